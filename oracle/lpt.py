@@ -1,0 +1,114 @@
+"""Cost-aware LPT planning of KV chunks onto workers (oracle; test infrastructure).
+
+[news] "Balance actual attention work": each context chunk gets a cost equal to
+its actual attention usage; LPT sorts chunks by cost and hands the expensive
+ones first to the least-loaded eligible worker, keeping chunk counts equal
+(device mode).  [digest] Abstract: "cost-aware longest-processing-time-first".
+
+Readings where the pages are silent (integer arithmetic, so bit-exact):
+
+* work item = (chunk c, KV head g[, slice]); cost = realised pairs served by the
+  item = G * pairs_c (G query heads read KV head g), or G * bs * sum(hi - lo)
+  over the blocks of a slice;
+* slicing: the chunk's entries are ordered by (lo, hi, b) and cut into query
+  tiles of rows_per_tile // (G * bs) blocks; consecutive groups of q_slice tiles
+  form the slices of the item;
+* items are ordered by cost descending, ties by (c, g, slice) ascending;
+* each goes to the eligible worker of minimum load, ties to the lowest id;
+* zero-cost items are dropped;
+* equal-count mode, n items on W workers, n = q W + r: a worker is eligible
+  while it holds fewer than q items, or holds q and fewer than r workers hold
+  q + 1;
+* imbalance = max load / mean load - 1 over all W workers;
+* the "unbalanced" baseline keeps chunks in contiguous order: the n_chunks * Hkv
+  unsliced items in (c, g) order, item i to worker floor(i W / n).
+"""
+
+from __future__ import annotations
+
+from typing import Dict, List, Tuple
+
+from .mask import chunk_entries, chunk_pairs
+
+
+def work_items(sample_lens, anchors, block_size: int, kv_chunk: int, num_q_heads: int,
+               num_kv_heads: int, q_slice: int = 0, rows_per_tile: int = 128
+               ) -> List[Tuple[Tuple[int, int, int], int]]:
+    """All work items ((c, g, slice), cost), zero-cost ones included."""
+    G = num_q_heads // num_kv_heads
+    bs = int(block_size)
+    items = []
+    if q_slice <= 0:
+        pairs = chunk_pairs(sample_lens, anchors, bs, kv_chunk)
+        for c, p in enumerate(pairs):
+            for g in range(num_kv_heads):
+                items.append(((c, g, 0), int(G * p)))
+        return items
+    blocks_per_tile = rows_per_tile // (G * bs)
+    per_chunk: Dict[int, list] = {}
+    for (c, b, lo, hi) in chunk_entries(sample_lens, anchors, kv_chunk):
+        per_chunk.setdefault(c, []).append((lo, hi, b))
+    for c in sorted(per_chunk):
+        ents = sorted(per_chunk[c])
+        per_slice = blocks_per_tile * q_slice
+        for s0 in range(0, len(ents), per_slice):
+            cost = G * bs * sum(hi - lo for (lo, hi, _) in ents[s0:s0 + per_slice])
+            for g in range(num_kv_heads):
+                items.append(((c, g, s0 // per_slice), int(cost)))
+    return items
+
+
+def lpt(items, num_workers: int, equal_count: bool = False):
+    """Assign items to workers longest-first; returns (lists, loads).
+
+    lists[w] holds the item keys of worker w in assignment order.
+    """
+    live = [(key, cost) for (key, cost) in items if cost > 0]
+    live.sort(key=lambda it: (-it[1], it[0]))
+    W = int(num_workers)
+    n = len(live)
+    q, r = divmod(n, W)
+    loads = [0] * W
+    counts = [0] * W
+    lists: List[list] = [[] for _ in range(W)]
+    for key, cost in live:
+        n_full = sum(1 for x in counts if x == q + 1)
+        best = -1
+        for w in range(W):
+            if equal_count:
+                ok = counts[w] < q or (counts[w] == q and n_full < r)
+            else:
+                ok = True
+            if ok and (best < 0 or loads[w] < loads[best]):
+                best = w
+        loads[best] += cost
+        counts[best] += 1
+        lists[best].append(key)
+    return lists, loads
+
+
+def contiguous(items, num_workers: int):
+    """Chunks left in contiguous order: item i of n (c, g order) -> worker floor(i W / n)."""
+    ordered = sorted(items, key=lambda it: it[0])
+    W = int(num_workers)
+    n = len(ordered)
+    loads = [0] * W
+    lists: List[list] = [[] for _ in range(W)]
+    for i, (key, cost) in enumerate(ordered):
+        w = (i * W) // n
+        loads[w] += cost
+        lists[w].append(key)
+    return lists, loads
+
+
+def imbalance(loads) -> float:
+    """max load / mean load - 1 (0 for an all-zero load vector)."""
+    total = sum(loads)
+    if total == 0:
+        return 0.0
+    mean = total / len(loads)
+    return max(loads) / mean - 1.0
+
+
+def makespan(loads) -> int:
+    return max(loads) if loads else 0

@@ -1,0 +1,118 @@
+"""Pins of the oracle's LPT planner (CPU only).
+
+LPT as stated on the news page, section "Balance actual attention work", and
+in the digest Abstract.  Pins: hand-worked assignments, Graham's makespan bound
+(4/3 - 1/(3m)) against an exhaustive optimum, the equal-count rule against an
+exhaustive equal-count optimum, and the cost bookkeeping.
+"""
+
+import itertools
+import json
+import os
+
+import numpy as np
+import pytest
+
+from oracle import lpt, mask
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _items(costs):
+    return [((i, 0, 0), int(c)) for i, c in enumerate(costs)]
+
+
+def test_hand_worked_cases():
+    g = json.load(open(os.path.join(GOLDEN, "lpt_hand.json")))
+    for case in g["cases"]:
+        lists, loads = lpt.lpt(_items(case["costs"]), case["workers"], case["equal_count"])
+        assert [[k[0] for k in l] for l in lists] == case["lists"], case["_worked"]
+        assert loads == case["loads"]
+
+
+def _opt(costs, m, equal_count=False):
+    n = len(costs)
+    best = None
+    q, r = divmod(n, m)
+    for assign in itertools.product(range(m), repeat=n):
+        if equal_count:
+            cnt = np.bincount(assign, minlength=m)
+            if sorted(cnt.tolist()) != sorted([q + 1] * r + [q] * (m - r)):
+                continue
+        loads = [0] * m
+        for c, w in zip(costs, assign):
+            loads[w] += c
+        ms = max(loads)
+        best = ms if best is None else min(best, ms)
+    return best
+
+
+@pytest.mark.parametrize("seed", range(40))
+def test_graham_bound_vs_exhaustive(seed):
+    rng = np.random.default_rng(seed)
+    m = int(rng.integers(2, 5))
+    n = int(rng.integers(m + 1, 9))
+    costs = rng.integers(1, 50, size=n).tolist()
+    _, loads = lpt.lpt(_items(costs), m)
+    opt = _opt(costs, m)
+    assert max(loads) <= (4.0 / 3.0 - 1.0 / (3 * m)) * opt + 1e-9
+
+
+@pytest.mark.parametrize("seed", range(40))
+def test_equal_count_counts_and_bound(seed):
+    """Counts differ by at most one; makespan within 4/3 - 1/(3m) of the equal-count optimum
+    on these instances (the bound observed; the pages state only that counts stay equal)."""
+    rng = np.random.default_rng(1000 + seed)
+    m = int(rng.integers(2, 4))
+    n = int(rng.integers(m + 1, 9))
+    costs = rng.integers(1, 50, size=n).tolist()
+    lists, loads = lpt.lpt(_items(costs), m, equal_count=True)
+    cnt = sorted(len(l) for l in lists)
+    q, r = divmod(n, m)
+    assert cnt == sorted([q + 1] * r + [q] * (m - r))
+    opt = _opt(costs, m, equal_count=True)
+    assert max(loads) <= (4.0 / 3.0 - 1.0 / (3 * m)) * opt + 1e-9
+
+
+def test_every_item_assigned_once_and_order_is_longest_first():
+    rng = np.random.default_rng(3)
+    costs = rng.integers(0, 100, size=60).tolist()
+    lists, loads = lpt.lpt(_items(costs), 7)
+    got = sorted(k[0] for l in lists for k in l)
+    assert got == [i for i, c in enumerate(costs) if c > 0]
+    for l in lists:
+        cs = [costs[k[0]] for k in l]
+        assert cs == sorted(cs, reverse=True)
+    assert loads == [sum(costs[k[0]] for k in l) for l in lists]
+
+
+def test_imbalance_definition():
+    assert lpt.imbalance([10, 10, 10]) == 0.0
+    assert abs(lpt.imbalance([12, 6, 6]) - (12 / 8 - 1)) < 1e-15
+    assert lpt.imbalance([0, 0]) == 0.0
+
+
+def test_contiguous_baseline_equal_lengths():
+    items = _items([5, 0, 3, 9, 1, 1, 2])
+    lists, loads = lpt.contiguous(items, 3)
+    # floor(i*3/7): i=0,1,2 -> 0; 3,4 -> 1; 5,6 -> 2
+    assert [[k[0] for k in l] for l in lists] == [[0, 1, 2], [3, 4], [5, 6]]
+    assert loads == [8, 10, 3]
+
+
+@pytest.mark.parametrize("q_slice", [0, 1, 2])
+def test_item_costs_sum_to_realised_pairs(q_slice):
+    rng = np.random.default_rng(11)
+    lens = rng.integers(20, 200, size=5).astype(np.int32)
+    N = int(lens.sum())
+    anchors = np.sort(rng.choice(N, size=24, replace=False)).astype(np.int32)
+    bs, C, Hq, Hkv = 4, 64, 8, 2
+    items = lpt.work_items(lens, anchors, bs, C, Hq, Hkv, q_slice=q_slice, rows_per_tile=32)
+    pairs = mask.chunk_pairs(lens, anchors, bs, C)
+    total = sum(c for _, c in items)
+    assert total == Hq * int(pairs.sum())
+    per_chunk = {}
+    for (c, g, s), cost in items:
+        per_chunk[c] = per_chunk.get(c, 0) + cost
+    for c, p in enumerate(pairs):
+        assert per_chunk.get(c, 0) == Hq * int(p)
