@@ -1,0 +1,232 @@
+"""Split-KV block-sparse anchor attention on NVIDIA B200 (sm_100a).
+
+Thin Python binding of libsplitkv.so.  The functions carry the C entry points'
+names and only marshal arguments (torch tensors -> device pointers, the
+current CUDA stream -> cudaStream_t); every step of the computation runs in the
+library's CUDA kernels.  Importing this package loads the shared library and
+raises ImportError if it has not been built.
+
+Method: "Split-KV: Efficient Context Parallelism for Training Diffusion
+Drafters" (digest page, Abstract) and the news page "Split-KV speeds
+diffusion drafter training by keeping long-context data local" (sections "Why
+short queries change the problem", "Exchange the smaller side", "Balance actual
+attention work").
+"""
+
+from __future__ import annotations
+
+import ctypes
+from typing import Optional, Sequence
+
+import numpy as np
+
+from . import _abi
+from ._abi import (  # noqa: F401
+    DTYPE_BF16, DTYPE_F32, EXPORT_BWD_LOADS, EXPORT_BWD_SCHEDULE, EXPORT_CHUNK_PAIRS,
+    EXPORT_CONTIG_LOADS, EXPORT_ENTRIES, EXPORT_FWD_LOADS, EXPORT_FWD_SCHEDULE,
+    FLAG_EQUAL_COUNT, WS_BWD, WS_FWD,
+)
+
+_lib = _abi.load()
+
+
+class SplitKVError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        self.status = status
+        msg = _lib.splitkv_error_string(status).decode()
+        super().__init__(f"{fn}: {msg} ({status})")
+
+
+def _check(fn: str, status: int) -> None:
+    if status != _abi.OK:
+        raise SplitKVError(fn, status)
+
+
+def _stream_ptr(stream) -> Optional[int]:
+    if stream is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    if hasattr(stream, "cuda_stream"):
+        return stream.cuda_stream
+    return int(stream)
+
+
+def _ptr(t) -> Optional[int]:
+    if t is None:
+        return None
+    if not t.is_cuda or not t.is_contiguous():
+        raise ValueError("tensors must be contiguous CUDA tensors")
+    return t.data_ptr()
+
+
+def _bf16_ptr(t) -> int:
+    import torch
+    if t.dtype != torch.bfloat16:
+        raise ValueError("q, k, v, kb, vb and dout must be bfloat16")
+    return _ptr(t)
+
+
+def _f32_ptr(t) -> int:
+    import torch
+    if t.dtype != torch.float32:
+        raise ValueError("lse, dq, dk, dv, dkb and dvb must be float32")
+    return _ptr(t)
+
+
+def _o_dtype(o) -> int:
+    import torch
+    if o.dtype == torch.float32:
+        return DTYPE_F32
+    if o.dtype == torch.bfloat16:
+        return DTYPE_BF16
+    raise ValueError("o must be float32 or bfloat16")
+
+
+class Plan:
+    """Owner of a splitkv_plan_t handle (see splitkv_plan)."""
+
+    def __init__(self, handle: ctypes.c_void_p, problem: _abi.Problem, keep):
+        self._h = handle
+        self.problem = problem
+        self._keep = keep
+
+    @property
+    def handle(self) -> ctypes.c_void_p:
+        if not self._h:
+            raise ValueError("plan has been destroyed")
+        return self._h
+
+    def stats(self) -> dict:
+        return splitkv_plan_stats(self)
+
+    def export(self, what: int) -> np.ndarray:
+        return splitkv_plan_export(self, what)
+
+    def upload(self, stream=None) -> "Plan":
+        splitkv_plan_upload(self, stream)
+        return self
+
+    def destroy(self) -> None:
+        splitkv_plan_destroy(self)
+
+    def __del__(self):
+        try:
+            if self._h:
+                _lib.splitkv_plan_destroy(self._h)
+                self._h = None
+        except Exception:
+            pass
+
+
+def _problem(sample_lens, anchors, block_size, num_q_heads, num_kv_heads, head_dim, kv_chunk,
+             num_workers, num_bwd_workers, q_slice, equal_count):
+    lens = np.ascontiguousarray(sample_lens, dtype=np.int32)
+    anc = np.ascontiguousarray(anchors, dtype=np.int32)
+    p = _abi.Problem()
+    p.num_samples = lens.size
+    p.sample_lens = lens.ctypes.data_as(ctypes.POINTER(ctypes.c_int32))
+    p.num_anchors = anc.size
+    p.anchors = anc.ctypes.data_as(ctypes.POINTER(ctypes.c_int32))
+    p.block_size = int(block_size)
+    p.num_q_heads = int(num_q_heads)
+    p.num_kv_heads = int(num_kv_heads)
+    p.head_dim = int(head_dim)
+    p.kv_chunk = int(kv_chunk)
+    p.num_workers = int(num_workers)
+    p.num_bwd_workers = int(num_bwd_workers)
+    p.q_slice = int(q_slice)
+    p.flags = FLAG_EQUAL_COUNT if equal_count else 0
+    return p, (lens, anc)
+
+
+def splitkv_plan(sample_lens: Sequence[int], anchors: Sequence[int], block_size: int, num_q_heads: int,
+                 num_kv_heads: int, head_dim: int, kv_chunk: int, num_workers: int,
+                 num_bwd_workers: int = 0, q_slice: int = 0, equal_count: bool = False) -> Plan:
+    """Host-side mask metadata + LPT schedules (no CUDA call)."""
+    p, keep = _problem(sample_lens, anchors, block_size, num_q_heads, num_kv_heads, head_dim, kv_chunk,
+                       num_workers, num_bwd_workers, q_slice, equal_count)
+    h = ctypes.c_void_p()
+    _check("splitkv_plan", _lib.splitkv_plan(ctypes.byref(p), ctypes.byref(h)))
+    return Plan(h, p, keep)
+
+
+def splitkv_plan_update(plan: Plan, sample_lens, anchors, **kw) -> Plan:
+    """Rebuild `plan` in place for new sample lengths / anchors (other fields kept unless given)."""
+    old = plan.problem
+    args = dict(block_size=old.block_size, num_q_heads=old.num_q_heads, num_kv_heads=old.num_kv_heads,
+                head_dim=old.head_dim, kv_chunk=old.kv_chunk, num_workers=old.num_workers,
+                num_bwd_workers=old.num_bwd_workers, q_slice=old.q_slice,
+                equal_count=bool(old.flags & FLAG_EQUAL_COUNT))
+    args.update(kw)
+    p, keep = _problem(sample_lens, anchors, **args)
+    _check("splitkv_plan_update", _lib.splitkv_plan_update(plan.handle, ctypes.byref(p)))
+    plan.problem, plan._keep = p, keep
+    return plan
+
+
+def splitkv_plan_upload(plan: Plan, stream=None) -> None:
+    _check("splitkv_plan_upload", _lib.splitkv_plan_upload(plan.handle, _stream_ptr(stream)))
+
+
+def splitkv_plan_destroy(plan: Plan) -> None:
+    if plan._h:
+        h, plan._h = plan._h, None
+        _check("splitkv_plan_destroy", _lib.splitkv_plan_destroy(h))
+
+
+def splitkv_plan_stats(plan: Plan) -> dict:
+    s = _abi.Stats()
+    _check("splitkv_plan_stats", _lib.splitkv_plan_stats(plan.handle, ctypes.byref(s)))
+    return s.as_dict()
+
+
+def splitkv_plan_export(plan: Plan, what: int) -> np.ndarray:
+    n = ctypes.c_int64()
+    _check("splitkv_plan_export", _lib.splitkv_plan_export(plan.handle, what, None, 0, ctypes.byref(n)))
+    out = np.zeros(max(n.value, 1), dtype=np.int64)
+    _check("splitkv_plan_export", _lib.splitkv_plan_export(
+        plan.handle, what, out.ctypes.data_as(ctypes.POINTER(ctypes.c_int64)), out.size, ctypes.byref(n)))
+    return out[:n.value]
+
+
+def splitkv_workspace_size(plan: Plan, which: int) -> int:
+    n = ctypes.c_size_t()
+    _check("splitkv_workspace_size", _lib.splitkv_workspace_size(plan.handle, which, ctypes.byref(n)))
+    return n.value
+
+
+def splitkv_attn_fwd(plan: Plan, q, k, v, scale: float, ws, stream=None) -> None:
+    """Chunk partial records into ws (uint8 CUDA tensor of splitkv_workspace_size(plan, WS_FWD) bytes)."""
+    _check("splitkv_attn_fwd", _lib.splitkv_attn_fwd(
+        plan.handle, _bf16_ptr(q), _bf16_ptr(k), _bf16_ptr(v), float(scale), _ptr(ws), ws.numel() * ws.element_size(),
+        _stream_ptr(stream)))
+
+
+def splitkv_merge(plan: Plan, q, kb, vb, scale: float, ws, o, lse, stream=None) -> None:
+    """In-block term + exact LSE merge of the chunk records -> o (f32 or bf16), lse (f32)."""
+    _check("splitkv_merge", _lib.splitkv_merge(
+        plan.handle, _bf16_ptr(q), _bf16_ptr(kb), _bf16_ptr(vb), float(scale), _ptr(ws),
+        ws.numel() * ws.element_size(), _ptr(o), _o_dtype(o), _f32_ptr(lse), _stream_ptr(stream)))
+
+
+def splitkv_attn_bwd(plan: Plan, q, k, v, kb, vb, o, lse, dout, dq, dk, dv, dkb, dvb, scale: float, ws,
+                     stream=None) -> None:
+    """Gradients dq, dk, dv, dkb, dvb (float32) recomputed from the saved lse."""
+    _check("splitkv_attn_bwd", _lib.splitkv_attn_bwd(
+        plan.handle, _bf16_ptr(q), _bf16_ptr(k), _bf16_ptr(v), _bf16_ptr(kb), _bf16_ptr(vb), _ptr(o),
+        _o_dtype(o), _f32_ptr(lse), _bf16_ptr(dout), _f32_ptr(dq), _f32_ptr(dk), _f32_ptr(dv), _f32_ptr(dkb),
+        _f32_ptr(dvb), float(scale), _ptr(ws), ws.numel() * ws.element_size(), _stream_ptr(stream)))
+
+
+def splitkv_read_cta_times(plan: Plan, which: int, stream=None) -> np.ndarray:
+    """Per-CTA busy nanoseconds of the last forward (WS_FWD) or backward (WS_BWD) partial kernel."""
+    st = plan.stats()
+    n = st["num_workers"] if which == WS_FWD else st["num_bwd_workers"]
+    out = np.zeros(n, dtype=np.int64)
+    _check("splitkv_read_cta_times", _lib.splitkv_read_cta_times(
+        plan.handle, which, out.ctypes.data_as(ctypes.POINTER(ctypes.c_int64)), n, _stream_ptr(stream)))
+    return out
+
+
+def library_path() -> str:
+    return _abi.LIB_PATH

@@ -1,0 +1,128 @@
+// C-ABI attention entry points of libsplitkv.so: argument checks, workspace
+// carving and kernel dispatch.  Every step of the computation runs in the
+// sm_100a kernels; this file only validates and launches.
+#include <cstdint>
+#include <new>
+
+#include "splitkv.h"
+#include "splitkv_internal.h"
+
+namespace splitkv {
+const DevPlan* plan_device_view(const splitkv_plan_t* P);
+}
+
+namespace {
+
+using splitkv::DevPlan;
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+// Shared checks of every attention call; on success *out points at the device view.
+int check_plan(const splitkv_plan_t* plan, const DevPlan** out) {
+  if (!plan) return SPLITKV_ERR_INVALID_ARG;
+  const DevPlan* dp = splitkv::plan_device_view(plan);
+  if (!dp) return SPLITKV_ERR_NOT_UPLOADED;
+  if (dp->d != 64 && dp->d != 128) return SPLITKV_ERR_UNSUPPORTED;
+  *out = dp;
+  return SPLITKV_OK;
+}
+
+int cuda_status(cudaError_t e) {
+  if (e == cudaSuccess) return SPLITKV_OK;
+  cudaGetLastError();
+  return SPLITKV_ERR_CUDA;
+}
+
+template <typename... Ps>
+bool all_aligned16(Ps... ps) {
+  return ((ps != nullptr && aligned(ps, 16)) && ...);
+}
+
+}  // namespace
+
+extern "C" {
+
+int splitkv_attn_fwd(const splitkv_plan_t* plan, const void* q, const void* k, const void* v, float scale,
+                     void* ws, size_t ws_bytes, void* stream) {
+  const DevPlan* dp = nullptr;
+  int st = check_plan(plan, &dp);
+  if (st != SPLITKV_OK) return st;
+  if (!all_aligned16(q, k, v, ws)) return SPLITKV_ERR_INVALID_ARG;
+  const splitkv::FwdWs L = splitkv::fwd_ws_layout(dp->E, dp->bs, dp->Hq, dp->d);
+  if (ws_bytes < L.total) return SPLITKV_ERR_WORKSPACE_TOO_SMALL;
+  char* w = static_cast<char*>(ws);
+  return cuda_status(splitkv::launch_fwd_partial(
+      *dp, static_cast<const uint16_t*>(q), static_cast<const uint16_t*>(k), static_cast<const uint16_t*>(v),
+      scale, reinterpret_cast<float*>(w + L.o_off), reinterpret_cast<float*>(w + L.m_off),
+      reinterpret_cast<float*>(w + L.l_off), static_cast<cudaStream_t>(stream)));
+}
+
+int splitkv_merge(const splitkv_plan_t* plan, const void* q, const void* kb, const void* vb, float scale,
+                  const void* ws, size_t ws_bytes, void* o, int o_dtype, float* lse, void* stream) {
+  const DevPlan* dp = nullptr;
+  int st = check_plan(plan, &dp);
+  if (st != SPLITKV_OK) return st;
+  if (!all_aligned16(q, kb, vb, ws, o) || !lse || !aligned(lse, 4)) return SPLITKV_ERR_INVALID_ARG;
+  if (o_dtype != SPLITKV_DTYPE_F32 && o_dtype != SPLITKV_DTYPE_BF16) return SPLITKV_ERR_INVALID_ARG;
+  const splitkv::FwdWs L = splitkv::fwd_ws_layout(dp->E, dp->bs, dp->Hq, dp->d);
+  if (ws_bytes < L.total) return SPLITKV_ERR_WORKSPACE_TOO_SMALL;
+  const char* w = static_cast<const char*>(ws);
+  return cuda_status(splitkv::launch_merge(
+      *dp, static_cast<const uint16_t*>(q), static_cast<const uint16_t*>(kb), static_cast<const uint16_t*>(vb),
+      scale, reinterpret_cast<const float*>(w + L.o_off), reinterpret_cast<const float*>(w + L.m_off),
+      reinterpret_cast<const float*>(w + L.l_off), o, o_dtype == SPLITKV_DTYPE_BF16 ? 1 : 0, lse,
+      static_cast<cudaStream_t>(stream)));
+}
+
+int splitkv_attn_bwd(const splitkv_plan_t* plan, const void* q, const void* k, const void* v, const void* kb,
+                     const void* vb, const void* o, int o_dtype, const float* lse, const void* dout, float* dq,
+                     float* dk, float* dv, float* dkb, float* dvb, float scale, void* ws, size_t ws_bytes,
+                     void* stream) {
+  const DevPlan* dp = nullptr;
+  int st = check_plan(plan, &dp);
+  if (st != SPLITKV_OK) return st;
+  if (!all_aligned16(q, k, v, kb, vb, o, dout, dq, dk, dv, dkb, dvb, ws) || !lse || !aligned(lse, 4))
+    return SPLITKV_ERR_INVALID_ARG;
+  if (o_dtype != SPLITKV_DTYPE_F32 && o_dtype != SPLITKV_DTYPE_BF16) return SPLITKV_ERR_INVALID_ARG;
+  const splitkv::BwdWs L = splitkv::bwd_ws_layout(dp->E, dp->Nq, dp->bs, dp->Hq, dp->d);
+  if (ws_bytes < L.total) return SPLITKV_ERR_WORKSPACE_TOO_SMALL;
+  char* w = static_cast<char*>(ws);
+  float* dq_part = reinterpret_cast<float*>(w + L.dq_off);
+  float* delta = reinterpret_cast<float*>(w + L.delta_off);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const auto* q16 = static_cast<const uint16_t*>(q);
+  const auto* do16 = static_cast<const uint16_t*>(dout);
+  const int obf = o_dtype == SPLITKV_DTYPE_BF16 ? 1 : 0;
+  st = cuda_status(splitkv::launch_bwd_delta(*dp, o, obf, do16, delta, s));
+  if (st != SPLITKV_OK) return st;
+  st = cuda_status(splitkv::launch_bwd_partial(*dp, q16, static_cast<const uint16_t*>(k),
+                                               static_cast<const uint16_t*>(v), do16, lse, delta, scale, dk, dv,
+                                               dq_part, s));
+  if (st != SPLITKV_OK) return st;
+  return cuda_status(splitkv::launch_bwd_reduce(*dp, q16, static_cast<const uint16_t*>(kb),
+                                                static_cast<const uint16_t*>(vb), do16, lse, delta, dq_part,
+                                                scale, dq, dkb, dvb, s));
+}
+
+int splitkv_read_cta_times(const splitkv_plan_t* plan, int which, int64_t* out_ns, int64_t capacity,
+                           void* stream) {
+  if (!plan || !out_ns) return SPLITKV_ERR_INVALID_ARG;
+  const DevPlan* dp = splitkv::plan_device_view(plan);
+  if (!dp) return SPLITKV_ERR_NOT_UPLOADED;
+  if (which != SPLITKV_WS_FWD && which != SPLITKV_WS_BWD) return SPLITKV_ERR_INVALID_ARG;
+  const int n = which == SPLITKV_WS_FWD ? dp->W : dp->Wb;
+  if (capacity < n) return SPLITKV_ERR_WORKSPACE_TOO_SMALL;
+  const long long* src = dp->timers + (which == SPLITKV_WS_FWD ? 0 : 2 * size_t(dp->W));
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  // stamps are small: copy to a host array synchronously on the stream
+  long long* host = new (std::nothrow) long long[2 * size_t(n)];
+  if (!host) return SPLITKV_ERR_NO_MEMORY;
+  int st = cuda_status(cudaMemcpyAsync(host, src, 2 * size_t(n) * sizeof(long long), cudaMemcpyDeviceToHost, s));
+  if (st == SPLITKV_OK) st = cuda_status(cudaStreamSynchronize(s));
+  if (st == SPLITKV_OK)
+    for (int i = 0; i < n; ++i) out_ns[i] = host[2 * i + 1] - host[2 * i];
+  delete[] host;
+  return st;
+}
+
+}  // extern "C"

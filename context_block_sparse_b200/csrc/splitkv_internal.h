@@ -1,0 +1,86 @@
+// Internal declarations shared by the host planner, the C-ABI layer and the
+// sm_100a kernels of libsplitkv.so.  Not part of the public ABI.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+
+#include <cuda_runtime.h>
+
+namespace splitkv {
+
+// Rows of one query tile: 128 / (G * bs) blocks x G heads x bs tokens.
+constexpr int kTileRows = 128;
+
+// Device view of a plan.  Every table lives in one device allocation owned by
+// the plan; this struct is passed by value as a kernel parameter.
+struct DevPlan {
+  const int4* entries;          // [E]   {block, lo, hi, chunk}, record order
+  const int4* tiles;            // [T]   {e0, e1, klo, khi}: entries [e0, e1), key union [klo, khi)
+  const int4* fwd_items;        // [If]  {chunk, kv head, t0, t1} grouped by worker
+  const int*  fwd_worker_ptr;   // [W+1]
+  const int4* bwd_items;        // [Ib]  same, backward schedule (whole chunks)
+  const int*  bwd_worker_ptr;   // [W+1]
+  const int*  block_entry_ptr;  // [A+1]
+  const int*  block_entries;    // [E]   entry ids of each block, ascending chunk
+  const int*  zero_chunks;      // [Z]   chunks no block reads (backward zero fill)
+  long long*  timers;           // [W + Wb][2] global-timer stamps: forward CTAs, then backward CTAs
+  int num_zero_chunks;
+  int N, Nq, A, bs, Hq, Hkv, G, d, C, num_chunks, E, W, Wb;
+};
+
+// Byte offsets of the forward workspace (partial records).
+struct FwdWs {
+  size_t o_off, m_off, l_off, total;
+};
+// Byte offsets of the backward workspace (dq partials, Delta).
+struct BwdWs {
+  size_t dq_off, delta_off, total;
+};
+
+inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+inline FwdWs fwd_ws_layout(long long E, int bs, int Hq, int d) {
+  FwdWs w;
+  const size_t rows = size_t(E) * bs * Hq;
+  w.o_off = 0;
+  w.m_off = align_up(rows * d * sizeof(float), 256);
+  w.l_off = w.m_off + align_up(rows * sizeof(float), 256);
+  w.total = w.l_off + align_up(rows * sizeof(float), 256);
+  if (w.total == 0) w.total = 256;
+  return w;
+}
+
+inline BwdWs bwd_ws_layout(long long E, int Nq, int bs, int Hq, int d) {
+  BwdWs w;
+  const size_t rows = size_t(E) * bs * Hq;
+  w.dq_off = 0;
+  w.delta_off = align_up(rows * d * sizeof(float), 256);
+  w.total = w.delta_off + align_up(size_t(Nq) * Hq * sizeof(float), 256);
+  return w;
+}
+
+// ---- kernel launchers (defined in the .cu files) ---------------------------
+cudaError_t launch_fwd_partial(const DevPlan& p, const uint16_t* q, const uint16_t* k,
+                               const uint16_t* v, float scale, float* part_o, float* part_m,
+                               float* part_l, cudaStream_t s);
+
+cudaError_t launch_merge(const DevPlan& p, const uint16_t* q, const uint16_t* kb,
+                         const uint16_t* vb, float scale, const float* part_o,
+                         const float* part_m, const float* part_l, void* o, int o_bf16,
+                         float* lse, cudaStream_t s);
+
+cudaError_t launch_bwd_delta(const DevPlan& p, const void* o, int o_bf16, const uint16_t* dout,
+                             float* delta, cudaStream_t s);
+
+cudaError_t launch_bwd_partial(const DevPlan& p, const uint16_t* q, const uint16_t* k,
+                               const uint16_t* v, const uint16_t* dout, const float* lse,
+                               const float* delta, float scale, float* dk, float* dv,
+                               float* dq_part, cudaStream_t s);
+
+cudaError_t launch_bwd_reduce(const DevPlan& p, const uint16_t* q, const uint16_t* kb,
+                              const uint16_t* vb, const uint16_t* dout, const float* lse,
+                              const float* delta, const float* dq_part, float scale, float* dq,
+                              float* dkb, float* dvb, cudaStream_t s);
+
+}  // namespace splitkv

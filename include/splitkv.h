@@ -1,0 +1,241 @@
+/*
+ * splitkv.h -- C ABI of the Split-KV block-sparse anchor attention library
+ * (libsplitkv.so, NVIDIA B200 / sm_100a).
+ *
+ * The method ("Split-KV: Efficient Context Parallelism for Training Diffusion
+ * Drafters", paper digest page, Abstract; news page "Split-KV speeds diffusion
+ * drafter training by keeping long-context data local"):
+ *
+ *   - anchors sampled from a packed context open blocks of block_size draft
+ *     query tokens; block b attends to the preceding context of its own sample,
+ *     keys [S_s, a_b), plus the block_size keys of its own block (news page,
+ *     "Why short queries change the problem");
+ *   - the context is cut into KV chunks; every chunk computes partial attention
+ *     for each query block it touches and the partials are combined exactly with
+ *     their normalisation statistics (news page, "Exchange the smaller side");
+ *   - chunks are scheduled longest-processing-time-first by realised attention
+ *     cost onto the least-loaded eligible worker (news page, "Balance actual
+ *     attention work").  On one GPU a worker is a persistent CTA.
+ *
+ * Conventions for every entry point:
+ *   - Return value: SPLITKV_OK (0) or a negative SPLITKV_ERR_* code; no C++
+ *     exception crosses this boundary.  splitkv_error_string() names a code.
+ *   - Tensors are caller-owned, contiguous DEVICE memory in these layouts
+ *     (row-major, last index fastest), 16-byte aligned:
+ *         q, dout      [Nq, Hq, d]   bfloat16 (raw 16-bit storage)
+ *         k, v         [N, Hkv, d]   bfloat16
+ *         kb, vb       [Nq, Hkv, d]  bfloat16  (the draft block's own keys/values,
+ *                                                one row per draft token)
+ *         o            [Nq, Hq, d]   float32 or bfloat16 (see o_dtype)
+ *         lse          [Nq, Hq]      float32, natural log
+ *         dq           [Nq, Hq, d]   float32
+ *         dk, dv       [N, Hkv, d]   float32
+ *         dkb, dvb     [Nq, Hkv, d]  float32
+ *     where N = sum of sample lengths, Nq = num_anchors * block_size, query
+ *     token i belongs to block i / block_size, and query head h reads KV head
+ *     h / (Hq / Hkv).
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *     stream).  Attention calls are asynchronous on it.  splitkv_plan,
+ *     splitkv_plan_update and the stats/export calls are host-only;
+ *     splitkv_plan_upload enqueues a copy on the stream.
+ *   - Workspaces are caller-allocated device memory of at least the size
+ *     splitkv_workspace_size reports; the library allocates no per-call memory.
+ *   - Calls that share a plan or a workspace must not run concurrently on
+ *     different streams.
+ */
+#ifndef SPLITKV_H_
+#define SPLITKV_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* ---- status codes -------------------------------------------------------- */
+#define SPLITKV_OK                        0
+#define SPLITKV_ERR_INVALID_ARG          -1  /* bad pointer, size, layout or problem      */
+#define SPLITKV_ERR_UNSUPPORTED          -2  /* valid problem outside the kernels' shapes */
+#define SPLITKV_ERR_WORKSPACE_TOO_SMALL  -3
+#define SPLITKV_ERR_CUDA                 -4  /* a CUDA runtime call failed                */
+#define SPLITKV_ERR_TIMEOUT              -5  /* reserved: a bounded device wait gave up   */
+#define SPLITKV_ERR_NOT_UPLOADED         -6  /* plan has no device copy yet               */
+#define SPLITKV_ERR_NO_MEMORY            -7  /* host or device allocation failed          */
+
+/* ---- plan flags -------------------------------------------------------------- */
+/* Equal-count LPT (the pages' device rule: chunk counts kept equal).  Off by
+ * default: CTAs have no memory limit, and plain LPT keeps Graham's bound. */
+#define SPLITKV_FLAG_EQUAL_COUNT  1u
+
+/* ---- dtype codes (o) ------------------------------------------------------- */
+#define SPLITKV_DTYPE_F32   0
+#define SPLITKV_DTYPE_BF16  1
+
+/* ---- workspace kinds --------------------------------------------------------- */
+#define SPLITKV_WS_FWD  0
+#define SPLITKV_WS_BWD  1
+
+/* ---- export selectors (splitkv_plan_export) ------------------------------- */
+#define SPLITKV_EXPORT_ENTRIES        0  /* 4 per entry: chunk, block, lo, hi (record order)      */
+#define SPLITKV_EXPORT_CHUNK_PAIRS    1  /* 1 per chunk: allowed (row, key) pairs per query head  */
+#define SPLITKV_EXPORT_FWD_SCHEDULE   2  /* 5 per assigned item: worker, chunk, kv head, slice, cost */
+#define SPLITKV_EXPORT_BWD_SCHEDULE   3  /* same, for the backward schedule (never sliced)        */
+#define SPLITKV_EXPORT_FWD_LOADS      4  /* 1 per forward worker: summed cost                      */
+#define SPLITKV_EXPORT_BWD_LOADS      5  /* 1 per backward worker                                  */
+#define SPLITKV_EXPORT_CONTIG_LOADS   6  /* 1 per forward worker: the contiguous ("unbalanced")
+                                            baseline                                               */
+
+/* The problem, as the news page states it ("Why short queries change the
+ * problem"): packed sample lengths, anchor positions, block size, and the
+ * GQA head layout.  All pointers are HOST memory, read during the call only. */
+typedef struct splitkv_problem {
+  int32_t        num_samples;   /* S >= 1                                                  */
+  const int32_t* sample_lens;   /* [S], every L_s >= 1; N = sum L_s < 2^31                 */
+  int32_t        num_anchors;   /* A >= 1                                                  */
+  const int32_t* anchors;       /* [A] global packed positions in [0, N); block b = anchors[b];
+                                   any order, repeats allowed                                */
+  int32_t        block_size;    /* bs >= 1                                                 */
+  int32_t        num_q_heads;   /* Hq, a multiple of Hkv                                   */
+  int32_t        num_kv_heads;  /* Hkv >= 1                                                */
+  int32_t        head_dim;      /* d (the kernels take 64 or 128)                          */
+  int32_t        kv_chunk;      /* C >= 1: chunk c covers keys [cC, min((c+1)C, N))         */
+  int32_t        num_workers;   /* W >= 1: persistent CTAs of the forward partial kernel    */
+  int32_t        num_bwd_workers; /* persistent CTAs of the backward partial kernel; 0 = W   */
+  int32_t        q_slice;       /* 0 = one item per (chunk, KV head); k > 0 = items of at most
+                                   k 128-row query tiles (forward schedule only)             */
+  uint32_t       flags;         /* SPLITKV_FLAG_*                                          */
+} splitkv_problem;
+
+typedef struct splitkv_plan splitkv_plan_t;   /* opaque, owned by the library */
+
+typedef struct splitkv_stats {
+  int64_t  context_len;        /* N                                                        */
+  int64_t  num_queries;        /* Nq                                                       */
+  int32_t  num_chunks;
+  int32_t  num_entries;        /* (chunk, block) pairs with a non-empty key interval        */
+  int32_t  num_tiles;          /* 128-row query tiles over all chunks                       */
+  int32_t  num_fwd_items;      /* non-zero-cost items of the forward schedule               */
+  int32_t  num_bwd_items;
+  int32_t  num_workers;
+  int32_t  num_bwd_workers;
+  uint64_t context_pairs;      /* sum over heads, rows and context keys of allowed pairs     */
+  uint64_t block_pairs;        /* Hq * A * bs * bs (the in-block term)                      */
+  uint64_t fwd_max_load;
+  uint64_t bwd_max_load;
+  double   fwd_imbalance;      /* max / mean - 1 over the W workers                         */
+  double   bwd_imbalance;
+  double   contig_imbalance;   /* same metric for the contiguous baseline                   */
+  double   plan_us;            /* host time of the last splitkv_plan / splitkv_plan_update  */
+} splitkv_stats;
+
+/* Name of a status code (static string, never NULL). */
+const char* splitkv_error_string(int status);
+
+/* Build the mask metadata and both LPT schedules on the host (no CUDA call).
+ * Metadata (news page, "Why short queries change the problem"; "Balance actual
+ * attention work"): per block its context interval [S_s, a_b); per chunk the
+ * blocks whose interval meets it, clipped to [lo, hi) and ordered by
+ * (lo, hi, block) -- the "entries", whose order is also the order of partial
+ * records in the workspace; 128-row query tiles of consecutive entries (a tile
+ * holds 128 / (G * bs) blocks, G = Hq / Hkv, which must divide 128).
+ * Schedule (digest Abstract; news page "Balance actual attention work"): items
+ * (chunk, KV head[, slice]) of integer cost G * bs * sum(hi - lo); sorted by
+ * cost descending, ties by (chunk, head, slice) ascending; each goes to the
+ * eligible worker of least load, ties to the lowest id; zero-cost items are
+ * dropped.  *out receives a plan the caller frees with splitkv_plan_destroy.
+ * Errors: INVALID_ARG (NULL, non-positive sizes, an anchor outside [0, N),
+ * Hq % Hkv != 0), UNSUPPORTED (128 % (G * bs) != 0), NO_MEMORY. */
+int splitkv_plan(const splitkv_problem* problem, splitkv_plan_t** out);
+
+/* Rebuild `plan` in place for a new problem (same rules as splitkv_plan),
+ * keeping its host and device buffers for reuse.  Blocks only until the
+ * plan's previous upload has been consumed from its pinned staging buffer.
+ * The device copy is stale until the next splitkv_plan_upload. */
+int splitkv_plan_update(splitkv_plan_t* plan, const splitkv_problem* problem);
+
+/* Copy the plan's tables to device memory owned by the plan (allocated or
+ * grown on first need, which synchronises `stream`), through a pinned
+ * staging buffer, asynchronously on `stream`.  Attention calls need it.
+ * Errors: INVALID_ARG, CUDA, NO_MEMORY. */
+int splitkv_plan_upload(splitkv_plan_t* plan, void* stream);
+
+/* Free the plan and its host, pinned and device buffers (synchronises the
+ * device if a device copy exists).  NULL is accepted. */
+int splitkv_plan_destroy(splitkv_plan_t* plan);
+
+/* Summary numbers of the plan (host only). */
+int splitkv_plan_stats(const splitkv_plan_t* plan, splitkv_stats* out);
+
+/* Copy one of the plan's host tables (SPLITKV_EXPORT_*) into out[0..capacity)
+ * as int64 values; *count receives the number of values the table holds.
+ * out may be NULL with capacity 0 to query the size.  Errors: INVALID_ARG,
+ * WORKSPACE_TOO_SMALL (capacity < *count; *count is still set). */
+int splitkv_plan_export(const splitkv_plan_t* plan, int what, int64_t* out,
+                        int64_t capacity, int64_t* count);
+
+/* Bytes of workspace an attention call needs (host only).
+ *   SPLITKV_WS_FWD: the chunk partial records, as float32
+ *       O_c [E][bs][Hq][d], then m_c [E][bs][Hq], then l_c [E][bs][Hq]
+ *     (E = number of entries, in entry order; each array starts on a 256-byte
+ *     boundary).  m_c is the row's max of scale * q.k over the entry's keys
+ *     (natural units), l_c = sum exp(s - m_c), O_c = sum exp(s - m_c) v / l_c.
+ *   SPLITKV_WS_BWD: dQ partials float32 [E][bs][Hq][d], then
+ *     Delta = rowsum(dout * o) float32 [Nq][Hq]. */
+int splitkv_workspace_size(const splitkv_plan_t* plan, int which, size_t* bytes);
+
+/* Partial attention of every entry (news page, "Exchange the smaller side":
+ * each shard evaluates all queries against its own keys).  For every entry
+ * (chunk c, block b, [lo, hi)) and every query row of b and head h, over the
+ * context keys j in [lo, hi) of KV head h / G: s = scale * q . k_j, and the
+ * record (m_c, l_c, O_c) defined at splitkv_workspace_size is written to ws.
+ * One persistent CTA per worker walks its forward schedule.  kb and vb are
+ * not read here (the in-block term is formed by splitkv_merge).
+ * Errors: INVALID_ARG (NULL/misaligned pointer, plan), NOT_UPLOADED,
+ * UNSUPPORTED (d not 64 or 128), WORKSPACE_TOO_SMALL, CUDA (launch failure). */
+int splitkv_attn_fwd(const splitkv_plan_t* plan, const void* q, const void* k,
+                     const void* v, float scale, void* ws, size_t ws_bytes,
+                     void* stream);
+
+/* Exact combine (news page, "Exchange the smaller side"): for every query row
+ * and head, the in-block term over the bs keys kb/vb of its own block gives a
+ * record (m_b, l_b, O_b); with the row's chunk records x (in chunk order),
+ * M = max m_x, L = sum l_x exp(m_x - M), o = sum l_x exp(m_x - M) O_x / L,
+ * lse = M + log L.  Records with l = 0 are skipped.  o is written as float32
+ * or bfloat16 (o_dtype), lse as float32.  ws must hold a forward result of
+ * the same plan.  Errors: as splitkv_attn_fwd. */
+int splitkv_merge(const splitkv_plan_t* plan, const void* q, const void* kb,
+                  const void* vb, float scale, const void* ws, size_t ws_bytes,
+                  void* o, int o_dtype, float* lse, void* stream);
+
+/* Backward with keys and values local to their chunk (news page, "Exchange
+ * the smaller side": K/V stay local through forward and backward), recomputing
+ * P = exp(s - lse) from the saved lse.  Per allowed (row i, key j):
+ *   dv_j += P_ij dout_i;  dP_ij = dout_i . v_j;  dS_ij = P_ij (dP_ij - Delta_i);
+ *   dk_j += scale dS_ij q_i;  dq_i += scale dS_ij k_j,
+ * with Delta_i = dout_i . o_i.  dk/dv of a chunk are owned by the CTA of its
+ * (chunk, KV head) item and summed over the G query heads; dq is written per
+ * entry as a partial and reduced over chunks in ascending chunk order, then the
+ * in-block term adds its dq and produces dkb/dvb (summed over the block's rows
+ * and the G heads).  Keys no query reads get dk = dv = 0.  Deterministic.
+ * o has dtype o_dtype.  Errors: as splitkv_attn_fwd. */
+int splitkv_attn_bwd(const splitkv_plan_t* plan, const void* q, const void* k,
+                     const void* v, const void* kb, const void* vb,
+                     const void* o, int o_dtype, const float* lse,
+                     const void* dout, float* dq, float* dk, float* dv,
+                     float* dkb, float* dvb, float scale, void* ws,
+                     size_t ws_bytes, void* stream);
+
+/* Per-CTA busy time of the last splitkv_attn_fwd (which = SPLITKV_WS_FWD) or
+ * backward partial kernel (SPLITKV_WS_BWD) on this plan: out_ns[w] = end - start
+ * of worker w's CTA in nanoseconds (device global timer), for the schedule's
+ * worker count.  Synchronises `stream`.  Errors: INVALID_ARG, NOT_UPLOADED,
+ * WORKSPACE_TOO_SMALL (capacity below the worker count), CUDA. */
+int splitkv_read_cta_times(const splitkv_plan_t* plan, int which, int64_t* out_ns,
+                           int64_t capacity, void* stream);
+
+#ifdef __cplusplus
+}  /* extern "C" */
+#endif
+
+#endif  /* SPLITKV_H_ */

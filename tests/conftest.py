@@ -11,3 +11,21 @@ if ROOT not in sys.path:
 def pytest_configure(config):
     config.addinivalue_line("markers", "gpu: needs a CUDA device (B200, sm_100a)")
     config.addinivalue_line("markers", "slow: long-running CPU test")
+
+
+@pytest.fixture(scope="session")
+def splitkv():
+    """The Python binding with libsplitkv.so built in-tree (nvcc cross-compiles; no GPU needed)."""
+    from context_block_sparse_b200 import build as _build
+    if not os.path.exists(_build.LIB):
+        _build.build()
+    import context_block_sparse_b200 as skv
+    return skv
+
+
+def gpu_available():
+    try:
+        import torch
+        return torch.cuda.is_available()
+    except Exception:
+        return False

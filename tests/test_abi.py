@@ -1,0 +1,62 @@
+"""The C-ABI library loads and exports exactly what include/splitkv.h declares (CPU only, no CUDA calls)."""
+
+import ctypes
+import os
+import re
+
+from context_block_sparse_b200 import _abi
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    src = open(os.path.join(ROOT, "include", "splitkv.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(splitkv_\w+)\s*\(", src)))
+
+
+def test_header_declarations_are_exported(splitkv):
+    names = _declared()
+    assert len(names) >= 12
+    lib = ctypes.CDLL(_abi.LIB_PATH)
+    for n in names:
+        assert hasattr(lib, n), n
+    assert sorted(_abi.SIGNATURES) == names
+
+
+def test_only_splitkv_symbols_exported(splitkv):
+    import subprocess
+    out = subprocess.run(["nm", "-D", "--defined-only", _abi.LIB_PATH], capture_output=True, text=True).stdout
+    syms = [l.split()[-1] for l in out.splitlines() if l.strip()]
+    funcs = [s for s in syms if not s.startswith("splitkv_")]
+    assert funcs == [] or all(s.startswith(("_init", "_fini")) for s in funcs), funcs
+
+
+def test_error_strings(splitkv):
+    lib = splitkv._lib
+    for code in range(0, -8, -1):
+        s = lib.splitkv_error_string(code).decode()
+        assert s and s != "unknown status"
+    assert lib.splitkv_error_string(-99).decode() == "unknown status"
+
+
+def _c_layout(struct, fields, tmp_path):
+    """sizeof and field offsets of a header struct, as gcc lays it out."""
+    import subprocess
+    body = "".join(f'  printf("%zu\\n", offsetof({struct}, {f}));\n' for f in fields)
+    src = (f'#include <stddef.h>\n#include <stdio.h>\n#include "splitkv.h"\n'
+           f'int main(void) {{\n  printf("%zu\\n", sizeof({struct}));\n{body}  return 0;\n}}\n')
+    c = tmp_path / "layout.c"
+    c.write_text(src)
+    exe = tmp_path / "layout"
+    subprocess.run(["gcc", "-I", os.path.join(ROOT, "include"), str(c), "-o", str(exe)], check=True)
+    vals = [int(x) for x in subprocess.run([str(exe)], capture_output=True, text=True, check=True).stdout.split()]
+    return vals[0], vals[1:]
+
+
+def test_struct_layouts_match_header(tmp_path):
+    for struct, cls in (("splitkv_problem", _abi.Problem), ("splitkv_stats", _abi.Stats)):
+        fields = [f for f, _ in cls._fields_]
+        size, offs = _c_layout(struct, fields, tmp_path)
+        assert ctypes.sizeof(cls) == size, struct
+        assert [getattr(cls, f).offset for f in fields] == offs, struct

@@ -1,0 +1,153 @@
+"""Host planner (C++, through the C ABI) against the oracle: bit-exact (CPU only).
+
+Mask metadata and LPT schedules are integer computations, so the library's
+entries, pair counts, schedules and loads must equal the oracle's exactly
+(news page "Balance actual attention work"; digest Abstract).
+"""
+
+import numpy as np
+import pytest
+from hypothesis import given, settings, strategies as st
+
+from oracle import lpt as olpt
+from oracle import mask as omask
+from synth import CONFIGS, make_workload
+
+
+def _plan(skv, lens, anchors, bs, Hq, Hkv, d, C, W, Wb=0, q_slice=0, eq=False):
+    return skv.splitkv_plan(lens, anchors, bs, Hq, Hkv, d, C, W, num_bwd_workers=Wb, q_slice=q_slice,
+                            equal_count=eq)
+
+
+def _check_against_oracle(skv, lens, anchors, bs, Hq, Hkv, C, W, Wb=0, q_slice=0, eq=False, d=64):
+    plan = _plan(skv, lens, anchors, bs, Hq, Hkv, d, C, W, Wb, q_slice, eq)
+    G = Hq // Hkv
+    # entries: same set per chunk, record order sorted by (lo, hi, block) inside each chunk
+    ent = plan.export(skv.EXPORT_ENTRIES).reshape(-1, 4)
+    want = omask.chunk_entries(lens, anchors, C)
+    assert sorted(map(tuple, ent.tolist())) == sorted(want)
+    keys = [(c, lo, hi, b) for (c, b, lo, hi) in ent.tolist()]
+    assert keys == sorted(keys)
+    # pair counts
+    pairs = plan.export(skv.EXPORT_CHUNK_PAIRS)
+    assert pairs.tolist() == omask.chunk_pairs(lens, anchors, bs, C).tolist()
+    # forward schedule (possibly sliced) and backward schedule (whole chunks)
+    for what, loads_what, workers, qs in ((skv.EXPORT_FWD_SCHEDULE, skv.EXPORT_FWD_LOADS, W, q_slice),
+                                          (skv.EXPORT_BWD_SCHEDULE, skv.EXPORT_BWD_LOADS, Wb or W, 0)):
+        items = olpt.work_items(lens, anchors, bs, C, Hq, Hkv, q_slice=qs, rows_per_tile=128)
+        lists, loads = olpt.lpt(items, workers, equal_count=eq)
+        cost = dict(items)
+        sched = plan.export(what).reshape(-1, 5)
+        got = [[] for _ in range(workers)]
+        for w, c, g, s, cst in sched.tolist():
+            got[w].append((c, g, s))
+            assert cst == cost[(c, g, s)]
+        assert got == [list(l) for l in lists]
+        assert plan.export(loads_what).tolist() == loads
+    # contiguous baseline
+    _, cl = olpt.contiguous(olpt.work_items(lens, anchors, bs, C, Hq, Hkv), W)
+    assert plan.export(skv.EXPORT_CONTIG_LOADS).tolist() == cl
+    st_ = plan.stats()
+    assert st_["context_pairs"] == Hq * int(pairs.sum())
+    assert st_["block_pairs"] == Hq * len(anchors) * bs * bs
+    _, fl = olpt.lpt(olpt.work_items(lens, anchors, bs, C, Hq, Hkv, q_slice=q_slice), W, equal_count=eq)
+    assert abs(st_["fwd_imbalance"] - olpt.imbalance(fl)) < 1e-12
+    assert abs(st_["contig_imbalance"] - olpt.imbalance(cl)) < 1e-12
+    plan.destroy()
+
+
+@settings(max_examples=120, deadline=None)
+@given(
+    lens=st.lists(st.integers(1, 300), min_size=1, max_size=6),
+    n_anchor=st.integers(1, 40),
+    heads=st.sampled_from([(1, 1), (2, 1), (4, 1), (4, 2), (8, 2), (32, 8)]),
+    bs=st.sampled_from([1, 2, 4, 8, 16]),
+    C=st.integers(1, 200),
+    W=st.integers(1, 20),
+    Wb=st.integers(0, 9),
+    q_slice=st.integers(0, 3),
+    eq=st.booleans(),
+    seed=st.integers(0, 2 ** 31 - 1),
+)
+def test_random_problems_bit_exact(splitkv, lens, n_anchor, heads, bs, C, W, Wb, q_slice, eq, seed):
+    Hq, Hkv = heads
+    if 128 % ((Hq // Hkv) * bs):
+        return
+    rng = np.random.default_rng(seed)
+    N = sum(lens)
+    anchors = rng.integers(0, N, size=n_anchor).astype(np.int32)   # any order, repeats allowed
+    _check_against_oracle(splitkv, lens, anchors, bs, Hq, Hkv, C, W, Wb, q_slice, eq)
+
+
+@pytest.mark.parametrize("name", ["tiny", "drafter", "budget", "skew", "bwd"])
+@pytest.mark.parametrize("q_slice,eq", [(0, False), (2, False), (0, True)])
+def test_workload_plans_bit_exact(splitkv, name, q_slice, eq):
+    w = make_workload(name, tensors=False)
+    _check_against_oracle(splitkv, w.sample_lens, w.anchors, w.block_size, w.num_q_heads, w.num_kv_heads,
+                          w.kv_chunk, 148, 0, q_slice, eq, d=w.head_dim)
+
+
+def test_anchor_at_sample_start_and_chunk_straddle(splitkv):
+    _check_against_oracle(splitkv, [4, 4, 9], [0, 4, 5, 16, 8], 2, 2, 1, 3, 2)
+
+
+@pytest.mark.parametrize("bad", [
+    dict(lens=[0, 5]), dict(lens=[-1]), dict(anchors=[9]), dict(anchors=[-1]),
+    dict(Hq=3, Hkv=2), dict(bs=0), dict(C=0), dict(W=0), dict(Wb=-1), dict(q_slice=-1),
+])
+def test_invalid_problems_rejected(splitkv, bad):
+    a = dict(lens=[5, 4], anchors=[3, 7], bs=4, Hq=2, Hkv=1, d=64, C=4, W=2, Wb=0, q_slice=0)
+    a.update(bad)
+    with pytest.raises(splitkv.SplitKVError) as ei:
+        _plan(splitkv, a["lens"], a["anchors"], a["bs"], a["Hq"], a["Hkv"], a["d"], a["C"], a["W"], a["Wb"],
+              a["q_slice"])
+    assert ei.value.status == -1
+
+
+def test_unsupported_tile_shape(splitkv):
+    # G * bs must divide the 128-row query tile
+    with pytest.raises(splitkv.SplitKVError) as ei:
+        _plan(splitkv, [50], [10], 3, 2, 1, 64, 8, 4)
+    assert ei.value.status == -2
+
+
+def test_attention_calls_need_an_uploaded_plan(splitkv):
+    """Host-side checks only: a plan without a device copy is refused before any CUDA call."""
+    import ctypes
+    plan = _plan(splitkv, [64, 64], [10, 70], 16, 1, 1, 64, 32, 4)
+    lib = splitkv._lib
+    fake = ctypes.c_void_p(16)
+    assert lib.splitkv_attn_fwd(plan.handle, fake, fake, fake, 1.0, fake, 1 << 20, None) == -6
+    assert lib.splitkv_merge(plan.handle, fake, fake, fake, 1.0, fake, 1 << 20, fake, 0, fake, None) == -6
+    assert lib.splitkv_attn_bwd(plan.handle, *([fake] * 6), 0, fake, fake, *([fake] * 5), 1.0, fake, 1 << 20,
+                                None) == -6
+    assert lib.splitkv_attn_fwd(None, fake, fake, fake, 1.0, fake, 1 << 20, None) == -1
+    plan.destroy()
+
+
+def test_update_in_place_matches_fresh_plan(splitkv):
+    w1 = make_workload("drafter", tensors=False)
+    w2 = make_workload("drafter", tensors=False, seed=7)
+    p = _plan(splitkv, w1.sample_lens, w1.anchors, 16, 32, 8, 128, 256, 148)
+    splitkv.splitkv_plan_update(p, w2.sample_lens, w2.anchors)
+    q = _plan(splitkv, w2.sample_lens, w2.anchors, 16, 32, 8, 128, 256, 148)
+    for what in range(7):
+        assert np.array_equal(p.export(what), q.export(what)), what
+
+
+def test_workspace_sizes(splitkv):
+    w = make_workload("tiny", tensors=False)
+    p = _plan(splitkv, w.sample_lens, w.anchors, 16, 1, 1, 64, 128, 148)
+    E = p.stats()["num_entries"]
+    fwd = splitkv.splitkv_workspace_size(p, splitkv.WS_FWD)
+    bwd = splitkv.splitkv_workspace_size(p, splitkv.WS_BWD)
+    assert fwd >= E * 16 * 1 * 64 * 4 + 2 * E * 16 * 4
+    assert bwd >= E * 16 * 64 * 4 + 128 * 4
+
+
+def test_lpt_beats_contiguous_on_skew(splitkv):
+    w = make_workload("skew", tensors=False)
+    p = _plan(splitkv, w.sample_lens, w.anchors, 16, 32, 8, 128, 512, 148)
+    st_ = p.stats()
+    assert st_["fwd_imbalance"] < 0.05
+    assert st_["contig_imbalance"] > 1.0
