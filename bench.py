@@ -1,0 +1,505 @@
+#!/usr/bin/env python
+"""Throughput of one Split-KV anchor-attention training step on B200.
+
+A step is one pass of the whole path over one batch of synthetic input:
+  host plan (mask metadata + LPT) -> plan upload -> chunk partial forward ->
+  merge (in-block term + exact LSE combine) -> backward Delta -> chunk partial
+  backward (dK, dV local per chunk, dQ partials) -> dQ reduce + in-block backward.
+
+Default workload (N=1): 32 query / 8 KV heads, head_dim 128, a 65536-token
+packed context (sample lengths uniform in [2048, 16384]), 512 anchors x 16 =
+8192 draft queries, KV chunk 512, bf16 inputs drawn N(0,1), fp32 outputs.
+
+Metric: masked-pair TFLOP/s = (4 + 10) * d * (allowed (query, key, head)
+pairs) per step / step time; allowed pairs are counted exactly (context pairs
+from the plan plus the in-block pairs).  Timing: CUDA events on the launch
+stream, W untimed warm-up steps, barrier + synchronize around K timed steps,
+max over ranks.  Every step's inputs and outputs (~4 GB with the workspaces)
+exceed the 126 MB L2, so no flush is needed between steps.
+
+With --gpus N > 1 (torchrun, one process per GPU) every rank runs an
+independent replica of the workload (the path has no exchange step on one
+GPU: replicas only), and the value is the sum of their work over the max time.
+
+--impl reference times the fp64 CPU oracle on a bounded sample of the same
+workload (rank 0 only).
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "masked-pair attn TFLOP/s fwd/bwd, % of BF16 tensor peak; LPT imbalance %"
+
+# DRAM bytes per launch from ncu captures (dram__bytes_read.sum + dram__bytes_write.sum),
+# keyed by kernel, with the sha256 of the kernel source they were taken on; a
+# changed source voids the figure.
+NCU_TRAFFIC = {}
+
+
+def _src_hash(name: str) -> str:
+    path = os.path.join(ROOT, "context_block_sparse_b200", "csrc", name)
+    with open(path, "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def _peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return {"hbm_gbs": float(d["hbm_gbs"]), "bf16_tflops": float(d["bf16_tflops"]),
+                "bf16_tflops_sustained": float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
+                "source": "measured"}
+    except Exception:
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples while the timed region runs."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str):
+        self.gpu_id = gpu_id
+        self.rows = []
+        self.proc = None
+        self.t = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", self.gpu_id, f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+            return
+        self.t = threading.Thread(target=self._read, daemon=True)
+        self.t.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) == 7:
+                self.rows.append((time.time(), parts))
+
+    def stop(self):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self, t0: float, t1: float):
+        rows = [r for (t, r) in self.rows if t0 - 0.15 <= t <= t1 + 0.15] or [r for (_, r) in self.rows]
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+
+        def num(x):
+            try:
+                return float(x)
+            except ValueError:
+                return None
+
+        sm = [num(r[0]) for r in rows if num(r[0]) is not None]
+        mx = [num(r[1]) for r in rows if num(r[1]) is not None]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[3 + i].lower() == "active"})
+        return {"sm_mhz": float(np.median(sm)) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+def _dist():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+# ---------------------------------------------------------------------------
+# our arm
+# ---------------------------------------------------------------------------
+
+def _kernel_work(st, w, E):
+    """Algorithmic FLOPs or bytes of one launch of each kernel."""
+    d, Hq, Hkv, bs, Nq = w.head_dim, w.num_q_heads, w.num_kv_heads, w.block_size, w.num_queries
+    ctx = st["context_pairs"]
+    rec_rows = E * bs * Hq
+    return {
+        "fwd_partial": ("tensor", 4.0 * d * ctx),
+        "bwd_partial": ("tensor", 10.0 * d * ctx),
+        # partial records (O_c, m, l) read; o, lse written; q, kb, vb read once
+        "merge": ("hbm", rec_rows * (4.0 * d + 8) + Nq * Hq * (4.0 * d + 4) + Nq * Hq * d * 2.0
+                  + 2.0 * Nq * Hkv * d * 2),
+        # o (fp32) and dout read, Delta written
+        "bwd_delta": ("hbm", Nq * Hq * d * (4.0 + 2.0) + Nq * Hq * 4.0),
+        # dq partials read; q, dout, kb, vb, lse, Delta read; dq, dkb, dvb written
+        "bwd_reduce": ("hbm", rec_rows * d * 4.0 + Nq * Hq * (d * 4.0 + 8) + Nq * Hq * d * 4.0
+                       + 2.0 * Nq * Hkv * d * 2 + 2.0 * Nq * Hkv * d * 4),
+    }
+
+
+def run_ours(args, world, rank, local):
+    import torch
+    import torch.distributed as dist
+
+    import context_block_sparse_b200 as skv
+    from synth import make_workload
+
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=180), device_id=dev)
+
+    w = make_workload(args.workload, num_anchors=args.anchors, with_grad=True)
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    W = args.workers or sms
+    Wb = args.bwd_workers or 2 * sms
+    stream = torch.cuda.current_stream(dev)
+
+    def up(name):
+        return torch.from_numpy(w.bits[name].view(np.int16)).view(torch.bfloat16).to(dev)
+
+    t = {n: up(n) for n in ("q", "k", "v", "kb", "vb", "dout")}
+    d, Hq, Nq = w.head_dim, w.num_q_heads, w.num_queries
+    plan = skv.splitkv_plan(w.sample_lens, w.anchors, w.block_size, Hq, w.num_kv_heads, d, w.kv_chunk, W,
+                            num_bwd_workers=Wb, q_slice=args.q_slice)
+    plan.upload(stream)
+    st = plan.stats()
+    ws_f = torch.empty(skv.splitkv_workspace_size(plan, skv.WS_FWD), dtype=torch.uint8, device=dev)
+    ws_b = torch.empty(skv.splitkv_workspace_size(plan, skv.WS_BWD), dtype=torch.uint8, device=dev)
+    f32 = dict(dtype=torch.float32, device=dev)
+    o = torch.empty((Nq, Hq, d), **f32)
+    lse = torch.empty((Nq, Hq), **f32)
+    g = {"dq": torch.empty(t["q"].shape, **f32), "dk": torch.empty(t["k"].shape, **f32),
+         "dv": torch.empty(t["v"].shape, **f32), "dkb": torch.empty(t["kb"].shape, **f32),
+         "dvb": torch.empty(t["vb"].shape, **f32)}
+    kernels = ["fwd_partial", "merge", "bwd_delta", "bwd_partial", "bwd_reduce"]
+    plan_us = []
+
+    def step(ev=None):
+        skv.splitkv_plan_update(plan, w.sample_lens, w.anchors)
+        plan_us.append(plan.stats()["plan_us"])
+        plan.upload(stream)
+        if ev is not None:
+            ev[0].record(stream)
+        skv.splitkv_attn_fwd(plan, t["q"], t["k"], t["v"], w.scale, ws_f, stream)
+        if ev is not None:
+            ev[1].record(stream)
+        skv.splitkv_merge(plan, t["q"], t["kb"], t["vb"], w.scale, ws_f, o, lse, stream)
+        if ev is not None:
+            ev[2].record(stream)
+        skv.splitkv_bwd_delta(plan, o, t["dout"], ws_b, stream)
+        if ev is not None:
+            ev[3].record(stream)
+        skv.splitkv_bwd_partial(plan, t["q"], t["k"], t["v"], lse, t["dout"], g["dk"], g["dv"], w.scale, ws_b,
+                                stream)
+        if ev is not None:
+            ev[4].record(stream)
+        skv.splitkv_bwd_reduce(plan, t["q"], t["kb"], t["vb"], lse, t["dout"], g["dq"], g["dkb"], g["dvb"],
+                               w.scale, ws_b, stream)
+        if ev is not None:
+            ev[5].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+
+    sampler = None
+    if rank == 0 and not args.no_clocks:
+        props = torch.cuda.get_device_properties(dev)
+        sampler = ClockSampler("GPU-" + str(props.uuid))
+        sampler.start()
+        time.sleep(0.3)
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(args.steps)]
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    plan_us.clear()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    wall0 = time.time()
+    start.record(stream)
+    for i in range(args.steps):
+        step(evs[i])
+    end.record(stream)
+    torch.cuda.synchronize(dev)
+    wall1 = time.time()
+    if world > 1:
+        dist.barrier()
+    ms = start.elapsed_time(end)
+    if world > 1:
+        x = torch.tensor([ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(x, op=dist.ReduceOp.MAX)
+        ms = float(x.item())
+    per_kernel = {k: float(np.mean([evs[i][j].elapsed_time(evs[i][j + 1]) for i in range(args.steps)]))
+                  for j, k in enumerate(kernels)}
+    clocks = sampler.summary(wall0, wall1) if sampler else {"sm_mhz": None, "sm_max_mhz": None,
+                                                              "reasons": ["unsampled"]}
+    if sampler:
+        sampler.stop()
+
+    # measured per-CTA busy time of the last step (untimed read)
+    cta_f = skv.splitkv_read_cta_times(plan, skv.WS_FWD, stream)
+    cta_b = skv.splitkv_read_cta_times(plan, skv.WS_BWD, stream)
+
+    def imb(x):
+        x = np.asarray(x, dtype=np.float64)
+        return float(x.max() / x.mean() - 1.0) if x.size and x.mean() > 0 else 0.0
+
+    pairs = st["context_pairs"] + st["block_pairs"]
+    flops_fwd = 4.0 * d * pairs
+    flops_bwd = 10.0 * d * pairs
+    flops_step = flops_fwd + flops_bwd
+    value = world * args.steps * flops_step / (ms * 1e-3) / 1e12
+    peaks = _peaks()
+    work = _kernel_work(st, w, st["num_entries"])
+    dom = max(kernels, key=lambda k: per_kernel[k])
+    bound, amount = work[dom]
+    dom_s = per_kernel[dom] * 1e-3
+    src_file = {"fwd_partial": "fwd_partial_mma.cu", "bwd_partial": "bwd_partial_mma.cu"}.get(dom, "merge.cu")
+    tr = NCU_TRAFFIC.get(dom)
+    traffic = tr["bytes"] if tr and tr.get("src") == _src_hash(src_file) else None
+    if bound == "tensor":
+        achieved = amount / dom_s / 1e12
+        roof = {"kernel": dom, "bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"],
+                "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops"], "traffic": traffic,
+                "peak_source": f"{peaks['source']} bf16 (burst)", "launch_ms": per_kernel[dom]}
+    else:
+        achieved = amount / dom_s / 1e9
+        roof = {"kernel": dom, "bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": achieved / peaks["hbm_gbs"], "traffic": traffic,
+                "peak_source": f"{peaks['source']} copy", "launch_ms": per_kernel[dom]}
+    kern = {}
+    for k in kernels:
+        b_, a_ = work[k]
+        s_ = per_kernel[k] * 1e-3
+        kern[k] = {"ms": per_kernel[k],
+                   ("tflops" if b_ == "tensor" else "gbs"): (a_ / s_ / 1e12 if b_ == "tensor" else a_ / s_ / 1e9)}
+    fwd_ms = per_kernel["fwd_partial"] + per_kernel["merge"]
+    bwd_ms = per_kernel["bwd_delta"] + per_kernel["bwd_partial"] + per_kernel["bwd_reduce"]
+
+    result = {
+        "metric": METRIC,
+        "value": value,
+        "unit": "TFLOP/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": ms / args.steps,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": w.config.description, "context_len": w.context_len, "num_queries": Nq,
+                   "num_anchors": int(w.anchors.size), "block_size": w.block_size, "heads": [Hq, w.num_kv_heads],
+                   "head_dim": d, "kv_chunk": w.kv_chunk, "fwd_workers": W, "bwd_workers": Wb,
+                   "q_slice": args.q_slice, "parallelism": "replicas" if world > 1 else "single",
+                   "l2": "no flush: each step touches ~4 GB (> 126 MB L2)"},
+        "fwd_tflops": flops_fwd / (fwd_ms * 1e-3) / 1e12,
+        "bwd_tflops": flops_bwd / (bwd_ms * 1e-3) / 1e12,
+        "pct_of_bf16_peak": 100.0 * value / world / peaks["bf16_tflops"],
+        "lpt_imbalance_pct": {"fwd_plan": 100 * st["fwd_imbalance"], "bwd_plan": 100 * st["bwd_imbalance"],
+                              "contiguous_plan": 100 * st["contig_imbalance"], "fwd_measured": 100 * imb(cta_f),
+                              "bwd_measured": 100 * imb(cta_b)},
+        "plan_us": float(np.median(plan_us)) if plan_us else None,
+        "kernels": kern,
+        "roofline": roof,
+        "gpu_launches": len(kernels) * args.steps,
+        "clocks": clocks,
+    }
+
+    if not args.no_e2e:
+        result["e2e"] = run_e2e(args, w, plan, dev, stream, flops_step, world=world)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        result["cpu_baseline"] = cpu_baseline(w, budget_s=args.cpu_seconds)
+    if world > 1:
+        dist.destroy_process_group()
+    return result if rank == 0 else None
+
+
+def run_e2e(args, w, plan, dev, stream, flops_step, world=1):
+    """Same metric through the public API from pinned HOST buffers: every step copies its inputs in and
+    its results (o, lse, dq, dk, dv, dkb, dvb) out inside the timed region."""
+    import torch
+    import torch.distributed as dist
+
+    import context_block_sparse_b200 as skv
+    from context_block_sparse_b200.torch_api import SplitKVAttention
+
+    host = {n: torch.from_numpy(w.bits[n].view(np.int16)).view(torch.bfloat16).pin_memory()
+            for n in ("q", "k", "v", "kb", "vb", "dout")}
+    d, Hq, Nq = w.head_dim, w.num_q_heads, w.num_queries
+    att = SplitKVAttention(w.sample_lens, w.anchors, w.block_size, Hq, w.num_kv_heads, d, w.kv_chunk,
+                           num_workers=plan.problem.num_workers, num_bwd_workers=plan.problem.num_bwd_workers,
+                           device=dev)
+    dv = {n: torch.empty(x.shape, dtype=x.dtype, device=dev) for n, x in host.items()}
+    outs_h = {"o": torch.empty((Nq, Hq, d), dtype=torch.float32).pin_memory(),
+              "lse": torch.empty((Nq, Hq), dtype=torch.float32).pin_memory()}
+    for n in ("q", "k", "v", "kb", "vb"):
+        outs_h["d" + n] = torch.empty(host[n].shape, dtype=torch.float32).pin_memory()
+    h2d = sum(x.numel() * x.element_size() for x in host.values()) + 4 * (w.sample_lens.size + w.anchors.size)
+    d2h = sum(x.numel() * x.element_size() for x in outs_h.values())
+    steps = max(1, min(args.steps, args.e2e_steps))
+
+    def step():
+        for n in host:
+            dv[n].copy_(host[n], non_blocking=True)
+        skv.splitkv_plan_update(att.plan, w.sample_lens, w.anchors)
+        att.plan.upload(stream)
+        o, lse = att.forward(dv["q"], dv["k"], dv["v"], dv["kb"], dv["vb"], w.scale)
+        g = att.backward(dv["q"], dv["k"], dv["v"], dv["kb"], dv["vb"], o, lse, dv["dout"], w.scale)
+        outs_h["o"].copy_(o, non_blocking=True)
+        outs_h["lse"].copy_(lse, non_blocking=True)
+        for n, x in g.items():
+            outs_h[n].copy_(x, non_blocking=True)
+
+    for _ in range(2):
+        step()
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(steps):
+        step()
+    b.record(stream)
+    torch.cuda.synchronize(dev)
+    ms = a.elapsed_time(b)
+    if world > 1:
+        x = torch.tensor([ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(x, op=dist.ReduceOp.MAX)
+        ms = float(x.item())
+        dist.barrier()
+    return {"value": world * steps * flops_step / (ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+            "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "steps": steps,
+            "ms_per_step": ms / steps}
+
+
+# ---------------------------------------------------------------------------
+# the fp64 CPU oracle, timed on a bounded sample of the same workload
+# ---------------------------------------------------------------------------
+
+def _oracle_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return int(max(n)) if n else 1
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def _oracle_blocks(w, budget_s: float, start: int = 0, stride: int = 37):
+    """Run the oracle forward + backward block by block until budget_s elapses; returns (flops, seconds, n)."""
+    from oracle import attention as oatt
+    from oracle import mask as omask
+    f = {n: w.f64(n) for n in ("q", "k", "v", "kb", "vb", "dout")}
+    iv = omask.context_interval(w.sample_lens, w.anchors)
+    A = len(iv)
+    flops = 0.0
+    n = 0
+    t0 = time.perf_counter()
+    b = start % A
+    while True:
+        oatt.attention_fwd(f["q"], f["k"], f["v"], f["kb"], f["vb"], w.sample_lens, w.anchors, w.block_size,
+                           w.scale, blocks=[b])
+        oatt.attention_bwd(f["q"], f["k"], f["v"], f["kb"], f["vb"], f["dout"], w.sample_lens, w.anchors,
+                           w.block_size, w.scale, blocks=[b])
+        S, a = iv[b]
+        flops += 14.0 * w.head_dim * w.num_q_heads * w.block_size * ((a - S) + w.block_size)
+        n += 1
+        b = (b + stride) % A
+        if time.perf_counter() - t0 >= budget_s:
+            break
+    return flops, time.perf_counter() - t0, n
+
+
+def cpu_baseline(w, budget_s=15.0):
+    flops, secs, n = _oracle_blocks(w, budget_s)
+    return {"value": flops / secs / 1e12, "unit": "TFLOP/s", "cores": _oracle_threads(), "kind": "oracle",
+            "sample": f"fp64 numpy oracle, forward + backward of {n} of {w.anchors.size} anchor blocks "
+                      f"(every 37th, all {w.num_q_heads} heads), {secs:.1f} s; same masked-pair FLOP count",
+            "host_cpu_count": os.cpu_count()}
+
+
+def run_reference(args, world, rank):
+    from synth import make_workload
+    if rank != 0:
+        return None
+    w = make_workload(args.workload, num_anchors=args.anchors, with_grad=True)
+    per_step = max(0.2, min(args.cpu_seconds, 120.0) / max(1, args.steps + args.warmup))
+    for i in range(args.warmup):
+        _oracle_blocks(w, per_step, start=i)
+    flops = secs = 0.0
+    n = 0
+    for i in range(args.steps):
+        f_, s_, n_ = _oracle_blocks(w, per_step, start=1000 + 7 * i)
+        flops += f_
+        secs += s_
+        n += n_
+    value = flops / secs / 1e12
+    sample = (f"fp64 numpy oracle, forward + backward of {n} anchor blocks over {args.steps} steps "
+              f"(about {per_step:.1f} s each) of the {args.workload} workload")
+    return {"impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * secs / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic",
+            "config": {"workload": w.config.description, "context_len": w.context_len,
+                       "num_queries": w.num_queries, "parallelism": "single"},
+            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": _oracle_threads(), "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+            "gpu_launches": 0}
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="bwd", choices=["tiny", "drafter", "budget", "skew", "bwd"])
+    ap.add_argument("--anchors", type=int, default=None)
+    ap.add_argument("--workers", type=int, default=0, help="forward CTAs (default: SM count)")
+    ap.add_argument("--bwd-workers", type=int, default=0, help="backward CTAs (default: 2 x SM count)")
+    ap.add_argument("--q-slice", type=int, default=0)
+    ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-clocks", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+    world, rank, local = _dist()
+    if world != args.gpus:
+        print(f"warning: --gpus {args.gpus} but WORLD_SIZE={world}", file=sys.stderr)
+    if args.impl == "reference":
+        res = run_reference(args, world, rank)
+    else:
+        res = run_ours(args, world, rank, local)
+    if res is not None:
+        print(json.dumps(res), flush=True)
+
+
+if __name__ == "__main__":
+    main()

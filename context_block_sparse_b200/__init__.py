@@ -218,6 +218,25 @@ def splitkv_attn_bwd(plan: Plan, q, k, v, kb, vb, o, lse, dout, dq, dk, dv, dkb,
         _f32_ptr(dvb), float(scale), _ptr(ws), ws.numel() * ws.element_size(), _stream_ptr(stream)))
 
 
+def splitkv_bwd_delta(plan: Plan, o, dout, ws, stream=None) -> None:
+    _check("splitkv_bwd_delta", _lib.splitkv_bwd_delta(
+        plan.handle, _ptr(o), _o_dtype(o), _bf16_ptr(dout), _ptr(ws), ws.numel() * ws.element_size(),
+        _stream_ptr(stream)))
+
+
+def splitkv_bwd_partial(plan: Plan, q, k, v, lse, dout, dk, dv, scale: float, ws, stream=None) -> None:
+    _check("splitkv_bwd_partial", _lib.splitkv_bwd_partial(
+        plan.handle, _bf16_ptr(q), _bf16_ptr(k), _bf16_ptr(v), _f32_ptr(lse), _bf16_ptr(dout), _f32_ptr(dk),
+        _f32_ptr(dv), float(scale), _ptr(ws), ws.numel() * ws.element_size(), _stream_ptr(stream)))
+
+
+def splitkv_bwd_reduce(plan: Plan, q, kb, vb, lse, dout, dq, dkb, dvb, scale: float, ws, stream=None) -> None:
+    _check("splitkv_bwd_reduce", _lib.splitkv_bwd_reduce(
+        plan.handle, _bf16_ptr(q), _bf16_ptr(kb), _bf16_ptr(vb), _f32_ptr(lse), _bf16_ptr(dout), _f32_ptr(dq),
+        _f32_ptr(dkb), _f32_ptr(dvb), float(scale), _ptr(ws), ws.numel() * ws.element_size(),
+        _stream_ptr(stream)))
+
+
 def splitkv_read_cta_times(plan: Plan, which: int, stream=None) -> np.ndarray:
     """Per-CTA busy nanoseconds of the last forward (WS_FWD) or backward (WS_BWD) partial kernel."""
     st = plan.stats()

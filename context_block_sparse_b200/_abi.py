@@ -99,6 +99,9 @@ SIGNATURES = {
     "splitkv_attn_fwd": (_I, [_P, _P, _P, _P, _F, _P, _SZ, _P]),
     "splitkv_merge": (_I, [_P, _P, _P, _P, _F, _P, _SZ, _P, _I, _P, _P]),
     "splitkv_attn_bwd": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _P, _P, _P, _P, _P, _P, _P, _F, _P, _SZ, _P]),
+    "splitkv_bwd_delta": (_I, [_P, _P, _I, _P, _P, _SZ, _P]),
+    "splitkv_bwd_partial": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _F, _P, _SZ, _P]),
+    "splitkv_bwd_reduce": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _F, _P, _SZ, _P]),
     "splitkv_read_cta_times": (_I, [_P, _I, ctypes.POINTER(ctypes.c_int64), ctypes.c_int64, _P]),
 }
 

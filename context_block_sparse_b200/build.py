@@ -1,6 +1,8 @@
 """Build libsplitkv.so in-tree with nvcc for sm_100a (B200).
 
-    python -m context_block_sparse_b200.build [-v]
+    python context_block_sparse_b200/build.py [-v] [-f] [--ptxas]
+
+(Run it as a script: importing the package itself needs the built library.)
 
 Objects go to _build/ at the repository root; the shared library lands next
 to this file so the Python binding finds it.  Only splitkv_* symbols are

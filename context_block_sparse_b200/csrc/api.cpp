@@ -74,6 +74,54 @@ int splitkv_merge(const splitkv_plan_t* plan, const void* q, const void* kb, con
       static_cast<cudaStream_t>(stream)));
 }
 
+int splitkv_bwd_delta(const splitkv_plan_t* plan, const void* o, int o_dtype, const void* dout, void* ws,
+                      size_t ws_bytes, void* stream) {
+  const DevPlan* dp = nullptr;
+  int st = check_plan(plan, &dp);
+  if (st != SPLITKV_OK) return st;
+  if (!all_aligned16(o, dout, ws)) return SPLITKV_ERR_INVALID_ARG;
+  if (o_dtype != SPLITKV_DTYPE_F32 && o_dtype != SPLITKV_DTYPE_BF16) return SPLITKV_ERR_INVALID_ARG;
+  const splitkv::BwdWs L = splitkv::bwd_ws_layout(dp->E, dp->Nq, dp->bs, dp->Hq, dp->d);
+  if (ws_bytes < L.total) return SPLITKV_ERR_WORKSPACE_TOO_SMALL;
+  float* delta = reinterpret_cast<float*>(static_cast<char*>(ws) + L.delta_off);
+  return cuda_status(splitkv::launch_bwd_delta(*dp, o, o_dtype == SPLITKV_DTYPE_BF16 ? 1 : 0,
+                                               static_cast<const uint16_t*>(dout), delta,
+                                               static_cast<cudaStream_t>(stream)));
+}
+
+int splitkv_bwd_partial(const splitkv_plan_t* plan, const void* q, const void* k, const void* v, const float* lse,
+                        const void* dout, float* dk, float* dv, float scale, void* ws, size_t ws_bytes,
+                        void* stream) {
+  const DevPlan* dp = nullptr;
+  int st = check_plan(plan, &dp);
+  if (st != SPLITKV_OK) return st;
+  if (!all_aligned16(q, k, v, dout, dk, dv, ws) || !lse || !aligned(lse, 4)) return SPLITKV_ERR_INVALID_ARG;
+  const splitkv::BwdWs L = splitkv::bwd_ws_layout(dp->E, dp->Nq, dp->bs, dp->Hq, dp->d);
+  if (ws_bytes < L.total) return SPLITKV_ERR_WORKSPACE_TOO_SMALL;
+  char* w = static_cast<char*>(ws);
+  return cuda_status(splitkv::launch_bwd_partial(
+      *dp, static_cast<const uint16_t*>(q), static_cast<const uint16_t*>(k), static_cast<const uint16_t*>(v),
+      static_cast<const uint16_t*>(dout), lse, reinterpret_cast<const float*>(w + L.delta_off), scale, dk, dv,
+      reinterpret_cast<float*>(w + L.dq_off), static_cast<cudaStream_t>(stream)));
+}
+
+int splitkv_bwd_reduce(const splitkv_plan_t* plan, const void* q, const void* kb, const void* vb, const float* lse,
+                       const void* dout, float* dq, float* dkb, float* dvb, float scale, const void* ws,
+                       size_t ws_bytes, void* stream) {
+  const DevPlan* dp = nullptr;
+  int st = check_plan(plan, &dp);
+  if (st != SPLITKV_OK) return st;
+  if (!all_aligned16(q, kb, vb, dout, dq, dkb, dvb, ws) || !lse || !aligned(lse, 4))
+    return SPLITKV_ERR_INVALID_ARG;
+  const splitkv::BwdWs L = splitkv::bwd_ws_layout(dp->E, dp->Nq, dp->bs, dp->Hq, dp->d);
+  if (ws_bytes < L.total) return SPLITKV_ERR_WORKSPACE_TOO_SMALL;
+  const char* w = static_cast<const char*>(ws);
+  return cuda_status(splitkv::launch_bwd_reduce(
+      *dp, static_cast<const uint16_t*>(q), static_cast<const uint16_t*>(kb), static_cast<const uint16_t*>(vb),
+      static_cast<const uint16_t*>(dout), lse, reinterpret_cast<const float*>(w + L.delta_off),
+      reinterpret_cast<const float*>(w + L.dq_off), scale, dq, dkb, dvb, static_cast<cudaStream_t>(stream)));
+}
+
 int splitkv_attn_bwd(const splitkv_plan_t* plan, const void* q, const void* k, const void* v, const void* kb,
                      const void* vb, const void* o, int o_dtype, const float* lse, const void* dout, float* dq,
                      float* dk, float* dv, float* dkb, float* dvb, float scale, void* ws, size_t ws_bytes,
@@ -81,27 +129,17 @@ int splitkv_attn_bwd(const splitkv_plan_t* plan, const void* q, const void* k, c
   const DevPlan* dp = nullptr;
   int st = check_plan(plan, &dp);
   if (st != SPLITKV_OK) return st;
+  // check everything up front so that no launch happens on a call that fails
   if (!all_aligned16(q, k, v, kb, vb, o, dout, dq, dk, dv, dkb, dvb, ws) || !lse || !aligned(lse, 4))
     return SPLITKV_ERR_INVALID_ARG;
   if (o_dtype != SPLITKV_DTYPE_F32 && o_dtype != SPLITKV_DTYPE_BF16) return SPLITKV_ERR_INVALID_ARG;
   const splitkv::BwdWs L = splitkv::bwd_ws_layout(dp->E, dp->Nq, dp->bs, dp->Hq, dp->d);
   if (ws_bytes < L.total) return SPLITKV_ERR_WORKSPACE_TOO_SMALL;
-  char* w = static_cast<char*>(ws);
-  float* dq_part = reinterpret_cast<float*>(w + L.dq_off);
-  float* delta = reinterpret_cast<float*>(w + L.delta_off);
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-  const auto* q16 = static_cast<const uint16_t*>(q);
-  const auto* do16 = static_cast<const uint16_t*>(dout);
-  const int obf = o_dtype == SPLITKV_DTYPE_BF16 ? 1 : 0;
-  st = cuda_status(splitkv::launch_bwd_delta(*dp, o, obf, do16, delta, s));
+  st = splitkv_bwd_delta(plan, o, o_dtype, dout, ws, ws_bytes, stream);
   if (st != SPLITKV_OK) return st;
-  st = cuda_status(splitkv::launch_bwd_partial(*dp, q16, static_cast<const uint16_t*>(k),
-                                               static_cast<const uint16_t*>(v), do16, lse, delta, scale, dk, dv,
-                                               dq_part, s));
+  st = splitkv_bwd_partial(plan, q, k, v, lse, dout, dk, dv, scale, ws, ws_bytes, stream);
   if (st != SPLITKV_OK) return st;
-  return cuda_status(splitkv::launch_bwd_reduce(*dp, q16, static_cast<const uint16_t*>(kb),
-                                                static_cast<const uint16_t*>(vb), do16, lse, delta, dq_part,
-                                                scale, dq, dkb, dvb, s));
+  return splitkv_bwd_reduce(plan, q, kb, vb, lse, dout, dq, dkb, dvb, scale, ws, ws_bytes, stream);
 }
 
 int splitkv_read_cta_times(const splitkv_plan_t* plan, int which, int64_t* out_ns, int64_t capacity,

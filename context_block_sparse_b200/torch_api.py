@@ -1,0 +1,68 @@
+"""Convenience wrapper over the C entry points for torch users.
+
+Allocates the outputs and workspaces with torch (device memory only) and calls
+splitkv_attn_fwd / splitkv_merge / splitkv_attn_bwd in order on the current
+stream.  No arithmetic happens here.
+"""
+
+from __future__ import annotations
+
+from typing import Optional
+
+import torch
+
+from . import (
+    WS_BWD, WS_FWD, Plan, splitkv_attn_bwd, splitkv_attn_fwd, splitkv_merge, splitkv_plan,
+    splitkv_plan_upload, splitkv_workspace_size,
+)
+
+
+class SplitKVAttention:
+    """One problem (packed samples + anchors + head layout) bound to a device plan."""
+
+    def __init__(self, sample_lens, anchors, block_size: int, num_q_heads: int, num_kv_heads: int,
+                 head_dim: int, kv_chunk: int, num_workers: Optional[int] = None,
+                 num_bwd_workers: int = 0, q_slice: int = 0, equal_count: bool = False,
+                 device: Optional[torch.device] = None):
+        self.device = torch.device("cuda") if device is None else torch.device(device)
+        if num_workers is None:
+            num_workers = torch.cuda.get_device_properties(self.device).multi_processor_count
+        self.plan: Plan = splitkv_plan(sample_lens, anchors, block_size, num_q_heads, num_kv_heads, head_dim,
+                                       kv_chunk, num_workers, num_bwd_workers, q_slice, equal_count)
+        splitkv_plan_upload(self.plan)
+        self.block_size = block_size
+        self.num_q_heads = num_q_heads
+        self.num_kv_heads = num_kv_heads
+        self.head_dim = head_dim
+        self.ws_fwd = torch.empty(splitkv_workspace_size(self.plan, WS_FWD), dtype=torch.uint8, device=self.device)
+        self._ws_bwd = None
+
+    def ws_bwd(self) -> torch.Tensor:
+        if self._ws_bwd is None:
+            self._ws_bwd = torch.empty(splitkv_workspace_size(self.plan, WS_BWD), dtype=torch.uint8,
+                                       device=self.device)
+        return self._ws_bwd
+
+    def forward(self, q, k, v, kb, vb, scale: float, out_dtype=torch.float32, o=None, lse=None):
+        Nq = q.shape[0]
+        if o is None:
+            o = torch.empty((Nq, self.num_q_heads, self.head_dim), dtype=out_dtype, device=q.device)
+        if lse is None:
+            lse = torch.empty((Nq, self.num_q_heads), dtype=torch.float32, device=q.device)
+        splitkv_attn_fwd(self.plan, q, k, v, scale, self.ws_fwd)
+        splitkv_merge(self.plan, q, kb, vb, scale, self.ws_fwd, o, lse)
+        return o, lse
+
+    def backward(self, q, k, v, kb, vb, o, lse, dout, scale: float, grads=None):
+        if grads is None:
+            f32 = dict(dtype=torch.float32, device=q.device)
+            grads = {
+                "dq": torch.empty(q.shape, **f32),
+                "dk": torch.empty(k.shape, **f32),
+                "dv": torch.empty(v.shape, **f32),
+                "dkb": torch.empty(kb.shape, **f32),
+                "dvb": torch.empty(vb.shape, **f32),
+            }
+        splitkv_attn_bwd(self.plan, q, k, v, kb, vb, o, lse, dout, grads["dq"], grads["dk"], grads["dv"],
+                         grads["dkb"], grads["dvb"], scale, self.ws_bwd())
+        return grads

@@ -226,6 +226,24 @@ int splitkv_attn_bwd(const splitkv_plan_t* plan, const void* q, const void* k,
                      float* dkb, float* dvb, float scale, void* ws,
                      size_t ws_bytes, void* stream);
 
+/* The three launches of splitkv_attn_bwd, exposed so that callers can time or
+ * overlap them; splitkv_attn_bwd is exactly these three in this order on one
+ * stream, with the same arguments:
+ *   splitkv_bwd_delta    Delta = rowsum(dout * o) into the backward workspace;
+ *   splitkv_bwd_partial  the persistent chunk kernel: dk, dv (chunk-owned) and the
+ *                        per-entry dq partials in the workspace;
+ *   splitkv_bwd_reduce   dq = sum of the partials in ascending chunk order plus the
+ *                        in-block term's dq; dkb, dvb of the in-block term.
+ * Errors: as splitkv_attn_bwd. */
+int splitkv_bwd_delta(const splitkv_plan_t* plan, const void* o, int o_dtype, const void* dout,
+                      void* ws, size_t ws_bytes, void* stream);
+int splitkv_bwd_partial(const splitkv_plan_t* plan, const void* q, const void* k, const void* v,
+                        const float* lse, const void* dout, float* dk, float* dv, float scale,
+                        void* ws, size_t ws_bytes, void* stream);
+int splitkv_bwd_reduce(const splitkv_plan_t* plan, const void* q, const void* kb, const void* vb,
+                       const float* lse, const void* dout, float* dq, float* dkb, float* dvb,
+                       float scale, const void* ws, size_t ws_bytes, void* stream);
+
 /* Per-CTA busy time of the last splitkv_attn_fwd (which = SPLITKV_WS_FWD) or
  * backward partial kernel (SPLITKV_WS_BWD) on this plan: out_ns[w] = end - start
  * of worker w's CTA in nanoseconds (device global timer), for the schedule's

@@ -75,14 +75,16 @@ def attention_fwd(q, k, v, kb, vb, sample_lens, anchors, block_size: int, scale:
     return O, LSE
 
 
-def attention_bwd(q, k, v, kb, vb, dout, sample_lens, anchors, block_size: int, scale: float
-                  ) -> Dict[str, np.ndarray]:
+def attention_bwd(q, k, v, kb, vb, dout, sample_lens, anchors, block_size: int, scale: float,
+                  blocks: Optional[Iterable[int]] = None) -> Dict[str, np.ndarray]:
     """Analytic gradients dq, dk, dv, dkb, dvb (float64) of sum(dout * O).
 
     Per block b and head h with P = softmax(s) over the allowed keys:
     dvalues = P^T dout; dP = dout values^T; Delta = rowsum(P * dP);
     dS = P * (dP - Delta); dq = scale * dS keys; dkeys = scale * dS^T q.
     Context-key gradients are summed over every (block, head) that reads the key.
+    `blocks` restricts the sum to some blocks (then dk/dv are exact only on keys
+    that no other block reads).
     """
     Nq, Hq, d = q.shape
     N, Hkv, _ = k.shape
@@ -93,7 +95,9 @@ def attention_bwd(q, k, v, kb, vb, dout, sample_lens, anchors, block_size: int, 
     dv = np.zeros_like(v)
     dkb = np.zeros_like(kb)
     dvb = np.zeros_like(vb)
-    for b, (S, a) in enumerate(context_interval(sample_lens, anchors)):
+    iv = context_interval(sample_lens, anchors)
+    for b in (range(len(iv)) if blocks is None else blocks):
+        S, a = iv[b]
         rows = slice(b * bs, (b + 1) * bs)
         n_ctx = a - S
         for h in range(Hq):

@@ -16,11 +16,21 @@ def pytest_configure(config):
 @pytest.fixture(scope="session")
 def splitkv():
     """The Python binding with libsplitkv.so built in-tree (nvcc cross-compiles; no GPU needed)."""
-    from context_block_sparse_b200 import build as _build
+    _build = load_build_module()
     if not os.path.exists(_build.LIB):
         _build.build()
     import context_block_sparse_b200 as skv
     return skv
+
+
+def load_build_module():
+    """context_block_sparse_b200/build.py, loaded by path (importing the package needs the built library)."""
+    import importlib.util
+    path = os.path.join(ROOT, "context_block_sparse_b200", "build.py")
+    spec = importlib.util.spec_from_file_location("_splitkv_build", path)
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    return mod
 
 
 def gpu_available():

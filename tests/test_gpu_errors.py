@@ -1,0 +1,57 @@
+"""Bad arguments come back as status codes from host-side checks; no kernel is given a bad pointer."""
+
+import numpy as np
+import pytest
+
+from gpu_util import small, to_dev
+
+pytestmark = pytest.mark.gpu
+
+
+def test_host_checks_before_launch(splitkv):
+    import torch
+    skv = splitkv
+    w = small(Hq=4, Hkv=1, d=64)
+    plan = skv.splitkv_plan(w.sample_lens, w.anchors, w.block_size, w.num_q_heads, w.num_kv_heads, w.head_dim,
+                            w.kv_chunk, 148)
+    t = {n: to_dev(b) for n, b in w.bits.items()}
+    ws = torch.empty(skv.splitkv_workspace_size(plan, skv.WS_FWD), dtype=torch.uint8, device="cuda")
+    with pytest.raises(skv.SplitKVError) as ei:          # no device copy yet
+        skv.splitkv_attn_fwd(plan, t["q"], t["k"], t["v"], w.scale, ws)
+    assert ei.value.status == -6
+    plan.upload()
+    with pytest.raises(skv.SplitKVError) as ei:          # workspace one byte short
+        skv.splitkv_attn_fwd(plan, t["q"], t["k"], t["v"], w.scale, ws[:-1])
+    assert ei.value.status == -3
+    lib = skv._lib
+    q = t["q"].data_ptr()
+    st = lib.splitkv_attn_fwd(plan.handle, q + 2, t["k"].data_ptr(), t["v"].data_ptr(), 1.0, ws.data_ptr(),
+                              ws.numel(), None)
+    assert st == -1                                       # misaligned q
+    st = lib.splitkv_attn_fwd(plan.handle, None, t["k"].data_ptr(), t["v"].data_ptr(), 1.0, ws.data_ptr(),
+                              ws.numel(), None)
+    assert st == -1                                       # NULL q
+    o = torch.empty((w.num_queries, 4, 64), dtype=torch.float16, device="cuda")
+    with pytest.raises(ValueError):
+        skv.splitkv_merge(plan, t["q"], t["kb"], t["vb"], w.scale, ws, o,
+                          torch.empty((w.num_queries, 4), device="cuda"))
+    st = lib.splitkv_merge(plan.handle, q, t["kb"].data_ptr(), t["vb"].data_ptr(), 1.0, ws.data_ptr(),
+                           ws.numel(), o.data_ptr(), 7, o.data_ptr(), None)
+    assert st == -1                                       # unknown o dtype
+    # the context still works afterwards
+    skv.splitkv_attn_fwd(plan, t["q"], t["k"], t["v"], w.scale, ws)
+    torch.cuda.synchronize()
+
+
+def test_unsupported_head_dim(splitkv):
+    import torch
+    skv = splitkv
+    w = small(Hq=2, Hkv=1, d=64)
+    plan = skv.splitkv_plan(w.sample_lens, w.anchors, w.block_size, 2, 1, 96, w.kv_chunk, 148)
+    plan.upload()
+    ws = torch.empty(skv.splitkv_workspace_size(plan, skv.WS_FWD), dtype=torch.uint8, device="cuda")
+    x = torch.zeros(16, dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(skv.SplitKVError) as ei:
+        skv.splitkv_attn_fwd(plan, x, x, x, 1.0, ws)
+    assert ei.value.status == -2
+    torch.cuda.synchronize()

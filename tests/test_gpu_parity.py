@@ -1,0 +1,222 @@
+"""CUDA path (through the C ABI) against the fp64 oracle on the same seeded bf16 inputs.
+
+Tolerances: max-abs 2e-2 on O, dQ, dK, dV, dKb, dVb and 1e-3 on LSE (bf16
+inputs, fp32 accumulation).  Small workloads are compared element by element;
+the full-size workloads on sampled blocks/keys, which the oracle computes one
+by one.
+"""
+
+import numpy as np
+import pytest
+
+from gpu_util import TOL_LSE, TOL_OUT, assert_close, oracle_bwd, oracle_fwd, run, small
+from oracle import mask as omask
+from synth import make_workload
+
+pytestmark = pytest.mark.gpu
+
+
+def _check_fwd(w, out, blocks=None):
+    O, L = oracle_fwd(w, blocks)
+    if blocks is not None:
+        rows = np.concatenate([np.arange(b * w.block_size, (b + 1) * w.block_size) for b in blocks])
+        O, L = O[rows], L[rows]
+        got_o, got_l = out["o"][rows], out["lse"][rows]
+    else:
+        got_o, got_l = out["o"], out["lse"]
+    e1 = assert_close("O", got_o, O, TOL_OUT)
+    e2 = assert_close("LSE", got_l, L, TOL_LSE)
+    return e1, e2
+
+
+def _check_bwd(w, out):
+    g = oracle_bwd(w)
+    for n in ("dq", "dk", "dv", "dkb", "dvb"):
+        assert_close(n, out[n], g[n], TOL_OUT)
+
+
+def test_tiny_fwd_bwd_elementwise(splitkv):
+    w = make_workload("tiny")
+    out, _, _ = run(w, bwd=True)
+    _check_fwd(w, out)
+    _check_bwd(w, out)
+
+
+SMALL_CASES = {
+    "gqa4_d128": dict(Hq=8, Hkv=2, d=128),
+    "mha_d64": dict(Hq=2, Hkv=2, d=64),
+    "gqa8_d64": dict(Hq=8, Hkv=1, d=64),
+    "gqa4_bs8": dict(Hq=4, Hkv=1, d=128, bs=8, anchors=40),
+    "bs1_mha": dict(Hq=1, Hkv=1, d=64, bs=1, anchors=300, C=64),
+    "bs32_g4": dict(Hq=4, Hkv=1, d=64, bs=32, anchors=10),
+    "chunk_not_dividing": dict(Hq=4, Hkv=1, d=128, C=100, lens=(257, 3, 1000, 61)),
+    "one_sample": dict(Hq=4, Hkv=2, d=64, lens=(3001,), anchors=20, C=512),
+}
+
+
+@pytest.mark.parametrize("case", list(SMALL_CASES))
+def test_small_ragged_fwd_bwd_elementwise(splitkv, case):
+    w = small(**SMALL_CASES[case])
+    out, _, _ = run(w, bwd=True)
+    _check_fwd(w, out)
+    _check_bwd(w, out)
+
+
+@pytest.mark.parametrize("opts", [
+    dict(W=7), dict(W=1), dict(W=300, Wb=5), dict(q_slice=1), dict(q_slice=2, equal_count=True),
+    dict(o_dtype="bf16"),
+])
+def test_schedules_and_options_same_result(splitkv, opts):
+    w = small()
+    out, _, _ = run(w, bwd=True, **opts)
+    _check_fwd(w, out)
+    _check_bwd(w, out)
+
+
+def test_anchor_at_sample_start_and_adjacent_anchors(splitkv):
+    """Empty context interval (block sees only its own keys) and neighbouring anchors."""
+    w = small(lens=(300, 200), anchors=6, Hq=4, Hkv=1, d=64)
+    w.anchors[:] = np.array([0, 1, 2, 299, 300, 301], dtype=np.int32)
+    out, _, _ = run(w, bwd=True)
+    _check_fwd(w, out)
+    _check_bwd(w, out)
+
+
+def test_partial_records_match_oracle_split(splitkv):
+    """The workspace records (m_c, l_c, O_c) equal the oracle's per-chunk partials."""
+    import torch
+    from oracle import attention as oatt
+    w = small(Hq=4, Hkv=2, d=64)
+    _, att, _ = run(w)
+    E = att.plan.stats()["num_entries"]
+    bs, Hq, d = w.block_size, w.num_q_heads, w.head_dim
+    ws = att.ws_fwd.cpu().numpy()
+    rows = E * bs * Hq
+
+    def arr(off, n):
+        return ws[off:off + 4 * n].view(np.float32)
+
+    o_bytes = -(-rows * d * 4 // 256) * 256
+    ml_bytes = -(-rows * 4 // 256) * 256
+    O = arr(0, rows * d).reshape(E, bs, Hq, d)
+    m = arr(o_bytes, rows).reshape(E, bs, Hq)
+    l = arr(o_bytes + ml_bytes, rows).reshape(E, bs, Hq)
+    ent = att.plan.export(0).reshape(-1, 4)
+    parts = {(p["c"], p["b"]): p for p in oatt.chunk_partials(
+        w.f64("q"), w.f64("k"), w.f64("v"), w.sample_lens, w.anchors, bs, w.kv_chunk, w.scale)}
+    for e, (c, b, lo, hi) in enumerate(ent.tolist()):
+        p = parts[(c, b)]
+        assert (p["lo"], p["hi"]) == (lo, hi)
+        assert_close("O_c", O[e].astype(np.float64), p["O"], TOL_OUT)
+        # compare m + log l (the chunk's log-sum-exp) and m itself
+        assert_close("lse_c", (m[e] + np.log(l[e])).astype(np.float64), p["m"] + np.log(p["l"]), TOL_LSE)
+        assert_close("m_c", m[e].astype(np.float64), p["m"], TOL_LSE)
+    torch.cuda.synchronize()
+
+
+def test_merge_alone_on_oracle_partials(splitkv):
+    """splitkv_merge fed with oracle-computed partial records reproduces the oracle output."""
+    import torch
+    import context_block_sparse_b200 as skv
+    from gpu_util import to_dev
+    from oracle import attention as oatt
+    w = small(Hq=4, Hkv=1, d=128)
+    plan = skv.splitkv_plan(w.sample_lens, w.anchors, w.block_size, w.num_q_heads, w.num_kv_heads,
+                            w.head_dim, w.kv_chunk, 148)
+    plan.upload()
+    E = plan.stats()["num_entries"]
+    bs, Hq, d = w.block_size, w.num_q_heads, w.head_dim
+    rows = E * bs * Hq
+    o_bytes = -(-rows * d * 4 // 256) * 256
+    ml_bytes = -(-rows * 4 // 256) * 256
+    ws = np.zeros(skv.splitkv_workspace_size(plan, skv.WS_FWD), dtype=np.uint8)
+    parts = {(p["c"], p["b"]): p for p in oatt.chunk_partials(
+        w.f64("q"), w.f64("k"), w.f64("v"), w.sample_lens, w.anchors, bs, w.kv_chunk, w.scale)}
+    O = ws[:rows * d * 4].view(np.float32).reshape(E, bs, Hq, d)
+    m = ws[o_bytes:o_bytes + rows * 4].view(np.float32).reshape(E, bs, Hq)
+    l = ws[o_bytes + ml_bytes:o_bytes + ml_bytes + rows * 4].view(np.float32).reshape(E, bs, Hq)
+    for e, (c, b, lo, hi) in enumerate(plan.export(0).reshape(-1, 4).tolist()):
+        p = parts[(c, b)]
+        O[e], m[e], l[e] = p["O"], p["m"], p["l"]
+    ws_d = torch.from_numpy(ws).cuda()
+    o = torch.empty((w.num_queries, Hq, d), dtype=torch.float32, device="cuda")
+    lse = torch.empty((w.num_queries, Hq), dtype=torch.float32, device="cuda")
+    skv.splitkv_merge(plan, to_dev(w.bits["q"]), to_dev(w.bits["kb"]), to_dev(w.bits["vb"]), w.scale, ws_d, o, lse)
+    Oref, Lref = oracle_fwd(w)
+    assert_close("O", o.cpu().numpy().astype(np.float64), Oref, TOL_OUT)
+    assert_close("LSE", lse.cpu().numpy().astype(np.float64), Lref, TOL_LSE)
+
+
+def test_backward_is_deterministic(splitkv):
+    w = small()
+    a, _, _ = run(w, bwd=True)
+    b, _, _ = run(w, bwd=True)
+    for n in ("o", "lse", "dq", "dk", "dv", "dkb", "dvb"):
+        assert np.array_equal(a[n], b[n]), n
+
+
+# ---------------------------------------------------------------------------
+# full-size workloads, in the launch configuration the bench times
+# ---------------------------------------------------------------------------
+
+def _sample_blocks(w, n=10, seed=0):
+    rng = np.random.default_rng(seed)
+    A = w.anchors.size
+    pick = {0, A - 1} | set(rng.choice(A, size=min(n, A), replace=False).tolist())
+    return sorted(pick)
+
+
+def test_drafter_fwd_full(splitkv):
+    w = make_workload("drafter")
+    out, _, _ = run(w)
+    _check_fwd(w, out)
+
+
+@pytest.mark.parametrize("anchors", [128, 256, 512])
+def test_budget_fwd_sampled(splitkv, anchors):
+    w = make_workload("budget", num_anchors=anchors)
+    out, _, _ = run(w)
+    _check_fwd(w, out, _sample_blocks(w))
+    assert np.isfinite(out["o"]).all() and np.isfinite(out["lse"]).all()
+
+
+def test_skew_fwd_sampled(splitkv):
+    w = make_workload("skew")
+    out, _, _ = run(w)
+    _check_fwd(w, out, _sample_blocks(w))
+    assert np.isfinite(out["o"]).all()
+
+
+def test_bwd_config_sampled(splitkv):
+    """fwd+bwd at 64k context / 8k queries: O, LSE, dQ, dKb, dVb on sampled blocks; dK, dV on the keys of
+    sampled chunks, with the oracle summing over every block that reads them."""
+    w = make_workload("bwd")
+    out, _, _ = run(w, bwd=True)
+    blocks = _sample_blocks(w, n=6)
+    _check_fwd(w, out, blocks)
+    g = oracle_bwd(w, blocks)
+    bs = w.block_size
+    rows = np.concatenate([np.arange(b * bs, (b + 1) * bs) for b in blocks])
+    for n in ("dq", "dkb", "dvb"):
+        assert_close(n, out[n][rows], g[n][rows], TOL_OUT)
+    # dK, dV on two chunks: the last chunks of the first and of a middle sample (few readers each)
+    C = w.kv_chunk
+    starts = omask.sample_starts(w.sample_lens) + [w.context_len]
+    mid = len(w.sample_lens) // 2
+    chunks = sorted({(starts[1] - 1) // C, (starts[mid + 1] - 1) // C})
+    iv = omask.context_interval(w.sample_lens, w.anchors)
+    readers = [b for b, (S, a) in enumerate(iv) if any(S < (c + 1) * C and a > c * C for c in chunks)]
+    g2 = oracle_bwd(w, readers)
+    keys = np.concatenate([np.arange(c * C, min((c + 1) * C, w.context_len)) for c in chunks])
+    for n in ("dk", "dv"):
+        assert_close(n, out[n][keys], g2[n][keys], TOL_OUT)
+    for n in ("dq", "dk", "dv", "dkb", "dvb"):
+        assert np.isfinite(out[n]).all(), n
+
+
+def test_cta_timers_recorded(splitkv):
+    import context_block_sparse_b200 as skv
+    w = make_workload("drafter")
+    out, att, _ = run(w)
+    t = skv.splitkv_read_cta_times(att.plan, skv.WS_FWD)
+    assert t.shape == (148,) and (t > 0).all()
