@@ -124,6 +124,22 @@ class ClockSampler:
                 "reasons": reasons, "samples": len(rows)}
 
 
+def max_over_ranks(ms: float, device) -> float:
+    """The slowest rank's time: every rank of an N-GPU run reports the max (all-reduce MAX)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(ms)
+    x = torch.tensor([ms], dtype=torch.float64, device=device)
+    dist.all_reduce(x, op=dist.ReduceOp.MAX)
+    return float(x.item())
+
+
+def whole_job_tflops(world: int, steps: int, flops_per_step: float, max_ms: float) -> float:
+    """Work of all ranks (each runs one replica) over the slowest rank's time, in TFLOP/s."""
+    return world * steps * flops_per_step / (max_ms * 1e-3) / 1e12
+
+
 def _dist():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -244,11 +260,7 @@ def run_ours(args, world, rank, local):
     wall1 = time.time()
     if world > 1:
         dist.barrier()
-    ms = start.elapsed_time(end)
-    if world > 1:
-        x = torch.tensor([ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(x, op=dist.ReduceOp.MAX)
-        ms = float(x.item())
+    ms = max_over_ranks(start.elapsed_time(end), dev)
     per_kernel = {k: float(np.mean([evs[i][j].elapsed_time(evs[i][j + 1]) for i in range(args.steps)]))
                   for j, k in enumerate(kernels)}
     clocks = sampler.summary(wall0, wall1) if sampler else {"sm_mhz": None, "sm_max_mhz": None,
@@ -268,7 +280,7 @@ def run_ours(args, world, rank, local):
     flops_fwd = 4.0 * d * pairs
     flops_bwd = 10.0 * d * pairs
     flops_step = flops_fwd + flops_bwd
-    value = world * args.steps * flops_step / (ms * 1e-3) / 1e12
+    value = whole_job_tflops(world, args.steps, flops_step, ms)
     peaks = _peaks()
     work = _kernel_work(st, w, st["num_entries"])
     dom = max(kernels, key=lambda k: per_kernel[k])
@@ -384,13 +396,10 @@ def run_e2e(args, w, plan, dev, stream, flops_step, world=1):
         step()
     b.record(stream)
     torch.cuda.synchronize(dev)
-    ms = a.elapsed_time(b)
+    ms = max_over_ranks(a.elapsed_time(b), dev)
     if world > 1:
-        x = torch.tensor([ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(x, op=dist.ReduceOp.MAX)
-        ms = float(x.item())
         dist.barrier()
-    return {"value": world * steps * flops_step / (ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+    return {"value": whole_job_tflops(world, steps, flops_step, ms), "unit": "TFLOP/s",
             "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "steps": steps,
             "ms_per_step": ms / steps}
 

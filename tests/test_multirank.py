@@ -1,0 +1,57 @@
+"""N > 1 host logic of the bench on CPU: world-size-2 gloo ranks (replicas only, no data-path collective)."""
+
+import os
+import sys
+
+import pytest
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _worker(rank, world, port, q):
+    import torch
+    import torch.distributed as dist
+    sys.path.insert(0, ROOT)
+    import bench
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank), WORLD_SIZE=str(world),
+                      LOCAL_RANK=str(rank))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        ms = bench.max_over_ranks(10.0 + 5.0 * rank, torch.device("cpu"))
+        w, r, l = bench._dist()
+        # the reference arm runs on rank 0 only; other ranks exit without work
+        class A:
+            workload, anchors, steps, warmup, cpu_seconds = "tiny", None, 1, 3, 0.2
+        ref = bench.run_reference(A, w, r)
+        q.put((rank, ms, (w, r, l), ref is None))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_two_gloo_ranks_take_the_max_time_and_only_rank0_runs_reference():
+    import socket
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    port = s.getsockname()[1]
+    s.close()
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    procs = [ctx.Process(target=_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    out = sorted(q.get(timeout=300) for _ in procs)
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    assert [o[1] for o in out] == [15.0, 15.0]            # both ranks see the slowest rank's time
+    assert [o[2] for o in out] == [(2, 0, 0), (2, 1, 1)]
+    assert [o[3] for o in out] == [False, True]            # rank 0 produced the reference line
+
+
+def test_whole_job_value_is_sum_of_replicas_over_max_time():
+    sys.path.insert(0, ROOT)
+    import bench
+    one = bench.whole_job_tflops(1, 10, 1e12, 1000.0)
+    two = bench.whole_job_tflops(2, 10, 1e12, 1000.0)
+    assert one == pytest.approx(10.0) and two == pytest.approx(20.0)
