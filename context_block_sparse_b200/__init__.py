@@ -24,7 +24,7 @@ from . import _abi
 from ._abi import (  # noqa: F401
     DTYPE_BF16, DTYPE_F32, EXPORT_BWD_LOADS, EXPORT_BWD_SCHEDULE, EXPORT_CHUNK_PAIRS,
     EXPORT_CONTIG_LOADS, EXPORT_ENTRIES, EXPORT_FWD_LOADS, EXPORT_FWD_SCHEDULE,
-    FLAG_EQUAL_COUNT, WS_BWD, WS_FWD,
+    FLAG_EQUAL_COUNT, STATIC_SCRATCH_BYTES, WS_BWD, WS_FWD,
 )
 
 _lib = _abi.load()
@@ -235,6 +235,13 @@ def splitkv_bwd_reduce(plan: Plan, q, kb, vb, lse, dout, dq, dkb, dvb, scale: fl
         plan.handle, _bf16_ptr(q), _bf16_ptr(kb), _bf16_ptr(vb), _f32_ptr(lse), _bf16_ptr(dout), _f32_ptr(dq),
         _f32_ptr(dkb), _f32_ptr(dvb), float(scale), _ptr(ws), ws.numel() * ws.element_size(),
         _stream_ptr(stream)))
+
+
+def splitkv_attn_fwd_static_scratch(plan: Plan, q, k, v, kb, vb, scale: float, o, lse, stream=None) -> None:
+    """Forward + merge with the partial records in the library's static device buffer (no allocation)."""
+    _check("splitkv_attn_fwd_static_scratch", _lib.splitkv_attn_fwd_static_scratch(
+        plan.handle, _bf16_ptr(q), _bf16_ptr(k), _bf16_ptr(v), _bf16_ptr(kb), _bf16_ptr(vb), float(scale),
+        _ptr(o), _o_dtype(o), _f32_ptr(lse), _stream_ptr(stream)))
 
 
 def splitkv_read_cta_times(plan: Plan, which: int, stream=None) -> np.ndarray:

@@ -22,6 +22,8 @@ ERR_NO_MEMORY = -7
 
 FLAG_EQUAL_COUNT = 1
 
+STATIC_SCRATCH_BYTES = 16 << 20
+
 DTYPE_F32 = 0
 DTYPE_BF16 = 1
 
@@ -102,6 +104,7 @@ SIGNATURES = {
     "splitkv_bwd_delta": (_I, [_P, _P, _I, _P, _P, _SZ, _P]),
     "splitkv_bwd_partial": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _F, _P, _SZ, _P]),
     "splitkv_bwd_reduce": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _F, _P, _SZ, _P]),
+    "splitkv_attn_fwd_static_scratch": (_I, [_P, _P, _P, _P, _P, _P, _F, _P, _I, _P, _P]),
     "splitkv_read_cta_times": (_I, [_P, _I, ctypes.POINTER(ctypes.c_int64), ctypes.c_int64, _P]),
 }
 

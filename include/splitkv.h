@@ -244,6 +244,33 @@ int splitkv_bwd_reduce(const splitkv_plan_t* plan, const void* q, const void* kb
                        const float* lse, const void* dout, float* dq, float* dkb, float* dvb,
                        float scale, const void* ws, size_t ws_bytes, void* stream);
 
+/* Size of the library's static device scratch buffer (16 MiB): see
+ * splitkv_attn_fwd_static_scratch. */
+#define SPLITKV_STATIC_SCRATCH_BYTES (16u << 20)
+
+/* Forward attention that allocates nothing: splitkv_attn_fwd followed by
+ * splitkv_merge, with the partial records held in a buffer of
+ * SPLITKV_STATIC_SCRATCH_BYTES that is a static array of the library's device
+ * code (every GPU that loads the library keeps it until the process exits).
+ * The pages have no counterpart to this call: it exists for callers that may
+ * not call cudaMalloc per call (a framework whose caching allocator holds the
+ * device memory, latency-critical loops that cannot take cudaMalloc's implicit
+ * synchronisation, plug-ins handed raw pointers without an allocator).
+ * The caller passes the inputs and outputs exactly as for splitkv_attn_fwd and
+ * splitkv_merge; the plan must already have its device copy
+ * (splitkv_plan_upload, a set-up step) on the current device.  The first call
+ * on a device looks up the buffer's device address (cudaGetSymbolAddress),
+ * so make that first call before any stream capture.  Every call shares the one
+ * buffer, and calls whose kernels overlap on the GPU (different streams, or
+ * different host threads) race on it: serialise them.  Each call writes every
+ * record it reads, so left-over contents of an earlier call are never used.
+ * Errors: as splitkv_merge, plus WORKSPACE_TOO_SMALL when the problem's forward
+ * workspace (splitkv_workspace_size, SPLITKV_WS_FWD) exceeds
+ * SPLITKV_STATIC_SCRATCH_BYTES. */
+int splitkv_attn_fwd_static_scratch(const splitkv_plan_t* plan, const void* q, const void* k,
+                                    const void* v, const void* kb, const void* vb, float scale,
+                                    void* o, int o_dtype, float* lse, void* stream);
+
 /* Per-CTA busy time of the last splitkv_attn_fwd (which = SPLITKV_WS_FWD) or
  * backward partial kernel (SPLITKV_WS_BWD) on this plan: out_ns[w] = end - start
  * of worker w's CTA in nanoseconds (device global timer), for the schedule's
