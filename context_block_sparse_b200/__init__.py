@@ -244,6 +244,11 @@ def splitkv_attn_fwd_static_scratch(plan: Plan, q, k, v, kb, vb, scale: float, o
         _ptr(o), _o_dtype(o), _f32_ptr(lse), _stream_ptr(stream)))
 
 
+def splitkv_plan_status(plan: Plan, stream=None) -> None:
+    """Raise SplitKVError if a kernel of this plan recorded an error (e.g. a timed-out wait)."""
+    _check("splitkv_plan_status", _lib.splitkv_plan_status(plan.handle, _stream_ptr(stream)))
+
+
 def splitkv_read_cta_times(plan: Plan, which: int, stream=None) -> np.ndarray:
     """Per-CTA busy nanoseconds of the last forward (WS_FWD) or backward (WS_BWD) partial kernel."""
     st = plan.stats()

@@ -13,6 +13,8 @@
 // accumulate), masks every row to its block's [lo, hi), keeps a base-2 online
 // softmax per row in registers and accumulates O += P V.  Each warp owns 16 rows.
 #include <cfloat>
+#include <cstdlib>
+#include <cstring>
 
 #include "common.cuh"
 #include "splitkv_internal.h"
@@ -264,9 +266,22 @@ cudaError_t launch_fwd_d(const DevPlan& p, const uint16_t* q, const uint16_t* k,
 
 }  // namespace
 
+bool fwd_sm100_supported(const DevPlan& p);
+cudaError_t launch_fwd_partial_sm100(const DevPlan& p, const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                                     float scale, float* part_o, float* part_m, float* part_l, cudaStream_t s);
+
+// The tcgen05 kernel serves head_dim 128 with G * bs a multiple of 8; every
+// other shape runs the mma.sync kernel.  SPLITKV_FWD_KERNEL=mma selects the
+// mma.sync kernel for every shape (for comparisons).
 cudaError_t launch_fwd_partial(const DevPlan& p, const uint16_t* q, const uint16_t* k,
                                const uint16_t* v, float scale, float* part_o, float* part_m,
                                float* part_l, cudaStream_t s) {
+  static const bool force_mma = [] {
+    const char* e = std::getenv("SPLITKV_FWD_KERNEL");
+    return e != nullptr && std::strcmp(e, "mma") == 0;
+  }();
+  if (!force_mma && fwd_sm100_supported(p))
+    return launch_fwd_partial_sm100(p, q, k, v, scale, part_o, part_m, part_l, s);
   if (p.d == 64) return launch_fwd_d<64>(p, q, k, v, scale, part_o, part_m, part_l, s);
   return launch_fwd_d<128>(p, q, k, v, scale, part_o, part_m, part_l, s);
 }

@@ -1,0 +1,478 @@
+// Partial attention of every (chunk, block) entry on the 5th-generation tensor
+// cores (tcgen05 / TMEM / TMA), head_dim 128.
+//
+// News page "Split-KV speeds diffusion drafter training by keeping long-context
+// data local", section "Exchange the smaller side": each key/value shard (here
+// a KV chunk) evaluates every query that reads it and emits a partial result
+// with its normalisation statistics; section "Balance actual attention work":
+// the shards are spread over workers (here persistent CTAs) by LPT.
+//
+// One persistent CTA per worker walks its LPT items; every item's 128-row query
+// tiles are taken two at a time (A and B) so that each K/V tile loaded into
+// shared memory feeds two 128x128 score tiles.  Roles (384 threads):
+//   warp 0      TMA producer: Q tiles (3-D boxes of bs tokens x G heads per
+//               block) and 128-key K/V tiles into a 2-stage ring;
+//   warp 1      MMA issuer (one thread): S_X = Q_X K^T into TMEM, then
+//               O_X += P_X V with P_X read from TMEM (bf16, aliasing S_X);
+//   warp 2      tensor-memory allocation (512 columns: S_A, S_B, O_A, O_B);
+//   warps 4-7   softmax / epilogue of tile A (thread = row = TMEM lane);
+//   warps 8-11  softmax / epilogue of tile B.
+// The softmax keeps, per row, a reference maximum m_ref and rescales O in TMEM
+// only when a new key tile raises the maximum by more than 2^8 (the result is
+// the same; the reference is exact bookkeeping).  The record written is
+// m_c = the row's true maximum (natural units), l_c = sum exp(s - m_c) and
+// O_c = sum exp(s - m_c) v / l_c.  Rows are masked to their block's [lo, hi).
+//
+// Every mbarrier wait is bounded; on a timeout the kernel records
+// SPLITKV_ERR_TIMEOUT in the plan's status word, lets every role wind down,
+// waits for its own copies in flight and frees its tensor memory.
+#include <cfloat>
+
+#include "sm100.cuh"
+#include "splitkv.h"
+#include "splitkv_internal.h"
+
+namespace splitkv {
+namespace {
+
+using namespace sm100;
+
+constexpr int D = 128;
+constexpr int BM = 128;               // query rows per tile
+constexpr int BN = 128;               // keys per key tile
+constexpr int kStages = 2;            // K/V ring depth
+constexpr int kThreads = 384;
+constexpr uint32_t kHalf = 128 * 128; // bytes of one 64-column half of a 128-row tile
+constexpr uint32_t kTile = 2 * kHalf; // 32 KB: a 128 x 128 bf16 tile
+constexpr uint32_t kIdescQK = idesc_bf16_f32(128, 128, 0);
+constexpr uint32_t kIdescPV = idesc_bf16_f32(128, D, 1);
+constexpr float kRescaleLog2 = 8.0f;  // rescale O only when the max grows by more than 2^8
+
+// shared-memory map (offsets from a 1024-aligned base)
+constexpr uint32_t kOffQ = 0;                              // Q_A, Q_B
+constexpr uint32_t kOffK = kOffQ + 2 * kTile;              // K stages
+constexpr uint32_t kOffV = kOffK + kStages * kTile;        // V stages
+constexpr uint32_t kOffBar = kOffV + kStages * kTile;      // mbarriers
+constexpr uint32_t kSmemBytes = kOffBar + 256 + 1024;      // + alignment slack
+
+struct Bars {
+  uint64_t q_full, q_empty;
+  uint64_t k_full[kStages], v_full[kStages], kv_empty[kStages];
+  uint64_t s_ready[2], p_ready[2], o_ready[2], o_free[2];
+  uint64_t mma_done;
+  uint32_t tmem_base;
+  int abort_flag;
+};
+static_assert(sizeof(Bars) <= 256, "barrier block");
+
+// The sequence of tile pairs a worker processes (identical in every role).
+struct PairIter {
+  const DevPlan* p;
+  int it, it_end;   // item cursor
+  int t, t_end;     // tile cursor inside the item
+  int g;
+  __device__ void init(const DevPlan* plan, int w) {
+    p = plan;
+    it = plan->fwd_worker_ptr[w];
+    it_end = plan->fwd_worker_ptr[w + 1];
+    t = t_end = 0;
+    g = 0;
+  }
+  // tA, tB (-1 if absent), kv head, key union [klo, khi)
+  __device__ bool next(int& tA, int& tB, int& head, int& klo, int& khi) {
+    while (t >= t_end) {
+      if (it >= it_end) return false;
+      const int4 item = p->fwd_items[it++];
+      g = item.y;
+      t = item.z;
+      t_end = item.w;
+    }
+    tA = t++;
+    tB = (t < t_end) ? t++ : -1;
+    head = g;
+    const int4 a = p->tiles[tA];
+    klo = a.z;
+    khi = a.w;
+    if (tB >= 0) {
+      const int4 b = p->tiles[tB];
+      klo = min(klo, b.z);
+      khi = max(khi, b.w);
+    }
+    return true;
+  }
+};
+
+__device__ __forceinline__ void record_abort(Bars* bars, const DevPlan& p) {
+  bars->abort_flag = 1;
+  atomicExch(p.status, SPLITKV_ERR_TIMEOUT);
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+    fwd_partial_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                             const __grid_constant__ CUtensorMap tm_v, DevPlan p, float scale_log2,
+                             float* __restrict__ part_o, float* __restrict__ part_m,
+                             float* __restrict__ part_l) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  Bars* bars = reinterpret_cast<Bars*>(smem + kOffBar);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int w = blockIdx.x;
+  volatile int* abort_flag = &bars->abort_flag;
+
+  if (tid == 0) {
+    p.timers[w * 2 + 0] = global_timer_ns();
+    mbar_init(&bars->q_full, 1);
+    mbar_init(&bars->q_empty, 1);
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&bars->k_full[s], 1);
+      mbar_init(&bars->v_full[s], 1);
+      mbar_init(&bars->kv_empty[s], 1);
+    }
+    for (int x = 0; x < 2; ++x) {
+      mbar_init(&bars->s_ready[x], 1);
+      mbar_init(&bars->p_ready[x], 128);
+      mbar_init(&bars->o_ready[x], 1);
+      mbar_init(&bars->o_free[x], 128);
+    }
+    mbar_init(&bars->mma_done, 1);
+    bars->abort_flag = 0;
+    mbar_fence_init();
+  }
+  if (warp == 2) {
+    tmem_alloc(&bars->tmem_base, 512);
+    tmem_relinquish();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(&tm_q);
+    prefetch_tmap(&tm_k);
+    prefetch_tmap(&tm_v);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = bars->tmem_base;
+  const int rows_per_slot = p.G * p.bs;
+  const uint32_t slot_bytes = uint32_t(rows_per_slot) * 128;   // one slot's rows of one 64-column half
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      PairIter pi;
+      pi.init(&p, w);
+      int tA, tB, g, klo, khi;
+      uint32_t kv_count = 0, pair_count = 0, q_issued = 0;
+      bool ok = true;
+      while (ok && pi.next(tA, tB, g, klo, khi)) {
+        if (!mbar_wait(&bars->q_empty, (pair_count & 1) ^ 1, abort_flag)) { ok = false; break; }
+        const int4 ta = p.tiles[tA];
+        const int nA = ta.y - ta.x;
+        int nB = 0;
+        int4 tb = make_int4(0, 0, 0, 0);
+        if (tB >= 0) {
+          tb = p.tiles[tB];
+          nB = tb.y - tb.x;
+        }
+        mbar_expect_tx(&bars->q_full, uint32_t(nA + nB) * 2u * slot_bytes);
+        for (int x = 0; x < 2; ++x) {
+          const int n = x == 0 ? nA : nB;
+          const int e0 = x == 0 ? ta.x : tb.x;
+          uint8_t* qbuf = smem + kOffQ + x * kTile;
+          for (int s = 0; s < n; ++s) {
+            const int blk = p.entries[e0 + s].x;
+            for (int dh = 0; dh < 2; ++dh)
+              tma_load_3d(qbuf + dh * kHalf + s * slot_bytes, &tm_q, &bars->q_full, dh * 64, g * p.G, blk * p.bs);
+          }
+        }
+        ++q_issued;
+        const int n_kt = (khi - klo + BN - 1) / BN;
+        for (int j = 0; j < n_kt; ++j, ++kv_count) {
+          const int s = kv_count % kStages;
+          if (!mbar_wait(&bars->kv_empty[s], ((kv_count / kStages) & 1) ^ 1, abort_flag)) { ok = false; break; }
+          const int k0 = klo + j * BN;
+          mbar_expect_tx(&bars->k_full[s], kTile);
+          for (int dh = 0; dh < 2; ++dh)
+            tma_load_3d(smem + kOffK + s * kTile + dh * kHalf, &tm_k, &bars->k_full[s], dh * 64, g, k0);
+          mbar_expect_tx(&bars->v_full[s], kTile);
+          for (int dh = 0; dh < 2; ++dh)
+            tma_load_3d(smem + kOffV + s * kTile + dh * kHalf, &tm_v, &bars->v_full[s], dh * 64, g, k0);
+        }
+        ++pair_count;
+      }
+      if (!ok) record_abort(bars, p);
+      // copies still in flight land before the CTA may exit: wait for the last
+      // fill of every buffer (bounded; completed phases return at once)
+      if (q_issued > 0) mbar_drain(&bars->q_full, (q_issued - 1) & 1);
+      for (uint32_t c = kv_count >= kStages ? kv_count - kStages : 0; c < kv_count; ++c) {
+        mbar_drain(&bars->k_full[c % kStages], (c / kStages) & 1);
+        mbar_drain(&bars->v_full[c % kStages], (c / kStages) & 1);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      PairIter pi;
+      pi.init(&p, w);
+      int tA, tB, g, klo, khi;
+      uint32_t kv_count = 0, pair_count = 0;
+      uint32_t p_cnt[2] = {0, 0}, of_cnt[2] = {0, 0};
+      bool ok = true;
+      const uint32_t sQ = smem_u32(smem + kOffQ);
+      const uint32_t sK = smem_u32(smem + kOffK);
+      const uint32_t sV = smem_u32(smem + kOffV);
+      while (ok && pi.next(tA, tB, g, klo, khi)) {
+        const int nx = tB >= 0 ? 2 : 1;
+        const int n_kt = (khi - klo + BN - 1) / BN;
+        if (!mbar_wait(&bars->q_full, pair_count & 1, abort_flag)) { ok = false; break; }
+        {
+          const int s0 = kv_count % kStages;
+          if (!mbar_wait(&bars->k_full[s0], (kv_count / kStages) & 1, abort_flag)) { ok = false; break; }
+          tc_fence_after();
+          for (int x = 0; x < nx; ++x) {
+            for (int kk = 0; kk < D / 16; ++kk) {
+              const uint64_t a = smem_desc_sw128(sQ + x * kTile + (kk >> 2) * kHalf + (kk & 3) * 32, 16, 1024);
+              const uint64_t b = smem_desc_sw128(sK + s0 * kTile + (kk >> 2) * kHalf + (kk & 3) * 32, 16, 1024);
+              mma_ss(tmem + x * 128, a, b, kIdescQK, kk > 0 ? 1u : 0u);
+            }
+            mma_commit(&bars->s_ready[x]);
+          }
+        }
+        for (int j = 0; j < n_kt && ok; ++j) {
+          const uint32_t c = kv_count + j;
+          const int s = c % kStages;
+          const int s1 = (c + 1) % kStages;
+          const bool more = j + 1 < n_kt;
+          for (int x = 0; x < nx; ++x) {
+            if (!mbar_wait(&bars->p_ready[x], p_cnt[x] & 1, abort_flag)) { ok = false; break; }
+            ++p_cnt[x];
+            if (j == 0) {
+              if (!mbar_wait(&bars->o_free[x], (of_cnt[x] & 1) ^ 1, abort_flag)) { ok = false; break; }
+              ++of_cnt[x];
+            }
+            if (x == 0) {
+              if (!mbar_wait(&bars->v_full[s], (c / kStages) & 1, abort_flag)) { ok = false; break; }
+            }
+            tc_fence_after();
+            // O_X (+)= P_X V : P in TMEM (columns 0..63 of S_X), V MN-major in smem
+            for (int kk = 0; kk < BN / 16; ++kk) {
+              const uint64_t b = smem_desc_sw128(sV + s * kTile + kk * 2048, kHalf, 1024);
+              mma_ts(tmem + 256 + x * 128, tmem + x * 128 + kk * 8, b, kIdescPV, (j > 0 || kk > 0) ? 1u : 0u);
+            }
+            mma_commit(&bars->o_ready[x]);
+            if (more) {
+              if (x == 0) {
+                if (!mbar_wait(&bars->k_full[s1], ((c + 1) / kStages) & 1, abort_flag)) { ok = false; break; }
+                tc_fence_after();
+              }
+              for (int kk = 0; kk < D / 16; ++kk) {
+                const uint64_t a = smem_desc_sw128(sQ + x * kTile + (kk >> 2) * kHalf + (kk & 3) * 32, 16, 1024);
+                const uint64_t b =
+                    smem_desc_sw128(sK + s1 * kTile + (kk >> 2) * kHalf + (kk & 3) * 32, 16, 1024);
+                mma_ss(tmem + x * 128, a, b, kIdescQK, kk > 0 ? 1u : 0u);
+              }
+              mma_commit(&bars->s_ready[x]);
+            }
+          }
+          if (!ok) break;
+          mma_commit(&bars->kv_empty[s]);   // K_s, V_s free once everything issued so far completes
+        }
+        if (!ok) break;
+        mma_commit(&bars->q_empty);
+        kv_count += n_kt;
+        ++pair_count;
+      }
+      if (!ok) record_abort(bars, p);
+      // every MMA must finish before tensor memory is released
+      mma_commit(&bars->mma_done);
+      mbar_drain(&bars->mma_done, 0);
+    }
+  } else if (warp >= 4) {
+    // ------------------------------------------------------------ softmax + epilogue
+    const int x = (warp - 4) >> 2;            // tile A (warps 4-7) or B (warps 8-11)
+    const int r = ((warp & 3) << 5) + lane;   // row of the tile = TMEM lane
+    const uint32_t lane_addr = uint32_t((warp & 3) << 5) << 16;
+    const uint32_t tS = tmem + lane_addr + x * 128;
+    const uint32_t tO = tmem + lane_addr + 256 + x * 128;
+    PairIter pi;
+    pi.init(&p, w);
+    int tA, tB, g, klo, khi;
+    uint32_t s_cnt = 0, o_cnt = 0;
+    bool ok = true;
+    while (ok && pi.next(tA, tB, g, klo, khi)) {
+      const int t = x == 0 ? tA : tB;
+      if (t < 0) continue;                    // no tile B in this pair
+      const int n_kt = (khi - klo + BN - 1) / BN;
+      const int4 tile = p.tiles[t];
+      const int slot = r / rows_per_slot;
+      const int within = r - slot * rows_per_slot;
+      const int tt = within / p.G, hh = within - tt * p.G;
+      const bool valid = slot < tile.y - tile.x;
+      int lo = 0, hi = 0, rec = 0;
+      if (valid) {
+        const int e = tile.x + slot;
+        const int4 ent = p.entries[e];
+        lo = ent.y;
+        hi = ent.z;
+        rec = (e * p.bs + tt) * p.Hq + g * p.G + hh;
+      }
+      float m_ref = -INFINITY, m_true = -INFINITY, l = 0.f;
+      for (int j = 0; j < n_kt; ++j) {
+        if (!warp_wait(&bars->s_ready[x], s_cnt & 1, abort_flag)) { ok = false; break; }
+        ++s_cnt;
+        tc_fence_after();
+        const int k0 = klo + j * BN;
+        // pass 1: masked row maximum
+        float mx = -INFINITY;
+#pragma unroll 1
+        for (int cch = 0; cch < 4; ++cch) {
+          uint32_t v[32];
+          tmem_ld32(tS + cch * 32, v);
+          tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const int key = k0 + cch * 32 + i;
+            const float sv = __uint_as_float(v[i]) * scale_log2;
+            mx = (key >= lo && key < hi) ? fmaxf(mx, sv) : mx;
+          }
+        }
+        m_true = fmaxf(m_true, mx);
+        // rescale decision (warp-uniform for the TMEM traffic)
+        const bool need = (mx > m_ref + kRescaleLog2) || (m_ref == -INFINITY && mx > -INFINITY);
+        const bool rescale_o = need && m_ref > -INFINITY;      // only after a previous tile added to O
+        if (__any_sync(0xffffffffu, rescale_o)) {
+          // PV(j-1) must have completed before O is touched
+          if (!warp_wait(&bars->o_ready[x], (o_cnt + j - 1) & 1, abort_flag)) { ok = false; break; }
+          tc_fence_after();
+          const float f = rescale_o ? fast_exp2(m_ref - mx) : 1.f;
+#pragma unroll 1
+          for (int cch = 0; cch < D / 32; ++cch) {
+            uint32_t v[32];
+            tmem_ld32(tO + cch * 32, v);
+            tmem_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 32; ++i) v[i] = __float_as_uint(__uint_as_float(v[i]) * f);
+            tmem_st32(tO + cch * 32, v);
+          }
+          tmem_wait_st();
+          l *= f;
+        }
+        if (need) m_ref = mx;
+        const float m_use = (m_ref == -INFINITY) ? 0.f : m_ref;
+        // pass 2: P = exp2(s - m_ref) (masked -> 0), row sum, bf16 P into TMEM columns 0..63 of S_X
+#pragma unroll 1
+        for (int cch = 0; cch < 4; ++cch) {
+          uint32_t v[32];
+          tmem_ld32(tS + cch * 32, v);
+          tmem_wait_ld();
+          uint32_t pk[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const int key = k0 + cch * 32 + 2 * i;
+            const float s0 = __uint_as_float(v[2 * i]) * scale_log2 - m_use;
+            const float s1 = __uint_as_float(v[2 * i + 1]) * scale_log2 - m_use;
+            const float p0 = (key >= lo && key < hi) ? fast_exp2(s0) : 0.f;
+            const float p1 = (key + 1 >= lo && key + 1 < hi) ? fast_exp2(s1) : 0.f;
+            l += p0 + p1;
+            pk[i] = pack_bf16(p0, p1);
+          }
+          tmem_st16(tS + cch * 16, pk);
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(&bars->p_ready[x]);
+      }
+      if (!ok) break;
+      // epilogue: wait for the last PV of this tile, then write the record
+      if (!warp_wait(&bars->o_ready[x], (o_cnt + n_kt - 1) & 1, abort_flag)) { ok = false; break; }
+      o_cnt += n_kt;
+      tc_fence_after();
+      const float inv = l > 0.f ? 1.f / l : 0.f;
+      float* dst = part_o + size_t(rec) * D;
+#pragma unroll 1
+      for (int cch = 0; cch < D / 32; ++cch) {
+        uint32_t v[32];
+        tmem_ld32(tO + cch * 32, v);
+        tmem_wait_ld();
+        if (valid) {
+#pragma unroll
+          for (int i = 0; i < 32; i += 4) {
+            *reinterpret_cast<float4*>(dst + cch * 32 + i) =
+                make_float4(__uint_as_float(v[i]) * inv, __uint_as_float(v[i + 1]) * inv,
+                            __uint_as_float(v[i + 2]) * inv, __uint_as_float(v[i + 3]) * inv);
+          }
+        }
+      }
+      if (valid) {
+        // record (true max, sum relative to it)
+        part_m[rec] = (l > 0.f) ? m_true * kLn2 : -INFINITY;
+        part_l[rec] = (l > 0.f) ? l * fast_exp2(m_ref - m_true) : 0.f;
+      }
+      tc_fence_before();
+      mbar_arrive(&bars->o_free[x]);
+    }
+    if (!ok) record_abort(bars, p);
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 2) tmem_dealloc(tmem, 512);
+  if (tid == 0) p.timers[w * 2 + 1] = global_timer_ns();
+}
+
+// ---------------------------------------------------------------- host side
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static bool tried = false;
+  if (!tried) {
+    tried = true;
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+    else
+      cudaGetLastError();
+  }
+  return fn;
+}
+
+// 3-D bf16 tensor [dim2][dim1][dim0] (dim0 contiguous), box {64, box1, box2}, 128-byte swizzle.
+bool make_map(CUtensorMap* m, const void* base, uint64_t dim0, uint64_t dim1, uint64_t dim2, uint32_t box1,
+              uint32_t box2) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[3] = {dim0, dim1, dim2};
+  const cuuint64_t strides[2] = {dim0 * 2, dim0 * dim1 * 2};
+  const cuuint32_t box[3] = {64, box1, box2};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+bool fwd_sm100_supported(const DevPlan& p) {
+  const int rows = p.G * p.bs;
+  return p.d == D && rows % 8 == 0 && rows <= BM && encode_fn() != nullptr;
+}
+
+cudaError_t launch_fwd_partial_sm100(const DevPlan& p, const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                                     float scale, float* part_o, float* part_m, float* part_l, cudaStream_t s) {
+  CUtensorMap tq, tk, tv;
+  if (!make_map(&tq, q, D, p.Hq, p.Nq, p.G, p.bs)) return cudaErrorInvalidValue;
+  if (!make_map(&tk, k, D, p.Hkv, p.N, 1, BN)) return cudaErrorInvalidValue;
+  if (!make_map(&tv, v, D, p.Hkv, p.N, 1, BN)) return cudaErrorInvalidValue;
+  cudaError_t e = cudaFuncSetAttribute(fwd_partial_sm100_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       int(kSmemBytes));
+  if (e != cudaSuccess) return e;
+  fwd_partial_sm100_kernel<<<p.W, kThreads, kSmemBytes, s>>>(tq, tk, tv, p, scale * kLog2e, part_o, part_m,
+                                                             part_l);
+  return cudaGetLastError();
+}
+
+}  // namespace splitkv

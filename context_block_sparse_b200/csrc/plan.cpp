@@ -434,7 +434,8 @@ int splitkv_plan_upload(splitkv_plan_t* P, void* stream) {
   }
   const size_t table_bytes = off;
   const size_t timer_off = table_bytes;
-  const size_t total = timer_off + splitkv::align_up(size_t(P->W + P->Wb) * 2 * sizeof(long long), 256);
+  const size_t status_off = timer_off + splitkv::align_up(size_t(P->W + P->Wb) * 2 * sizeof(long long), 256);
+  const size_t total = status_off + 256;
 
   if (P->upload_pending) {
     if (cudaEventSynchronize(P->upload_ev) != cudaSuccess) return SPLITKV_ERR_CUDA;
@@ -492,6 +493,7 @@ int splitkv_plan_upload(splitkv_plan_t* P, void* stream) {
   v.block_entries = reinterpret_cast<const int*>(d + segs[7].off);
   v.zero_chunks = reinterpret_cast<const int*>(d + segs[8].off);
   v.timers = reinterpret_cast<long long*>(d + timer_off);
+  v.status = reinterpret_cast<int*>(d + status_off);
   v.num_zero_chunks = int(P->zero_chunks.size());
   v.N = int(P->N);
   v.Nq = int(P->Nq);

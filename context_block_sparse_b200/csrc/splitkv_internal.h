@@ -25,6 +25,7 @@ struct DevPlan {
   const int*  block_entries;    // [E]   entry ids of each block, ascending chunk
   const int*  zero_chunks;      // [Z]   chunks no block reads (backward zero fill)
   long long*  timers;           // [W + Wb][2] global-timer stamps: forward CTAs, then backward CTAs
+  int*        status;           // device status word: 0, or a SPLITKV_ERR_* code a kernel recorded
   int num_zero_chunks;
   int N, Nq, A, bs, Hq, Hkv, G, d, C, num_chunks, E, W, Wb;
 };

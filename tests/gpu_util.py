@@ -45,6 +45,8 @@ def run(w, bwd=False, o_dtype="f32", W=148, Wb=0, q_slice=0, equal_count=False, 
             for n, x in g.items():
                 out[n] = x.cpu().numpy().astype(np.float64)
     torch.cuda.synchronize()
+    import context_block_sparse_b200 as skv
+    skv.splitkv_plan_status(att.plan)
     return out, att, t
 
 
