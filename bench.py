@@ -170,6 +170,11 @@ def _kernel_work(st, w, E):
     }
 
 
+def _bwd_is_two_launches(w) -> bool:
+    return (w.head_dim == 128 and (w.num_q_heads // w.num_kv_heads * w.block_size) % 8 == 0
+            and os.environ.get("SPLITKV_BWD_KERNEL") != "mma")
+
+
 def run_ours(args, world, rank, local):
     import torch
     import torch.distributed as dist
@@ -186,7 +191,7 @@ def run_ours(args, world, rank, local):
     w = make_workload(args.workload, num_anchors=args.anchors, with_grad=True)
     sms = torch.cuda.get_device_properties(dev).multi_processor_count
     W = args.workers or sms
-    Wb = args.bwd_workers or 2 * sms
+    Wb = args.bwd_workers or sms
     stream = torch.cuda.current_stream(dev)
 
     def up(name):
@@ -335,7 +340,9 @@ def run_ours(args, world, rank, local):
         "plan_us": float(np.median(plan_us)) if plan_us else None,
         "kernels": kern,
         "roofline": roof,
-        "gpu_launches": len(kernels) * args.steps,
+        # the backward partial step is two launches (dK/dV kernel + dQ kernel) on the tcgen05
+        # path (head_dim 128, G * bs a multiple of 8), one on the mma.sync path
+        "gpu_launches": (len(kernels) + (1 if _bwd_is_two_launches(w) else 0)) * args.steps,
         "clocks": clocks,
     }
 
@@ -489,7 +496,7 @@ def main(argv=None):
     ap.add_argument("--workload", default="bwd", choices=["tiny", "drafter", "budget", "skew", "bwd"])
     ap.add_argument("--anchors", type=int, default=None)
     ap.add_argument("--workers", type=int, default=0, help="forward CTAs (default: SM count)")
-    ap.add_argument("--bwd-workers", type=int, default=0, help="backward CTAs (default: 2 x SM count)")
+    ap.add_argument("--bwd-workers", type=int, default=0, help="backward CTAs (default: SM count)")
     ap.add_argument("--q-slice", type=int, default=0)
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--cpu-seconds", type=float, default=15.0)

@@ -1,0 +1,645 @@
+// Backward of the chunk partial attention on the 5th-generation tensor cores
+// (tcgen05 / TMEM / TMA), head_dim 128.
+//
+// News page "Split-KV speeds diffusion drafter training by keeping long-context
+// data local", section "Exchange the smaller side": keys and values stay local
+// to their shard through the backward pass, and the query-side result is
+// reduced across shards.  Here a shard is a KV chunk owned by one persistent CTA.
+//
+// Tensor memory (512 columns) cannot hold dK, dV, S, dP and dQ of a 128-key by
+// 128-row tile pair at once, so the backward runs as two kernels that both
+// recompute P = exp(s - lse) from the saved log-sum-exp:
+//
+//  dkdv kernel (KV-stationary, backward LPT schedule, whole chunks): for every
+//    128-key tile of the chunk, for every query tile that meets it:
+//      S^T = K Q^T, dP^T = V dO^T          (TMEM, keys as lanes)
+//      P^T, dS^T = P^T (dP^T - Delta)      (thread = key; bf16, written back
+//                                           over S^T / dP^T)
+//      dV += P^T dO, dK += dS^T Q          (A operand from TMEM)
+//    then dK (times scale) and dV of the tile's keys go to global memory; keys
+//    that no query reads get zeros.
+//  dq kernel (Q-stationary, forward LPT schedule): for every query tile, over
+//    the 128-key tiles of its chunk:
+//      S = Q K^T (double-buffered), dP = dO V^T, dS = P (dP - Delta)
+//      dQ += dS K                           (A operand from TMEM)
+//    then scale * dQ is written once as the (chunk, block) entry's dq partial.
+//
+// Roles per CTA (256 threads): warp 0 TMA producer, warp 1 MMA issuer (one
+// thread), warp 2 tensor-memory allocation, warps 4-7 element-wise work and
+// epilogue (thread = TMEM lane).  Waits are bounded; a timeout is recorded in
+// the plan's status word and every role winds down.
+#include <cfloat>
+
+#include "sm100.cuh"
+#include "splitkv.h"
+#include "splitkv_internal.h"
+
+namespace splitkv {
+namespace {
+
+using namespace sm100;
+
+constexpr int D = 128;
+constexpr int BT = 128;                // keys per key tile = rows per query tile
+constexpr int kThreads = 256;
+constexpr uint32_t kHalf = 128 * 128;  // one 64-column half of a 128-row bf16 tile
+constexpr uint32_t kTile = 2 * kHalf;  // 32 KB
+constexpr uint32_t kIdescKM = idesc_bf16_f32(128, 128, 0);  // B K-major
+constexpr uint32_t kIdescMN = idesc_bf16_f32(128, D, 1);    // B MN-major
+constexpr uint32_t kSmemBytes = 6 * kTile + 4096 + 256 + 1024;
+
+__device__ __forceinline__ void abort_kernel(volatile int* flag, const DevPlan& p) {
+  *flag = 1;
+  atomicExch(p.status, SPLITKV_ERR_TIMEOUT);
+}
+
+// K-major SW128 descriptor of the k-th 16-column step of a 128-row tile.
+__device__ __forceinline__ uint64_t kmajor(uint32_t tile, int kk) {
+  return smem_desc_sw128(tile + (kk >> 2) * kHalf + (kk & 3) * 32, 16, 1024);
+}
+// MN-major SW128 descriptor of the k-th 16-row step of a 128-row tile (N = 128 columns).
+__device__ __forceinline__ uint64_t mnmajor(uint32_t tile, int kk) {
+  return smem_desc_sw128(tile + kk * 2048, kHalf, 1024);
+}
+
+// Row metadata of query-tile row r (rows ordered slot, token, head).
+struct RowMeta {
+  bool valid;
+  int lo, hi, rec;
+  size_t qrow;
+};
+__device__ __forceinline__ RowMeta row_meta(const DevPlan& p, const int4& tile, int g, int r) {
+  RowMeta m;
+  const int rps = p.G * p.bs;
+  const int slot = r / rps;
+  const int within = r - slot * rps;
+  const int tt = within / p.G, hh = within - tt * p.G;
+  m.valid = slot < tile.y - tile.x;
+  m.lo = m.hi = m.rec = 0;
+  m.qrow = 0;
+  if (m.valid) {
+    const int e = tile.x + slot;
+    const int4 ent = p.entries[e];
+    m.lo = ent.y;
+    m.hi = ent.z;
+    m.rec = (e * p.bs + tt) * p.Hq + g * p.G + hh;
+    m.qrow = size_t(ent.x * p.bs + tt) * p.Hq + g * p.G + hh;
+  }
+  return m;
+}
+
+// TMA of one query tile's rows (Q or dO layout) into a 128-row SW128 tile
+// (kTile bytes).  Slots past the tile's last block are loaded from token
+// coordinate Nq, outside the tensor, so that the hardware fills them with
+// zeros: the dK/dV products contract over all 128 rows.
+__device__ __forceinline__ void load_query_tile(const DevPlan& p, const int4& tile, int g, uint8_t* dst,
+                                                const CUtensorMap* map, uint64_t* bar) {
+  const int rps = p.G * p.bs;
+  const uint32_t slot_bytes = uint32_t(rps) * 128;
+  const int n = tile.y - tile.x;
+  for (int s = 0; s < BT / rps; ++s) {
+    const int z = s < n ? p.entries[tile.x + s].x * p.bs : p.Nq;
+    for (int dh = 0; dh < 2; ++dh) tma_load_3d(dst + dh * kHalf + s * slot_bytes, map, bar, dh * 64, g * p.G, z);
+  }
+}
+
+__device__ __forceinline__ void setup_common(uint64_t* bars, int nbars, const uint32_t* counts, uint32_t* tmem_slot,
+                                             int warp) {
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < nbars; ++i) mbar_init(&bars[i], counts[i]);
+    mbar_fence_init();
+  }
+  if (warp == 2) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+}
+
+// ============================================================================
+// dkdv kernel
+// ============================================================================
+struct DkdvBars {
+  uint64_t kv_full, kv_empty, qd_full[2], qd_empty[2], st_ready, pds_ready, dkv_ready, dkv_free, mma_done,
+      meta_ready[2];
+  uint32_t tmem_base;
+  int abort_flag;
+};
+constexpr int kDkdvNumBars = 13;
+
+__global__ void __launch_bounds__(kThreads, 1)
+    bwd_dkdv_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_do,
+                          const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                          DevPlan p, const float* __restrict__ lse, const float* __restrict__ delta, float scale,
+                          float* __restrict__ dk, float* __restrict__ dv) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sK = smem;
+  uint8_t* sV = smem + kTile;
+  uint8_t* sQ = smem + 2 * kTile;   // [2 stages]
+  uint8_t* sdO = smem + 4 * kTile;  // [2 stages]
+  int2* meta_lohi = reinterpret_cast<int2*>(smem + 6 * kTile);                // [2][128]
+  float2* meta_ld = reinterpret_cast<float2*>(smem + 6 * kTile + 2048);       // [2][128] (lse2, delta)
+  DkdvBars* B = reinterpret_cast<DkdvBars*>(smem + 6 * kTile + 4096);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int w = blockIdx.x;
+  volatile int* abort_flag = &B->abort_flag;
+  if (tid == 0) {
+    p.timers[(p.W + w) * 2 + 0] = global_timer_ns();
+    B->abort_flag = 0;
+  }
+  {
+    const uint32_t counts[kDkdvNumBars] = {1, 1, 1, 1, 1, 1, 1, 128, 1, 128, 1, 128, 128};
+    setup_common(&B->kv_full, kDkdvNumBars, counts, &B->tmem_base, warp);
+  }
+  const uint32_t tmem = B->tmem_base;
+  const size_t kv_row = size_t(p.Hkv) * D;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      prefetch_tmap(&tm_q);
+      prefetch_tmap(&tm_do);
+      prefetch_tmap(&tm_k);
+      prefetch_tmap(&tm_v);
+      uint32_t kt_count = 0, qd_count = 0;
+      bool ok = true;
+      for (int it = p.bwd_worker_ptr[w]; ok && it < p.bwd_worker_ptr[w + 1]; ++it) {
+        const int4 item = p.bwd_items[it];
+        const int g = item.y, c0 = item.x * p.C, c1 = min(c0 + p.C, p.N);
+        for (int k0 = c0; ok && k0 < c1; k0 += BT) {
+          if (!mbar_wait(&B->kv_empty, (kt_count & 1) ^ 1, abort_flag)) { ok = false; break; }
+          mbar_expect_tx(&B->kv_full, 2 * kTile);
+          for (int dh = 0; dh < 2; ++dh) {
+            tma_load_3d(sK + dh * kHalf, &tm_k, &B->kv_full, dh * 64, g, k0);
+            tma_load_3d(sV + dh * kHalf, &tm_v, &B->kv_full, dh * 64, g, k0);
+          }
+          ++kt_count;
+          for (int t = item.z; t < item.w; ++t) {
+            const int4 tile = p.tiles[t];
+            if (!(tile.z < k0 + BT && tile.w > k0)) continue;
+            const int s = qd_count & 1;
+            if (!mbar_wait(&B->qd_empty[s], ((qd_count >> 1) & 1) ^ 1, abort_flag)) { ok = false; break; }
+            mbar_expect_tx(&B->qd_full[s], 2 * kTile);
+            load_query_tile(p, tile, g, sQ + s * kTile, &tm_q, &B->qd_full[s]);
+            load_query_tile(p, tile, g, sdO + s * kTile, &tm_do, &B->qd_full[s]);
+            ++qd_count;
+          }
+        }
+      }
+      if (!ok) abort_kernel(abort_flag, p);
+      if (kt_count > 0) mbar_drain(&B->kv_full, (kt_count - 1) & 1);
+      for (uint32_t c = qd_count >= 2 ? qd_count - 2 : 0; c < qd_count; ++c) mbar_drain(&B->qd_full[c & 1], (c >> 1) & 1);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      const uint32_t aK = smem_u32(sK), aV = smem_u32(sV), aQ = smem_u32(sQ), adO = smem_u32(sdO);
+      uint32_t kt_count = 0, qd_count = 0, pds_cnt = 0, dkvf_cnt = 0;
+      bool ok = true;
+      for (int it = p.bwd_worker_ptr[w]; ok && it < p.bwd_worker_ptr[w + 1]; ++it) {
+        const int4 item = p.bwd_items[it];
+        const int c0 = item.x * p.C, c1 = min(c0 + p.C, p.N);
+        for (int k0 = c0; ok && k0 < c1; k0 += BT) {
+          if (!mbar_wait(&B->kv_full, kt_count & 1, abort_flag)) { ok = false; break; }
+          tc_fence_after();
+          int u = 0;
+          for (int t = item.z; t < item.w; ++t) {
+            const int4 tile = p.tiles[t];
+            if (!(tile.z < k0 + BT && tile.w > k0)) continue;
+            const int s = qd_count & 1;
+            if (!mbar_wait(&B->qd_full[s], (qd_count >> 1) & 1, abort_flag)) { ok = false; break; }
+            tc_fence_after();
+            // S^T = K Q^T (cols 0..127), dP^T = V dO^T (cols 128..255)
+            for (int kk = 0; kk < D / 16; ++kk)
+              mma_ss(tmem + 0, kmajor(aK, kk), kmajor(aQ + s * kTile, kk), kIdescKM, kk > 0 ? 1u : 0u);
+            for (int kk = 0; kk < D / 16; ++kk)
+              mma_ss(tmem + 128, kmajor(aV, kk), kmajor(adO + s * kTile, kk), kIdescKM, kk > 0 ? 1u : 0u);
+            mma_commit(&B->st_ready);
+            if (!mbar_wait(&B->pds_ready, pds_cnt & 1, abort_flag)) { ok = false; break; }
+            ++pds_cnt;
+            if (u == 0) {
+              if (!mbar_wait(&B->dkv_free, (dkvf_cnt & 1) ^ 1, abort_flag)) { ok = false; break; }
+              ++dkvf_cnt;
+            }
+            tc_fence_after();
+            // dV (cols 384..) += P^T dO ; dK (cols 256..) += dS^T Q  -- A operands from TMEM
+            for (int kk = 0; kk < BT / 16; ++kk)
+              mma_ts(tmem + 384, tmem + 0 + kk * 8, mnmajor(adO + s * kTile, kk), kIdescMN,
+                     (u > 0 || kk > 0) ? 1u : 0u);
+            for (int kk = 0; kk < BT / 16; ++kk)
+              mma_ts(tmem + 256, tmem + 128 + kk * 8, mnmajor(aQ + s * kTile, kk), kIdescMN,
+                     (u > 0 || kk > 0) ? 1u : 0u);
+            mma_commit(&B->qd_empty[s]);
+            ++qd_count;
+            ++u;
+          }
+          if (!ok) break;
+          if (u > 0) mma_commit(&B->dkv_ready);
+          mma_commit(&B->kv_empty);
+          ++kt_count;
+        }
+      }
+      if (!ok) abort_kernel(abort_flag, p);
+      mma_commit(&B->mma_done);
+      mbar_drain(&B->mma_done, 0);
+    }
+  } else if (warp >= 4) {
+    const int r = ((warp & 3) << 5) + lane;   // key of the tile = TMEM lane; also the row this thread describes
+    const uint32_t lane_addr = uint32_t((warp & 3) << 5) << 16;
+    const uint32_t tSt = tmem + lane_addr;          // S^T / P^T
+    const uint32_t tdPt = tmem + lane_addr + 128;   // dP^T / dS^T
+    const uint32_t tdK = tmem + lane_addr + 256;
+    const uint32_t tdV = tmem + lane_addr + 384;
+    const float scale_log2 = scale * kLog2e;
+    // chunks no block reads: zeros for every KV head
+    for (int z = w; z < p.num_zero_chunks; z += p.Wb) {
+      const int c = p.zero_chunks[z];
+      const size_t first = size_t(c) * p.C * kv_row;
+      const size_t last = size_t(min(c * p.C + p.C, p.N)) * kv_row;
+      for (size_t i = first + size_t(r) * 4; i < last; i += size_t(128) * 4) {
+        *reinterpret_cast<float4*>(dk + i) = make_float4(0.f, 0.f, 0.f, 0.f);
+        *reinterpret_cast<float4*>(dv + i) = make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+    }
+    uint32_t qd_count = 0, st_cnt = 0, dkv_cnt = 0;
+    bool ok = true;
+    for (int it = p.bwd_worker_ptr[w]; ok && it < p.bwd_worker_ptr[w + 1]; ++it) {
+      const int4 item = p.bwd_items[it];
+      const int g = item.y, c0 = item.x * p.C, c1 = min(c0 + p.C, p.N);
+      for (int k0 = c0; ok && k0 < c1; k0 += BT) {
+        const int key = k0 + r;
+        int n_meet = 0;
+        for (int t = item.z; t < item.w; ++t) {
+          const int4 tile = p.tiles[t];
+          if (!(tile.z < k0 + BT && tile.w > k0)) continue;
+          const int s = qd_count & 1;
+          {
+            // this thread describes row r of the query tile
+            const RowMeta m = row_meta(p, tile, g, r);
+            float l2 = INFINITY, dl = 0.f;
+            if (m.valid) {
+              const float L = lse[m.qrow];
+              l2 = (L == -INFINITY) ? INFINITY : L * kLog2e;
+              dl = delta[m.qrow];
+            }
+            meta_lohi[s * 128 + r] = make_int2(m.lo, m.hi);
+            meta_ld[s * 128 + r] = make_float2(l2, dl);
+          }
+          // every thread needs all 128 rows' metadata: bounded handoff through an mbarrier
+          mbar_arrive(&B->meta_ready[s]);
+          if (!warp_wait(&B->meta_ready[s], (qd_count >> 1) & 1, abort_flag)) { ok = false; break; }
+          if (!warp_wait(&B->st_ready, st_cnt & 1, abort_flag)) { ok = false; break; }
+          ++st_cnt;
+          tc_fence_after();
+#pragma unroll 1
+          for (int cc = 0; cc < 4; ++cc) {
+            uint32_t sv[32], dpv[32];
+            tmem_ld32(tSt + cc * 32, sv);
+            tmem_ld32(tdPt + cc * 32, dpv);
+            tmem_wait_ld();
+            uint32_t pk[16], dk16[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              float pr[2], ds[2];
+#pragma unroll
+              for (int e = 0; e < 2; ++e) {
+                const int row = cc * 32 + 2 * i + e;
+                const int2 lh = meta_lohi[s * 128 + row];
+                const float2 ld = meta_ld[s * 128 + row];
+                const bool in = key >= lh.x && key < lh.y;
+                pr[e] = in ? fast_exp2(__uint_as_float(sv[2 * i + e]) * scale_log2 - ld.x) : 0.f;
+                ds[e] = pr[e] * (__uint_as_float(dpv[2 * i + e]) - ld.y);
+              }
+              pk[i] = pack_bf16(pr[0], pr[1]);
+              dk16[i] = pack_bf16(ds[0], ds[1]);
+            }
+            tmem_st16(tSt + cc * 16, pk);
+            tmem_st16(tdPt + cc * 16, dk16);
+          }
+          tmem_wait_st();
+          tc_fence_before();
+          mbar_arrive(&B->pds_ready);
+          ++qd_count;
+          ++n_meet;
+        }
+        if (!ok) break;
+        // epilogue of the key tile: dK * scale, dV (zeros when no query met it)
+        float* dkr = dk + (size_t(key) * p.Hkv + g) * D;
+        float* dvr = dv + (size_t(key) * p.Hkv + g) * D;
+        const bool own = key < c1;
+        if (n_meet > 0) {
+          if (!warp_wait(&B->dkv_ready, dkv_cnt & 1, abort_flag)) { ok = false; break; }
+          ++dkv_cnt;
+          tc_fence_after();
+#pragma unroll 1
+          for (int cc = 0; cc < D / 32; ++cc) {
+            uint32_t a[32], b[32];
+            tmem_ld32(tdK + cc * 32, a);
+            tmem_ld32(tdV + cc * 32, b);
+            tmem_wait_ld();
+            if (own) {
+#pragma unroll
+              for (int i = 0; i < 32; i += 4) {
+                *reinterpret_cast<float4*>(dkr + cc * 32 + i) =
+                    make_float4(scale * __uint_as_float(a[i]), scale * __uint_as_float(a[i + 1]),
+                                scale * __uint_as_float(a[i + 2]), scale * __uint_as_float(a[i + 3]));
+                *reinterpret_cast<float4*>(dvr + cc * 32 + i) =
+                    make_float4(__uint_as_float(b[i]), __uint_as_float(b[i + 1]), __uint_as_float(b[i + 2]),
+                                __uint_as_float(b[i + 3]));
+              }
+            }
+          }
+          tc_fence_before();
+          mbar_arrive(&B->dkv_free);
+        } else if (own) {
+          for (int i = 0; i < D; i += 4) {
+            *reinterpret_cast<float4*>(dkr + i) = make_float4(0.f, 0.f, 0.f, 0.f);
+            *reinterpret_cast<float4*>(dvr + i) = make_float4(0.f, 0.f, 0.f, 0.f);
+          }
+        }
+      }
+    }
+    if (!ok) abort_kernel(abort_flag, p);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 2) tmem_dealloc(tmem, 512);
+  if (tid == 0) p.timers[(p.W + w) * 2 + 1] = global_timer_ns();
+}
+
+// ============================================================================
+// dq kernel
+// ============================================================================
+struct DqBars {
+  uint64_t qd_full, qd_empty, k_full[2], v_full[2], kv_empty[2], s_ready[2], dp_ready, ds_ready, dq_ready, dq_free,
+      mma_done;
+  uint32_t tmem_base;
+  int abort_flag;
+};
+constexpr int kDqNumBars = 15;
+
+// The query tiles of a worker's forward schedule, one at a time.
+struct TileIter {
+  const DevPlan* p;
+  int it, it_end, t, t_end, g;
+  __device__ void init(const DevPlan* plan, int w) {
+    p = plan;
+    it = plan->fwd_worker_ptr[w];
+    it_end = plan->fwd_worker_ptr[w + 1];
+    t = t_end = 0;
+    g = 0;
+  }
+  __device__ bool next(int& tile_id, int& head) {
+    while (t >= t_end) {
+      if (it >= it_end) return false;
+      const int4 item = p->fwd_items[it++];
+      g = item.y;
+      t = item.z;
+      t_end = item.w;
+    }
+    tile_id = t++;
+    head = g;
+    return true;
+  }
+};
+
+__global__ void __launch_bounds__(kThreads, 1)
+    bwd_dq_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_do,
+                        const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                        DevPlan p, const float* __restrict__ lse, const float* __restrict__ delta, float scale,
+                        float* __restrict__ dq_part) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sQ = smem;
+  uint8_t* sdO = smem + kTile;
+  uint8_t* sK = smem + 2 * kTile;   // [2 stages]
+  uint8_t* sV = smem + 4 * kTile;   // [2 stages]
+  DqBars* B = reinterpret_cast<DqBars*>(smem + 6 * kTile + 4096);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int w = blockIdx.x;
+  volatile int* abort_flag = &B->abort_flag;
+  if (tid == 0) B->abort_flag = 0;
+  {
+    const uint32_t counts[kDqNumBars] = {1, 1, 1, 1, 1, 1, 1, 1, 1, 1, 1, 128, 1, 128, 1};
+    setup_common(&B->qd_full, kDqNumBars, counts, &B->tmem_base, warp);
+  }
+  const uint32_t tmem = B->tmem_base;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      prefetch_tmap(&tm_q);
+      prefetch_tmap(&tm_do);
+      prefetch_tmap(&tm_k);
+      prefetch_tmap(&tm_v);
+      TileIter ti;
+      ti.init(&p, w);
+      int t, g;
+      uint32_t tile_count = 0, kv_count = 0, q_issued = 0;
+      bool ok = true;
+      while (ok && ti.next(t, g)) {
+        const int4 tile = p.tiles[t];
+        if (!mbar_wait(&B->qd_empty, (tile_count & 1) ^ 1, abort_flag)) { ok = false; break; }
+        mbar_expect_tx(&B->qd_full, 2 * kTile);
+        load_query_tile(p, tile, g, sQ, &tm_q, &B->qd_full);
+        load_query_tile(p, tile, g, sdO, &tm_do, &B->qd_full);
+        ++q_issued;
+        const int n_kt = (tile.w - tile.z + BT - 1) / BT;
+        for (int j = 0; j < n_kt; ++j, ++kv_count) {
+          const int s = kv_count & 1;
+          if (!mbar_wait(&B->kv_empty[s], ((kv_count >> 1) & 1) ^ 1, abort_flag)) { ok = false; break; }
+          const int k0 = tile.z + j * BT;
+          mbar_expect_tx(&B->k_full[s], kTile);
+          for (int dh = 0; dh < 2; ++dh) tma_load_3d(sK + s * kTile + dh * kHalf, &tm_k, &B->k_full[s], dh * 64, g, k0);
+          mbar_expect_tx(&B->v_full[s], kTile);
+          for (int dh = 0; dh < 2; ++dh) tma_load_3d(sV + s * kTile + dh * kHalf, &tm_v, &B->v_full[s], dh * 64, g, k0);
+        }
+        ++tile_count;
+      }
+      if (!ok) abort_kernel(abort_flag, p);
+      if (q_issued > 0) mbar_drain(&B->qd_full, (q_issued - 1) & 1);
+      for (uint32_t c = kv_count >= 2 ? kv_count - 2 : 0; c < kv_count; ++c) {
+        mbar_drain(&B->k_full[c & 1], (c >> 1) & 1);
+        mbar_drain(&B->v_full[c & 1], (c >> 1) & 1);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      const uint32_t aK = smem_u32(sK), aV = smem_u32(sV), aQ = smem_u32(sQ), adO = smem_u32(sdO);
+      TileIter ti;
+      ti.init(&p, w);
+      int t, g;
+      uint32_t tile_count = 0, kv_count = 0, ds_cnt = 0, dqf_cnt = 0;
+      bool ok = true;
+      while (ok && ti.next(t, g)) {
+        const int4 tile = p.tiles[t];
+        const int n_kt = (tile.w - tile.z + BT - 1) / BT;
+        if (!mbar_wait(&B->qd_full, tile_count & 1, abort_flag)) { ok = false; break; }
+        const uint32_t c0 = kv_count;
+        {
+          const int s = c0 & 1;
+          if (!mbar_wait(&B->k_full[s], (c0 >> 1) & 1, abort_flag)) { ok = false; break; }
+          tc_fence_after();
+          for (int kk = 0; kk < D / 16; ++kk)
+            mma_ss(tmem + s * 128, kmajor(aQ, kk), kmajor(aK + s * kTile, kk), kIdescKM, kk > 0 ? 1u : 0u);
+          mma_commit(&B->s_ready[s]);
+          if (!mbar_wait(&B->v_full[s], (c0 >> 1) & 1, abort_flag)) { ok = false; break; }
+          tc_fence_after();
+          for (int kk = 0; kk < D / 16; ++kk)
+            mma_ss(tmem + 256, kmajor(adO, kk), kmajor(aV + s * kTile, kk), kIdescKM, kk > 0 ? 1u : 0u);
+          mma_commit(&B->dp_ready);
+        }
+        for (int j = 0; j < n_kt; ++j) {
+          const uint32_t c = c0 + j;
+          const int s = c & 1, s1 = (c + 1) & 1;
+          const bool more = j + 1 < n_kt;
+          if (more) {   // next S into the other buffer while this tile's dS is formed
+            if (!mbar_wait(&B->k_full[s1], ((c + 1) >> 1) & 1, abort_flag)) { ok = false; break; }
+            tc_fence_after();
+            for (int kk = 0; kk < D / 16; ++kk)
+              mma_ss(tmem + s1 * 128, kmajor(aQ, kk), kmajor(aK + s1 * kTile, kk), kIdescKM, kk > 0 ? 1u : 0u);
+            mma_commit(&B->s_ready[s1]);
+          }
+          if (!mbar_wait(&B->ds_ready, ds_cnt & 1, abort_flag)) { ok = false; break; }
+          ++ds_cnt;
+          if (j == 0) {
+            if (!mbar_wait(&B->dq_free, (dqf_cnt & 1) ^ 1, abort_flag)) { ok = false; break; }
+            ++dqf_cnt;
+          }
+          tc_fence_after();
+          // dQ (cols 384..) += dS K : dS in TMEM (columns 0..63 of S buffer s), K MN-major
+          for (int kk = 0; kk < BT / 16; ++kk)
+            mma_ts(tmem + 384, tmem + s * 128 + kk * 8, mnmajor(aK + s * kTile, kk), kIdescMN,
+                   (j > 0 || kk > 0) ? 1u : 0u);
+          mma_commit(&B->kv_empty[s]);
+          if (more) {
+            if (!mbar_wait(&B->v_full[s1], ((c + 1) >> 1) & 1, abort_flag)) { ok = false; break; }
+            tc_fence_after();
+            for (int kk = 0; kk < D / 16; ++kk)
+              mma_ss(tmem + 256, kmajor(adO, kk), kmajor(aV + s1 * kTile, kk), kIdescKM, kk > 0 ? 1u : 0u);
+            mma_commit(&B->dp_ready);
+          }
+        }
+        if (!ok) break;
+        mma_commit(&B->dq_ready);
+        mma_commit(&B->qd_empty);
+        kv_count += n_kt;
+        ++tile_count;
+      }
+      if (!ok) abort_kernel(abort_flag, p);
+      mma_commit(&B->mma_done);
+      mbar_drain(&B->mma_done, 0);
+    }
+  } else if (warp >= 4) {
+    const int r = ((warp & 3) << 5) + lane;
+    const uint32_t lane_addr = uint32_t((warp & 3) << 5) << 16;
+    const uint32_t tdP = tmem + lane_addr + 256;
+    const uint32_t tdQ = tmem + lane_addr + 384;
+    const float scale_log2 = scale * kLog2e;
+    TileIter ti;
+    ti.init(&p, w);
+    int t, g;
+    uint32_t kv_count = 0, dp_cnt = 0, dq_cnt = 0;
+    bool ok = true;
+    while (ok && ti.next(t, g)) {
+      const int4 tile = p.tiles[t];
+      const int n_kt = (tile.w - tile.z + BT - 1) / BT;
+      const RowMeta m = row_meta(p, tile, g, r);
+      float l2 = INFINITY, dl = 0.f;
+      if (m.valid) {
+        const float L = lse[m.qrow];
+        l2 = (L == -INFINITY) ? INFINITY : L * kLog2e;
+        dl = delta[m.qrow];
+      }
+      for (int j = 0; j < n_kt; ++j) {
+        const uint32_t c = kv_count + j;
+        const int s = c & 1;
+        if (!warp_wait(&B->s_ready[s], (c >> 1) & 1, abort_flag)) { ok = false; break; }
+        if (!warp_wait(&B->dp_ready, dp_cnt & 1, abort_flag)) { ok = false; break; }
+        ++dp_cnt;
+        tc_fence_after();
+        const uint32_t tS = tmem + lane_addr + s * 128;
+        const int k0 = tile.z + j * BT;
+#pragma unroll 1
+        for (int cc = 0; cc < 4; ++cc) {
+          uint32_t sv[32], dpv[32];
+          tmem_ld32(tS + cc * 32, sv);
+          tmem_ld32(tdP + cc * 32, dpv);
+          tmem_wait_ld();
+          uint32_t pk[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            float ds[2];
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+              const int key = k0 + cc * 32 + 2 * i + e;
+              const bool in = key >= m.lo && key < m.hi;
+              const float pr = in ? fast_exp2(__uint_as_float(sv[2 * i + e]) * scale_log2 - l2) : 0.f;
+              ds[e] = pr * (__uint_as_float(dpv[2 * i + e]) - dl);
+            }
+            pk[i] = pack_bf16(ds[0], ds[1]);
+          }
+          tmem_st16(tS + cc * 16, pk);
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(&B->ds_ready);
+      }
+      if (!ok) break;
+      kv_count += n_kt;
+      if (!warp_wait(&B->dq_ready, dq_cnt & 1, abort_flag)) { ok = false; break; }
+      ++dq_cnt;
+      tc_fence_after();
+      float* dst = dq_part + size_t(m.rec) * D;
+#pragma unroll 1
+      for (int cc = 0; cc < D / 32; ++cc) {
+        uint32_t v[32];
+        tmem_ld32(tdQ + cc * 32, v);
+        tmem_wait_ld();
+        if (m.valid) {
+#pragma unroll
+          for (int i = 0; i < 32; i += 4)
+            *reinterpret_cast<float4*>(dst + cc * 32 + i) =
+                make_float4(scale * __uint_as_float(v[i]), scale * __uint_as_float(v[i + 1]),
+                            scale * __uint_as_float(v[i + 2]), scale * __uint_as_float(v[i + 3]));
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&B->dq_free);
+    }
+    if (!ok) abort_kernel(abort_flag, p);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 2) tmem_dealloc(tmem, 512);
+}
+
+}  // namespace
+
+bool bwd_sm100_supported(const DevPlan& p) {
+  const int rows = p.G * p.bs;
+  return p.d == D && rows % 8 == 0 && rows <= BT && tensor_maps_available();
+}
+
+cudaError_t launch_bwd_partial_sm100(const DevPlan& p, const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                                     const uint16_t* dout, const float* lse, const float* delta, float scale,
+                                     float* dk, float* dv, float* dq_part, cudaStream_t s) {
+  CUtensorMap tq, tdo, tk, tv;
+  if (!make_bf16_map_3d(&tq, q, D, p.Hq, p.Nq, p.G, p.bs) || !make_bf16_map_3d(&tdo, dout, D, p.Hq, p.Nq, p.G, p.bs) ||
+      !make_bf16_map_3d(&tk, k, D, p.Hkv, p.N, 1, BT) || !make_bf16_map_3d(&tv, v, D, p.Hkv, p.N, 1, BT))
+    return cudaErrorInvalidValue;
+  cudaError_t e = cudaFuncSetAttribute(bwd_dkdv_sm100_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       int(kSmemBytes));
+  if (e != cudaSuccess) return e;
+  e = cudaFuncSetAttribute(bwd_dq_sm100_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(kSmemBytes));
+  if (e != cudaSuccess) return e;
+  bwd_dkdv_sm100_kernel<<<p.Wb, kThreads, kSmemBytes, s>>>(tq, tdo, tk, tv, p, lse, delta, scale, dk, dv);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  bwd_dq_sm100_kernel<<<p.W, kThreads, kSmemBytes, s>>>(tq, tdo, tk, tv, p, lse, delta, scale, dq_part);
+  return cudaGetLastError();
+}
+
+}  // namespace splitkv

@@ -172,15 +172,18 @@ __global__ void __launch_bounds__(kThreads, 1)
           tb = p.tiles[tB];
           nB = tb.y - tb.x;
         }
-        mbar_expect_tx(&bars->q_full, uint32_t(nA + nB) * 2u * slot_bytes);
-        for (int x = 0; x < 2; ++x) {
+        // whole tiles: slots past a tile's last block come from token coordinate
+        // Nq (outside the tensor) and are zero-filled
+        const int nx = tB >= 0 ? 2 : 1;
+        mbar_expect_tx(&bars->q_full, uint32_t(nx) * kTile);
+        for (int x = 0; x < nx; ++x) {
           const int n = x == 0 ? nA : nB;
           const int e0 = x == 0 ? ta.x : tb.x;
           uint8_t* qbuf = smem + kOffQ + x * kTile;
-          for (int s = 0; s < n; ++s) {
-            const int blk = p.entries[e0 + s].x;
+          for (int s = 0; s < BM / rows_per_slot; ++s) {
+            const int z = s < n ? p.entries[e0 + s].x * p.bs : p.Nq;
             for (int dh = 0; dh < 2; ++dh)
-              tma_load_3d(qbuf + dh * kHalf + s * slot_bytes, &tm_q, &bars->q_full, dh * 64, g * p.G, blk * p.bs);
+              tma_load_3d(qbuf + dh * kHalf + s * slot_bytes, &tm_q, &bars->q_full, dh * 64, g * p.G, z);
           }
         }
         ++q_issued;
@@ -419,54 +422,19 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (tid == 0) p.timers[w * 2 + 1] = global_timer_ns();
 }
 
-// ---------------------------------------------------------------- host side
-using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
-                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
-                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn encode_fn() {
-  static EncodeTiledFn fn = nullptr;
-  static bool tried = false;
-  if (!tried) {
-    tried = true;
-    void* ptr = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeTiledFn>(ptr);
-    else
-      cudaGetLastError();
-  }
-  return fn;
-}
-
-// 3-D bf16 tensor [dim2][dim1][dim0] (dim0 contiguous), box {64, box1, box2}, 128-byte swizzle.
-bool make_map(CUtensorMap* m, const void* base, uint64_t dim0, uint64_t dim1, uint64_t dim2, uint32_t box1,
-              uint32_t box2) {
-  EncodeTiledFn fn = encode_fn();
-  if (!fn) return false;
-  const cuuint64_t dims[3] = {dim0, dim1, dim2};
-  const cuuint64_t strides[2] = {dim0 * 2, dim0 * dim1 * 2};
-  const cuuint32_t box[3] = {64, box1, box2};
-  const cuuint32_t estr[3] = {1, 1, 1};
-  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 }  // namespace
 
 bool fwd_sm100_supported(const DevPlan& p) {
   const int rows = p.G * p.bs;
-  return p.d == D && rows % 8 == 0 && rows <= BM && encode_fn() != nullptr;
+  return p.d == D && rows % 8 == 0 && rows <= BM && tensor_maps_available();
 }
 
 cudaError_t launch_fwd_partial_sm100(const DevPlan& p, const uint16_t* q, const uint16_t* k, const uint16_t* v,
                                      float scale, float* part_o, float* part_m, float* part_l, cudaStream_t s) {
   CUtensorMap tq, tk, tv;
-  if (!make_map(&tq, q, D, p.Hq, p.Nq, p.G, p.bs)) return cudaErrorInvalidValue;
-  if (!make_map(&tk, k, D, p.Hkv, p.N, 1, BN)) return cudaErrorInvalidValue;
-  if (!make_map(&tv, v, D, p.Hkv, p.N, 1, BN)) return cudaErrorInvalidValue;
+  if (!make_bf16_map_3d(&tq, q, D, p.Hq, p.Nq, p.G, p.bs)) return cudaErrorInvalidValue;
+  if (!make_bf16_map_3d(&tk, k, D, p.Hkv, p.N, 1, BN)) return cudaErrorInvalidValue;
+  if (!make_bf16_map_3d(&tv, v, D, p.Hkv, p.N, 1, BN)) return cudaErrorInvalidValue;
   cudaError_t e = cudaFuncSetAttribute(fwd_partial_sm100_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        int(kSmemBytes));
   if (e != cudaSuccess) return e;

@@ -61,6 +61,13 @@ inline BwdWs bwd_ws_layout(long long E, int Nq, int bs, int Hq, int d) {
   return w;
 }
 
+// ---- TMA tensor maps (tensor_maps.cpp) ------------------------------------
+// 3-D bf16 tensor [dim2][dim1][dim0] (dim0 contiguous), box {64, box1, box2},
+// 128-byte swizzle, zero fill out of bounds; `map` points at a CUtensorMap.
+bool tensor_maps_available();
+bool make_bf16_map_3d(void* map, const void* base, uint64_t dim0, uint64_t dim1, uint64_t dim2, uint32_t box1,
+                      uint32_t box2);
+
 // ---- kernel launchers (defined in the .cu files) ---------------------------
 cudaError_t launch_fwd_partial(const DevPlan& p, const uint16_t* q, const uint16_t* k,
                                const uint16_t* v, float scale, float* part_o, float* part_m,
