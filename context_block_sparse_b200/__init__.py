@@ -37,6 +37,12 @@ class SplitKVError(RuntimeError):
         super().__init__(f"{fn}: {msg} ({status})")
 
 
+def _with_site(err: "SplitKVError", site: int) -> "SplitKVError":
+    if site:
+        err.args = (f"{err.args[0]} [first timed-out wait: file {site // 10000}, line {site % 10000}]",)
+    return err
+
+
 def _check(fn: str, status: int) -> None:
     if status != _abi.OK:
         raise SplitKVError(fn, status)
@@ -246,7 +252,12 @@ def splitkv_attn_fwd_static_scratch(plan: Plan, q, k, v, kb, vb, scale: float, o
 
 def splitkv_plan_status(plan: Plan, stream=None) -> None:
     """Raise SplitKVError if a kernel of this plan recorded an error (e.g. a timed-out wait)."""
-    _check("splitkv_plan_status", _lib.splitkv_plan_status(plan.handle, _stream_ptr(stream)))
+    site = ctypes.c_int32(0)
+    st = _lib.splitkv_plan_status(plan.handle, _stream_ptr(stream), ctypes.byref(site))
+    if st != _abi.OK:
+        err = SplitKVError("splitkv_plan_status", st)
+        err.site = site.value
+        raise _with_site(err, site.value)
 
 
 def splitkv_read_cta_times(plan: Plan, which: int, stream=None) -> np.ndarray:

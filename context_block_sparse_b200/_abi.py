@@ -105,7 +105,7 @@ SIGNATURES = {
     "splitkv_bwd_partial": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _F, _P, _SZ, _P]),
     "splitkv_bwd_reduce": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _F, _P, _SZ, _P]),
     "splitkv_attn_fwd_static_scratch": (_I, [_P, _P, _P, _P, _P, _P, _F, _P, _I, _P, _P]),
-    "splitkv_plan_status": (_I, [_P, _P]),
+    "splitkv_plan_status": (_I, [_P, _P, ctypes.POINTER(ctypes.c_int32)]),
     "splitkv_read_cta_times": (_I, [_P, _I, ctypes.POINTER(ctypes.c_int64), ctypes.c_int64, _P]),
 }
 

@@ -53,11 +53,16 @@ def build(verbose: bool = False, force: bool = False, ptxas_info: bool = False) 
                 and os.path.getmtime(obj) >= max(os.path.getmtime(path), newest_header)):
             continue
         cmd = [nvcc, *ARCH, *COMMON, "-c", path, "-o", obj]
-        if ptxas_info and src.endswith(".cu"):
+        if src.endswith(".cu"):
             cmd.insert(1, "-Xptxas=-v")
         if verbose:
             print(" ".join(cmd), flush=True)
-        subprocess.run(cmd, check=True)
+        res = subprocess.run(cmd, capture_output=True, text=True)
+        if ptxas_info or res.returncode != 0:
+            sys.stderr.write(res.stderr)
+        if res.returncode != 0:
+            raise subprocess.CalledProcessError(res.returncode, cmd)
+
     link = [nvcc, *ARCH, "-shared", "-o", LIB, *objs,
             "-Xlinker", "--version-script=" + os.path.join(CSRC, "exports.map"), "-lcuda"]
     if verbose:

@@ -142,19 +142,20 @@ int splitkv_attn_bwd(const splitkv_plan_t* plan, const void* q, const void* k, c
   return splitkv_bwd_reduce(plan, q, kb, vb, lse, dout, dq, dkb, dvb, scale, ws, ws_bytes, stream);
 }
 
-int splitkv_plan_status(const splitkv_plan_t* plan, void* stream) {
+int splitkv_plan_status(const splitkv_plan_t* plan, void* stream, int32_t* site) {
   if (!plan) return SPLITKV_ERR_INVALID_ARG;
   const DevPlan* dp = splitkv::plan_device_view(plan);
   if (!dp) return SPLITKV_ERR_NOT_UPLOADED;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  int word = 0;
-  int st = cuda_status(cudaMemcpyAsync(&word, dp->status, sizeof(int), cudaMemcpyDeviceToHost, s));
+  int words[2] = {0, 0};
+  int st = cuda_status(cudaMemcpyAsync(words, dp->status, sizeof(words), cudaMemcpyDeviceToHost, s));
   if (st == SPLITKV_OK) st = cuda_status(cudaStreamSynchronize(s));
   if (st != SPLITKV_OK) return st;
-  if (word == 0) return SPLITKV_OK;
-  st = cuda_status(cudaMemsetAsync(dp->status, 0, sizeof(int), s));
+  if (site) *site = words[1];
+  if (words[0] == 0 && words[1] == 0) return SPLITKV_OK;
+  st = cuda_status(cudaMemsetAsync(dp->status, 0, sizeof(words), s));
   if (st == SPLITKV_OK) st = cuda_status(cudaStreamSynchronize(s));
-  return st != SPLITKV_OK ? st : word;
+  return st != SPLITKV_OK ? st : (words[0] != 0 ? words[0] : SPLITKV_ERR_TIMEOUT);
 }
 
 int splitkv_read_cta_times(const splitkv_plan_t* plan, int which, int64_t* out_ns, int64_t capacity,

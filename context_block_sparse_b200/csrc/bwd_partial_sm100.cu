@@ -48,10 +48,6 @@ constexpr uint32_t kIdescKM = idesc_bf16_f32(128, 128, 0);  // B K-major
 constexpr uint32_t kIdescMN = idesc_bf16_f32(128, D, 1);    // B MN-major
 constexpr uint32_t kSmemBytes = 6 * kTile + 4096 + 256 + 1024;
 
-__device__ __forceinline__ void abort_kernel(volatile int* flag, const DevPlan& p) {
-  *flag = 1;
-  atomicExch(p.status, SPLITKV_ERR_TIMEOUT);
-}
 
 // K-major SW128 descriptor of the k-th 16-column step of a 128-row tile.
 __device__ __forceinline__ uint64_t kmajor(uint32_t tile, int kk) {
@@ -118,6 +114,75 @@ __device__ __forceinline__ void setup_common(uint64_t* bars, int nbars, const ui
   tc_fence_after();
 }
 
+// dq kernel, one key tile of one row (thread = TMEM lane): dS = P (dP - Delta)
+// with P = exp2(s * c - lse2), zero outside the row's columns [a, b); bf16 dS
+// pairs go to TMEM columns [0, 64) of the score buffer.  Two 64-column halves.
+template <bool kMasked>
+__device__ __forceinline__ void ds_tile(uint32_t tS, uint32_t tdP, int a, int b, float c, float l2, float dl) {
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    uint32_t sv[64], dpv[64];
+    tmem_ld32p(tS + h * 64, sv);
+    tmem_ld32p(tS + h * 64 + 32, sv + 32);
+    tmem_ld32p(tdP + h * 64, dpv);
+    tmem_ld32p(tdP + h * 64 + 32, dpv + 32);
+    tmem_wait_ld();
+    uint32_t pk[32];
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+      const int col = h * 64 + 2 * i;
+      float x0, x1, d0, d1, g0, g1;
+      ffma2(x0, x1, __uint_as_float(sv[2 * i]), __uint_as_float(sv[2 * i + 1]), c, c, -l2, -l2);
+      float p0 = fast_exp2(x0), p1 = fast_exp2(x1);
+      if (kMasked) {
+        p0 = (col >= a && col < b) ? p0 : 0.f;
+        p1 = (col + 1 >= a && col + 1 < b) ? p1 : 0.f;
+      }
+      fadd2(d0, d1, __uint_as_float(dpv[2 * i]), __uint_as_float(dpv[2 * i + 1]), -dl, -dl);
+      fmul2(g0, g1, p0, p1, d0, d1);
+      pk[i] = pack_bf16(g0, g1);
+    }
+    tmem_st16p(tS + h * 32, pk);
+    tmem_st16p(tS + h * 32 + 16, pk + 16);
+  }
+}
+
+// dkdv kernel, one query tile for one key (thread = TMEM lane): P^T and
+// dS^T = P^T (dP^T - Delta) over the 128 rows, P = exp2(s * c - lse2[row]),
+// zero for rows whose slot bit (slot = row >> lg) is clear.  bf16 pairs
+// of rows go to TMEM columns [0, 64) of S^T and of dP^T.
+template <bool kMasked>
+__device__ __forceinline__ void pds_tile(uint32_t tSt, uint32_t tdPt, uint32_t smask, int lg,
+                                         const float4* ld4, float c) {
+#pragma unroll 1
+  for (int q = 0; q < 4; ++q) {        // 32 rows per TMEM round trip
+    uint32_t sv[32], dpv[32];
+    tmem_ld32(tSt + q * 32, sv);
+    tmem_ld32(tdPt + q * 32, dpv);
+    tmem_wait_ld();
+    uint32_t pp[16], pd[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const int row = q * 32 + 2 * i;
+      const float4 m = ld4[row >> 1];    // lse2[row], delta[row], lse2[row + 1], delta[row + 1]
+      float x0, x1, d0, d1, g0, g1;
+      ffma2(x0, x1, __uint_as_float(sv[2 * i]), __uint_as_float(sv[2 * i + 1]), c, c, -m.x, -m.z);
+      float p0 = fast_exp2(x0), p1 = fast_exp2(x1);
+      if (kMasked) {   // rows row and row + 1 share a slot (slots hold >= 8 rows)
+        const bool in = (smask >> (row >> lg)) & 1u;
+        p0 = in ? p0 : 0.f;
+        p1 = in ? p1 : 0.f;
+      }
+      fadd2(d0, d1, __uint_as_float(dpv[2 * i]), __uint_as_float(dpv[2 * i + 1]), -m.y, -m.w);
+      fmul2(g0, g1, p0, p1, d0, d1);
+      pp[i] = pack_bf16(p0, p1);
+      pd[i] = pack_bf16(g0, g1);
+    }
+    tmem_st16p(tSt + q * 16, pp);
+    tmem_st16p(tdPt + q * 16, pd);
+  }
+}
+
 // ============================================================================
 // dkdv kernel
 // ============================================================================
@@ -140,12 +205,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* sV = smem + kTile;
   uint8_t* sQ = smem + 2 * kTile;   // [2 stages]
   uint8_t* sdO = smem + 4 * kTile;  // [2 stages]
-  int2* meta_lohi = reinterpret_cast<int2*>(smem + 6 * kTile);                // [2][128]
-  float2* meta_ld = reinterpret_cast<float2*>(smem + 6 * kTile + 2048);       // [2][128] (lse2, delta)
+  float2* meta_ld = reinterpret_cast<float2*>(smem + 6 * kTile);             // [2][128] (lse2, delta) per row
+  int2* meta_slot = reinterpret_cast<int2*>(smem + 6 * kTile + 2048);         // [2][16] (lo, hi) per slot
   DkdvBars* B = reinterpret_cast<DkdvBars*>(smem + 6 * kTile + 4096);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int w = blockIdx.x;
   volatile int* abort_flag = &B->abort_flag;
+  const WaitCtx wctx{abort_flag, p.status};
   if (tid == 0) {
     p.timers[(p.W + w) * 2 + 0] = global_timer_ns();
     B->abort_flag = 0;
@@ -169,7 +235,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int4 item = p.bwd_items[it];
         const int g = item.y, c0 = item.x * p.C, c1 = min(c0 + p.C, p.N);
         for (int k0 = c0; ok && k0 < c1; k0 += BT) {
-          if (!mbar_wait(&B->kv_empty, (kt_count & 1) ^ 1, abort_flag)) { ok = false; break; }
+          if (!mbar_wait(&B->kv_empty, (kt_count & 1) ^ 1, wctx, 2 * 10000 + __LINE__)) { ok = false; break; }
           mbar_expect_tx(&B->kv_full, 2 * kTile);
           for (int dh = 0; dh < 2; ++dh) {
             tma_load_3d(sK + dh * kHalf, &tm_k, &B->kv_full, dh * 64, g, k0);
@@ -180,7 +246,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int4 tile = p.tiles[t];
             if (!(tile.z < k0 + BT && tile.w > k0)) continue;
             const int s = qd_count & 1;
-            if (!mbar_wait(&B->qd_empty[s], ((qd_count >> 1) & 1) ^ 1, abort_flag)) { ok = false; break; }
+            if (!mbar_wait(&B->qd_empty[s], ((qd_count >> 1) & 1) ^ 1, wctx, 2 * 10000 + __LINE__)) { ok = false; break; }
             mbar_expect_tx(&B->qd_full[s], 2 * kTile);
             load_query_tile(p, tile, g, sQ + s * kTile, &tm_q, &B->qd_full[s]);
             load_query_tile(p, tile, g, sdO + s * kTile, &tm_do, &B->qd_full[s]);
@@ -188,9 +254,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       }
-      if (!ok) abort_kernel(abort_flag, p);
-      if (kt_count > 0) mbar_drain(&B->kv_full, (kt_count - 1) & 1);
-      for (uint32_t c = qd_count >= 2 ? qd_count - 2 : 0; c < qd_count; ++c) mbar_drain(&B->qd_full[c & 1], (c >> 1) & 1);
+      if (!ok) *abort_flag = 1;
+      if (kt_count > 0) mbar_drain(&B->kv_full, (kt_count - 1) & 1, wctx, 2 * 10000 + __LINE__);
+      for (uint32_t c = qd_count >= 2 ? qd_count - 2 : 0; c < qd_count; ++c) mbar_drain(&B->qd_full[c & 1], (c >> 1) & 1, wctx, 2 * 10000 + __LINE__);
     }
   } else if (warp == 1) {
     if (lane == 0) {
@@ -201,14 +267,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int4 item = p.bwd_items[it];
         const int c0 = item.x * p.C, c1 = min(c0 + p.C, p.N);
         for (int k0 = c0; ok && k0 < c1; k0 += BT) {
-          if (!mbar_wait(&B->kv_full, kt_count & 1, abort_flag)) { ok = false; break; }
+          if (!mbar_wait(&B->kv_full, kt_count & 1, wctx, 2 * 10000 + __LINE__)) { ok = false; break; }
           tc_fence_after();
           int u = 0;
           for (int t = item.z; t < item.w; ++t) {
             const int4 tile = p.tiles[t];
             if (!(tile.z < k0 + BT && tile.w > k0)) continue;
             const int s = qd_count & 1;
-            if (!mbar_wait(&B->qd_full[s], (qd_count >> 1) & 1, abort_flag)) { ok = false; break; }
+            if (!mbar_wait(&B->qd_full[s], (qd_count >> 1) & 1, wctx, 2 * 10000 + __LINE__)) { ok = false; break; }
             tc_fence_after();
             // S^T = K Q^T (cols 0..127), dP^T = V dO^T (cols 128..255)
             for (int kk = 0; kk < D / 16; ++kk)
@@ -216,10 +282,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int kk = 0; kk < D / 16; ++kk)
               mma_ss(tmem + 128, kmajor(aV, kk), kmajor(adO + s * kTile, kk), kIdescKM, kk > 0 ? 1u : 0u);
             mma_commit(&B->st_ready);
-            if (!mbar_wait(&B->pds_ready, pds_cnt & 1, abort_flag)) { ok = false; break; }
+            if (!mbar_wait(&B->pds_ready, pds_cnt & 1, wctx, 2 * 10000 + __LINE__)) { ok = false; break; }
             ++pds_cnt;
             if (u == 0) {
-              if (!mbar_wait(&B->dkv_free, (dkvf_cnt & 1) ^ 1, abort_flag)) { ok = false; break; }
+              if (!mbar_wait(&B->dkv_free, (dkvf_cnt & 1) ^ 1, wctx, 2 * 10000 + __LINE__)) { ok = false; break; }
               ++dkvf_cnt;
             }
             tc_fence_after();
@@ -240,9 +306,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           ++kt_count;
         }
       }
-      if (!ok) abort_kernel(abort_flag, p);
+      if (!ok) *abort_flag = 1;
       mma_commit(&B->mma_done);
-      mbar_drain(&B->mma_done, 0);
+      mbar_drain(&B->mma_done, 0, wctx, 2 * 10000 + __LINE__);
     }
   } else if (warp >= 4) {
     const int r = ((warp & 3) << 5) + lane;   // key of the tile = TMEM lane; also the row this thread describes
@@ -274,8 +340,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int4 tile = p.tiles[t];
           if (!(tile.z < k0 + BT && tile.w > k0)) continue;
           const int s = qd_count & 1;
+          const int rps = p.G * p.bs;
           {
-            // this thread describes row r of the query tile
+            // this thread describes row r of the query tile (and slot r / rps's interval)
             const RowMeta m = row_meta(p, tile, g, r);
             float l2 = INFINITY, dl = 0.f;
             if (m.valid) {
@@ -283,40 +350,32 @@ __global__ void __launch_bounds__(kThreads, 1)
               l2 = (L == -INFINITY) ? INFINITY : L * kLog2e;
               dl = delta[m.qrow];
             }
-            meta_lohi[s * 128 + r] = make_int2(m.lo, m.hi);
             meta_ld[s * 128 + r] = make_float2(l2, dl);
+            if (r % rps == 0) meta_slot[s * 16 + r / rps] = make_int2(m.lo, m.hi);
           }
           // every thread needs all 128 rows' metadata: bounded handoff through an mbarrier
           mbar_arrive(&B->meta_ready[s]);
-          if (!warp_wait(&B->meta_ready[s], (qd_count >> 1) & 1, abort_flag)) { ok = false; break; }
-          if (!warp_wait(&B->st_ready, st_cnt & 1, abort_flag)) { ok = false; break; }
+          if (!warp_wait(&B->meta_ready[s], (qd_count >> 1) & 1, wctx, 2 * 10000 + __LINE__)) { ok = false; break; }
+          // slots (blocks) that may read this thread's key: one bit per slot.  Padding
+          // slots count as "in": their rows have lse2 = +inf, so P = 0 there anyway.
+          const int nslots = BT / rps;             // rps is a power of two (8 .. 128)
+          const int lg = 31 - __clz(rps);
+          uint32_t smask = ~((1u << (tile.y - tile.x)) - 1u);
+          for (int sl = 0; sl < tile.y - tile.x; ++sl) {
+            const int2 lh = meta_slot[s * 16 + sl];
+            if (key >= lh.x && key < lh.y) smask |= 1u << sl;
+          }
+          const uint32_t all = nslots >= 32 ? 0xffffffffu : ((1u << nslots) - 1u);
+          // warp-uniform choice: both paths issue warp-collective tcgen05.ld/st
+          const bool all_in = __all_sync(0xffffffffu, (smask & all) == all);
+          if (!warp_wait(&B->st_ready, st_cnt & 1, wctx, 2 * 10000 + __LINE__)) { ok = false; break; }
           ++st_cnt;
           tc_fence_after();
-#pragma unroll 1
-          for (int cc = 0; cc < 4; ++cc) {
-            uint32_t sv[32], dpv[32];
-            tmem_ld32(tSt + cc * 32, sv);
-            tmem_ld32(tdPt + cc * 32, dpv);
-            tmem_wait_ld();
-            uint32_t pk[16], dk16[16];
-#pragma unroll
-            for (int i = 0; i < 16; ++i) {
-              float pr[2], ds[2];
-#pragma unroll
-              for (int e = 0; e < 2; ++e) {
-                const int row = cc * 32 + 2 * i + e;
-                const int2 lh = meta_lohi[s * 128 + row];
-                const float2 ld = meta_ld[s * 128 + row];
-                const bool in = key >= lh.x && key < lh.y;
-                pr[e] = in ? fast_exp2(__uint_as_float(sv[2 * i + e]) * scale_log2 - ld.x) : 0.f;
-                ds[e] = pr[e] * (__uint_as_float(dpv[2 * i + e]) - ld.y);
-              }
-              pk[i] = pack_bf16(pr[0], pr[1]);
-              dk16[i] = pack_bf16(ds[0], ds[1]);
-            }
-            tmem_st16(tSt + cc * 16, pk);
-            tmem_st16(tdPt + cc * 16, dk16);
-          }
+          const float4* ld4 = reinterpret_cast<const float4*>(meta_ld + s * 128);
+          if (all_in)
+            pds_tile<false>(tSt, tdPt, smask, lg, ld4, scale_log2);
+          else
+            pds_tile<true>(tSt, tdPt, smask, lg, ld4, scale_log2);
           tmem_wait_st();
           tc_fence_before();
           mbar_arrive(&B->pds_ready);
@@ -329,7 +388,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         float* dvr = dv + (size_t(key) * p.Hkv + g) * D;
         const bool own = key < c1;
         if (n_meet > 0) {
-          if (!warp_wait(&B->dkv_ready, dkv_cnt & 1, abort_flag)) { ok = false; break; }
+          if (!warp_wait(&B->dkv_ready, dkv_cnt & 1, wctx, 2 * 10000 + __LINE__)) { ok = false; break; }
           ++dkv_cnt;
           tc_fence_after();
 #pragma unroll 1
@@ -360,7 +419,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
     }
-    if (!ok) abort_kernel(abort_flag, p);
+    if (!ok) *abort_flag = 1;
   }
   tc_fence_before();
   __syncthreads();
@@ -420,6 +479,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int w = blockIdx.x;
   volatile int* abort_flag = &B->abort_flag;
+  const WaitCtx wctx{abort_flag, p.status};
   if (tid == 0) B->abort_flag = 0;
   {
     const uint32_t counts[kDqNumBars] = {1, 1, 1, 1, 1, 1, 1, 1, 1, 1, 1, 128, 1, 128, 1};
@@ -440,7 +500,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok = true;
       while (ok && ti.next(t, g)) {
         const int4 tile = p.tiles[t];
-        if (!mbar_wait(&B->qd_empty, (tile_count & 1) ^ 1, abort_flag)) { ok = false; break; }
+        if (!mbar_wait(&B->qd_empty, (tile_count & 1) ^ 1, wctx, 2 * 10000 + __LINE__)) { ok = false; break; }
         mbar_expect_tx(&B->qd_full, 2 * kTile);
         load_query_tile(p, tile, g, sQ, &tm_q, &B->qd_full);
         load_query_tile(p, tile, g, sdO, &tm_do, &B->qd_full);
@@ -448,7 +508,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int n_kt = (tile.w - tile.z + BT - 1) / BT;
         for (int j = 0; j < n_kt; ++j, ++kv_count) {
           const int s = kv_count & 1;
-          if (!mbar_wait(&B->kv_empty[s], ((kv_count >> 1) & 1) ^ 1, abort_flag)) { ok = false; break; }
+          if (!mbar_wait(&B->kv_empty[s], ((kv_count >> 1) & 1) ^ 1, wctx, 2 * 10000 + __LINE__)) { ok = false; break; }
           const int k0 = tile.z + j * BT;
           mbar_expect_tx(&B->k_full[s], kTile);
           for (int dh = 0; dh < 2; ++dh) tma_load_3d(sK + s * kTile + dh * kHalf, &tm_k, &B->k_full[s], dh * 64, g, k0);
@@ -457,11 +517,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         ++tile_count;
       }
-      if (!ok) abort_kernel(abort_flag, p);
-      if (q_issued > 0) mbar_drain(&B->qd_full, (q_issued - 1) & 1);
+      if (!ok) *abort_flag = 1;
+      if (q_issued > 0) mbar_drain(&B->qd_full, (q_issued - 1) & 1, wctx, 2 * 10000 + __LINE__);
       for (uint32_t c = kv_count >= 2 ? kv_count - 2 : 0; c < kv_count; ++c) {
-        mbar_drain(&B->k_full[c & 1], (c >> 1) & 1);
-        mbar_drain(&B->v_full[c & 1], (c >> 1) & 1);
+        mbar_drain(&B->k_full[c & 1], (c >> 1) & 1, wctx, 2 * 10000 + __LINE__);
+        mbar_drain(&B->v_full[c & 1], (c >> 1) & 1, wctx, 2 * 10000 + __LINE__);
       }
     }
   } else if (warp == 1) {
@@ -475,16 +535,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       while (ok && ti.next(t, g)) {
         const int4 tile = p.tiles[t];
         const int n_kt = (tile.w - tile.z + BT - 1) / BT;
-        if (!mbar_wait(&B->qd_full, tile_count & 1, abort_flag)) { ok = false; break; }
+        if (!mbar_wait(&B->qd_full, tile_count & 1, wctx, 2 * 10000 + __LINE__)) { ok = false; break; }
         const uint32_t c0 = kv_count;
         {
           const int s = c0 & 1;
-          if (!mbar_wait(&B->k_full[s], (c0 >> 1) & 1, abort_flag)) { ok = false; break; }
+          if (!mbar_wait(&B->k_full[s], (c0 >> 1) & 1, wctx, 2 * 10000 + __LINE__)) { ok = false; break; }
           tc_fence_after();
           for (int kk = 0; kk < D / 16; ++kk)
             mma_ss(tmem + s * 128, kmajor(aQ, kk), kmajor(aK + s * kTile, kk), kIdescKM, kk > 0 ? 1u : 0u);
           mma_commit(&B->s_ready[s]);
-          if (!mbar_wait(&B->v_full[s], (c0 >> 1) & 1, abort_flag)) { ok = false; break; }
+          if (!mbar_wait(&B->v_full[s], (c0 >> 1) & 1, wctx, 2 * 10000 + __LINE__)) { ok = false; break; }
           tc_fence_after();
           for (int kk = 0; kk < D / 16; ++kk)
             mma_ss(tmem + 256, kmajor(adO, kk), kmajor(aV + s * kTile, kk), kIdescKM, kk > 0 ? 1u : 0u);
@@ -495,16 +555,16 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int s = c & 1, s1 = (c + 1) & 1;
           const bool more = j + 1 < n_kt;
           if (more) {   // next S into the other buffer while this tile's dS is formed
-            if (!mbar_wait(&B->k_full[s1], ((c + 1) >> 1) & 1, abort_flag)) { ok = false; break; }
+            if (!mbar_wait(&B->k_full[s1], ((c + 1) >> 1) & 1, wctx, 2 * 10000 + __LINE__)) { ok = false; break; }
             tc_fence_after();
             for (int kk = 0; kk < D / 16; ++kk)
               mma_ss(tmem + s1 * 128, kmajor(aQ, kk), kmajor(aK + s1 * kTile, kk), kIdescKM, kk > 0 ? 1u : 0u);
             mma_commit(&B->s_ready[s1]);
           }
-          if (!mbar_wait(&B->ds_ready, ds_cnt & 1, abort_flag)) { ok = false; break; }
+          if (!mbar_wait(&B->ds_ready, ds_cnt & 1, wctx, 2 * 10000 + __LINE__)) { ok = false; break; }
           ++ds_cnt;
           if (j == 0) {
-            if (!mbar_wait(&B->dq_free, (dqf_cnt & 1) ^ 1, abort_flag)) { ok = false; break; }
+            if (!mbar_wait(&B->dq_free, (dqf_cnt & 1) ^ 1, wctx, 2 * 10000 + __LINE__)) { ok = false; break; }
             ++dqf_cnt;
           }
           tc_fence_after();
@@ -514,7 +574,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                    (j > 0 || kk > 0) ? 1u : 0u);
           mma_commit(&B->kv_empty[s]);
           if (more) {
-            if (!mbar_wait(&B->v_full[s1], ((c + 1) >> 1) & 1, abort_flag)) { ok = false; break; }
+            if (!mbar_wait(&B->v_full[s1], ((c + 1) >> 1) & 1, wctx, 2 * 10000 + __LINE__)) { ok = false; break; }
             tc_fence_after();
             for (int kk = 0; kk < D / 16; ++kk)
               mma_ss(tmem + 256, kmajor(adO, kk), kmajor(aV + s1 * kTile, kk), kIdescKM, kk > 0 ? 1u : 0u);
@@ -527,9 +587,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         kv_count += n_kt;
         ++tile_count;
       }
-      if (!ok) abort_kernel(abort_flag, p);
+      if (!ok) *abort_flag = 1;
       mma_commit(&B->mma_done);
-      mbar_drain(&B->mma_done, 0);
+      mbar_drain(&B->mma_done, 0, wctx, 2 * 10000 + __LINE__);
     }
   } else if (warp >= 4) {
     const int r = ((warp & 3) << 5) + lane;
@@ -555,40 +615,25 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int j = 0; j < n_kt; ++j) {
         const uint32_t c = kv_count + j;
         const int s = c & 1;
-        if (!warp_wait(&B->s_ready[s], (c >> 1) & 1, abort_flag)) { ok = false; break; }
-        if (!warp_wait(&B->dp_ready, dp_cnt & 1, abort_flag)) { ok = false; break; }
+        if (!warp_wait(&B->s_ready[s], (c >> 1) & 1, wctx, 2 * 10000 + __LINE__)) { ok = false; break; }
+        if (!warp_wait(&B->dp_ready, dp_cnt & 1, wctx, 2 * 10000 + __LINE__)) { ok = false; break; }
         ++dp_cnt;
         tc_fence_after();
         const uint32_t tS = tmem + lane_addr + s * 128;
         const int k0 = tile.z + j * BT;
-#pragma unroll 1
-        for (int cc = 0; cc < 4; ++cc) {
-          uint32_t sv[32], dpv[32];
-          tmem_ld32(tS + cc * 32, sv);
-          tmem_ld32(tdP + cc * 32, dpv);
-          tmem_wait_ld();
-          uint32_t pk[16];
-#pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            float ds[2];
-#pragma unroll
-            for (int e = 0; e < 2; ++e) {
-              const int key = k0 + cc * 32 + 2 * i + e;
-              const bool in = key >= m.lo && key < m.hi;
-              const float pr = in ? fast_exp2(__uint_as_float(sv[2 * i + e]) * scale_log2 - l2) : 0.f;
-              ds[e] = pr * (__uint_as_float(dpv[2 * i + e]) - dl);
-            }
-            pk[i] = pack_bf16(ds[0], ds[1]);
-          }
-          tmem_st16(tS + cc * 16, pk);
-        }
+        const int a = m.lo - k0, b = m.hi - k0;   // the row's allowed columns of this key tile
+        // warp-uniform choice: both paths issue warp-collective tcgen05.ld/st
+        if (__all_sync(0xffffffffu, a <= 0 && b >= BT))
+          ds_tile<false>(tS, tdP, a, b, scale_log2, l2, dl);
+        else
+          ds_tile<true>(tS, tdP, a, b, scale_log2, l2, dl);
         tmem_wait_st();
         tc_fence_before();
         mbar_arrive(&B->ds_ready);
       }
       if (!ok) break;
       kv_count += n_kt;
-      if (!warp_wait(&B->dq_ready, dq_cnt & 1, abort_flag)) { ok = false; break; }
+      if (!warp_wait(&B->dq_ready, dq_cnt & 1, wctx, 2 * 10000 + __LINE__)) { ok = false; break; }
       ++dq_cnt;
       tc_fence_after();
       float* dst = dq_part + size_t(m.rec) * D;
@@ -608,7 +653,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_before();
       mbar_arrive(&B->dq_free);
     }
-    if (!ok) abort_kernel(abort_flag, p);
+    if (!ok) *abort_flag = 1;
   }
   tc_fence_before();
   __syncthreads();

@@ -102,9 +102,53 @@ struct PairIter {
   }
 };
 
-__device__ __forceinline__ void record_abort(Bars* bars, const DevPlan& p) {
-  bars->abort_flag = 1;
-  atomicExch(p.status, SPLITKV_ERR_TIMEOUT);
+
+// Maximum of 64 raw scores of one row over its allowed columns [a, b) of them.
+template <bool kMasked>
+__device__ __forceinline__ float row_max(const uint32_t (&v)[64], int a, int b) {
+  float m0 = -INFINITY, m1 = -INFINITY, m2 = -INFINITY, m3 = -INFINITY;
+#pragma unroll
+  for (int i = 0; i < 64; i += 4) {
+    if (kMasked) {
+      m0 = (i >= a && i < b) ? fmaxf(m0, __uint_as_float(v[i])) : m0;
+      m1 = (i + 1 >= a && i + 1 < b) ? fmaxf(m1, __uint_as_float(v[i + 1])) : m1;
+      m2 = (i + 2 >= a && i + 2 < b) ? fmaxf(m2, __uint_as_float(v[i + 2])) : m2;
+      m3 = (i + 3 >= a && i + 3 < b) ? fmaxf(m3, __uint_as_float(v[i + 3])) : m3;
+    } else {
+      m0 = fmaxf(m0, __uint_as_float(v[i]));
+      m1 = fmaxf(m1, __uint_as_float(v[i + 1]));
+      m2 = fmaxf(m2, __uint_as_float(v[i + 2]));
+      m3 = fmaxf(m3, __uint_as_float(v[i + 3]));
+    }
+  }
+  return fmaxf(fmaxf(m0, m1), fmaxf(m2, m3));
+}
+
+// P = exp2(v * c + nm) over 64 columns of a row (0 outside [a, b)), packed to
+// bf16 pairs into 32 TMEM columns at tS; returns the row sum of the fp32 P.
+template <bool kMasked>
+__device__ __forceinline__ float exp_pack_store(const uint32_t (&v)[64], int a, int b, float c, float nm,
+                                                uint32_t tS) {
+  float s0 = 0.f, s1 = 0.f;
+#pragma unroll
+  for (int cch = 0; cch < 2; ++cch) {
+    uint32_t pk[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const int col = cch * 32 + 2 * i;
+      float x0, x1;
+      ffma2(x0, x1, __uint_as_float(v[col]), __uint_as_float(v[col + 1]), c, c, nm, nm);
+      float p0 = fast_exp2(x0), p1 = fast_exp2(x1);
+      if (kMasked) {
+        p0 = (col >= a && col < b) ? p0 : 0.f;
+        p1 = (col + 1 >= a && col + 1 < b) ? p1 : 0.f;
+      }
+      fadd2(s0, s1, s0, s1, p0, p1);
+      pk[i] = pack_bf16(p0, p1);
+    }
+    tmem_st16p(tS + cch * 16, pk);
+  }
+  return s0 + s1;
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -118,6 +162,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int w = blockIdx.x;
   volatile int* abort_flag = &bars->abort_flag;
+  const WaitCtx wctx{abort_flag, p.status};
 
   if (tid == 0) {
     p.timers[w * 2 + 0] = global_timer_ns();
@@ -153,7 +198,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem = bars->tmem_base;
   const int rows_per_slot = p.G * p.bs;
   const uint32_t slot_bytes = uint32_t(rows_per_slot) * 128;   // one slot's rows of one 64-column half
-
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
@@ -163,7 +207,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t kv_count = 0, pair_count = 0, q_issued = 0;
       bool ok = true;
       while (ok && pi.next(tA, tB, g, klo, khi)) {
-        if (!mbar_wait(&bars->q_empty, (pair_count & 1) ^ 1, abort_flag)) { ok = false; break; }
+        if (!mbar_wait(&bars->q_empty, (pair_count & 1) ^ 1, wctx, 1 * 10000 + __LINE__)) { ok = false; break; }
         const int4 ta = p.tiles[tA];
         const int nA = ta.y - ta.x;
         int nB = 0;
@@ -190,7 +234,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int n_kt = (khi - klo + BN - 1) / BN;
         for (int j = 0; j < n_kt; ++j, ++kv_count) {
           const int s = kv_count % kStages;
-          if (!mbar_wait(&bars->kv_empty[s], ((kv_count / kStages) & 1) ^ 1, abort_flag)) { ok = false; break; }
+          if (!mbar_wait(&bars->kv_empty[s], ((kv_count / kStages) & 1) ^ 1, wctx, 1 * 10000 + __LINE__)) { ok = false; break; }
           const int k0 = klo + j * BN;
           mbar_expect_tx(&bars->k_full[s], kTile);
           for (int dh = 0; dh < 2; ++dh)
@@ -201,13 +245,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         ++pair_count;
       }
-      if (!ok) record_abort(bars, p);
+      if (!ok) *abort_flag = 1;
       // copies still in flight land before the CTA may exit: wait for the last
       // fill of every buffer (bounded; completed phases return at once)
-      if (q_issued > 0) mbar_drain(&bars->q_full, (q_issued - 1) & 1);
+      if (q_issued > 0) mbar_drain(&bars->q_full, (q_issued - 1) & 1, wctx, 1 * 10000 + __LINE__);
       for (uint32_t c = kv_count >= kStages ? kv_count - kStages : 0; c < kv_count; ++c) {
-        mbar_drain(&bars->k_full[c % kStages], (c / kStages) & 1);
-        mbar_drain(&bars->v_full[c % kStages], (c / kStages) & 1);
+        mbar_drain(&bars->k_full[c % kStages], (c / kStages) & 1, wctx, 1 * 10000 + __LINE__);
+        mbar_drain(&bars->v_full[c % kStages], (c / kStages) & 1, wctx, 1 * 10000 + __LINE__);
       }
     }
   } else if (warp == 1) {
@@ -225,10 +269,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       while (ok && pi.next(tA, tB, g, klo, khi)) {
         const int nx = tB >= 0 ? 2 : 1;
         const int n_kt = (khi - klo + BN - 1) / BN;
-        if (!mbar_wait(&bars->q_full, pair_count & 1, abort_flag)) { ok = false; break; }
+        if (!mbar_wait(&bars->q_full, pair_count & 1, wctx, 1 * 10000 + __LINE__)) { ok = false; break; }
         {
           const int s0 = kv_count % kStages;
-          if (!mbar_wait(&bars->k_full[s0], (kv_count / kStages) & 1, abort_flag)) { ok = false; break; }
+          if (!mbar_wait(&bars->k_full[s0], (kv_count / kStages) & 1, wctx, 1 * 10000 + __LINE__)) { ok = false; break; }
           tc_fence_after();
           for (int x = 0; x < nx; ++x) {
             for (int kk = 0; kk < D / 16; ++kk) {
@@ -245,14 +289,14 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int s1 = (c + 1) % kStages;
           const bool more = j + 1 < n_kt;
           for (int x = 0; x < nx; ++x) {
-            if (!mbar_wait(&bars->p_ready[x], p_cnt[x] & 1, abort_flag)) { ok = false; break; }
+            if (!mbar_wait(&bars->p_ready[x], p_cnt[x] & 1, wctx, 1 * 10000 + __LINE__)) { ok = false; break; }
             ++p_cnt[x];
             if (j == 0) {
-              if (!mbar_wait(&bars->o_free[x], (of_cnt[x] & 1) ^ 1, abort_flag)) { ok = false; break; }
+              if (!mbar_wait(&bars->o_free[x], (of_cnt[x] & 1) ^ 1, wctx, 1 * 10000 + __LINE__)) { ok = false; break; }
               ++of_cnt[x];
             }
             if (x == 0) {
-              if (!mbar_wait(&bars->v_full[s], (c / kStages) & 1, abort_flag)) { ok = false; break; }
+              if (!mbar_wait(&bars->v_full[s], (c / kStages) & 1, wctx, 1 * 10000 + __LINE__)) { ok = false; break; }
             }
             tc_fence_after();
             // O_X (+)= P_X V : P in TMEM (columns 0..63 of S_X), V MN-major in smem
@@ -263,7 +307,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             mma_commit(&bars->o_ready[x]);
             if (more) {
               if (x == 0) {
-                if (!mbar_wait(&bars->k_full[s1], ((c + 1) / kStages) & 1, abort_flag)) { ok = false; break; }
+                if (!mbar_wait(&bars->k_full[s1], ((c + 1) / kStages) & 1, wctx, 1 * 10000 + __LINE__)) { ok = false; break; }
                 tc_fence_after();
               }
               for (int kk = 0; kk < D / 16; ++kk) {
@@ -283,10 +327,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         kv_count += n_kt;
         ++pair_count;
       }
-      if (!ok) record_abort(bars, p);
+      if (!ok) *abort_flag = 1;
       // every MMA must finish before tensor memory is released
       mma_commit(&bars->mma_done);
-      mbar_drain(&bars->mma_done, 0);
+      mbar_drain(&bars->mma_done, 0, wctx, 1 * 10000 + __LINE__);
     }
   } else if (warp >= 4) {
     // ------------------------------------------------------------ softmax + epilogue
@@ -319,65 +363,62 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       float m_ref = -INFINITY, m_true = -INFINITY, l = 0.f;
       for (int j = 0; j < n_kt; ++j) {
-        if (!warp_wait(&bars->s_ready[x], s_cnt & 1, abort_flag)) { ok = false; break; }
+        if (!warp_wait(&bars->s_ready[x], s_cnt & 1, wctx, 1 * 10000 + __LINE__)) { ok = false; break; }
         ++s_cnt;
         tc_fence_after();
         const int k0 = klo + j * BN;
-        // pass 1: masked row maximum
-        float mx = -INFINITY;
+        // the row's allowed columns in this key tile: [a, b)
+        const int a = lo - k0, b = hi - k0;
+        const bool none = b <= 0 || a >= BN;
+        // warp-uniform: the two exp_pack_store variants issue warp-collective tcgen05.st
+        const bool full = __all_sync(0xffffffffu, a <= 0 && b >= BN);
+        // pass 1: maximum of the raw scores, 64 columns per TMEM round trip
+        float mxr = -INFINITY;
+        if (__any_sync(0xffffffffu, !none)) {
 #pragma unroll 1
-        for (int cch = 0; cch < 4; ++cch) {
-          uint32_t v[32];
-          tmem_ld32(tS + cch * 32, v);
-          tmem_wait_ld();
-#pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            const int key = k0 + cch * 32 + i;
-            const float sv = __uint_as_float(v[i]) * scale_log2;
-            mx = (key >= lo && key < hi) ? fmaxf(mx, sv) : mx;
+          for (int h = 0; h < BN / 64; ++h) {
+            uint32_t v[64];
+            tmem_ld32p(tS + h * 64, v);
+            tmem_ld32p(tS + h * 64 + 32, v + 32);
+            tmem_wait_ld();
+            const float mh = full ? row_max<false>(v, a - h * 64, b - h * 64) : row_max<true>(v, a - h * 64, b - h * 64);
+            mxr = fmaxf(mxr, mh);
           }
         }
+        const float mx = none ? -INFINITY : mxr * scale_log2;
         m_true = fmaxf(m_true, mx);
         // rescale decision (warp-uniform for the TMEM traffic)
         const bool need = (mx > m_ref + kRescaleLog2) || (m_ref == -INFINITY && mx > -INFINITY);
         const bool rescale_o = need && m_ref > -INFINITY;      // only after a previous tile added to O
         if (__any_sync(0xffffffffu, rescale_o)) {
           // PV(j-1) must have completed before O is touched
-          if (!warp_wait(&bars->o_ready[x], (o_cnt + j - 1) & 1, abort_flag)) { ok = false; break; }
+          if (!warp_wait(&bars->o_ready[x], (o_cnt + j - 1) & 1, wctx, 1 * 10000 + __LINE__)) { ok = false; break; }
           tc_fence_after();
           const float f = rescale_o ? fast_exp2(m_ref - mx) : 1.f;
 #pragma unroll 1
-          for (int cch = 0; cch < D / 32; ++cch) {
-            uint32_t v[32];
-            tmem_ld32(tO + cch * 32, v);
+          for (int cch = 0; cch < D / 16; ++cch) {
+            uint32_t o[16];
+            tmem_ld16(tO + cch * 16, o);
             tmem_wait_ld();
 #pragma unroll
-            for (int i = 0; i < 32; ++i) v[i] = __float_as_uint(__uint_as_float(v[i]) * f);
-            tmem_st32(tO + cch * 32, v);
+            for (int i = 0; i < 16; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * f);
+            tmem_st16(tO + cch * 16, o);
           }
           tmem_wait_st();
           l *= f;
         }
         if (need) m_ref = mx;
         const float m_use = (m_ref == -INFINITY) ? 0.f : m_ref;
-        // pass 2: P = exp2(s - m_ref) (masked -> 0), row sum, bf16 P into TMEM columns 0..63 of S_X
+        // pass 2: P = exp2(s * scale_log2 - m_ref) (masked -> 0), row sum, bf16 P into
+        // TMEM columns 0..63 of S_X (half h -> columns 32h..32h+31, already read)
 #pragma unroll 1
-        for (int cch = 0; cch < 4; ++cch) {
-          uint32_t v[32];
-          tmem_ld32(tS + cch * 32, v);
+        for (int h = 0; h < BN / 64; ++h) {
+          uint32_t v[64];
+          tmem_ld32p(tS + h * 64, v);
+          tmem_ld32p(tS + h * 64 + 32, v + 32);
           tmem_wait_ld();
-          uint32_t pk[16];
-#pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            const int key = k0 + cch * 32 + 2 * i;
-            const float s0 = __uint_as_float(v[2 * i]) * scale_log2 - m_use;
-            const float s1 = __uint_as_float(v[2 * i + 1]) * scale_log2 - m_use;
-            const float p0 = (key >= lo && key < hi) ? fast_exp2(s0) : 0.f;
-            const float p1 = (key + 1 >= lo && key + 1 < hi) ? fast_exp2(s1) : 0.f;
-            l += p0 + p1;
-            pk[i] = pack_bf16(p0, p1);
-          }
-          tmem_st16(tS + cch * 16, pk);
+          l += full ? exp_pack_store<false>(v, a - h * 64, b - h * 64, scale_log2, -m_use, tS + h * 32)
+                    : exp_pack_store<true>(v, a - h * 64, b - h * 64, scale_log2, -m_use, tS + h * 32);
         }
         tmem_wait_st();
         tc_fence_before();
@@ -385,7 +426,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (!ok) break;
       // epilogue: wait for the last PV of this tile, then write the record
-      if (!warp_wait(&bars->o_ready[x], (o_cnt + n_kt - 1) & 1, abort_flag)) { ok = false; break; }
+      if (!warp_wait(&bars->o_ready[x], (o_cnt + n_kt - 1) & 1, wctx, 1 * 10000 + __LINE__)) { ok = false; break; }
       o_cnt += n_kt;
       tc_fence_after();
       const float inv = l > 0.f ? 1.f / l : 0.f;
@@ -412,7 +453,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_before();
       mbar_arrive(&bars->o_free[x]);
     }
-    if (!ok) record_abort(bars, p);
+    if (!ok) *abort_flag = 1;
   }
 
   tc_fence_before();

@@ -273,10 +273,11 @@ int splitkv_attn_fwd_static_scratch(const splitkv_plan_t* plan, const void* q, c
 
 /* Device status of the plan's kernels: synchronises `stream`, returns
  * SPLITKV_OK, or the SPLITKV_ERR_* code a kernel recorded since the last call
- * (SPLITKV_ERR_TIMEOUT: a bounded wait inside a kernel gave up and the kernel
- * wound down; its outputs are invalid), and clears the word.
- * Errors: INVALID_ARG, NOT_UPLOADED, CUDA. */
-int splitkv_plan_status(const splitkv_plan_t* plan, void* stream);
+ * (SPLITKV_ERR_TIMEOUT: a wait inside a kernel passed its 2-second limit and
+ * the kernel wound down; its outputs are invalid), and clears the words.
+ * If `site` is not NULL it receives the source site of the first wait that
+ * timed out (0 if none).  Errors: INVALID_ARG, NOT_UPLOADED, CUDA. */
+int splitkv_plan_status(const splitkv_plan_t* plan, void* stream, int32_t* site);
 
 /* Per-CTA busy time of the last splitkv_attn_fwd (which = SPLITKV_WS_FWD) or
  * backward partial kernel (SPLITKV_WS_BWD) on this plan: out_ns[w] = end - start
