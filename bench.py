@@ -497,7 +497,8 @@ def main(argv=None):
     ap.add_argument("--anchors", type=int, default=None)
     ap.add_argument("--workers", type=int, default=0, help="forward CTAs (default: SM count)")
     ap.add_argument("--bwd-workers", type=int, default=0, help="backward CTAs (default: SM count)")
-    ap.add_argument("--q-slice", type=int, default=0)
+    ap.add_argument("--q-slice", type=int, default=2,
+                    help="forward items of at most this many 128-row query tiles (0 = whole chunks)")
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-e2e", action="store_true")

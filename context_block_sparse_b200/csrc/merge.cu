@@ -25,6 +25,12 @@ namespace {
 
 constexpr int kMergeThreads = 256;
 
+__device__ __forceinline__ float warp_max(float x) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, o));
+  return x;
+}
+
 __device__ __forceinline__ float warp_sum(float x) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
@@ -113,30 +119,55 @@ __global__ void __launch_bounds__(kMergeThreads)
       for (int i = 0; i < DPL; ++i) ob[i] = ob[i] * corr + pr * vv[i];
       mb = mn;
     }
-    // pass 1: global max and normaliser over the in-block record and the chunk records
-    float M = mb;
-    for (int x = e0; x < e1; ++x) {
-      const int e = p.block_entries[x];
-      const size_t rec = size_t(e * p.bs + tt) * p.Hq + head;
-      if (part_l[rec] > 0.f) M = fmaxf(M, part_m[rec] * kLog2e);
+    // the chunk records of this row: one entry per lane, 32 at a time
+    const int n = e1 - e0;
+    float Mc = -INFINITY;
+    for (int base = 0; base < n; base += 32) {
+      float m2 = -INFINITY;
+      if (base + lane < n) {
+        const int rec = (p.block_entries[e0 + base + lane] * p.bs + tt) * p.Hq + head;
+        if (part_l[rec] > 0.f) m2 = part_m[rec] * kLog2e;
+      }
+      Mc = fmaxf(Mc, warp_max(m2));
     }
-    float L = lb * fast_exp2(mb - M);
-    float acc[DPL];
+    const float M = fmaxf(mb, Mc);
     const float wb = fast_exp2(mb - M);   // ob is unnormalised: weight exp2(mb - M)
+    float L = lb * wb;
+    float acc[DPL];
 #pragma unroll
     for (int i = 0; i < DPL; ++i) acc[i] = ob[i] * wb;
-    // pass 2: weighted sum of the normalised chunk outputs, ascending chunk
-#pragma unroll 4
-    for (int x = e0; x < e1; ++x) {
-      const int e = p.block_entries[x];
-      const size_t rec = size_t(e * p.bs + tt) * p.Hq + head;
-      const float lx = part_l[rec];
-      const float wx = lx > 0.f ? lx * fast_exp2(part_m[rec] * kLog2e - M) : 0.f;
-      float ov[DPL];
-      load_f32_row<DPL>(part_o + rec * D + lane * DPL, ov);
-      L += wx;
+    // weighted sum of the normalised chunk outputs in ascending chunk order, 8 rows in flight
+    for (int base = 0; base < n; base += 32) {
+      float wl = 0.f;
+      int recl = 0;
+      if (base + lane < n) {
+        recl = (p.block_entries[e0 + base + lane] * p.bs + tt) * p.Hq + head;
+        const float lx = part_l[recl];
+        wl = lx > 0.f ? lx * fast_exp2(part_m[recl] * kLog2e - M) : 0.f;
+      }
+      L += warp_sum(wl);
+      const int cnt = min(32, n - base);
+      for (int j0 = 0; j0 < cnt; j0 += 8) {
+        float w8[8];
+        float ov[8][DPL];
 #pragma unroll
-      for (int i = 0; i < DPL; ++i) acc[i] = fmaf(wx, ov[i], acc[i]);
+        for (int u = 0; u < 8; ++u) {
+          const int j = j0 + u;
+          const float wj = __shfl_sync(0xffffffffu, wl, j & 31);
+          const int rj = __shfl_sync(0xffffffffu, recl, j & 31);
+          w8[u] = j < cnt ? wj : 0.f;
+          if (j < cnt) {
+            load_f32_row<DPL>(part_o + size_t(rj) * D + lane * DPL, ov[u]);
+          } else {
+#pragma unroll
+            for (int i = 0; i < DPL; ++i) ov[u][i] = 0.f;
+          }
+        }
+#pragma unroll
+        for (int u = 0; u < 8; ++u)
+#pragma unroll
+          for (int i = 0; i < DPL; ++i) acc[i] = fmaf(w8[u], ov[u][i], acc[i]);
+      }
     }
     const float inv = L > 0.f ? 1.f / L : 0.f;
     if (o_bf16) {
@@ -197,7 +228,7 @@ __global__ void __launch_bounds__(kMergeThreads)
                       const uint16_t* __restrict__ vb, const uint16_t* __restrict__ dout,
                       const float* __restrict__ lse, const float* __restrict__ delta,
                       const float* __restrict__ dq_part, float scale, float* __restrict__ dq,
-                      float* __restrict__ dkb, float* __restrict__ dvb) {
+                      float* __restrict__ dkb, float* __restrict__ dvb, int stage_rows) {
   constexpr int DPL = D / 32;
   extern __shared__ __align__(16) uint8_t smem_raw[];
   const int bs = p.bs;
@@ -206,6 +237,8 @@ __global__ void __launch_bounds__(kMergeThreads)
   uint16_t* sVb = sKb + bs * D;
   float* sP = reinterpret_cast<float*>(sVb + bs * D);    // [rows][bs]
   float* sdS = sP + rows * bs;                            // [rows][bs]
+  uint16_t* sQr = reinterpret_cast<uint16_t*>(sdS + rows * bs);   // [rows][D] when stage_rows
+  uint16_t* sDr = sQr + rows * D;
   const int b = blockIdx.x, g = blockIdx.y;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int nwarps = blockDim.x >> 5;
@@ -252,18 +285,44 @@ __global__ void __launch_bounds__(kMergeThreads)
 #pragma unroll
       for (int i = 0; i < DPL; ++i) acc[i] = fmaf(ds, kv[i], acc[i]);
     }
-    // chunk partials in ascending chunk order, then the in-block term
+    // chunk partials in ascending chunk order (8 rows in flight), then the in-block term
     float tot[DPL];
 #pragma unroll
     for (int i = 0; i < DPL; ++i) tot[i] = 0.f;
-#pragma unroll 4
-    for (int x = e0; x < e1; ++x) {
-      const int e = p.block_entries[x];
-      const size_t rec = size_t(e * bs + tt) * p.Hq + head;
-      float pv[DPL];
-      load_f32_row<DPL>(dq_part + rec * D + lane * DPL, pv);
+    const int n = e1 - e0;
+    for (int base = 0; base < n; base += 32) {
+      int recl = 0;
+      if (base + lane < n) recl = (p.block_entries[e0 + base + lane] * bs + tt) * p.Hq + head;
+      const int cnt = min(32, n - base);
+      for (int j0 = 0; j0 < cnt; j0 += 8) {
+        float pv[8][DPL];
 #pragma unroll
-      for (int i = 0; i < DPL; ++i) tot[i] += pv[i];
+        for (int u = 0; u < 8; ++u) {
+          const int j = j0 + u;
+          const int rj = __shfl_sync(0xffffffffu, recl, j & 31);
+          if (j < cnt) {
+            load_f32_row<DPL>(dq_part + size_t(rj) * D + lane * DPL, pv[u]);
+          } else {
+#pragma unroll
+            for (int i = 0; i < DPL; ++i) pv[u][i] = 0.f;
+          }
+        }
+#pragma unroll
+        for (int u = 0; u < 8; ++u)
+#pragma unroll
+          for (int i = 0; i < DPL; ++i) tot[i] += pv[u][i];
+      }
+    }
+    if (stage_rows) {   // keep q and dout of this row for the dkb / dvb pass
+      uint16_t* sq = sQr + r * D + lane * DPL;
+      uint16_t* sd = sDr + r * D + lane * DPL;
+      if constexpr (DPL == 4) {
+        *reinterpret_cast<uint2*>(sq) = *reinterpret_cast<const uint2*>(q + qrow * D + lane * DPL);
+        *reinterpret_cast<uint2*>(sd) = *reinterpret_cast<const uint2*>(dout + qrow * D + lane * DPL);
+      } else {
+        *reinterpret_cast<uint32_t*>(sq) = *reinterpret_cast<const uint32_t*>(q + qrow * D + lane * DPL);
+        *reinterpret_cast<uint32_t*>(sd) = *reinterpret_cast<const uint32_t*>(dout + qrow * D + lane * DPL);
+      }
     }
     float* dst = dq + qrow * D + lane * DPL;
 #pragma unroll
@@ -281,11 +340,16 @@ __global__ void __launch_bounds__(kMergeThreads)
 #pragma unroll
     for (int i = 0; i < DPL; ++i) ak[i] = av[i] = 0.f;
     for (int r = 0; r < rows; ++r) {
-      const int hh = r / bs, tt = r % bs;
-      const size_t qrow = size_t(b * bs + tt) * p.Hq + g * p.G + hh;
       float qv[DPL], dov[DPL];
-      load_bf16_row<DPL>(q + qrow * D + lane * DPL, qv);
-      load_bf16_row<DPL>(dout + qrow * D + lane * DPL, dov);
+      if (stage_rows) {
+        load_bf16_row<DPL>(sQr + r * D + lane * DPL, qv);
+        load_bf16_row<DPL>(sDr + r * D + lane * DPL, dov);
+      } else {
+        const int hh = r / bs, tt = r % bs;
+        const size_t qrow = size_t(b * bs + tt) * p.Hq + g * p.G + hh;
+        load_bf16_row<DPL>(q + qrow * D + lane * DPL, qv);
+        load_bf16_row<DPL>(dout + qrow * D + lane * DPL, dov);
+      }
       const float ds = sdS[r * bs + key], pr = sP[r * bs + key];
 #pragma unroll
       for (int i = 0; i < DPL; ++i) {
@@ -323,12 +387,15 @@ cudaError_t reduce_d(const DevPlan& p, const uint16_t* q, const uint16_t* kb, co
                      const uint16_t* dout, const float* lse, const float* delta, const float* dq_part,
                      float scale, float* dq, float* dkb, float* dvb, cudaStream_t s) {
   const size_t rows = size_t(p.G) * p.bs;
-  const size_t smem = size_t(2) * p.bs * D * sizeof(uint16_t) + 2 * rows * p.bs * sizeof(float);
+  const size_t base = size_t(2) * p.bs * D * sizeof(uint16_t) + 2 * rows * p.bs * sizeof(float);
+  const size_t staged = base + 2 * rows * D * sizeof(uint16_t);
+  const int stage_rows = staged <= size_t(64) * 1024 ? 1 : 0;   // small enough to keep occupancy
+  const size_t smem = stage_rows ? staged : base;
   cudaError_t e =
       cudaFuncSetAttribute(bwd_reduce_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
   if (e != cudaSuccess) return e;
   bwd_reduce_kernel<D><<<dim3(p.A, p.Hkv), kMergeThreads, smem, s>>>(p, q, kb, vb, dout, lse, delta, dq_part,
-                                                                       scale, dq, dkb, dvb);
+                                                                       scale, dq, dkb, dvb, stage_rows);
   return cudaGetLastError();
 }
 
