@@ -24,10 +24,15 @@
 //      dQ += dS K                           (A operand from TMEM)
 //    then scale * dQ is written once as the (chunk, block) entry's dq partial.
 //
-// Roles per CTA (256 threads): warp 0 TMA producer, warp 1 MMA issuer (one
-// thread), warp 2 tensor-memory allocation, warps 4-7 element-wise work and
-// epilogue (thread = TMEM lane).  Waits are bounded; a timeout is recorded in
-// the plan's status word and every role winds down.
+// Roles per CTA (384 threads): warp 0 TMA producer, warp 1 MMA issuer (one
+// thread), warp 2 tensor-memory allocation, warp 3 prefetches the row
+// metadata of upcoming query tiles into shared memory, warps 4-11 element-wise work and
+// epilogue in two warpgroups that split the 128 columns of every tile between
+// them (thread = TMEM lane; warpgroup h takes columns 64h..64h+63).  Each
+// warpgroup writes its bf16 results into its own columns (the MMA addresses the
+// 16-wide K-steps one by one), so neither overwrites scores the other has not
+// read yet.  Waits are bounded; a timeout is recorded in the plan's status word
+// and every role winds down.
 #include <cfloat>
 
 #include "sm100.cuh"
@@ -41,12 +46,12 @@ using namespace sm100;
 
 constexpr int D = 128;
 constexpr int BT = 128;                // keys per key tile = rows per query tile
-constexpr int kThreads = 256;
+constexpr int kThreads = 384;
 constexpr uint32_t kHalf = 128 * 128;  // one 64-column half of a 128-row bf16 tile
 constexpr uint32_t kTile = 2 * kHalf;  // 32 KB
 constexpr uint32_t kIdescKM = idesc_bf16_f32(128, 128, 0);  // B K-major
 constexpr uint32_t kIdescMN = idesc_bf16_f32(128, D, 1);    // B MN-major
-constexpr uint32_t kSmemBytes = 6 * kTile + 4096 + 256 + 1024;
+constexpr uint32_t kSmemBytes = 6 * kTile + 8192 + 256 + 1024;
 
 
 // K-major SW128 descriptor of the k-th 16-column step of a 128-row tile.
@@ -57,6 +62,11 @@ __device__ __forceinline__ uint64_t kmajor(uint32_t tile, int kk) {
 __device__ __forceinline__ uint64_t mnmajor(uint32_t tile, int kk) {
   return smem_desc_sw128(tile + kk * 2048, kHalf, 1024);
 }
+// TMEM column (relative to a 128-column score buffer) of the bf16 pairs of the
+// k-th 16-wide K-step: steps 0..3 (written by warpgroup 0) sit in columns 0..31,
+// steps 4..7 (warpgroup 1) in columns 64..95 -- inside each warpgroup's own
+// half of the buffer, over scores it has already read.
+__device__ __forceinline__ uint32_t packed_col(int kk) { return (kk < 4 ? 0u : 64u) + 8u * uint32_t(kk & 3); }
 
 // Row metadata of query-tile row r (rows ordered slot, token, head).
 struct RowMeta {
@@ -114,23 +124,22 @@ __device__ __forceinline__ void setup_common(uint64_t* bars, int nbars, const ui
   tc_fence_after();
 }
 
-// dq kernel, one key tile of one row (thread = TMEM lane): dS = P (dP - Delta)
-// with P = exp2(s * c - lse2), zero outside the row's columns [a, b); bf16 dS
-// pairs go to TMEM columns [0, 64) of the score buffer.  Two 64-column halves.
+// dq kernel, half hf of one key tile for one row (thread = TMEM lane): dS =
+// P (dP - Delta) with P = exp2(s * c - lse2), zero outside the row's columns
+// [a, b) of the tile; bf16 pairs of dS go to packed_col() of the score buffer.
 template <bool kMasked>
-__device__ __forceinline__ void ds_tile(uint32_t tS, uint32_t tdP, int a, int b, float c, float l2, float dl) {
-#pragma unroll
-  for (int h = 0; h < 2; ++h) {
-    uint32_t sv[64], dpv[64];
-    tmem_ld32p(tS + h * 64, sv);
-    tmem_ld32p(tS + h * 64 + 32, sv + 32);
-    tmem_ld32p(tdP + h * 64, dpv);
-    tmem_ld32p(tdP + h * 64 + 32, dpv + 32);
+__device__ __forceinline__ void ds_tile(uint32_t tS, uint32_t tdP, int hf, int a, int b, float c, float l2,
+                                        float dl) {
+#pragma unroll 1
+  for (int q = 2 * hf; q < 2 * hf + 2; ++q) {   // 32 keys per TMEM round trip
+    uint32_t sv[32], dpv[32];
+    tmem_ld32(tS + q * 32, sv);
+    tmem_ld32(tdP + q * 32, dpv);
     tmem_wait_ld();
-    uint32_t pk[32];
+    uint32_t pk[16];
 #pragma unroll
-    for (int i = 0; i < 32; ++i) {
-      const int col = h * 64 + 2 * i;
+    for (int i = 0; i < 16; ++i) {
+      const int col = q * 32 + 2 * i;
       float x0, x1, d0, d1, g0, g1;
       ffma2(x0, x1, __uint_as_float(sv[2 * i]), __uint_as_float(sv[2 * i + 1]), c, c, -l2, -l2);
       float p0 = fast_exp2(x0), p1 = fast_exp2(x1);
@@ -142,20 +151,19 @@ __device__ __forceinline__ void ds_tile(uint32_t tS, uint32_t tdP, int a, int b,
       fmul2(g0, g1, p0, p1, d0, d1);
       pk[i] = pack_bf16(g0, g1);
     }
-    tmem_st16p(tS + h * 32, pk);
-    tmem_st16p(tS + h * 32 + 16, pk + 16);
+    tmem_st16p(tS + packed_col(2 * q), pk);
   }
 }
 
-// dkdv kernel, one query tile for one key (thread = TMEM lane): P^T and
-// dS^T = P^T (dP^T - Delta) over the 128 rows, P = exp2(s * c - lse2[row]),
-// zero for rows whose slot bit (slot = row >> lg) is clear.  bf16 pairs
-// of rows go to TMEM columns [0, 64) of S^T and of dP^T.
+// dkdv kernel, rows 64hf..64hf+63 of one query tile for one key (thread = TMEM
+// lane): P^T and dS^T = P^T (dP^T - Delta), P = exp2(s * c - lse2[row]), zero
+// for rows whose slot bit (slot = row >> lg) is clear; bf16 pairs of rows go to
+// packed_col() of S^T and of dP^T.
 template <bool kMasked>
-__device__ __forceinline__ void pds_tile(uint32_t tSt, uint32_t tdPt, uint32_t smask, int lg,
+__device__ __forceinline__ void pds_tile(uint32_t tSt, uint32_t tdPt, int hf, uint32_t smask, int lg,
                                          const float4* ld4, float c) {
 #pragma unroll 1
-  for (int q = 0; q < 4; ++q) {        // 32 rows per TMEM round trip
+  for (int q = 2 * hf; q < 2 * hf + 2; ++q) {   // 32 rows per TMEM round trip
     uint32_t sv[32], dpv[32];
     tmem_ld32(tSt + q * 32, sv);
     tmem_ld32(tdPt + q * 32, dpv);
@@ -178,8 +186,8 @@ __device__ __forceinline__ void pds_tile(uint32_t tSt, uint32_t tdPt, uint32_t s
       pp[i] = pack_bf16(p0, p1);
       pd[i] = pack_bf16(g0, g1);
     }
-    tmem_st16p(tSt + q * 16, pp);
-    tmem_st16p(tdPt + q * 16, pd);
+    tmem_st16p(tSt + packed_col(2 * q), pp);
+    tmem_st16p(tdPt + packed_col(2 * q), pd);
   }
 }
 
@@ -188,11 +196,11 @@ __device__ __forceinline__ void pds_tile(uint32_t tSt, uint32_t tdPt, uint32_t s
 // ============================================================================
 struct DkdvBars {
   uint64_t kv_full, kv_empty, qd_full[2], qd_empty[2], st_ready, pds_ready, dkv_ready, dkv_free, mma_done,
-      meta_ready[2];
+      meta_ready[2], meta_free[2];
   uint32_t tmem_base;
   int abort_flag;
 };
-constexpr int kDkdvNumBars = 13;
+constexpr int kDkdvNumBars = 15;
 
 __global__ void __launch_bounds__(kThreads, 1)
     bwd_dkdv_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_do,
@@ -207,7 +215,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* sdO = smem + 4 * kTile;  // [2 stages]
   float2* meta_ld = reinterpret_cast<float2*>(smem + 6 * kTile);             // [2][128] (lse2, delta) per row
   int2* meta_slot = reinterpret_cast<int2*>(smem + 6 * kTile + 2048);         // [2][16] (lo, hi) per slot
-  DkdvBars* B = reinterpret_cast<DkdvBars*>(smem + 6 * kTile + 4096);
+  DkdvBars* B = reinterpret_cast<DkdvBars*>(smem + 6 * kTile + 8192);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int w = blockIdx.x;
   volatile int* abort_flag = &B->abort_flag;
@@ -217,7 +225,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     B->abort_flag = 0;
   }
   {
-    const uint32_t counts[kDkdvNumBars] = {1, 1, 1, 1, 1, 1, 1, 128, 1, 128, 1, 128, 128};
+    const uint32_t counts[kDkdvNumBars] = {1, 1, 1, 1, 1, 1, 1, 256, 1, 256, 1, 32, 32, 256, 256};
     setup_common(&B->kv_full, kDkdvNumBars, counts, &B->tmem_base, warp);
   }
   const uint32_t tmem = B->tmem_base;
@@ -282,6 +290,14 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int kk = 0; kk < D / 16; ++kk)
               mma_ss(tmem + 128, kmajor(aV, kk), kmajor(adO + s * kTile, kk), kIdescKM, kk > 0 ? 1u : 0u);
             mma_commit(&B->st_ready);
+            {   // K and V are read only by S^T / dP^T: release them after the key tile's last pair
+              bool later = false;
+              for (int t2 = t + 1; t2 < item.w && !later; ++t2) {
+                const int4 tl2 = p.tiles[t2];
+                later = tl2.z < k0 + BT && tl2.w > k0;
+              }
+              if (!later) mma_commit(&B->kv_empty);
+            }
             if (!mbar_wait(&B->pds_ready, pds_cnt & 1, wctx, 2 * 10000 + __LINE__)) { ok = false; break; }
             ++pds_cnt;
             if (u == 0) {
@@ -291,10 +307,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             tc_fence_after();
             // dV (cols 384..) += P^T dO ; dK (cols 256..) += dS^T Q  -- A operands from TMEM
             for (int kk = 0; kk < BT / 16; ++kk)
-              mma_ts(tmem + 384, tmem + 0 + kk * 8, mnmajor(adO + s * kTile, kk), kIdescMN,
+              mma_ts(tmem + 384, tmem + 0 + packed_col(kk), mnmajor(adO + s * kTile, kk), kIdescMN,
                      (u > 0 || kk > 0) ? 1u : 0u);
             for (int kk = 0; kk < BT / 16; ++kk)
-              mma_ts(tmem + 256, tmem + 128 + kk * 8, mnmajor(aQ + s * kTile, kk), kIdescMN,
+              mma_ts(tmem + 256, tmem + 128 + packed_col(kk), mnmajor(aQ + s * kTile, kk), kIdescMN,
                      (u > 0 || kk > 0) ? 1u : 0u);
             mma_commit(&B->qd_empty[s]);
             ++qd_count;
@@ -302,7 +318,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           if (!ok) break;
           if (u > 0) mma_commit(&B->dkv_ready);
-          mma_commit(&B->kv_empty);
+          else mma_commit(&B->kv_empty);   // no pair met this key tile
           ++kt_count;
         }
       }
@@ -310,20 +326,52 @@ __global__ void __launch_bounds__(kThreads, 1)
       mma_commit(&B->mma_done);
       mbar_drain(&B->mma_done, 0, wctx, 2 * 10000 + __LINE__);
     }
+  } else if (warp == 3) {
+    // metadata of the query tiles, in the element-wise order, up to two tiles ahead
+    uint32_t mcount = 0;
+    bool ok = true;
+    for (int it = p.bwd_worker_ptr[w]; ok && it < p.bwd_worker_ptr[w + 1]; ++it) {
+      const int4 item = p.bwd_items[it];
+      const int g = item.y, c0 = item.x * p.C, c1 = min(c0 + p.C, p.N);
+      for (int k0 = c0; ok && k0 < c1; k0 += BT) {
+        for (int t = item.z; t < item.w; ++t) {
+          const int4 tile = p.tiles[t];
+          if (!(tile.z < k0 + BT && tile.w > k0)) continue;
+          const int s = mcount & 1;
+          if (!warp_wait(&B->meta_free[s], ((mcount >> 1) & 1) ^ 1, wctx, 2 * 10000 + __LINE__)) { ok = false; break; }
+          const int rps = p.G * p.bs;
+          for (int rr = lane; rr < BT; rr += 32) {
+            const RowMeta m = row_meta(p, tile, g, rr);
+            float l2 = INFINITY, dl = 0.f;
+            if (m.valid) {
+              const float L = lse[m.qrow];
+              l2 = (L == -INFINITY) ? INFINITY : L * kLog2e;
+              dl = delta[m.qrow];
+            }
+            meta_ld[s * 128 + rr] = make_float2(l2, dl);
+            if (rr % rps == 0) meta_slot[s * 16 + rr / rps] = make_int2(m.lo, m.hi);
+          }
+          mbar_arrive(&B->meta_ready[s]);
+          ++mcount;
+        }
+      }
+    }
+    if (!ok) *abort_flag = 1;
   } else if (warp >= 4) {
-    const int r = ((warp & 3) << 5) + lane;   // key of the tile = TMEM lane; also the row this thread describes
+    const int hf = (warp - 4) >> 2;           // warpgroup: rows 64hf..64hf+63 of every query tile
+    const int r = ((warp & 3) << 5) + lane;   // key of the tile = TMEM lane
     const uint32_t lane_addr = uint32_t((warp & 3) << 5) << 16;
     const uint32_t tSt = tmem + lane_addr;          // S^T / P^T
     const uint32_t tdPt = tmem + lane_addr + 128;   // dP^T / dS^T
-    const uint32_t tdK = tmem + lane_addr + 256;
-    const uint32_t tdV = tmem + lane_addr + 384;
+    const uint32_t tAcc = tmem + lane_addr + 256 + hf * 128;   // dK (warpgroup 0) or dV (warpgroup 1)
     const float scale_log2 = scale * kLog2e;
     // chunks no block reads: zeros for every KV head
+    const int et = tid - 128;
     for (int z = w; z < p.num_zero_chunks; z += p.Wb) {
       const int c = p.zero_chunks[z];
       const size_t first = size_t(c) * p.C * kv_row;
       const size_t last = size_t(min(c * p.C + p.C, p.N)) * kv_row;
-      for (size_t i = first + size_t(r) * 4; i < last; i += size_t(128) * 4) {
+      for (size_t i = first + size_t(et) * 4; i < last; i += size_t(256) * 4) {
         *reinterpret_cast<float4*>(dk + i) = make_float4(0.f, 0.f, 0.f, 0.f);
         *reinterpret_cast<float4*>(dv + i) = make_float4(0.f, 0.f, 0.f, 0.f);
       }
@@ -341,20 +389,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (!(tile.z < k0 + BT && tile.w > k0)) continue;
           const int s = qd_count & 1;
           const int rps = p.G * p.bs;
-          {
-            // this thread describes row r of the query tile (and slot r / rps's interval)
-            const RowMeta m = row_meta(p, tile, g, r);
-            float l2 = INFINITY, dl = 0.f;
-            if (m.valid) {
-              const float L = lse[m.qrow];
-              l2 = (L == -INFINITY) ? INFINITY : L * kLog2e;
-              dl = delta[m.qrow];
-            }
-            meta_ld[s * 128 + r] = make_float2(l2, dl);
-            if (r % rps == 0) meta_slot[s * 16 + r / rps] = make_int2(m.lo, m.hi);
-          }
-          // every thread needs all 128 rows' metadata: bounded handoff through an mbarrier
-          mbar_arrive(&B->meta_ready[s]);
+          // the tile's row metadata, prefetched by warp 3
           if (!warp_wait(&B->meta_ready[s], (qd_count >> 1) & 1, wctx, 2 * 10000 + __LINE__)) { ok = false; break; }
           // slots (blocks) that may read this thread's key: one bit per slot.  Padding
           // slots count as "in": their rows have lse2 = +inf, so P = 0 there anyway.
@@ -373,19 +408,21 @@ __global__ void __launch_bounds__(kThreads, 1)
           tc_fence_after();
           const float4* ld4 = reinterpret_cast<const float4*>(meta_ld + s * 128);
           if (all_in)
-            pds_tile<false>(tSt, tdPt, smask, lg, ld4, scale_log2);
+            pds_tile<false>(tSt, tdPt, hf, smask, lg, ld4, scale_log2);
           else
-            pds_tile<true>(tSt, tdPt, smask, lg, ld4, scale_log2);
+            pds_tile<true>(tSt, tdPt, hf, smask, lg, ld4, scale_log2);
           tmem_wait_st();
           tc_fence_before();
           mbar_arrive(&B->pds_ready);
+          mbar_arrive(&B->meta_free[s]);
           ++qd_count;
           ++n_meet;
         }
         if (!ok) break;
-        // epilogue of the key tile: dK * scale, dV (zeros when no query met it)
-        float* dkr = dk + (size_t(key) * p.Hkv + g) * D;
-        float* dvr = dv + (size_t(key) * p.Hkv + g) * D;
+        // epilogue of the key tile: warpgroup 0 writes dK * scale, warpgroup 1 dV
+        // (zeros when no query met the tile)
+        float* dst = (hf == 0 ? dk : dv) + (size_t(key) * p.Hkv + g) * D;
+        const float f = hf == 0 ? scale : 1.f;
         const bool own = key < c1;
         if (n_meet > 0) {
           if (!warp_wait(&B->dkv_ready, dkv_cnt & 1, wctx, 2 * 10000 + __LINE__)) { ok = false; break; }
@@ -393,29 +430,21 @@ __global__ void __launch_bounds__(kThreads, 1)
           tc_fence_after();
 #pragma unroll 1
           for (int cc = 0; cc < D / 32; ++cc) {
-            uint32_t a[32], b[32];
-            tmem_ld32(tdK + cc * 32, a);
-            tmem_ld32(tdV + cc * 32, b);
+            uint32_t a[32];
+            tmem_ld32(tAcc + cc * 32, a);
             tmem_wait_ld();
             if (own) {
 #pragma unroll
-              for (int i = 0; i < 32; i += 4) {
-                *reinterpret_cast<float4*>(dkr + cc * 32 + i) =
-                    make_float4(scale * __uint_as_float(a[i]), scale * __uint_as_float(a[i + 1]),
-                                scale * __uint_as_float(a[i + 2]), scale * __uint_as_float(a[i + 3]));
-                *reinterpret_cast<float4*>(dvr + cc * 32 + i) =
-                    make_float4(__uint_as_float(b[i]), __uint_as_float(b[i + 1]), __uint_as_float(b[i + 2]),
-                                __uint_as_float(b[i + 3]));
-              }
+              for (int i = 0; i < 32; i += 4)
+                *reinterpret_cast<float4*>(dst + cc * 32 + i) =
+                    make_float4(f * __uint_as_float(a[i]), f * __uint_as_float(a[i + 1]),
+                                f * __uint_as_float(a[i + 2]), f * __uint_as_float(a[i + 3]));
             }
           }
           tc_fence_before();
           mbar_arrive(&B->dkv_free);
         } else if (own) {
-          for (int i = 0; i < D; i += 4) {
-            *reinterpret_cast<float4*>(dkr + i) = make_float4(0.f, 0.f, 0.f, 0.f);
-            *reinterpret_cast<float4*>(dvr + i) = make_float4(0.f, 0.f, 0.f, 0.f);
-          }
+          for (int i = 0; i < D; i += 4) *reinterpret_cast<float4*>(dst + i) = make_float4(0.f, 0.f, 0.f, 0.f);
         }
       }
     }
@@ -433,11 +462,17 @@ __global__ void __launch_bounds__(kThreads, 1)
 // ============================================================================
 struct DqBars {
   uint64_t qd_full, qd_empty, k_full[2], v_full[2], kv_empty[2], s_ready[2], dp_ready, ds_ready, dq_ready, dq_free,
-      mma_done;
+      mma_done, meta_ready[2], meta_free[2];
   uint32_t tmem_base;
   int abort_flag;
 };
-constexpr int kDqNumBars = 15;
+constexpr int kDqNumBars = 19;
+
+// Per-row metadata of a query tile for the dq kernel (shared memory).
+struct DqRow {
+  int lo, hi, rec, valid;
+  float l2, dl;
+};
 
 // The query tiles of a worker's forward schedule, one at a time.
 struct TileIter {
@@ -475,14 +510,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* sdO = smem + kTile;
   uint8_t* sK = smem + 2 * kTile;   // [2 stages]
   uint8_t* sV = smem + 4 * kTile;   // [2 stages]
-  DqBars* B = reinterpret_cast<DqBars*>(smem + 6 * kTile + 4096);
+  DqRow* meta = reinterpret_cast<DqRow*>(smem + 6 * kTile);   // [2][128]
+  DqBars* B = reinterpret_cast<DqBars*>(smem + 6 * kTile + 8192);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int w = blockIdx.x;
   volatile int* abort_flag = &B->abort_flag;
   const WaitCtx wctx{abort_flag, p.status};
   if (tid == 0) B->abort_flag = 0;
   {
-    const uint32_t counts[kDqNumBars] = {1, 1, 1, 1, 1, 1, 1, 1, 1, 1, 1, 128, 1, 128, 1};
+    const uint32_t counts[kDqNumBars] = {1, 1, 1, 1, 1, 1, 1, 1, 1, 1, 1, 256, 1, 256, 1, 32, 32, 256, 256};
     setup_common(&B->qd_full, kDqNumBars, counts, &B->tmem_base, warp);
   }
   const uint32_t tmem = B->tmem_base;
@@ -570,7 +606,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           tc_fence_after();
           // dQ (cols 384..) += dS K : dS in TMEM (columns 0..63 of S buffer s), K MN-major
           for (int kk = 0; kk < BT / 16; ++kk)
-            mma_ts(tmem + 384, tmem + s * 128 + kk * 8, mnmajor(aK + s * kTile, kk), kIdescMN,
+            mma_ts(tmem + 384, tmem + s * 128 + packed_col(kk), mnmajor(aK + s * kTile, kk), kIdescMN,
                    (j > 0 || kk > 0) ? 1u : 0u);
           mma_commit(&B->kv_empty[s]);
           if (more) {
@@ -579,11 +615,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int kk = 0; kk < D / 16; ++kk)
               mma_ss(tmem + 256, kmajor(adO, kk), kmajor(aV + s1 * kTile, kk), kIdescKM, kk > 0 ? 1u : 0u);
             mma_commit(&B->dp_ready);
+            if (j + 2 == n_kt) mma_commit(&B->qd_empty);   // Q, dO: no further reader after this S / dP
           }
         }
         if (!ok) break;
         mma_commit(&B->dq_ready);
-        mma_commit(&B->qd_empty);
+        if (n_kt == 1) mma_commit(&B->qd_empty);
         kv_count += n_kt;
         ++tile_count;
       }
@@ -591,27 +628,58 @@ __global__ void __launch_bounds__(kThreads, 1)
       mma_commit(&B->mma_done);
       mbar_drain(&B->mma_done, 0, wctx, 2 * 10000 + __LINE__);
     }
+  } else if (warp == 3) {
+    // row metadata of upcoming query tiles, up to two tiles ahead
+    TileIter ti;
+    ti.init(&p, w);
+    int t, g;
+    uint32_t mcount = 0;
+    bool ok = true;
+    while (ok && ti.next(t, g)) {
+      const int4 tile = p.tiles[t];
+      const int s = mcount & 1;
+      if (!warp_wait(&B->meta_free[s], ((mcount >> 1) & 1) ^ 1, wctx, 2 * 10000 + __LINE__)) { ok = false; break; }
+      for (int rr = lane; rr < BT; rr += 32) {
+        const RowMeta m = row_meta(p, tile, g, rr);
+        DqRow d;
+        d.lo = m.lo;
+        d.hi = m.hi;
+        d.rec = m.rec;
+        d.valid = m.valid ? 1 : 0;
+        d.l2 = INFINITY;
+        d.dl = 0.f;
+        if (m.valid) {
+          const float L = lse[m.qrow];
+          d.l2 = (L == -INFINITY) ? INFINITY : L * kLog2e;
+          d.dl = delta[m.qrow];
+        }
+        meta[s * 128 + rr] = d;
+      }
+      mbar_arrive(&B->meta_ready[s]);
+      ++mcount;
+    }
+    if (!ok) *abort_flag = 1;
   } else if (warp >= 4) {
+    const int hf = (warp - 4) >> 2;           // warpgroup: keys 64hf..64hf+63 of every key tile
     const int r = ((warp & 3) << 5) + lane;
     const uint32_t lane_addr = uint32_t((warp & 3) << 5) << 16;
     const uint32_t tdP = tmem + lane_addr + 256;
-    const uint32_t tdQ = tmem + lane_addr + 384;
+    const uint32_t tdQ = tmem + lane_addr + 384 + hf * 64;   // this warpgroup's 64 dQ columns
     const float scale_log2 = scale * kLog2e;
     TileIter ti;
     ti.init(&p, w);
     int t, g;
-    uint32_t kv_count = 0, dp_cnt = 0, dq_cnt = 0;
+    uint32_t kv_count = 0, dp_cnt = 0, dq_cnt = 0, mcount = 0;
     bool ok = true;
     while (ok && ti.next(t, g)) {
       const int4 tile = p.tiles[t];
       const int n_kt = (tile.w - tile.z + BT - 1) / BT;
-      const RowMeta m = row_meta(p, tile, g, r);
-      float l2 = INFINITY, dl = 0.f;
-      if (m.valid) {
-        const float L = lse[m.qrow];
-        l2 = (L == -INFINITY) ? INFINITY : L * kLog2e;
-        dl = delta[m.qrow];
-      }
+      const int ms = mcount & 1;
+      if (!warp_wait(&B->meta_ready[ms], (mcount >> 1) & 1, wctx, 2 * 10000 + __LINE__)) { ok = false; break; }
+      const DqRow m = meta[ms * 128 + r];
+      mbar_arrive(&B->meta_free[ms]);
+      ++mcount;
+      const float l2 = m.l2, dl = m.dl;
       for (int j = 0; j < n_kt; ++j) {
         const uint32_t c = kv_count + j;
         const int s = c & 1;
@@ -623,10 +691,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int k0 = tile.z + j * BT;
         const int a = m.lo - k0, b = m.hi - k0;   // the row's allowed columns of this key tile
         // warp-uniform choice: both paths issue warp-collective tcgen05.ld/st
-        if (__all_sync(0xffffffffu, a <= 0 && b >= BT))
-          ds_tile<false>(tS, tdP, a, b, scale_log2, l2, dl);
+        if (__all_sync(0xffffffffu, a <= hf * 64 && b >= hf * 64 + 64))
+          ds_tile<false>(tS, tdP, hf, a, b, scale_log2, l2, dl);
         else
-          ds_tile<true>(tS, tdP, a, b, scale_log2, l2, dl);
+          ds_tile<true>(tS, tdP, hf, a, b, scale_log2, l2, dl);
         tmem_wait_st();
         tc_fence_before();
         mbar_arrive(&B->ds_ready);
@@ -636,9 +704,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!warp_wait(&B->dq_ready, dq_cnt & 1, wctx, 2 * 10000 + __LINE__)) { ok = false; break; }
       ++dq_cnt;
       tc_fence_after();
-      float* dst = dq_part + size_t(m.rec) * D;
+      float* dst = dq_part + size_t(m.rec) * D + hf * 64;
 #pragma unroll 1
-      for (int cc = 0; cc < D / 32; ++cc) {
+      for (int cc = 0; cc < 2; ++cc) {
         uint32_t v[32];
         tmem_ld32(tdQ + cc * 32, v);
         tmem_wait_ld();
