@@ -51,7 +51,12 @@ constexpr uint32_t kHalf = 128 * 128;  // one 64-column half of a 128-row bf16 t
 constexpr uint32_t kTile = 2 * kHalf;  // 32 KB
 constexpr uint32_t kIdescKM = idesc_bf16_f32(128, 128, 0);  // B K-major
 constexpr uint32_t kIdescMN = idesc_bf16_f32(128, D, 1);    // B MN-major
-constexpr uint32_t kSmemBytes = 6 * kTile + 8192 + 256 + 1024;
+// 6 tiles | row metadata (8 KB) | epilogue scratch (2 KB per element-wise warp) | barriers
+constexpr uint32_t kOffMeta = 6 * kTile;
+constexpr uint32_t kOffScratch = kOffMeta + 8192;
+constexpr uint32_t kOffBars = kOffScratch + 8 * 2048;
+constexpr uint32_t kSmemBytes = kOffBars + 256 + 1024;
+static_assert(kSmemBytes <= 232448, "shared memory per block");
 
 
 // K-major SW128 descriptor of the k-th 16-column step of a 128-row tile.
@@ -215,7 +220,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* sdO = smem + 4 * kTile;  // [2 stages]
   float2* meta_ld = reinterpret_cast<float2*>(smem + 6 * kTile);             // [2][128] (lse2, delta) per row
   int2* meta_slot = reinterpret_cast<int2*>(smem + 6 * kTile + 2048);         // [2][16] (lo, hi) per slot
-  DkdvBars* B = reinterpret_cast<DkdvBars*>(smem + 6 * kTile + 8192);
+  DkdvBars* B = reinterpret_cast<DkdvBars*>(smem + kOffBars);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int w = blockIdx.x;
   volatile int* abort_flag = &B->abort_flag;
@@ -428,18 +433,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (!warp_wait(&B->dkv_ready, dkv_cnt & 1, wctx, 2 * 10000 + __LINE__)) { ok = false; break; }
           ++dkv_cnt;
           tc_fence_after();
+          float* scratch = reinterpret_cast<float*>(smem + kOffScratch) + (warp - 4) * 512;
 #pragma unroll 1
-          for (int cc = 0; cc < D / 32; ++cc) {
-            uint32_t a[32];
-            tmem_ld32(tAcc + cc * 32, a);
+          for (int cc = 0; cc < D / 16; ++cc) {
+            uint32_t a[16];
+            tmem_ld16(tAcc + cc * 16, a);
             tmem_wait_ld();
-            if (own) {
-#pragma unroll
-              for (int i = 0; i < 32; i += 4)
-                *reinterpret_cast<float4*>(dst + cc * 32 + i) =
-                    make_float4(f * __uint_as_float(a[i]), f * __uint_as_float(a[i + 1]),
-                                f * __uint_as_float(a[i + 2]), f * __uint_as_float(a[i + 3]));
-            }
+            warp_store_rows<16>(scratch, reinterpret_cast<const float*>(a), f, own ? dst + cc * 16 : nullptr);
           }
           tc_fence_before();
           mbar_arrive(&B->dkv_free);
@@ -511,7 +511,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* sK = smem + 2 * kTile;   // [2 stages]
   uint8_t* sV = smem + 4 * kTile;   // [2 stages]
   DqRow* meta = reinterpret_cast<DqRow*>(smem + 6 * kTile);   // [2][128]
-  DqBars* B = reinterpret_cast<DqBars*>(smem + 6 * kTile + 8192);
+  DqBars* B = reinterpret_cast<DqBars*>(smem + kOffBars);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int w = blockIdx.x;
   volatile int* abort_flag = &B->abort_flag;
@@ -705,18 +705,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       ++dq_cnt;
       tc_fence_after();
       float* dst = dq_part + size_t(m.rec) * D + hf * 64;
+      float* scratch = reinterpret_cast<float*>(smem + kOffScratch) + (warp - 4) * 512;
 #pragma unroll 1
-      for (int cc = 0; cc < 2; ++cc) {
-        uint32_t v[32];
-        tmem_ld32(tdQ + cc * 32, v);
+      for (int cc = 0; cc < 4; ++cc) {
+        uint32_t v[16];
+        tmem_ld16(tdQ + cc * 16, v);
         tmem_wait_ld();
-        if (m.valid) {
-#pragma unroll
-          for (int i = 0; i < 32; i += 4)
-            *reinterpret_cast<float4*>(dst + cc * 32 + i) =
-                make_float4(scale * __uint_as_float(v[i]), scale * __uint_as_float(v[i + 1]),
-                            scale * __uint_as_float(v[i + 2]), scale * __uint_as_float(v[i + 3]));
-        }
+        warp_store_rows<16>(scratch, reinterpret_cast<const float*>(v), scale, m.valid ? dst + cc * 16 : nullptr);
       }
       tc_fence_before();
       mbar_arrive(&B->dq_free);

@@ -52,8 +52,10 @@ constexpr float kRescaleLog2 = 8.0f;  // rescale O only when the max grows by mo
 constexpr uint32_t kOffQ = 0;                              // Q_A, Q_B
 constexpr uint32_t kOffK = kOffQ + 2 * kTile;              // K stages
 constexpr uint32_t kOffV = kOffK + kStages * kTile;        // V stages
-constexpr uint32_t kOffBar = kOffV + kStages * kTile;      // mbarriers
+constexpr uint32_t kOffScratch = kOffV + kStages * kTile; // epilogue scratch, 4 KB per softmax warp
+constexpr uint32_t kOffBar = kOffScratch + 8 * 4096;       // mbarriers
 constexpr uint32_t kSmemBytes = kOffBar + 256 + 1024;      // + alignment slack
+static_assert(kSmemBytes <= 232448, "shared memory per block");
 
 struct Bars {
   uint64_t q_full, q_empty;
@@ -317,13 +319,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                 mma_ss(tmem + x * 128, a, b, kIdescQK, kk > 0 ? 1u : 0u);
               }
               mma_commit(&bars->s_ready[x]);
+              // the pair's last S: Q_A / Q_B have no further reader
+              if (j + 2 == n_kt && x == nx - 1) mma_commit(&bars->q_empty);
             }
           }
           if (!ok) break;
           mma_commit(&bars->kv_empty[s]);   // K_s, V_s free once everything issued so far completes
         }
         if (!ok) break;
-        mma_commit(&bars->q_empty);
+        if (n_kt == 1) mma_commit(&bars->q_empty);
         kv_count += n_kt;
         ++pair_count;
       }
@@ -430,20 +434,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       o_cnt += n_kt;
       tc_fence_after();
       const float inv = l > 0.f ? 1.f / l : 0.f;
-      float* dst = part_o + size_t(rec) * D;
+      float* scratch = reinterpret_cast<float*>(smem + kOffScratch) + (warp - 4) * 1024;
 #pragma unroll 1
       for (int cch = 0; cch < D / 32; ++cch) {
         uint32_t v[32];
         tmem_ld32(tO + cch * 32, v);
         tmem_wait_ld();
-        if (valid) {
-#pragma unroll
-          for (int i = 0; i < 32; i += 4) {
-            *reinterpret_cast<float4*>(dst + cch * 32 + i) =
-                make_float4(__uint_as_float(v[i]) * inv, __uint_as_float(v[i + 1]) * inv,
-                            __uint_as_float(v[i + 2]) * inv, __uint_as_float(v[i + 3]) * inv);
-          }
-        }
+        warp_store_rows<32>(scratch, reinterpret_cast<const float*>(v), inv,
+                            valid ? part_o + size_t(rec) * D + cch * 32 : nullptr);
       }
       if (valid) {
         // record (true max, sum relative to it)

@@ -271,5 +271,36 @@ __device__ __forceinline__ void fmul2(float& d0, float& d1, float a0, float a1, 
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
+// ---------------------------------------------------------------- epilogue stores
+// Lane i of a warp holds W consecutive fp32 values of its own output row
+// (vals[0..W)); dst is that row's destination (NULL for a row that is not
+// written).  The values go through a per-warp scratch of 32 x W floats in
+// shared memory so that every global store instruction writes whole 4W-byte
+// row segments of 128 / W rows instead of 32 scattered 16-byte pieces.
+// W is 16 or 32; the scratch is XOR-swizzled by 16-byte granule.
+template <int W>
+__device__ __forceinline__ void warp_store_rows(float* scratch, const float* vals, float mul, float* dst) {
+  constexpr int kG = W / 4;          // 16-byte granules per row
+  constexpr int kRows = 32 / kG;     // rows per store instruction
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int g = 0; g < kG; ++g) {
+    const float4 x = make_float4(vals[4 * g] * mul, vals[4 * g + 1] * mul, vals[4 * g + 2] * mul,
+                                 vals[4 * g + 3] * mul);
+    *reinterpret_cast<float4*>(scratch + lane * W + ((g ^ (lane & (kG - 1))) << 2)) = x;
+  }
+  __syncwarp();
+  const unsigned long long mine = reinterpret_cast<unsigned long long>(dst);
+#pragma unroll
+  for (int k = 0; k < kG; ++k) {
+    const int r = k * kRows + lane / kG;
+    const int gi = lane % kG;
+    const float4 x = *reinterpret_cast<const float4*>(scratch + r * W + ((gi ^ (r & (kG - 1))) << 2));
+    float* d = reinterpret_cast<float*>(__shfl_sync(0xffffffffu, mine, r));
+    if (d != nullptr) *reinterpret_cast<float4*>(d + 4 * gi) = x;
+  }
+  __syncwarp();
+}
+
 }  // namespace sm100
 }  // namespace splitkv
