@@ -158,7 +158,10 @@ def _kernel_work(st, w, E):
     rec_rows = E * bs * Hq
     return {
         "fwd_partial": ("tensor", 4.0 * d * ctx),
-        "bwd_partial": ("tensor", 10.0 * d * ctx),
+        # the backward partial step is two kernels that each recompute S and dP:
+        # dK/dV kernel S, dP, dV, dK = 8d per allowed pair; dQ kernel S, dP, dQ = 6d
+        "bwd_dkdv": ("tensor", 8.0 * d * ctx),
+        "bwd_dq": ("tensor", 6.0 * d * ctx),
         # partial records (O_c, m, l) read; o, lse written; q, kb, vb read once
         "merge": ("hbm", rec_rows * (4.0 * d + 8) + Nq * Hq * (4.0 * d + 4) + Nq * Hq * d * 2.0
                   + 2.0 * Nq * Hkv * d * 2),
@@ -211,7 +214,7 @@ def run_ours(args, world, rank, local):
     g = {"dq": torch.empty(t["q"].shape, **f32), "dk": torch.empty(t["k"].shape, **f32),
          "dv": torch.empty(t["v"].shape, **f32), "dkb": torch.empty(t["kb"].shape, **f32),
          "dvb": torch.empty(t["vb"].shape, **f32)}
-    kernels = ["fwd_partial", "merge", "bwd_delta", "bwd_partial", "bwd_reduce"]
+    kernels = ["fwd_partial", "merge", "bwd_delta", "bwd_dkdv", "bwd_dq", "bwd_reduce"]
     plan_us = []
 
     def step(ev=None):
@@ -229,14 +232,16 @@ def run_ours(args, world, rank, local):
         skv.splitkv_bwd_delta(plan, o, t["dout"], ws_b, stream)
         if ev is not None:
             ev[3].record(stream)
-        skv.splitkv_bwd_partial(plan, t["q"], t["k"], t["v"], lse, t["dout"], g["dk"], g["dv"], w.scale, ws_b,
-                                stream)
+        skv.splitkv_bwd_dkdv(plan, t["q"], t["k"], t["v"], lse, t["dout"], g["dk"], g["dv"], w.scale, ws_b, stream)
         if ev is not None:
             ev[4].record(stream)
+        skv.splitkv_bwd_dq(plan, t["q"], t["k"], t["v"], lse, t["dout"], w.scale, ws_b, stream)
+        if ev is not None:
+            ev[5].record(stream)
         skv.splitkv_bwd_reduce(plan, t["q"], t["kb"], t["vb"], lse, t["dout"], g["dq"], g["dkb"], g["dvb"],
                                w.scale, ws_b, stream)
         if ev is not None:
-            ev[5].record(stream)
+            ev[6].record(stream)
 
     for _ in range(args.warmup):
         step()
@@ -249,7 +254,7 @@ def run_ours(args, world, rank, local):
         sampler.start()
         time.sleep(0.3)
 
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(args.steps)]
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(len(kernels) + 1)] for _ in range(args.steps)]
     start = torch.cuda.Event(enable_timing=True)
     end = torch.cuda.Event(enable_timing=True)
     plan_us.clear()
@@ -291,7 +296,8 @@ def run_ours(args, world, rank, local):
     dom = max(kernels, key=lambda k: per_kernel[k])
     bound, amount = work[dom]
     dom_s = per_kernel[dom] * 1e-3
-    src_file = {"fwd_partial": "fwd_partial_mma.cu", "bwd_partial": "bwd_partial_mma.cu"}.get(dom, "merge.cu")
+    src_file = {"fwd_partial": "fwd_partial_sm100.cu", "bwd_dkdv": "bwd_partial_sm100.cu",
+                "bwd_dq": "bwd_partial_sm100.cu"}.get(dom, "merge.cu")
     tr = NCU_TRAFFIC.get(dom)
     traffic = tr["bytes"] if tr and tr.get("src") == _src_hash(src_file) else None
     if bound == "tensor":
@@ -307,11 +313,11 @@ def run_ours(args, world, rank, local):
     kern = {}
     for k in kernels:
         b_, a_ = work[k]
-        s_ = per_kernel[k] * 1e-3
+        s_ = max(per_kernel[k] * 1e-3, 1e-9)
         kern[k] = {"ms": per_kernel[k],
                    ("tflops" if b_ == "tensor" else "gbs"): (a_ / s_ / 1e12 if b_ == "tensor" else a_ / s_ / 1e9)}
     fwd_ms = per_kernel["fwd_partial"] + per_kernel["merge"]
-    bwd_ms = per_kernel["bwd_delta"] + per_kernel["bwd_partial"] + per_kernel["bwd_reduce"]
+    bwd_ms = sum(per_kernel[k] for k in ("bwd_delta", "bwd_dkdv", "bwd_dq", "bwd_reduce"))
 
     result = {
         "metric": METRIC,
@@ -340,9 +346,10 @@ def run_ours(args, world, rank, local):
         "plan_us": float(np.median(plan_us)) if plan_us else None,
         "kernels": kern,
         "roofline": roof,
-        # the backward partial step is two launches (dK/dV kernel + dQ kernel) on the tcgen05
-        # path (head_dim 128, G * bs a multiple of 8), one on the mma.sync path
-        "gpu_launches": (len(kernels) + (1 if _bwd_is_two_launches(w) else 0)) * args.steps,
+        # the dQ kernel is a separate launch on the tcgen05 path (head_dim 128, G * bs a
+        # multiple of 8); on the mma.sync path the dK/dV launch also writes dQ and the
+        # dQ call launches nothing
+        "gpu_launches": (len(kernels) - (0 if _bwd_is_two_launches(w) else 1)) * args.steps,
         "clocks": clocks,
     }
 

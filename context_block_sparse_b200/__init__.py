@@ -236,6 +236,18 @@ def splitkv_bwd_partial(plan: Plan, q, k, v, lse, dout, dk, dv, scale: float, ws
         _f32_ptr(dv), float(scale), _ptr(ws), ws.numel() * ws.element_size(), _stream_ptr(stream)))
 
 
+def splitkv_bwd_dkdv(plan: Plan, q, k, v, lse, dout, dk, dv, scale: float, ws, stream=None) -> None:
+    _check("splitkv_bwd_dkdv", _lib.splitkv_bwd_dkdv(
+        plan.handle, _bf16_ptr(q), _bf16_ptr(k), _bf16_ptr(v), _f32_ptr(lse), _bf16_ptr(dout), _f32_ptr(dk),
+        _f32_ptr(dv), float(scale), _ptr(ws), ws.numel() * ws.element_size(), _stream_ptr(stream)))
+
+
+def splitkv_bwd_dq(plan: Plan, q, k, v, lse, dout, scale: float, ws, stream=None) -> None:
+    _check("splitkv_bwd_dq", _lib.splitkv_bwd_dq(
+        plan.handle, _bf16_ptr(q), _bf16_ptr(k), _bf16_ptr(v), _f32_ptr(lse), _bf16_ptr(dout), float(scale),
+        _ptr(ws), ws.numel() * ws.element_size(), _stream_ptr(stream)))
+
+
 def splitkv_bwd_reduce(plan: Plan, q, kb, vb, lse, dout, dq, dkb, dvb, scale: float, ws, stream=None) -> None:
     _check("splitkv_bwd_reduce", _lib.splitkv_bwd_reduce(
         plan.handle, _bf16_ptr(q), _bf16_ptr(kb), _bf16_ptr(vb), _f32_ptr(lse), _bf16_ptr(dout), _f32_ptr(dq),

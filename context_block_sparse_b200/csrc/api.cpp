@@ -89,20 +89,40 @@ int splitkv_bwd_delta(const splitkv_plan_t* plan, const void* o, int o_dtype, co
                                                static_cast<cudaStream_t>(stream)));
 }
 
-int splitkv_bwd_partial(const splitkv_plan_t* plan, const void* q, const void* k, const void* v, const float* lse,
-                        const void* dout, float* dk, float* dv, float scale, void* ws, size_t ws_bytes,
-                        void* stream) {
+namespace {
+int bwd_partial_part(const splitkv_plan_t* plan, const void* q, const void* k, const void* v, const float* lse,
+                     const void* dout, float* dk, float* dv, float scale, void* ws, size_t ws_bytes, void* stream,
+                     int which) {
   const DevPlan* dp = nullptr;
   int st = check_plan(plan, &dp);
   if (st != SPLITKV_OK) return st;
-  if (!all_aligned16(q, k, v, dout, dk, dv, ws) || !lse || !aligned(lse, 4)) return SPLITKV_ERR_INVALID_ARG;
+  if (!all_aligned16(q, k, v, dout, ws) || !lse || !aligned(lse, 4)) return SPLITKV_ERR_INVALID_ARG;
+  if (which != 2 && !all_aligned16(dk, dv)) return SPLITKV_ERR_INVALID_ARG;
   const splitkv::BwdWs L = splitkv::bwd_ws_layout(dp->E, dp->Nq, dp->bs, dp->Hq, dp->d);
   if (ws_bytes < L.total) return SPLITKV_ERR_WORKSPACE_TOO_SMALL;
   char* w = static_cast<char*>(ws);
   return cuda_status(splitkv::launch_bwd_partial(
       *dp, static_cast<const uint16_t*>(q), static_cast<const uint16_t*>(k), static_cast<const uint16_t*>(v),
       static_cast<const uint16_t*>(dout), lse, reinterpret_cast<const float*>(w + L.delta_off), scale, dk, dv,
-      reinterpret_cast<float*>(w + L.dq_off), static_cast<cudaStream_t>(stream)));
+      reinterpret_cast<float*>(w + L.dq_off), static_cast<cudaStream_t>(stream), which));
+}
+}  // namespace
+
+int splitkv_bwd_partial(const splitkv_plan_t* plan, const void* q, const void* k, const void* v, const float* lse,
+                        const void* dout, float* dk, float* dv, float scale, void* ws, size_t ws_bytes,
+                        void* stream) {
+  return bwd_partial_part(plan, q, k, v, lse, dout, dk, dv, scale, ws, ws_bytes, stream, 0);
+}
+
+int splitkv_bwd_dkdv(const splitkv_plan_t* plan, const void* q, const void* k, const void* v, const float* lse,
+                     const void* dout, float* dk, float* dv, float scale, void* ws, size_t ws_bytes,
+                     void* stream) {
+  return bwd_partial_part(plan, q, k, v, lse, dout, dk, dv, scale, ws, ws_bytes, stream, 1);
+}
+
+int splitkv_bwd_dq(const splitkv_plan_t* plan, const void* q, const void* k, const void* v, const float* lse,
+                   const void* dout, float scale, void* ws, size_t ws_bytes, void* stream) {
+  return bwd_partial_part(plan, q, k, v, lse, dout, nullptr, nullptr, scale, ws, ws_bytes, stream, 2);
 }
 
 int splitkv_bwd_reduce(const splitkv_plan_t* plan, const void* q, const void* kb, const void* vb, const float* lse,

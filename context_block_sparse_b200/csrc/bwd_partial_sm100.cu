@@ -147,7 +147,8 @@ __device__ __forceinline__ void ds_tile(uint32_t tS, uint32_t tdP, int hf, int a
       const int col = q * 32 + 2 * i;
       float x0, x1, d0, d1, g0, g1;
       ffma2(x0, x1, __uint_as_float(sv[2 * i]), __uint_as_float(sv[2 * i + 1]), c, c, -l2, -l2);
-      float p0 = fast_exp2(x0), p1 = fast_exp2(x1);
+      float p0, p1;
+      exp2_pair((i % kPolyEvery) == 1, x0, x1, p0, p1);
       if (kMasked) {
         p0 = (col >= a && col < b) ? p0 : 0.f;
         p1 = (col + 1 >= a && col + 1 < b) ? p1 : 0.f;
@@ -180,7 +181,8 @@ __device__ __forceinline__ void pds_tile(uint32_t tSt, uint32_t tdPt, int hf, ui
       const float4 m = ld4[row >> 1];    // lse2[row], delta[row], lse2[row + 1], delta[row + 1]
       float x0, x1, d0, d1, g0, g1;
       ffma2(x0, x1, __uint_as_float(sv[2 * i]), __uint_as_float(sv[2 * i + 1]), c, c, -m.x, -m.z);
-      float p0 = fast_exp2(x0), p1 = fast_exp2(x1);
+      float p0, p1;
+      exp2_pair((i % kPolyEvery) == 1, x0, x1, p0, p1);
       if (kMasked) {   // rows row and row + 1 share a slot (slots hold >= 8 rows)
         const bool in = (smask >> (row >> lg)) & 1u;
         p0 = in ? p0 : 0.f;
@@ -733,7 +735,7 @@ bool bwd_sm100_supported(const DevPlan& p) {
 
 cudaError_t launch_bwd_partial_sm100(const DevPlan& p, const uint16_t* q, const uint16_t* k, const uint16_t* v,
                                      const uint16_t* dout, const float* lse, const float* delta, float scale,
-                                     float* dk, float* dv, float* dq_part, cudaStream_t s) {
+                                     float* dk, float* dv, float* dq_part, cudaStream_t s, int which) {
   CUtensorMap tq, tdo, tk, tv;
   if (!make_bf16_map_3d(&tq, q, D, p.Hq, p.Nq, p.G, p.bs) || !make_bf16_map_3d(&tdo, dout, D, p.Hq, p.Nq, p.G, p.bs) ||
       !make_bf16_map_3d(&tk, k, D, p.Hkv, p.N, 1, BT) || !make_bf16_map_3d(&tv, v, D, p.Hkv, p.N, 1, BT))
@@ -743,11 +745,16 @@ cudaError_t launch_bwd_partial_sm100(const DevPlan& p, const uint16_t* q, const 
   if (e != cudaSuccess) return e;
   e = cudaFuncSetAttribute(bwd_dq_sm100_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(kSmemBytes));
   if (e != cudaSuccess) return e;
-  bwd_dkdv_sm100_kernel<<<p.Wb, kThreads, kSmemBytes, s>>>(tq, tdo, tk, tv, p, lse, delta, scale, dk, dv);
-  e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
-  bwd_dq_sm100_kernel<<<p.W, kThreads, kSmemBytes, s>>>(tq, tdo, tk, tv, p, lse, delta, scale, dq_part);
-  return cudaGetLastError();
+  if (which != 2) {
+    bwd_dkdv_sm100_kernel<<<p.Wb, kThreads, kSmemBytes, s>>>(tq, tdo, tk, tv, p, lse, delta, scale, dk, dv);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  if (which != 1) {
+    bwd_dq_sm100_kernel<<<p.W, kThreads, kSmemBytes, s>>>(tq, tdo, tk, tv, p, lse, delta, scale, dq_part);
+    e = cudaGetLastError();
+  }
+  return e;
 }
 
 }  // namespace splitkv

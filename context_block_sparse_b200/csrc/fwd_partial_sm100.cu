@@ -140,7 +140,8 @@ __device__ __forceinline__ float exp_pack_store(const uint32_t (&v)[64], int a, 
       const int col = cch * 32 + 2 * i;
       float x0, x1;
       ffma2(x0, x1, __uint_as_float(v[col]), __uint_as_float(v[col + 1]), c, c, nm, nm);
-      float p0 = fast_exp2(x0), p1 = fast_exp2(x1);
+      float p0, p1;
+      exp2_pair((i % kPolyEvery) == 1, x0, x1, p0, p1);
       if (kMasked) {
         p0 = (col >= a && col < b) ? p0 : 0.f;
         p1 = (col + 1 >= a && col + 1 < b) ? p1 : 0.f;

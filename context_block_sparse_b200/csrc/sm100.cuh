@@ -104,6 +104,43 @@ __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, u
       "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y), "r"(z)
       : "memory");
 }
+// Bulk tensor store shared -> global (bulk-group completion) and its waits.
+__device__ __forceinline__ void tma_store_3d(const CUtensorMap* map, const void* src, int x, int y, int z) {
+  asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%2, %3, %4}], [%1];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(smem_u32(src)), "r"(x), "r"(y), "r"(z)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_read0() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait0() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+__device__ __forceinline__ void fence_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// One warp's 32 rows x 32 fp32 columns through a 4 KB shared chunk laid out as a
+// 128-byte-swizzled box (row = lane), then one bulk tensor store at (x, y, z) of
+// `map`.  Lane 0 owns the bulk group; the chunk may be rewritten once
+// bulk_wait_read0 has returned (done here before the writes).
+__device__ __forceinline__ void warp_bulk_store_rows32(float* chunk, const float* vals, float mul,
+                                                       const CUtensorMap* map, int x, int y, int z, bool store) {
+  const int lane = threadIdx.x & 31;
+  if (lane == 0) bulk_wait_read0();   // the previous store from this chunk has read it
+  __syncwarp();
+#pragma unroll
+  for (int g = 0; g < 8; ++g) {
+    const float4 v = make_float4(vals[4 * g] * mul, vals[4 * g + 1] * mul, vals[4 * g + 2] * mul,
+                                 vals[4 * g + 3] * mul);
+    *reinterpret_cast<float4*>(chunk + lane * 32 + ((g ^ (lane & 7)) << 2)) = v;
+  }
+  fence_async_smem();
+  __syncwarp();
+  if (lane == 0 && store) {
+    tma_store_3d(map, chunk, x, y, z);
+    bulk_commit();
+  }
+}
+
 __device__ __forceinline__ void prefetch_tmap(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
@@ -270,6 +307,45 @@ __device__ __forceinline__ void fmul2(float& d0, float& d1, float a0, float a1, 
 
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+// ---------------------------------------------------------------- exp2 on the FMA pipe
+// 2^x for two lanes without the MUFU unit (which computes only 16 exp2 per
+// clock per SM): Cody-Waite range reduction x = n + f, n = round(x) (by adding
+// and subtracting 1.5 * 2^23), f in [-0.5, 0.5], a cubic fitted here to 2^f on
+// that interval (weighted least squares on the relative error, max relative
+// error 7.6e-5 in fp32, far below bf16's 3.9e-3), and the exponent n added
+// to the result's bits.  x is clamped at -126 (the result is then below 2^-125,
+// i.e. zero for bf16 P and negligible in fp32 sums).
+constexpr float kExpMagic = 12582912.0f;   // 1.5 * 2^23
+constexpr float kExpC0 = 0.99992758f, kExpC1 = 0.69326109f, kExpC2 = 0.24261758f, kExpC3 = 0.055174146f;
+
+__device__ __forceinline__ void exp2_poly2(float x0, float x1, float& y0, float& y1) {
+  x0 = fmaxf(x0, -126.f);
+  x1 = fmaxf(x1, -126.f);
+  float t0, t1, n0, n1, f0, f1, p0, p1;
+  fadd2(t0, t1, x0, x1, kExpMagic, kExpMagic);     // round(x) in the low mantissa bits
+  fadd2(n0, n1, t0, t1, -kExpMagic, -kExpMagic);   // round(x) as a float
+  fadd2(f0, f1, x0, x1, -n0, -n1);                 // f = x - n
+  ffma2(p0, p1, f0, f1, kExpC3, kExpC3, kExpC2, kExpC2);
+  ffma2(p0, p1, p0, p1, f0, f1, kExpC1, kExpC1);
+  ffma2(p0, p1, p0, p1, f0, f1, kExpC0, kExpC0);
+  y0 = __uint_as_float(__float_as_uint(p0) + (__float_as_uint(t0) << 23));
+  y1 = __uint_as_float(__float_as_uint(p1) + (__float_as_uint(t1) << 23));
+}
+
+// exp2 of two lanes on MUFU (poly = false) or on the FMA pipe (poly = true);
+// callers pass a condition on an unrolled loop index, so the branch folds away.
+__device__ __forceinline__ void exp2_pair(bool poly, float x0, float x1, float& y0, float& y1) {
+  if (poly) {
+    exp2_poly2(x0, x1, y0, y1);
+  } else {
+    y0 = fast_exp2(x0);
+    y1 = fast_exp2(x1);
+  }
+}
+
+// One pair in kPolyEvery goes through the polynomial (keeps MUFU and FMA busy).
+constexpr int kPolyEvery = 4;
 
 // ---------------------------------------------------------------- epilogue stores
 // Lane i of a warp holds W consecutive fp32 values of its own output row

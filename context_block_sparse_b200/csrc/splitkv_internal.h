@@ -67,6 +67,10 @@ inline BwdWs bwd_ws_layout(long long E, int Nq, int bs, int Hq, int d) {
 bool tensor_maps_available();
 bool make_bf16_map_3d(void* map, const void* base, uint64_t dim0, uint64_t dim1, uint64_t dim2, uint32_t box1,
                       uint32_t box2);
+// 3-D fp32 tensor [dim2][dim1][dim0], box {box0, box1, box2} with box0 * 4 =
+// 128 bytes, 128-byte swizzle (used for bulk stores of epilogue chunks).
+bool make_f32_map_3d(void* map, void* base, uint64_t dim0, uint64_t dim1, uint64_t dim2, uint32_t box0,
+                     uint32_t box1, uint32_t box2);
 
 // ---- kernel launchers (defined in the .cu files) ---------------------------
 cudaError_t launch_fwd_partial(const DevPlan& p, const uint16_t* q, const uint16_t* k,
@@ -81,10 +85,12 @@ cudaError_t launch_merge(const DevPlan& p, const uint16_t* q, const uint16_t* kb
 cudaError_t launch_bwd_delta(const DevPlan& p, const void* o, int o_bf16, const uint16_t* dout,
                              float* delta, cudaStream_t s);
 
+// which: 0 = both parts, 1 = the dK/dV part (everything on the mma.sync path),
+// 2 = the dQ part (nothing on the mma.sync path).
 cudaError_t launch_bwd_partial(const DevPlan& p, const uint16_t* q, const uint16_t* k,
                                const uint16_t* v, const uint16_t* dout, const float* lse,
                                const float* delta, float scale, float* dk, float* dv,
-                               float* dq_part, cudaStream_t s);
+                               float* dq_part, cudaStream_t s, int which = 0);
 
 cudaError_t launch_bwd_reduce(const DevPlan& p, const uint16_t* q, const uint16_t* kb,
                               const uint16_t* vb, const uint16_t* dout, const float* lse,

@@ -244,6 +244,19 @@ int splitkv_bwd_reduce(const splitkv_plan_t* plan, const void* q, const void* kb
                        const float* lse, const void* dout, float* dq, float* dkb, float* dvb,
                        float scale, const void* ws, size_t ws_bytes, void* stream);
 
+/* splitkv_bwd_partial is itself two launches on the tcgen05 path (head_dim
+ * 128, G * bs a multiple of 8), exposed for timing: splitkv_bwd_dkdv (the
+ * KV-stationary kernel: dk, dv) followed by splitkv_bwd_dq (the Q-stationary
+ * kernel: the dq partials).  On other shapes one kernel produces all three and
+ * runs in splitkv_bwd_dkdv; splitkv_bwd_dq then launches nothing.  Same
+ * arguments and errors as splitkv_bwd_partial. */
+int splitkv_bwd_dkdv(const splitkv_plan_t* plan, const void* q, const void* k, const void* v,
+                     const float* lse, const void* dout, float* dk, float* dv, float scale,
+                     void* ws, size_t ws_bytes, void* stream);
+int splitkv_bwd_dq(const splitkv_plan_t* plan, const void* q, const void* k, const void* v,
+                   const float* lse, const void* dout, float scale, void* ws, size_t ws_bytes,
+                   void* stream);
+
 /* Size of the library's static device scratch buffer (16 MiB): see
  * splitkv_attn_fwd_static_scratch. */
 #define SPLITKV_STATIC_SCRATCH_BYTES (16u << 20)
@@ -278,6 +291,13 @@ int splitkv_attn_fwd_static_scratch(const splitkv_plan_t* plan, const void* q, c
  * If `site` is not NULL it receives the source site of the first wait that
  * timed out (0 if none).  Errors: INVALID_ARG, NOT_UPLOADED, CUDA. */
 int splitkv_plan_status(const splitkv_plan_t* plan, void* stream, int32_t* site);
+
+/* Self-test of the FMA-pipe exp2 the attention kernels use for part of their
+ * exponentials (Cody-Waite range reduction and a fitted cubic): y[i] = 2^x[i]
+ * for n device floats, asynchronously on `stream`.  Not part of the method;
+ * it lets a test compare the approximation with CUDA's exp2f.
+ * Errors: INVALID_ARG, CUDA. */
+int splitkv_selftest_exp2(const float* x, float* y, int64_t n, void* stream);
 
 /* Per-CTA busy time of the last splitkv_attn_fwd (which = SPLITKV_WS_FWD) or
  * backward partial kernel (SPLITKV_WS_BWD) on this plan: out_ns[w] = end - start
