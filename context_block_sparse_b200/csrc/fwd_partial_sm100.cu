@@ -17,16 +17,22 @@
 //   warp 2      tensor-memory allocation (512 columns: S_A, S_B, O_A, O_B);
 //   warps 4-7   softmax / epilogue of tile A (thread = row = TMEM lane);
 //   warps 8-11  softmax / epilogue of tile B.
-// The softmax keeps, per row, a reference maximum m_ref and rescales O in TMEM
-// only when a new key tile raises the maximum by more than 2^8 (the result is
-// the same; the reference is exact bookkeeping).  The record written is
-// m_c = the row's true maximum (natural units), l_c = sum exp(s - m_c) and
-// O_c = sum exp(s - m_c) v / l_c.  Rows are masked to their block's [lo, hi).
+// The softmax keeps, per row, a reference maximum m_ref, taken from the first
+// key tile in which the row has allowed keys (the only tile that reads S from
+// TMEM twice); later tiles exponentiate against it in one pass and only when a
+// score exceeds m_ref by more than 2^32 (in P) are O, l and the P already
+// written rescaled to a new reference -- the result is the same, the reference
+// is exact bookkeeping.  The record written is m_c = the row's true maximum
+// (natural units), l_c = sum exp(s - m_c) and O_c = sum exp(s - m_c) v / l_c.
+// Rows are masked to their block's [lo, hi).  When a warp's 32 rows are whole
+// tokens of one block (G * bs a multiple of 32), O_c leaves through bulk tensor
+// stores of 32-row x 16-column boxes staged in two 2 KB buffers per warp.
 //
 // Every mbarrier wait is bounded; on a timeout the kernel records
 // SPLITKV_ERR_TIMEOUT in the plan's status word, lets every role wind down,
 // waits for its own copies in flight and frees its tensor memory.
 #include <cfloat>
+#include <cstring>
 
 #include "sm100.cuh"
 #include "splitkv.h"
@@ -46,13 +52,16 @@ constexpr uint32_t kHalf = 128 * 128; // bytes of one 64-column half of a 128-ro
 constexpr uint32_t kTile = 2 * kHalf; // 32 KB: a 128 x 128 bf16 tile
 constexpr uint32_t kIdescQK = idesc_bf16_f32(128, 128, 0);
 constexpr uint32_t kIdescPV = idesc_bf16_f32(128, D, 1);
-constexpr float kRescaleLog2 = 8.0f;  // rescale O only when the max grows by more than 2^8
+// A row's reference maximum stays while P = exp2(s - m_ref) <= 2^kHeadroomLog2;
+// P (bf16), l and O (fp32) hold such values exactly as well as near 1, and
+// O = sum P v stays far inside the fp32 range.
+constexpr float kHeadroomLog2 = 32.0f;
 
 // shared-memory map (offsets from a 1024-aligned base)
 constexpr uint32_t kOffQ = 0;                              // Q_A, Q_B
 constexpr uint32_t kOffK = kOffQ + 2 * kTile;              // K stages
 constexpr uint32_t kOffV = kOffK + kStages * kTile;        // V stages
-constexpr uint32_t kOffScratch = kOffV + kStages * kTile; // epilogue scratch, 4 KB per softmax warp
+constexpr uint32_t kOffScratch = kOffV + kStages * kTile; // epilogue buffers, 4 KB per softmax warp
 constexpr uint32_t kOffBar = kOffScratch + 8 * 4096;       // mbarriers
 constexpr uint32_t kSmemBytes = kOffBar + 256 + 1024;      // + alignment slack
 static_assert(kSmemBytes <= 232448, "shared memory per block");
@@ -105,23 +114,21 @@ struct PairIter {
 };
 
 
-// Maximum of 64 raw scores of one row over its allowed columns [a, b) of them.
+// Maximum of 64 raw scores of one row over its allowed columns [a, b) of them
+// (-inf when none is allowed).
 template <bool kMasked>
 __device__ __forceinline__ float row_max(const uint32_t (&v)[64], int a, int b) {
   float m0 = -INFINITY, m1 = -INFINITY, m2 = -INFINITY, m3 = -INFINITY;
 #pragma unroll
-  for (int i = 0; i < 64; i += 4) {
-    if (kMasked) {
-      m0 = (i >= a && i < b) ? fmaxf(m0, __uint_as_float(v[i])) : m0;
-      m1 = (i + 1 >= a && i + 1 < b) ? fmaxf(m1, __uint_as_float(v[i + 1])) : m1;
-      m2 = (i + 2 >= a && i + 2 < b) ? fmaxf(m2, __uint_as_float(v[i + 2])) : m2;
-      m3 = (i + 3 >= a && i + 3 < b) ? fmaxf(m3, __uint_as_float(v[i + 3])) : m3;
-    } else {
-      m0 = fmaxf(m0, __uint_as_float(v[i]));
-      m1 = fmaxf(m1, __uint_as_float(v[i + 1]));
-      m2 = fmaxf(m2, __uint_as_float(v[i + 2]));
-      m3 = fmaxf(m3, __uint_as_float(v[i + 3]));
-    }
+  for (int i = 0; i < 64; i += 8) {
+    float u[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k)
+      u[k] = (!kMasked || (i + k >= a && i + k < b)) ? __uint_as_float(v[i + k]) : -INFINITY;
+    m0 = fmax3(m0, u[0], u[1]);
+    m1 = fmax3(m1, u[2], u[3]);
+    m2 = fmax3(m2, u[4], u[5]);
+    m3 = fmax3(m3, u[6], u[7]);
   }
   return fmaxf(fmaxf(m0, m1), fmaxf(m2, m3));
 }
@@ -156,9 +163,9 @@ __device__ __forceinline__ float exp_pack_store(const uint32_t (&v)[64], int a, 
 
 __global__ void __launch_bounds__(kThreads, 1)
     fwd_partial_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                             const __grid_constant__ CUtensorMap tm_v, DevPlan p, float scale_log2,
-                             float* __restrict__ part_o, float* __restrict__ part_m,
-                             float* __restrict__ part_l) {
+                             const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
+                             DevPlan p, float scale_log2, int bulk_o, float* __restrict__ part_o,
+                             float* __restrict__ part_m, float* __restrict__ part_l) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   Bars* bars = reinterpret_cast<Bars*>(smem + kOffBar);
@@ -367,7 +374,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         rec = (e * p.bs + tt) * p.Hq + g * p.G + hh;
       }
       float m_ref = -INFINITY, m_true = -INFINITY, l = 0.f;
-      for (int j = 0; j < n_kt; ++j) {
+      for (int j = 0; j < n_kt && ok; ++j) {
         if (!warp_wait(&bars->s_ready[x], s_cnt & 1, wctx, 1 * 10000 + __LINE__)) { ok = false; break; }
         ++s_cnt;
         tc_fence_after();
@@ -377,54 +384,82 @@ __global__ void __launch_bounds__(kThreads, 1)
         const bool none = b <= 0 || a >= BN;
         // warp-uniform: the two exp_pack_store variants issue warp-collective tcgen05.st
         const bool full = __all_sync(0xffffffffu, a <= 0 && b >= BN);
-        // pass 1: maximum of the raw scores, 64 columns per TMEM round trip
-        float mxr = -INFINITY;
-        if (__any_sync(0xffffffffu, !none)) {
+        // first allowed keys of a row: its reference is this tile's maximum (O and
+        // l of the row are still zero, nothing to rescale)
+        if (__any_sync(0xffffffffu, m_ref == -INFINITY && !none)) {
+          float mxr = -INFINITY;
 #pragma unroll 1
           for (int h = 0; h < BN / 64; ++h) {
             uint32_t v[64];
             tmem_ld32p(tS + h * 64, v);
             tmem_ld32p(tS + h * 64 + 32, v + 32);
             tmem_wait_ld();
-            const float mh = full ? row_max<false>(v, a - h * 64, b - h * 64) : row_max<true>(v, a - h * 64, b - h * 64);
-            mxr = fmaxf(mxr, mh);
+            reg_fence<64>(v);
+            mxr = fmaxf(mxr, full ? row_max<false>(v, a - h * 64, b - h * 64)
+                                  : row_max<true>(v, a - h * 64, b - h * 64));
           }
+          if (m_ref == -INFINITY && !none) m_ref = mxr * scale_log2;
         }
-        const float mx = none ? -INFINITY : mxr * scale_log2;
-        m_true = fmaxf(m_true, mx);
-        // rescale decision (warp-uniform for the TMEM traffic)
-        const bool need = (mx > m_ref + kRescaleLog2) || (m_ref == -INFINITY && mx > -INFINITY);
-        const bool rescale_o = need && m_ref > -INFINITY;      // only after a previous tile added to O
-        if (__any_sync(0xffffffffu, rescale_o)) {
-          // PV(j-1) must have completed before O is touched
-          if (!warp_wait(&bars->o_ready[x], (o_cnt + j - 1) & 1, wctx, 1 * 10000 + __LINE__)) { ok = false; break; }
-          tc_fence_after();
-          const float f = rescale_o ? fast_exp2(m_ref - mx) : 1.f;
-#pragma unroll 1
-          for (int cch = 0; cch < D / 16; ++cch) {
-            uint32_t o[16];
-            tmem_ld16(tO + cch * 16, o);
-            tmem_wait_ld();
-#pragma unroll
-            for (int i = 0; i < 16; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * f);
-            tmem_st16(tO + cch * 16, o);
-          }
-          tmem_wait_st();
-          l *= f;
-        }
-        if (need) m_ref = mx;
-        const float m_use = (m_ref == -INFINITY) ? 0.f : m_ref;
-        // pass 2: P = exp2(s * scale_log2 - m_ref) (masked -> 0), row sum, bf16 P into
-        // TMEM columns 0..63 of S_X (half h -> columns 32h..32h+31, already read)
+        // one pass per 64-column half: maximum, P = exp2(s * scale_log2 - m_ref)
+        // (masked -> 0), row sum, bf16 P into TMEM columns 32h..32h+31 of S_X
+        // (columns already read)
+        float mx = -INFINITY;
 #pragma unroll 1
         for (int h = 0; h < BN / 64; ++h) {
           uint32_t v[64];
           tmem_ld32p(tS + h * 64, v);
           tmem_ld32p(tS + h * 64 + 32, v + 32);
           tmem_wait_ld();
+          reg_fence<64>(v);
+          const float mh = scale_log2 * (full ? row_max<false>(v, a - h * 64, b - h * 64)
+                                              : row_max<true>(v, a - h * 64, b - h * 64));
+          mx = fmaxf(mx, mh);
+          const bool over = mh > m_ref + kHeadroomLog2;
+          if (__any_sync(0xffffffffu, over)) {
+            // new reference for the rows past the headroom: rescale O (after PV(j-1)),
+            // the P of half 0 already in TMEM, and l
+            const float f = over ? fast_exp2(m_ref - mh) : 1.f;
+            if (j > 0) {
+              if (!warp_wait(&bars->o_ready[x], (o_cnt + j - 1) & 1, wctx, 1 * 10000 + __LINE__)) {
+                ok = false;
+                break;
+              }
+              tc_fence_after();
+#pragma unroll 1
+              for (int cch = 0; cch < D / 16; ++cch) {
+                uint32_t o[16];
+                tmem_ld16(tO + cch * 16, o);
+                tmem_wait_ld();
+                reg_fence<16>(o);
+#pragma unroll
+                for (int i = 0; i < 16; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * f);
+                tmem_st16(tO + cch * 16, o);
+              }
+            }
+            if (h > 0) {
+              tmem_wait_st();
+#pragma unroll 1
+              for (int cch = 0; cch < 2; ++cch) {
+                uint32_t pk[16];
+                tmem_ld16(tS + cch * 16, pk);
+                tmem_wait_ld();
+                reg_fence<16>(pk);
+#pragma unroll
+                for (int i = 0; i < 16; ++i)
+                  pk[i] = pack_bf16(__uint_as_float(pk[i] << 16) * f, __uint_as_float(pk[i] & 0xffff0000u) * f);
+                tmem_st16(tS + cch * 16, pk);
+              }
+            }
+            tmem_wait_st();
+            l *= f;
+            if (over) m_ref = mh;
+          }
+          const float m_use = (m_ref == -INFINITY) ? 0.f : m_ref;
           l += full ? exp_pack_store<false>(v, a - h * 64, b - h * 64, scale_log2, -m_use, tS + h * 32)
                     : exp_pack_store<true>(v, a - h * 64, b - h * 64, scale_log2, -m_use, tS + h * 32);
         }
+        if (!ok) break;
+        m_true = fmaxf(m_true, none ? -INFINITY : mx);
         tmem_wait_st();
         tc_fence_before();
         mbar_arrive(&bars->p_ready[x]);
@@ -436,22 +471,52 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       const float inv = l > 0.f ? 1.f / l : 0.f;
       float* scratch = reinterpret_cast<float*>(smem + kOffScratch) + (warp - 4) * 1024;
+      if (bulk_o) {
+        // the warp's rows: tokens tt0 .. tt0 + 32/G - 1 of one block, all G heads
+        // (valid is warp-uniform here: a slot holds whole warps)
+        const int z0 = __shfl_sync(0xffffffffu, valid ? rec / p.Hq : 0, 0);
+        if (valid) {
+          uint32_t va[32], vb[32];
+          tmem_ld32(tO, va);
+          tmem_wait_ld();
+          reg_fence<32>(va);
+#pragma unroll
+          for (int cch = 0; cch < D / 32; cch += 2) {
+            tmem_ld32(tO + (cch + 1) * 32, vb);
+            warp_bulk_store16(scratch, va, inv, &tm_o, cch * 32, g * p.G, z0);
+            warp_bulk_store16(scratch + 512, va + 16, inv, &tm_o, cch * 32 + 16, g * p.G, z0);
+            tmem_wait_ld();
+            reg_fence<32>(vb);
+            if (cch + 2 < D / 32) tmem_ld32(tO + (cch + 2) * 32, va);
+            warp_bulk_store16(scratch, vb, inv, &tm_o, (cch + 1) * 32, g * p.G, z0);
+            warp_bulk_store16(scratch + 512, vb + 16, inv, &tm_o, (cch + 1) * 32 + 16, g * p.G, z0);
+            tmem_wait_ld();
+            reg_fence<32>(va);
+          }
+        }
+      } else {
 #pragma unroll 1
-      for (int cch = 0; cch < D / 32; ++cch) {
-        uint32_t v[32];
-        tmem_ld32(tO + cch * 32, v);
-        tmem_wait_ld();
-        warp_store_rows<32>(scratch, reinterpret_cast<const float*>(v), inv,
-                            valid ? part_o + size_t(rec) * D + cch * 32 : nullptr);
+        for (int cch = 0; cch < D / 32; ++cch) {
+          uint32_t v[32];
+          tmem_ld32(tO + cch * 32, v);
+          tmem_wait_ld();
+          reg_fence<32>(v);
+          warp_store_rows<32>(scratch, reinterpret_cast<const float*>(v), inv,
+                              valid ? part_o + size_t(rec) * D + cch * 32 : nullptr);
+        }
       }
       if (valid) {
         // record (true max, sum relative to it)
         part_m[rec] = (l > 0.f) ? m_true * kLn2 : -INFINITY;
         part_l[rec] = (l > 0.f) ? l * fast_exp2(m_ref - m_true) : 0.f;
       }
+      __syncwarp();
       tc_fence_before();
       mbar_arrive(&bars->o_free[x]);
     }
+    // bulk stores of this warp complete before the CTA exits
+    if (lane == 0) bulk_wait0();
+    __syncwarp();
     if (!ok) *abort_flag = 1;
   }
 
@@ -471,15 +536,22 @@ bool fwd_sm100_supported(const DevPlan& p) {
 
 cudaError_t launch_fwd_partial_sm100(const DevPlan& p, const uint16_t* q, const uint16_t* k, const uint16_t* v,
                                      float scale, float* part_o, float* part_m, float* part_l, cudaStream_t s) {
-  CUtensorMap tq, tk, tv;
+  CUtensorMap tq, tk, tv, to;
   if (!make_bf16_map_3d(&tq, q, D, p.Hq, p.Nq, p.G, p.bs)) return cudaErrorInvalidValue;
+  // bulk record stores when a warp's 32 rows are 32/G whole tokens of one block
+  const bool bulk = 32 % p.G == 0 && (p.G * p.bs) % 32 == 0 && p.E > 0;
+  if (bulk) {
+    if (!make_f32_map_3d(&to, part_o, D, p.Hq, uint64_t(p.E) * p.bs, 16, p.G, 32 / p.G)) return cudaErrorInvalidValue;
+  } else {
+    memset(&to, 0, sizeof(to));
+  }
   if (!make_bf16_map_3d(&tk, k, D, p.Hkv, p.N, 1, BN)) return cudaErrorInvalidValue;
   if (!make_bf16_map_3d(&tv, v, D, p.Hkv, p.N, 1, BN)) return cudaErrorInvalidValue;
   cudaError_t e = cudaFuncSetAttribute(fwd_partial_sm100_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        int(kSmemBytes));
   if (e != cudaSuccess) return e;
-  fwd_partial_sm100_kernel<<<p.W, kThreads, kSmemBytes, s>>>(tq, tk, tv, p, scale * kLog2e, part_o, part_m,
-                                                             part_l);
+  fwd_partial_sm100_kernel<<<p.W, kThreads, kSmemBytes, s>>>(tq, tk, tv, to, p, scale * kLog2e, bulk ? 1 : 0,
+                                                             part_o, part_m, part_l);
   return cudaGetLastError();
 }
 

@@ -118,27 +118,36 @@ __device__ __forceinline__ void fence_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
-// One warp's 32 rows x 32 fp32 columns through a 4 KB shared chunk laid out as a
-// 128-byte-swizzled box (row = lane), then one bulk tensor store at (x, y, z) of
-// `map`.  Lane 0 owns the bulk group; the chunk may be rewritten once
-// bulk_wait_read0 has returned (done here before the writes).
-__device__ __forceinline__ void warp_bulk_store_rows32(float* chunk, const float* vals, float mul,
-                                                       const CUtensorMap* map, int x, int y, int z, bool store) {
+// One warp's 32 rows x 16 fp32 columns (vals[0..16) of the lane's row, times
+// mul) through a 2 KB shared buffer laid out as the 64-byte-swizzled box of
+// `map` (row = lane), then one bulk tensor store at (x, y, z).  A warp
+// alternates two such buffers: before a buffer is rewritten, the store issued
+// from it two calls earlier must have read it (wait_group.read 1; lane 0 owns
+// the bulk groups).  The buffer must be 512-byte aligned.
+__device__ __forceinline__ void warp_bulk_store16(float* buf, const uint32_t* vals, float mul,
+                                                  const CUtensorMap* map, int x, int y, int z) {
   const int lane = threadIdx.x & 31;
-  if (lane == 0) bulk_wait_read0();   // the previous store from this chunk has read it
+  if (lane == 0) asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
   __syncwarp();
 #pragma unroll
-  for (int g = 0; g < 8; ++g) {
-    const float4 v = make_float4(vals[4 * g] * mul, vals[4 * g + 1] * mul, vals[4 * g + 2] * mul,
-                                 vals[4 * g + 3] * mul);
-    *reinterpret_cast<float4*>(chunk + lane * 32 + ((g ^ (lane & 7)) << 2)) = v;
+  for (int g = 0; g < 4; ++g) {
+    const float4 v = make_float4(__uint_as_float(vals[4 * g]) * mul, __uint_as_float(vals[4 * g + 1]) * mul,
+                                 __uint_as_float(vals[4 * g + 2]) * mul, __uint_as_float(vals[4 * g + 3]) * mul);
+    *reinterpret_cast<float4*>(buf + lane * 16 + ((g ^ ((lane >> 1) & 3)) << 2)) = v;
   }
   fence_async_smem();
   __syncwarp();
-  if (lane == 0 && store) {
-    tma_store_3d(map, chunk, x, y, z);
+  if (lane == 0) {
+    tma_store_3d(map, buf, x, y, z);
     bulk_commit();
   }
+}
+
+// Three-input maximum (one instruction on sm_100).
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
 }
 
 __device__ __forceinline__ void prefetch_tmap(const CUtensorMap* map) {
@@ -230,6 +239,15 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
       : "r"(taddr)
       : "memory");
 }
+// tcgen05.ld writes its destination registers asynchronously: after
+// tmem_wait_ld, pass the loaded values through this empty asm so that the
+// compiler cannot move any use of them above the wait.
+template <int N>
+__device__ __forceinline__ void reg_fence(uint32_t* r) {
+#pragma unroll
+  for (int i = 0; i < N; ++i) asm volatile("" : "+r"(r[i]));
+}
+
 __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
   asm volatile(
       "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "

@@ -67,8 +67,9 @@ inline BwdWs bwd_ws_layout(long long E, int Nq, int bs, int Hq, int d) {
 bool tensor_maps_available();
 bool make_bf16_map_3d(void* map, const void* base, uint64_t dim0, uint64_t dim1, uint64_t dim2, uint32_t box1,
                       uint32_t box2);
-// 3-D fp32 tensor [dim2][dim1][dim0], box {box0, box1, box2} with box0 * 4 =
-// 128 bytes, 128-byte swizzle (used for bulk stores of epilogue chunks).
+// 3-D fp32 tensor [dim2][dim1][dim0], box {box0, box1, box2}; box0 * 4 is 64
+// or 128 bytes and selects the 64- or 128-byte swizzle (bulk stores of
+// epilogue chunks).
 bool make_f32_map_3d(void* map, void* base, uint64_t dim0, uint64_t dim1, uint64_t dim2, uint32_t box0,
                      uint32_t box1, uint32_t box2);
 
