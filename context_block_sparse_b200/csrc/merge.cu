@@ -2,8 +2,8 @@
 //   merge_kernel        exact log-sum-exp combine of a block's chunk records plus
 //                       its in-block term -> o, lse
 //   delta_kernel        Delta_i = dout_i . o_i (backward preamble)
-//   bwd_reduce_kernel   dq = sum of chunk dq partials (ascending chunk) + the
-//                       in-block term's dq; dkb, dvb of the in-block term
+//   bwd_reduce_kernel   dq = the in-block term's dq + the chunk dq partials
+//                       (ascending chunk); dkb, dvb of the in-block term
 //
 // News page "Split-KV speeds diffusion drafter training by keeping long-context
 // data local", section "Exchange the smaller side" (partials combined exactly
@@ -12,9 +12,8 @@
 // bs keys are the draft block's own kb/vb rows).
 //
 // One CTA per (block b, KV head g) handles the G*bs query rows (G heads x bs
-// tokens) that read the same bs block keys; one warp per row, each lane owning
-// D/32 consecutive dimensions, so every record row is a coalesced 256/512-byte
-// read.  All loops run in a fixed order, so results are deterministic.
+// tokens) that read the same bs block keys, four threads per row (see the row
+// layout below).  All loops run in a fixed order, so results are deterministic.
 #include <cfloat>
 
 #include "common.cuh"
@@ -68,127 +67,181 @@ __device__ __forceinline__ void load_f32_row(const float* src, float (&x)[DPL]) 
 }
 
 // ---------------------------------------------------------------------------
-// merge: grid (A, Hkv), smem kb/vb rows of the block (bf16)
+// Row layout of the merge and reduce kernels: four threads (a quad) per query
+// row; thread u of the quad owns the 16-byte fp32 granules u, u + 4, u + 8, ...
+// of the row (NG = D / 16 of them, 4 * NG dimensions), so one load instruction
+// of a warp reads 8 rows x 64 contiguous bytes.  Dot products over the row are
+// quad sums (two shuffles).  The block's chunk entries are staged in shared
+// memory kEStage at a time.
+// ---------------------------------------------------------------------------
+constexpr int kEStage = 512;
+constexpr int kRowsPerPass = kMergeThreads / 4;
+
+__device__ __forceinline__ float quad_sum(float x) {
+  x += __shfl_xor_sync(0xffffffffu, x, 1);
+  x += __shfl_xor_sync(0xffffffffu, x, 2);
+  return x;
+}
+
+// the thread's dimensions of a bf16 row: granule k covers dims 4 (u + 4k) .. +3
+template <int NG>
+__device__ __forceinline__ void load_bf16_quad(const uint16_t* row, int u, float (&x)[NG][4]) {
+#pragma unroll
+  for (int k = 0; k < NG; ++k) {
+    const uint2 w = *reinterpret_cast<const uint2*>(row + 4 * (u + 4 * k));
+    x[k][0] = __uint_as_float(w.x << 16);
+    x[k][1] = __uint_as_float(w.x & 0xffff0000u);
+    x[k][2] = __uint_as_float(w.y << 16);
+    x[k][3] = __uint_as_float(w.y & 0xffff0000u);
+  }
+}
+
+template <int NG>
+__device__ __forceinline__ void load_f32_quad(const float* row, int u, float4 (&x)[NG]) {
+#pragma unroll
+  for (int k = 0; k < NG; ++k) x[k] = __ldg(reinterpret_cast<const float4*>(row + 4 * (u + 4 * k)));
+}
+
+// Stage entries [c0, c0 + cnt) of the block into sE (whole CTA; barriers inside).
+__device__ __forceinline__ void stage_entries(int* sE, const int* __restrict__ entries, int c0, int cnt) {
+  __syncthreads();
+  for (int i = threadIdx.x; i < cnt; i += blockDim.x) sE[i] = entries[c0 + i];
+  __syncthreads();
+}
+
+// ---------------------------------------------------------------------------
+// merge: grid (A, Hkv); smem kb/vb rows of the block (bf16), staged entry ids
 // ---------------------------------------------------------------------------
 template <int D>
-__global__ void __launch_bounds__(kMergeThreads)
+__global__ void __launch_bounds__(kMergeThreads, 2)
     merge_kernel(DevPlan p, const uint16_t* __restrict__ q, const uint16_t* __restrict__ kb,
                  const uint16_t* __restrict__ vb, float scale_log2, const float* __restrict__ part_o,
                  const float* __restrict__ part_m, const float* __restrict__ part_l, void* __restrict__ o,
                  int o_bf16, float* __restrict__ lse) {
-  constexpr int DPL = D / 32;
+  constexpr int NG = D / 16;
+  constexpr int EG = 16 / NG;          // entries whose records are in flight together
   extern __shared__ __align__(16) uint8_t smem_raw[];
   uint16_t* sKb = reinterpret_cast<uint16_t*>(smem_raw);   // [bs][D]
   uint16_t* sVb = sKb + p.bs * D;
+  int* sE = reinterpret_cast<int*>(sVb + p.bs * D);        // [kEStage]
   const int b = blockIdx.x, g = blockIdx.y;
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int nwarps = blockDim.x >> 5;
-  // stage the block's own keys/values of KV head g
+  const int tid = threadIdx.x, u = tid & 3;
   for (int idx = tid; idx < p.bs * (D / 8); idx += blockDim.x) {
     const int t = idx / (D / 8), ch = idx % (D / 8);
     const size_t src = (size_t(b * p.bs + t) * p.Hkv + g) * D + ch * 8;
     *reinterpret_cast<uint4*>(sKb + t * D + ch * 8) = *reinterpret_cast<const uint4*>(kb + src);
     *reinterpret_cast<uint4*>(sVb + t * D + ch * 8) = *reinterpret_cast<const uint4*>(vb + src);
   }
-  __syncthreads();
-  const int e0 = p.block_entry_ptr[b], e1 = p.block_entry_ptr[b + 1];
-  const int rows = p.G * p.bs;
-  for (int r = warp; r < rows; r += nwarps) {
-    const int hh = r / p.bs, tt = r % p.bs;
+  const int e0 = p.block_entry_ptr[b], n = p.block_entry_ptr[b + 1] - e0;
+  const int R = p.G * p.bs;
+  for (int r0 = 0; r0 < R; r0 += kRowsPerPass) {
+    // rows ordered (token, head): the 8 rows of a warp are contiguous records
+    const int r = min(r0 + (tid >> 2), R - 1);          // rows past R compute, never store
+    const bool active = r0 + (tid >> 2) < R;
+    const int tt = r / p.G, hh = r - tt * p.G;
     const int head = g * p.G + hh;
     const size_t qrow = size_t(b * p.bs + tt) * p.Hq + head;
-    float qv[DPL];
-    load_bf16_row<DPL>(q + qrow * D + lane * DPL, qv);
-    // in-block term: online softmax over the bs block keys (base 2)
-    float mb = -INFINITY, lb = 0.f, ob[DPL];
+    stage_entries(sE, p.block_entries + e0, 0, min(n, kEStage));
+    // in-block term: online softmax over the bs block keys (base 2), unnormalised
+    float acc[NG][4];
+    float M = -INFINITY, L = 0.f;
+    {
+      float qv[NG][4];
+      load_bf16_quad<NG>(q + qrow * D, u, qv);
 #pragma unroll
-    for (int i = 0; i < DPL; ++i) ob[i] = 0.f;
-    for (int key = 0; key < p.bs; ++key) {
-      float kv[DPL], vv[DPL];
-      load_bf16_row<DPL>(sKb + key * D + lane * DPL, kv);
-      float dot = 0.f;
+      for (int k = 0; k < NG; ++k)
 #pragma unroll
-      for (int i = 0; i < DPL; ++i) dot = fmaf(qv[i], kv[i], dot);
-      const float s = warp_sum(dot) * scale_log2;
-      const float mn = fmaxf(mb, s);
-      const float corr = fast_exp2(mb - mn);
-      const float pr = fast_exp2(s - mn);
-      lb = lb * corr + pr;
-      load_bf16_row<DPL>(sVb + key * D + lane * DPL, vv);
+        for (int i = 0; i < 4; ++i) acc[k][i] = 0.f;
+      for (int key = 0; key < p.bs; ++key) {
+        float kv[NG][4];
+        load_bf16_quad<NG>(sKb + key * D, u, kv);
+        float dot = 0.f;
 #pragma unroll
-      for (int i = 0; i < DPL; ++i) ob[i] = ob[i] * corr + pr * vv[i];
-      mb = mn;
-    }
-    // the chunk records of this row: one entry per lane, 32 at a time
-    const int n = e1 - e0;
-    float Mc = -INFINITY;
-    for (int base = 0; base < n; base += 32) {
-      float m2 = -INFINITY;
-      if (base + lane < n) {
-        const int rec = (p.block_entries[e0 + base + lane] * p.bs + tt) * p.Hq + head;
-        if (part_l[rec] > 0.f) m2 = part_m[rec] * kLog2e;
+        for (int k = 0; k < NG; ++k)
+#pragma unroll
+          for (int i = 0; i < 4; ++i) dot = fmaf(qv[k][i], kv[k][i], dot);
+        const float sc = quad_sum(dot) * scale_log2;
+        const float mn = fmaxf(M, sc);
+        const float corr = fast_exp2(M - mn);
+        const float pr = fast_exp2(sc - mn);
+        L = L * corr + pr;
+        float vv[NG][4];
+        load_bf16_quad<NG>(sVb + key * D, u, vv);
+#pragma unroll
+        for (int k = 0; k < NG; ++k)
+#pragma unroll
+          for (int i = 0; i < 4; ++i) acc[k][i] = fmaf(pr, vv[k][i], acc[k][i] * corr);
+        M = mn;
       }
-      Mc = fmaxf(Mc, warp_max(m2));
     }
-    const float M = fmaxf(mb, Mc);
-    const float wb = fast_exp2(mb - M);   // ob is unnormalised: weight exp2(mb - M)
-    float L = lb * wb;
-    float acc[DPL];
+    // chunk records in ascending chunk order, EG in flight; online reference M
+    for (int c0 = 0; c0 < n; c0 += kEStage) {
+      const int cnt = min(kEStage, n - c0);
+      if (c0 > 0) stage_entries(sE, p.block_entries + e0, c0, cnt);
+      for (int i0 = 0; i0 < cnt; i0 += EG) {
+        float4 ov[EG][NG];
+        float mx[EG], lx[EG];
 #pragma unroll
-    for (int i = 0; i < DPL; ++i) acc[i] = ob[i] * wb;
-    // weighted sum of the normalised chunk outputs in ascending chunk order, 8 rows in flight
-    for (int base = 0; base < n; base += 32) {
-      float wl = 0.f;
-      int recl = 0;
-      if (base + lane < n) {
-        recl = (p.block_entries[e0 + base + lane] * p.bs + tt) * p.Hq + head;
-        const float lx = part_l[recl];
-        wl = lx > 0.f ? lx * fast_exp2(part_m[recl] * kLog2e - M) : 0.f;
-      }
-      L += warp_sum(wl);
-      const int cnt = min(32, n - base);
-      for (int j0 = 0; j0 < cnt; j0 += 8) {
-        float w8[8];
-        float ov[8][DPL];
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          const int j = j0 + u;
-          const float wj = __shfl_sync(0xffffffffu, wl, j & 31);
-          const int rj = __shfl_sync(0xffffffffu, recl, j & 31);
-          w8[u] = j < cnt ? wj : 0.f;
-          if (j < cnt) {
-            load_f32_row<DPL>(part_o + size_t(rj) * D + lane * DPL, ov[u]);
+        for (int v = 0; v < EG; ++v) {
+          lx[v] = 0.f;
+          mx[v] = -INFINITY;
+          if (i0 + v < cnt) {
+            const size_t rec = size_t(sE[i0 + v] * p.bs + tt) * p.Hq + head;
+            load_f32_quad<NG>(part_o + rec * D, u, ov[v]);
+            const float lr = __ldg(part_l + rec), mr = __ldg(part_m + rec);
+            lx[v] = lr;
+            mx[v] = lr > 0.f ? mr * kLog2e : -INFINITY;
           } else {
 #pragma unroll
-            for (int i = 0; i < DPL; ++i) ov[u][i] = 0.f;
+            for (int k = 0; k < NG; ++k) ov[v][k] = make_float4(0.f, 0.f, 0.f, 0.f);
           }
         }
+        float mg = mx[0];
 #pragma unroll
-        for (int u = 0; u < 8; ++u)
+        for (int v = 1; v < EG; ++v) mg = fmaxf(mg, mx[v]);
+        if (mg > M) {
+          const float f = fast_exp2(M - mg);
 #pragma unroll
-          for (int i = 0; i < DPL; ++i) acc[i] = fmaf(w8[u], ov[u][i], acc[i]);
+          for (int k = 0; k < NG; ++k)
+#pragma unroll
+            for (int i = 0; i < 4; ++i) acc[k][i] *= f;
+          L *= f;
+          M = mg;
+        }
+#pragma unroll
+        for (int v = 0; v < EG; ++v) {
+          const float wv = lx[v] > 0.f ? lx[v] * fast_exp2(mx[v] - M) : 0.f;
+          L += wv;
+#pragma unroll
+          for (int k = 0; k < NG; ++k) {
+            acc[k][0] = fmaf(wv, ov[v][k].x, acc[k][0]);
+            acc[k][1] = fmaf(wv, ov[v][k].y, acc[k][1]);
+            acc[k][2] = fmaf(wv, ov[v][k].z, acc[k][2]);
+            acc[k][3] = fmaf(wv, ov[v][k].w, acc[k][3]);
+          }
+        }
       }
     }
-    const float inv = L > 0.f ? 1.f / L : 0.f;
-    if (o_bf16) {
-      uint16_t* dst = static_cast<uint16_t*>(o) + qrow * D + lane * DPL;
-      if constexpr (DPL == 4) {
-        uint2 u;
-        u.x = pack_bf16(acc[0] * inv, acc[1] * inv);
-        u.y = pack_bf16(acc[2] * inv, acc[3] * inv);
-        *reinterpret_cast<uint2*>(dst) = u;
+    if (active) {
+      const float inv = L > 0.f ? 1.f / L : 0.f;
+      if (o_bf16) {
+        uint16_t* dst = static_cast<uint16_t*>(o) + qrow * D;
+#pragma unroll
+        for (int k = 0; k < NG; ++k) {
+          uint2 w;
+          w.x = pack_bf16(acc[k][0] * inv, acc[k][1] * inv);
+          w.y = pack_bf16(acc[k][2] * inv, acc[k][3] * inv);
+          *reinterpret_cast<uint2*>(dst + 4 * (u + 4 * k)) = w;
+        }
       } else {
-        *reinterpret_cast<uint32_t*>(dst) = pack_bf16(acc[0] * inv, acc[1] * inv);
+        float* dst = static_cast<float*>(o) + qrow * D;
+#pragma unroll
+        for (int k = 0; k < NG; ++k)
+          *reinterpret_cast<float4*>(dst + 4 * (u + 4 * k)) =
+              make_float4(acc[k][0] * inv, acc[k][1] * inv, acc[k][2] * inv, acc[k][3] * inv);
       }
-    } else {
-      float* dst = static_cast<float*>(o) + qrow * D + lane * DPL;
-      if constexpr (DPL == 4) {
-        *reinterpret_cast<float4*>(dst) = make_float4(acc[0] * inv, acc[1] * inv, acc[2] * inv, acc[3] * inv);
-      } else {
-        *reinterpret_cast<float2*>(dst) = make_float2(acc[0] * inv, acc[1] * inv);
-      }
+      if (u == 0) lse[qrow] = L > 0.f ? (M + __log2f(L)) * kLn2 : -INFINITY;
     }
-    if (lane == 0) lse[qrow] = L > 0.f ? (M + __log2f(L)) * kLn2 : -INFINITY;
   }
 }
 
@@ -220,27 +273,31 @@ __global__ void __launch_bounds__(kMergeThreads)
 
 // ---------------------------------------------------------------------------
 // dq reduce + in-block backward: grid (A, Hkv)
-// smem: kb, vb [bs][D] bf16; P, dS [rows][bs] fp32 (rows = G*bs)
+// smem: kb, vb [bs][D] bf16; P, dS [rows][bs] fp32 (rows = G*bs, ordered
+// (token, head)); q, dout [rows][D] bf16 when stage_rows; entry ids
 // ---------------------------------------------------------------------------
 template <int D>
-__global__ void __launch_bounds__(kMergeThreads)
+__global__ void __launch_bounds__(kMergeThreads, 2)
     bwd_reduce_kernel(DevPlan p, const uint16_t* __restrict__ q, const uint16_t* __restrict__ kb,
                       const uint16_t* __restrict__ vb, const uint16_t* __restrict__ dout,
                       const float* __restrict__ lse, const float* __restrict__ delta,
                       const float* __restrict__ dq_part, float scale, float* __restrict__ dq,
                       float* __restrict__ dkb, float* __restrict__ dvb, int stage_rows) {
+  constexpr int NG = D / 16;
+  constexpr int EG = 16 / NG;
   constexpr int DPL = D / 32;
   extern __shared__ __align__(16) uint8_t smem_raw[];
   const int bs = p.bs;
-  const int rows = p.G * bs;
+  const int R = p.G * bs;
   uint16_t* sKb = reinterpret_cast<uint16_t*>(smem_raw);
   uint16_t* sVb = sKb + bs * D;
   float* sP = reinterpret_cast<float*>(sVb + bs * D);    // [rows][bs]
-  float* sdS = sP + rows * bs;                            // [rows][bs]
-  uint16_t* sQr = reinterpret_cast<uint16_t*>(sdS + rows * bs);   // [rows][D] when stage_rows
-  uint16_t* sDr = sQr + rows * D;
+  float* sdS = sP + R * bs;                               // [rows][bs]
+  int* sE = reinterpret_cast<int*>(sdS + R * bs);         // [kEStage]
+  uint16_t* sQr = reinterpret_cast<uint16_t*>(sE + kEStage);   // [rows][D] when stage_rows
+  uint16_t* sDr = sQr + R * D;
   const int b = blockIdx.x, g = blockIdx.y;
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int tid = threadIdx.x, u = tid & 3, warp = tid >> 5, lane = tid & 31;
   const int nwarps = blockDim.x >> 5;
   for (int idx = tid; idx < bs * (D / 8); idx += blockDim.x) {
     const int t = idx / (D / 8), ch = idx % (D / 8);
@@ -248,89 +305,100 @@ __global__ void __launch_bounds__(kMergeThreads)
     *reinterpret_cast<uint4*>(sKb + t * D + ch * 8) = *reinterpret_cast<const uint4*>(kb + src);
     *reinterpret_cast<uint4*>(sVb + t * D + ch * 8) = *reinterpret_cast<const uint4*>(vb + src);
   }
-  __syncthreads();
   const float scale_log2 = scale * kLog2e;
-  const int e0 = p.block_entry_ptr[b], e1 = p.block_entry_ptr[b + 1];
-  // phase 1, one warp per row: P, dS of the in-block keys; dq = sum of partials + in-block dq
-  for (int r = warp; r < rows; r += nwarps) {
-    const int hh = r / bs, tt = r % bs;
+  const int e0 = p.block_entry_ptr[b], n = p.block_entry_ptr[b + 1] - e0;
+  // phase 1, a quad per row: P, dS of the in-block keys; dq = in-block dq + sum of partials
+  for (int r0 = 0; r0 < R; r0 += kRowsPerPass) {
+    const int r = min(r0 + (tid >> 2), R - 1);          // rows past R compute, never store
+    const bool active = r0 + (tid >> 2) < R;
+    const int tt = r / p.G, hh = r - tt * p.G;
     const int head = g * p.G + hh;
     const size_t qrow = size_t(b * bs + tt) * p.Hq + head;
-    float qv[DPL], dov[DPL];
-    load_bf16_row<DPL>(q + qrow * D + lane * DPL, qv);
-    load_bf16_row<DPL>(dout + qrow * D + lane * DPL, dov);
-    const float l2 = lse[qrow] * kLog2e;
-    const float dl = delta[qrow];
-    float acc[DPL];
+    stage_entries(sE, p.block_entries + e0, 0, min(n, kEStage));
+    float acc[NG][4];
+    {
+      float qv[NG][4], dov[NG][4];
+      load_bf16_quad<NG>(q + qrow * D, u, qv);
+      load_bf16_quad<NG>(dout + qrow * D, u, dov);
+      const float l2 = lse[qrow] * kLog2e;
+      const float dl = delta[qrow];
 #pragma unroll
-    for (int i = 0; i < DPL; ++i) acc[i] = 0.f;
-    for (int key = 0; key < bs; ++key) {
-      float kv[DPL], vv[DPL];
-      load_bf16_row<DPL>(sKb + key * D + lane * DPL, kv);
-      load_bf16_row<DPL>(sVb + key * D + lane * DPL, vv);
-      float s = 0.f, dp = 0.f;
+      for (int k = 0; k < NG; ++k)
 #pragma unroll
-      for (int i = 0; i < DPL; ++i) {
-        s = fmaf(qv[i], kv[i], s);
-        dp = fmaf(dov[i], vv[i], dp);
+        for (int i = 0; i < 4; ++i) acc[k][i] = 0.f;
+      for (int key = 0; key < bs; ++key) {
+        float sd = 0.f, dp = 0.f;
+#pragma unroll
+        for (int k = 0; k < NG; ++k) {
+          float kv[1][4], vv[1][4];
+          load_bf16_quad<1>(sKb + key * D + 16 * k, u, kv);
+          load_bf16_quad<1>(sVb + key * D + 16 * k, u, vv);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            sd = fmaf(qv[k][i], kv[0][i], sd);
+            dp = fmaf(dov[k][i], vv[0][i], dp);
+          }
+        }
+        sd = quad_sum(sd);
+        dp = quad_sum(dp);
+        const float pr = (l2 == -INFINITY) ? 0.f : fast_exp2(sd * scale_log2 - l2);
+        const float ds = pr * (dp - dl);
+        if (active && u == 0) {
+          sP[r * bs + key] = pr;
+          sdS[r * bs + key] = ds;
+        }
+#pragma unroll
+        for (int k = 0; k < NG; ++k) {
+          float kv[1][4];
+          load_bf16_quad<1>(sKb + key * D + 16 * k, u, kv);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) acc[k][i] = fmaf(ds, kv[0][i], acc[k][i]);
+        }
       }
-      s = warp_sum(s);
-      dp = warp_sum(dp);
-      const float pr = (l2 == -INFINITY) ? 0.f : fast_exp2(s * scale_log2 - l2);
-      const float ds = pr * (dp - dl);
-      if (lane == 0) {
-        sP[r * bs + key] = pr;
-        sdS[r * bs + key] = ds;
-      }
+      if (stage_rows && active) {   // keep q and dout of this row for the dkb / dvb pass
 #pragma unroll
-      for (int i = 0; i < DPL; ++i) acc[i] = fmaf(ds, kv[i], acc[i]);
+        for (int k = 0; k < NG; ++k) {
+          const int off = r * D + 4 * (u + 4 * k);
+          *reinterpret_cast<uint2*>(sQr + off) = *reinterpret_cast<const uint2*>(q + qrow * D + 4 * (u + 4 * k));
+          *reinterpret_cast<uint2*>(sDr + off) = *reinterpret_cast<const uint2*>(dout + qrow * D + 4 * (u + 4 * k));
+        }
+      }
     }
-    // chunk partials in ascending chunk order (8 rows in flight), then the in-block term
-    float tot[DPL];
+    // the in-block term, then the chunk partials in ascending chunk order, EG in flight
+    float4 tot[NG];
 #pragma unroll
-    for (int i = 0; i < DPL; ++i) tot[i] = 0.f;
-    const int n = e1 - e0;
-    for (int base = 0; base < n; base += 32) {
-      int recl = 0;
-      if (base + lane < n) recl = (p.block_entries[e0 + base + lane] * bs + tt) * p.Hq + head;
-      const int cnt = min(32, n - base);
-      for (int j0 = 0; j0 < cnt; j0 += 8) {
-        float pv[8][DPL];
+    for (int k = 0; k < NG; ++k)
+      tot[k] = make_float4(scale * acc[k][0], scale * acc[k][1], scale * acc[k][2], scale * acc[k][3]);
+    for (int c0 = 0; c0 < n; c0 += kEStage) {
+      const int cnt = min(kEStage, n - c0);
+      if (c0 > 0) stage_entries(sE, p.block_entries + e0, c0, cnt);
+      for (int i0 = 0; i0 < cnt; i0 += EG) {
+        float4 pv[EG][NG];
 #pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          const int j = j0 + u;
-          const int rj = __shfl_sync(0xffffffffu, recl, j & 31);
-          if (j < cnt) {
-            load_f32_row<DPL>(dq_part + size_t(rj) * D + lane * DPL, pv[u]);
+        for (int v = 0; v < EG; ++v) {
+          if (i0 + v < cnt) {
+            const size_t rec = size_t(sE[i0 + v] * bs + tt) * p.Hq + head;
+            load_f32_quad<NG>(dq_part + rec * D, u, pv[v]);
           } else {
 #pragma unroll
-            for (int i = 0; i < DPL; ++i) pv[u][i] = 0.f;
+            for (int k = 0; k < NG; ++k) pv[v][k] = make_float4(0.f, 0.f, 0.f, 0.f);
           }
         }
 #pragma unroll
-        for (int u = 0; u < 8; ++u)
+        for (int v = 0; v < EG; ++v)
 #pragma unroll
-          for (int i = 0; i < DPL; ++i) tot[i] += pv[u][i];
+          for (int k = 0; k < NG; ++k) {
+            tot[k].x += pv[v][k].x;
+            tot[k].y += pv[v][k].y;
+            tot[k].z += pv[v][k].z;
+            tot[k].w += pv[v][k].w;
+          }
       }
     }
-    if (stage_rows) {   // keep q and dout of this row for the dkb / dvb pass
-      uint16_t* sq = sQr + r * D + lane * DPL;
-      uint16_t* sd = sDr + r * D + lane * DPL;
-      if constexpr (DPL == 4) {
-        *reinterpret_cast<uint2*>(sq) = *reinterpret_cast<const uint2*>(q + qrow * D + lane * DPL);
-        *reinterpret_cast<uint2*>(sd) = *reinterpret_cast<const uint2*>(dout + qrow * D + lane * DPL);
-      } else {
-        *reinterpret_cast<uint32_t*>(sq) = *reinterpret_cast<const uint32_t*>(q + qrow * D + lane * DPL);
-        *reinterpret_cast<uint32_t*>(sd) = *reinterpret_cast<const uint32_t*>(dout + qrow * D + lane * DPL);
-      }
-    }
-    float* dst = dq + qrow * D + lane * DPL;
+    if (active) {
+      float* dst = dq + qrow * D;
 #pragma unroll
-    for (int i = 0; i < DPL; ++i) tot[i] += scale * acc[i];
-    if constexpr (DPL == 4) {
-      *reinterpret_cast<float4*>(dst) = make_float4(tot[0], tot[1], tot[2], tot[3]);
-    } else {
-      *reinterpret_cast<float2*>(dst) = make_float2(tot[0], tot[1]);
+      for (int k = 0; k < NG; ++k) *reinterpret_cast<float4*>(dst + 4 * (u + 4 * k)) = tot[k];
     }
   }
   __syncthreads();
@@ -339,13 +407,13 @@ __global__ void __launch_bounds__(kMergeThreads)
     float ak[DPL], av[DPL];
 #pragma unroll
     for (int i = 0; i < DPL; ++i) ak[i] = av[i] = 0.f;
-    for (int r = 0; r < rows; ++r) {
+    for (int r = 0; r < R; ++r) {
       float qv[DPL], dov[DPL];
       if (stage_rows) {
         load_bf16_row<DPL>(sQr + r * D + lane * DPL, qv);
         load_bf16_row<DPL>(sDr + r * D + lane * DPL, dov);
       } else {
-        const int hh = r / bs, tt = r % bs;
+        const int tt = r / p.G, hh = r - tt * p.G;
         const size_t qrow = size_t(b * bs + tt) * p.Hq + g * p.G + hh;
         load_bf16_row<DPL>(q + qrow * D + lane * DPL, qv);
         load_bf16_row<DPL>(dout + qrow * D + lane * DPL, dov);
@@ -374,7 +442,7 @@ template <int D>
 cudaError_t merge_d(const DevPlan& p, const uint16_t* q, const uint16_t* kb, const uint16_t* vb,
                     float scale, const float* po, const float* pm, const float* pl, void* o, int o_bf16,
                     float* lse, cudaStream_t s) {
-  const size_t smem = size_t(2) * p.bs * D * sizeof(uint16_t);
+  const size_t smem = size_t(2) * p.bs * D * sizeof(uint16_t) + kEStage * sizeof(int);
   cudaError_t e = cudaFuncSetAttribute(merge_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
   if (e != cudaSuccess) return e;
   merge_kernel<D><<<dim3(p.A, p.Hkv), kMergeThreads, smem, s>>>(p, q, kb, vb, scale * kLog2e, po, pm, pl, o,
@@ -387,7 +455,8 @@ cudaError_t reduce_d(const DevPlan& p, const uint16_t* q, const uint16_t* kb, co
                      const uint16_t* dout, const float* lse, const float* delta, const float* dq_part,
                      float scale, float* dq, float* dkb, float* dvb, cudaStream_t s) {
   const size_t rows = size_t(p.G) * p.bs;
-  const size_t base = size_t(2) * p.bs * D * sizeof(uint16_t) + 2 * rows * p.bs * sizeof(float);
+  const size_t base =
+      size_t(2) * p.bs * D * sizeof(uint16_t) + 2 * rows * p.bs * sizeof(float) + kEStage * sizeof(int);
   const size_t staged = base + 2 * rows * D * sizeof(uint16_t);
   const int stage_rows = staged <= size_t(64) * 1024 ? 1 : 0;   // small enough to keep occupancy
   const size_t smem = stage_rows ? staged : base;
