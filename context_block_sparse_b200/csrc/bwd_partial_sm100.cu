@@ -12,10 +12,12 @@
 //
 //  dkdv kernel (KV-stationary, backward LPT schedule, whole chunks): for every
 //    128-key tile of the chunk, for every query tile that meets it:
-//      S^T = K Q^T, dP^T = V dO^T          (TMEM, keys as lanes)
-//      P^T, dS^T = P^T (dP^T - Delta)      (thread = key; bf16, written back
-//                                           over S^T / dP^T)
-//      dV += P^T dO, dK += dS^T Q          (A operand from TMEM)
+//      S^T = K Q^T, dP^T = V dO^T          (TMEM, keys as lanes; two commits)
+//      P^T                                 (thread = key; bf16 over S^T, as soon
+//                                           as S^T lands)
+//      dV += P^T dO                        (A operand from TMEM, overlapping...)
+//      dS^T = P^T (dP^T - Delta)           (... the dS^T pass; bf16 over dP^T)
+//      dK += dS^T Q
 //    then dK (times scale) and dV of the tile's keys go to global memory; keys
 //    that no query reads get zeros.
 //  dq kernel (Q-stationary, forward LPT schedule): for every query tile, over
@@ -162,24 +164,25 @@ __device__ __forceinline__ void ds_tile(uint32_t tS, uint32_t tdP, int hf, int a
 }
 
 // dkdv kernel, rows 64hf..64hf+63 of one query tile for one key (thread = TMEM
-// lane): P^T and dS^T = P^T (dP^T - Delta), P = exp2(s * c - lse2[row]), zero
-// for rows whose slot bit (slot = row >> lg) is clear; bf16 pairs of rows go to
-// packed_col() of S^T and of dP^T.
+// lane), first half of the element-wise step: P^T = exp2(s * c - lse2[row]),
+// zero for rows whose slot bit (slot = row >> lg) is clear.  P stays in pv
+// (fp32, for dS^T) and goes as bf16 pairs to packed_col() of S^T.
 template <bool kMasked>
-__device__ __forceinline__ void pds_tile(uint32_t tSt, uint32_t tdPt, int hf, uint32_t smask, int lg,
-                                         const float4* ld4, float c) {
-#pragma unroll 1
-  for (int q = 2 * hf; q < 2 * hf + 2; ++q) {   // 32 rows per TMEM round trip
-    uint32_t sv[32], dpv[32];
+__device__ __forceinline__ void pt_tile(uint32_t tSt, int hf, uint32_t smask, int lg, const float4* ld4, float c,
+                                        float (&pv)[64]) {
+#pragma unroll
+  for (int qq = 0; qq < 2; ++qq) {   // 32 rows per TMEM round trip
+    const int q = 2 * hf + qq;
+    uint32_t sv[32];
     tmem_ld32(tSt + q * 32, sv);
-    tmem_ld32(tdPt + q * 32, dpv);
     tmem_wait_ld();
-    uint32_t pp[16], pd[16];
+    reg_fence<32>(sv);
+    uint32_t pp[16];
 #pragma unroll
     for (int i = 0; i < 16; ++i) {
       const int row = q * 32 + 2 * i;
       const float4 m = ld4[row >> 1];    // lse2[row], delta[row], lse2[row + 1], delta[row + 1]
-      float x0, x1, d0, d1, g0, g1;
+      float x0, x1;
       ffma2(x0, x1, __uint_as_float(sv[2 * i]), __uint_as_float(sv[2 * i + 1]), c, c, -m.x, -m.z);
       float p0, p1;
       exp2_pair((i % kPolyEvery) == 1, x0, x1, p0, p1);
@@ -188,12 +191,33 @@ __device__ __forceinline__ void pds_tile(uint32_t tSt, uint32_t tdPt, int hf, ui
         p0 = in ? p0 : 0.f;
         p1 = in ? p1 : 0.f;
       }
-      fadd2(d0, d1, __uint_as_float(dpv[2 * i]), __uint_as_float(dpv[2 * i + 1]), -m.y, -m.w);
-      fmul2(g0, g1, p0, p1, d0, d1);
+      pv[qq * 32 + 2 * i] = p0;
+      pv[qq * 32 + 2 * i + 1] = p1;
       pp[i] = pack_bf16(p0, p1);
-      pd[i] = pack_bf16(g0, g1);
     }
     tmem_st16p(tSt + packed_col(2 * q), pp);
+  }
+}
+
+// Second half: dS^T = P^T (dP^T - Delta[row]) as bf16 pairs to packed_col() of dP^T.
+__device__ __forceinline__ void dst_tile(uint32_t tdPt, int hf, const float4* ld4, const float (&pv)[64]) {
+#pragma unroll
+  for (int qq = 0; qq < 2; ++qq) {
+    const int q = 2 * hf + qq;
+    uint32_t dpv[32];
+    tmem_ld32(tdPt + q * 32, dpv);
+    tmem_wait_ld();
+    reg_fence<32>(dpv);
+    uint32_t pd[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const int row = q * 32 + 2 * i;
+      const float4 m = ld4[row >> 1];
+      float d0, d1, g0, g1;
+      fadd2(d0, d1, __uint_as_float(dpv[2 * i]), __uint_as_float(dpv[2 * i + 1]), -m.y, -m.w);
+      fmul2(g0, g1, pv[qq * 32 + 2 * i], pv[qq * 32 + 2 * i + 1], d0, d1);
+      pd[i] = pack_bf16(g0, g1);
+    }
     tmem_st16p(tdPt + packed_col(2 * q), pd);
   }
 }
@@ -202,12 +226,12 @@ __device__ __forceinline__ void pds_tile(uint32_t tSt, uint32_t tdPt, int hf, ui
 // dkdv kernel
 // ============================================================================
 struct DkdvBars {
-  uint64_t kv_full, kv_empty, qd_full[2], qd_empty[2], st_ready, pds_ready, dkv_ready, dkv_free, mma_done,
-      meta_ready[2], meta_free[2];
+  uint64_t kv_full, kv_empty, qd_full[2], qd_empty[2], st_ready, dpt_ready, pt_ready, dst_ready, dkv_ready,
+      dkv_free, mma_done, meta_ready[2], meta_free[2];
   uint32_t tmem_base;
   int abort_flag;
 };
-constexpr int kDkdvNumBars = 15;
+constexpr int kDkdvNumBars = 17;
 
 __global__ void __launch_bounds__(kThreads, 1)
     bwd_dkdv_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_do,
@@ -232,7 +256,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     B->abort_flag = 0;
   }
   {
-    const uint32_t counts[kDkdvNumBars] = {1, 1, 1, 1, 1, 1, 1, 256, 1, 256, 1, 32, 32, 256, 256};
+    // commits count 1; element-wise / metadata signals count warps (warp_arrive)
+    const uint32_t counts[kDkdvNumBars] = {1, 1, 1, 1, 1, 1, 1, 1, 8, 8, 1, 8, 1, 1, 1, 8, 8};
     setup_common(&B->kv_full, kDkdvNumBars, counts, &B->tmem_base, warp);
   }
   const uint32_t tmem = B->tmem_base;
@@ -291,12 +316,14 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int s = qd_count & 1;
             if (!mbar_wait(&B->qd_full[s], (qd_count >> 1) & 1, wctx, 2 * 10000 + __LINE__)) { ok = false; break; }
             tc_fence_after();
-            // S^T = K Q^T (cols 0..127), dP^T = V dO^T (cols 128..255)
+            // S^T = K Q^T (cols 0..127), dP^T = V dO^T (cols 128..255); the P^T pass
+            // starts when S^T lands, while dP^T is still being computed
             for (int kk = 0; kk < D / 16; ++kk)
               mma_ss(tmem + 0, kmajor(aK, kk), kmajor(aQ + s * kTile, kk), kIdescKM, kk > 0 ? 1u : 0u);
+            mma_commit(&B->st_ready);
             for (int kk = 0; kk < D / 16; ++kk)
               mma_ss(tmem + 128, kmajor(aV, kk), kmajor(adO + s * kTile, kk), kIdescKM, kk > 0 ? 1u : 0u);
-            mma_commit(&B->st_ready);
+            mma_commit(&B->dpt_ready);
             {   // K and V are read only by S^T / dP^T: release them after the key tile's last pair
               bool later = false;
               for (int t2 = t + 1; t2 < item.w && !later; ++t2) {
@@ -305,17 +332,20 @@ __global__ void __launch_bounds__(kThreads, 1)
               }
               if (!later) mma_commit(&B->kv_empty);
             }
-            if (!mbar_wait(&B->pds_ready, pds_cnt & 1, wctx, 2 * 10000 + __LINE__)) { ok = false; break; }
-            ++pds_cnt;
+            if (!mbar_wait(&B->pt_ready, pds_cnt & 1, wctx, 2 * 10000 + __LINE__)) { ok = false; break; }
             if (u == 0) {
               if (!mbar_wait(&B->dkv_free, (dkvf_cnt & 1) ^ 1, wctx, 2 * 10000 + __LINE__)) { ok = false; break; }
               ++dkvf_cnt;
             }
             tc_fence_after();
-            // dV (cols 384..) += P^T dO ; dK (cols 256..) += dS^T Q  -- A operands from TMEM
+            // dV (cols 384..) += P^T dO while dS^T is formed -- A operand from TMEM
             for (int kk = 0; kk < BT / 16; ++kk)
               mma_ts(tmem + 384, tmem + 0 + packed_col(kk), mnmajor(adO + s * kTile, kk), kIdescMN,
                      (u > 0 || kk > 0) ? 1u : 0u);
+            if (!mbar_wait(&B->dst_ready, pds_cnt & 1, wctx, 2 * 10000 + __LINE__)) { ok = false; break; }
+            ++pds_cnt;
+            tc_fence_after();
+            // dK (cols 256..) += dS^T Q
             for (int kk = 0; kk < BT / 16; ++kk)
               mma_ts(tmem + 256, tmem + 128 + packed_col(kk), mnmajor(aQ + s * kTile, kk), kIdescMN,
                      (u > 0 || kk > 0) ? 1u : 0u);
@@ -358,7 +388,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             meta_ld[s * 128 + rr] = make_float2(l2, dl);
             if (rr % rps == 0) meta_slot[s * 16 + rr / rps] = make_int2(m.lo, m.hi);
           }
-          mbar_arrive(&B->meta_ready[s]);
+          warp_arrive(&B->meta_ready[s]);
           ++mcount;
         }
       }
@@ -411,17 +441,24 @@ __global__ void __launch_bounds__(kThreads, 1)
           // warp-uniform choice: both paths issue warp-collective tcgen05.ld/st
           const bool all_in = __all_sync(0xffffffffu, (smask & all) == all);
           if (!warp_wait(&B->st_ready, st_cnt & 1, wctx, 2 * 10000 + __LINE__)) { ok = false; break; }
-          ++st_cnt;
           tc_fence_after();
           const float4* ld4 = reinterpret_cast<const float4*>(meta_ld + s * 128);
+          float pv[64];
           if (all_in)
-            pds_tile<false>(tSt, tdPt, hf, smask, lg, ld4, scale_log2);
+            pt_tile<false>(tSt, hf, smask, lg, ld4, scale_log2, pv);
           else
-            pds_tile<true>(tSt, tdPt, hf, smask, lg, ld4, scale_log2);
+            pt_tile<true>(tSt, hf, smask, lg, ld4, scale_log2, pv);
           tmem_wait_st();
           tc_fence_before();
-          mbar_arrive(&B->pds_ready);
-          mbar_arrive(&B->meta_free[s]);
+          warp_arrive(&B->pt_ready);
+          if (!warp_wait(&B->dpt_ready, st_cnt & 1, wctx, 2 * 10000 + __LINE__)) { ok = false; break; }
+          ++st_cnt;
+          tc_fence_after();
+          dst_tile(tdPt, hf, ld4, pv);
+          tmem_wait_st();
+          tc_fence_before();
+          warp_arrive(&B->dst_ready);
+          warp_arrive(&B->meta_free[s]);
           ++qd_count;
           ++n_meet;
         }
@@ -444,7 +481,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             warp_store_rows<16>(scratch, reinterpret_cast<const float*>(a), f, own ? dst + cc * 16 : nullptr);
           }
           tc_fence_before();
-          mbar_arrive(&B->dkv_free);
+          warp_arrive(&B->dkv_free);
         } else if (own) {
           for (int i = 0; i < D; i += 4) *reinterpret_cast<float4*>(dst + i) = make_float4(0.f, 0.f, 0.f, 0.f);
         }
@@ -520,7 +557,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   const WaitCtx wctx{abort_flag, p.status};
   if (tid == 0) B->abort_flag = 0;
   {
-    const uint32_t counts[kDqNumBars] = {1, 1, 1, 1, 1, 1, 1, 1, 1, 1, 1, 256, 1, 256, 1, 32, 32, 256, 256};
+    // commits count 1; element-wise / metadata signals count warps (warp_arrive)
+    const uint32_t counts[kDqNumBars] = {1, 1, 1, 1, 1, 1, 1, 1, 1, 1, 1, 8, 1, 8, 1, 1, 1, 8, 8};
     setup_common(&B->qd_full, kDqNumBars, counts, &B->tmem_base, warp);
   }
   const uint32_t tmem = B->tmem_base;
@@ -606,11 +644,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             ++dqf_cnt;
           }
           tc_fence_after();
+          // the next dP first (the element-wise step of key tile j + 1 waits on it), then
           // dQ (cols 384..) += dS K : dS in TMEM (columns 0..63 of S buffer s), K MN-major
-          for (int kk = 0; kk < BT / 16; ++kk)
-            mma_ts(tmem + 384, tmem + s * 128 + packed_col(kk), mnmajor(aK + s * kTile, kk), kIdescMN,
-                   (j > 0 || kk > 0) ? 1u : 0u);
-          mma_commit(&B->kv_empty[s]);
           if (more) {
             if (!mbar_wait(&B->v_full[s1], ((c + 1) >> 1) & 1, wctx, 2 * 10000 + __LINE__)) { ok = false; break; }
             tc_fence_after();
@@ -619,6 +654,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             mma_commit(&B->dp_ready);
             if (j + 2 == n_kt) mma_commit(&B->qd_empty);   // Q, dO: no further reader after this S / dP
           }
+          for (int kk = 0; kk < BT / 16; ++kk)
+            mma_ts(tmem + 384, tmem + s * 128 + packed_col(kk), mnmajor(aK + s * kTile, kk), kIdescMN,
+                   (j > 0 || kk > 0) ? 1u : 0u);
+          mma_commit(&B->kv_empty[s]);
         }
         if (!ok) break;
         mma_commit(&B->dq_ready);
@@ -657,7 +696,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         meta[s * 128 + rr] = d;
       }
-      mbar_arrive(&B->meta_ready[s]);
+      warp_arrive(&B->meta_ready[s]);
       ++mcount;
     }
     if (!ok) *abort_flag = 1;
@@ -679,7 +718,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int ms = mcount & 1;
       if (!warp_wait(&B->meta_ready[ms], (mcount >> 1) & 1, wctx, 2 * 10000 + __LINE__)) { ok = false; break; }
       const DqRow m = meta[ms * 128 + r];
-      mbar_arrive(&B->meta_free[ms]);
+      warp_arrive(&B->meta_free[ms]);
       ++mcount;
       const float l2 = m.l2, dl = m.dl;
       for (int j = 0; j < n_kt; ++j) {
@@ -699,7 +738,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           ds_tile<true>(tS, tdP, hf, a, b, scale_log2, l2, dl);
         tmem_wait_st();
         tc_fence_before();
-        mbar_arrive(&B->ds_ready);
+        warp_arrive(&B->ds_ready);
       }
       if (!ok) break;
       kv_count += n_kt;
@@ -716,7 +755,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         warp_store_rows<16>(scratch, reinterpret_cast<const float*>(v), scale, m.valid ? dst + cc * 16 : nullptr);
       }
       tc_fence_before();
-      mbar_arrive(&B->dq_free);
+      warp_arrive(&B->dq_free);
     }
     if (!ok) *abort_flag = 1;
   }

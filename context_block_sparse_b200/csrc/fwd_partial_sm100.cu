@@ -185,9 +185,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int x = 0; x < 2; ++x) {
       mbar_init(&bars->s_ready[x], 1);
-      mbar_init(&bars->p_ready[x], 128);
+      mbar_init(&bars->p_ready[x], 4);    // one arrival per softmax warp
       mbar_init(&bars->o_ready[x], 1);
-      mbar_init(&bars->o_free[x], 128);
+      mbar_init(&bars->o_free[x], 4);
     }
     mbar_init(&bars->mma_done, 1);
     bars->abort_flag = 0;
@@ -462,7 +462,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         m_true = fmaxf(m_true, none ? -INFINITY : mx);
         tmem_wait_st();
         tc_fence_before();
-        mbar_arrive(&bars->p_ready[x]);
+        warp_arrive(&bars->p_ready[x]);
       }
       if (!ok) break;
       // epilogue: wait for the last PV of this tile, then write the record
@@ -510,9 +510,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         part_m[rec] = (l > 0.f) ? m_true * kLn2 : -INFINITY;
         part_l[rec] = (l > 0.f) ? l * fast_exp2(m_ref - m_true) : 0.f;
       }
-      __syncwarp();
       tc_fence_before();
-      mbar_arrive(&bars->o_free[x]);
+      warp_arrive(&bars->o_free[x]);
     }
     // bulk stores of this warp complete before the CTA exits
     if (lane == 0) bulk_wait0();
