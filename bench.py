@@ -43,16 +43,31 @@ sys.path.insert(0, ROOT)
 
 METRIC = "masked-pair attn TFLOP/s fwd/bwd, % of BF16 tensor peak; LPT imbalance %"
 
-# DRAM bytes per launch from ncu captures (dram__bytes_read.sum + dram__bytes_write.sum),
-# keyed by kernel, with the sha256 of the kernel source they were taken on; a
-# changed source voids the figure.
-NCU_TRAFFIC = {}
+# DRAM bytes per launch at the default (64k context / 8k queries) workload, from
+# one ncu capture (dram__bytes_read.sum + dram__bytes_write.sum, mean of 5
+# launches), keyed by kernel, with the sha256 of the sources the kernel was
+# built from when it was taken; a changed source voids the figure.
+NCU_TRAFFIC = {
+    "fwd_partial": {"bytes": 2078109286, "src": "58a8dc50e8d73802"},
+    "merge": {"bytes": 1558072269, "src": "747751e396772082"},
+    "bwd_delta": {"bytes": 201895065, "src": "747751e396772082"},
+    "bwd_dkdv": {"bytes": 1727694080, "src": "4f1f3b56d6418672"},
+    "bwd_dq": {"bytes": 2309566618, "src": "4f1f3b56d6418672"},
+    "bwd_reduce": {"bytes": 1553884058, "src": "747751e396772082"},
+}
+_KERNEL_SOURCES = {
+    "fwd_partial": ("fwd_partial_sm100.cu", "sm100.cuh", "splitkv_internal.h"),
+    "bwd_dkdv": ("bwd_partial_sm100.cu", "sm100.cuh", "splitkv_internal.h"),
+    "bwd_dq": ("bwd_partial_sm100.cu", "sm100.cuh", "splitkv_internal.h"),
+}
 
 
-def _src_hash(name: str) -> str:
-    path = os.path.join(ROOT, "context_block_sparse_b200", "csrc", name)
-    with open(path, "rb") as f:
-        return hashlib.sha256(f.read()).hexdigest()[:16]
+def _src_hash(kernel: str) -> str:
+    m = hashlib.sha256()
+    for name in _KERNEL_SOURCES.get(kernel, ("merge.cu", "common.cuh", "splitkv_internal.h")):
+        with open(os.path.join(ROOT, "context_block_sparse_b200", "csrc", name), "rb") as f:
+            m.update(f.read())
+    return m.hexdigest()[:16]
 
 
 def _peaks():
@@ -68,19 +83,52 @@ def _peaks():
 
 
 class ClockSampler:
-    """nvidia-smi clock / throttle-reason samples while the timed region runs."""
+    """SM clock, power and clock-event reasons sampled while the timed region runs.
+
+    NVML (read-only queries) polled every 2 ms from a thread, so that a timed region
+    of a few tens of milliseconds still gets samples; nvidia-smi at 100 ms when NVML
+    cannot be opened."""
 
     FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
               "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
               "clocks_event_reasons.sw_power_cap")
+    NAMES = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
 
     def __init__(self, gpu_id: str):
         self.gpu_id = gpu_id
-        self.rows = []
+        self.rows = []          # (time, sm_mhz, max_mhz, {reason names})
         self.proc = None
         self.t = None
+        self.stop_flag = False
+        self.source = None
 
     def start(self):
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            h = pynvml.nvmlDeviceGetHandleByUUID(self.gpu_id)
+            mx = pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM)
+            bits = (pynvml.nvmlClocksEventReasonHwSlowdown, pynvml.nvmlClocksEventReasonHwThermalSlowdown,
+                    pynvml.nvmlClocksEventReasonSwThermalSlowdown, pynvml.nvmlClocksEventReasonSwPowerCap)
+        except Exception:
+            return self._start_smi()
+        self.source = "nvml"
+
+        def poll():
+            while not self.stop_flag:
+                try:
+                    sm = pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM)
+                    rs = pynvml.nvmlDeviceGetCurrentClocksEventReasons(h)
+                except Exception:
+                    break
+                self.rows.append((time.time(), float(sm), float(mx),
+                                  {n for n, b in zip(self.NAMES, bits) if rs & b}))
+                time.sleep(0.002)
+
+        self.t = threading.Thread(target=poll, daemon=True)
+        self.t.start()
+
+    def _start_smi(self):
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", self.gpu_id, f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
@@ -88,27 +136,7 @@ class ClockSampler:
         except Exception:
             self.proc = None
             return
-        self.t = threading.Thread(target=self._read, daemon=True)
-        self.t.start()
-
-    def _read(self):
-        for line in self.proc.stdout:
-            parts = [p.strip() for p in line.split(",")]
-            if len(parts) == 7:
-                self.rows.append((time.time(), parts))
-
-    def stop(self):
-        if self.proc is not None:
-            self.proc.terminate()
-            try:
-                self.proc.wait(timeout=5)
-            except Exception:
-                self.proc.kill()
-
-    def summary(self, t0: float, t1: float):
-        rows = [r for (t, r) in self.rows if t0 - 0.15 <= t <= t1 + 0.15] or [r for (_, r) in self.rows]
-        if not rows:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        self.source = "nvidia-smi"
 
         def num(x):
             try:
@@ -116,12 +144,36 @@ class ClockSampler:
             except ValueError:
                 return None
 
-        sm = [num(r[0]) for r in rows if num(r[0]) is not None]
-        mx = [num(r[1]) for r in rows if num(r[1]) is not None]
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({names[i] for r in rows for i in range(4) if r[3 + i].lower() == "active"})
+        def read():
+            for line in self.proc.stdout:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) == 7:
+                    self.rows.append((time.time(), num(parts[0]), num(parts[1]),
+                                      {n for n, v in zip(self.NAMES, parts[3:]) if v.lower() == "active"}))
+
+        self.t = threading.Thread(target=read, daemon=True)
+        self.t.start()
+
+    def stop(self):
+        self.stop_flag = True
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+        if self.t is not None:
+            self.t.join(timeout=1.0)
+
+    def summary(self, t0: float, t1: float):
+        rows = [r for r in self.rows if t0 <= r[0] <= t1] or [r for r in self.rows if t0 - 0.15 <= r[0] <= t1 + 0.15]
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        sm = [r[1] for r in rows if r[1] is not None]
+        mx = [r[2] for r in rows if r[2] is not None]
+        reasons = sorted(set().union(*[r[3] for r in rows]))
         return {"sm_mhz": float(np.median(sm)) if sm else None, "sm_max_mhz": max(mx) if mx else None,
-                "reasons": reasons, "samples": len(rows)}
+                "reasons": reasons, "samples": len(rows), "source": self.source}
 
 
 def max_over_ranks(ms: float, device) -> float:
@@ -296,10 +348,8 @@ def run_ours(args, world, rank, local):
     dom = max(kernels, key=lambda k: per_kernel[k])
     bound, amount = work[dom]
     dom_s = per_kernel[dom] * 1e-3
-    src_file = {"fwd_partial": "fwd_partial_sm100.cu", "bwd_dkdv": "bwd_partial_sm100.cu",
-                "bwd_dq": "bwd_partial_sm100.cu"}.get(dom, "merge.cu")
     tr = NCU_TRAFFIC.get(dom)
-    traffic = tr["bytes"] if tr and tr.get("src") == _src_hash(src_file) else None
+    traffic = tr["bytes"] if tr and tr.get("src") == _src_hash(dom) else None
     if bound == "tensor":
         achieved = amount / dom_s / 1e12
         roof = {"kernel": dom, "bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"],
