@@ -166,27 +166,39 @@ __device__ __forceinline__ void ds_tile(uint32_t tS, uint32_t tdP, int hf, int a
 // dkdv kernel, rows 64hf..64hf+63 of one query tile for one key (thread = TMEM
 // lane), first half of the element-wise step: P^T = exp2(s * c - lse2[row]),
 // zero for rows whose slot bit (slot = row >> lg) is clear.  P stays in pv
-// (fp32, for dS^T) and goes as bf16 pairs to packed_col() of S^T.
+// (fp32, for dS^T) and goes as bf16 pairs to packed_col() of S^T.  The rows
+// are the columns of S^T, so every element needs its own row statistic: the
+// 32 of a TMEM round trip are loaded together (eight 16-byte shared loads)
+// before the scores, not one per element inside the loop.
 template <bool kMasked>
-__device__ __forceinline__ void pt_tile(uint32_t tSt, int hf, uint32_t smask, int lg, const float4* ld4, float c,
+__device__ __forceinline__ void pt_tile(uint32_t tSt, int hf, uint32_t smask, int lg, const float* l2tile, float c,
                                         float (&pv)[64]) {
 #pragma unroll
   for (int qq = 0; qq < 2; ++qq) {   // 32 rows per TMEM round trip
     const int q = 2 * hf + qq;
+    float l2[32];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const float4 v = reinterpret_cast<const float4*>(l2tile + q * 32)[k];
+      l2[4 * k] = v.x;
+      l2[4 * k + 1] = v.y;
+      l2[4 * k + 2] = v.z;
+      l2[4 * k + 3] = v.w;
+    }
     uint32_t sv[32];
     tmem_ld32(tSt + q * 32, sv);
     tmem_wait_ld();
     reg_fence<32>(sv);
+    reg_fence<32>(reinterpret_cast<uint32_t*>(l2));
     uint32_t pp[16];
 #pragma unroll
     for (int i = 0; i < 16; ++i) {
       const int row = q * 32 + 2 * i;
-      const float4 m = ld4[row >> 1];    // lse2[row], delta[row], lse2[row + 1], delta[row + 1]
       float x0, x1;
-      ffma2(x0, x1, __uint_as_float(sv[2 * i]), __uint_as_float(sv[2 * i + 1]), c, c, -m.x, -m.z);
+      ffma2(x0, x1, __uint_as_float(sv[2 * i]), __uint_as_float(sv[2 * i + 1]), c, c, -l2[2 * i], -l2[2 * i + 1]);
       float p0, p1;
       exp2_pair((i % kPolyEvery) == 1, x0, x1, p0, p1);
-      if (kMasked) {   // rows row and row + 1 share a slot (slots hold >= 8 rows)
+      if (kMasked) {
         const bool in = (smask >> (row >> lg)) & 1u;
         p0 = in ? p0 : 0.f;
         p1 = in ? p1 : 0.f;
@@ -200,21 +212,29 @@ __device__ __forceinline__ void pt_tile(uint32_t tSt, int hf, uint32_t smask, in
 }
 
 // Second half: dS^T = P^T (dP^T - Delta[row]) as bf16 pairs to packed_col() of dP^T.
-__device__ __forceinline__ void dst_tile(uint32_t tdPt, int hf, const float4* ld4, const float (&pv)[64]) {
+__device__ __forceinline__ void dst_tile(uint32_t tdPt, int hf, const float* dltile, const float (&pv)[64]) {
 #pragma unroll
   for (int qq = 0; qq < 2; ++qq) {
     const int q = 2 * hf + qq;
+    float dl[32];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const float4 v = reinterpret_cast<const float4*>(dltile + q * 32)[k];
+      dl[4 * k] = v.x;
+      dl[4 * k + 1] = v.y;
+      dl[4 * k + 2] = v.z;
+      dl[4 * k + 3] = v.w;
+    }
     uint32_t dpv[32];
     tmem_ld32(tdPt + q * 32, dpv);
     tmem_wait_ld();
     reg_fence<32>(dpv);
+    reg_fence<32>(reinterpret_cast<uint32_t*>(dl));
     uint32_t pd[16];
 #pragma unroll
     for (int i = 0; i < 16; ++i) {
-      const int row = q * 32 + 2 * i;
-      const float4 m = ld4[row >> 1];
       float d0, d1, g0, g1;
-      fadd2(d0, d1, __uint_as_float(dpv[2 * i]), __uint_as_float(dpv[2 * i + 1]), -m.y, -m.w);
+      fadd2(d0, d1, __uint_as_float(dpv[2 * i]), __uint_as_float(dpv[2 * i + 1]), -dl[2 * i], -dl[2 * i + 1]);
       fmul2(g0, g1, pv[qq * 32 + 2 * i], pv[qq * 32 + 2 * i + 1], d0, d1);
       pd[i] = pack_bf16(g0, g1);
     }
@@ -244,7 +264,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* sV = smem + kTile;
   uint8_t* sQ = smem + 2 * kTile;   // [2 stages]
   uint8_t* sdO = smem + 4 * kTile;  // [2 stages]
-  float2* meta_ld = reinterpret_cast<float2*>(smem + 6 * kTile);             // [2][128] (lse2, delta) per row
+  float* meta_l2 = reinterpret_cast<float*>(smem + 6 * kTile);               // [2][128] lse2 per row
+  float* meta_dl = reinterpret_cast<float*>(smem + 6 * kTile + 1024);        // [2][128] delta per row
   int2* meta_slot = reinterpret_cast<int2*>(smem + 6 * kTile + 2048);         // [2][16] (lo, hi) per slot
   DkdvBars* B = reinterpret_cast<DkdvBars*>(smem + kOffBars);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -385,7 +406,8 @@ __global__ void __launch_bounds__(kThreads, 1)
               l2 = (L == -INFINITY) ? INFINITY : L * kLog2e;
               dl = delta[m.qrow];
             }
-            meta_ld[s * 128 + rr] = make_float2(l2, dl);
+            meta_l2[s * 128 + rr] = l2;
+            meta_dl[s * 128 + rr] = dl;
             if (rr % rps == 0) meta_slot[s * 16 + rr / rps] = make_int2(m.lo, m.hi);
           }
           warp_arrive(&B->meta_ready[s]);
@@ -442,19 +464,18 @@ __global__ void __launch_bounds__(kThreads, 1)
           const bool all_in = __all_sync(0xffffffffu, (smask & all) == all);
           if (!warp_wait(&B->st_ready, st_cnt & 1, wctx, 2 * 10000 + __LINE__)) { ok = false; break; }
           tc_fence_after();
-          const float4* ld4 = reinterpret_cast<const float4*>(meta_ld + s * 128);
           float pv[64];
           if (all_in)
-            pt_tile<false>(tSt, hf, smask, lg, ld4, scale_log2, pv);
+            pt_tile<false>(tSt, hf, smask, lg, meta_l2 + s * 128, scale_log2, pv);
           else
-            pt_tile<true>(tSt, hf, smask, lg, ld4, scale_log2, pv);
+            pt_tile<true>(tSt, hf, smask, lg, meta_l2 + s * 128, scale_log2, pv);
           tmem_wait_st();
           tc_fence_before();
           warp_arrive(&B->pt_ready);
           if (!warp_wait(&B->dpt_ready, st_cnt & 1, wctx, 2 * 10000 + __LINE__)) { ok = false; break; }
           ++st_cnt;
           tc_fence_after();
-          dst_tile(tdPt, hf, ld4, pv);
+          dst_tile(tdPt, hf, meta_dl + s * 128, pv);
           tmem_wait_st();
           tc_fence_before();
           warp_arrive(&B->dst_ready);
