@@ -36,6 +36,7 @@
 // read yet.  Waits are bounded; a timeout is recorded in the plan's status word
 // and every role winds down.
 #include <cfloat>
+#include <cstring>
 
 #include "sm100.cuh"
 #include "splitkv.h"
@@ -256,6 +257,7 @@ constexpr int kDkdvNumBars = 17;
 __global__ void __launch_bounds__(kThreads, 1)
     bwd_dkdv_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_do,
                           const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                          const __grid_constant__ CUtensorMap tm_dk, const __grid_constant__ CUtensorMap tm_dv,
                           DevPlan p, const float* __restrict__ lse, const float* __restrict__ delta, float scale,
                           float* __restrict__ dk, float* __restrict__ dv) {
   extern __shared__ uint8_t smem_raw[];
@@ -494,12 +496,27 @@ __global__ void __launch_bounds__(kThreads, 1)
           ++dkv_cnt;
           tc_fence_after();
           float* scratch = reinterpret_cast<float*>(smem + kOffScratch) + (warp - 4) * 512;
+          if (__all_sync(0xffffffffu, own)) {
+            // the warp's 32 keys all belong to this chunk (and lie below N): bulk
+            // tensor stores of 32 keys x 16 columns
+            const CUtensorMap* map = hf == 0 ? &tm_dk : &tm_dv;
 #pragma unroll 1
-          for (int cc = 0; cc < D / 16; ++cc) {
-            uint32_t a[16];
-            tmem_ld16(tAcc + cc * 16, a);
-            tmem_wait_ld();
-            warp_store_rows<16>(scratch, reinterpret_cast<const float*>(a), f, own ? dst + cc * 16 : nullptr);
+            for (int cc = 0; cc < D / 16; ++cc) {
+              uint32_t a[16];
+              tmem_ld16(tAcc + cc * 16, a);
+              tmem_wait_ld();
+              reg_fence<16>(a);
+              warp_bulk_store16<0>(scratch, a, f, map, cc * 16, g, k0 + ((warp & 3) << 5));
+            }
+          } else {
+#pragma unroll 1
+            for (int cc = 0; cc < D / 16; ++cc) {
+              uint32_t a[16];
+              tmem_ld16(tAcc + cc * 16, a);
+              tmem_wait_ld();
+              reg_fence<16>(a);
+              warp_store_rows<16>(scratch, reinterpret_cast<const float*>(a), f, own ? dst + cc * 16 : nullptr);
+            }
           }
           tc_fence_before();
           warp_arrive(&B->dkv_free);
@@ -508,6 +525,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
     }
+    // bulk stores of this warp complete before the CTA exits
+    if (lane == 0) bulk_wait0();
+    __syncwarp();
     if (!ok) *abort_flag = 1;
   }
   tc_fence_before();
@@ -562,8 +582,8 @@ struct TileIter {
 __global__ void __launch_bounds__(kThreads, 1)
     bwd_dq_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_do,
                         const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
-                        DevPlan p, const float* __restrict__ lse, const float* __restrict__ delta, float scale,
-                        float* __restrict__ dq_part) {
+                        const __grid_constant__ CUtensorMap tm_dq, DevPlan p, const float* __restrict__ lse,
+                        const float* __restrict__ delta, float scale, int bulk, float* __restrict__ dq_part) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sQ = smem;
@@ -766,18 +786,37 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!warp_wait(&B->dq_ready, dq_cnt & 1, wctx, 2 * 10000 + __LINE__)) { ok = false; break; }
       ++dq_cnt;
       tc_fence_after();
-      float* dst = dq_part + size_t(m.rec) * D + hf * 64;
       float* scratch = reinterpret_cast<float*>(smem + kOffScratch) + (warp - 4) * 512;
+      if (bulk) {
+        // the warp's 32 rows are 32/G whole tokens of one block, all G heads of KV
+        // head g (valid is warp-uniform): bulk tensor stores of 32 x 16 boxes
+        const int z0 = __shfl_sync(0xffffffffu, m.valid ? m.rec / p.Hq : 0, 0);
+        const bool wv = __shfl_sync(0xffffffffu, m.valid ? 1 : 0, 0) != 0;
 #pragma unroll 1
-      for (int cc = 0; cc < 4; ++cc) {
-        uint32_t v[16];
-        tmem_ld16(tdQ + cc * 16, v);
-        tmem_wait_ld();
-        warp_store_rows<16>(scratch, reinterpret_cast<const float*>(v), scale, m.valid ? dst + cc * 16 : nullptr);
+        for (int cc = 0; cc < 4; ++cc) {
+          uint32_t v[16];
+          tmem_ld16(tdQ + cc * 16, v);
+          tmem_wait_ld();
+          reg_fence<16>(v);
+          warp_bulk_store16<0>(scratch, v, scale, &tm_dq, hf * 64 + cc * 16, g * p.G, z0, wv);
+        }
+      } else {
+        float* dst = dq_part + size_t(m.rec) * D + hf * 64;
+#pragma unroll 1
+        for (int cc = 0; cc < 4; ++cc) {
+          uint32_t v[16];
+          tmem_ld16(tdQ + cc * 16, v);
+          tmem_wait_ld();
+          reg_fence<16>(v);
+          warp_store_rows<16>(scratch, reinterpret_cast<const float*>(v), scale, m.valid ? dst + cc * 16 : nullptr);
+        }
       }
       tc_fence_before();
       warp_arrive(&B->dq_free);
     }
+    // bulk stores of this warp complete before the CTA exits
+    if (lane == 0) bulk_wait0();
+    __syncwarp();
     if (!ok) *abort_flag = 1;
   }
   tc_fence_before();
@@ -796,22 +835,31 @@ bool bwd_sm100_supported(const DevPlan& p) {
 cudaError_t launch_bwd_partial_sm100(const DevPlan& p, const uint16_t* q, const uint16_t* k, const uint16_t* v,
                                      const uint16_t* dout, const float* lse, const float* delta, float scale,
                                      float* dk, float* dv, float* dq_part, cudaStream_t s, int which) {
-  CUtensorMap tq, tdo, tk, tv;
+  CUtensorMap tq, tdo, tk, tv, tdk, tdv, tdq;
   if (!make_bf16_map_3d(&tq, q, D, p.Hq, p.Nq, p.G, p.bs) || !make_bf16_map_3d(&tdo, dout, D, p.Hq, p.Nq, p.G, p.bs) ||
-      !make_bf16_map_3d(&tk, k, D, p.Hkv, p.N, 1, BT) || !make_bf16_map_3d(&tv, v, D, p.Hkv, p.N, 1, BT))
+      !make_bf16_map_3d(&tk, k, D, p.Hkv, p.N, 1, BT) || !make_bf16_map_3d(&tv, v, D, p.Hkv, p.N, 1, BT) ||
+      !make_f32_map_3d(&tdk, dk, D, p.Hkv, p.N, 16, 1, 32) || !make_f32_map_3d(&tdv, dv, D, p.Hkv, p.N, 16, 1, 32))
     return cudaErrorInvalidValue;
+  // dq partial records by bulk stores when a warp's 32 rows are 32/G whole tokens of one block
+  const bool bulk_dq = 32 % p.G == 0 && (p.G * p.bs) % 32 == 0 && p.E > 0;
+  if (bulk_dq) {
+    if (!make_f32_map_3d(&tdq, dq_part, D, p.Hq, uint64_t(p.E) * p.bs, 16, p.G, 32 / p.G)) return cudaErrorInvalidValue;
+  } else {
+    memset(&tdq, 0, sizeof(tdq));
+  }
   cudaError_t e = cudaFuncSetAttribute(bwd_dkdv_sm100_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        int(kSmemBytes));
   if (e != cudaSuccess) return e;
   e = cudaFuncSetAttribute(bwd_dq_sm100_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(kSmemBytes));
   if (e != cudaSuccess) return e;
   if (which != 2) {
-    bwd_dkdv_sm100_kernel<<<p.Wb, kThreads, kSmemBytes, s>>>(tq, tdo, tk, tv, p, lse, delta, scale, dk, dv);
+    bwd_dkdv_sm100_kernel<<<p.Wb, kThreads, kSmemBytes, s>>>(tq, tdo, tk, tv, tdk, tdv, p, lse, delta, scale, dk, dv);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
   if (which != 1) {
-    bwd_dq_sm100_kernel<<<p.W, kThreads, kSmemBytes, s>>>(tq, tdo, tk, tv, p, lse, delta, scale, dq_part);
+    bwd_dq_sm100_kernel<<<p.W, kThreads, kSmemBytes, s>>>(tq, tdo, tk, tv, tdq, p, lse, delta, scale,
+                                                          bulk_dq ? 1 : 0, dq_part);
     e = cudaGetLastError();
   }
   return e;

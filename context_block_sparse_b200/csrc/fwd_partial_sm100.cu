@@ -483,13 +483,13 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int cch = 0; cch < D / 32; cch += 2) {
             tmem_ld32(tO + (cch + 1) * 32, vb);
-            warp_bulk_store16(scratch, va, inv, &tm_o, cch * 32, g * p.G, z0);
-            warp_bulk_store16(scratch + 512, va + 16, inv, &tm_o, cch * 32 + 16, g * p.G, z0);
+            warp_bulk_store16<1>(scratch, va, inv, &tm_o, cch * 32, g * p.G, z0);
+            warp_bulk_store16<1>(scratch + 512, va + 16, inv, &tm_o, cch * 32 + 16, g * p.G, z0);
             tmem_wait_ld();
             reg_fence<32>(vb);
             if (cch + 2 < D / 32) tmem_ld32(tO + (cch + 2) * 32, va);
-            warp_bulk_store16(scratch, vb, inv, &tm_o, (cch + 1) * 32, g * p.G, z0);
-            warp_bulk_store16(scratch + 512, vb + 16, inv, &tm_o, (cch + 1) * 32 + 16, g * p.G, z0);
+            warp_bulk_store16<1>(scratch, vb, inv, &tm_o, (cch + 1) * 32, g * p.G, z0);
+            warp_bulk_store16<1>(scratch + 512, vb + 16, inv, &tm_o, (cch + 1) * 32 + 16, g * p.G, z0);
             tmem_wait_ld();
             reg_fence<32>(va);
           }

@@ -128,14 +128,16 @@ __device__ __forceinline__ void fence_async_smem() {
 
 // One warp's 32 rows x 16 fp32 columns (vals[0..16) of the lane's row, times
 // mul) through a 2 KB shared buffer laid out as the 64-byte-swizzled box of
-// `map` (row = lane), then one bulk tensor store at (x, y, z).  A warp
-// alternates two such buffers: before a buffer is rewritten, the store issued
-// from it two calls earlier must have read it (wait_group.read 1; lane 0 owns
-// the bulk groups).  The buffer must be 512-byte aligned.
+// `map` (row = lane), then one bulk tensor store at (x, y, z) when `store`.
+// Before the buffer is rewritten, at most kPending of this lane-0's earlier bulk
+// stores may still be reading shared memory: 1 for a warp alternating two
+// buffers, 0 for a warp with one.  The buffer must be 512-byte aligned; lane 0
+// owns the bulk groups (bulk_wait0 before the CTA exits).
+template <int kPending>
 __device__ __forceinline__ void warp_bulk_store16(float* buf, const uint32_t* vals, float mul,
-                                                  const CUtensorMap* map, int x, int y, int z) {
+                                                  const CUtensorMap* map, int x, int y, int z, bool store = true) {
   const int lane = threadIdx.x & 31;
-  if (lane == 0) asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
+  if (lane == 0) asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(kPending) : "memory");
   __syncwarp();
 #pragma unroll
   for (int g = 0; g < 4; ++g) {
@@ -145,10 +147,11 @@ __device__ __forceinline__ void warp_bulk_store16(float* buf, const uint32_t* va
   }
   fence_async_smem();
   __syncwarp();
-  if (lane == 0) {
+  if (lane == 0 && store) {
     tma_store_3d(map, buf, x, y, z);
     bulk_commit();
   }
+  __syncwarp();
 }
 
 // Three-input maximum (one instruction on sm_100).
