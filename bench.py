@@ -403,6 +403,8 @@ def run_ours(args, world, rank, local):
         "clocks": clocks,
     }
 
+    if rank == 0:
+        result["device_lpt"] = device_lpt_report(skv, w)
     if not args.no_e2e:
         result["e2e"] = run_e2e(args, w, plan, dev, stream, flops_step, world=world)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -410,6 +412,29 @@ def run_ours(args, world, rank, local):
     if world > 1:
         dist.destroy_process_group()
     return result if rank == 0 else None
+
+
+def device_lpt_report(skv, w, workers=(8, 16, 32, 64)):
+    """The planner in the pages' device regime (news page, "Balance actual attention
+    work": W devices, equal chunk counts, against leaving chunks unbalanced), on the
+    host, untimed: for each W, plan latency and max/mean load imbalance of plain LPT,
+    equal-count LPT and the contiguous assignment, over whole (chunk, KV head) items;
+    `makespan_ratio` = (1 + contiguous) / (1 + equal-count LPT), the step-time ratio the
+    imbalance alone implies."""
+    out = {}
+    for W in workers:
+        row = {}
+        for mode, eq in (("lpt", False), ("equal_count", True)):
+            plan = skv.splitkv_plan(w.sample_lens, w.anchors, w.block_size, w.num_q_heads, w.num_kv_heads,
+                                    w.head_dim, w.kv_chunk, W, num_bwd_workers=W, q_slice=0, equal_count=eq)
+            st = plan.stats()
+            row[f"{mode}_imbalance_pct"] = 100 * st["fwd_imbalance"]
+            row[f"{mode}_plan_us"] = st["plan_us"]
+            row["contiguous_imbalance_pct"] = 100 * st["contig_imbalance"]
+            plan.destroy()
+        row["makespan_ratio"] = (1 + row["contiguous_imbalance_pct"] / 100) / (1 + row["equal_count_imbalance_pct"] / 100)
+        out[str(W)] = row
+    return out
 
 
 def run_e2e(args, w, plan, dev, stream, flops_step, world=1):

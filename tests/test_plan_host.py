@@ -151,3 +151,24 @@ def test_lpt_beats_contiguous_on_skew(splitkv):
     st_ = p.stats()
     assert st_["fwd_imbalance"] < 0.05
     assert st_["contig_imbalance"] > 1.0
+
+
+@pytest.mark.parametrize("name", ["bwd", "skew"])
+def test_device_regime_report(splitkv, name):
+    """The planner in the pages' device regime (news page, "Balance actual attention
+    work": imbalance below 1 % with LPT, clearly better than leaving chunks unbalanced)
+    on whole (chunk, KV head) items for W = 8 .. 64, as bench.py reports it."""
+    import importlib.util
+    import os
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    spec = importlib.util.spec_from_file_location("_bench", os.path.join(root, "bench.py"))
+    bench = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(bench)
+    w = make_workload(name, with_grad=False)
+    rep = bench.device_lpt_report(splitkv, w)
+    assert sorted(rep, key=int) == ["8", "16", "32", "64"]
+    for W, row in rep.items():
+        assert row["equal_count_imbalance_pct"] < 1.0, (W, row)
+        assert row["lpt_imbalance_pct"] < 1.0, (W, row)
+        assert row["makespan_ratio"] > 1.1, (W, row)
+        assert row["equal_count_plan_us"] > 0 and row["lpt_plan_us"] > 0
