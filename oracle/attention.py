@@ -9,6 +9,10 @@ smaller side"; [digest] Abstract):
 * Allowed keys of every row of block b, head h: the context keys
   j in [S_{s(b)}, a_b) of KV head g, then the bs in-block keys
   kb[b*bs : (b+1)*bs, g] (values likewise).
+* Reading B (`block_keys_in_context`): the block's own tokens are the context
+  positions after its anchor; the allowed keys are the context keys
+  j in [S_{s(b)}, min(a_b + bs, S_{s(b)} + L_{s(b)})) and nothing else (kb, vb
+  unused; dkb, dvb returned as None).
 * s = scale * q . key; O = softmax(s) . values; LSE = log(sum(exp(s))) (natural
   log).  Gradients are the analytic gradients of O with respect to q, k, v, kb,
   vb contracted with dout.
@@ -40,14 +44,17 @@ def _group(Hq: int, Hkv: int) -> int:
     return Hq // Hkv
 
 
-def _block_keys(k, v, kb, vb, S, a, b, bs, g):
+def _block_keys(k, v, kb, vb, S, a, b, bs, g, in_context=False):
+    if in_context:
+        return k[S:a, g, :], v[S:a, g, :]
     keys = np.concatenate([k[S:a, g, :], kb[b * bs:(b + 1) * bs, g, :]], axis=0)
     vals = np.concatenate([v[S:a, g, :], vb[b * bs:(b + 1) * bs, g, :]], axis=0)
     return keys, vals
 
 
 def attention_fwd(q, k, v, kb, vb, sample_lens, anchors, block_size: int, scale: float,
-                  blocks: Optional[Iterable[int]] = None) -> Tuple[np.ndarray, np.ndarray]:
+                  blocks: Optional[Iterable[int]] = None, block_keys_in_context: bool = False
+                  ) -> Tuple[np.ndarray, np.ndarray]:
     """O [Nq, Hq, d] and LSE [Nq, Hq] by the plain definition (all inputs float64).
 
     `blocks` restricts the work to some blocks; other rows are left NaN.
@@ -58,14 +65,14 @@ def attention_fwd(q, k, v, kb, vb, sample_lens, anchors, block_size: int, scale:
     bs = int(block_size)
     O = np.full((Nq, Hq, d), np.nan)
     LSE = np.full((Nq, Hq), np.nan)
-    iv = context_interval(sample_lens, anchors)
+    iv = context_interval(sample_lens, anchors, bs, block_keys_in_context)
     todo = range(len(iv)) if blocks is None else blocks
     for b in todo:
         S, a = iv[b]
         rows = slice(b * bs, (b + 1) * bs)
         for h in range(Hq):
             g = h // G
-            keys, vals = _block_keys(k, v, kb, vb, S, a, b, bs, g)
+            keys, vals = _block_keys(k, v, kb, vb, S, a, b, bs, g, block_keys_in_context)
             s = scale * (q[rows, h, :] @ keys.T)              # [bs, n_keys]
             m = s.max(axis=1, keepdims=True)
             p = np.exp(s - m)
@@ -76,7 +83,8 @@ def attention_fwd(q, k, v, kb, vb, sample_lens, anchors, block_size: int, scale:
 
 
 def attention_bwd(q, k, v, kb, vb, dout, sample_lens, anchors, block_size: int, scale: float,
-                  blocks: Optional[Iterable[int]] = None) -> Dict[str, np.ndarray]:
+                  blocks: Optional[Iterable[int]] = None, block_keys_in_context: bool = False
+                  ) -> Dict[str, np.ndarray]:
     """Analytic gradients dq, dk, dv, dkb, dvb (float64) of sum(dout * O).
 
     Per block b and head h with P = softmax(s) over the allowed keys:
@@ -93,16 +101,16 @@ def attention_bwd(q, k, v, kb, vb, dout, sample_lens, anchors, block_size: int, 
     dq = np.zeros_like(q)
     dk = np.zeros_like(k)
     dv = np.zeros_like(v)
-    dkb = np.zeros_like(kb)
-    dvb = np.zeros_like(vb)
-    iv = context_interval(sample_lens, anchors)
+    dkb = None if block_keys_in_context else np.zeros_like(kb)
+    dvb = None if block_keys_in_context else np.zeros_like(vb)
+    iv = context_interval(sample_lens, anchors, bs, block_keys_in_context)
     for b in (range(len(iv)) if blocks is None else blocks):
         S, a = iv[b]
         rows = slice(b * bs, (b + 1) * bs)
         n_ctx = a - S
         for h in range(Hq):
             g = h // G
-            keys, vals = _block_keys(k, v, kb, vb, S, a, b, bs, g)
+            keys, vals = _block_keys(k, v, kb, vb, S, a, b, bs, g, block_keys_in_context)
             s = scale * (q[rows, h, :] @ keys.T)
             p = np.exp(s - s.max(axis=1, keepdims=True))
             P = p / p.sum(axis=1, keepdims=True)
@@ -115,8 +123,9 @@ def attention_bwd(q, k, v, kb, vb, dout, sample_lens, anchors, block_size: int, 
             dkeys = scale * (dS.T @ q[rows, h, :])
             dk[S:a, g, :] += dkeys[:n_ctx]
             dv[S:a, g, :] += dvals[:n_ctx]
-            dkb[rows, g, :] += dkeys[n_ctx:]
-            dvb[rows, g, :] += dvals[n_ctx:]
+            if not block_keys_in_context:
+                dkb[rows, g, :] += dkeys[n_ctx:]
+                dvb[rows, g, :] += dvals[n_ctx:]
     return {"dq": dq, "dk": dk, "dv": dv, "dkb": dkb, "dvb": dvb}
 
 
@@ -149,8 +158,8 @@ def merge(records: List[Tuple[np.ndarray, np.ndarray, np.ndarray]]) -> Tuple[np.
     return out, lse
 
 
-def chunk_partials(q, k, v, sample_lens, anchors, block_size: int, kv_chunk: int, scale: float
-                   ) -> List[Dict]:
+def chunk_partials(q, k, v, sample_lens, anchors, block_size: int, kv_chunk: int, scale: float,
+                   block_keys_in_context: bool = False) -> List[Dict]:
     """Per (chunk, block) partial records over the block's keys inside the chunk.
 
     Returns a list in chunk_entries order of dicts with keys c, b, lo, hi,
@@ -161,7 +170,7 @@ def chunk_partials(q, k, v, sample_lens, anchors, block_size: int, kv_chunk: int
     G = _group(Hq, Hkv)
     bs = int(block_size)
     out = []
-    for (c, b, lo, hi) in chunk_entries(sample_lens, anchors, kv_chunk):
+    for (c, b, lo, hi) in chunk_entries(sample_lens, anchors, kv_chunk, bs, block_keys_in_context):
         rows = slice(b * bs, (b + 1) * bs)
         m = np.zeros((bs, Hq))
         l = np.zeros((bs, Hq))
@@ -192,18 +201,21 @@ def block_partials(q, kb, vb, num_blocks: int, block_size: int, scale: float):
     return m, l, O
 
 
-def split_fwd(q, k, v, kb, vb, sample_lens, anchors, block_size: int, kv_chunk: int, scale: float):
-    """Forward by the split form: chunk partials + in-block partial, then merge."""
+def split_fwd(q, k, v, kb, vb, sample_lens, anchors, block_size: int, kv_chunk: int, scale: float,
+              block_keys_in_context: bool = False):
+    """Forward by the split form: chunk partials (+ the in-block partial under reading A), then merge."""
     Nq, Hq, d = q.shape
     bs = int(block_size)
     A = len(anchors)
-    parts = chunk_partials(q, k, v, sample_lens, anchors, bs, kv_chunk, scale)
-    bm, bl, bO = block_partials(q, kb, vb, A, bs, scale)
+    parts = chunk_partials(q, k, v, sample_lens, anchors, bs, kv_chunk, scale, block_keys_in_context)
+    if not block_keys_in_context:
+        bm, bl, bO = block_partials(q, kb, vb, A, bs, scale)
     O = np.zeros((Nq, Hq, d))
     LSE = np.zeros((Nq, Hq))
     for b in range(A):
         rows = slice(b * bs, (b + 1) * bs)
-        recs = [(bm[rows].reshape(-1), bl[rows].reshape(-1), bO[rows].reshape(-1, d))]
+        recs = [] if block_keys_in_context else [(bm[rows].reshape(-1), bl[rows].reshape(-1),
+                                                   bO[rows].reshape(-1, d))]
         for p in parts:
             if p["b"] == b:
                 recs.append((p["m"].reshape(-1), p["l"].reshape(-1), p["O"].reshape(-1, d)))

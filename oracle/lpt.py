@@ -32,21 +32,21 @@ from .mask import chunk_entries, chunk_pairs
 
 
 def work_items(sample_lens, anchors, block_size: int, kv_chunk: int, num_q_heads: int,
-               num_kv_heads: int, q_slice: int = 0, rows_per_tile: int = 128
-               ) -> List[Tuple[Tuple[int, int, int], int]]:
+               num_kv_heads: int, q_slice: int = 0, rows_per_tile: int = 128,
+               block_keys_in_context: bool = False) -> List[Tuple[Tuple[int, int, int], int]]:
     """All work items ((c, g, slice), cost), zero-cost ones included."""
     G = num_q_heads // num_kv_heads
     bs = int(block_size)
     items = []
     if q_slice <= 0:
-        pairs = chunk_pairs(sample_lens, anchors, bs, kv_chunk)
+        pairs = chunk_pairs(sample_lens, anchors, bs, kv_chunk, block_keys_in_context)
         for c, p in enumerate(pairs):
             for g in range(num_kv_heads):
                 items.append(((c, g, 0), int(G * p)))
         return items
     blocks_per_tile = rows_per_tile // (G * bs)
     per_chunk: Dict[int, list] = {}
-    for (c, b, lo, hi) in chunk_entries(sample_lens, anchors, kv_chunk):
+    for (c, b, lo, hi) in chunk_entries(sample_lens, anchors, kv_chunk, bs, block_keys_in_context):
         per_chunk.setdefault(c, []).append((lo, hi, b))
     for c in sorted(per_chunk):
         ents = sorted(per_chunk[c])

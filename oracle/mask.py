@@ -5,6 +5,13 @@ tokens; each block attends to the preceding context within its own sample and
 to all tokens inside the block.  Samples are packed back to back into one
 context (sample s occupies [S_s, S_s + L_s)).
 
+Where the block's own tokens live is not fixed by the pages.  Reading A (the
+default): they are the draft block's own keys and values, separate from the
+context, so a block's context interval ends at its anchor.  Reading B
+(`block_keys_in_context`): they are the context positions after the anchor, so
+the interval runs on to min(a_b + bs, end of the sample) and the block has no
+keys besides the context.
+
 [news] "Balance actual attention work": the context is cut into chunks and a
 chunk's cost is its actual attention usage, i.e. the number of allowed
 (query, key) pairs that fall into it.  Chunks are fixed-length pieces of the
@@ -45,23 +52,33 @@ def anchor_sample(sample_lens, anchors) -> List[int]:
     return out
 
 
-def context_interval(sample_lens, anchors) -> List[Tuple[int, int]]:
-    """Allowed context keys of block b: [S_{s(b)}, a_b) (preceding context of its own sample)."""
+def context_interval(sample_lens, anchors, block_size: int = 0,
+                     block_keys_in_context: bool = False) -> List[Tuple[int, int]]:
+    """Allowed context keys of block b: [S_{s(b)}, a_b) (preceding context of its own sample);
+    under reading B, [S_{s(b)}, min(a_b + bs, S_{s(b)} + L_{s(b)}))."""
     starts = sample_starts(sample_lens)
-    return [(starts[s], int(a)) for s, a in zip(anchor_sample(sample_lens, anchors), anchors)]
+    out = []
+    for s, a in zip(anchor_sample(sample_lens, anchors), anchors):
+        end = int(a)
+        if block_keys_in_context:
+            end = min(int(a) + int(block_size), starts[s] + int(sample_lens[s]))
+        out.append((starts[s], end))
+    return out
 
 
 def num_chunks(context_len: int, kv_chunk: int) -> int:
     return (int(context_len) + kv_chunk - 1) // kv_chunk
 
 
-def chunk_entries(sample_lens, anchors, kv_chunk: int) -> List[Tuple[int, int, int, int]]:
+def chunk_entries(sample_lens, anchors, kv_chunk: int, block_size: int = 0,
+                  block_keys_in_context: bool = False) -> List[Tuple[int, int, int, int]]:
     """Every (chunk c, block b, lo, hi) whose clipped interval [lo, hi) is non-empty.
 
-    lo = max(S_s, c*C), hi = min(a_b, (c+1)*C, N).  Ordered by chunk, then block.
+    lo = max(S_s, c*C), hi = min(e_b, (c+1)*C, N), with e_b the interval end
+    (a_b, or the reading-B end).  Ordered by chunk, then block.
     """
     N = int(np.sum(sample_lens))
-    iv = context_interval(sample_lens, anchors)
+    iv = context_interval(sample_lens, anchors, block_size, block_keys_in_context)
     out = []
     for c in range(num_chunks(N, kv_chunk)):
         c0, c1 = c * kv_chunk, min((c + 1) * kv_chunk, N)
@@ -72,29 +89,31 @@ def chunk_entries(sample_lens, anchors, kv_chunk: int) -> List[Tuple[int, int, i
     return out
 
 
-def chunk_pairs(sample_lens, anchors, block_size: int, kv_chunk: int) -> np.ndarray:
+def chunk_pairs(sample_lens, anchors, block_size: int, kv_chunk: int,
+                block_keys_in_context: bool = False) -> np.ndarray:
     """pairs_c: allowed (query row, context key) pairs inside each chunk, per query head.
 
     Evaluated straight from the definition: for every block, mark the context
     keys it may read, count the marks that fall into each chunk, and multiply
-    by the block's bs query rows.  (The in-block keys are not context keys and
-    belong to no chunk.)
+    by the block's bs query rows.  (Under reading A the in-block keys are not
+    context keys and belong to no chunk.)
     """
     N = int(np.sum(sample_lens))
     nc = num_chunks(N, kv_chunk)
     counts = np.zeros(nc, dtype=np.int64)
     keys = np.arange(N, dtype=np.int64)
     chunk_of_key = keys // kv_chunk
-    for S, a in context_interval(sample_lens, anchors):
+    for S, a in context_interval(sample_lens, anchors, block_size, block_keys_in_context):
         allowed = (keys >= S) & (keys < a)
         counts += np.bincount(chunk_of_key[allowed], minlength=nc).astype(np.int64)
     return counts * int(block_size)
 
 
-def chunk_pairs_loops(sample_lens, anchors, block_size: int, kv_chunk: int) -> List[int]:
+def chunk_pairs_loops(sample_lens, anchors, block_size: int, kv_chunk: int,
+                      block_keys_in_context: bool = False) -> List[int]:
     """Same count as chunk_pairs by a plain triple loop (chunks x blocks x keys); small inputs only."""
     N = int(np.sum(sample_lens))
-    iv = context_interval(sample_lens, anchors)
+    iv = context_interval(sample_lens, anchors, block_size, block_keys_in_context)
     out = []
     for c in range(num_chunks(N, kv_chunk)):
         total = 0

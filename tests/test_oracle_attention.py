@@ -221,7 +221,7 @@ def test_planted_inclusive_anchor_is_caught(monkeypatch):
     assert _fwd_matches_dense(lens, anchors, bs, t)
     orig = mask.context_interval
     monkeypatch.setattr(att, "context_interval",
-                        lambda L, A: [(S, a + 1) for (S, a) in orig(L, A)])
+                        lambda L, A, *rest: [(S, a + 1) for (S, a) in orig(L, A, *rest)])
     assert not _fwd_matches_dense(lens, anchors, bs, t)
 
 
@@ -230,7 +230,8 @@ def test_planted_wrong_kv_head_is_caught(monkeypatch):
     assert _fwd_matches_dense(lens, anchors, bs, t)
     orig = att._block_keys
     monkeypatch.setattr(att, "_block_keys",
-                        lambda k, v, kb, vb, S, a, b, bs_, g: orig(k, v, kb, vb, S, a, b, bs_, (g + 1) % 2))
+                        lambda k, v, kb, vb, S, a, b, bs_, g, *rest: orig(k, v, kb, vb, S, a, b, bs_, (g + 1) % 2,
+                                                                           *rest))
     assert not _fwd_matches_dense(lens, anchors, bs, t)
 
 
@@ -238,7 +239,7 @@ def test_planted_swapped_key_value_is_caught(monkeypatch):
     lens, anchors, bs, t = _problem(3)
     orig = att._block_keys
     monkeypatch.setattr(att, "_block_keys",
-                        lambda k, v, kb, vb, S, a, b, bs_, g: orig(k, v, vb, kb, S, a, b, bs_, g))
+                        lambda k, v, kb, vb, S, a, b, bs_, g, *rest: orig(k, v, vb, kb, S, a, b, bs_, g, *rest))
     assert not _fwd_matches_dense(lens, anchors, bs, t)
 
 
