@@ -24,7 +24,7 @@ from . import _abi
 from ._abi import (  # noqa: F401
     DTYPE_BF16, DTYPE_F32, EXPORT_BWD_LOADS, EXPORT_BWD_SCHEDULE, EXPORT_CHUNK_PAIRS,
     EXPORT_CONTIG_LOADS, EXPORT_ENTRIES, EXPORT_FWD_LOADS, EXPORT_FWD_SCHEDULE,
-    FLAG_EQUAL_COUNT, STATIC_SCRATCH_BYTES, WS_BWD, WS_FWD,
+    FLAG_BLOCK_KEYS_IN_CONTEXT, FLAG_EQUAL_COUNT, STATIC_SCRATCH_BYTES, WS_BWD, WS_FWD,
 )
 
 _lib = _abi.load()
@@ -67,6 +67,8 @@ def _ptr(t) -> Optional[int]:
 
 def _bf16_ptr(t) -> int:
     import torch
+    if t is None:
+        return None
     if t.dtype != torch.bfloat16:
         raise ValueError("q, k, v, kb, vb and dout must be bfloat16")
     return _ptr(t)
@@ -74,6 +76,8 @@ def _bf16_ptr(t) -> int:
 
 def _f32_ptr(t) -> int:
     import torch
+    if t is None:
+        return None
     if t.dtype != torch.float32:
         raise ValueError("lse, dq, dk, dv, dkb and dvb must be float32")
     return _ptr(t)
@@ -125,7 +129,7 @@ class Plan:
 
 
 def _problem(sample_lens, anchors, block_size, num_q_heads, num_kv_heads, head_dim, kv_chunk,
-             num_workers, num_bwd_workers, q_slice, equal_count):
+             num_workers, num_bwd_workers, q_slice, equal_count, block_keys_in_context=False):
     lens = np.ascontiguousarray(sample_lens, dtype=np.int32)
     anc = np.ascontiguousarray(anchors, dtype=np.int32)
     p = _abi.Problem()
@@ -141,16 +145,18 @@ def _problem(sample_lens, anchors, block_size, num_q_heads, num_kv_heads, head_d
     p.num_workers = int(num_workers)
     p.num_bwd_workers = int(num_bwd_workers)
     p.q_slice = int(q_slice)
-    p.flags = FLAG_EQUAL_COUNT if equal_count else 0
+    p.flags = (FLAG_EQUAL_COUNT if equal_count else 0) | (FLAG_BLOCK_KEYS_IN_CONTEXT if block_keys_in_context else 0)
     return p, (lens, anc)
 
 
 def splitkv_plan(sample_lens: Sequence[int], anchors: Sequence[int], block_size: int, num_q_heads: int,
                  num_kv_heads: int, head_dim: int, kv_chunk: int, num_workers: int,
-                 num_bwd_workers: int = 0, q_slice: int = 0, equal_count: bool = False) -> Plan:
-    """Host-side mask metadata + LPT schedules (no CUDA call)."""
+                 num_bwd_workers: int = 0, q_slice: int = 0, equal_count: bool = False,
+                 block_keys_in_context: bool = False) -> Plan:
+    """Host-side mask metadata + LPT schedules (no CUDA call).  block_keys_in_context
+    selects reading B of the block keys (SPLITKV_FLAG_BLOCK_KEYS_IN_CONTEXT)."""
     p, keep = _problem(sample_lens, anchors, block_size, num_q_heads, num_kv_heads, head_dim, kv_chunk,
-                       num_workers, num_bwd_workers, q_slice, equal_count)
+                       num_workers, num_bwd_workers, q_slice, equal_count, block_keys_in_context)
     h = ctypes.c_void_p()
     _check("splitkv_plan", _lib.splitkv_plan(ctypes.byref(p), ctypes.byref(h)))
     return Plan(h, p, keep)
@@ -162,7 +168,8 @@ def splitkv_plan_update(plan: Plan, sample_lens, anchors, **kw) -> Plan:
     args = dict(block_size=old.block_size, num_q_heads=old.num_q_heads, num_kv_heads=old.num_kv_heads,
                 head_dim=old.head_dim, kv_chunk=old.kv_chunk, num_workers=old.num_workers,
                 num_bwd_workers=old.num_bwd_workers, q_slice=old.q_slice,
-                equal_count=bool(old.flags & FLAG_EQUAL_COUNT))
+                equal_count=bool(old.flags & FLAG_EQUAL_COUNT),
+                block_keys_in_context=bool(old.flags & FLAG_BLOCK_KEYS_IN_CONTEXT))
     args.update(kw)
     p, keep = _problem(sample_lens, anchors, **args)
     _check("splitkv_plan_update", _lib.splitkv_plan_update(plan.handle, ctypes.byref(p)))

@@ -21,6 +21,7 @@ ERR_NOT_UPLOADED = -6
 ERR_NO_MEMORY = -7
 
 FLAG_EQUAL_COUNT = 1
+FLAG_BLOCK_KEYS_IN_CONTEXT = 2
 
 STATIC_SCRATCH_BYTES = 16 << 20
 

@@ -38,6 +38,14 @@ bool all_aligned16(Ps... ps) {
   return ((ps != nullptr && aligned(ps, 16)) && ...);
 }
 
+// Block-key tensors (kb, vb, dkb, dvb): required under reading A; under reading B
+// they may be NULL (never read or written) and are checked only for alignment.
+template <typename... Ps>
+bool block_ptrs_ok(const DevPlan* dp, Ps... ps) {
+  if (dp->block_term) return all_aligned16(ps...);
+  return ((ps == nullptr || aligned(ps, 16)) && ...);
+}
+
 }  // namespace
 
 extern "C" {
@@ -62,7 +70,8 @@ int splitkv_merge(const splitkv_plan_t* plan, const void* q, const void* kb, con
   const DevPlan* dp = nullptr;
   int st = check_plan(plan, &dp);
   if (st != SPLITKV_OK) return st;
-  if (!all_aligned16(q, kb, vb, ws, o) || !lse || !aligned(lse, 4)) return SPLITKV_ERR_INVALID_ARG;
+  if (!all_aligned16(q, ws, o) || !block_ptrs_ok(dp, kb, vb) || !lse || !aligned(lse, 4))
+    return SPLITKV_ERR_INVALID_ARG;
   if (o_dtype != SPLITKV_DTYPE_F32 && o_dtype != SPLITKV_DTYPE_BF16) return SPLITKV_ERR_INVALID_ARG;
   const splitkv::FwdWs L = splitkv::fwd_ws_layout(dp->E, dp->bs, dp->Hq, dp->d);
   if (ws_bytes < L.total) return SPLITKV_ERR_WORKSPACE_TOO_SMALL;
@@ -131,7 +140,7 @@ int splitkv_bwd_reduce(const splitkv_plan_t* plan, const void* q, const void* kb
   const DevPlan* dp = nullptr;
   int st = check_plan(plan, &dp);
   if (st != SPLITKV_OK) return st;
-  if (!all_aligned16(q, kb, vb, dout, dq, dkb, dvb, ws) || !lse || !aligned(lse, 4))
+  if (!all_aligned16(q, dout, dq, ws) || !block_ptrs_ok(dp, kb, vb, dkb, dvb) || !lse || !aligned(lse, 4))
     return SPLITKV_ERR_INVALID_ARG;
   const splitkv::BwdWs L = splitkv::bwd_ws_layout(dp->E, dp->Nq, dp->bs, dp->Hq, dp->d);
   if (ws_bytes < L.total) return SPLITKV_ERR_WORKSPACE_TOO_SMALL;
@@ -150,7 +159,8 @@ int splitkv_attn_bwd(const splitkv_plan_t* plan, const void* q, const void* k, c
   int st = check_plan(plan, &dp);
   if (st != SPLITKV_OK) return st;
   // check everything up front so that no launch happens on a call that fails
-  if (!all_aligned16(q, k, v, kb, vb, o, dout, dq, dk, dv, dkb, dvb, ws) || !lse || !aligned(lse, 4))
+  if (!all_aligned16(q, k, v, o, dout, dq, dk, dv, ws) || !block_ptrs_ok(dp, kb, vb, dkb, dvb) || !lse ||
+      !aligned(lse, 4))
     return SPLITKV_ERR_INVALID_ARG;
   if (o_dtype != SPLITKV_DTYPE_F32 && o_dtype != SPLITKV_DTYPE_BF16) return SPLITKV_ERR_INVALID_ARG;
   const splitkv::BwdWs L = splitkv::bwd_ws_layout(dp->E, dp->Nq, dp->bs, dp->Hq, dp->d);

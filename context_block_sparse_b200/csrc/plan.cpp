@@ -75,7 +75,7 @@ int validate(const splitkv_problem* p) {
       p->num_bwd_workers < 0 || p->q_slice < 0)
     return SPLITKV_ERR_INVALID_ARG;
   if (p->num_q_heads % p->num_kv_heads) return SPLITKV_ERR_INVALID_ARG;
-  if (p->flags & ~uint32_t(SPLITKV_FLAG_EQUAL_COUNT)) return SPLITKV_ERR_INVALID_ARG;
+  if (p->flags & ~uint32_t(SPLITKV_FLAG_EQUAL_COUNT | SPLITKV_FLAG_BLOCK_KEYS_IN_CONTEXT)) return SPLITKV_ERR_INVALID_ARG;
   int64_t N = 0;
   for (int s = 0; s < p->num_samples; ++s) {
     if (p->sample_lens[s] < 1) return SPLITKV_ERR_INVALID_ARG;
@@ -177,6 +177,7 @@ int build(splitkv_plan_t* P, const splitkv_problem* p) {
   P->blocks_per_tile = splitkv::kTileRows / (P->G * P->bs);
 
   // sample starts; block intervals [S_s, a_b) by binary search over the starts
+  // (reading B of the block keys: [S_s, min(a_b + bs, S_s + L_s)))
   std::vector<int64_t> starts(P->S + 1, 0);
   for (int s = 0; s < P->S; ++s) starts[s + 1] = starts[s] + P->lens[s];
   P->N = starts[P->S];
@@ -188,7 +189,9 @@ int build(splitkv_plan_t* P, const splitkv_problem* p) {
     const int64_t a = P->anchors[b];
     const int s = int(std::upper_bound(starts.begin(), starts.end(), a) - starts.begin()) - 1;
     P->block_lo[b] = int32_t(starts[s]);
-    P->block_hi[b] = int32_t(a);
+    P->block_hi[b] = (P->flags & SPLITKV_FLAG_BLOCK_KEYS_IN_CONTEXT)
+                         ? int32_t(std::min<int64_t>(a + P->bs, starts[s + 1]))
+                         : int32_t(a);
   }
 
   // entries: each block's interval covers chunks lo/C .. (hi-1)/C; bucket by chunk
@@ -508,6 +511,7 @@ int splitkv_plan_upload(splitkv_plan_t* P, void* stream) {
   v.E = int(P->entries.size());
   v.W = P->W;
   v.Wb = P->Wb;
+  v.block_term = (P->flags & SPLITKV_FLAG_BLOCK_KEYS_IN_CONTEXT) ? 0 : 1;
   P->uploaded = true;
   return SPLITKV_OK;
 }
@@ -540,7 +544,9 @@ int splitkv_plan_stats(const splitkv_plan_t* P, splitkv_stats* out) {
   uint64_t ctx = 0;
   for (uint64_t x : P->chunk_pairs) ctx += x;
   out->context_pairs = ctx * uint64_t(P->Hq);
-  out->block_pairs = uint64_t(P->Hq) * uint64_t(P->A) * uint64_t(P->bs) * uint64_t(P->bs);
+  out->block_pairs = (P->flags & SPLITKV_FLAG_BLOCK_KEYS_IN_CONTEXT)
+                         ? 0
+                         : uint64_t(P->Hq) * uint64_t(P->A) * uint64_t(P->bs) * uint64_t(P->bs);
   out->fwd_max_load = P->fwd_loads.empty() ? 0 : *std::max_element(P->fwd_loads.begin(), P->fwd_loads.end());
   out->bwd_max_load = P->bwd_loads.empty() ? 0 : *std::max_element(P->bwd_loads.begin(), P->bwd_loads.end());
   out->fwd_imbalance = imbalance(P->fwd_loads);

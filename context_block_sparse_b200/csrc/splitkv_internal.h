@@ -28,6 +28,7 @@ struct DevPlan {
   int*        status;           // device status word: 0, or a SPLITKV_ERR_* code a kernel recorded
   int num_zero_chunks;
   int N, Nq, A, bs, Hq, Hkv, G, d, C, num_chunks, E, W, Wb;
+  int block_term;               // 1: separate block keys kb, vb (reading A); 0: block keys in the context
 };
 
 // Byte offsets of the forward workspace (partial records).

@@ -66,8 +66,11 @@ extern "C" int splitkv_attn_fwd_static_scratch(const splitkv_plan_t* plan, const
   const splitkv::DevPlan* dp = splitkv::plan_device_view(plan);
   if (!dp) return SPLITKV_ERR_NOT_UPLOADED;
   if (dp->d != 64 && dp->d != 128) return SPLITKV_ERR_UNSUPPORTED;
-  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(kb) || !aligned16(vb) || !aligned16(o) ||
-      !lse || (reinterpret_cast<uintptr_t>(lse) % 4) != 0)
+  // kb, vb: required under reading A; may be NULL under SPLITKV_FLAG_BLOCK_KEYS_IN_CONTEXT
+  const bool blk_ok = dp->block_term ? (aligned16(kb) && aligned16(vb))
+                                     : ((!kb || aligned16(kb)) && (!vb || aligned16(vb)));
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !blk_ok || !aligned16(o) || !lse ||
+      (reinterpret_cast<uintptr_t>(lse) % 4) != 0)
     return SPLITKV_ERR_INVALID_ARG;
   if (o_dtype != SPLITKV_DTYPE_F32 && o_dtype != SPLITKV_DTYPE_BF16) return SPLITKV_ERR_INVALID_ARG;
   const splitkv::FwdWs L = splitkv::fwd_ws_layout(dp->E, dp->bs, dp->Hq, dp->d);

@@ -23,12 +23,17 @@ class SplitKVAttention:
     def __init__(self, sample_lens, anchors, block_size: int, num_q_heads: int, num_kv_heads: int,
                  head_dim: int, kv_chunk: int, num_workers: Optional[int] = None,
                  num_bwd_workers: int = 0, q_slice: int = 0, equal_count: bool = False,
-                 device: Optional[torch.device] = None):
+                 device: Optional[torch.device] = None, block_keys_in_context: bool = False):
+        """block_keys_in_context: reading B of the block keys (the block's own tokens are
+        the context positions after its anchor); kb, vb are then unused (pass None)
+        and backward() returns no dkb, dvb."""
         self.device = torch.device("cuda") if device is None else torch.device(device)
         if num_workers is None:
             num_workers = torch.cuda.get_device_properties(self.device).multi_processor_count
         self.plan: Plan = splitkv_plan(sample_lens, anchors, block_size, num_q_heads, num_kv_heads, head_dim,
-                                       kv_chunk, num_workers, num_bwd_workers, q_slice, equal_count)
+                                       kv_chunk, num_workers, num_bwd_workers, q_slice, equal_count,
+                                       block_keys_in_context)
+        self.block_keys_in_context = bool(block_keys_in_context)
         splitkv_plan_upload(self.plan)
         self.block_size = block_size
         self.num_q_heads = num_q_heads
@@ -60,8 +65,8 @@ class SplitKVAttention:
                 "dq": torch.empty(q.shape, **f32),
                 "dk": torch.empty(k.shape, **f32),
                 "dv": torch.empty(v.shape, **f32),
-                "dkb": torch.empty(kb.shape, **f32),
-                "dvb": torch.empty(vb.shape, **f32),
+                "dkb": None if self.block_keys_in_context else torch.empty(kb.shape, **f32),
+                "dvb": None if self.block_keys_in_context else torch.empty(vb.shape, **f32),
             }
         splitkv_attn_bwd(self.plan, q, k, v, kb, vb, o, lse, dout, grads["dq"], grads["dk"], grads["dv"],
                          grads["dkb"], grads["dvb"], scale, self.ws_bwd())

@@ -67,6 +67,15 @@ extern "C" {
 /* Equal-count LPT (the pages' device rule: chunk counts kept equal).  Off by
  * default: CTAs have no memory limit, and plain LPT keeps Graham's bound. */
 #define SPLITKV_FLAG_EQUAL_COUNT  1u
+/* Reading B of the block keys (news page, "Why short queries change the
+ * problem": every block also attends to "all tokens inside the block"): the
+ * block's own tokens are the context positions after its anchor, so block b's
+ * context interval is [S_s, min(a_b + bs, S_s + L_s)) and there are no
+ * separate block keys.  Under this flag kb, vb (splitkv_merge,
+ * splitkv_attn_fwd_static_scratch, splitkv_bwd_reduce, splitkv_attn_bwd) and
+ * dkb, dvb may be NULL; they are neither read nor written.  Default (flag
+ * clear, reading A): the block keys are the separate query-sized kb, vb. */
+#define SPLITKV_FLAG_BLOCK_KEYS_IN_CONTEXT  2u
 
 /* ---- dtype codes (o) ------------------------------------------------------- */
 #define SPLITKV_DTYPE_F32   0

@@ -26,38 +26,43 @@ def small(name="tiny", lens=(700, 1100, 333), anchors=24, Hq=8, Hkv=2, d=128, bs
         value_scale=1.0))
 
 
-def run(w, bwd=False, o_dtype="f32", W=148, Wb=0, q_slice=0, equal_count=False, repeat=1):
-    """Run plan/fwd/merge (and bwd) on cuda:0; returns numpy outputs (+ the attention object)."""
+def run(w, bwd=False, o_dtype="f32", W=148, Wb=0, q_slice=0, equal_count=False, repeat=1, rb=False):
+    """Run plan/fwd/merge (and bwd) on cuda:0; returns numpy outputs (+ the attention object).
+    rb: reading B of the block keys (kb, vb not passed; no dkb, dvb)."""
     import torch
     from context_block_sparse_b200.torch_api import SplitKVAttention
     att = SplitKVAttention(w.sample_lens, w.anchors, w.block_size, w.num_q_heads, w.num_kv_heads, w.head_dim,
                            w.kv_chunk, num_workers=W, num_bwd_workers=Wb, q_slice=q_slice,
-                           equal_count=equal_count)
+                           equal_count=equal_count, block_keys_in_context=rb)
     t = {n: to_dev(b) for n, b in w.bits.items()}
+    kb, vb = (None, None) if rb else (t["kb"], t["vb"])
     odt = torch.float32 if o_dtype == "f32" else torch.bfloat16
     out = {}
     for _ in range(repeat):
-        o, lse = att.forward(t["q"], t["k"], t["v"], t["kb"], t["vb"], w.scale, out_dtype=odt)
+        o, lse = att.forward(t["q"], t["k"], t["v"], kb, vb, w.scale, out_dtype=odt)
         out["o"] = o.float().cpu().numpy().astype(np.float64)
         out["lse"] = lse.cpu().numpy().astype(np.float64)
         if bwd:
-            g = att.backward(t["q"], t["k"], t["v"], t["kb"], t["vb"], o, lse, t["dout"], w.scale)
+            g = att.backward(t["q"], t["k"], t["v"], kb, vb, o, lse, t["dout"], w.scale)
             for n, x in g.items():
-                out[n] = x.cpu().numpy().astype(np.float64)
+                if x is not None:
+                    out[n] = x.cpu().numpy().astype(np.float64)
     torch.cuda.synchronize()
     import context_block_sparse_b200 as skv
     skv.splitkv_plan_status(att.plan)
     return out, att, t
 
 
-def oracle_fwd(w, blocks=None):
+def oracle_fwd(w, blocks=None, rb=False):
     return oatt.attention_fwd(w.f64("q"), w.f64("k"), w.f64("v"), w.f64("kb"), w.f64("vb"),
-                              w.sample_lens, w.anchors, w.block_size, w.scale, blocks=blocks)
+                              w.sample_lens, w.anchors, w.block_size, w.scale, blocks=blocks,
+                              block_keys_in_context=rb)
 
 
-def oracle_bwd(w, blocks=None):
+def oracle_bwd(w, blocks=None, rb=False):
     return oatt.attention_bwd(w.f64("q"), w.f64("k"), w.f64("v"), w.f64("kb"), w.f64("vb"), w.f64("dout"),
-                              w.sample_lens, w.anchors, w.block_size, w.scale, blocks=blocks)
+                              w.sample_lens, w.anchors, w.block_size, w.scale, blocks=blocks,
+                              block_keys_in_context=rb)
 
 
 def max_abs(a, b):

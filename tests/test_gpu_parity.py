@@ -150,6 +150,33 @@ def test_partial_records_match_oracle_split(splitkv, d):
     torch.cuda.synchronize()
 
 
+READING_B_CASES = {
+    "gqa4_d128": dict(Hq=8, Hkv=2, d=128),
+    "mha_d64": dict(Hq=2, Hkv=2, d=64),
+    "g1_bs8_d128": dict(Hq=2, Hkv=2, d=128, bs=8, anchors=40),
+    "chunk_not_dividing": dict(Hq=4, Hkv=1, d=128, C=100, lens=(257, 3, 1000, 61)),
+}
+
+
+@pytest.mark.parametrize("case", list(READING_B_CASES))
+def test_block_keys_in_context_fwd_bwd(splitkv, case):
+    """Reading B of the block keys (plan flag): every row reads its sample's context up to
+    min(a_b + bs, sample end); kb, vb are not passed and no dkb, dvb come back."""
+    w = small(**READING_B_CASES[case])
+    # an anchor within bs of its sample's end, so the interval end is clipped
+    starts = np.concatenate([[0], np.cumsum(w.sample_lens)])
+    w.anchors[0] = int(starts[1]) - 2
+    w.anchors[-1] = int(starts[-1]) - 1
+    out, _, _ = run(w, bwd=True, rb=True)
+    assert "dkb" not in out and "dvb" not in out
+    O, L = oracle_fwd(w, rb=True)
+    assert_close("O", out["o"], O, TOL_OUT)
+    assert_close("LSE", out["lse"], L, TOL_LSE)
+    g = oracle_bwd(w, rb=True)
+    for n in ("dq", "dk", "dv"):
+        assert_close(n, out[n], g[n], TOL_OUT)
+
+
 def test_merge_alone_on_oracle_partials(splitkv):
     """splitkv_merge fed with oracle-computed partial records reproduces the oracle output."""
     import torch

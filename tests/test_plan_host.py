@@ -14,27 +14,29 @@ from oracle import mask as omask
 from synth import CONFIGS, make_workload
 
 
-def _plan(skv, lens, anchors, bs, Hq, Hkv, d, C, W, Wb=0, q_slice=0, eq=False):
+def _plan(skv, lens, anchors, bs, Hq, Hkv, d, C, W, Wb=0, q_slice=0, eq=False, rb=False):
     return skv.splitkv_plan(lens, anchors, bs, Hq, Hkv, d, C, W, num_bwd_workers=Wb, q_slice=q_slice,
-                            equal_count=eq)
+                            equal_count=eq, block_keys_in_context=rb)
 
 
-def _check_against_oracle(skv, lens, anchors, bs, Hq, Hkv, C, W, Wb=0, q_slice=0, eq=False, d=64):
-    plan = _plan(skv, lens, anchors, bs, Hq, Hkv, d, C, W, Wb, q_slice, eq)
+def _check_against_oracle(skv, lens, anchors, bs, Hq, Hkv, C, W, Wb=0, q_slice=0, eq=False, d=64, rb=False):
+    """rb: reading B of the block keys (block keys in the context)."""
+    plan = _plan(skv, lens, anchors, bs, Hq, Hkv, d, C, W, Wb, q_slice, eq, rb)
     G = Hq // Hkv
     # entries: same set per chunk, record order sorted by (lo, hi, block) inside each chunk
     ent = plan.export(skv.EXPORT_ENTRIES).reshape(-1, 4)
-    want = omask.chunk_entries(lens, anchors, C)
+    want = omask.chunk_entries(lens, anchors, C, bs, rb)
     assert sorted(map(tuple, ent.tolist())) == sorted(want)
     keys = [(c, lo, hi, b) for (c, b, lo, hi) in ent.tolist()]
     assert keys == sorted(keys)
     # pair counts
     pairs = plan.export(skv.EXPORT_CHUNK_PAIRS)
-    assert pairs.tolist() == omask.chunk_pairs(lens, anchors, bs, C).tolist()
+    assert pairs.tolist() == omask.chunk_pairs(lens, anchors, bs, C, rb).tolist()
     # forward schedule (possibly sliced) and backward schedule (whole chunks)
     for what, loads_what, workers, qs in ((skv.EXPORT_FWD_SCHEDULE, skv.EXPORT_FWD_LOADS, W, q_slice),
                                           (skv.EXPORT_BWD_SCHEDULE, skv.EXPORT_BWD_LOADS, Wb or W, 0)):
-        items = olpt.work_items(lens, anchors, bs, C, Hq, Hkv, q_slice=qs, rows_per_tile=128)
+        items = olpt.work_items(lens, anchors, bs, C, Hq, Hkv, q_slice=qs, rows_per_tile=128,
+                                block_keys_in_context=rb)
         lists, loads = olpt.lpt(items, workers, equal_count=eq)
         cost = dict(items)
         sched = plan.export(what).reshape(-1, 5)
@@ -45,12 +47,13 @@ def _check_against_oracle(skv, lens, anchors, bs, Hq, Hkv, C, W, Wb=0, q_slice=0
         assert got == [list(l) for l in lists]
         assert plan.export(loads_what).tolist() == loads
     # contiguous baseline
-    _, cl = olpt.contiguous(olpt.work_items(lens, anchors, bs, C, Hq, Hkv), W)
+    _, cl = olpt.contiguous(olpt.work_items(lens, anchors, bs, C, Hq, Hkv, block_keys_in_context=rb), W)
     assert plan.export(skv.EXPORT_CONTIG_LOADS).tolist() == cl
     st_ = plan.stats()
     assert st_["context_pairs"] == Hq * int(pairs.sum())
-    assert st_["block_pairs"] == Hq * len(anchors) * bs * bs
-    _, fl = olpt.lpt(olpt.work_items(lens, anchors, bs, C, Hq, Hkv, q_slice=q_slice), W, equal_count=eq)
+    assert st_["block_pairs"] == (0 if rb else Hq * len(anchors) * bs * bs)
+    _, fl = olpt.lpt(olpt.work_items(lens, anchors, bs, C, Hq, Hkv, q_slice=q_slice, block_keys_in_context=rb), W,
+                     equal_count=eq)
     assert abs(st_["fwd_imbalance"] - olpt.imbalance(fl)) < 1e-12
     assert abs(st_["contig_imbalance"] - olpt.imbalance(cl)) < 1e-12
     plan.destroy()
@@ -67,28 +70,31 @@ def _check_against_oracle(skv, lens, anchors, bs, Hq, Hkv, C, W, Wb=0, q_slice=0
     Wb=st.integers(0, 9),
     q_slice=st.integers(0, 3),
     eq=st.booleans(),
+    rb=st.booleans(),
     seed=st.integers(0, 2 ** 31 - 1),
 )
-def test_random_problems_bit_exact(splitkv, lens, n_anchor, heads, bs, C, W, Wb, q_slice, eq, seed):
+def test_random_problems_bit_exact(splitkv, lens, n_anchor, heads, bs, C, W, Wb, q_slice, eq, rb, seed):
     Hq, Hkv = heads
     if 128 % ((Hq // Hkv) * bs):
         return
     rng = np.random.default_rng(seed)
     N = sum(lens)
     anchors = rng.integers(0, N, size=n_anchor).astype(np.int32)   # any order, repeats allowed
-    _check_against_oracle(splitkv, lens, anchors, bs, Hq, Hkv, C, W, Wb, q_slice, eq)
+    _check_against_oracle(splitkv, lens, anchors, bs, Hq, Hkv, C, W, Wb, q_slice, eq, rb=rb)
 
 
 @pytest.mark.parametrize("name", ["tiny", "drafter", "budget", "skew", "bwd"])
-@pytest.mark.parametrize("q_slice,eq", [(0, False), (2, False), (0, True)])
-def test_workload_plans_bit_exact(splitkv, name, q_slice, eq):
+@pytest.mark.parametrize("q_slice,eq,rb", [(0, False, False), (2, False, False), (0, True, False), (2, False, True)])
+def test_workload_plans_bit_exact(splitkv, name, q_slice, eq, rb):
     w = make_workload(name, tensors=False)
     _check_against_oracle(splitkv, w.sample_lens, w.anchors, w.block_size, w.num_q_heads, w.num_kv_heads,
-                          w.kv_chunk, 148, 0, q_slice, eq, d=w.head_dim)
+                          w.kv_chunk, 148, 0, q_slice, eq, d=w.head_dim, rb=rb)
 
 
 def test_anchor_at_sample_start_and_chunk_straddle(splitkv):
     _check_against_oracle(splitkv, [4, 4, 9], [0, 4, 5, 16, 8], 2, 2, 1, 3, 2)
+    # reading B: anchors 3 and 16 sit within bs of their sample's end (clipped)
+    _check_against_oracle(splitkv, [4, 4, 9], [0, 3, 5, 16, 8], 2, 2, 1, 3, 2, rb=True)
 
 
 @pytest.mark.parametrize("bad", [
