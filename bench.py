@@ -203,8 +203,9 @@ def _dist():
 # our arm
 # ---------------------------------------------------------------------------
 
-def _kernel_work(st, w, E):
-    """Algorithmic FLOPs or bytes of one launch of each kernel."""
+def _kernel_work(st, w, E, rec_bytes=4.0):
+    """Algorithmic FLOPs or bytes of one launch of each kernel; rec_bytes: bytes of one
+    O_c / dQ-partial element (4, or 2 with bf16 partial records)."""
     d, Hq, Hkv, bs, Nq = w.head_dim, w.num_q_heads, w.num_kv_heads, w.block_size, w.num_queries
     ctx = st["context_pairs"]
     rec_rows = E * bs * Hq
@@ -215,12 +216,12 @@ def _kernel_work(st, w, E):
         "bwd_dkdv": ("tensor", 8.0 * d * ctx),
         "bwd_dq": ("tensor", 6.0 * d * ctx),
         # partial records (O_c, m, l) read; o, lse written; q, kb, vb read once
-        "merge": ("hbm", rec_rows * (4.0 * d + 8) + Nq * Hq * (4.0 * d + 4) + Nq * Hq * d * 2.0
+        "merge": ("hbm", rec_rows * (rec_bytes * d + 8) + Nq * Hq * (4.0 * d + 4) + Nq * Hq * d * 2.0
                   + 2.0 * Nq * Hkv * d * 2),
         # o (fp32) and dout read, Delta written
         "bwd_delta": ("hbm", Nq * Hq * d * (4.0 + 2.0) + Nq * Hq * 4.0),
         # dq partials read; q, dout, kb, vb, lse, Delta read; dq, dkb, dvb written
-        "bwd_reduce": ("hbm", rec_rows * d * 4.0 + Nq * Hq * (d * 4.0 + 8) + Nq * Hq * d * 4.0
+        "bwd_reduce": ("hbm", rec_rows * d * rec_bytes + Nq * Hq * (d * 4.0 + 8) + Nq * Hq * d * 4.0
                        + 2.0 * Nq * Hkv * d * 2 + 2.0 * Nq * Hkv * d * 4),
     }
 
@@ -255,7 +256,7 @@ def run_ours(args, world, rank, local):
     t = {n: up(n) for n in ("q", "k", "v", "kb", "vb", "dout")}
     d, Hq, Nq = w.head_dim, w.num_q_heads, w.num_queries
     plan = skv.splitkv_plan(w.sample_lens, w.anchors, w.block_size, Hq, w.num_kv_heads, d, w.kv_chunk, W,
-                            num_bwd_workers=Wb, q_slice=args.q_slice)
+                            num_bwd_workers=Wb, q_slice=args.q_slice, partial_bf16=args.partial_bf16)
     plan.upload(stream)
     st = plan.stats()
     ws_f = torch.empty(skv.splitkv_workspace_size(plan, skv.WS_FWD), dtype=torch.uint8, device=dev)
@@ -344,7 +345,7 @@ def run_ours(args, world, rank, local):
     flops_step = flops_fwd + flops_bwd
     value = whole_job_tflops(world, args.steps, flops_step, ms)
     peaks = _peaks()
-    work = _kernel_work(st, w, st["num_entries"])
+    work = _kernel_work(st, w, st["num_entries"], 2.0 if args.partial_bf16 else 4.0)
     dom = max(kernels, key=lambda k: per_kernel[k])
     bound, amount = work[dom]
     dom_s = per_kernel[dom] * 1e-3
@@ -385,7 +386,8 @@ def run_ours(args, world, rank, local):
         "config": {"workload": w.config.description, "context_len": w.context_len, "num_queries": Nq,
                    "num_anchors": int(w.anchors.size), "block_size": w.block_size, "heads": [Hq, w.num_kv_heads],
                    "head_dim": d, "kv_chunk": w.kv_chunk, "fwd_workers": W, "bwd_workers": Wb,
-                   "q_slice": args.q_slice, "parallelism": "replicas" if world > 1 else "single",
+                   "q_slice": args.q_slice, "partial_records": "bf16" if args.partial_bf16 else "f32",
+                   "parallelism": "replicas" if world > 1 else "single",
                    "l2": "no flush: each step touches ~4 GB (> 126 MB L2)"},
         "fwd_tflops": flops_fwd / (fwd_ms * 1e-3) / 1e12,
         "bwd_tflops": flops_bwd / (bwd_ms * 1e-3) / 1e12,
@@ -451,7 +453,7 @@ def run_e2e(args, w, plan, dev, stream, flops_step, world=1):
     d, Hq, Nq = w.head_dim, w.num_q_heads, w.num_queries
     att = SplitKVAttention(w.sample_lens, w.anchors, w.block_size, Hq, w.num_kv_heads, d, w.kv_chunk,
                            num_workers=plan.problem.num_workers, num_bwd_workers=plan.problem.num_bwd_workers,
-                           device=dev)
+                           q_slice=plan.problem.q_slice, device=dev, partial_bf16=args.partial_bf16)
     dv = {n: torch.empty(x.shape, dtype=x.dtype, device=dev) for n, x in host.items()}
     outs_h = {"o": torch.empty((Nq, Hq, d), dtype=torch.float32).pin_memory(),
               "lse": torch.empty((Nq, Hq), dtype=torch.float32).pin_memory()}
@@ -586,6 +588,8 @@ def main(argv=None):
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-clocks", action="store_true")
+    ap.add_argument("--partial-bf16", action="store_true",
+                    help="store the partial records (O_c, dQ partials) as bf16 (plan flag; default float32)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")

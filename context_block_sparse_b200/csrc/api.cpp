@@ -23,9 +23,12 @@ int check_plan(const splitkv_plan_t* plan, const DevPlan** out) {
   const DevPlan* dp = splitkv::plan_device_view(plan);
   if (!dp) return SPLITKV_ERR_NOT_UPLOADED;
   if (dp->d != 64 && dp->d != 128) return SPLITKV_ERR_UNSUPPORTED;
+  if (dp->partial_bf16 && !splitkv::partial_bf16_supported(*dp)) return SPLITKV_ERR_UNSUPPORTED;
   *out = dp;
   return SPLITKV_OK;
 }
+
+size_t rec_bytes(const DevPlan* dp) { return dp->partial_bf16 ? 2 : 4; }
 
 int cuda_status(cudaError_t e) {
   if (e == cudaSuccess) return SPLITKV_OK;
@@ -56,12 +59,12 @@ int splitkv_attn_fwd(const splitkv_plan_t* plan, const void* q, const void* k, c
   int st = check_plan(plan, &dp);
   if (st != SPLITKV_OK) return st;
   if (!all_aligned16(q, k, v, ws)) return SPLITKV_ERR_INVALID_ARG;
-  const splitkv::FwdWs L = splitkv::fwd_ws_layout(dp->E, dp->bs, dp->Hq, dp->d);
+  const splitkv::FwdWs L = splitkv::fwd_ws_layout(dp->E, dp->bs, dp->Hq, dp->d, rec_bytes(dp));
   if (ws_bytes < L.total) return SPLITKV_ERR_WORKSPACE_TOO_SMALL;
   char* w = static_cast<char*>(ws);
   return cuda_status(splitkv::launch_fwd_partial(
       *dp, static_cast<const uint16_t*>(q), static_cast<const uint16_t*>(k), static_cast<const uint16_t*>(v),
-      scale, reinterpret_cast<float*>(w + L.o_off), reinterpret_cast<float*>(w + L.m_off),
+      scale, static_cast<void*>(w + L.o_off), reinterpret_cast<float*>(w + L.m_off),
       reinterpret_cast<float*>(w + L.l_off), static_cast<cudaStream_t>(stream)));
 }
 
@@ -73,12 +76,12 @@ int splitkv_merge(const splitkv_plan_t* plan, const void* q, const void* kb, con
   if (!all_aligned16(q, ws, o) || !block_ptrs_ok(dp, kb, vb) || !lse || !aligned(lse, 4))
     return SPLITKV_ERR_INVALID_ARG;
   if (o_dtype != SPLITKV_DTYPE_F32 && o_dtype != SPLITKV_DTYPE_BF16) return SPLITKV_ERR_INVALID_ARG;
-  const splitkv::FwdWs L = splitkv::fwd_ws_layout(dp->E, dp->bs, dp->Hq, dp->d);
+  const splitkv::FwdWs L = splitkv::fwd_ws_layout(dp->E, dp->bs, dp->Hq, dp->d, rec_bytes(dp));
   if (ws_bytes < L.total) return SPLITKV_ERR_WORKSPACE_TOO_SMALL;
   const char* w = static_cast<const char*>(ws);
   return cuda_status(splitkv::launch_merge(
       *dp, static_cast<const uint16_t*>(q), static_cast<const uint16_t*>(kb), static_cast<const uint16_t*>(vb),
-      scale, reinterpret_cast<const float*>(w + L.o_off), reinterpret_cast<const float*>(w + L.m_off),
+      scale, static_cast<const void*>(w + L.o_off), reinterpret_cast<const float*>(w + L.m_off),
       reinterpret_cast<const float*>(w + L.l_off), o, o_dtype == SPLITKV_DTYPE_BF16 ? 1 : 0, lse,
       static_cast<cudaStream_t>(stream)));
 }
@@ -90,7 +93,7 @@ int splitkv_bwd_delta(const splitkv_plan_t* plan, const void* o, int o_dtype, co
   if (st != SPLITKV_OK) return st;
   if (!all_aligned16(o, dout, ws)) return SPLITKV_ERR_INVALID_ARG;
   if (o_dtype != SPLITKV_DTYPE_F32 && o_dtype != SPLITKV_DTYPE_BF16) return SPLITKV_ERR_INVALID_ARG;
-  const splitkv::BwdWs L = splitkv::bwd_ws_layout(dp->E, dp->Nq, dp->bs, dp->Hq, dp->d);
+  const splitkv::BwdWs L = splitkv::bwd_ws_layout(dp->E, dp->Nq, dp->bs, dp->Hq, dp->d, rec_bytes(dp));
   if (ws_bytes < L.total) return SPLITKV_ERR_WORKSPACE_TOO_SMALL;
   float* delta = reinterpret_cast<float*>(static_cast<char*>(ws) + L.delta_off);
   return cuda_status(splitkv::launch_bwd_delta(*dp, o, o_dtype == SPLITKV_DTYPE_BF16 ? 1 : 0,
@@ -107,7 +110,7 @@ int bwd_partial_part(const splitkv_plan_t* plan, const void* q, const void* k, c
   if (st != SPLITKV_OK) return st;
   if (!all_aligned16(q, k, v, dout, ws) || !lse || !aligned(lse, 4)) return SPLITKV_ERR_INVALID_ARG;
   if (which != 2 && !all_aligned16(dk, dv)) return SPLITKV_ERR_INVALID_ARG;
-  const splitkv::BwdWs L = splitkv::bwd_ws_layout(dp->E, dp->Nq, dp->bs, dp->Hq, dp->d);
+  const splitkv::BwdWs L = splitkv::bwd_ws_layout(dp->E, dp->Nq, dp->bs, dp->Hq, dp->d, rec_bytes(dp));
   if (ws_bytes < L.total) return SPLITKV_ERR_WORKSPACE_TOO_SMALL;
   char* w = static_cast<char*>(ws);
   return cuda_status(splitkv::launch_bwd_partial(
@@ -142,13 +145,13 @@ int splitkv_bwd_reduce(const splitkv_plan_t* plan, const void* q, const void* kb
   if (st != SPLITKV_OK) return st;
   if (!all_aligned16(q, dout, dq, ws) || !block_ptrs_ok(dp, kb, vb, dkb, dvb) || !lse || !aligned(lse, 4))
     return SPLITKV_ERR_INVALID_ARG;
-  const splitkv::BwdWs L = splitkv::bwd_ws_layout(dp->E, dp->Nq, dp->bs, dp->Hq, dp->d);
+  const splitkv::BwdWs L = splitkv::bwd_ws_layout(dp->E, dp->Nq, dp->bs, dp->Hq, dp->d, rec_bytes(dp));
   if (ws_bytes < L.total) return SPLITKV_ERR_WORKSPACE_TOO_SMALL;
   const char* w = static_cast<const char*>(ws);
   return cuda_status(splitkv::launch_bwd_reduce(
       *dp, static_cast<const uint16_t*>(q), static_cast<const uint16_t*>(kb), static_cast<const uint16_t*>(vb),
       static_cast<const uint16_t*>(dout), lse, reinterpret_cast<const float*>(w + L.delta_off),
-      reinterpret_cast<const float*>(w + L.dq_off), scale, dq, dkb, dvb, static_cast<cudaStream_t>(stream)));
+      static_cast<const void*>(w + L.dq_off), scale, dq, dkb, dvb, static_cast<cudaStream_t>(stream)));
 }
 
 int splitkv_attn_bwd(const splitkv_plan_t* plan, const void* q, const void* k, const void* v, const void* kb,
@@ -163,7 +166,7 @@ int splitkv_attn_bwd(const splitkv_plan_t* plan, const void* q, const void* k, c
       !aligned(lse, 4))
     return SPLITKV_ERR_INVALID_ARG;
   if (o_dtype != SPLITKV_DTYPE_F32 && o_dtype != SPLITKV_DTYPE_BF16) return SPLITKV_ERR_INVALID_ARG;
-  const splitkv::BwdWs L = splitkv::bwd_ws_layout(dp->E, dp->Nq, dp->bs, dp->Hq, dp->d);
+  const splitkv::BwdWs L = splitkv::bwd_ws_layout(dp->E, dp->Nq, dp->bs, dp->Hq, dp->d, rec_bytes(dp));
   if (ws_bytes < L.total) return SPLITKV_ERR_WORKSPACE_TOO_SMALL;
   st = splitkv_bwd_delta(plan, o, o_dtype, dout, ws, ws_bytes, stream);
   if (st != SPLITKV_OK) return st;

@@ -360,7 +360,7 @@ cudaError_t launch_bwd_d(const DevPlan& p, const uint16_t* q, const uint16_t* k,
 bool bwd_sm100_supported(const DevPlan& p);
 cudaError_t launch_bwd_partial_sm100(const DevPlan& p, const uint16_t* q, const uint16_t* k, const uint16_t* v,
                                      const uint16_t* dout, const float* lse, const float* delta, float scale,
-                                     float* dk, float* dv, float* dq_part, cudaStream_t s, int which);
+                                     float* dk, float* dv, void* dq_part, cudaStream_t s, int which);
 
 // The tcgen05 kernels serve head_dim 128 with G * bs a multiple of 8; every
 // other shape runs the mma.sync kernel.  SPLITKV_BWD_KERNEL=mma selects the
@@ -368,16 +368,18 @@ cudaError_t launch_bwd_partial_sm100(const DevPlan& p, const uint16_t* q, const 
 cudaError_t launch_bwd_partial(const DevPlan& p, const uint16_t* q, const uint16_t* k,
                                const uint16_t* v, const uint16_t* dout, const float* lse,
                                const float* delta, float scale, float* dk, float* dv,
-                               float* dq_part, cudaStream_t s, int which) {
+                               void* dq_part, cudaStream_t s, int which) {
   static const bool force_mma = [] {
     const char* e = std::getenv("SPLITKV_BWD_KERNEL");
     return e != nullptr && std::strcmp(e, "mma") == 0;
   }();
   if (!force_mma && bwd_sm100_supported(p))
     return launch_bwd_partial_sm100(p, q, k, v, dout, lse, delta, scale, dk, dv, dq_part, s, which);
+  if (p.partial_bf16) return cudaErrorNotSupported;   // the entry points check this first
   if (which == 2) return cudaSuccess;   // the single mma.sync kernel ran in the dK/dV part
-  if (p.d == 64) return launch_bwd_d<64>(p, q, k, v, dout, lse, delta, scale, dk, dv, dq_part, s);
-  return launch_bwd_d<128>(p, q, k, v, dout, lse, delta, scale, dk, dv, dq_part, s);
+  float* dqp = static_cast<float*>(dq_part);
+  if (p.d == 64) return launch_bwd_d<64>(p, q, k, v, dout, lse, delta, scale, dk, dv, dqp, s);
+  return launch_bwd_d<128>(p, q, k, v, dout, lse, delta, scale, dk, dv, dqp, s);
 }
 
 }  // namespace splitkv

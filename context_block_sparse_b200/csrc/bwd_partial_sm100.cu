@@ -583,7 +583,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     bwd_dq_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_do,
                         const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                         const __grid_constant__ CUtensorMap tm_dq, DevPlan p, const float* __restrict__ lse,
-                        const float* __restrict__ delta, float scale, int bulk, float* __restrict__ dq_part) {
+                        const float* __restrict__ delta, float scale, int bulk, void* __restrict__ dq_part) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sQ = smem;
@@ -787,7 +787,22 @@ __global__ void __launch_bounds__(kThreads, 1)
       ++dq_cnt;
       tc_fence_after();
       float* scratch = reinterpret_cast<float*>(smem + kOffScratch) + (warp - 4) * 512;
-      if (bulk) {
+      if (p.partial_bf16) {
+        // bf16 dq partials: two 32-column chunks of this warpgroup's 64 columns
+        const int z0 = __shfl_sync(0xffffffffu, m.valid ? m.rec / p.Hq : 0, 0);
+        const bool wv = __shfl_sync(0xffffffffu, m.valid ? 1 : 0, 0) != 0;
+#pragma unroll 1
+        for (int cc = 0; cc < 2; ++cc) {
+          uint32_t v[32];
+          tmem_ld32(tdQ + cc * 32, v);
+          tmem_wait_ld();
+          reg_fence<32>(v);
+          if (bulk)
+            warp_bulk_store32_bf16<0>(scratch, v, scale, &tm_dq, hf * 64 + cc * 32, g * p.G, z0, wv);
+          else if (m.valid)
+            lane_store32_bf16(static_cast<uint16_t*>(dq_part) + size_t(m.rec) * D + hf * 64 + cc * 32, v, scale);
+        }
+      } else if (bulk) {
         // the warp's 32 rows are 32/G whole tokens of one block, all G heads of KV
         // head g (valid is warp-uniform): bulk tensor stores of 32 x 16 boxes
         const int z0 = __shfl_sync(0xffffffffu, m.valid ? m.rec / p.Hq : 0, 0);
@@ -801,7 +816,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           warp_bulk_store16<0>(scratch, v, scale, &tm_dq, hf * 64 + cc * 16, g * p.G, z0, wv);
         }
       } else {
-        float* dst = dq_part + size_t(m.rec) * D + hf * 64;
+        float* dst = static_cast<float*>(dq_part) + size_t(m.rec) * D + hf * 64;
 #pragma unroll 1
         for (int cc = 0; cc < 4; ++cc) {
           uint32_t v[16];
@@ -834,7 +849,7 @@ bool bwd_sm100_supported(const DevPlan& p) {
 
 cudaError_t launch_bwd_partial_sm100(const DevPlan& p, const uint16_t* q, const uint16_t* k, const uint16_t* v,
                                      const uint16_t* dout, const float* lse, const float* delta, float scale,
-                                     float* dk, float* dv, float* dq_part, cudaStream_t s, int which) {
+                                     float* dk, float* dv, void* dq_part, cudaStream_t s, int which) {
   CUtensorMap tq, tdo, tk, tv, tdk, tdv, tdq;
   if (!make_bf16_map_3d(&tq, q, D, p.Hq, p.Nq, p.G, p.bs) || !make_bf16_map_3d(&tdo, dout, D, p.Hq, p.Nq, p.G, p.bs) ||
       !make_bf16_map_3d(&tk, k, D, p.Hkv, p.N, 1, BT) || !make_bf16_map_3d(&tv, v, D, p.Hkv, p.N, 1, BT) ||
@@ -843,7 +858,10 @@ cudaError_t launch_bwd_partial_sm100(const DevPlan& p, const uint16_t* q, const 
   // dq partial records by bulk stores when a warp's 32 rows are 32/G whole tokens of one block
   const bool bulk_dq = 32 % p.G == 0 && (p.G * p.bs) % 32 == 0 && p.E > 0;
   if (bulk_dq) {
-    if (!make_f32_map_3d(&tdq, dq_part, D, p.Hq, uint64_t(p.E) * p.bs, 16, p.G, 32 / p.G)) return cudaErrorInvalidValue;
+    const bool ok = p.partial_bf16
+                        ? make_bf16_store_map_3d(&tdq, dq_part, D, p.Hq, uint64_t(p.E) * p.bs, p.G, 32 / p.G)
+                        : make_f32_map_3d(&tdq, dq_part, D, p.Hq, uint64_t(p.E) * p.bs, 16, p.G, 32 / p.G);
+    if (!ok) return cudaErrorInvalidValue;
   } else {
     memset(&tdq, 0, sizeof(tdq));
   }

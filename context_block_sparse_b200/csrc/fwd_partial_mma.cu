@@ -268,22 +268,34 @@ cudaError_t launch_fwd_d(const DevPlan& p, const uint16_t* q, const uint16_t* k,
 
 bool fwd_sm100_supported(const DevPlan& p);
 cudaError_t launch_fwd_partial_sm100(const DevPlan& p, const uint16_t* q, const uint16_t* k, const uint16_t* v,
-                                     float scale, float* part_o, float* part_m, float* part_l, cudaStream_t s);
+                                     float scale, void* part_o, float* part_m, float* part_l, cudaStream_t s);
+bool bwd_sm100_supported(const DevPlan& p);
+
+namespace {
+bool env_is_mma(const char* name) {
+  const char* e = std::getenv(name);
+  return e != nullptr && std::strcmp(e, "mma") == 0;
+}
+}  // namespace
+
+bool partial_bf16_supported(const DevPlan& p) {
+  static const bool forced = env_is_mma("SPLITKV_FWD_KERNEL") || env_is_mma("SPLITKV_BWD_KERNEL");
+  return !forced && fwd_sm100_supported(p) && bwd_sm100_supported(p);
+}
 
 // The tcgen05 kernel serves head_dim 128 with G * bs a multiple of 8; every
 // other shape runs the mma.sync kernel.  SPLITKV_FWD_KERNEL=mma selects the
 // mma.sync kernel for every shape (for comparisons).
 cudaError_t launch_fwd_partial(const DevPlan& p, const uint16_t* q, const uint16_t* k,
-                               const uint16_t* v, float scale, float* part_o, float* part_m,
+                               const uint16_t* v, float scale, void* part_o, float* part_m,
                                float* part_l, cudaStream_t s) {
-  static const bool force_mma = [] {
-    const char* e = std::getenv("SPLITKV_FWD_KERNEL");
-    return e != nullptr && std::strcmp(e, "mma") == 0;
-  }();
+  static const bool force_mma = env_is_mma("SPLITKV_FWD_KERNEL");
   if (!force_mma && fwd_sm100_supported(p))
     return launch_fwd_partial_sm100(p, q, k, v, scale, part_o, part_m, part_l, s);
-  if (p.d == 64) return launch_fwd_d<64>(p, q, k, v, scale, part_o, part_m, part_l, s);
-  return launch_fwd_d<128>(p, q, k, v, scale, part_o, part_m, part_l, s);
+  if (p.partial_bf16) return cudaErrorNotSupported;   // the entry points check this first
+  float* po = static_cast<float*>(part_o);
+  if (p.d == 64) return launch_fwd_d<64>(p, q, k, v, scale, po, part_m, part_l, s);
+  return launch_fwd_d<128>(p, q, k, v, scale, po, part_m, part_l, s);
 }
 
 }  // namespace splitkv

@@ -26,7 +26,8 @@
 // (natural units), l_c = sum exp(s - m_c) and O_c = sum exp(s - m_c) v / l_c.
 // Rows are masked to their block's [lo, hi).  When a warp's 32 rows are whole
 // tokens of one block (G * bs a multiple of 32), O_c leaves through bulk tensor
-// stores of 32-row x 16-column boxes staged in two 2 KB buffers per warp.
+// stores of 32-row x 16-column boxes staged in two 2 KB buffers per warp (32-row x
+// 32-column bf16 boxes when the plan stores bf16 records).
 //
 // Every mbarrier wait is bounded; on a timeout the kernel records
 // SPLITKV_ERR_TIMEOUT in the plan's status word, lets every role wind down,
@@ -164,7 +165,7 @@ __device__ __forceinline__ float exp_pack_store(const uint32_t (&v)[64], int a, 
 __global__ void __launch_bounds__(kThreads, 1)
     fwd_partial_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                              const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
-                             DevPlan p, float scale_log2, int bulk_o, float* __restrict__ part_o,
+                             DevPlan p, float scale_log2, int bulk_o, void* __restrict__ part_o,
                              float* __restrict__ part_m, float* __restrict__ part_l) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -471,7 +472,36 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       const float inv = l > 0.f ? 1.f / l : 0.f;
       float* scratch = reinterpret_cast<float*>(smem + kOffScratch) + (warp - 4) * 1024;
-      if (bulk_o) {
+      if (bulk_o && p.partial_bf16) {
+        // bf16 records: one 32-row x 32-column box per TMEM load, two buffers
+        const int z0 = __shfl_sync(0xffffffffu, valid ? rec / p.Hq : 0, 0);
+        if (valid) {
+          uint32_t va[32], vb[32];
+          tmem_ld32(tO, va);
+          tmem_wait_ld();
+          reg_fence<32>(va);
+#pragma unroll
+          for (int cch = 0; cch < D / 32; cch += 2) {
+            tmem_ld32(tO + (cch + 1) * 32, vb);
+            warp_bulk_store32_bf16<1>(scratch, va, inv, &tm_o, cch * 32, g * p.G, z0);
+            tmem_wait_ld();
+            reg_fence<32>(vb);
+            if (cch + 2 < D / 32) tmem_ld32(tO + (cch + 2) * 32, va);
+            warp_bulk_store32_bf16<1>(scratch + 512, vb, inv, &tm_o, (cch + 1) * 32, g * p.G, z0);
+            tmem_wait_ld();
+            reg_fence<32>(va);
+          }
+        }
+      } else if (p.partial_bf16) {
+#pragma unroll 1
+        for (int cch = 0; cch < D / 32; ++cch) {
+          uint32_t v[32];
+          tmem_ld32(tO + cch * 32, v);
+          tmem_wait_ld();
+          reg_fence<32>(v);
+          if (valid) lane_store32_bf16(static_cast<uint16_t*>(part_o) + size_t(rec) * D + cch * 32, v, inv);
+        }
+      } else if (bulk_o) {
         // the warp's rows: tokens tt0 .. tt0 + 32/G - 1 of one block, all G heads
         // (valid is warp-uniform here: a slot holds whole warps)
         const int z0 = __shfl_sync(0xffffffffu, valid ? rec / p.Hq : 0, 0);
@@ -502,7 +532,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           tmem_wait_ld();
           reg_fence<32>(v);
           warp_store_rows<32>(scratch, reinterpret_cast<const float*>(v), inv,
-                              valid ? part_o + size_t(rec) * D + cch * 32 : nullptr);
+                              valid ? static_cast<float*>(part_o) + size_t(rec) * D + cch * 32 : nullptr);
         }
       }
       if (valid) {
@@ -534,13 +564,15 @@ bool fwd_sm100_supported(const DevPlan& p) {
 }
 
 cudaError_t launch_fwd_partial_sm100(const DevPlan& p, const uint16_t* q, const uint16_t* k, const uint16_t* v,
-                                     float scale, float* part_o, float* part_m, float* part_l, cudaStream_t s) {
+                                     float scale, void* part_o, float* part_m, float* part_l, cudaStream_t s) {
   CUtensorMap tq, tk, tv, to;
   if (!make_bf16_map_3d(&tq, q, D, p.Hq, p.Nq, p.G, p.bs)) return cudaErrorInvalidValue;
   // bulk record stores when a warp's 32 rows are 32/G whole tokens of one block
   const bool bulk = 32 % p.G == 0 && (p.G * p.bs) % 32 == 0 && p.E > 0;
   if (bulk) {
-    if (!make_f32_map_3d(&to, part_o, D, p.Hq, uint64_t(p.E) * p.bs, 16, p.G, 32 / p.G)) return cudaErrorInvalidValue;
+    const bool ok = p.partial_bf16 ? make_bf16_store_map_3d(&to, part_o, D, p.Hq, uint64_t(p.E) * p.bs, p.G, 32 / p.G)
+                                   : make_f32_map_3d(&to, part_o, D, p.Hq, uint64_t(p.E) * p.bs, 16, p.G, 32 / p.G);
+    if (!ok) return cudaErrorInvalidValue;
   } else {
     memset(&to, 0, sizeof(to));
   }

@@ -102,6 +102,45 @@ __device__ __forceinline__ void load_f32_quad(const float* row, int u, float4 (&
   for (int k = 0; k < NG; ++k) x[k] = __ldg(reinterpret_cast<const float4*>(row + 4 * (u + 4 * k)));
 }
 
+// Record rows of either element type, held as raw 32-bit words until use: a
+// granule (4 dimensions) is RW words -- 4 for float32, 2 for bf16 pairs -- so
+// that bf16 records keep twice as many entries in flight in the same registers.
+template <bool kBf16>
+struct Rec {
+  static constexpr int RW = kBf16 ? 2 : 4;
+  template <int NG>
+  __device__ __forceinline__ static void load(const void* base, size_t row, int u, uint32_t (&x)[NG][RW]) {
+#pragma unroll
+    for (int k = 0; k < NG; ++k) {
+      if constexpr (kBf16) {
+        const uint2 w = __ldg(reinterpret_cast<const uint2*>(static_cast<const uint16_t*>(base) + row + 4 * (u + 4 * k)));
+        x[k][0] = w.x;
+        x[k][1] = w.y;
+      } else {
+        const uint4 w = __ldg(reinterpret_cast<const uint4*>(static_cast<const float*>(base) + row + 4 * (u + 4 * k)));
+        x[k][0] = w.x;
+        x[k][1] = w.y;
+        x[k][2] = w.z;
+        x[k][3] = w.w;
+      }
+    }
+  }
+  __device__ __forceinline__ static float4 get(const uint32_t (&x)[RW]) {
+    if constexpr (kBf16)
+      return make_float4(__uint_as_float(x[0] << 16), __uint_as_float(x[0] & 0xffff0000u),
+                         __uint_as_float(x[1] << 16), __uint_as_float(x[1] & 0xffff0000u));
+    else
+      return make_float4(__uint_as_float(x[0]), __uint_as_float(x[1]), __uint_as_float(x[2]), __uint_as_float(x[3]));
+  }
+  template <int NG>
+  __device__ __forceinline__ static void zero(uint32_t (&x)[NG][RW]) {
+#pragma unroll
+    for (int k = 0; k < NG; ++k)
+#pragma unroll
+      for (int i = 0; i < RW; ++i) x[k][i] = 0u;
+  }
+};
+
 // Stage entries [c0, c0 + cnt) of the block into sE (whole CTA; barriers inside).
 __device__ __forceinline__ void stage_entries(int* sE, const int* __restrict__ entries, int c0, int cnt) {
   __syncthreads();
@@ -112,14 +151,15 @@ __device__ __forceinline__ void stage_entries(int* sE, const int* __restrict__ e
 // ---------------------------------------------------------------------------
 // merge: grid (A, Hkv); smem kb/vb rows of the block (bf16), staged entry ids
 // ---------------------------------------------------------------------------
-template <int D>
+template <int D, bool kBf16Rec>
 __global__ void __launch_bounds__(kMergeThreads, 2)
     merge_kernel(DevPlan p, const uint16_t* __restrict__ q, const uint16_t* __restrict__ kb,
-                 const uint16_t* __restrict__ vb, float scale_log2, const float* __restrict__ part_o,
+                 const uint16_t* __restrict__ vb, float scale_log2, const void* __restrict__ part_o,
                  const float* __restrict__ part_m, const float* __restrict__ part_l, void* __restrict__ o,
                  int o_bf16, float* __restrict__ lse) {
   constexpr int NG = D / 16;
-  constexpr int EG = 16 / NG;          // entries whose records are in flight together
+  using RecT = Rec<kBf16Rec>;
+  constexpr int EG = 64 / (NG * RecT::RW);   // entries whose records are in flight together
   extern __shared__ __align__(16) uint8_t smem_raw[];
   uint16_t* sKb = reinterpret_cast<uint16_t*>(smem_raw);   // [bs][D]
   uint16_t* sVb = sKb + p.bs * D;
@@ -180,7 +220,7 @@ __global__ void __launch_bounds__(kMergeThreads, 2)
       const int cnt = min(kEStage, n - c0);
       if (c0 > 0) stage_entries(sE, p.block_entries + e0, c0, cnt);
       for (int i0 = 0; i0 < cnt; i0 += EG) {
-        float4 ov[EG][NG];
+        uint32_t ov[EG][NG][RecT::RW];
         float mx[EG], lx[EG];
 #pragma unroll
         for (int v = 0; v < EG; ++v) {
@@ -188,13 +228,12 @@ __global__ void __launch_bounds__(kMergeThreads, 2)
           mx[v] = -INFINITY;
           if (i0 + v < cnt) {
             const size_t rec = size_t(sE[i0 + v] * p.bs + tt) * p.Hq + head;
-            load_f32_quad<NG>(part_o + rec * D, u, ov[v]);
+            RecT::template load<NG>(part_o, rec * D, u, ov[v]);
             const float lr = __ldg(part_l + rec), mr = __ldg(part_m + rec);
             lx[v] = lr;
             mx[v] = lr > 0.f ? mr * kLog2e : -INFINITY;
           } else {
-#pragma unroll
-            for (int k = 0; k < NG; ++k) ov[v][k] = make_float4(0.f, 0.f, 0.f, 0.f);
+            RecT::template zero<NG>(ov[v]);
           }
         }
         float mg = mx[0];
@@ -215,10 +254,11 @@ __global__ void __launch_bounds__(kMergeThreads, 2)
           L += wv;
 #pragma unroll
           for (int k = 0; k < NG; ++k) {
-            acc[k][0] = fmaf(wv, ov[v][k].x, acc[k][0]);
-            acc[k][1] = fmaf(wv, ov[v][k].y, acc[k][1]);
-            acc[k][2] = fmaf(wv, ov[v][k].z, acc[k][2]);
-            acc[k][3] = fmaf(wv, ov[v][k].w, acc[k][3]);
+            const float4 x = RecT::get(ov[v][k]);
+            acc[k][0] = fmaf(wv, x.x, acc[k][0]);
+            acc[k][1] = fmaf(wv, x.y, acc[k][1]);
+            acc[k][2] = fmaf(wv, x.z, acc[k][2]);
+            acc[k][3] = fmaf(wv, x.w, acc[k][3]);
           }
         }
       }
@@ -277,15 +317,16 @@ __global__ void __launch_bounds__(kMergeThreads)
 // smem: kb, vb [bs][D] bf16; P, dS [rows][bs] fp32 (rows = G*bs, ordered
 // (token, head)); q, dout [rows][D] bf16 when stage_rows; entry ids
 // ---------------------------------------------------------------------------
-template <int D>
+template <int D, bool kBf16Rec>
 __global__ void __launch_bounds__(kMergeThreads, 2)
     bwd_reduce_kernel(DevPlan p, const uint16_t* __restrict__ q, const uint16_t* __restrict__ kb,
                       const uint16_t* __restrict__ vb, const uint16_t* __restrict__ dout,
                       const float* __restrict__ lse, const float* __restrict__ delta,
-                      const float* __restrict__ dq_part, float scale, float* __restrict__ dq,
+                      const void* __restrict__ dq_part, float scale, float* __restrict__ dq,
                       float* __restrict__ dkb, float* __restrict__ dvb, int stage_rows) {
   constexpr int NG = D / 16;
-  constexpr int EG = 16 / NG;
+  using RecT = Rec<kBf16Rec>;
+  constexpr int EG = 64 / (NG * RecT::RW);   // entries whose partials are in flight together
   constexpr int DPL = D / 32;
   extern __shared__ __align__(16) uint8_t smem_raw[];
   const int bs = p.bs;
@@ -375,25 +416,25 @@ __global__ void __launch_bounds__(kMergeThreads, 2)
       const int cnt = min(kEStage, n - c0);
       if (c0 > 0) stage_entries(sE, p.block_entries + e0, c0, cnt);
       for (int i0 = 0; i0 < cnt; i0 += EG) {
-        float4 pv[EG][NG];
+        uint32_t pv[EG][NG][RecT::RW];
 #pragma unroll
         for (int v = 0; v < EG; ++v) {
           if (i0 + v < cnt) {
             const size_t rec = size_t(sE[i0 + v] * bs + tt) * p.Hq + head;
-            load_f32_quad<NG>(dq_part + rec * D, u, pv[v]);
+            RecT::template load<NG>(dq_part, rec * D, u, pv[v]);
           } else {
-#pragma unroll
-            for (int k = 0; k < NG; ++k) pv[v][k] = make_float4(0.f, 0.f, 0.f, 0.f);
+            RecT::template zero<NG>(pv[v]);
           }
         }
 #pragma unroll
         for (int v = 0; v < EG; ++v)
 #pragma unroll
           for (int k = 0; k < NG; ++k) {
-            tot[k].x += pv[v][k].x;
-            tot[k].y += pv[v][k].y;
-            tot[k].z += pv[v][k].z;
-            tot[k].w += pv[v][k].w;
+            const float4 x = RecT::get(pv[v][k]);
+            tot[k].x += x.x;
+            tot[k].y += x.y;
+            tot[k].z += x.z;
+            tot[k].w += x.w;
           }
       }
     }
@@ -440,21 +481,22 @@ __global__ void __launch_bounds__(kMergeThreads, 2)
   }
 }
 
-template <int D>
+template <int D, bool kBf16Rec>
 cudaError_t merge_d(const DevPlan& p, const uint16_t* q, const uint16_t* kb, const uint16_t* vb,
-                    float scale, const float* po, const float* pm, const float* pl, void* o, int o_bf16,
+                    float scale, const void* po, const float* pm, const float* pl, void* o, int o_bf16,
                     float* lse, cudaStream_t s) {
   const size_t smem = size_t(2) * p.bs * D * sizeof(uint16_t) + kEStage * sizeof(int);
-  cudaError_t e = cudaFuncSetAttribute(merge_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+  cudaError_t e =
+      cudaFuncSetAttribute(merge_kernel<D, kBf16Rec>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
   if (e != cudaSuccess) return e;
-  merge_kernel<D><<<dim3(p.A, p.Hkv), kMergeThreads, smem, s>>>(p, q, kb, vb, scale * kLog2e, po, pm, pl, o,
-                                                                  o_bf16, lse);
+  merge_kernel<D, kBf16Rec><<<dim3(p.A, p.Hkv), kMergeThreads, smem, s>>>(p, q, kb, vb, scale * kLog2e, po, pm,
+                                                                            pl, o, o_bf16, lse);
   return cudaGetLastError();
 }
 
-template <int D>
+template <int D, bool kBf16Rec>
 cudaError_t reduce_d(const DevPlan& p, const uint16_t* q, const uint16_t* kb, const uint16_t* vb,
-                     const uint16_t* dout, const float* lse, const float* delta, const float* dq_part,
+                     const uint16_t* dout, const float* lse, const float* delta, const void* dq_part,
                      float scale, float* dq, float* dkb, float* dvb, cudaStream_t s) {
   const size_t rows = size_t(p.G) * p.bs;
   const size_t base =
@@ -462,21 +504,25 @@ cudaError_t reduce_d(const DevPlan& p, const uint16_t* q, const uint16_t* kb, co
   const size_t staged = base + 2 * rows * D * sizeof(uint16_t);
   const int stage_rows = staged <= size_t(64) * 1024 ? 1 : 0;   // small enough to keep occupancy
   const size_t smem = stage_rows ? staged : base;
-  cudaError_t e =
-      cudaFuncSetAttribute(bwd_reduce_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+  cudaError_t e = cudaFuncSetAttribute(bwd_reduce_kernel<D, kBf16Rec>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       int(smem));
   if (e != cudaSuccess) return e;
-  bwd_reduce_kernel<D><<<dim3(p.A, p.Hkv), kMergeThreads, smem, s>>>(p, q, kb, vb, dout, lse, delta, dq_part,
-                                                                       scale, dq, dkb, dvb, stage_rows);
+  bwd_reduce_kernel<D, kBf16Rec><<<dim3(p.A, p.Hkv), kMergeThreads, smem, s>>>(
+      p, q, kb, vb, dout, lse, delta, dq_part, scale, dq, dkb, dvb, stage_rows);
   return cudaGetLastError();
 }
 
 }  // namespace
 
 cudaError_t launch_merge(const DevPlan& p, const uint16_t* q, const uint16_t* kb, const uint16_t* vb,
-                         float scale, const float* part_o, const float* part_m, const float* part_l,
+                         float scale, const void* part_o, const float* part_m, const float* part_l,
                          void* o, int o_bf16, float* lse, cudaStream_t s) {
-  if (p.d == 64) return merge_d<64>(p, q, kb, vb, scale, part_o, part_m, part_l, o, o_bf16, lse, s);
-  return merge_d<128>(p, q, kb, vb, scale, part_o, part_m, part_l, o, o_bf16, lse, s);
+  if (p.partial_bf16) {
+    if (p.d == 64) return merge_d<64, true>(p, q, kb, vb, scale, part_o, part_m, part_l, o, o_bf16, lse, s);
+    return merge_d<128, true>(p, q, kb, vb, scale, part_o, part_m, part_l, o, o_bf16, lse, s);
+  }
+  if (p.d == 64) return merge_d<64, false>(p, q, kb, vb, scale, part_o, part_m, part_l, o, o_bf16, lse, s);
+  return merge_d<128, false>(p, q, kb, vb, scale, part_o, part_m, part_l, o, o_bf16, lse, s);
 }
 
 cudaError_t launch_bwd_delta(const DevPlan& p, const void* o, int o_bf16, const uint16_t* dout,
@@ -495,10 +541,14 @@ cudaError_t launch_bwd_delta(const DevPlan& p, const void* o, int o_bf16, const 
 
 cudaError_t launch_bwd_reduce(const DevPlan& p, const uint16_t* q, const uint16_t* kb,
                               const uint16_t* vb, const uint16_t* dout, const float* lse,
-                              const float* delta, const float* dq_part, float scale, float* dq,
+                              const float* delta, const void* dq_part, float scale, float* dq,
                               float* dkb, float* dvb, cudaStream_t s) {
-  if (p.d == 64) return reduce_d<64>(p, q, kb, vb, dout, lse, delta, dq_part, scale, dq, dkb, dvb, s);
-  return reduce_d<128>(p, q, kb, vb, dout, lse, delta, dq_part, scale, dq, dkb, dvb, s);
+  if (p.partial_bf16) {
+    if (p.d == 64) return reduce_d<64, true>(p, q, kb, vb, dout, lse, delta, dq_part, scale, dq, dkb, dvb, s);
+    return reduce_d<128, true>(p, q, kb, vb, dout, lse, delta, dq_part, scale, dq, dkb, dvb, s);
+  }
+  if (p.d == 64) return reduce_d<64, false>(p, q, kb, vb, dout, lse, delta, dq_part, scale, dq, dkb, dvb, s);
+  return reduce_d<128, false>(p, q, kb, vb, dout, lse, delta, dq_part, scale, dq, dkb, dvb, s);
 }
 
 }  // namespace splitkv

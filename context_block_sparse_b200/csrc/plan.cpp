@@ -75,7 +75,8 @@ int validate(const splitkv_problem* p) {
       p->num_bwd_workers < 0 || p->q_slice < 0)
     return SPLITKV_ERR_INVALID_ARG;
   if (p->num_q_heads % p->num_kv_heads) return SPLITKV_ERR_INVALID_ARG;
-  if (p->flags & ~uint32_t(SPLITKV_FLAG_EQUAL_COUNT | SPLITKV_FLAG_BLOCK_KEYS_IN_CONTEXT)) return SPLITKV_ERR_INVALID_ARG;
+  if (p->flags & ~uint32_t(SPLITKV_FLAG_EQUAL_COUNT | SPLITKV_FLAG_BLOCK_KEYS_IN_CONTEXT | SPLITKV_FLAG_PARTIAL_BF16))
+    return SPLITKV_ERR_INVALID_ARG;
   int64_t N = 0;
   for (int s = 0; s < p->num_samples; ++s) {
     if (p->sample_lens[s] < 1) return SPLITKV_ERR_INVALID_ARG;
@@ -512,6 +513,7 @@ int splitkv_plan_upload(splitkv_plan_t* P, void* stream) {
   v.W = P->W;
   v.Wb = P->Wb;
   v.block_term = (P->flags & SPLITKV_FLAG_BLOCK_KEYS_IN_CONTEXT) ? 0 : 1;
+  v.partial_bf16 = (P->flags & SPLITKV_FLAG_PARTIAL_BF16) ? 1 : 0;
   P->uploaded = true;
   return SPLITKV_OK;
 }
@@ -606,10 +608,11 @@ int splitkv_plan_export(const splitkv_plan_t* P, int what, int64_t* out, int64_t
 int splitkv_workspace_size(const splitkv_plan_t* P, int which, size_t* bytes) {
   if (!P || !bytes) return SPLITKV_ERR_INVALID_ARG;
   const long long E = (long long)P->entries.size();
+  const size_t rb = (P->flags & SPLITKV_FLAG_PARTIAL_BF16) ? 2 : 4;
   if (which == SPLITKV_WS_FWD) {
-    *bytes = splitkv::fwd_ws_layout(E, P->bs, P->Hq, P->d).total;
+    *bytes = splitkv::fwd_ws_layout(E, P->bs, P->Hq, P->d, rb).total;
   } else if (which == SPLITKV_WS_BWD) {
-    *bytes = splitkv::bwd_ws_layout(E, int(P->Nq), P->bs, P->Hq, P->d).total;
+    *bytes = splitkv::bwd_ws_layout(E, int(P->Nq), P->bs, P->Hq, P->d, rb).total;
   } else {
     return SPLITKV_ERR_INVALID_ARG;
   }

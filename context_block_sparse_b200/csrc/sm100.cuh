@@ -154,6 +154,50 @@ __device__ __forceinline__ void warp_bulk_store16(float* buf, const uint32_t* va
   __syncwarp();
 }
 
+// The bf16 counterpart: one warp's 32 rows x 32 columns (vals[0..32) of the
+// lane's row, times mul, rounded to bf16 with round-to-nearest-even) through a
+// 2 KB buffer laid out as the 64-byte-swizzled box {32, ...} of a bf16 `map`,
+// then one bulk tensor store at (x, y, z) when `store`.  Same buffer rules as
+// warp_bulk_store16.
+template <int kPending>
+__device__ __forceinline__ void warp_bulk_store32_bf16(float* bufp, const uint32_t* vals, float mul,
+                                                       const CUtensorMap* map, int x, int y, int z, bool store = true) {
+  const int lane = threadIdx.x & 31;
+  if (lane == 0) asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(kPending) : "memory");
+  __syncwarp();
+  uint32_t* buf = reinterpret_cast<uint32_t*>(bufp);
+#pragma unroll
+  for (int g = 0; g < 4; ++g) {
+    uint4 w;
+    w.x = pack_bf16(__uint_as_float(vals[8 * g]) * mul, __uint_as_float(vals[8 * g + 1]) * mul);
+    w.y = pack_bf16(__uint_as_float(vals[8 * g + 2]) * mul, __uint_as_float(vals[8 * g + 3]) * mul);
+    w.z = pack_bf16(__uint_as_float(vals[8 * g + 4]) * mul, __uint_as_float(vals[8 * g + 5]) * mul);
+    w.w = pack_bf16(__uint_as_float(vals[8 * g + 6]) * mul, __uint_as_float(vals[8 * g + 7]) * mul);
+    *reinterpret_cast<uint4*>(buf + lane * 16 + ((g ^ ((lane >> 1) & 3)) << 2)) = w;
+  }
+  fence_async_smem();
+  __syncwarp();
+  if (lane == 0 && store) {
+    tma_store_3d(map, buf, x, y, z);
+    bulk_commit();
+  }
+  __syncwarp();
+}
+
+// 32 values of the lane's own row, times mul, as bf16 to dst (64 bytes, 16-byte
+// aligned): four 16-byte stores (rows that are not one bulk box).
+__device__ __forceinline__ void lane_store32_bf16(uint16_t* dst, const uint32_t* vals, float mul) {
+#pragma unroll
+  for (int g = 0; g < 4; ++g) {
+    uint4 w;
+    w.x = pack_bf16(__uint_as_float(vals[8 * g]) * mul, __uint_as_float(vals[8 * g + 1]) * mul);
+    w.y = pack_bf16(__uint_as_float(vals[8 * g + 2]) * mul, __uint_as_float(vals[8 * g + 3]) * mul);
+    w.z = pack_bf16(__uint_as_float(vals[8 * g + 4]) * mul, __uint_as_float(vals[8 * g + 5]) * mul);
+    w.w = pack_bf16(__uint_as_float(vals[8 * g + 6]) * mul, __uint_as_float(vals[8 * g + 7]) * mul);
+    reinterpret_cast<uint4*>(dst)[g] = w;
+  }
+}
+
 // Three-input maximum (one instruction on sm_100).
 __device__ __forceinline__ float fmax3(float a, float b, float c) {
   float r;

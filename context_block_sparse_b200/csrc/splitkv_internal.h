@@ -29,6 +29,7 @@ struct DevPlan {
   int num_zero_chunks;
   int N, Nq, A, bs, Hq, Hkv, G, d, C, num_chunks, E, W, Wb;
   int block_term;               // 1: separate block keys kb, vb (reading A); 0: block keys in the context
+  int partial_bf16;             // 1: O_c records and dQ partials stored as bf16
 };
 
 // Byte offsets of the forward workspace (partial records).
@@ -42,22 +43,23 @@ struct BwdWs {
 
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
-inline FwdWs fwd_ws_layout(long long E, int bs, int Hq, int d) {
+// rec_bytes: bytes of one O_c / dQ-partial element (4, or 2 under bf16 partials)
+inline FwdWs fwd_ws_layout(long long E, int bs, int Hq, int d, size_t rec_bytes) {
   FwdWs w;
   const size_t rows = size_t(E) * bs * Hq;
   w.o_off = 0;
-  w.m_off = align_up(rows * d * sizeof(float), 256);
+  w.m_off = align_up(rows * d * rec_bytes, 256);
   w.l_off = w.m_off + align_up(rows * sizeof(float), 256);
   w.total = w.l_off + align_up(rows * sizeof(float), 256);
   if (w.total == 0) w.total = 256;
   return w;
 }
 
-inline BwdWs bwd_ws_layout(long long E, int Nq, int bs, int Hq, int d) {
+inline BwdWs bwd_ws_layout(long long E, int Nq, int bs, int Hq, int d, size_t rec_bytes) {
   BwdWs w;
   const size_t rows = size_t(E) * bs * Hq;
   w.dq_off = 0;
-  w.delta_off = align_up(rows * d * sizeof(float), 256);
+  w.delta_off = align_up(rows * d * rec_bytes, 256);
   w.total = w.delta_off + align_up(size_t(Nq) * Hq * sizeof(float), 256);
   return w;
 }
@@ -73,14 +75,19 @@ bool make_bf16_map_3d(void* map, const void* base, uint64_t dim0, uint64_t dim1,
 // epilogue chunks).
 bool make_f32_map_3d(void* map, void* base, uint64_t dim0, uint64_t dim1, uint64_t dim2, uint32_t box0,
                      uint32_t box1, uint32_t box2);
+// 3-D bf16 tensor [dim2][dim1][dim0], box {32, box1, box2} (64-byte rows),
+// 64-byte swizzle (bulk stores of bf16 epilogue chunks).
+bool make_bf16_store_map_3d(void* map, void* base, uint64_t dim0, uint64_t dim1, uint64_t dim2, uint32_t box1,
+                            uint32_t box2);
 
 // ---- kernel launchers (defined in the .cu files) ---------------------------
+// part_o / dq_part: float32 records, or bf16 when p.partial_bf16 (tcgen05 path only)
 cudaError_t launch_fwd_partial(const DevPlan& p, const uint16_t* q, const uint16_t* k,
-                               const uint16_t* v, float scale, float* part_o, float* part_m,
+                               const uint16_t* v, float scale, void* part_o, float* part_m,
                                float* part_l, cudaStream_t s);
 
 cudaError_t launch_merge(const DevPlan& p, const uint16_t* q, const uint16_t* kb,
-                         const uint16_t* vb, float scale, const float* part_o,
+                         const uint16_t* vb, float scale, const void* part_o,
                          const float* part_m, const float* part_l, void* o, int o_bf16,
                          float* lse, cudaStream_t s);
 
@@ -92,11 +99,15 @@ cudaError_t launch_bwd_delta(const DevPlan& p, const void* o, int o_bf16, const 
 cudaError_t launch_bwd_partial(const DevPlan& p, const uint16_t* q, const uint16_t* k,
                                const uint16_t* v, const uint16_t* dout, const float* lse,
                                const float* delta, float scale, float* dk, float* dv,
-                               float* dq_part, cudaStream_t s, int which = 0);
+                               void* dq_part, cudaStream_t s, int which = 0);
 
 cudaError_t launch_bwd_reduce(const DevPlan& p, const uint16_t* q, const uint16_t* kb,
                               const uint16_t* vb, const uint16_t* dout, const float* lse,
-                              const float* delta, const float* dq_part, float scale, float* dq,
+                              const float* delta, const void* dq_part, float scale, float* dq,
                               float* dkb, float* dvb, cudaStream_t s);
+
+// bf16 partial records need the tcgen05 forward and backward kernels for this plan
+// (and no SPLITKV_FWD_KERNEL / SPLITKV_BWD_KERNEL override selecting mma.sync).
+bool partial_bf16_supported(const DevPlan& p);
 
 }  // namespace splitkv

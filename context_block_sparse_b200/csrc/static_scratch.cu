@@ -66,6 +66,7 @@ extern "C" int splitkv_attn_fwd_static_scratch(const splitkv_plan_t* plan, const
   const splitkv::DevPlan* dp = splitkv::plan_device_view(plan);
   if (!dp) return SPLITKV_ERR_NOT_UPLOADED;
   if (dp->d != 64 && dp->d != 128) return SPLITKV_ERR_UNSUPPORTED;
+  if (dp->partial_bf16 && !splitkv::partial_bf16_supported(*dp)) return SPLITKV_ERR_UNSUPPORTED;
   // kb, vb: required under reading A; may be NULL under SPLITKV_FLAG_BLOCK_KEYS_IN_CONTEXT
   const bool blk_ok = dp->block_term ? (aligned16(kb) && aligned16(vb))
                                      : ((!kb || aligned16(kb)) && (!vb || aligned16(vb)));
@@ -73,13 +74,13 @@ extern "C" int splitkv_attn_fwd_static_scratch(const splitkv_plan_t* plan, const
       (reinterpret_cast<uintptr_t>(lse) % 4) != 0)
     return SPLITKV_ERR_INVALID_ARG;
   if (o_dtype != SPLITKV_DTYPE_F32 && o_dtype != SPLITKV_DTYPE_BF16) return SPLITKV_ERR_INVALID_ARG;
-  const splitkv::FwdWs L = splitkv::fwd_ws_layout(dp->E, dp->bs, dp->Hq, dp->d);
+  const splitkv::FwdWs L = splitkv::fwd_ws_layout(dp->E, dp->bs, dp->Hq, dp->d, dp->partial_bf16 ? 2 : 4);
   if (L.total > kScratchBytes) return SPLITKV_ERR_WORKSPACE_TOO_SMALL;   // problem too large for the buffer
   void* base = nullptr;
   const int st = scratch_address(&base);
   if (st != SPLITKV_OK) return st;
   char* w = static_cast<char*>(base);
-  float* po = reinterpret_cast<float*>(w + L.o_off);
+  void* po = w + L.o_off;
   float* pm = reinterpret_cast<float*>(w + L.m_off);
   float* pl = reinterpret_cast<float*>(w + L.l_off);
   cudaStream_t s = static_cast<cudaStream_t>(stream);

@@ -76,6 +76,14 @@ extern "C" {
  * dkb, dvb may be NULL; they are neither read nor written.  Default (flag
  * clear, reading A): the block keys are the separate query-sized kb, vb. */
 #define SPLITKV_FLAG_BLOCK_KEYS_IN_CONTEXT  2u
+/* bfloat16 partial records: the chunk outputs O_c of the forward workspace and
+ * the dQ partials of the backward workspace are stored as bf16 (m_c, l_c and
+ * every output stay float32).  Halves the record traffic of the partial
+ * kernels, the merge and the dQ reduce, at one more bf16 rounding (relative
+ * 2^-9) of each record element before the fp32 combine.  Served by the
+ * tcgen05 kernels only (head_dim 128, G * bs a multiple of 8): attention calls
+ * of other plans return SPLITKV_ERR_UNSUPPORTED. */
+#define SPLITKV_FLAG_PARTIAL_BF16  4u
 
 /* ---- dtype codes (o) ------------------------------------------------------- */
 #define SPLITKV_DTYPE_F32   0
@@ -184,12 +192,14 @@ int splitkv_plan_export(const splitkv_plan_t* plan, int what, int64_t* out,
                         int64_t capacity, int64_t* count);
 
 /* Bytes of workspace an attention call needs (host only).
- *   SPLITKV_WS_FWD: the chunk partial records, as float32
+ *   SPLITKV_WS_FWD: the chunk partial records, as float32 (O_c as bfloat16
+ *       under SPLITKV_FLAG_PARTIAL_BF16)
  *       O_c [E][bs][Hq][d], then m_c [E][bs][Hq], then l_c [E][bs][Hq]
  *     (E = number of entries, in entry order; each array starts on a 256-byte
  *     boundary).  m_c is the row's max of scale * q.k over the entry's keys
  *     (natural units), l_c = sum exp(s - m_c), O_c = sum exp(s - m_c) v / l_c.
- *   SPLITKV_WS_BWD: dQ partials float32 [E][bs][Hq][d], then
+ *   SPLITKV_WS_BWD: dQ partials float32 [E][bs][Hq][d] (bfloat16 under
+ *       SPLITKV_FLAG_PARTIAL_BF16), then
  *     Delta = rowsum(dout * o) float32 [Nq][Hq]. */
 int splitkv_workspace_size(const splitkv_plan_t* plan, int which, size_t* bytes);
 

@@ -177,6 +177,53 @@ def test_block_keys_in_context_fwd_bwd(splitkv, case):
         assert_close(n, out[n], g[n], TOL_OUT)
 
 
+BF16_CASES = {
+    "gqa4_d128": dict(Hq=8, Hkv=2, d=128),                           # records by bulk tensor stores
+    "g1_bs8_d128": dict(Hq=2, Hkv=2, d=128, bs=8, anchors=40),      # 8-row slots: per-lane stores
+    "gqa8_d128": dict(Hq=8, Hkv=1, d=128),
+    "chunk_not_dividing": dict(Hq=4, Hkv=1, d=128, C=100, lens=(257, 3, 1000, 61)),
+}
+
+
+@pytest.mark.parametrize("case", list(BF16_CASES))
+def test_partial_bf16_fwd_bwd(splitkv, case):
+    """bf16 partial records (plan flag): one more bf16 rounding (relative 2^-9) of each
+    O_c and dQ-partial element before the fp32 combine, within the same tolerances."""
+    w = small(**BF16_CASES[case])
+    out, _, _ = run(w, bwd=True, partial_bf16=True)
+    _check_fwd(w, out)
+    _check_bwd(w, out)
+
+
+def test_partial_bf16_records(splitkv):
+    """The bf16 O_c records (and fp32 m_c, l_c) match the oracle's per-chunk partials."""
+    from oracle import attention as oatt
+    w = small(Hq=4, Hkv=2, d=128)
+    _, att, _ = run(w, partial_bf16=True)
+    E = att.plan.stats()["num_entries"]
+    bs, Hq, d = w.block_size, w.num_q_heads, w.head_dim
+    ws = att.ws_fwd.cpu().numpy()
+    rows = E * bs * Hq
+    o_bytes = -(-rows * d * 2 // 256) * 256
+    ml_bytes = -(-rows * 4 // 256) * 256
+    O = (ws[:rows * d * 2].view(np.uint16).astype(np.uint32) << 16).view(np.float32).reshape(E, bs, Hq, d)
+    m = ws[o_bytes:o_bytes + rows * 4].view(np.float32).reshape(E, bs, Hq)
+    ent = att.plan.export(0).reshape(-1, 4)
+    parts = {(p["c"], p["b"]): p for p in oatt.chunk_partials(
+        w.f64("q"), w.f64("k"), w.f64("v"), w.sample_lens, w.anchors, bs, w.kv_chunk, w.scale)}
+    for e, (c, b, lo, hi) in enumerate(ent.tolist()):
+        p = parts[(c, b)]
+        assert_close("O_c", O[e].astype(np.float64), p["O"], TOL_OUT)
+        assert_close("m_c", m[e].astype(np.float64), p["m"], TOL_LSE)
+
+
+def test_partial_bf16_needs_the_tcgen05_path(splitkv):
+    w = small(Hq=2, Hkv=2, d=64)
+    with pytest.raises(splitkv.SplitKVError) as ei:
+        run(w, partial_bf16=True)
+    assert ei.value.status == -2   # SPLITKV_ERR_UNSUPPORTED
+
+
 def test_merge_alone_on_oracle_partials(splitkv):
     """splitkv_merge fed with oracle-computed partial records reproduces the oracle output."""
     import torch
@@ -239,6 +286,13 @@ def test_drafter_fwd_full(splitkv):
 def test_budget_fwd_sampled(splitkv, anchors):
     w = make_workload("budget", num_anchors=anchors)
     out, _, _ = run(w)
+    _check_fwd(w, out, _sample_blocks(w))
+    assert np.isfinite(out["o"]).all() and np.isfinite(out["lse"]).all()
+
+
+def test_budget_fwd_sampled_bf16_partials(splitkv):
+    w = make_workload("budget", num_anchors=512)
+    out, _, _ = run(w, partial_bf16=True)
     _check_fwd(w, out, _sample_blocks(w))
     assert np.isfinite(out["o"]).all() and np.isfinite(out["lse"]).all()
 
