@@ -48,12 +48,12 @@ METRIC = "masked-pair attn TFLOP/s fwd/bwd, % of BF16 tensor peak; LPT imbalance
 # launches), keyed by kernel, with the sha256 of the sources the kernel was
 # built from when it was taken; a changed source voids the figure.
 NCU_TRAFFIC = {
-    "fwd_partial": {"bytes": 2077623910, "src": "a3476331464989c3"},
-    "merge": {"bytes": 1558117734, "src": "747751e396772082"},
-    "bwd_delta": {"bytes": 201976883, "src": "747751e396772082"},
-    "bwd_dkdv": {"bytes": 1716478925, "src": "ec4a2afa5314f31c"},
-    "bwd_dq": {"bytes": 2314637670, "src": "ec4a2afa5314f31c"},
-    "bwd_reduce": {"bytes": 1553852672, "src": "747751e396772082"},
+    "fwd_partial": {"bytes": 2079296922, "src": "28cc87a4c859dafd"},
+    "merge": {"bytes": 1557832397, "src": "66938df79d9cc3b1"},
+    "bwd_delta": {"bytes": 202124698, "src": "66938df79d9cc3b1"},
+    "bwd_dkdv": {"bytes": 1651303680, "src": "93057d0c2a816242"},
+    "bwd_dq": {"bytes": 2309377331, "src": "93057d0c2a816242"},
+    "bwd_reduce": {"bytes": 1554064230, "src": "66938df79d9cc3b1"},
 }
 _KERNEL_SOURCES = {
     "fwd_partial": ("fwd_partial_sm100.cu", "sm100.cuh", "splitkv_internal.h"),
