@@ -64,10 +64,6 @@ __device__ __forceinline__ float fast_exp2(float x) {
   return y;
 }
 
-__device__ __forceinline__ float bf16_bits_to_float(uint16_t b) {
-  return __uint_as_float(uint32_t(b) << 16);
-}
-
 // Element offset of (row r, 16-byte chunk ch) in a row-major [rows][D] bf16 smem
 // tile whose 16-byte chunks are XOR-swizzled by (r & 7): ldmatrix over 8
 // consecutive rows then touches 8 distinct bank groups.

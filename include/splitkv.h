@@ -25,12 +25,14 @@
  *         q, dout      [Nq, Hq, d]   bfloat16 (raw 16-bit storage)
  *         k, v         [N, Hkv, d]   bfloat16
  *         kb, vb       [Nq, Hkv, d]  bfloat16  (the draft block's own keys/values,
- *                                                one row per draft token)
+ *                                                one row per draft token; unused
+ *                                                and may be NULL under
+ *                                                SPLITKV_FLAG_BLOCK_KEYS_IN_CONTEXT)
  *         o            [Nq, Hq, d]   float32 or bfloat16 (see o_dtype)
  *         lse          [Nq, Hq]      float32, natural log
  *         dq           [Nq, Hq, d]   float32
  *         dk, dv       [N, Hkv, d]   float32
- *         dkb, dvb     [Nq, Hkv, d]  float32
+ *         dkb, dvb     [Nq, Hkv, d]  float32   (likewise)
  *     where N = sum of sample lengths, Nq = num_anchors * block_size, query
  *     token i belongs to block i / block_size, and query head h reads KV head
  *     h / (Hq / Hkv).
@@ -218,7 +220,8 @@ int splitkv_attn_fwd(const splitkv_plan_t* plan, const void* q, const void* k,
 
 /* Exact combine (news page, "Exchange the smaller side"): for every query row
  * and head, the in-block term over the bs keys kb/vb of its own block gives a
- * record (m_b, l_b, O_b); with the row's chunk records x (in chunk order),
+ * record (m_b, l_b, O_b) (none under SPLITKV_FLAG_BLOCK_KEYS_IN_CONTEXT, where
+ * the block's keys are context keys); with the row's chunk records x (in chunk order),
  * M = max m_x, L = sum l_x exp(m_x - M), o = sum l_x exp(m_x - M) O_x / L,
  * lse = M + log L.  Records with l = 0 are skipped.  o is written as float32
  * or bfloat16 (o_dtype), lse as float32.  ws must hold a forward result of
