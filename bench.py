@@ -48,12 +48,12 @@ METRIC = "masked-pair attn TFLOP/s fwd/bwd, % of BF16 tensor peak; LPT imbalance
 # launches), keyed by kernel, with the sha256 of the sources the kernel was
 # built from when it was taken; a changed source voids the figure.
 NCU_TRAFFIC = {
-    "fwd_partial": {"bytes": 2079296922, "src": "28cc87a4c859dafd"},
-    "merge": {"bytes": 1557832397, "src": "66938df79d9cc3b1"},
-    "bwd_delta": {"bytes": 202124698, "src": "66938df79d9cc3b1"},
-    "bwd_dkdv": {"bytes": 1651303680, "src": "93057d0c2a816242"},
-    "bwd_dq": {"bytes": 2309377331, "src": "93057d0c2a816242"},
-    "bwd_reduce": {"bytes": 1554064230, "src": "66938df79d9cc3b1"},
+    "fwd_partial": {"bytes": 2082256026, "src": "9a3f68c6308f2a0e"},
+    "merge": {"bytes": 1557937152, "src": "b87601659b20c86d"},
+    "bwd_delta": {"bytes": 201935719, "src": "b87601659b20c86d"},
+    "bwd_dkdv": {"bytes": 1651331277, "src": "1ddaa484886212e9"},
+    "bwd_dq": {"bytes": 2313403597, "src": "1ddaa484886212e9"},
+    "bwd_reduce": {"bytes": 1554807655, "src": "b87601659b20c86d"},
 }
 _KERNEL_SOURCES = {
     "fwd_partial": ("fwd_partial_sm100.cu", "sm100.cuh", "splitkv_internal.h"),
