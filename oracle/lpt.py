@@ -22,22 +22,87 @@ Readings where the pages are silent (integer arithmetic, so bit-exact):
 * imbalance = max load / mean load - 1 over all W workers;
 * the "unbalanced" baseline keeps chunks in contiguous order: the n_chunks * Hkv
   unsliced items in (c, g) order, item i to worker floor(i W / n).
+
+Optional tile cost (this library's refinement for its kernels, not the pages'
+rule): the cost of an item is the work its kernel executes, in (row, key) pairs
+of whole tiles -- rows_per_tile-row query tiles against key_tile-key key tiles --
+so that partly filled tiles count as full ones:
+
+* forward schedule ("fwd"): the item's tiles, in order, are taken two at a time;
+  a pair of n tiles with key union [lo, hi) executes n * ceil((hi - lo) / key_tile)
+  tile steps;
+* backward schedule ("bwd", whole chunks): for every key tile [k0, k0 + key_tile)
+  of the chunk, k0 = cC, cC + key_tile, ..., below min((c+1)C, N), one step per
+  query tile whose key range meets it;
+* cost = steps * rows_per_tile * key_tile.
 """
 
 from __future__ import annotations
 
 from typing import Dict, List, Tuple
 
-from .mask import chunk_entries, chunk_pairs
+from .mask import chunk_entries, chunk_pairs, num_chunks
+
+
+def query_tiles(sample_lens, anchors, block_size: int, kv_chunk: int, G: int, rows_per_tile: int = 128,
+                block_keys_in_context: bool = False) -> Dict[int, List[Tuple[int, int]]]:
+    """Per chunk, its query tiles' key ranges [min lo, max hi): consecutive groups of
+    rows_per_tile // (G * bs) entries in (lo, hi, block) order."""
+    bs = int(block_size)
+    bpt = rows_per_tile // (G * bs)
+    per_chunk: Dict[int, list] = {}
+    for (c, b, lo, hi) in chunk_entries(sample_lens, anchors, kv_chunk, bs, block_keys_in_context):
+        per_chunk.setdefault(c, []).append((lo, hi, b))
+    out = {}
+    for c in sorted(per_chunk):
+        ents = sorted(per_chunk[c])
+        out[c] = [(min(e[0] for e in ents[i:i + bpt]), max(e[1] for e in ents[i:i + bpt]))
+                  for i in range(0, len(ents), bpt)]
+    return out
+
+
+def fwd_tile_cost(tiles, rows_per_tile: int = 128, key_tile: int = 128) -> int:
+    """Executed (row, key) pairs of the forward kernel over these tiles, taken two at a time."""
+    steps = 0
+    for i in range(0, len(tiles), 2):
+        pair = tiles[i:i + 2]
+        lo = min(t[0] for t in pair)
+        hi = max(t[1] for t in pair)
+        steps += len(pair) * ((hi - lo + key_tile - 1) // key_tile)
+    return steps * rows_per_tile * key_tile
+
+
+def bwd_tile_cost(tiles, c: int, kv_chunk: int, context_len: int, rows_per_tile: int = 128,
+                  key_tile: int = 128) -> int:
+    """Executed (row, key) pairs of the dK/dV kernel on chunk c: per key tile of the chunk,
+    one step per query tile meeting it."""
+    steps = 0
+    for k0 in range(c * kv_chunk, min((c + 1) * kv_chunk, context_len), key_tile):
+        steps += sum(1 for (lo, hi) in tiles if lo < k0 + key_tile and hi > k0)
+    return steps * rows_per_tile * key_tile
 
 
 def work_items(sample_lens, anchors, block_size: int, kv_chunk: int, num_q_heads: int,
                num_kv_heads: int, q_slice: int = 0, rows_per_tile: int = 128,
-               block_keys_in_context: bool = False) -> List[Tuple[Tuple[int, int, int], int]]:
-    """All work items ((c, g, slice), cost), zero-cost ones included."""
+               block_keys_in_context: bool = False, tile_cost: str = ""
+               ) -> List[Tuple[Tuple[int, int, int], int]]:
+    """All work items ((c, g, slice), cost), zero-cost ones included.  tile_cost: "" (the
+    pages' pair cost), "fwd" or "bwd" (executed tile work of that schedule's kernel)."""
     G = num_q_heads // num_kv_heads
     bs = int(block_size)
     items = []
+    if tile_cost:
+        N = int(sum(int(L) for L in sample_lens))
+        tiles = query_tiles(sample_lens, anchors, bs, kv_chunk, G, rows_per_tile, block_keys_in_context)
+        for c in range(num_chunks(N, kv_chunk)):
+            ts = tiles.get(c, [])
+            groups = [ts] if q_slice <= 0 else [ts[i:i + q_slice] for i in range(0, len(ts), q_slice)]
+            for s, grp in enumerate(groups):
+                cost = (bwd_tile_cost(grp, c, kv_chunk, N, rows_per_tile) if tile_cost == "bwd"
+                        else fwd_tile_cost(grp, rows_per_tile))
+                for g in range(num_kv_heads):
+                    items.append(((c, g, s), int(cost)))
+        return items
     if q_slice <= 0:
         pairs = chunk_pairs(sample_lens, anchors, bs, kv_chunk, block_keys_in_context)
         for c, p in enumerate(pairs):
