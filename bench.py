@@ -43,17 +43,18 @@ sys.path.insert(0, ROOT)
 
 METRIC = "masked-pair attn TFLOP/s fwd/bwd, % of BF16 tensor peak; LPT imbalance %"
 
-# DRAM bytes per launch at the default (64k context / 8k queries) workload, from
-# one ncu capture (dram__bytes_read.sum + dram__bytes_write.sum, mean of 5
-# launches), keyed by kernel, with the sha256 of the sources the kernel was
-# built from when it was taken; a changed source voids the figure.
+# DRAM bytes per launch at the default (64k context / 8k queries) workload and
+# schedule (backward LPT by tile cost), from one ncu capture
+# (dram__bytes_read.sum + dram__bytes_write.sum, mean of 5 launches), keyed by
+# kernel, with the sha256 of the sources the kernel was built from when it was
+# taken; a changed source voids the figure.
 NCU_TRAFFIC = {
-    "fwd_partial": {"bytes": 2082256026, "src": "9a3f68c6308f2a0e"},
-    "merge": {"bytes": 1557937152, "src": "b87601659b20c86d"},
-    "bwd_delta": {"bytes": 201935719, "src": "b87601659b20c86d"},
-    "bwd_dkdv": {"bytes": 1651331277, "src": "1ddaa484886212e9"},
-    "bwd_dq": {"bytes": 2313403597, "src": "1ddaa484886212e9"},
-    "bwd_reduce": {"bytes": 1554807655, "src": "b87601659b20c86d"},
+    "fwd_partial": {"bytes": 2075161140, "src": "9a3f68c6308f2a0e"},
+    "merge": {"bytes": 1558043085, "src": "b87601659b20c86d"},
+    "bwd_delta": {"bytes": 201970791, "src": "b87601659b20c86d"},
+    "bwd_dkdv": {"bytes": 1653801319, "src": "1ddaa484886212e9"},
+    "bwd_dq": {"bytes": 2306389299, "src": "1ddaa484886212e9"},
+    "bwd_reduce": {"bytes": 1554170317, "src": "b87601659b20c86d"},
 }
 _KERNEL_SOURCES = {
     "fwd_partial": ("fwd_partial_sm100.cu", "sm100.cuh", "splitkv_internal.h"),
@@ -256,7 +257,8 @@ def run_ours(args, world, rank, local):
     t = {n: up(n) for n in ("q", "k", "v", "kb", "vb", "dout")}
     d, Hq, Nq = w.head_dim, w.num_q_heads, w.num_queries
     plan = skv.splitkv_plan(w.sample_lens, w.anchors, w.block_size, Hq, w.num_kv_heads, d, w.kv_chunk, W,
-                            num_bwd_workers=Wb, q_slice=args.q_slice, partial_bf16=args.partial_bf16)
+                            num_bwd_workers=Wb, q_slice=args.q_slice, partial_bf16=args.partial_bf16,
+                            tile_cost=args.lpt_cost == "tiles")
     plan.upload(stream)
     st = plan.stats()
     ws_f = torch.empty(skv.splitkv_workspace_size(plan, skv.WS_FWD), dtype=torch.uint8, device=dev)
@@ -387,6 +389,7 @@ def run_ours(args, world, rank, local):
                    "num_anchors": int(w.anchors.size), "block_size": w.block_size, "heads": [Hq, w.num_kv_heads],
                    "head_dim": d, "kv_chunk": w.kv_chunk, "fwd_workers": W, "bwd_workers": Wb,
                    "q_slice": args.q_slice, "partial_records": "bf16" if args.partial_bf16 else "f32",
+                   "lpt_cost": args.lpt_cost,
                    "parallelism": "replicas" if world > 1 else "single",
                    "l2": "no flush: each step touches ~4 GB (> 126 MB L2)"},
         "fwd_tflops": flops_fwd / (fwd_ms * 1e-3) / 1e12,
@@ -453,7 +456,8 @@ def run_e2e(args, w, plan, dev, stream, flops_step, world=1):
     d, Hq, Nq = w.head_dim, w.num_q_heads, w.num_queries
     att = SplitKVAttention(w.sample_lens, w.anchors, w.block_size, Hq, w.num_kv_heads, d, w.kv_chunk,
                            num_workers=plan.problem.num_workers, num_bwd_workers=plan.problem.num_bwd_workers,
-                           q_slice=plan.problem.q_slice, device=dev, partial_bf16=args.partial_bf16)
+                           q_slice=plan.problem.q_slice, device=dev, partial_bf16=args.partial_bf16,
+                           tile_cost=args.lpt_cost == "tiles")
     dv = {n: torch.empty(x.shape, dtype=x.dtype, device=dev) for n, x in host.items()}
     outs_h = {"o": torch.empty((Nq, Hq, d), dtype=torch.float32).pin_memory(),
               "lse": torch.empty((Nq, Hq), dtype=torch.float32).pin_memory()}
@@ -588,6 +592,9 @@ def main(argv=None):
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-clocks", action="store_true")
+    ap.add_argument("--lpt-cost", choices=["tiles", "pairs"], default="tiles",
+                    help="LPT item cost of the backward (dK/dV) schedule: executed tile work (default) or "
+                         "the allowed pairs of the pages' rule; the forward schedule uses the pairs")
     ap.add_argument("--partial-bf16", action="store_true",
                     help="store the partial records (O_c, dQ partials) as bf16 (plan flag; default float32)")
     args = ap.parse_args(argv)

@@ -75,7 +75,8 @@ int validate(const splitkv_problem* p) {
       p->num_bwd_workers < 0 || p->q_slice < 0)
     return SPLITKV_ERR_INVALID_ARG;
   if (p->num_q_heads % p->num_kv_heads) return SPLITKV_ERR_INVALID_ARG;
-  if (p->flags & ~uint32_t(SPLITKV_FLAG_EQUAL_COUNT | SPLITKV_FLAG_BLOCK_KEYS_IN_CONTEXT | SPLITKV_FLAG_PARTIAL_BF16))
+  if (p->flags & ~uint32_t(SPLITKV_FLAG_EQUAL_COUNT | SPLITKV_FLAG_BLOCK_KEYS_IN_CONTEXT | SPLITKV_FLAG_PARTIAL_BF16 |
+                           SPLITKV_FLAG_TILE_COST))
     return SPLITKV_ERR_INVALID_ARG;
   int64_t N = 0;
   for (int s = 0; s < p->num_samples; ++s) {
@@ -255,6 +256,19 @@ int build(splitkv_plan_t* P, const splitkv_problem* p) {
     for (int e = P->tiles[t].x; e < P->tiles[t].y; ++e) keys += uint64_t(P->entries[e].z - P->entries[e].y);
     return keys * uint64_t(P->bs) * uint64_t(P->G);
   };
+  // tile cost of the backward schedule (SPLITKV_FLAG_TILE_COST): executed (row, key)
+  // pairs of whole tile steps of the dK/dV kernel, whose key tiles hold 128 keys
+  constexpr int kKeyTile = 128;
+  const bool by_tiles = (P->flags & SPLITKV_FLAG_TILE_COST) != 0;
+  const uint64_t step_pairs = uint64_t(splitkv::kTileRows) * uint64_t(kKeyTile);
+  auto bwd_exec = [&](int c, int t0, int t1) {   // per key tile of chunk c, the tiles that meet it
+    const int64_t c0 = int64_t(c) * P->C, c1 = std::min<int64_t>(c0 + P->C, P->N);
+    uint64_t steps = 0;
+    for (int64_t k0 = c0; k0 < c1; k0 += kKeyTile)
+      for (int t = t0; t < t1; ++t)
+        if (P->tiles[t].z < k0 + kKeyTile && P->tiles[t].w > k0) ++steps;
+    return steps * step_pairs;
+  };
   P->fwd_items.clear();
   P->bwd_items.clear();
   P->zero_chunks.clear();
@@ -265,7 +279,8 @@ int build(splitkv_plan_t* P, const splitkv_problem* p) {
       continue;
     }
     const uint64_t whole = P->chunk_pairs[c] * uint64_t(P->G);
-    for (int g = 0; g < P->Hkv; ++g) P->bwd_items.push_back(Item{c, g, 0, t0, t1, whole});
+    const uint64_t bcost = by_tiles ? bwd_exec(c, t0, t1) : whole;
+    for (int g = 0; g < P->Hkv; ++g) P->bwd_items.push_back(Item{c, g, 0, t0, t1, bcost});
     if (P->q_slice <= 0) {
       for (int g = 0; g < P->Hkv; ++g) P->fwd_items.push_back(Item{c, g, 0, t0, t1, whole});
     } else {

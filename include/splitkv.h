@@ -86,6 +86,15 @@ extern "C" {
  * tcgen05 kernels only (head_dim 128, G * bs a multiple of 8): attention calls
  * of other plans return SPLITKV_ERR_UNSUPPORTED. */
 #define SPLITKV_FLAG_PARTIAL_BF16  4u
+/* Tile cost for the backward LPT schedule: a (chunk, KV head) item of the
+ * dK/dV kernel costs the work that kernel executes, in (row, key) pairs of
+ * whole 128-row x 128-key tile steps -- for every 128-key tile of the chunk,
+ * the query tiles that meet it -- instead of the allowed pairs (the pages'
+ * "actual attention usage", the default).  Partly filled tiles then count as
+ * what they cost, which evens out the measured per-CTA busy time of the dK/dV
+ * kernel.  The forward schedule (used by the forward and dQ kernels), the
+ * contiguous baseline and the pair counts keep the pair cost. */
+#define SPLITKV_FLAG_TILE_COST  8u
 
 /* ---- dtype codes (o) ------------------------------------------------------- */
 #define SPLITKV_DTYPE_F32   0

@@ -23,18 +23,13 @@ Readings where the pages are silent (integer arithmetic, so bit-exact):
 * the "unbalanced" baseline keeps chunks in contiguous order: the n_chunks * Hkv
   unsliced items in (c, g) order, item i to worker floor(i W / n).
 
-Optional tile cost (this library's refinement for its kernels, not the pages'
-rule): the cost of an item is the work its kernel executes, in (row, key) pairs
-of whole tiles -- rows_per_tile-row query tiles against key_tile-key key tiles --
-so that partly filled tiles count as full ones:
-
-* forward schedule ("fwd"): the item's tiles, in order, are taken two at a time;
-  a pair of n tiles with key union [lo, hi) executes n * ceil((hi - lo) / key_tile)
-  tile steps;
-* backward schedule ("bwd", whole chunks): for every key tile [k0, k0 + key_tile)
-  of the chunk, k0 = cC, cC + key_tile, ..., below min((c+1)C, N), one step per
-  query tile whose key range meets it;
-* cost = steps * rows_per_tile * key_tile.
+Optional tile cost of the backward schedule (this library's refinement for its
+dK/dV kernel, not the pages' rule): the cost of a (chunk, head) item is the work
+that kernel executes, in (row, key) pairs of whole tiles -- rows_per_tile-row
+query tiles against key_tile-key key tiles -- so that partly filled tiles count
+as full ones: for every key tile [k0, k0 + key_tile) of the chunk, k0 = cC,
+cC + key_tile, ..., below min((c+1)C, N), one step per query tile whose key
+range meets it; cost = steps * rows_per_tile * key_tile.
 """
 
 from __future__ import annotations
@@ -61,17 +56,6 @@ def query_tiles(sample_lens, anchors, block_size: int, kv_chunk: int, G: int, ro
     return out
 
 
-def fwd_tile_cost(tiles, rows_per_tile: int = 128, key_tile: int = 128) -> int:
-    """Executed (row, key) pairs of the forward kernel over these tiles, taken two at a time."""
-    steps = 0
-    for i in range(0, len(tiles), 2):
-        pair = tiles[i:i + 2]
-        lo = min(t[0] for t in pair)
-        hi = max(t[1] for t in pair)
-        steps += len(pair) * ((hi - lo + key_tile - 1) // key_tile)
-    return steps * rows_per_tile * key_tile
-
-
 def bwd_tile_cost(tiles, c: int, kv_chunk: int, context_len: int, rows_per_tile: int = 128,
                   key_tile: int = 128) -> int:
     """Executed (row, key) pairs of the dK/dV kernel on chunk c: per key tile of the chunk,
@@ -84,24 +68,22 @@ def bwd_tile_cost(tiles, c: int, kv_chunk: int, context_len: int, rows_per_tile:
 
 def work_items(sample_lens, anchors, block_size: int, kv_chunk: int, num_q_heads: int,
                num_kv_heads: int, q_slice: int = 0, rows_per_tile: int = 128,
-               block_keys_in_context: bool = False, tile_cost: str = ""
+               block_keys_in_context: bool = False, tile_cost: bool = False
                ) -> List[Tuple[Tuple[int, int, int], int]]:
-    """All work items ((c, g, slice), cost), zero-cost ones included.  tile_cost: "" (the
-    pages' pair cost), "fwd" or "bwd" (executed tile work of that schedule's kernel)."""
+    """All work items ((c, g, slice), cost), zero-cost ones included.  tile_cost: whole-chunk
+    items of the backward schedule costed by the dK/dV kernel's executed tile work."""
     G = num_q_heads // num_kv_heads
     bs = int(block_size)
     items = []
     if tile_cost:
+        if q_slice > 0:
+            raise ValueError("the tile cost applies to the backward schedule (whole chunks)")
         N = int(sum(int(L) for L in sample_lens))
         tiles = query_tiles(sample_lens, anchors, bs, kv_chunk, G, rows_per_tile, block_keys_in_context)
         for c in range(num_chunks(N, kv_chunk)):
-            ts = tiles.get(c, [])
-            groups = [ts] if q_slice <= 0 else [ts[i:i + q_slice] for i in range(0, len(ts), q_slice)]
-            for s, grp in enumerate(groups):
-                cost = (bwd_tile_cost(grp, c, kv_chunk, N, rows_per_tile) if tile_cost == "bwd"
-                        else fwd_tile_cost(grp, rows_per_tile))
-                for g in range(num_kv_heads):
-                    items.append(((c, g, s), int(cost)))
+            cost = bwd_tile_cost(tiles.get(c, []), c, kv_chunk, N, rows_per_tile)
+            for g in range(num_kv_heads):
+                items.append(((c, g, 0), int(cost)))
         return items
     if q_slice <= 0:
         pairs = chunk_pairs(sample_lens, anchors, bs, kv_chunk, block_keys_in_context)

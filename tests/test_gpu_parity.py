@@ -68,7 +68,7 @@ def test_small_ragged_fwd_bwd_elementwise(splitkv, case):
 
 @pytest.mark.parametrize("opts", [
     dict(W=7), dict(W=1), dict(W=300, Wb=5), dict(q_slice=1), dict(q_slice=2, equal_count=True),
-    dict(o_dtype="bf16"),
+    dict(o_dtype="bf16"), dict(q_slice=2, tile_cost=True), dict(tile_cost=True, Wb=5),
 ])
 def test_schedules_and_options_same_result(splitkv, opts):
     w = small()

@@ -128,11 +128,9 @@ def test_tile_cost_hand_worked():
     tiles = lpt.query_tiles(lens, anchors, bs, C, 1, rows_per_tile=32)
     # chunk 0 entries (0,50),(0,60),(0,128),(0,128) -> tiles [0,60), [0,128); chunk 1: [128,250)
     assert tiles == {0: [(0, 60), (0, 128)], 1: [(128, 250)]}
-    assert lpt.fwd_tile_cost(tiles[0], 32) == 2 * 1 * 32 * 128      # one pair, one key tile
-    assert lpt.fwd_tile_cost(tiles[1], 32) == 1 * 1 * 32 * 128
     assert lpt.bwd_tile_cost(tiles[0], 0, C, 300, 32) == 2 * 32 * 128   # key tile [0,128): both tiles
     assert lpt.bwd_tile_cost(tiles[1], 1, C, 300, 32) == 1 * 32 * 128
-    items = dict(lpt.work_items(lens, anchors, bs, C, 1, 1, rows_per_tile=32, tile_cost="bwd"))
+    items = dict(lpt.work_items(lens, anchors, bs, C, 1, 1, rows_per_tile=32, tile_cost=True))
     assert items == {(0, 0, 0): 8192, (1, 0, 0): 4096, (2, 0, 0): 0}
     # the pages' pair cost of the same chunks: bs * sum(hi - lo)
     pairs = dict(lpt.work_items(lens, anchors, bs, C, 1, 1))
@@ -149,23 +147,17 @@ def test_tile_cost_bounds_pair_cost(seed):
     bs = [4, 8, 16][seed % 3]
     anchors = rng.integers(0, N, size=rng.integers(1, 30)).tolist()
     C = int(rng.integers(16, 300))
-    for q_slice, mode in ((0, "bwd"), (0, "fwd"), (1, "fwd"), (3, "fwd")):
-        tc = dict(lpt.work_items(lens, anchors, bs, C, heads[0], heads[1], q_slice=q_slice, tile_cost=mode))
-        pc = dict(lpt.work_items(lens, anchors, bs, C, heads[0], heads[1], q_slice=q_slice))
-        assert set(pc) <= set(tc)
-        for key, cost in pc.items():
-            assert tc[key] >= cost, (q_slice, mode, key)
+    tc = dict(lpt.work_items(lens, anchors, bs, C, heads[0], heads[1], tile_cost=True))
+    pc = dict(lpt.work_items(lens, anchors, bs, C, heads[0], heads[1]))
+    assert set(pc) == set(tc)
+    for key, cost in pc.items():
+        assert tc[key] >= cost, key
 
 
 def test_tile_cost_equals_pair_cost_for_full_aligned_tiles():
     # one block per 128-row tile (G * bs = 128) and every interval a whole number of key tiles
     lens, bs, C = [1024], 16, 256
     anchors = [512, 512, 768, 768]
-    for mode, q_slice in (("bwd", 0), ("fwd", 0), ("fwd", 2)):
-        tc = dict(lpt.work_items(lens, anchors, bs, C, 8, 1, q_slice=q_slice, tile_cost=mode))
-        pc = dict(lpt.work_items(lens, anchors, bs, C, 8, 1, q_slice=q_slice))
-        if mode == "bwd":
-            assert tc == pc
-        else:   # the forward pairs tiles over their key union: equal when a pair shares its interval
-            assert all(tc[k] >= pc[k] for k in pc)
-            assert tc[(0, 0, 0)] == pc[(0, 0, 0)]
+    tc = dict(lpt.work_items(lens, anchors, bs, C, 8, 1, tile_cost=True))
+    pc = dict(lpt.work_items(lens, anchors, bs, C, 8, 1))
+    assert tc == pc

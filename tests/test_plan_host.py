@@ -14,14 +14,15 @@ from oracle import mask as omask
 from synth import CONFIGS, make_workload
 
 
-def _plan(skv, lens, anchors, bs, Hq, Hkv, d, C, W, Wb=0, q_slice=0, eq=False, rb=False):
+def _plan(skv, lens, anchors, bs, Hq, Hkv, d, C, W, Wb=0, q_slice=0, eq=False, rb=False, tc=False):
     return skv.splitkv_plan(lens, anchors, bs, Hq, Hkv, d, C, W, num_bwd_workers=Wb, q_slice=q_slice,
-                            equal_count=eq, block_keys_in_context=rb)
+                            equal_count=eq, block_keys_in_context=rb, tile_cost=tc)
 
 
-def _check_against_oracle(skv, lens, anchors, bs, Hq, Hkv, C, W, Wb=0, q_slice=0, eq=False, d=64, rb=False):
-    """rb: reading B of the block keys (block keys in the context)."""
-    plan = _plan(skv, lens, anchors, bs, Hq, Hkv, d, C, W, Wb, q_slice, eq, rb)
+def _check_against_oracle(skv, lens, anchors, bs, Hq, Hkv, C, W, Wb=0, q_slice=0, eq=False, d=64, rb=False,
+                          tc=False):
+    """rb: reading B of the block keys (block keys in the context); tc: tile cost."""
+    plan = _plan(skv, lens, anchors, bs, Hq, Hkv, d, C, W, Wb, q_slice, eq, rb, tc)
     G = Hq // Hkv
     # entries: same set per chunk, record order sorted by (lo, hi, block) inside each chunk
     ent = plan.export(skv.EXPORT_ENTRIES).reshape(-1, 4)
@@ -33,10 +34,11 @@ def _check_against_oracle(skv, lens, anchors, bs, Hq, Hkv, C, W, Wb=0, q_slice=0
     pairs = plan.export(skv.EXPORT_CHUNK_PAIRS)
     assert pairs.tolist() == omask.chunk_pairs(lens, anchors, bs, C, rb).tolist()
     # forward schedule (possibly sliced) and backward schedule (whole chunks)
-    for what, loads_what, workers, qs in ((skv.EXPORT_FWD_SCHEDULE, skv.EXPORT_FWD_LOADS, W, q_slice),
-                                          (skv.EXPORT_BWD_SCHEDULE, skv.EXPORT_BWD_LOADS, Wb or W, 0)):
+    for what, loads_what, workers, qs, mode in (
+            (skv.EXPORT_FWD_SCHEDULE, skv.EXPORT_FWD_LOADS, W, q_slice, False),
+            (skv.EXPORT_BWD_SCHEDULE, skv.EXPORT_BWD_LOADS, Wb or W, 0, tc)):
         items = olpt.work_items(lens, anchors, bs, C, Hq, Hkv, q_slice=qs, rows_per_tile=128,
-                                block_keys_in_context=rb)
+                                block_keys_in_context=rb, tile_cost=mode)
         lists, loads = olpt.lpt(items, workers, equal_count=eq)
         cost = dict(items)
         sched = plan.export(what).reshape(-1, 5)
@@ -71,24 +73,27 @@ def _check_against_oracle(skv, lens, anchors, bs, Hq, Hkv, C, W, Wb=0, q_slice=0
     q_slice=st.integers(0, 3),
     eq=st.booleans(),
     rb=st.booleans(),
+    tc=st.booleans(),
     seed=st.integers(0, 2 ** 31 - 1),
 )
-def test_random_problems_bit_exact(splitkv, lens, n_anchor, heads, bs, C, W, Wb, q_slice, eq, rb, seed):
+def test_random_problems_bit_exact(splitkv, lens, n_anchor, heads, bs, C, W, Wb, q_slice, eq, rb, tc, seed):
     Hq, Hkv = heads
     if 128 % ((Hq // Hkv) * bs):
         return
     rng = np.random.default_rng(seed)
     N = sum(lens)
     anchors = rng.integers(0, N, size=n_anchor).astype(np.int32)   # any order, repeats allowed
-    _check_against_oracle(splitkv, lens, anchors, bs, Hq, Hkv, C, W, Wb, q_slice, eq, rb=rb)
+    _check_against_oracle(splitkv, lens, anchors, bs, Hq, Hkv, C, W, Wb, q_slice, eq, rb=rb, tc=tc)
 
 
 @pytest.mark.parametrize("name", ["tiny", "drafter", "budget", "skew", "bwd"])
-@pytest.mark.parametrize("q_slice,eq,rb", [(0, False, False), (2, False, False), (0, True, False), (2, False, True)])
-def test_workload_plans_bit_exact(splitkv, name, q_slice, eq, rb):
+@pytest.mark.parametrize("q_slice,eq,rb,tc", [(0, False, False, False), (2, False, False, False),
+                                               (0, True, False, False), (2, False, True, False),
+                                               (2, False, False, True), (0, True, False, True)])
+def test_workload_plans_bit_exact(splitkv, name, q_slice, eq, rb, tc):
     w = make_workload(name, tensors=False)
     _check_against_oracle(splitkv, w.sample_lens, w.anchors, w.block_size, w.num_q_heads, w.num_kv_heads,
-                          w.kv_chunk, 148, 0, q_slice, eq, d=w.head_dim, rb=rb)
+                          w.kv_chunk, 148, 0, q_slice, eq, d=w.head_dim, rb=rb, tc=tc)
 
 
 def test_anchor_at_sample_start_and_chunk_straddle(splitkv):
