@@ -1,6 +1,6 @@
-// TMA tensor-map encoding for the tcgen05 kernels (host side).  The driver
-// entry point is looked up through the runtime, so the library carries no
-// link-time dependency on libcuda.
+// TMA tensor-map encoding for the tcgen05 kernels (host side).  The CUDA
+// driver's cuTensorMapEncodeTiled is looked up through the runtime, so the
+// library carries no link-time dependency on libcuda.
 #include <cuda.h>
 #include <cuda_runtime.h>
 
