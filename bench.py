@@ -341,6 +341,13 @@ def run_ours(args, world, rank, local):
         x = np.asarray(x, dtype=np.float64)
         return float(x.max() / x.mean() - 1.0) if x.size and x.mean() > 0 else 0.0
 
+    if args.dump_cta_times and rank == 0:
+        with open(args.dump_cta_times, "w") as f:
+            json.dump({"workload": args.workload, "anchors": int(w.anchors.size), "q_slice": args.q_slice,
+                       "lpt_cost": args.lpt_cost, "partial_bf16": bool(args.partial_bf16),
+                       "fwd_workers": W, "bwd_workers": Wb,
+                       "fwd_ns": [int(x) for x in cta_f], "bwd_ns": [int(x) for x in cta_b]}, f)
+
     pairs = st["context_pairs"] + st["block_pairs"]
     flops_fwd = 4.0 * d * pairs
     flops_bwd = 10.0 * d * pairs
@@ -595,6 +602,9 @@ def main(argv=None):
     ap.add_argument("--lpt-cost", choices=["tiles", "pairs"], default="tiles",
                     help="LPT item cost of the backward (dK/dV) schedule: executed tile work (default) or "
                          "the allowed pairs of the pages' rule; the forward schedule uses the pairs")
+    ap.add_argument("--dump-cta-times", default=None, metavar="PATH",
+                    help="write the measured per-CTA busy times of the last step (fwd partial and dK/dV "
+                         "kernels, ns) with the schedule options to PATH as JSON")
     ap.add_argument("--partial-bf16", action="store_true",
                     help="store the partial records (O_c, dQ partials) as bf16 (plan flag; default float32)")
     args = ap.parse_args(argv)
