@@ -232,6 +232,24 @@ def _bwd_is_two_launches(w) -> bool:
             and os.environ.get("SPLITKV_BWD_KERNEL") != "mma")
 
 
+def bench_config(args, w, W, Wb, world):
+    """The workload and launch options of a bench line (both arms report the same)."""
+    return {"workload": w.config.description, "context_len": w.context_len, "num_queries": w.num_queries,
+            "num_anchors": int(w.anchors.size), "block_size": w.block_size, "heads": [w.num_q_heads, w.num_kv_heads],
+            "head_dim": w.head_dim, "kv_chunk": w.kv_chunk, "fwd_workers": W, "bwd_workers": Wb,
+            "q_slice": args.q_slice, "partial_records": "bf16" if args.partial_bf16 else "f32",
+            "lpt_cost": args.lpt_cost,
+            "parallelism": "replicas" if world > 1 else "single",
+            "l2": "no flush: each step touches ~4 GB (> 126 MB L2)"}
+
+
+def _workers(args):
+    """Forward and backward CTA counts: the options, else the SM count of the GPU (None without one)."""
+    import torch
+    sms = torch.cuda.get_device_properties(0).multi_processor_count if torch.cuda.is_available() else None
+    return args.workers or sms, args.bwd_workers or sms
+
+
 def run_ours(args, world, rank, local):
     import torch
     import torch.distributed as dist
@@ -392,13 +410,7 @@ def run_ours(args, world, rank, local):
         "vs_baseline": None,
         "dtype": "bf16",
         "data": "synthetic",
-        "config": {"workload": w.config.description, "context_len": w.context_len, "num_queries": Nq,
-                   "num_anchors": int(w.anchors.size), "block_size": w.block_size, "heads": [Hq, w.num_kv_heads],
-                   "head_dim": d, "kv_chunk": w.kv_chunk, "fwd_workers": W, "bwd_workers": Wb,
-                   "q_slice": args.q_slice, "partial_records": "bf16" if args.partial_bf16 else "f32",
-                   "lpt_cost": args.lpt_cost,
-                   "parallelism": "replicas" if world > 1 else "single",
-                   "l2": "no flush: each step touches ~4 GB (> 126 MB L2)"},
+        "config": bench_config(args, w, W, Wb, world),
         "fwd_tflops": flops_fwd / (fwd_ms * 1e-3) / 1e12,
         "bwd_tflops": flops_bwd / (bwd_ms * 1e-3) / 1e12,
         "pct_of_bf16_peak": 100.0 * value / world / peaks["bf16_tflops"],
@@ -574,15 +586,14 @@ def run_reference(args, world, rank):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * secs / args.steps,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic",
-            "config": {"workload": w.config.description, "context_len": w.context_len,
-                       "num_queries": w.num_queries, "parallelism": "single"},
+            "config": bench_config(args, w, *_workers(args), world),
             "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": _oracle_threads(), "kind": "oracle",
                              "sample": sample},
             "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
             "gpu_launches": 0}
 
 
-def main(argv=None):
+def parse_args(argv=None):
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=20)
@@ -610,6 +621,11 @@ def main(argv=None):
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
+    return args
+
+
+def main(argv=None):
+    args = parse_args(argv)
     world, rank, local = _dist()
     if world != args.gpus:
         print(f"warning: --gpus {args.gpus} but WORLD_SIZE={world}", file=sys.stderr)

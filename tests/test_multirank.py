@@ -21,9 +21,9 @@ def _worker(rank, world, port, q):
         ms = bench.max_over_ranks(10.0 + 5.0 * rank, torch.device("cpu"))
         w, r, l = bench._dist()
         # the reference arm runs on rank 0 only; other ranks exit without work
-        class A:
-            workload, anchors, steps, warmup, cpu_seconds = "tiny", None, 1, 3, 0.2
-        ref = bench.run_reference(A, w, r)
+        args = bench.parse_args(["--impl", "reference", "--workload", "tiny", "--steps", "1", "--warmup", "3",
+                                 "--cpu-seconds", "0.2"])
+        ref = bench.run_reference(args, w, r)
         q.put((rank, ms, (w, r, l), ref is None))
     finally:
         dist.destroy_process_group()
@@ -55,3 +55,24 @@ def test_whole_job_value_is_sum_of_replicas_over_max_time():
     one = bench.whole_job_tflops(1, 10, 1e12, 1000.0)
     two = bench.whole_job_tflops(2, 10, 1e12, 1000.0)
     assert one == pytest.approx(10.0) and two == pytest.approx(20.0)
+
+
+def test_reference_line_keeps_the_contract():
+    """The reference arm (the oracle on the host cores) prints the bench's metric, unit,
+    direction and config, with its own cpu_baseline and a zero-copy e2e."""
+    sys.path.insert(0, ROOT)
+    import bench
+    from synth import make_workload
+    args = bench.parse_args(["--impl", "reference", "--workload", "tiny", "--steps", "2", "--warmup", "3",
+                             "--cpu-seconds", "0.5"])
+    line = bench.run_reference(args, 1, 0)
+    assert line["impl"] == "reference" and line["metric"] == bench.METRIC and line["unit"] == "TFLOP/s"
+    assert line["higher_is_better"] is True and line["steps"] == 2 and line["warmup"] == 3
+    w = make_workload("tiny", with_grad=True)
+    assert line["config"] == bench.bench_config(args, w, *bench._workers(args), 1)
+    assert line["value"] > 0 and line["cpu_baseline"]["value"] == line["value"]
+    assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["cores"] >= 1
+    assert line["e2e"] == {"value": line["value"], "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                           "d2h_bytes_per_step": 0}
+    import json
+    json.dumps(line)
