@@ -24,6 +24,7 @@ FLAG_EQUAL_COUNT = 1
 FLAG_BLOCK_KEYS_IN_CONTEXT = 2
 FLAG_PARTIAL_BF16 = 4
 FLAG_TILE_COST = 8
+FLAG_FWD_TILE_COST = 16
 
 STATIC_SCRATCH_BYTES = 16 << 20
 

@@ -76,7 +76,7 @@ int validate(const splitkv_problem* p) {
     return SPLITKV_ERR_INVALID_ARG;
   if (p->num_q_heads % p->num_kv_heads) return SPLITKV_ERR_INVALID_ARG;
   if (p->flags & ~uint32_t(SPLITKV_FLAG_EQUAL_COUNT | SPLITKV_FLAG_BLOCK_KEYS_IN_CONTEXT | SPLITKV_FLAG_PARTIAL_BF16 |
-                           SPLITKV_FLAG_TILE_COST))
+                           SPLITKV_FLAG_TILE_COST | SPLITKV_FLAG_FWD_TILE_COST))
     return SPLITKV_ERR_INVALID_ARG;
   int64_t N = 0;
   for (int s = 0; s < p->num_samples; ++s) {
@@ -269,6 +269,23 @@ int build(splitkv_plan_t* P, const splitkv_problem* p) {
         if (P->tiles[t].z < k0 + kKeyTile && P->tiles[t].w > k0) ++steps;
     return steps * step_pairs;
   };
+  // tile cost of the forward schedule (SPLITKV_FLAG_FWD_TILE_COST): the forward
+  // kernel runs tiles t0, t0 + 1 (then t0 + 2, t0 + 3, ...) together over the key
+  // tiles of their joint key range
+  const bool fwd_by_tiles = (P->flags & SPLITKV_FLAG_FWD_TILE_COST) != 0;
+  auto fwd_exec = [&](int t0, int t1) {
+    uint64_t steps = 0;
+    for (int t = t0; t < t1; t += 2) {
+      const int n = std::min(2, t1 - t);
+      int klo = P->tiles[t].z, khi = P->tiles[t].w;
+      if (n == 2) {
+        klo = std::min(klo, P->tiles[t + 1].z);
+        khi = std::max(khi, P->tiles[t + 1].w);
+      }
+      steps += uint64_t(n) * uint64_t((int64_t(khi) - klo + kKeyTile - 1) / kKeyTile);
+    }
+    return steps * step_pairs;
+  };
   P->fwd_items.clear();
   P->bwd_items.clear();
   P->zero_chunks.clear();
@@ -282,7 +299,8 @@ int build(splitkv_plan_t* P, const splitkv_problem* p) {
     const uint64_t bcost = by_tiles ? bwd_exec(c, t0, t1) : whole;
     for (int g = 0; g < P->Hkv; ++g) P->bwd_items.push_back(Item{c, g, 0, t0, t1, bcost});
     if (P->q_slice <= 0) {
-      for (int g = 0; g < P->Hkv; ++g) P->fwd_items.push_back(Item{c, g, 0, t0, t1, whole});
+      const uint64_t fcost = fwd_by_tiles ? fwd_exec(t0, t1) : whole;
+      for (int g = 0; g < P->Hkv; ++g) P->fwd_items.push_back(Item{c, g, 0, t0, t1, fcost});
     } else {
       // generated in (chunk, head, slice) order: the LPT sort relies on it for ties
       const size_t first = P->fwd_items.size();
@@ -290,7 +308,10 @@ int build(splitkv_plan_t* P, const splitkv_problem* p) {
       for (int s0 = t0; s0 < t1; s0 += P->q_slice, ++slice) {
         const int s1 = std::min(s0 + P->q_slice, t1);
         uint64_t cost = 0;
-        for (int t = s0; t < s1; ++t) cost += tile_cost(t);
+        if (fwd_by_tiles)
+          cost = fwd_exec(s0, s1);
+        else
+          for (int t = s0; t < s1; ++t) cost += tile_cost(t);
         P->fwd_items.push_back(Item{c, 0, slice, s0, s1, cost});
       }
       const size_t ns = P->fwd_items.size() - first;

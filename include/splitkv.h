@@ -95,6 +95,16 @@ extern "C" {
  * kernel.  The forward schedule (used by the forward and dQ kernels), the
  * contiguous baseline and the pair counts keep the pair cost. */
 #define SPLITKV_FLAG_TILE_COST  8u
+/* Tile cost for the forward LPT schedule: a forward item (a chunk, or a slice of
+ * q_slice query tiles, of one KV head) costs the work the forward kernel
+ * executes on it, in (row, key) pairs of whole 128 x 128 tile steps.  That
+ * kernel takes the item's query tiles two at a time, from the item's first
+ * tile, and runs both over the 128-key tiles of their joint key range, so a
+ * pair of tiles whose key ranges are [lo1, hi1) and [lo2, hi2) executes
+ * 2 * ceil((max(hi) - min(lo)) / 128) steps (1 * ... for a last single tile).
+ * The backward schedule, the contiguous baseline and the pair counts are not
+ * affected (see SPLITKV_FLAG_TILE_COST for the backward schedule). */
+#define SPLITKV_FLAG_FWD_TILE_COST  16u
 
 /* ---- dtype codes (o) ------------------------------------------------------- */
 #define SPLITKV_DTYPE_F32   0

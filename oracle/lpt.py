@@ -30,6 +30,13 @@ query tiles against key_tile-key key tiles -- so that partly filled tiles count
 as full ones: for every key tile [k0, k0 + key_tile) of the chunk, k0 = cC,
 cC + key_tile, ..., below min((c+1)C, N), one step per query tile whose key
 range meets it; cost = steps * rows_per_tile * key_tile.
+
+Optional tile cost of the forward schedule (the same refinement for the forward
+kernel): a forward item's query tiles are taken two at a time from its first
+tile, and each pair runs over the key tiles of its joint key range [min lo,
+max hi), starting at min lo; a pair costs 2 * ceil((max hi - min lo) / key_tile)
+steps (a last single tile, 1 * ceil((hi - lo) / key_tile)); cost = steps *
+rows_per_tile * key_tile.
 """
 
 from __future__ import annotations
@@ -66,15 +73,46 @@ def bwd_tile_cost(tiles, c: int, kv_chunk: int, context_len: int, rows_per_tile:
     return steps * rows_per_tile * key_tile
 
 
+def forward_tile_cost(tiles, rows_per_tile: int = 128, key_tile: int = 128) -> int:
+    """Executed (row, key) pairs of the forward kernel on one item's query tiles (their
+    key ranges, in item order): the tiles go in twos, each two over their joint key range."""
+    steps = 0
+    for i in range(0, len(tiles), 2):
+        two = tiles[i:i + 2]
+        lo = min(t[0] for t in two)
+        hi = max(t[1] for t in two)
+        n_key_tiles = -(-(hi - lo) // key_tile)
+        steps += len(two) * n_key_tiles
+    return steps * rows_per_tile * key_tile
+
+
 def work_items(sample_lens, anchors, block_size: int, kv_chunk: int, num_q_heads: int,
                num_kv_heads: int, q_slice: int = 0, rows_per_tile: int = 128,
-               block_keys_in_context: bool = False, tile_cost: bool = False
-               ) -> List[Tuple[Tuple[int, int, int], int]]:
+               block_keys_in_context: bool = False, tile_cost: bool = False,
+               fwd_tile_cost: bool = False) -> List[Tuple[Tuple[int, int, int], int]]:
     """All work items ((c, g, slice), cost), zero-cost ones included.  tile_cost: whole-chunk
-    items of the backward schedule costed by the dK/dV kernel's executed tile work."""
+    items of the backward schedule costed by the dK/dV kernel's executed tile work;
+    fwd_tile_cost: items of the forward schedule (sliced or not) costed by the forward
+    kernel's executed tile work."""
     G = num_q_heads // num_kv_heads
     bs = int(block_size)
     items = []
+    if fwd_tile_cost:
+        if tile_cost:
+            raise ValueError("tile_cost and fwd_tile_cost describe different schedules")
+        N = int(sum(int(L) for L in sample_lens))
+        tiles = query_tiles(sample_lens, anchors, bs, kv_chunk, G, rows_per_tile, block_keys_in_context)
+        for c in range(num_chunks(N, kv_chunk)):
+            ts = tiles.get(c, [])
+            if q_slice <= 0:
+                groups = [ts]
+            else:
+                groups = [ts[i:i + q_slice] for i in range(0, len(ts), q_slice)]
+            for s, grp in enumerate(groups):
+                cost = forward_tile_cost(grp, rows_per_tile)
+                for g in range(num_kv_heads):
+                    items.append(((c, g, s), int(cost)))
+        return items
     if tile_cost:
         if q_slice > 0:
             raise ValueError("the tile cost applies to the backward schedule (whole chunks)")

@@ -161,3 +161,56 @@ def test_tile_cost_equals_pair_cost_for_full_aligned_tiles():
     tc = dict(lpt.work_items(lens, anchors, bs, C, 8, 1, tile_cost=True))
     pc = dict(lpt.work_items(lens, anchors, bs, C, 8, 1))
     assert tc == pc
+
+
+# ---------------------------------------------------------------------------
+# optional tile cost of the forward schedule (tiles in twos over their joint key range)
+# ---------------------------------------------------------------------------
+
+def test_forward_tile_cost_hand_worked():
+    # samples [0, 300) and [300, 600); bs 16, G 1, 2-block (32-row) tiles, one 512-key chunk in use
+    lens, anchors, bs, C = [300, 300], [50, 60, 400, 410], 16, 512
+    tiles = lpt.query_tiles(lens, anchors, bs, C, 1, rows_per_tile=32)
+    # entries (0,50), (0,60), (300,400), (300,410) -> tiles [0,60), [300,410)
+    assert tiles == {0: [(0, 60), (300, 410)]}
+    # together they run over [0, 410): 4 key tiles each -> 8 steps
+    assert lpt.forward_tile_cost(tiles[0], 32) == 8 * 32 * 128
+    # alone: [0, 60) one key tile; [300, 410) one key tile starting at 300
+    assert lpt.forward_tile_cost(tiles[0][:1], 32) == 32 * 128
+    assert lpt.forward_tile_cost(tiles[0][1:], 32) == 32 * 128
+    whole = dict(lpt.work_items(lens, anchors, bs, C, 1, 1, rows_per_tile=32, fwd_tile_cost=True))
+    assert whole == {(0, 0, 0): 8 * 4096, (1, 0, 0): 0}
+    sliced = dict(lpt.work_items(lens, anchors, bs, C, 1, 1, q_slice=1, rows_per_tile=32, fwd_tile_cost=True))
+    assert sliced == {(0, 0, 0): 4096, (0, 0, 1): 4096}
+    # the pages' pair cost of the chunk: bs * sum(hi - lo)
+    assert dict(lpt.work_items(lens, anchors, bs, C, 1, 1)) == {(0, 0, 0): 16 * (50 + 60 + 100 + 110), (1, 0, 0): 0}
+    with pytest.raises(ValueError):
+        lpt.work_items(lens, anchors, bs, C, 1, 1, tile_cost=True, fwd_tile_cost=True)
+
+
+@pytest.mark.parametrize("seed", range(12))
+def test_forward_tile_cost_bounds_pair_cost(seed):
+    """Executed tile work covers every allowed pair, sliced or not."""
+    rng = np.random.default_rng(50 + seed)
+    lens = rng.integers(1, 400, size=rng.integers(1, 5)).tolist()
+    N = sum(lens)
+    heads = [(1, 1), (4, 1), (8, 2)][seed % 3]
+    bs = [4, 8, 16][seed % 3]
+    anchors = rng.integers(0, N, size=rng.integers(1, 30)).tolist()
+    C = int(rng.integers(16, 300))
+    for q_slice in (0, 1, 2, 3):
+        tc = dict(lpt.work_items(lens, anchors, bs, C, heads[0], heads[1], q_slice=q_slice, fwd_tile_cost=True))
+        pc = dict(lpt.work_items(lens, anchors, bs, C, heads[0], heads[1], q_slice=q_slice))
+        assert {k for k, v in pc.items() if v} == {k for k, v in tc.items() if v}
+        for key, cost in pc.items():
+            assert tc[key] >= cost, (q_slice, key)
+
+
+def test_forward_tile_cost_equals_pair_cost_for_full_aligned_tiles():
+    # one block per 128-row tile, every interval whole key tiles, tiles of a pair alike
+    lens, bs, C = [1024], 16, 256
+    anchors = [512, 512, 768, 768]
+    for q_slice in (0, 1, 2):
+        tc = dict(lpt.work_items(lens, anchors, bs, C, 8, 1, q_slice=q_slice, fwd_tile_cost=True))
+        pc = dict(lpt.work_items(lens, anchors, bs, C, 8, 1, q_slice=q_slice))
+        assert {k: v for k, v in tc.items() if v} == {k: v for k, v in pc.items() if v}

@@ -14,15 +14,16 @@ from oracle import mask as omask
 from synth import CONFIGS, make_workload
 
 
-def _plan(skv, lens, anchors, bs, Hq, Hkv, d, C, W, Wb=0, q_slice=0, eq=False, rb=False, tc=False):
+def _plan(skv, lens, anchors, bs, Hq, Hkv, d, C, W, Wb=0, q_slice=0, eq=False, rb=False, tc=False, ftc=False):
     return skv.splitkv_plan(lens, anchors, bs, Hq, Hkv, d, C, W, num_bwd_workers=Wb, q_slice=q_slice,
-                            equal_count=eq, block_keys_in_context=rb, tile_cost=tc)
+                            equal_count=eq, block_keys_in_context=rb, tile_cost=tc, fwd_tile_cost=ftc)
 
 
 def _check_against_oracle(skv, lens, anchors, bs, Hq, Hkv, C, W, Wb=0, q_slice=0, eq=False, d=64, rb=False,
-                          tc=False):
-    """rb: reading B of the block keys (block keys in the context); tc: tile cost."""
-    plan = _plan(skv, lens, anchors, bs, Hq, Hkv, d, C, W, Wb, q_slice, eq, rb, tc)
+                          tc=False, ftc=False):
+    """rb: reading B of the block keys (block keys in the context); tc / ftc: tile cost of the
+    backward / forward schedule."""
+    plan = _plan(skv, lens, anchors, bs, Hq, Hkv, d, C, W, Wb, q_slice, eq, rb, tc, ftc)
     G = Hq // Hkv
     # entries: same set per chunk, record order sorted by (lo, hi, block) inside each chunk
     ent = plan.export(skv.EXPORT_ENTRIES).reshape(-1, 4)
@@ -34,11 +35,11 @@ def _check_against_oracle(skv, lens, anchors, bs, Hq, Hkv, C, W, Wb=0, q_slice=0
     pairs = plan.export(skv.EXPORT_CHUNK_PAIRS)
     assert pairs.tolist() == omask.chunk_pairs(lens, anchors, bs, C, rb).tolist()
     # forward schedule (possibly sliced) and backward schedule (whole chunks)
-    for what, loads_what, workers, qs, mode in (
-            (skv.EXPORT_FWD_SCHEDULE, skv.EXPORT_FWD_LOADS, W, q_slice, False),
-            (skv.EXPORT_BWD_SCHEDULE, skv.EXPORT_BWD_LOADS, Wb or W, 0, tc)):
+    for what, loads_what, workers, qs, mode, fmode in (
+            (skv.EXPORT_FWD_SCHEDULE, skv.EXPORT_FWD_LOADS, W, q_slice, False, ftc),
+            (skv.EXPORT_BWD_SCHEDULE, skv.EXPORT_BWD_LOADS, Wb or W, 0, tc, False)):
         items = olpt.work_items(lens, anchors, bs, C, Hq, Hkv, q_slice=qs, rows_per_tile=128,
-                                block_keys_in_context=rb, tile_cost=mode)
+                                block_keys_in_context=rb, tile_cost=mode, fwd_tile_cost=fmode)
         lists, loads = olpt.lpt(items, workers, equal_count=eq)
         cost = dict(items)
         sched = plan.export(what).reshape(-1, 5)
@@ -54,8 +55,8 @@ def _check_against_oracle(skv, lens, anchors, bs, Hq, Hkv, C, W, Wb=0, q_slice=0
     st_ = plan.stats()
     assert st_["context_pairs"] == Hq * int(pairs.sum())
     assert st_["block_pairs"] == (0 if rb else Hq * len(anchors) * bs * bs)
-    _, fl = olpt.lpt(olpt.work_items(lens, anchors, bs, C, Hq, Hkv, q_slice=q_slice, block_keys_in_context=rb), W,
-                     equal_count=eq)
+    _, fl = olpt.lpt(olpt.work_items(lens, anchors, bs, C, Hq, Hkv, q_slice=q_slice, block_keys_in_context=rb,
+                                     fwd_tile_cost=ftc), W, equal_count=eq)
     assert abs(st_["fwd_imbalance"] - olpt.imbalance(fl)) < 1e-12
     assert abs(st_["contig_imbalance"] - olpt.imbalance(cl)) < 1e-12
     plan.destroy()
@@ -74,26 +75,29 @@ def _check_against_oracle(skv, lens, anchors, bs, Hq, Hkv, C, W, Wb=0, q_slice=0
     eq=st.booleans(),
     rb=st.booleans(),
     tc=st.booleans(),
+    ftc=st.booleans(),
     seed=st.integers(0, 2 ** 31 - 1),
 )
-def test_random_problems_bit_exact(splitkv, lens, n_anchor, heads, bs, C, W, Wb, q_slice, eq, rb, tc, seed):
+def test_random_problems_bit_exact(splitkv, lens, n_anchor, heads, bs, C, W, Wb, q_slice, eq, rb, tc, ftc, seed):
     Hq, Hkv = heads
     if 128 % ((Hq // Hkv) * bs):
         return
     rng = np.random.default_rng(seed)
     N = sum(lens)
     anchors = rng.integers(0, N, size=n_anchor).astype(np.int32)   # any order, repeats allowed
-    _check_against_oracle(splitkv, lens, anchors, bs, Hq, Hkv, C, W, Wb, q_slice, eq, rb=rb, tc=tc)
+    _check_against_oracle(splitkv, lens, anchors, bs, Hq, Hkv, C, W, Wb, q_slice, eq, rb=rb, tc=tc, ftc=ftc)
 
 
 @pytest.mark.parametrize("name", ["tiny", "drafter", "budget", "skew", "bwd"])
-@pytest.mark.parametrize("q_slice,eq,rb,tc", [(0, False, False, False), (2, False, False, False),
-                                               (0, True, False, False), (2, False, True, False),
-                                               (2, False, False, True), (0, True, False, True)])
-def test_workload_plans_bit_exact(splitkv, name, q_slice, eq, rb, tc):
+@pytest.mark.parametrize("q_slice,eq,rb,tc,ftc", [(0, False, False, False, False), (2, False, False, False, False),
+                                                   (0, True, False, False, False), (2, False, True, False, False),
+                                                   (2, False, False, True, False), (0, True, False, True, False),
+                                                   (2, False, False, True, True), (0, False, True, False, True),
+                                                   (1, True, False, False, True)])
+def test_workload_plans_bit_exact(splitkv, name, q_slice, eq, rb, tc, ftc):
     w = make_workload(name, tensors=False)
     _check_against_oracle(splitkv, w.sample_lens, w.anchors, w.block_size, w.num_q_heads, w.num_kv_heads,
-                          w.kv_chunk, 148, 0, q_slice, eq, d=w.head_dim, rb=rb, tc=tc)
+                          w.kv_chunk, 148, 0, q_slice, eq, d=w.head_dim, rb=rb, tc=tc, ftc=ftc)
 
 
 def test_anchor_at_sample_start_and_chunk_straddle(splitkv):
