@@ -239,6 +239,7 @@ def bench_config(args, w, W, Wb, world):
             "head_dim": w.head_dim, "kv_chunk": w.kv_chunk, "fwd_workers": W, "bwd_workers": Wb,
             "q_slice": args.q_slice, "partial_records": "bf16" if args.partial_bf16 else "f32",
             "lpt_cost": args.lpt_cost, "fwd_lpt_cost": args.fwd_lpt_cost,
+            "item_claims": "run-time" if args.dynamic_claim else "static",
             "parallelism": "replicas" if world > 1 else "single",
             "l2": "no flush: each step touches ~4 GB (> 126 MB L2)"}
 
@@ -276,7 +277,8 @@ def run_ours(args, world, rank, local):
     d, Hq, Nq = w.head_dim, w.num_q_heads, w.num_queries
     plan = skv.splitkv_plan(w.sample_lens, w.anchors, w.block_size, Hq, w.num_kv_heads, d, w.kv_chunk, W,
                             num_bwd_workers=Wb, q_slice=args.q_slice, partial_bf16=args.partial_bf16,
-                            tile_cost=args.lpt_cost == "tiles", fwd_tile_cost=args.fwd_lpt_cost == "tiles")
+                            tile_cost=args.lpt_cost == "tiles", fwd_tile_cost=args.fwd_lpt_cost == "tiles",
+                            dynamic_claim=args.dynamic_claim)
     plan.upload(stream)
     st = plan.stats()
     ws_f = torch.empty(skv.splitkv_workspace_size(plan, skv.WS_FWD), dtype=torch.uint8, device=dev)
@@ -363,7 +365,7 @@ def run_ours(args, world, rank, local):
         with open(args.dump_cta_times, "w") as f:
             json.dump({"workload": args.workload, "anchors": int(w.anchors.size), "q_slice": args.q_slice,
                        "lpt_cost": args.lpt_cost, "fwd_lpt_cost": args.fwd_lpt_cost,
-                       "partial_bf16": bool(args.partial_bf16),
+                       "dynamic_claim": bool(args.dynamic_claim), "partial_bf16": bool(args.partial_bf16),
                        "fwd_workers": W, "bwd_workers": Wb,
                        "fwd_ns": [int(x) for x in cta_f], "bwd_ns": [int(x) for x in cta_b]}, f)
 
@@ -477,7 +479,8 @@ def run_e2e(args, w, plan, dev, stream, flops_step, world=1):
     att = SplitKVAttention(w.sample_lens, w.anchors, w.block_size, Hq, w.num_kv_heads, d, w.kv_chunk,
                            num_workers=plan.problem.num_workers, num_bwd_workers=plan.problem.num_bwd_workers,
                            q_slice=plan.problem.q_slice, device=dev, partial_bf16=args.partial_bf16,
-                           tile_cost=args.lpt_cost == "tiles", fwd_tile_cost=args.fwd_lpt_cost == "tiles")
+                           tile_cost=args.lpt_cost == "tiles", fwd_tile_cost=args.fwd_lpt_cost == "tiles",
+                           dynamic_claim=args.dynamic_claim)
     dv = {n: torch.empty(x.shape, dtype=x.dtype, device=dev) for n, x in host.items()}
     outs_h = {"o": torch.empty((Nq, Hq, d), dtype=torch.float32).pin_memory(),
               "lse": torch.empty((Nq, Hq), dtype=torch.float32).pin_memory()}
@@ -617,6 +620,9 @@ def parse_args(argv=None):
     ap.add_argument("--fwd-lpt-cost", choices=["tiles", "pairs"], default="pairs",
                     help="LPT item cost of the forward schedule (forward and dQ kernels): the allowed pairs "
                          "of the pages' rule (default) or the forward kernel's executed tile work")
+    ap.add_argument("--dynamic-claim", action="store_true",
+                    help="CTAs claim the items in LPT order at run time (plan flag) instead of taking the "
+                         "static worker lists")
     ap.add_argument("--dump-cta-times", default=None, metavar="PATH",
                     help="write the measured per-CTA busy times of the last step (fwd partial and dK/dV "
                          "kernels, ns) with the schedule options to PATH as JSON")

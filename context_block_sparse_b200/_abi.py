@@ -25,6 +25,7 @@ FLAG_BLOCK_KEYS_IN_CONTEXT = 2
 FLAG_PARTIAL_BF16 = 4
 FLAG_TILE_COST = 8
 FLAG_FWD_TILE_COST = 16
+FLAG_DYNAMIC_CLAIM = 32
 
 STATIC_SCRATCH_BYTES = 16 << 20
 
@@ -41,6 +42,8 @@ EXPORT_BWD_SCHEDULE = 3
 EXPORT_FWD_LOADS = 4
 EXPORT_BWD_LOADS = 5
 EXPORT_CONTIG_LOADS = 6
+EXPORT_FWD_LPT_ORDER = 7
+EXPORT_BWD_LPT_ORDER = 8
 
 
 class Problem(ctypes.Structure):

@@ -23,7 +23,7 @@ int check_plan(const splitkv_plan_t* plan, const DevPlan** out) {
   const DevPlan* dp = splitkv::plan_device_view(plan);
   if (!dp) return SPLITKV_ERR_NOT_UPLOADED;
   if (dp->d != 64 && dp->d != 128) return SPLITKV_ERR_UNSUPPORTED;
-  if (dp->partial_bf16 && !splitkv::partial_bf16_supported(*dp)) return SPLITKV_ERR_UNSUPPORTED;
+  if ((dp->partial_bf16 || dp->dynamic) && !splitkv::tcgen05_supported(*dp)) return SPLITKV_ERR_UNSUPPORTED;
   *out = dp;
   return SPLITKV_OK;
 }

@@ -375,7 +375,7 @@ cudaError_t launch_bwd_partial(const DevPlan& p, const uint16_t* q, const uint16
   }();
   if (!force_mma && bwd_sm100_supported(p))
     return launch_bwd_partial_sm100(p, q, k, v, dout, lse, delta, scale, dk, dv, dq_part, s, which);
-  if (p.partial_bf16) return cudaErrorNotSupported;   // the entry points check this first
+  if (p.partial_bf16 || p.dynamic) return cudaErrorNotSupported;   // the entry points check this first
   if (which == 2) return cudaSuccess;   // the single mma.sync kernel ran in the dK/dV part
   float* dqp = static_cast<float*>(dq_part);
   if (p.d == 64) return launch_bwd_d<64>(p, q, k, v, dout, lse, delta, scale, dk, dv, dqp, s);

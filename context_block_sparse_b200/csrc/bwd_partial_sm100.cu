@@ -249,10 +249,23 @@ __device__ __forceinline__ void dst_tile(uint32_t tdPt, int hf, const float* dlt
 struct DkdvBars {
   uint64_t kv_full, kv_empty, qd_full[2], qd_empty[2], st_ready, dpt_ready, pt_ready, dst_ready, dkv_ready,
       dkv_free, mma_done, meta_ready[2], meta_free[2];
+  ClaimRing ring;   // run-time claims: producer -> MMA thread, metadata warp, 8 element-wise warps
   uint32_t tmem_base;
   int abort_flag;
 };
 constexpr int kDkdvNumBars = 17;
+static_assert(sizeof(DkdvBars) <= 256, "barrier block");
+// consumers of the claim ring in both backward kernels: the MMA thread, warp 3, warps 4-11
+constexpr uint32_t kClaimConsumers = 1 + 1 + 8;
+
+// The item sequence of one role of the dK/dV kernel: the worker's items of the
+// backward schedule, or its run-time claims.
+__device__ __forceinline__ void bwd_item_seq(ItemSeq& s, const DevPlan& p, int w, ClaimRing* ring, int role) {
+  if (p.dynamic)
+    s.init_claims(ring, p.claim + 1, p.n_bwd_items, role);
+  else
+    s.init_static(p.bwd_worker_ptr[w], p.bwd_worker_ptr[w + 1]);
+}
 
 __global__ void __launch_bounds__(kThreads, 1)
     bwd_dkdv_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_do,
@@ -281,6 +294,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   {
     // commits count 1; element-wise / metadata signals count warps (warp_arrive)
     const uint32_t counts[kDkdvNumBars] = {1, 1, 1, 1, 1, 1, 1, 1, 8, 8, 1, 8, 1, 1, 1, 8, 8};
+    if (tid == 0) claim_ring_init(&B->ring, kClaimConsumers);
     setup_common(&B->kv_full, kDkdvNumBars, counts, &B->tmem_base, warp);
   }
   const uint32_t tmem = B->tmem_base;
@@ -294,8 +308,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       prefetch_tmap(&tm_v);
       uint32_t kt_count = 0, qd_count = 0;
       bool ok = true;
-      for (int it = p.bwd_worker_ptr[w]; ok && it < p.bwd_worker_ptr[w + 1]; ++it) {
-        const int4 item = p.bwd_items[it];
+      ItemSeq seq;
+      bwd_item_seq(seq, p, w, &B->ring, kClaimProducer);
+      int idx;
+      while (ok && seq.next(idx, wctx, 2 * 10000 + __LINE__)) {
+        const int4 item = p.bwd_items[idx];
         const int g = item.y, c0 = item.x * p.C, c1 = min(c0 + p.C, p.N);
         for (int k0 = c0; ok && k0 < c1; k0 += BT) {
           if (!mbar_wait(&B->kv_empty, (kt_count & 1) ^ 1, wctx, 2 * 10000 + __LINE__)) { ok = false; break; }
@@ -326,8 +343,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t aK = smem_u32(sK), aV = smem_u32(sV), aQ = smem_u32(sQ), adO = smem_u32(sdO);
       uint32_t kt_count = 0, qd_count = 0, pds_cnt = 0, dkvf_cnt = 0;
       bool ok = true;
-      for (int it = p.bwd_worker_ptr[w]; ok && it < p.bwd_worker_ptr[w + 1]; ++it) {
-        const int4 item = p.bwd_items[it];
+      ItemSeq seq;
+      bwd_item_seq(seq, p, w, &B->ring, kClaimThread);
+      int idx;
+      while (ok && seq.next(idx, wctx, 2 * 10000 + __LINE__)) {
+        const int4 item = p.bwd_items[idx];
         const int c0 = item.x * p.C, c1 = min(c0 + p.C, p.N);
         for (int k0 = c0; ok && k0 < c1; k0 += BT) {
           if (!mbar_wait(&B->kv_full, kt_count & 1, wctx, 2 * 10000 + __LINE__)) { ok = false; break; }
@@ -390,8 +410,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     // metadata of the query tiles, in the element-wise order, up to two tiles ahead
     uint32_t mcount = 0;
     bool ok = true;
-    for (int it = p.bwd_worker_ptr[w]; ok && it < p.bwd_worker_ptr[w + 1]; ++it) {
-      const int4 item = p.bwd_items[it];
+    ItemSeq seq;
+    bwd_item_seq(seq, p, w, &B->ring, kClaimWarp);
+    int idx;
+    while (ok && seq.next(idx, wctx, 2 * 10000 + __LINE__)) {
+      const int4 item = p.bwd_items[idx];
       const int g = item.y, c0 = item.x * p.C, c1 = min(c0 + p.C, p.N);
       for (int k0 = c0; ok && k0 < c1; k0 += BT) {
         for (int t = item.z; t < item.w; ++t) {
@@ -439,8 +462,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     uint32_t qd_count = 0, st_cnt = 0, dkv_cnt = 0;
     bool ok = true;
-    for (int it = p.bwd_worker_ptr[w]; ok && it < p.bwd_worker_ptr[w + 1]; ++it) {
-      const int4 item = p.bwd_items[it];
+    ItemSeq seq;
+    bwd_item_seq(seq, p, w, &B->ring, kClaimWarp);
+    int idx;
+    while (ok && seq.next(idx, wctx, 2 * 10000 + __LINE__)) {
+      const int4 item = p.bwd_items[idx];
       const int g = item.y, c0 = item.x * p.C, c1 = min(c0 + p.C, p.N);
       for (int k0 = c0; ok && k0 < c1; k0 += BT) {
         const int key = k0 + r;
@@ -543,10 +569,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 struct DqBars {
   uint64_t qd_full, qd_empty, k_full[2], v_full[2], kv_empty[2], s_ready[2], dp_ready, ds_ready, dq_ready, dq_free,
       mma_done, meta_ready[2], meta_free[2];
+  ClaimRing ring;   // run-time claims: producer -> MMA thread, metadata warp, 8 element-wise warps
   uint32_t tmem_base;
   int abort_flag;
 };
 constexpr int kDqNumBars = 19;
+static_assert(sizeof(DqBars) <= 256, "barrier block");
 
 // Per-row metadata of a query tile for the dq kernel (shared memory).
 struct DqRow {
@@ -554,21 +582,29 @@ struct DqRow {
   float l2, dl;
 };
 
-// The query tiles of a worker's forward schedule, one at a time.
+// The query tiles of a worker's forward schedule (or of the forward items it
+// claims at run time), one at a time.
 struct TileIter {
   const DevPlan* p;
-  int it, it_end, t, t_end, g;
-  __device__ void init(const DevPlan* plan, int w) {
+  const WaitCtx* wc;
+  ItemSeq seq;
+  int t, t_end, g;
+  __device__ void init(const DevPlan* plan, int w, ClaimRing* ring, int role, const WaitCtx* wctx) {
     p = plan;
-    it = plan->fwd_worker_ptr[w];
-    it_end = plan->fwd_worker_ptr[w + 1];
+    wc = wctx;
+    if (plan->dynamic)
+      seq.init_claims(ring, plan->claim + 2, plan->n_fwd_items, role);
+    else
+      seq.init_static(plan->fwd_worker_ptr[w], plan->fwd_worker_ptr[w + 1]);
     t = t_end = 0;
     g = 0;
   }
+  // false at the end (or when a claim wait gave up, which the wait recorded)
   __device__ bool next(int& tile_id, int& head) {
     while (t >= t_end) {
-      if (it >= it_end) return false;
-      const int4 item = p->fwd_items[it++];
+      int idx;
+      if (!seq.next(idx, *wc, 2 * 10000 + __LINE__)) return false;
+      const int4 item = p->fwd_items[idx];
       g = item.y;
       t = item.z;
       t_end = item.w;
@@ -600,6 +636,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   {
     // commits count 1; element-wise / metadata signals count warps (warp_arrive)
     const uint32_t counts[kDqNumBars] = {1, 1, 1, 1, 1, 1, 1, 1, 1, 1, 1, 8, 1, 8, 1, 1, 1, 8, 8};
+    if (tid == 0) claim_ring_init(&B->ring, kClaimConsumers);
     setup_common(&B->qd_full, kDqNumBars, counts, &B->tmem_base, warp);
   }
   const uint32_t tmem = B->tmem_base;
@@ -611,7 +648,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       prefetch_tmap(&tm_k);
       prefetch_tmap(&tm_v);
       TileIter ti;
-      ti.init(&p, w);
+      ti.init(&p, w, &B->ring, kClaimProducer, &wctx);
       int t, g;
       uint32_t tile_count = 0, kv_count = 0, q_issued = 0;
       bool ok = true;
@@ -645,7 +682,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       const uint32_t aK = smem_u32(sK), aV = smem_u32(sV), aQ = smem_u32(sQ), adO = smem_u32(sdO);
       TileIter ti;
-      ti.init(&p, w);
+      ti.init(&p, w, &B->ring, kClaimThread, &wctx);
       int t, g;
       uint32_t tile_count = 0, kv_count = 0, ds_cnt = 0, dqf_cnt = 0;
       bool ok = true;
@@ -713,7 +750,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == 3) {
     // row metadata of upcoming query tiles, up to two tiles ahead
     TileIter ti;
-    ti.init(&p, w);
+    ti.init(&p, w, &B->ring, kClaimWarp, &wctx);
     int t, g;
     uint32_t mcount = 0;
     bool ok = true;
@@ -749,7 +786,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tdQ = tmem + lane_addr + 384 + hf * 64;   // this warpgroup's 64 dQ columns
     const float scale_log2 = scale * kLog2e;
     TileIter ti;
-    ti.init(&p, w);
+    ti.init(&p, w, &B->ring, kClaimWarp, &wctx);
     int t, g;
     uint32_t kv_count = 0, dp_cnt = 0, dq_cnt = 0, mcount = 0;
     bool ok = true;
@@ -870,12 +907,15 @@ cudaError_t launch_bwd_partial_sm100(const DevPlan& p, const uint16_t* q, const 
   if (e != cudaSuccess) return e;
   e = cudaFuncSetAttribute(bwd_dq_sm100_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(kSmemBytes));
   if (e != cudaSuccess) return e;
+  // run-time claims start from item 0 at every launch (each kernel its own cursor)
   if (which != 2) {
+    if (p.dynamic && (e = cudaMemsetAsync(p.claim + 1, 0, sizeof(int), s)) != cudaSuccess) return e;
     bwd_dkdv_sm100_kernel<<<p.Wb, kThreads, kSmemBytes, s>>>(tq, tdo, tk, tv, tdk, tdv, p, lse, delta, scale, dk, dv);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
   if (which != 1) {
+    if (p.dynamic && (e = cudaMemsetAsync(p.claim + 2, 0, sizeof(int), s)) != cudaSuccess) return e;
     bwd_dq_sm100_kernel<<<p.W, kThreads, kSmemBytes, s>>>(tq, tdo, tk, tv, tdq, p, lse, delta, scale,
                                                           bulk_dq ? 1 : 0, dq_part);
     e = cudaGetLastError();

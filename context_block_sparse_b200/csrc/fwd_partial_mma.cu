@@ -278,7 +278,7 @@ bool env_is_mma(const char* name) {
 }
 }  // namespace
 
-bool partial_bf16_supported(const DevPlan& p) {
+bool tcgen05_supported(const DevPlan& p) {
   static const bool forced = env_is_mma("SPLITKV_FWD_KERNEL") || env_is_mma("SPLITKV_BWD_KERNEL");
   return !forced && fwd_sm100_supported(p) && bwd_sm100_supported(p);
 }
@@ -292,7 +292,7 @@ cudaError_t launch_fwd_partial(const DevPlan& p, const uint16_t* q, const uint16
   static const bool force_mma = env_is_mma("SPLITKV_FWD_KERNEL");
   if (!force_mma && fwd_sm100_supported(p))
     return launch_fwd_partial_sm100(p, q, k, v, scale, part_o, part_m, part_l, s);
-  if (p.partial_bf16) return cudaErrorNotSupported;   // the entry points check this first
+  if (p.partial_bf16 || p.dynamic) return cudaErrorNotSupported;   // the entry points check this first
   float* po = static_cast<float*>(part_o);
   if (p.d == 64) return launch_fwd_d<64>(p, q, k, v, scale, po, part_m, part_l, s);
   return launch_fwd_d<128>(p, q, k, v, scale, po, part_m, part_l, s);

@@ -72,29 +72,38 @@ struct Bars {
   uint64_t k_full[kStages], v_full[kStages], kv_empty[kStages];
   uint64_t s_ready[2], p_ready[2], o_ready[2], o_free[2];
   uint64_t mma_done;
+  ClaimRing ring;   // run-time claims: the producer hands items to the MMA thread and the 8 softmax warps
   uint32_t tmem_base;
   int abort_flag;
 };
 static_assert(sizeof(Bars) <= 256, "barrier block");
+constexpr uint32_t kClaimConsumers = 1 + 8;
 
-// The sequence of tile pairs a worker processes (identical in every role).
+// The sequence of tile pairs a worker processes (identical in every role): the
+// worker's items of the static schedule, or the items it claims at run time.
 struct PairIter {
   const DevPlan* p;
-  int it, it_end;   // item cursor
+  const WaitCtx* wc;
+  ItemSeq seq;      // item cursor
   int t, t_end;     // tile cursor inside the item
   int g;
-  __device__ void init(const DevPlan* plan, int w) {
+  __device__ void init(const DevPlan* plan, int w, ClaimRing* ring, int role, const WaitCtx* wctx) {
     p = plan;
-    it = plan->fwd_worker_ptr[w];
-    it_end = plan->fwd_worker_ptr[w + 1];
+    wc = wctx;
+    if (plan->dynamic)
+      seq.init_claims(ring, plan->claim + 0, plan->n_fwd_items, role);
+    else
+      seq.init_static(plan->fwd_worker_ptr[w], plan->fwd_worker_ptr[w + 1]);
     t = t_end = 0;
     g = 0;
   }
-  // tA, tB (-1 if absent), kv head, key union [klo, khi)
+  // tA, tB (-1 if absent), kv head, key union [klo, khi); false at the end (or
+  // when a claim wait gave up, which the wait recorded)
   __device__ bool next(int& tA, int& tB, int& head, int& klo, int& khi) {
     while (t >= t_end) {
-      if (it >= it_end) return false;
-      const int4 item = p->fwd_items[it++];
+      int idx;
+      if (!seq.next(idx, *wc, 1 * 10000 + __LINE__)) return false;
+      const int4 item = p->fwd_items[idx];
       g = item.y;
       t = item.z;
       t_end = item.w;
@@ -191,6 +200,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&bars->o_free[x], 4);
     }
     mbar_init(&bars->mma_done, 1);
+    claim_ring_init(&bars->ring, kClaimConsumers);
     bars->abort_flag = 0;
     mbar_fence_init();
   }
@@ -213,7 +223,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
       PairIter pi;
-      pi.init(&p, w);
+      pi.init(&p, w, &bars->ring, kClaimProducer, &wctx);
       int tA, tB, g, klo, khi;
       uint32_t kv_count = 0, pair_count = 0, q_issued = 0;
       bool ok = true;
@@ -269,7 +279,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       PairIter pi;
-      pi.init(&p, w);
+      pi.init(&p, w, &bars->ring, kClaimThread, &wctx);
       int tA, tB, g, klo, khi;
       uint32_t kv_count = 0, pair_count = 0;
       uint32_t p_cnt[2] = {0, 0}, of_cnt[2] = {0, 0};
@@ -353,7 +363,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tS = tmem + lane_addr + x * 128;
     const uint32_t tO = tmem + lane_addr + 256 + x * 128;
     PairIter pi;
-    pi.init(&p, w);
+    pi.init(&p, w, &bars->ring, kClaimWarp, &wctx);
     int tA, tB, g, klo, khi;
     uint32_t s_cnt = 0, o_cnt = 0;
     bool ok = true;
@@ -581,6 +591,8 @@ cudaError_t launch_fwd_partial_sm100(const DevPlan& p, const uint16_t* q, const 
   cudaError_t e = cudaFuncSetAttribute(fwd_partial_sm100_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        int(kSmemBytes));
   if (e != cudaSuccess) return e;
+  // run-time claims start from item 0 at every launch
+  if (p.dynamic && (e = cudaMemsetAsync(p.claim + 0, 0, sizeof(int), s)) != cudaSuccess) return e;
   fwd_partial_sm100_kernel<<<p.W, kThreads, kSmemBytes, s>>>(tq, tk, tv, to, p, scale * kLog2e, bulk ? 1 : 0,
                                                              part_o, part_m, part_l);
   return cudaGetLastError();

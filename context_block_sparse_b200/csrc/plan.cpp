@@ -51,6 +51,7 @@ struct splitkv_plan {
   std::vector<Item> fwd_items, bwd_items;          // non-zero-cost items
   std::vector<int32_t> fwd_worker_ptr, bwd_worker_ptr;
   std::vector<int32_t> fwd_order, bwd_order;       // item indices grouped by worker
+  std::vector<int32_t> fwd_lpt, bwd_lpt;           // item indices in LPT order (cost desc, index asc)
   std::vector<uint64_t> fwd_loads, bwd_loads, contig_loads;
   std::vector<int32_t> block_entry_ptr, block_entries;
   std::vector<int32_t> zero_chunks;
@@ -76,7 +77,7 @@ int validate(const splitkv_problem* p) {
     return SPLITKV_ERR_INVALID_ARG;
   if (p->num_q_heads % p->num_kv_heads) return SPLITKV_ERR_INVALID_ARG;
   if (p->flags & ~uint32_t(SPLITKV_FLAG_EQUAL_COUNT | SPLITKV_FLAG_BLOCK_KEYS_IN_CONTEXT | SPLITKV_FLAG_PARTIAL_BF16 |
-                           SPLITKV_FLAG_TILE_COST | SPLITKV_FLAG_FWD_TILE_COST))
+                           SPLITKV_FLAG_TILE_COST | SPLITKV_FLAG_FWD_TILE_COST | SPLITKV_FLAG_DYNAMIC_CLAIM))
     return SPLITKV_ERR_INVALID_ARG;
   int64_t N = 0;
   for (int s = 0; s < p->num_samples; ++s) {
@@ -101,7 +102,7 @@ int validate(const splitkv_problem* p) {
 // removed for good.
 void lpt_schedule(const std::vector<Item>& items, int W, bool equal_count,
                   std::vector<int32_t>& worker_ptr, std::vector<int32_t>& order,
-                  std::vector<uint64_t>& loads) {
+                  std::vector<uint64_t>& loads, std::vector<int32_t>& sorted) {
   const int64_t n = int64_t(items.size());
   std::vector<std::pair<uint64_t, int32_t>> byc(n);
   for (int64_t i = 0; i < n; ++i) byc[i] = {items[i].cost, int32_t(i)};
@@ -156,6 +157,8 @@ void lpt_schedule(const std::vector<Item>& items, int W, bool equal_count,
   order.resize(n);
   std::vector<int32_t> fill(worker_ptr.begin(), worker_ptr.end() - 1);
   for (int64_t k = 0; k < n; ++k) order[fill[owner[k]]++] = byc[k].second;
+  sorted.resize(n);
+  for (int64_t k = 0; k < n; ++k) sorted[k] = byc[k].second;
 }
 
 int build(splitkv_plan_t* P, const splitkv_problem* p) {
@@ -330,8 +333,8 @@ int build(splitkv_plan_t* P, const splitkv_problem* p) {
   nonzero(P->fwd_items);
   nonzero(P->bwd_items);
   const bool eq = (P->flags & SPLITKV_FLAG_EQUAL_COUNT) != 0;
-  lpt_schedule(P->fwd_items, P->W, eq, P->fwd_worker_ptr, P->fwd_order, P->fwd_loads);
-  lpt_schedule(P->bwd_items, P->Wb, eq, P->bwd_worker_ptr, P->bwd_order, P->bwd_loads);
+  lpt_schedule(P->fwd_items, P->W, eq, P->fwd_worker_ptr, P->fwd_order, P->fwd_loads, P->fwd_lpt);
+  lpt_schedule(P->bwd_items, P->Wb, eq, P->bwd_worker_ptr, P->bwd_order, P->bwd_loads, P->bwd_lpt);
 
   // contiguous ("unbalanced") baseline: the num_chunks * Hkv (chunk, head) items in
   // order, item i to worker floor(i W / n), zero-cost items included
@@ -449,9 +452,11 @@ int splitkv_plan_upload(splitkv_plan_t* P, void* stream) {
       dst[4 * i + 3] = it.t1;
     }
   };
+  // run-time claims walk the whole lists in LPT order; otherwise each worker's items
+  const bool dynamic = (P->flags & SPLITKV_FLAG_DYNAMIC_CLAIM) != 0;
   try {
-    pack_items(P->fwd_items, P->fwd_order, fwd_items);
-    pack_items(P->bwd_items, P->bwd_order, bwd_items);
+    pack_items(P->fwd_items, dynamic ? P->fwd_lpt : P->fwd_order, fwd_items);
+    pack_items(P->bwd_items, dynamic ? P->bwd_lpt : P->bwd_order, bwd_items);
   } catch (...) {
     return SPLITKV_ERR_NO_MEMORY;
   }
@@ -550,6 +555,10 @@ int splitkv_plan_upload(splitkv_plan_t* P, void* stream) {
   v.Wb = P->Wb;
   v.block_term = (P->flags & SPLITKV_FLAG_BLOCK_KEYS_IN_CONTEXT) ? 0 : 1;
   v.partial_bf16 = (P->flags & SPLITKV_FLAG_PARTIAL_BF16) ? 1 : 0;
+  v.dynamic = dynamic ? 1 : 0;
+  v.n_fwd_items = int(P->fwd_items.size());
+  v.n_bwd_items = int(P->bwd_items.size());
+  v.claim = reinterpret_cast<int*>(d + status_off + 128);   // after the two status words
   P->uploaded = true;
   return SPLITKV_OK;
 }
@@ -629,6 +638,16 @@ int splitkv_plan_export(const splitkv_plan_t* P, int what, int64_t* out, int64_t
       case SPLITKV_EXPORT_CONTIG_LOADS:
         for (uint64_t x : P->contig_loads) v.push_back(int64_t(x));
         break;
+      case SPLITKV_EXPORT_FWD_LPT_ORDER:
+      case SPLITKV_EXPORT_BWD_LPT_ORDER: {
+        const bool f = what == SPLITKV_EXPORT_FWD_LPT_ORDER;
+        const auto& items = f ? P->fwd_items : P->bwd_items;
+        for (int32_t i : (f ? P->fwd_lpt : P->bwd_lpt)) {
+          const Item& it = items[i];
+          v.insert(v.end(), {int64_t(it.c), int64_t(it.g), int64_t(it.slice), int64_t(it.cost)});
+        }
+        break;
+      }
       default:
         return SPLITKV_ERR_INVALID_ARG;
     }

@@ -103,6 +103,88 @@ __device__ __forceinline__ void mbar_drain(uint64_t* bar, uint32_t parity, const
   }
 }
 
+// ---------------------------------------------------------------- run-time item claims
+// Items claimed at run time: whenever the producer thread of a CTA needs a new
+// item it takes the next index of a global cursor (one atomicAdd) and hands it
+// to the CTA's other roles through a ring of shared-memory slots, so that every
+// role walks the same sequence; an index past the list ends it (-1 in the ring).
+// A CTA therefore takes the next item of the list as soon as it is free: the
+// list order (longest first) with the actual, not the predicted, loads.
+constexpr int kClaimRing = 4;
+struct ClaimRing {
+  uint64_t full[kClaimRing];    // count 1: the producer's arrival after it wrote the slot
+  uint64_t empty[kClaimRing];   // count: the consumers' arrivals (threads or warps)
+  int item[kClaimRing];
+};
+// Thread 0, before the CTA's mbarrier-init fence.
+__device__ __forceinline__ void claim_ring_init(ClaimRing* r, uint32_t consumers) {
+  for (int s = 0; s < kClaimRing; ++s) {
+    mbar_init(&r->full[s], 1);
+    mbar_init(&r->empty[s], consumers);
+  }
+}
+
+enum ClaimRole { kClaimProducer = 0, kClaimThread = 1, kClaimWarp = 2 };
+
+// The item sequence one role of a CTA walks: a static range [it, end) of the
+// schedule's item list, or (cursor != nullptr) the run-time claims over the
+// whole list of `end` items.  A kClaimWarp role calls next() with all 32 lanes.
+struct ItemSeq {
+  ClaimRing* ring;
+  int* cursor;
+  int it, end;
+  uint32_t cnt;
+  int role;
+  __device__ void init_static(int first, int last) {
+    ring = nullptr;
+    cursor = nullptr;
+    it = first;
+    end = last;
+    cnt = 0;
+    role = kClaimThread;
+  }
+  __device__ void init_claims(ClaimRing* r, int* cur, int n_items, int role_) {
+    ring = r;
+    cursor = cur;
+    it = 0;
+    end = n_items;
+    cnt = 0;
+    role = role_;
+  }
+  // The next item index; false at the end of the sequence, or when a wait gave up
+  // (the wait recorded the timeout, or another role's abort stopped it).
+  __device__ bool next(int& idx, const WaitCtx& c, int site) {
+    if (cursor == nullptr) {
+      if (it >= end) return false;
+      idx = it++;
+      return true;
+    }
+    const int s = int(cnt % kClaimRing);
+    const uint32_t ph = (cnt / kClaimRing) & 1u;
+    ++cnt;
+    int v;
+    if (role == kClaimProducer) {
+      // the slot is free once every consumer took the item it held kClaimRing claims ago
+      if (!mbar_wait(&ring->empty[s], ph ^ 1u, c, site)) return false;
+      v = atomicAdd(cursor, 1);
+      if (v >= end) v = -1;
+      ring->item[s] = v;
+      mbar_arrive(&ring->full[s]);   // release: the slot's write before the arrival
+    } else if (role == kClaimThread) {
+      if (!mbar_wait(&ring->full[s], ph, c, site)) return false;
+      v = *reinterpret_cast<volatile int*>(&ring->item[s]);
+      mbar_arrive(&ring->empty[s]);
+    } else {
+      if (!warp_wait(&ring->full[s], ph, c, site)) return false;
+      v = *reinterpret_cast<volatile int*>(&ring->item[s]);
+      warp_arrive(&ring->empty[s]);
+    }
+    if (v < 0) return false;
+    idx = v;
+    return true;
+  }
+};
+
 // ---------------------------------------------------------------- TMA
 __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, uint64_t* bar, int x, int y,
                                             int z) {

@@ -30,6 +30,12 @@ struct DevPlan {
   int N, Nq, A, bs, Hq, Hkv, G, d, C, num_chunks, E, W, Wb;
   int block_term;               // 1: separate block keys kb, vb (reading A); 0: block keys in the context
   int partial_bf16;             // 1: O_c records and dQ partials stored as bf16
+  // run-time claims (SPLITKV_FLAG_DYNAMIC_CLAIM): fwd_items / bwd_items hold the whole
+  // lists in LPT order and the CTAs claim them through claim[0] (forward kernel),
+  // claim[1] (dK/dV kernel), claim[2] (dQ kernel), zeroed before each launch
+  int dynamic;
+  int n_fwd_items, n_bwd_items;
+  int* claim;                   // [4]
 };
 
 // Byte offsets of the forward workspace (partial records).
@@ -106,8 +112,9 @@ cudaError_t launch_bwd_reduce(const DevPlan& p, const uint16_t* q, const uint16_
                               const float* delta, const void* dq_part, float scale, float* dq,
                               float* dkb, float* dvb, cudaStream_t s);
 
-// bf16 partial records need the tcgen05 forward and backward kernels for this plan
-// (and no SPLITKV_FWD_KERNEL / SPLITKV_BWD_KERNEL override selecting mma.sync).
-bool partial_bf16_supported(const DevPlan& p);
+// True when the tcgen05 forward and backward kernels serve this plan (and no
+// SPLITKV_FWD_KERNEL / SPLITKV_BWD_KERNEL override selects mma.sync): bf16
+// partial records and run-time claims exist on those kernels only.
+bool tcgen05_supported(const DevPlan& p);
 
 }  // namespace splitkv

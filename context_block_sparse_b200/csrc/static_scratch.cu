@@ -66,7 +66,7 @@ extern "C" int splitkv_attn_fwd_static_scratch(const splitkv_plan_t* plan, const
   const splitkv::DevPlan* dp = splitkv::plan_device_view(plan);
   if (!dp) return SPLITKV_ERR_NOT_UPLOADED;
   if (dp->d != 64 && dp->d != 128) return SPLITKV_ERR_UNSUPPORTED;
-  if (dp->partial_bf16 && !splitkv::partial_bf16_supported(*dp)) return SPLITKV_ERR_UNSUPPORTED;
+  if ((dp->partial_bf16 || dp->dynamic) && !splitkv::tcgen05_supported(*dp)) return SPLITKV_ERR_UNSUPPORTED;
   // kb, vb: required under reading A; may be NULL under SPLITKV_FLAG_BLOCK_KEYS_IN_CONTEXT
   const bool blk_ok = dp->block_term ? (aligned16(kb) && aligned16(vb))
                                      : ((!kb || aligned16(kb)) && (!vb || aligned16(vb)));

@@ -105,6 +105,20 @@ extern "C" {
  * The backward schedule, the contiguous baseline and the pair counts are not
  * affected (see SPLITKV_FLAG_TILE_COST for the backward schedule). */
 #define SPLITKV_FLAG_FWD_TILE_COST  16u
+/* Run-time claims: the LPT order of each schedule is kept, but instead of the
+ * worker lists the CTAs of the forward, dK/dV and dQ kernels take the items of
+ * that order one at a time, each CTA the next item as soon as it is free (an
+ * atomic cursor per kernel in the plan's device memory, zeroed by every
+ * launch).  This is LPT's "next item to the least-loaded worker" with the
+ * loads the CTAs actually reach instead of the predicted costs, so per-SM speed
+ * differences and cost-model error do not add to the makespan.  Results are
+ * unchanged (every item writes only its own outputs); which CTA ran an item
+ * varies from launch to launch.  The worker lists (SPLITKV_EXPORT_*_SCHEDULE)
+ * and their loads are still computed: they are the static plan.  Served by the
+ * tcgen05 kernels only (head_dim 128, G * bs a multiple of 8): attention calls
+ * of other plans return SPLITKV_ERR_UNSUPPORTED.  Launches of one kernel on one
+ * plan must not overlap (they share its cursor). */
+#define SPLITKV_FLAG_DYNAMIC_CLAIM  32u
 
 /* ---- dtype codes (o) ------------------------------------------------------- */
 #define SPLITKV_DTYPE_F32   0
@@ -123,6 +137,9 @@ extern "C" {
 #define SPLITKV_EXPORT_BWD_LOADS      5  /* 1 per backward worker                                  */
 #define SPLITKV_EXPORT_CONTIG_LOADS   6  /* 1 per forward worker: the contiguous ("unbalanced")
                                             baseline                                               */
+#define SPLITKV_EXPORT_FWD_LPT_ORDER  7  /* 4 per forward item, in LPT order: chunk, kv head,
+                                            slice, cost (the order run-time claims take)         */
+#define SPLITKV_EXPORT_BWD_LPT_ORDER  8  /* same, backward items                                 */
 
 /* The problem, as the news page states it ("Why short queries change the
  * problem"): packed sample lengths, anchor positions, block size, and the

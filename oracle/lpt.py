@@ -143,13 +143,20 @@ def work_items(sample_lens, anchors, block_size: int, kv_chunk: int, num_q_heads
     return items
 
 
+def lpt_order(items):
+    """The order in which LPT hands out items: positive-cost items by cost descending,
+    ties by key ascending."""
+    live = [(key, cost) for (key, cost) in items if cost > 0]
+    live.sort(key=lambda it: (-it[1], it[0]))
+    return live
+
+
 def lpt(items, num_workers: int, equal_count: bool = False):
     """Assign items to workers longest-first; returns (lists, loads).
 
     lists[w] holds the item keys of worker w in assignment order.
     """
-    live = [(key, cost) for (key, cost) in items if cost > 0]
-    live.sort(key=lambda it: (-it[1], it[0]))
+    live = lpt_order(items)
     W = int(num_workers)
     n = len(live)
     q, r = divmod(n, W)

@@ -69,6 +69,8 @@ def test_small_ragged_fwd_bwd_elementwise(splitkv, case):
 @pytest.mark.parametrize("opts", [
     dict(W=7), dict(W=1), dict(W=300, Wb=5), dict(q_slice=1), dict(q_slice=2, equal_count=True),
     dict(o_dtype="bf16"), dict(q_slice=2, tile_cost=True), dict(tile_cost=True, Wb=5),
+    dict(dynamic_claim=True), dict(dynamic_claim=True, W=7, Wb=3, q_slice=1), dict(dynamic_claim=True, W=300),
+    dict(dynamic_claim=True, W=1, Wb=1, q_slice=2, partial_bf16=True),
 ])
 def test_schedules_and_options_same_result(splitkv, opts):
     w = small()
@@ -224,6 +226,28 @@ def test_partial_bf16_needs_the_tcgen05_path(splitkv):
     assert ei.value.status == -2   # SPLITKV_ERR_UNSUPPORTED
 
 
+def test_dynamic_claim_needs_the_tcgen05_path(splitkv):
+    w = small(Hq=2, Hkv=2, d=64)
+    with pytest.raises(splitkv.SplitKVError) as ei:
+        run(w, dynamic_claim=True)
+    assert ei.value.status == -2   # SPLITKV_ERR_UNSUPPORTED
+
+
+@pytest.mark.parametrize("case", list(BF16_CASES))
+def test_dynamic_claim_fwd_bwd(splitkv, case):
+    """Items claimed at run time: every item is run exactly once by some CTA, so the
+    results equal the oracle's (and repeat bit for bit, whichever CTA ran what)."""
+    w = small(**BF16_CASES[case])
+    out, _, _ = run(w, bwd=True, dynamic_claim=True, q_slice=2, tile_cost=True)
+    _check_fwd(w, out)
+    _check_bwd(w, out)
+    again, _, _ = run(w, bwd=True, dynamic_claim=True, q_slice=2, tile_cost=True)
+    static, _, _ = run(w, bwd=True, q_slice=2, tile_cost=True)
+    for n in out:
+        assert np.array_equal(out[n], again[n]), n
+        assert np.array_equal(out[n], static[n]), n
+
+
 def test_merge_alone_on_oracle_partials(splitkv):
     """splitkv_merge fed with oracle-computed partial records reproduces the oracle output."""
     import torch
@@ -288,6 +312,21 @@ def test_budget_fwd_sampled(splitkv, anchors):
     out, _, _ = run(w)
     _check_fwd(w, out, _sample_blocks(w))
     assert np.isfinite(out["o"]).all() and np.isfinite(out["lse"]).all()
+
+
+def test_bwd_config_dynamic_claim_matches_static(splitkv):
+    """The fwd+bwd workload in the bench's launch configuration with run-time claims:
+    bit-identical to the static schedule (the static run is checked against the oracle
+    in test_bwd_config_sampled), and repeated launches reuse the cursors correctly."""
+    w = make_workload("bwd")
+    dyn, att, _ = run(w, bwd=True, dynamic_claim=True, q_slice=2, tile_cost=True, repeat=2)
+    static, _, _ = run(w, bwd=True, q_slice=2, tile_cost=True)
+    for n in dyn:
+        assert np.array_equal(dyn[n], static[n]), n
+    import context_block_sparse_b200 as skv
+    for which in (skv.WS_FWD, skv.WS_BWD):
+        t = skv.splitkv_read_cta_times(att.plan, which)
+        assert (t > 0).all()
 
 
 def test_budget_fwd_sampled_bf16_partials(splitkv):

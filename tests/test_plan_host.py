@@ -14,9 +14,11 @@ from oracle import mask as omask
 from synth import CONFIGS, make_workload
 
 
-def _plan(skv, lens, anchors, bs, Hq, Hkv, d, C, W, Wb=0, q_slice=0, eq=False, rb=False, tc=False, ftc=False):
+def _plan(skv, lens, anchors, bs, Hq, Hkv, d, C, W, Wb=0, q_slice=0, eq=False, rb=False, tc=False, ftc=False,
+          dyn=False):
     return skv.splitkv_plan(lens, anchors, bs, Hq, Hkv, d, C, W, num_bwd_workers=Wb, q_slice=q_slice,
-                            equal_count=eq, block_keys_in_context=rb, tile_cost=tc, fwd_tile_cost=ftc)
+                            equal_count=eq, block_keys_in_context=rb, tile_cost=tc, fwd_tile_cost=ftc,
+                            dynamic_claim=dyn)
 
 
 def _check_against_oracle(skv, lens, anchors, bs, Hq, Hkv, C, W, Wb=0, q_slice=0, eq=False, d=64, rb=False,
@@ -49,6 +51,10 @@ def _check_against_oracle(skv, lens, anchors, bs, Hq, Hkv, C, W, Wb=0, q_slice=0
             assert cst == cost[(c, g, s)]
         assert got == [list(l) for l in lists]
         assert plan.export(loads_what).tolist() == loads
+        # the LPT order itself (the order run-time claims take)
+        order_what = skv.EXPORT_FWD_LPT_ORDER if what == skv.EXPORT_FWD_SCHEDULE else skv.EXPORT_BWD_LPT_ORDER
+        order = [((c, g, s), cst) for c, g, s, cst in plan.export(order_what).reshape(-1, 4).tolist()]
+        assert order == olpt.lpt_order(items)
     # contiguous baseline
     _, cl = olpt.contiguous(olpt.work_items(lens, anchors, bs, C, Hq, Hkv, block_keys_in_context=rb), W)
     assert plan.export(skv.EXPORT_CONTIG_LOADS).tolist() == cl
@@ -187,3 +193,19 @@ def test_device_regime_report(splitkv, name):
         assert row["lpt_imbalance_pct"] < 1.0, (W, row)
         assert row["makespan_ratio"] > 1.1, (W, row)
         assert row["equal_count_plan_us"] > 0 and row["lpt_plan_us"] > 0
+
+
+def test_dynamic_claim_keeps_the_static_plan(splitkv):
+    """SPLITKV_FLAG_DYNAMIC_CLAIM changes how the kernels take the items, not the plan:
+    every exported table is the same with and without it."""
+    w = make_workload("drafter", tensors=False)
+    a = _plan(splitkv, w.sample_lens, w.anchors, 16, 32, 8, 128, 256, 148, q_slice=2)
+    b = _plan(splitkv, w.sample_lens, w.anchors, 16, 32, 8, 128, 256, 148, q_slice=2, dyn=True)
+    for what in range(9):
+        assert np.array_equal(a.export(what), b.export(what)), what
+    sa, sb = a.stats(), b.stats()
+    sa.pop("plan_us", None)
+    sb.pop("plan_us", None)
+    assert sa == sb
+    a.destroy()
+    b.destroy()
