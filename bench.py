@@ -620,9 +620,9 @@ def parse_args(argv=None):
     ap.add_argument("--fwd-lpt-cost", choices=["tiles", "pairs"], default="pairs",
                     help="LPT item cost of the forward schedule (forward and dQ kernels): the allowed pairs "
                          "of the pages' rule (default) or the forward kernel's executed tile work")
-    ap.add_argument("--dynamic-claim", action="store_true",
-                    help="CTAs claim the items in LPT order at run time (plan flag) instead of taking the "
-                         "static worker lists")
+    ap.add_argument("--claims", choices=["run-time", "static"], default="run-time",
+                    help="how the CTAs of the partial kernels take their items: one at a time in LPT order at "
+                         "run time (default; plan flag) or from the static LPT worker lists")
     ap.add_argument("--dump-cta-times", default=None, metavar="PATH",
                     help="write the measured per-CTA busy times of the last step (fwd partial and dK/dV "
                          "kernels, ns) with the schedule options to PATH as JSON")
@@ -631,6 +631,7 @@ def parse_args(argv=None):
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
+    args.dynamic_claim = args.claims == "run-time"
     return args
 
 
