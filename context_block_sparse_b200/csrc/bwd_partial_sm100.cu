@@ -838,6 +838,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             warp_bulk_store32_bf16<0>(scratch, v, scale, &tm_dq, hf * 64 + cc * 32, g * p.G, z0, wv);
           else if (m.valid)
             lane_store32_bf16(static_cast<uint16_t*>(dq_part) + size_t(m.rec) * D + hf * 64 + cc * 32, v, scale);
+          __syncwarp();   // m.valid differs across the warp's rows: converge before the next tcgen05.ld
         }
       } else if (bulk) {
         // the warp's 32 rows are 32/G whole tokens of one block, all G heads of KV

@@ -510,6 +510,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           tmem_wait_ld();
           reg_fence<32>(v);
           if (valid) lane_store32_bf16(static_cast<uint16_t*>(part_o) + size_t(rec) * D + cch * 32, v, inv);
+          __syncwarp();   // valid differs across the warp's rows: converge before the next tcgen05.ld
         }
       } else if (bulk_o) {
         // the warp's rows: tokens tt0 .. tt0 + 32/G - 1 of one block, all G heads
