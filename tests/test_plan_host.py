@@ -209,3 +209,17 @@ def test_dynamic_claim_keeps_the_static_plan(splitkv):
     assert sa == sb
     a.destroy()
     b.destroy()
+
+
+def test_unknown_flag_bits_rejected(splitkv):
+    """Flags outside SPLITKV_FLAG_* (1, 2, 4, 8, 16, 32) are an invalid argument; each known bit alone is accepted."""
+    import ctypes
+    lib = splitkv._lib
+    for flags, want in [(1, 0), (2, 0), (4, 0), (8, 0), (16, 0), (32, 0), (63, 0), (64, -1), (1 << 31, -1)]:
+        p, keep = splitkv._problem([64, 64], [10, 70], 16, 2, 1, 128, 32, 4, 0, 0, False)
+        p.flags = flags
+        h = ctypes.c_void_p()
+        st = lib.splitkv_plan(ctypes.byref(p), ctypes.byref(h))
+        assert st == want, (flags, st)
+        if st == 0:
+            lib.splitkv_plan_destroy(h)
