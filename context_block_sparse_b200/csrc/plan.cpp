@@ -34,7 +34,7 @@ struct Item {
 
 }  // namespace
 
-struct splitkv_plan {
+struct splitkv_plan_s {
   // problem
   int32_t S = 0, A = 0, bs = 0, Hq = 0, Hkv = 0, d = 0, C = 0, W = 0, Wb = 0, q_slice = 0;
   uint32_t flags = 0;
@@ -162,7 +162,7 @@ void lpt_schedule(const std::vector<Item>& items, int W, bool equal_count,
 }
 
 int build(splitkv_plan_t* P, const splitkv_problem* p) {
-  const auto t0 = std::chrono::steady_clock::now();
+  const auto clock_start = std::chrono::steady_clock::now();
   int st = validate(p);
   if (st != SPLITKV_OK) return st;
   P->S = p->num_samples;
@@ -357,7 +357,7 @@ int build(splitkv_plan_t* P, const splitkv_problem* p) {
     for (int e = 0; e < E; ++e) P->block_entries[fill[P->entries[e].x]++] = e;  // e ascends with chunk
   }
   P->uploaded = false;
-  P->plan_us = std::chrono::duration<double, std::micro>(std::chrono::steady_clock::now() - t0).count();
+  P->plan_us = std::chrono::duration<double, std::micro>(std::chrono::steady_clock::now() - clock_start).count();
   return SPLITKV_OK;
 }
 

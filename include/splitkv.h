@@ -162,7 +162,7 @@ typedef struct splitkv_problem {
   uint32_t       flags;         /* SPLITKV_FLAG_*                                          */
 } splitkv_problem;
 
-typedef struct splitkv_plan splitkv_plan_t;   /* opaque, owned by the library */
+typedef struct splitkv_plan_s splitkv_plan_t;   /* opaque, owned by the library */
 
 typedef struct splitkv_stats {
   int64_t  context_len;        /* N                                                        */
