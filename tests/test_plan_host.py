@@ -223,3 +223,15 @@ def test_unknown_flag_bits_rejected(splitkv):
         assert st == want, (flags, st)
         if st == 0:
             lib.splitkv_plan_destroy(h)
+
+
+def test_context_at_int32_limit_rejected(splitkv):
+    """A packed context of 2^31 tokens or more is refused before anything is allocated."""
+    with pytest.raises(splitkv.SplitKVError) as ei:
+        _plan(splitkv, [2 ** 30, 2 ** 30], [5, 2 ** 30 + 7], 16, 2, 1, 128, 512, 4)
+    assert ei.value.status == -1
+    # one token below the limit is a valid problem size (planned here with a small chunk count)
+    lens = [2 ** 30, 2 ** 30 - 1]
+    plan = _plan(splitkv, lens, [5], 16, 2, 1, 128, 2 ** 28, 4)
+    assert plan.stats()["context_pairs"] == 2 * 16 * 5
+    plan.destroy()
