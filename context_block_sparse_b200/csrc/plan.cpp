@@ -100,16 +100,34 @@ int validate(const splitkv_problem* p) {
 // binary min-heap keyed by (load, id); eligibility is monotone (a worker that
 // stops being eligible never becomes eligible again), so an ineligible top is
 // removed for good.
+// Item indices by cost descending, equal costs in index order: an LSD radix sort on
+// the complemented cost, one stable counting pass per byte that differs between
+// keys (the same order as a stable sort by cost descending, in O(n) per pass).
+void sort_by_cost_desc(const std::vector<Item>& items, std::vector<int32_t>& out) {
+  const int64_t n = int64_t(items.size());
+  std::vector<int32_t> a(n), b(n);
+  for (int64_t i = 0; i < n; ++i) a[i] = int32_t(i);
+  uint64_t any_one = 0, all_one = ~uint64_t(0);
+  for (const Item& it : items) {
+    any_one |= ~it.cost;
+    all_one &= ~it.cost;
+  }
+  for (int shift = 0; shift < 64; shift += 8) {
+    if ((((any_one ^ all_one) >> shift) & 0xffu) == 0) continue;   // the same byte in every key
+    int64_t cnt[257] = {};
+    for (int64_t i = 0; i < n; ++i) cnt[((~items[a[i]].cost >> shift) & 0xffu) + 1]++;
+    for (int d = 0; d < 256; ++d) cnt[d + 1] += cnt[d];
+    for (int64_t i = 0; i < n; ++i) b[cnt[(~items[a[i]].cost >> shift) & 0xffu]++] = a[i];
+    a.swap(b);
+  }
+  out.swap(a);
+}
+
 void lpt_schedule(const std::vector<Item>& items, int W, bool equal_count,
                   std::vector<int32_t>& worker_ptr, std::vector<int32_t>& order,
                   std::vector<uint64_t>& loads, std::vector<int32_t>& sorted) {
   const int64_t n = int64_t(items.size());
-  std::vector<std::pair<uint64_t, int32_t>> byc(n);
-  for (int64_t i = 0; i < n; ++i) byc[i] = {items[i].cost, int32_t(i)};
-  std::stable_sort(byc.begin(), byc.end(),
-                   [](const std::pair<uint64_t, int32_t>& a, const std::pair<uint64_t, int32_t>& b) {
-                     return a.first > b.first;
-                   });
+  sort_by_cost_desc(items, sorted);
   const int64_t q = n / W, r = n % W;
   loads.assign(W, 0);
   std::vector<int64_t> counts(W, 0);
@@ -133,7 +151,7 @@ void lpt_schedule(const std::vector<Item>& items, int W, bool equal_count,
   };
   int64_t n_full = 0;  // workers holding q + 1 items
   for (int64_t k = 0; k < n; ++k) {
-    const int32_t it = byc[k].second;
+    const int32_t it = sorted[k];
     if (equal_count) {
       // drop tops that can no longer take an item; some worker always can
       for (;;) {
@@ -156,9 +174,7 @@ void lpt_schedule(const std::vector<Item>& items, int W, bool equal_count,
   for (int w = 0; w < W; ++w) worker_ptr[w + 1] += worker_ptr[w];
   order.resize(n);
   std::vector<int32_t> fill(worker_ptr.begin(), worker_ptr.end() - 1);
-  for (int64_t k = 0; k < n; ++k) order[fill[owner[k]]++] = byc[k].second;
-  sorted.resize(n);
-  for (int64_t k = 0; k < n; ++k) sorted[k] = byc[k].second;
+  for (int64_t k = 0; k < n; ++k) order[fill[owner[k]]++] = sorted[k];
 }
 
 int build(splitkv_plan_t* P, const splitkv_problem* p) {
@@ -292,6 +308,9 @@ int build(splitkv_plan_t* P, const splitkv_problem* p) {
   P->fwd_items.clear();
   P->bwd_items.clear();
   P->zero_chunks.clear();
+  // at most one forward item per tile and KV head, one backward item per chunk and KV head
+  P->fwd_items.reserve(P->tiles.size() * size_t(P->Hkv));
+  P->bwd_items.reserve(size_t(P->num_chunks) * size_t(P->Hkv));
   for (int c = 0; c < P->num_chunks; ++c) {
     const int t0 = P->chunk_tile_ptr[c], t1 = P->chunk_tile_ptr[c + 1];
     if (t0 == t1) {
