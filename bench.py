@@ -237,6 +237,7 @@ def bench_config(args, w, W, Wb, world):
     return {"workload": w.config.description, "context_len": w.context_len, "num_queries": w.num_queries,
             "num_anchors": int(w.anchors.size), "block_size": w.block_size, "heads": [w.num_q_heads, w.num_kv_heads],
             "head_dim": w.head_dim, "kv_chunk": w.kv_chunk, "fwd_workers": W, "bwd_workers": Wb,
+            "seed": args.seed if args.seed is not None else 1000 + w.config.index,
             "q_slice": args.q_slice, "partial_records": "bf16" if args.partial_bf16 else "f32",
             "lpt_cost": args.lpt_cost, "fwd_lpt_cost": args.fwd_lpt_cost,
             "item_claims": "run-time" if args.dynamic_claim else "static",
@@ -264,7 +265,7 @@ def run_ours(args, world, rank, local):
         import datetime
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=180), device_id=dev)
 
-    w = make_workload(args.workload, num_anchors=args.anchors, with_grad=True)
+    w = make_workload(args.workload, num_anchors=args.anchors, seed=args.seed, with_grad=True)
     sms = torch.cuda.get_device_properties(dev).multi_processor_count
     W = args.workers or sms
     Wb = args.bwd_workers or sms
@@ -562,17 +563,27 @@ def _oracle_blocks(w, budget_s: float, start: int = 0, stride: int = 37):
 
 def cpu_baseline(w, budget_s=15.0):
     flops, secs, n = _oracle_blocks(w, budget_s)
-    return {"value": flops / secs / 1e12, "unit": "TFLOP/s", "cores": _oracle_threads(), "kind": "oracle",
-            "sample": f"fp64 numpy oracle, forward + backward of {n} of {w.anchors.size} anchor blocks "
-                      f"(every 37th, all {w.num_q_heads} heads), {secs:.1f} s; same masked-pair FLOP count",
-            "host_cpu_count": os.cpu_count()}
+    out = {"value": flops / secs / 1e12, "unit": "TFLOP/s", "cores": _oracle_threads(), "kind": "oracle",
+           "sample": f"fp64 numpy oracle, forward + backward of {n} of {w.anchors.size} anchor blocks "
+                     f"(every 37th, all {w.num_q_heads} heads), {secs:.1f} s; same masked-pair FLOP count",
+           "host_cpu_count": os.cpu_count()}
+    # the same oracle on one thread, on a shorter sample
+    try:
+        from threadpoolctl import threadpool_limits
+        with threadpool_limits(limits=1):
+            f1, s1, n1 = _oracle_blocks(w, max(1.0, budget_s / 3), start=500)
+        out["value_one_thread"] = f1 / s1 / 1e12
+        out["sample_one_thread"] = f"{n1} anchor blocks, {s1:.1f} s, 1 BLAS thread"
+    except ImportError:
+        pass
+    return out
 
 
 def run_reference(args, world, rank):
     from synth import make_workload
     if rank != 0:
         return None
-    w = make_workload(args.workload, num_anchors=args.anchors, with_grad=True)
+    w = make_workload(args.workload, num_anchors=args.anchors, seed=args.seed, with_grad=True)
     per_step = max(0.2, min(args.cpu_seconds, 120.0) / max(1, args.steps + args.warmup))
     for i in range(args.warmup):
         _oracle_blocks(w, per_step, start=i)
@@ -605,6 +616,8 @@ def parse_args(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="bwd", choices=["tiny", "drafter", "budget", "skew", "bwd"])
     ap.add_argument("--anchors", type=int, default=None)
+    ap.add_argument("--seed", type=int, default=None,
+                    help="input seed of the workload (default: the workload's own, 1000 + its index)")
     ap.add_argument("--workers", type=int, default=0, help="forward CTAs (default: SM count)")
     ap.add_argument("--bwd-workers", type=int, default=0, help="backward CTAs (default: SM count)")
     ap.add_argument("--q-slice", type=int, default=2,

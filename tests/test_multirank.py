@@ -76,3 +76,24 @@ def test_reference_line_keeps_the_contract():
                            "d2h_bytes_per_step": 0}
     import json
     json.dumps(line)
+
+
+def test_cpu_baseline_reports_all_cores_and_one_thread():
+    sys.path.insert(0, ROOT)
+    import bench
+    from synth import make_workload
+    r = bench.cpu_baseline(make_workload("tiny", with_grad=True), budget_s=0.6)
+    assert r["kind"] == "oracle" and r["unit"] == "TFLOP/s" and r["cores"] >= 1
+    assert r["value"] > 0 and r["value_one_thread"] > 0
+    assert "1 BLAS thread" in r["sample_one_thread"]
+
+
+def test_seed_option_reaches_the_config():
+    sys.path.insert(0, ROOT)
+    import bench
+    from synth import make_workload
+    args = bench.parse_args(["--impl", "reference", "--workload", "tiny", "--seed", "7"])
+    w = make_workload("tiny", seed=7, with_grad=True)
+    assert bench.bench_config(args, w, 148, 148, 1)["seed"] == 7
+    args = bench.parse_args(["--workload", "tiny"])
+    assert bench.bench_config(args, w, 148, 148, 1)["seed"] == 1000 + w.config.index
