@@ -32,7 +32,9 @@ listed in the repository's design notes):
 
 Modules: mask (intervals, chunk entries, pair counts), attention (forward,
 backward, chunk partials, merge), lpt (work items, LPT, contiguous baseline,
-imbalance).  All floating point is float64.
+imbalance), context_parallel (chunk ownership over ranks, a rank's partial
+result and backward share, the combine over ranks).  All floating point is
+float64.
 """
 
-from . import mask, attention, lpt  # noqa: F401
+from . import mask, attention, lpt, context_parallel  # noqa: F401
