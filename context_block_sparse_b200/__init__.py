@@ -23,7 +23,8 @@ import numpy as np
 from . import _abi
 from ._abi import (  # noqa: F401
     DTYPE_BF16, DTYPE_F32, EXPORT_BWD_LOADS, EXPORT_BWD_SCHEDULE, EXPORT_CHUNK_PAIRS,
-    EXPORT_BWD_LPT_ORDER, EXPORT_CONTIG_LOADS, EXPORT_ENTRIES, EXPORT_FWD_LOADS, EXPORT_FWD_LPT_ORDER,
+    EXPORT_BWD_LPT_ORDER, EXPORT_CHUNK_OWNER, EXPORT_CONTIG_LOADS, EXPORT_ENTRIES, EXPORT_FWD_LOADS,
+    EXPORT_FWD_LPT_ORDER, EXPORT_QUERY_SHARD, MAX_RANKS,
     EXPORT_FWD_SCHEDULE, FLAG_BLOCK_KEYS_IN_CONTEXT, FLAG_DYNAMIC_CLAIM, FLAG_EQUAL_COUNT, FLAG_FWD_TILE_COST,
     FLAG_PARTIAL_BF16, FLAG_TILE_COST,
     STATIC_SCRATCH_BYTES, WS_BWD, WS_FWD,
@@ -174,6 +175,20 @@ def splitkv_plan(sample_lens: Sequence[int], anchors: Sequence[int], block_size:
     return Plan(h, p, keep)
 
 
+def splitkv_plan_shard(sample_lens: Sequence[int], anchors: Sequence[int], block_size: int, num_q_heads: int,
+                       num_kv_heads: int, head_dim: int, kv_chunk: int, num_workers: int, num_ranks: int,
+                       rank: int, **kw) -> Plan:
+    """Rank `rank`'s plan of Split-KV over `num_ranks` ranks (splitkv_plan_shard): the
+    chunks it owns and the in-block term of its block range; other options as
+    splitkv_plan."""
+    p, keep = _problem(sample_lens, anchors, block_size, num_q_heads, num_kv_heads, head_dim, kv_chunk,
+                       num_workers, kw.pop("num_bwd_workers", 0), kw.pop("q_slice", 0),
+                       kw.pop("equal_count", False), **kw)
+    h = ctypes.c_void_p()
+    _check("splitkv_plan_shard", _lib.splitkv_plan_shard(ctypes.byref(p), int(num_ranks), int(rank), ctypes.byref(h)))
+    return Plan(h, p, keep)
+
+
 def splitkv_plan_update(plan: Plan, sample_lens, anchors, **kw) -> Plan:
     """Rebuild `plan` in place for new sample lengths / anchors (other fields kept unless given)."""
     old = plan.problem
@@ -303,6 +318,28 @@ def splitkv_read_cta_times(plan: Plan, which: int, stream=None) -> np.ndarray:
     _check("splitkv_read_cta_times", _lib.splitkv_read_cta_times(
         plan.handle, which, out.ctypes.data_as(ctypes.POINTER(ctypes.c_int64)), n, _stream_ptr(stream)))
     return out
+
+
+def splitkv_combine_ranks(o_parts, lse_parts, o, lse, stream=None) -> None:
+    """o_parts [R, rows..., d] and lse_parts [R, rows...] float32 -> o [rows..., d] (float32 or
+    bfloat16) and lse [rows...]: the exact combine of R ranks' results."""
+    R = int(o_parts.shape[0])
+    d = int(o_parts.shape[-1])
+    rows = int(lse_parts[0].numel()) if R else 0
+    if tuple(lse_parts.shape) != tuple(o_parts.shape[:-1]) or o.numel() != rows * d or lse.numel() != rows:
+        raise ValueError("o_parts [R, rows..., d], lse_parts [R, rows...], o [rows..., d], lse [rows...]")
+    _check("splitkv_combine_ranks", _lib.splitkv_combine_ranks(R, rows, d, _f32_ptr(o_parts), _f32_ptr(lse_parts),
+                                                               _ptr(o), _o_dtype(o), _f32_ptr(lse),
+                                                               _stream_ptr(stream)))
+
+
+def splitkv_sum_ranks(parts, out, stream=None) -> None:
+    """parts [R, ...] float32 -> out [...] = the sum over R, in rank order."""
+    R = int(parts.shape[0])
+    n = int(out.numel())
+    if parts.numel() != R * n:
+        raise ValueError("parts must be [R, *out.shape]")
+    _check("splitkv_sum_ranks", _lib.splitkv_sum_ranks(R, n, _f32_ptr(parts), _f32_ptr(out), _stream_ptr(stream)))
 
 
 def library_path() -> str:

@@ -44,6 +44,9 @@ EXPORT_BWD_LOADS = 5
 EXPORT_CONTIG_LOADS = 6
 EXPORT_FWD_LPT_ORDER = 7
 EXPORT_BWD_LPT_ORDER = 8
+EXPORT_CHUNK_OWNER = 9
+EXPORT_QUERY_SHARD = 10
+MAX_RANKS = 4096
 
 
 class Problem(ctypes.Structure):
@@ -99,6 +102,9 @@ SIGNATURES = {
     "splitkv_error_string": (ctypes.c_char_p, [_I]),
     "splitkv_plan": (_I, [ctypes.POINTER(Problem), ctypes.POINTER(_P)]),
     "splitkv_plan_update": (_I, [_P, ctypes.POINTER(Problem)]),
+    "splitkv_plan_shard": (_I, [ctypes.POINTER(Problem), ctypes.c_int32, ctypes.c_int32, ctypes.POINTER(_P)]),
+    "splitkv_combine_ranks": (_I, [ctypes.c_int32, ctypes.c_int64, ctypes.c_int32, _P, _P, _P, _I, _P, _P]),
+    "splitkv_sum_ranks": (_I, [ctypes.c_int32, ctypes.c_int64, _P, _P, _P]),
     "splitkv_plan_upload": (_I, [_P, _P]),
     "splitkv_plan_destroy": (_I, [_P]),
     "splitkv_plan_stats": (_I, [_P, ctypes.POINTER(Stats)]),

@@ -160,7 +160,8 @@ __global__ void __launch_bounds__(kMergeThreads, 2)
   int* sE = reinterpret_cast<int*>(sVb + p.bs * D);        // [kEStage]
   const int b = blockIdx.x, g = blockIdx.y;
   const int tid = threadIdx.x, u = tid & 3;
-  for (int idx = tid; p.block_term && idx < p.bs * (D / 8); idx += blockDim.x) {
+  const bool bterm = p.block_term && b >= p.bt_lo && b < p.bt_hi;   // in-block term of this block here
+  for (int idx = tid; bterm && idx < p.bs * (D / 8); idx += blockDim.x) {
     const int t = idx / (D / 8), ch = idx % (D / 8);
     const size_t src = (size_t(b * p.bs + t) * p.Hkv + g) * D + ch * 8;
     *reinterpret_cast<uint4*>(sKb + t * D + ch * 8) = *reinterpret_cast<const uint4*>(kb + src);
@@ -168,7 +169,7 @@ __global__ void __launch_bounds__(kMergeThreads, 2)
   }
   const int e0 = p.block_entry_ptr[b], n = p.block_entry_ptr[b + 1] - e0;
   const int R = p.G * p.bs;
-  const int n_block_keys = p.block_term ? p.bs : 0;   // no block keys when they are context keys
+  const int n_block_keys = bterm ? p.bs : 0;   // none when they are context keys, or on another rank
   for (int r0 = 0; r0 < R; r0 += kRowsPerPass) {
     // rows ordered (token, head): the 8 rows of a warp are contiguous records
     const int r = min(r0 + (tid >> 2), R - 1);          // rows past R compute, never store
@@ -335,13 +336,14 @@ __global__ void __launch_bounds__(kMergeThreads, 2)
   const int b = blockIdx.x, g = blockIdx.y;
   const int tid = threadIdx.x, u = tid & 3, warp = tid >> 5, lane = tid & 31;
   const int nwarps = blockDim.x >> 5;
-  for (int idx = tid; p.block_term && idx < bs * (D / 8); idx += blockDim.x) {
+  const bool bterm = p.block_term && b >= p.bt_lo && b < p.bt_hi;   // in-block term of this block here
+  for (int idx = tid; bterm && idx < bs * (D / 8); idx += blockDim.x) {
     const int t = idx / (D / 8), ch = idx % (D / 8);
     const size_t src = (size_t(b * bs + t) * p.Hkv + g) * D + ch * 8;
     *reinterpret_cast<uint4*>(sKb + t * D + ch * 8) = *reinterpret_cast<const uint4*>(kb + src);
     *reinterpret_cast<uint4*>(sVb + t * D + ch * 8) = *reinterpret_cast<const uint4*>(vb + src);
   }
-  const int n_block_keys = p.block_term ? bs : 0;   // no block keys when they are context keys
+  const int n_block_keys = bterm ? bs : 0;   // none when they are context keys, or on another rank
   const float scale_log2 = scale * kLog2e;
   const int e0 = p.block_entry_ptr[b], n = p.block_entry_ptr[b + 1] - e0;
   // phase 1, a quad per row: P, dS of the in-block keys; dq = in-block dq + sum of partials
@@ -392,7 +394,7 @@ __global__ void __launch_bounds__(kMergeThreads, 2)
           for (int i = 0; i < 4; ++i) acc[k][i] = fmaf(ds, kv[0][i], acc[k][i]);
         }
       }
-      if (stage_rows && active && p.block_term) {   // keep q and dout of this row for the dkb / dvb pass
+      if (stage_rows && active && bterm) {   // keep q and dout of this row for the dkb / dvb pass
 #pragma unroll
         for (int k = 0; k < NG; ++k) {
           const int off = r * D + 4 * (u + 4 * k);

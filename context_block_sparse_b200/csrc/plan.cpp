@@ -55,6 +55,10 @@ struct splitkv_plan_s {
   std::vector<uint64_t> fwd_loads, bwd_loads, contig_loads;
   std::vector<int32_t> block_entry_ptr, block_entries;
   std::vector<int32_t> zero_chunks;
+  // ranks (splitkv_plan_shard): this plan holds the entries of the chunks rank `rank`
+  // owns and the in-block term of blocks [bt_lo, bt_hi); a plain plan is rank 0 of 1
+  int32_t R = 1, rank = 0, bt_lo = 0, bt_hi = 0;
+  std::vector<int32_t> chunk_owner;               // [num_chunks]
   double plan_us = 0.0;
   // device copy
   void* d_blob = nullptr;
@@ -225,7 +229,7 @@ int build(splitkv_plan_t* P, const splitkv_problem* p) {
   P->chunk_entry_ptr.assign(P->num_chunks + 1, 0);
   for (int c = 0; c < P->num_chunks; ++c) P->chunk_entry_ptr[c + 1] = P->chunk_entry_ptr[c] + cnt[c + 1];
   const int32_t E = P->chunk_entry_ptr[P->num_chunks];
-  P->entries.resize(E);
+  P->entries.resize(size_t(E));
   {
     std::vector<int32_t> fill(P->chunk_entry_ptr.begin(), P->chunk_entry_ptr.end() - 1);
     for (int b = 0; b < P->A; ++b) {
@@ -251,6 +255,38 @@ int build(splitkv_plan_t* P, const splitkv_problem* p) {
     for (auto it = first; it != last; ++it) keys += uint64_t(it->z - it->y);
     P->chunk_pairs[c] = keys * uint64_t(P->bs);
   }
+
+  // ranks: whole chunks to ranks by LPT with equal counts (the pages' device rule), every
+  // chunk an item -- zero-cost ones too, since its keys live somewhere -- of cost
+  // Hq * pairs_c; then keep this rank's entries (their pairs are the rank's work) and
+  // the in-block term of its contiguous block range [floor(r A / R), floor((r + 1) A / R))
+  P->chunk_owner.assign(size_t(P->num_chunks), 0);
+  P->bt_lo = int32_t(int64_t(P->rank) * P->A / P->R);
+  P->bt_hi = int32_t(int64_t(P->rank + 1) * P->A / P->R);
+  if (P->R > 1) {
+    std::vector<Item> chunk_items(size_t(P->num_chunks));
+    for (int c = 0; c < P->num_chunks; ++c)
+      chunk_items[size_t(c)] = Item{c, 0, 0, 0, 0, P->chunk_pairs[size_t(c)] * uint64_t(P->Hq)};
+    std::vector<int32_t> rank_ptr, rank_order, by_cost;
+    std::vector<uint64_t> rank_loads;
+    lpt_schedule(chunk_items, P->R, true, rank_ptr, rank_order, rank_loads, by_cost);
+    for (int r = 0; r < P->R; ++r)
+      for (int k = rank_ptr[size_t(r)]; k < rank_ptr[size_t(r) + 1]; ++k)
+        P->chunk_owner[size_t(chunk_items[size_t(rank_order[size_t(k)])].c)] = r;
+    std::vector<I4> kept;
+    std::vector<int32_t> kept_ptr(size_t(P->num_chunks) + 1, 0);
+    for (int c = 0; c < P->num_chunks; ++c) {
+      if (P->chunk_owner[size_t(c)] == P->rank)
+        kept.insert(kept.end(), P->entries.begin() + P->chunk_entry_ptr[size_t(c)],
+                    P->entries.begin() + P->chunk_entry_ptr[size_t(c) + 1]);
+      else
+        P->chunk_pairs[size_t(c)] = 0;
+      kept_ptr[size_t(c) + 1] = int32_t(kept.size());
+    }
+    P->entries.swap(kept);
+    P->chunk_entry_ptr.swap(kept_ptr);
+  }
+  const int32_t E_kept = int32_t(P->entries.size());
 
   // 128-row query tiles of consecutive entries inside each chunk
   P->tiles.clear();
@@ -314,7 +350,7 @@ int build(splitkv_plan_t* P, const splitkv_problem* p) {
   for (int c = 0; c < P->num_chunks; ++c) {
     const int t0 = P->chunk_tile_ptr[c], t1 = P->chunk_tile_ptr[c + 1];
     if (t0 == t1) {
-      P->zero_chunks.push_back(c);
+      if (P->chunk_owner[size_t(c)] == P->rank) P->zero_chunks.push_back(c);   // other ranks' keys: not ours
       continue;
     }
     const uint64_t whole = P->chunk_pairs[c] * uint64_t(P->G);
@@ -368,12 +404,12 @@ int build(splitkv_plan_t* P, const splitkv_problem* p) {
 
   // block -> entries (ascending chunk)
   P->block_entry_ptr.assign(P->A + 1, 0);
-  for (int e = 0; e < E; ++e) P->block_entry_ptr[P->entries[e].x + 1]++;
+  for (int e = 0; e < E_kept; ++e) P->block_entry_ptr[P->entries[e].x + 1]++;
   for (int b = 0; b < P->A; ++b) P->block_entry_ptr[b + 1] += P->block_entry_ptr[b];
-  P->block_entries.assign(E, 0);
+  P->block_entries.assign(size_t(E_kept), 0);
   {
     std::vector<int32_t> fill(P->block_entry_ptr.begin(), P->block_entry_ptr.end() - 1);
-    for (int e = 0; e < E; ++e) P->block_entries[fill[P->entries[e].x]++] = e;  // e ascends with chunk
+    for (int e = 0; e < E_kept; ++e) P->block_entries[fill[P->entries[e].x]++] = e;  // e ascends with chunk
   }
   P->uploaded = false;
   P->plan_us = std::chrono::duration<double, std::micro>(std::chrono::steady_clock::now() - clock_start).count();
@@ -416,6 +452,31 @@ int splitkv_plan(const splitkv_problem* problem, splitkv_plan_t** out) {
   splitkv_plan_t* P = nullptr;
   try {
     P = new splitkv_plan_t();
+    const int st = build(P, problem);
+    if (st != SPLITKV_OK) {
+      delete P;
+      return st;
+    }
+  } catch (const std::bad_alloc&) {
+    delete P;
+    return SPLITKV_ERR_NO_MEMORY;
+  } catch (...) {
+    delete P;
+    return SPLITKV_ERR_INVALID_ARG;
+  }
+  *out = P;
+  return SPLITKV_OK;
+}
+
+int splitkv_plan_shard(const splitkv_problem* problem, int32_t num_ranks, int32_t rank, splitkv_plan_t** out) {
+  if (!out) return SPLITKV_ERR_INVALID_ARG;
+  *out = nullptr;
+  if (num_ranks < 1 || rank < 0 || rank >= num_ranks) return SPLITKV_ERR_INVALID_ARG;
+  splitkv_plan_t* P = nullptr;
+  try {
+    P = new splitkv_plan_t();
+    P->R = num_ranks;
+    P->rank = rank;
     const int st = build(P, problem);
     if (st != SPLITKV_OK) {
       delete P;
@@ -573,6 +634,8 @@ int splitkv_plan_upload(splitkv_plan_t* P, void* stream) {
   v.W = P->W;
   v.Wb = P->Wb;
   v.block_term = (P->flags & SPLITKV_FLAG_BLOCK_KEYS_IN_CONTEXT) ? 0 : 1;
+  v.bt_lo = P->bt_lo;
+  v.bt_hi = P->bt_hi;
   v.partial_bf16 = (P->flags & SPLITKV_FLAG_PARTIAL_BF16) ? 1 : 0;
   v.dynamic = dynamic ? 1 : 0;
   v.n_fwd_items = int(P->fwd_items.size());
@@ -612,7 +675,7 @@ int splitkv_plan_stats(const splitkv_plan_t* P, splitkv_stats* out) {
   out->context_pairs = ctx * uint64_t(P->Hq);
   out->block_pairs = (P->flags & SPLITKV_FLAG_BLOCK_KEYS_IN_CONTEXT)
                          ? 0
-                         : uint64_t(P->Hq) * uint64_t(P->A) * uint64_t(P->bs) * uint64_t(P->bs);
+                         : uint64_t(P->Hq) * uint64_t(P->bt_hi - P->bt_lo) * uint64_t(P->bs) * uint64_t(P->bs);
   out->fwd_max_load = P->fwd_loads.empty() ? 0 : *std::max_element(P->fwd_loads.begin(), P->fwd_loads.end());
   out->bwd_max_load = P->bwd_loads.empty() ? 0 : *std::max_element(P->bwd_loads.begin(), P->bwd_loads.end());
   out->fwd_imbalance = imbalance(P->fwd_loads);
@@ -667,6 +730,12 @@ int splitkv_plan_export(const splitkv_plan_t* P, int what, int64_t* out, int64_t
         }
         break;
       }
+      case SPLITKV_EXPORT_CHUNK_OWNER:
+        for (int32_t r : P->chunk_owner) v.push_back(int64_t(r));
+        break;
+      case SPLITKV_EXPORT_QUERY_SHARD:
+        v.insert(v.end(), {int64_t(P->rank), int64_t(P->R), int64_t(P->bt_lo), int64_t(P->bt_hi)});
+        break;
       default:
         return SPLITKV_ERR_INVALID_ARG;
     }

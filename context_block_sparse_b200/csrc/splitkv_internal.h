@@ -29,6 +29,7 @@ struct DevPlan {
   int num_zero_chunks;
   int N, Nq, A, bs, Hq, Hkv, G, d, C, num_chunks, E, W, Wb;
   int block_term;               // 1: separate block keys kb, vb (reading A); 0: block keys in the context
+  int bt_lo, bt_hi;             // blocks [bt_lo, bt_hi) take the in-block term (all of them, but on a rank's shard)
   int partial_bf16;             // 1: O_c records and dQ partials stored as bf16
   // run-time claims (SPLITKV_FLAG_DYNAMIC_CLAIM): fwd_items / bwd_items hold the whole
   // lists in LPT order and the CTAs claim them through claim[0] (forward kernel),

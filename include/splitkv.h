@@ -140,6 +140,12 @@ extern "C" {
 #define SPLITKV_EXPORT_FWD_LPT_ORDER  7  /* 4 per forward item, in LPT order: chunk, kv head,
                                             slice, cost (the order run-time claims take)         */
 #define SPLITKV_EXPORT_BWD_LPT_ORDER  8  /* same, backward items                                 */
+#define SPLITKV_EXPORT_CHUNK_OWNER    9  /* 1 per chunk: the rank that owns it (0 for a plain plan) */
+#define SPLITKV_EXPORT_QUERY_SHARD   10  /* 4 values: rank, number of ranks, first block, end block
+                                            of the blocks whose in-block term the plan adds      */
+
+/* Largest number of ranks splitkv_combine_ranks / splitkv_sum_ranks take. */
+#define SPLITKV_MAX_RANKS 4096
 
 /* The problem, as the news page states it ("Why short queries change the
  * problem"): packed sample lengths, anchor positions, block size, and the
@@ -202,6 +208,40 @@ const char* splitkv_error_string(int status);
  * Errors: INVALID_ARG (NULL, non-positive sizes, an anchor outside [0, N),
  * Hq % Hkv != 0), UNSUPPORTED (128 % (G * bs) != 0), NO_MEMORY. */
 int splitkv_plan(const splitkv_problem* problem, splitkv_plan_t** out);
+
+/* One rank's plan of Split-KV over `num_ranks` ranks (news page, "Exchange the
+ * smaller side": every device keeps its own share of the long context and
+ * computes partial attention of all queries against it; "Balance actual
+ * attention work": chunks go to devices by LPT on their cost with equal chunk
+ * counts).  Ownership: every chunk, zero-cost ones included, is an item of cost
+ * Hq * pairs_c (its realised (row, key) pairs over all query heads), sorted by
+ * cost descending, ties by chunk ascending, each to the eligible rank of least
+ * load (ties to the lowest rank); with n = q R + r chunks a rank is eligible while
+ * it holds fewer than q chunks, or q while fewer than r ranks hold q + 1.  Query
+ * side: rank r holds blocks [floor(r A / R), floor((r + 1) A / R)) -- their
+ * queries, and their draft keys kb, vb (reading A) -- and adds their in-block
+ * term.  The plan is splitkv_plan's over the chunks this rank owns: its entries
+ * (and workspace), schedules and stats cover them only, and its chunk pairs are
+ * 0 on other ranks' chunks.  Used with the same entry points:
+ *   splitkv_attn_fwd + splitkv_merge give, for EVERY query row, the exact result
+ *     over the keys this rank holds (O_r, LSE_r; O_r = 0 and LSE_r = -inf for a
+ *     row that meets none of them); splitkv_combine_ranks merges the ranks'
+ *     results of a row;
+ *   splitkv_attn_bwd with the final o and lse gives every row's dq share (summed
+ *     over ranks by splitkv_sum_ranks), complete dk, dv on the rows of this rank's
+ *     chunks (rows of other ranks' chunks are not written) and complete dkb, dvb
+ *     on the rows of its blocks (other rows not written).
+ * q, dout, o and lse are full-size (every query row); k and v are addressed by
+ * global position, and only the rows of this rank's chunks are read, except that
+ * a 128-key tile starting in an owned chunk may read past the chunk end into rows
+ * whose scores it masks (finite values are enough there: zero them once); kb and
+ * vb are read on the rows of this rank's blocks only.  splitkv_plan_update keeps
+ * the plan's rank.  Exports SPLITKV_EXPORT_CHUNK_OWNER and
+ * SPLITKV_EXPORT_QUERY_SHARD give the assignment.
+ * Errors: as splitkv_plan, and INVALID_ARG for num_ranks < 1 or rank outside
+ * [0, num_ranks). */
+int splitkv_plan_shard(const splitkv_problem* problem, int32_t num_ranks, int32_t rank,
+                       splitkv_plan_t** out);
 
 /* Rebuild `plan` in place for a new problem (same rules as splitkv_plan),
  * keeping its host and device buffers for reuse.  Blocks only until the
@@ -356,6 +396,26 @@ int splitkv_plan_status(const splitkv_plan_t* plan, void* stream, int32_t* site)
  * it lets a test compare the approximation with CUDA's exp2f.
  * Errors: INVALID_ARG, CUDA. */
 int splitkv_selftest_exp2(const float* x, float* y, int64_t n, void* stream);
+
+/* Exact combine of the ranks' results (news page, "Exchange the smaller side":
+ * partials over disjoint key shares merged with their normalisation statistics).
+ * o_parts [R][rows][head_dim] and lse_parts [R][rows] float32 (device; row =
+ * query token x head, 16- and 4-byte aligned), rank r's exact result over its
+ * keys (lse natural-log, -inf where rank r holds no key of the row).  For every
+ * row: M = max_r lse_r, w_r = exp(lse_r - M), o = sum_r w_r o_r / sum_r w_r
+ * (ranks in ascending order), lse = M + log(sum_r w_r); a row with no finite
+ * lse_r gets o = 0, lse = -inf.  o is float32 (16-byte aligned) or bfloat16
+ * (8-byte aligned) per o_dtype, [rows][head_dim]; lse [rows].  Asynchronous on
+ * `stream`.  Errors: INVALID_ARG (num_ranks outside [1, SPLITKV_MAX_RANKS],
+ * head_dim not a positive multiple of 4, NULL or misaligned pointer), CUDA. */
+int splitkv_combine_ranks(int32_t num_ranks, int64_t rows, int32_t head_dim, const float* o_parts,
+                          const float* lse_parts, void* o, int o_dtype, float* lse, void* stream);
+
+/* Sum of the ranks' shares: out[i] = sum_r parts[r * n + i], ranks added in
+ * ascending order (the dq of Split-KV over ranks: every rank's dq share of the
+ * rows a rank owns).  parts [R][n] and out [n] float32, 16-byte aligned, n a
+ * multiple of 4.  Asynchronous on `stream`.  Errors: INVALID_ARG, CUDA. */
+int splitkv_sum_ranks(int32_t num_ranks, int64_t n, const float* parts, float* out, void* stream);
 
 /* Per-CTA busy time of the last splitkv_attn_fwd (which = SPLITKV_WS_FWD) or
  * backward partial kernel (SPLITKV_WS_BWD) on this plan: out_ns[w] = end - start
