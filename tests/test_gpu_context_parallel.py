@@ -1,0 +1,202 @@
+"""Split-KV over ranks on the GPU, through the C ABI, against the fp64 oracle.
+
+One GPU stands in for R ranks, one after another (no rank waits on another):
+each rank plan (splitkv_plan_shard) runs the attention kernels on keys and
+values that hold only its own chunks (zeros elsewhere), the ranks' results are
+combined by splitkv_combine_ranks and their dq shares summed by
+splitkv_sum_ranks, and the outputs must match the unsplit oracle at the fixed
+tolerances (max-abs 2e-2 on O and the gradients, 1e-3 on LSE).  Guard values in
+dk, dv, dkb, dvb show that a rank writes only the rows of its own chunks and
+blocks.  The combine and the sum are also checked alone against the oracle's
+combine and an fp32 sum in rank order, and SplitKVContextParallel runs end to end
+on a one-rank NCCL group.
+"""
+
+import numpy as np
+import pytest
+
+from gpu_util import TOL_LSE, TOL_OUT, assert_close, oracle_bwd, oracle_fwd, small, to_dev
+from oracle import context_parallel as ocp
+
+pytestmark = pytest.mark.gpu
+
+GUARD = 7.0
+
+CASES = {
+    "tcgen05_R2": dict(w=dict(), R=2, plan=dict()),
+    "tcgen05_R3_claims_bf16": dict(w=dict(), R=3, plan=dict(q_slice=2, tile_cost=True, dynamic_claim=True,
+                                                            partial_bf16=True)),
+    "mma_d64_R4": dict(w=dict(Hq=4, Hkv=2, d=64), R=4, plan=dict()),
+    "chunk_not_dividing_R2": dict(w=dict(Hq=4, Hkv=1, d=128, C=100, lens=(257, 3, 1000, 61)), R=2, plan=dict()),
+    "reading_b_R2": dict(w=dict(Hq=8, Hkv=1), R=2, plan=dict(block_keys_in_context=True)),
+}
+
+
+def _emulate(skv, w, R, plan_kw):
+    import torch
+    rb = plan_kw.get("block_keys_in_context", False)
+    t = {n: to_dev(b) for n, b in w.bits.items()}
+    Nq, N, Hq, Hkv, d = w.num_queries, w.context_len, w.num_q_heads, w.num_kv_heads, w.head_dim
+    f32 = dict(dtype=torch.float32, device="cuda")
+    args = (w.sample_lens, w.anchors, w.block_size, Hq, Hkv, d, w.kv_chunk, 148)
+    plans, keep = [], []
+    o_parts = torch.empty((R, Nq, Hq, d), **f32)
+    lse_parts = torch.empty((R, Nq, Hq), **f32)
+    for r in range(R):
+        plan = skv.splitkv_plan_shard(*args, R, r, **plan_kw).upload()
+        owner = plan.export(skv.EXPORT_CHUNK_OWNER)
+        rows = torch.from_numpy(np.repeat(owner == r, w.kv_chunk)[:N]).cuda()
+        k = torch.where(rows[:, None, None], t["k"], torch.zeros_like(t["k"]))
+        v = torch.where(rows[:, None, None], t["v"], torch.zeros_like(t["v"]))
+        b_lo, b_hi = plan.export(skv.EXPORT_QUERY_SHARD).tolist()[2:]
+        if rb:
+            kb = vb = None
+        else:   # the draft keys of other ranks' blocks are not there either
+            kb, vb = torch.zeros_like(t["kb"]), torch.zeros_like(t["vb"])
+            kb[b_lo * w.block_size:b_hi * w.block_size] = t["kb"][b_lo * w.block_size:b_hi * w.block_size]
+            vb[b_lo * w.block_size:b_hi * w.block_size] = t["vb"][b_lo * w.block_size:b_hi * w.block_size]
+        ws = torch.empty(skv.splitkv_workspace_size(plan, skv.WS_FWD), dtype=torch.uint8, device="cuda")
+        skv.splitkv_attn_fwd(plan, t["q"], k, v, w.scale, ws)
+        skv.splitkv_merge(plan, t["q"], kb, vb, w.scale, ws, o_parts[r], lse_parts[r])
+        plans.append((plan, rows, k, v, kb, vb, b_lo, b_hi))
+        keep.append(ws)
+    o = torch.empty((Nq, Hq, d), **f32)
+    lse = torch.empty((Nq, Hq), **f32)
+    skv.splitkv_combine_ranks(o_parts, lse_parts, o, lse)
+    # backward of every rank with the final o, lse
+    dq_parts = torch.empty((R, Nq, Hq, d), **f32)
+    dk = torch.full((N, Hkv, d), float("nan"), **f32)
+    dv = torch.full((N, Hkv, d), float("nan"), **f32)
+    dkb = None if rb else torch.full((Nq, Hkv, d), float("nan"), **f32)
+    dvb = None if rb else torch.full((Nq, Hkv, d), float("nan"), **f32)
+    bs = w.block_size
+    for r, (plan, rows, k, v, kb, vb, b_lo, b_hi) in enumerate(plans):
+        g = {n: torch.full(shape, GUARD, **f32) for n, shape in (("dk", (N, Hkv, d)), ("dv", (N, Hkv, d)),
+                                                                   ("dkb", (Nq, Hkv, d)), ("dvb", (Nq, Hkv, d)))}
+        if rb:
+            g["dkb"] = g["dvb"] = None
+        ws = torch.empty(skv.splitkv_workspace_size(plan, skv.WS_BWD), dtype=torch.uint8, device="cuda")
+        skv.splitkv_attn_bwd(plan, t["q"], k, v, kb, vb, o, lse, t["dout"], dq_parts[r], g["dk"], g["dv"],
+                             g["dkb"], g["dvb"], w.scale, ws)
+        torch.cuda.synchronize()
+        skv.splitkv_plan_status(plan)
+        # nothing outside the rank's chunks / blocks was written
+        for n in ("dk", "dv"):
+            assert bool((g[n][~rows] == GUARD).all()), f"rank {r} wrote {n} rows of other ranks' chunks"
+            (dk if n == "dk" else dv)[rows] = g[n][rows]
+        if not rb:
+            mine = slice(b_lo * bs, b_hi * bs)
+            for n, dst in (("dkb", dkb), ("dvb", dvb)):
+                outside = torch.ones(Nq, dtype=torch.bool, device="cuda")
+                outside[mine] = False
+                assert bool((g[n][outside] == GUARD).all()), f"rank {r} wrote {n} rows of other ranks' blocks"
+                dst[mine] = g[n][mine]
+    dq = torch.empty((Nq, Hq, d), **f32)
+    skv.splitkv_sum_ranks(dq_parts, dq)
+    torch.cuda.synchronize()
+    out = {"o": o, "lse": lse, "dq": dq, "dk": dk, "dv": dv, "dkb": dkb, "dvb": dvb}
+    for plan, *_ in plans:
+        plan.destroy()
+    return {n: None if x is None else x.cpu().numpy().astype(np.float64) for n, x in out.items()}
+
+
+@pytest.mark.parametrize("case", list(CASES))
+def test_rank_plans_reproduce_unsplit_attention(splitkv, case):
+    cfg = CASES[case]
+    w = small(**cfg["w"])
+    rb = cfg["plan"].get("block_keys_in_context", False)
+    out = _emulate(splitkv, w, cfg["R"], cfg["plan"])
+    O, L = oracle_fwd(w, rb=rb)
+    assert_close("O", out["o"], O, TOL_OUT)
+    assert_close("LSE", out["lse"], L, TOL_LSE)
+    g = oracle_bwd(w, rb=rb)
+    for n in ("dq", "dk", "dv", "dkb", "dvb"):
+        if g[n] is not None:
+            assert_close(n, out[n], g[n], TOL_OUT)
+
+
+@pytest.mark.parametrize("R,d,o_bf16", [(1, 128, False), (3, 128, False), (5, 64, True), (8, 128, True)])
+def test_combine_kernel_against_oracle(splitkv, R, d, o_bf16):
+    import torch
+    rng = np.random.default_rng(R * 100 + d)
+    rows = 3001
+    o_parts = rng.standard_normal((R, rows, d)).astype(np.float32)
+    lse_parts = (rng.standard_normal((R, rows)) * 30).astype(np.float32)
+    lse_parts[rng.random((R, rows)) < 0.3] = -np.inf           # ranks holding no key of a row
+    lse_parts[:, :7] = -np.inf                                  # rows no rank holds a key of
+    lse_parts[0, 7:9] = [88.0, -88.0]                          # far above / below the other ranks
+    O, L = ocp.combine_ranks(o_parts.astype(np.float64), lse_parts.astype(np.float64))
+    dev = lambda a: torch.from_numpy(a).cuda()
+    o = torch.empty((rows, d), dtype=torch.bfloat16 if o_bf16 else torch.float32, device="cuda")
+    lse = torch.empty((rows,), dtype=torch.float32, device="cuda")
+    splitkv.splitkv_combine_ranks(dev(o_parts), dev(lse_parts), o, lse)
+    got_o = o.float().cpu().numpy().astype(np.float64)
+    got_l = lse.cpu().numpy().astype(np.float64)
+    assert np.array_equal(np.isneginf(got_l), np.isneginf(L))
+    fin = np.isfinite(L)
+    assert np.all(got_o[~fin] == 0)
+    assert np.abs(got_l[fin] - L[fin]).max() <= 1e-4 * max(1.0, np.abs(L[fin]).max())
+    assert np.abs(got_o - O).max() <= (1e-2 if o_bf16 else 1e-5) * max(1.0, np.abs(O).max())
+
+
+def test_sum_kernel_is_the_fp32_sum_in_rank_order(splitkv):
+    import torch
+    rng = np.random.default_rng(9)
+    R, n = 6, 4 * 100003
+    parts = (rng.standard_normal((R, n)) * np.exp(rng.standard_normal((R, n)) * 4)).astype(np.float32)
+    want = parts[0].copy()
+    for r in range(1, R):
+        want = (want + parts[r]).astype(np.float32)
+    out = torch.empty(n, dtype=torch.float32, device="cuda")
+    splitkv.splitkv_sum_ranks(torch.from_numpy(parts).cuda(), out)
+    assert np.array_equal(out.cpu().numpy().view(np.uint32), want.view(np.uint32))
+
+
+def test_combine_and_sum_reject_bad_arguments(splitkv):
+    import torch
+    lib = splitkv._lib
+    a = torch.zeros((2, 8, 64), dtype=torch.float32, device="cuda")
+    l = torch.zeros((2, 8), dtype=torch.float32, device="cuda")
+    o = torch.zeros((8, 64), dtype=torch.float32, device="cuda")
+    lo = torch.zeros((8,), dtype=torch.float32, device="cuda")
+    assert lib.splitkv_combine_ranks(0, 8, 64, a.data_ptr(), l.data_ptr(), o.data_ptr(), 0, lo.data_ptr(), None) == -1
+    assert lib.splitkv_combine_ranks(2, 8, 62, a.data_ptr(), l.data_ptr(), o.data_ptr(), 0, lo.data_ptr(), None) == -1
+    assert lib.splitkv_combine_ranks(2, 8, 64, a.data_ptr() + 4, l.data_ptr(), o.data_ptr(), 0, lo.data_ptr(),
+                                     None) == -1
+    assert lib.splitkv_combine_ranks(2, 8, 64, a.data_ptr(), l.data_ptr(), o.data_ptr(), 5, lo.data_ptr(), None) == -1
+    assert lib.splitkv_sum_ranks(2, 6, a.data_ptr(), o.data_ptr(), None) == -1
+    assert lib.splitkv_sum_ranks(2, 8, a.data_ptr() + 8, o.data_ptr(), None) == -1
+    assert lib.splitkv_sum_ranks(2, 0, None, None, None) == 0
+
+
+def test_context_parallel_class_on_one_nccl_rank(splitkv):
+    """SplitKVContextParallel end to end (broadcasts, all-to-all, kernels) on a one-rank group."""
+    import socket
+
+    import torch
+    import torch.distributed as dist
+    from context_block_sparse_b200.context_parallel import SplitKVContextParallel
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    port = s.getsockname()[1]
+    s.close()
+    dist.init_process_group("nccl", init_method=f"tcp://127.0.0.1:{port}", rank=0, world_size=1,
+                            device_id=torch.device("cuda", 0))
+    try:
+        w = small()
+        t = {n: to_dev(b) for n, b in w.bits.items()}
+        cp = SplitKVContextParallel(w.sample_lens, w.anchors, w.block_size, w.num_q_heads, w.num_kv_heads,
+                                    w.head_dim, w.kv_chunk, q_slice=2, tile_cost=True, dynamic_claim=True)
+        assert cp.owned_rows() == [(c * w.kv_chunk, min((c + 1) * w.kv_chunk, w.context_len))
+                                   for c in range(-(-w.context_len // w.kv_chunk))]
+        o, lse = cp.forward(t["q"], t["k"], t["v"], t["kb"], t["vb"], w.scale)
+        g = cp.backward(t["k"], t["v"], o, lse, t["dout"], w.scale)
+        torch.cuda.synchronize()
+        O, L = oracle_fwd(w)
+        assert_close("O", o.cpu().numpy().astype(np.float64), O, TOL_OUT)
+        assert_close("LSE", lse.cpu().numpy().astype(np.float64), L, TOL_LSE)
+        ref = oracle_bwd(w)
+        for n in ("dq", "dk", "dv", "dkb", "dvb"):
+            assert_close(n, g[n].cpu().numpy().astype(np.float64), ref[n], TOL_OUT)
+    finally:
+        dist.destroy_process_group()
