@@ -115,6 +115,38 @@ def test_rank_plans_reproduce_unsplit_attention(splitkv, case):
             assert_close(n, out[n], g[n], TOL_OUT)
 
 
+def test_bwd_workload_over_four_ranks_sampled(splitkv):
+    """64k context, 8k queries, 32 / 8 heads over 4 emulated ranks (the bench's run-time
+    claims and tile cost): O, LSE, dQ, dKb, dVb on sampled blocks; dK, dV on the keys of
+    two chunks, the oracle summing over every block that reads them."""
+    from oracle import mask as omask
+    from synth import make_workload
+    w = make_workload("bwd")
+    out = _emulate(splitkv, w, 4, dict(q_slice=2, tile_cost=True, dynamic_claim=True))
+    rng = np.random.default_rng(0)
+    A, bs = w.anchors.size, w.block_size
+    blocks = sorted({0, A - 1, A // 4, A // 2, 3 * A // 4} | set(rng.choice(A, size=4, replace=False).tolist()))
+    rows = np.concatenate([np.arange(b * bs, (b + 1) * bs) for b in blocks])
+    O, L = oracle_fwd(w, blocks)
+    assert_close("O", out["o"][rows], O[rows], TOL_OUT)
+    assert_close("LSE", out["lse"][rows], L[rows], TOL_LSE)
+    g = oracle_bwd(w, blocks)
+    for n in ("dq", "dkb", "dvb"):
+        assert_close(n, out[n][rows], g[n][rows], TOL_OUT)
+    C = w.kv_chunk
+    starts = omask.sample_starts(w.sample_lens) + [w.context_len]
+    mid = len(w.sample_lens) // 2
+    chunks = sorted({(starts[1] - 1) // C, (starts[mid + 1] - 1) // C})
+    iv = omask.context_interval(w.sample_lens, w.anchors)
+    readers = [b for b, (S, a) in enumerate(iv) if any(S < (c + 1) * C and a > c * C for c in chunks)]
+    g2 = oracle_bwd(w, readers)
+    keys = np.concatenate([np.arange(c * C, min((c + 1) * C, w.context_len)) for c in chunks])
+    for n in ("dk", "dv"):
+        assert_close(n, out[n][keys], g2[n][keys], TOL_OUT)
+    for n in ("o", "lse", "dq", "dk", "dv", "dkb", "dvb"):
+        assert np.isfinite(out[n]).all(), n
+
+
 @pytest.mark.parametrize("R,d,o_bf16", [(1, 128, False), (3, 128, False), (5, 64, True), (8, 128, True)])
 def test_combine_kernel_against_oracle(splitkv, R, d, o_bf16):
     import torch
