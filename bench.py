@@ -433,6 +433,9 @@ def run_ours(args, world, rank, local):
 
     if rank == 0:
         result["device_lpt"] = device_lpt_report(skv, w)
+    if rank == 0 and world == 1 and args.emulate_ranks > 1:
+        result["split_kv_ranks"] = rank_emulation_report(skv, w, args, args.emulate_ranks, dev, stream, t, W, Wb,
+                                                          peaks)
     if not args.no_e2e:
         result["e2e"] = run_e2e(args, w, plan, dev, stream, flops_step, world=world)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -463,6 +466,96 @@ def device_lpt_report(skv, w, workers=(8, 16, 32, 64)):
         row["makespan_ratio"] = (1 + row["contiguous_imbalance_pct"] / 100) / (1 + row["equal_count_imbalance_pct"] / 100)
         out[str(W)] = row
     return out
+
+
+def rank_emulation_report(skv, w, args, R, dev, stream, t, W, Wb, peaks, reps=5):
+    """Split-KV over R ranks with one GPU standing in for each rank in turn (after the timed
+    region, untimed by the bench line): per rank, the device time of its forward
+    (splitkv_attn_fwd + splitkv_merge) and backward (splitkv_attn_bwd) on its rank plan, the
+    median of `reps`; the measured rank imbalance (max / mean - 1 of forward + backward)
+    against the planned one (the ranks' summed chunk costs, news page "Balance actual
+    attention work"); and the combine / sum kernels of the exchange against the HBM peak.
+    The collectives themselves are not timed (one GPU)."""
+    import torch
+    f32 = dict(dtype=torch.float32, device=dev)
+    d, Hq, Hkv, Nq, N = w.head_dim, w.num_q_heads, w.num_kv_heads, w.num_queries, w.context_len
+    kw = dict(num_bwd_workers=Wb, q_slice=args.q_slice, partial_bf16=args.partial_bf16,
+              tile_cost=args.lpt_cost == "tiles", dynamic_claim=args.dynamic_claim)
+    args_p = (w.sample_lens, w.anchors, w.block_size, Hq, Hkv, d, w.kv_chunk, W)
+    o_parts = torch.empty((R, Nq, Hq, d), **f32)
+    lse_parts = torch.empty((R, Nq, Hq), **f32)
+    dq_parts = torch.empty((R, Nq, Hq, d), **f32)
+    dk, dv = torch.zeros(t["k"].shape, **f32), torch.zeros(t["v"].shape, **f32)
+    dkb, dvb = torch.zeros(t["kb"].shape, **f32), torch.zeros(t["vb"].shape, **f32)
+    o = torch.empty((Nq, Hq, d), **f32)
+    lse = torch.empty((Nq, Hq), **f32)
+
+    def timed(fn):
+        out = []
+        for _ in range(reps + 1):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            fn()
+            b.record(stream)
+            torch.cuda.synchronize(dev)
+            out.append(a.elapsed_time(b))
+        return float(np.median(out[1:]))
+
+    fwd_ms, bwd_ms, loads = [], [], []
+    full = skv.splitkv_plan(*args_p, **kw)
+    full_pairs = full.export(skv.EXPORT_CHUNK_PAIRS)
+    full.destroy()
+    plans = []
+    for r in range(R):
+        plan = skv.splitkv_plan_shard(*args_p, R, r, **kw).upload(stream)
+        owner = plan.export(skv.EXPORT_CHUNK_OWNER)
+        loads.append(int(Hq * full_pairs[owner == r].sum()))
+        ws_f = torch.empty(skv.splitkv_workspace_size(plan, skv.WS_FWD), dtype=torch.uint8, device=dev)
+        ws_b = torch.empty(skv.splitkv_workspace_size(plan, skv.WS_BWD), dtype=torch.uint8, device=dev)
+        plans.append((plan, ws_f, ws_b))
+
+        def fwd(plan=plan, ws_f=ws_f, r=r):
+            skv.splitkv_attn_fwd(plan, t["q"], t["k"], t["v"], w.scale, ws_f, stream)
+            skv.splitkv_merge(plan, t["q"], t["kb"], t["vb"], w.scale, ws_f, o_parts[r], lse_parts[r], stream)
+
+        fwd_ms.append(timed(fwd))
+    # the backward of every rank runs with the combined o, lse
+    skv.splitkv_combine_ranks(o_parts, lse_parts, o, lse, stream)
+    for r, (plan, ws_f, ws_b) in enumerate(plans):
+        def bwd(plan=plan, ws_b=ws_b, r=r):
+            skv.splitkv_attn_bwd(plan, t["q"], t["k"], t["v"], t["kb"], t["vb"], o, lse, t["dout"], dq_parts[r],
+                                 dk, dv, dkb, dvb, w.scale, ws_b, stream)
+
+        bwd_ms.append(timed(bwd))
+        skv.splitkv_plan_status(plan, stream)
+    for plan, _, _ in plans:
+        plan.destroy()
+    plans.clear()
+    comb_ms = timed(lambda: skv.splitkv_combine_ranks(o_parts, lse_parts, o, lse, stream))
+    dq = torch.empty((Nq, Hq, d), **f32)
+    sum_ms = timed(lambda: skv.splitkv_sum_ranks(dq_parts, dq, stream))
+    rows = Nq * Hq
+    comb_bytes = (R + 1) * rows * (4 * d + 4)
+    sum_bytes = 4 * (R + 1) * rows * d
+    step = [f + b for f, b in zip(fwd_ms, bwd_ms)]
+
+    def imb(x):
+        x = np.asarray(x, dtype=np.float64)
+        return float(x.max() / x.mean() - 1.0) if x.size and x.mean() > 0 else 0.0
+
+    return {
+        "ranks": R,
+        "planned_loads": loads,
+        "planned_imbalance_pct": 100 * imb(loads),
+        "fwd_ms": fwd_ms,
+        "bwd_ms": bwd_ms,
+        "measured_imbalance_pct": 100 * imb(step),
+        "combine": {"ms": comb_ms, "gbs": comb_bytes / (comb_ms * 1e-3) / 1e9,
+                    "frac": comb_bytes / (comb_ms * 1e-3) / 1e9 / peaks["hbm_gbs"], "rows": rows},
+        "sum": {"ms": sum_ms, "gbs": sum_bytes / (sum_ms * 1e-3) / 1e9,
+                "frac": sum_bytes / (sum_ms * 1e-3) / 1e9 / peaks["hbm_gbs"]},
+        "note": "one GPU runs each rank plan in turn; combine / sum timed over all query rows at once",
+    }
 
 
 def run_e2e(args, w, plan, dev, stream, flops_step, world=1):
@@ -639,6 +732,8 @@ def parse_args(argv=None):
     ap.add_argument("--dump-cta-times", default=None, metavar="PATH",
                     help="write the measured per-CTA busy times of the last step (fwd partial and dK/dV "
                          "kernels, ns) with the schedule options to PATH as JSON")
+    ap.add_argument("--emulate-ranks", type=int, default=0, metavar="R",
+                    help="also report Split-KV over R ranks, one GPU running each rank plan in turn")
     ap.add_argument("--partial-bf16", action="store_true",
                     help="store the partial records (O_c, dQ partials) as bf16 (plan flag; default float32)")
     args = ap.parse_args(argv)

@@ -97,3 +97,11 @@ def test_seed_option_reaches_the_config():
     assert bench.bench_config(args, w, 148, 148, 1)["seed"] == 7
     args = bench.parse_args(["--workload", "tiny"])
     assert bench.bench_config(args, w, 148, 148, 1)["seed"] == 1000 + w.config.index
+
+
+def test_rank_emulation_option():
+    sys.path.insert(0, ROOT)
+    import bench
+    assert bench.parse_args([]).emulate_ranks == 0                 # not part of the default run
+    assert bench.parse_args(["--emulate-ranks", "4"]).emulate_ranks == 4
+    assert callable(bench.rank_emulation_report)
