@@ -1,6 +1,5 @@
 """Bad arguments come back as status codes from host-side checks; no kernel is given a bad pointer."""
 
-import numpy as np
 import pytest
 
 from gpu_util import small, to_dev

@@ -2,7 +2,6 @@
 
 import ctypes
 
-import numpy as np
 import pytest
 
 pytestmark = pytest.mark.gpu

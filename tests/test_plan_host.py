@@ -11,7 +11,7 @@ from hypothesis import given, settings, strategies as st
 
 from oracle import lpt as olpt
 from oracle import mask as omask
-from synth import CONFIGS, make_workload
+from synth import make_workload
 
 
 def _plan(skv, lens, anchors, bs, Hq, Hkv, d, C, W, Wb=0, q_slice=0, eq=False, rb=False, tc=False, ftc=False,
