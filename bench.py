@@ -282,6 +282,8 @@ def run_ours(args, world, rank, local):
                             dynamic_claim=args.dynamic_claim)
     plan.upload(stream)
     st = plan.stats()
+    if args.dump_plan and rank == 0:
+        plan.dump(args.dump_plan)
     ws_f = torch.empty(skv.splitkv_workspace_size(plan, skv.WS_FWD), dtype=torch.uint8, device=dev)
     ws_b = torch.empty(skv.splitkv_workspace_size(plan, skv.WS_BWD), dtype=torch.uint8, device=dev)
     f32 = dict(dtype=torch.float32, device=dev)
@@ -732,6 +734,8 @@ def parse_args(argv=None):
     ap.add_argument("--dump-cta-times", default=None, metavar="PATH",
                     help="write the measured per-CTA busy times of the last step (fwd partial and dK/dV "
                          "kernels, ns) with the schedule options to PATH as JSON")
+    ap.add_argument("--dump-plan", default=None, metavar="PATH",
+                    help="write the run's plan (problem, stats, every table) to PATH (.npz)")
     ap.add_argument("--emulate-ranks", type=int, default=0, metavar="R",
                     help="also report Split-KV over R ranks, one GPU running each rank plan in turn")
     ap.add_argument("--partial-bf16", action="store_true",

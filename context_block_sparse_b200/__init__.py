@@ -115,6 +115,10 @@ class Plan:
     def export(self, what: int) -> np.ndarray:
         return splitkv_plan_export(self, what)
 
+    def dump(self, path: str) -> None:
+        """Write the plan to `path` (.npz): the problem, the stats and every exported table."""
+        splitkv_plan_dump(self, path)
+
     def upload(self, stream=None) -> "Plan":
         splitkv_plan_upload(self, stream)
         return self
@@ -231,6 +235,35 @@ def splitkv_plan_export(plan: Plan, what: int) -> np.ndarray:
     _check("splitkv_plan_export", _lib.splitkv_plan_export(
         plan.handle, what, out.ctypes.data_as(ctypes.POINTER(ctypes.c_int64)), out.size, ctypes.byref(n)))
     return out[:n.value]
+
+
+_PROBLEM_FIELDS = ("block_size", "num_q_heads", "num_kv_heads", "head_dim", "kv_chunk", "num_workers",
+                   "num_bwd_workers", "q_slice", "flags")
+_EXPORTS = ("entries", "chunk_pairs", "fwd_schedule", "bwd_schedule", "fwd_loads", "bwd_loads", "contig_loads",
+            "fwd_lpt_order", "bwd_lpt_order", "chunk_owner", "query_shard")
+
+
+def splitkv_plan_dump(plan: Plan, path: str) -> None:
+    """The plan as a reproducible record (.npz): sample lengths, anchors and the other problem
+    fields, the stats (plan_us aside, which is a timing), and every SPLITKV_EXPORT_* table.
+    Two plans of the same problem give identical dumps (the planner is integer arithmetic)."""
+    p = plan.problem
+    rec = {"sample_lens": np.ctypeslib.as_array(p.sample_lens, shape=(p.num_samples,)).copy(),
+           "anchors": np.ctypeslib.as_array(p.anchors, shape=(p.num_anchors,)).copy()}
+    for f in _PROBLEM_FIELDS:
+        rec["problem_" + f] = np.int64(getattr(p, f))
+    for k, v in splitkv_plan_stats(plan).items():
+        if k != "plan_us":
+            rec["stats_" + k] = np.asarray(v)
+    for i, name in enumerate(_EXPORTS):
+        rec[name] = splitkv_plan_export(plan, i)
+    np.savez(path, **rec)
+
+
+def splitkv_plan_load_dump(path: str) -> dict:
+    """A dump written by splitkv_plan_dump, as a dict of numpy arrays."""
+    with np.load(path) as z:
+        return {k: z[k] for k in z.files}
 
 
 def splitkv_workspace_size(plan: Plan, which: int) -> int:

@@ -235,3 +235,28 @@ def test_context_at_int32_limit_rejected(splitkv):
     plan = _plan(splitkv, lens, [5], 16, 2, 1, 128, 2 ** 28, 4)
     assert plan.stats()["context_pairs"] == 2 * 16 * 5
     plan.destroy()
+
+
+def test_plan_dump_is_reproducible(splitkv, tmp_path):
+    """A dump (problem, stats, every exported table) of two plans of the same problem is
+    identical, and its tables are the plan's exports."""
+    w = make_workload("drafter", seed=1001, with_grad=False)
+    args = (w.sample_lens, w.anchors, w.block_size, w.num_q_heads, w.num_kv_heads, w.head_dim, w.kv_chunk, 148)
+    a = splitkv.splitkv_plan(*args, q_slice=2, tile_cost=True, dynamic_claim=True)
+    b = splitkv.splitkv_plan(*args, q_slice=2, tile_cost=True, dynamic_claim=True)
+    a.dump(str(tmp_path / "a.npz"))
+    b.dump(str(tmp_path / "b.npz"))
+    da = splitkv.splitkv_plan_load_dump(str(tmp_path / "a.npz"))
+    db = splitkv.splitkv_plan_load_dump(str(tmp_path / "b.npz"))
+    assert sorted(da) == sorted(db)
+    for k in da:
+        assert np.array_equal(da[k], db[k]), k
+    assert np.array_equal(da["fwd_schedule"], a.export(splitkv.EXPORT_FWD_SCHEDULE))
+    assert np.array_equal(da["anchors"], np.asarray(w.anchors, dtype=np.int32))
+    assert int(da["problem_flags"]) == splitkv.FLAG_TILE_COST | splitkv.FLAG_DYNAMIC_CLAIM
+    assert int(da["stats_num_entries"]) == a.stats()["num_entries"]
+    s = splitkv.splitkv_plan_shard(*args, 4, 3)
+    s.dump(str(tmp_path / "s.npz"))
+    ds = splitkv.splitkv_plan_load_dump(str(tmp_path / "s.npz"))
+    assert ds["query_shard"].tolist() == [3, 4, 3 * len(w.anchors) // 4, len(w.anchors)]
+    assert np.array_equal(ds["chunk_owner"], s.export(splitkv.EXPORT_CHUNK_OWNER))
