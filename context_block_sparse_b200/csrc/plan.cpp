@@ -109,6 +109,31 @@ int validate(const splitkv_problem* p) {
 // keys (the same order as a stable sort by cost descending, in O(n) per pass).
 void sort_by_cost_desc(const std::vector<Item>& items, std::vector<int32_t>& out) {
   const int64_t n = int64_t(items.size());
+  uint64_t max_cost = 0;
+  for (const Item& it : items) max_cost = std::max(max_cost, it.cost);
+  if (max_cost <= 0xffffffffull && n <= (int64_t(1) << 31)) {
+    // costs fit in 32 bits: sort packed keys ((~cost) << 32 | index) by their high half,
+    // stably, so equal costs keep index order -- one contiguous array, no indirection
+    std::vector<uint64_t> a(static_cast<size_t>(n)), b(static_cast<size_t>(n));
+    uint32_t any_one = 0, all_one = 0xffffffffu;
+    for (int64_t i = 0; i < n; ++i) {
+      const uint32_t k = ~uint32_t(items[size_t(i)].cost);
+      any_one |= k;
+      all_one &= k;
+      a[size_t(i)] = (uint64_t(k) << 32) | uint64_t(i);
+    }
+    for (int shift = 32; shift < 64; shift += 8) {
+      if ((((uint64_t(any_one ^ all_one) << 32) >> shift) & 0xffu) == 0) continue;   // a constant byte
+      int64_t cnt[257] = {};
+      for (int64_t i = 0; i < n; ++i) cnt[((a[size_t(i)] >> shift) & 0xffu) + 1]++;
+      for (int d = 0; d < 256; ++d) cnt[d + 1] += cnt[d];
+      for (int64_t i = 0; i < n; ++i) b[size_t(cnt[(a[size_t(i)] >> shift) & 0xffu]++)] = a[size_t(i)];
+      a.swap(b);
+    }
+    out.resize(size_t(n));
+    for (int64_t i = 0; i < n; ++i) out[size_t(i)] = int32_t(a[size_t(i)] & 0xffffffffu);
+    return;
+  }
   std::vector<int32_t> a(n), b(n);
   for (int64_t i = 0; i < n; ++i) a[i] = int32_t(i);
   uint64_t any_one = 0, all_one = ~uint64_t(0);
@@ -154,7 +179,47 @@ void lpt_schedule(const std::vector<Item>& items, int W, bool equal_count,
     heap[i] = x;
   };
   int64_t n_full = 0;  // workers holding q + 1 items
-  for (int64_t k = 0; k < n; ++k) {
+  // Plain LPT whose loads stay small enough: the heap holds keys (load << id_bits) | id,
+  // whose integer order is the (load, id) order, and the sift picks children without
+  // branches.  Distinct keys have one minimum, so every choice is the same as below.
+  int id_bits = 1;
+  while ((int64_t(1) << id_bits) < W) ++id_bits;
+  uint64_t total = 0;
+  bool fits = !equal_count;
+  for (const Item& it : items) {
+    total += it.cost;
+    if (total >= (uint64_t(1) << (63 - id_bits))) fits = false;
+  }
+  if (fits) {
+    std::vector<uint64_t> key(static_cast<size_t>(W));
+    for (int w = 0; w < W; ++w) key[size_t(w)] = uint64_t(w);   // all loads 0: ids ascending is a heap
+    const uint64_t id_mask = (uint64_t(1) << id_bits) - 1;
+    for (int64_t k = 0; k < n; ++k) {
+      const int32_t it = sorted[size_t(k)];
+      const uint64_t top = key[0];
+      const int32_t w = int32_t(top & id_mask);
+      const uint64_t x = top + (items[size_t(it)].cost << id_bits);
+      loads[size_t(w)] += items[size_t(it)].cost;
+      owner[size_t(k)] = w;
+      int i = 0;
+      for (;;) {
+        int c = 2 * i + 1;
+        if (c >= W) break;
+        uint64_t kc = key[size_t(c)];
+        if (c + 1 < W) {
+          const uint64_t k2 = key[size_t(c) + 1];
+          const bool right = k2 < kc;
+          c += right ? 1 : 0;
+          kc = right ? k2 : kc;
+        }
+        if (kc >= x) break;
+        key[size_t(i)] = kc;
+        i = c;
+      }
+      key[size_t(i)] = x;
+    }
+  }
+  for (int64_t k = 0; k < n && !fits; ++k) {
     const int32_t it = sorted[k];
     if (equal_count) {
       // drop tops that can no longer take an item; some worker always can

@@ -260,3 +260,14 @@ def test_plan_dump_is_reproducible(splitkv, tmp_path):
     ds = splitkv.splitkv_plan_load_dump(str(tmp_path / "s.npz"))
     assert ds["query_shard"].tolist() == [3, 4, 3 * len(w.anchors) // 4, len(w.anchors)]
     assert np.array_equal(ds["chunk_owner"], s.export(splitkv.EXPORT_CHUNK_OWNER))
+
+
+def test_costs_above_32_bits_bit_exact(splitkv):
+    """Item costs past 2^32 (72 blocks of 16 x 8 heads reading whole chunks of 2^19 keys)
+    take the planner's wide sort; the schedules still equal the oracle's."""
+    lens = [1 << 21, 1000]
+    anchors = [(1 << 21) - 1 - 3 * i for i in range(72)] + [(1 << 21) + 500, 1 << 20]
+    C = 1 << 19
+    assert max(omask.chunk_pairs(lens, anchors, 16, C)) * 8 > (1 << 32)
+    _check_against_oracle(splitkv, lens, anchors, 16, 8, 1, C, 3, q_slice=1)
+    _check_against_oracle(splitkv, lens, anchors, 16, 8, 1, C, 2, eq=True)
