@@ -86,6 +86,29 @@ def _f32_ptr(t) -> int:
     return _ptr(t)
 
 
+def _dims(plan: "Plan") -> dict:
+    """Element counts of every tensor of an attention call, from the plan's problem (cached on
+    the plan until splitkv_plan_update)."""
+    if plan._dims is not None:
+        return plan._dims
+    st = splitkv_plan_stats(plan)
+    p = plan.problem
+    N, Nq, Hq, Hkv, d = st["context_len"], st["num_queries"], p.num_q_heads, p.num_kv_heads, p.head_dim
+    qs, ks, bs_ = Nq * Hq * d, N * Hkv * d, Nq * Hkv * d
+    plan._dims = {"q": qs, "dout": qs, "o": qs, "dq": qs, "lse": Nq * Hq, "k": ks, "v": ks, "dk": ks, "dv": ks,
+            "kb": bs_, "vb": bs_, "dkb": bs_, "dvb": bs_}
+    return plan._dims
+
+
+def _sizes(plan: "Plan", **tensors) -> None:
+    """Every given tensor must hold exactly the elements the plan's layout gives it (the C
+    entry points take bare pointers; a short tensor would be read or written past its end)."""
+    want = _dims(plan)
+    for name, t in tensors.items():
+        if t is not None and t.numel() != want[name]:
+            raise ValueError(f"{name} has {t.numel()} elements; the plan's layout needs {want[name]}")
+
+
 def _o_dtype(o) -> int:
     import torch
     if o.dtype == torch.float32:
@@ -102,6 +125,7 @@ class Plan:
         self._h = handle
         self.problem = problem
         self._keep = keep
+        self._dims = None
 
     @property
     def handle(self) -> ctypes.c_void_p:
@@ -208,7 +232,7 @@ def splitkv_plan_update(plan: Plan, sample_lens, anchors, **kw) -> Plan:
     args.update(kw)
     p, keep = _problem(sample_lens, anchors, **args)
     _check("splitkv_plan_update", _lib.splitkv_plan_update(plan.handle, ctypes.byref(p)))
-    plan.problem, plan._keep = p, keep
+    plan.problem, plan._keep, plan._dims = p, keep, None
     return plan
 
 
@@ -274,6 +298,7 @@ def splitkv_workspace_size(plan: Plan, which: int) -> int:
 
 def splitkv_attn_fwd(plan: Plan, q, k, v, scale: float, ws, stream=None) -> None:
     """Chunk partial records into ws (uint8 CUDA tensor of splitkv_workspace_size(plan, WS_FWD) bytes)."""
+    _sizes(plan, q=q, k=k, v=v)
     _check("splitkv_attn_fwd", _lib.splitkv_attn_fwd(
         plan.handle, _bf16_ptr(q), _bf16_ptr(k), _bf16_ptr(v), float(scale), _ptr(ws), ws.numel() * ws.element_size(),
         _stream_ptr(stream)))
@@ -281,6 +306,7 @@ def splitkv_attn_fwd(plan: Plan, q, k, v, scale: float, ws, stream=None) -> None
 
 def splitkv_merge(plan: Plan, q, kb, vb, scale: float, ws, o, lse, stream=None) -> None:
     """In-block term + exact LSE merge of the chunk records -> o (f32 or bf16), lse (f32)."""
+    _sizes(plan, q=q, kb=kb, vb=vb, o=o, lse=lse)
     _check("splitkv_merge", _lib.splitkv_merge(
         plan.handle, _bf16_ptr(q), _bf16_ptr(kb), _bf16_ptr(vb), float(scale), _ptr(ws),
         ws.numel() * ws.element_size(), _ptr(o), _o_dtype(o), _f32_ptr(lse), _stream_ptr(stream)))
@@ -289,6 +315,7 @@ def splitkv_merge(plan: Plan, q, kb, vb, scale: float, ws, o, lse, stream=None) 
 def splitkv_attn_bwd(plan: Plan, q, k, v, kb, vb, o, lse, dout, dq, dk, dv, dkb, dvb, scale: float, ws,
                      stream=None) -> None:
     """Gradients dq, dk, dv, dkb, dvb (float32) recomputed from the saved lse."""
+    _sizes(plan, q=q, k=k, v=v, kb=kb, vb=vb, o=o, lse=lse, dout=dout, dq=dq, dk=dk, dv=dv, dkb=dkb, dvb=dvb)
     _check("splitkv_attn_bwd", _lib.splitkv_attn_bwd(
         plan.handle, _bf16_ptr(q), _bf16_ptr(k), _bf16_ptr(v), _bf16_ptr(kb), _bf16_ptr(vb), _ptr(o),
         _o_dtype(o), _f32_ptr(lse), _bf16_ptr(dout), _f32_ptr(dq), _f32_ptr(dk), _f32_ptr(dv), _f32_ptr(dkb),
@@ -296,30 +323,35 @@ def splitkv_attn_bwd(plan: Plan, q, k, v, kb, vb, o, lse, dout, dq, dk, dv, dkb,
 
 
 def splitkv_bwd_delta(plan: Plan, o, dout, ws, stream=None) -> None:
+    _sizes(plan, o=o, dout=dout)
     _check("splitkv_bwd_delta", _lib.splitkv_bwd_delta(
         plan.handle, _ptr(o), _o_dtype(o), _bf16_ptr(dout), _ptr(ws), ws.numel() * ws.element_size(),
         _stream_ptr(stream)))
 
 
 def splitkv_bwd_partial(plan: Plan, q, k, v, lse, dout, dk, dv, scale: float, ws, stream=None) -> None:
+    _sizes(plan, q=q, k=k, v=v, lse=lse, dout=dout, dk=dk, dv=dv)
     _check("splitkv_bwd_partial", _lib.splitkv_bwd_partial(
         plan.handle, _bf16_ptr(q), _bf16_ptr(k), _bf16_ptr(v), _f32_ptr(lse), _bf16_ptr(dout), _f32_ptr(dk),
         _f32_ptr(dv), float(scale), _ptr(ws), ws.numel() * ws.element_size(), _stream_ptr(stream)))
 
 
 def splitkv_bwd_dkdv(plan: Plan, q, k, v, lse, dout, dk, dv, scale: float, ws, stream=None) -> None:
+    _sizes(plan, q=q, k=k, v=v, lse=lse, dout=dout, dk=dk, dv=dv)
     _check("splitkv_bwd_dkdv", _lib.splitkv_bwd_dkdv(
         plan.handle, _bf16_ptr(q), _bf16_ptr(k), _bf16_ptr(v), _f32_ptr(lse), _bf16_ptr(dout), _f32_ptr(dk),
         _f32_ptr(dv), float(scale), _ptr(ws), ws.numel() * ws.element_size(), _stream_ptr(stream)))
 
 
 def splitkv_bwd_dq(plan: Plan, q, k, v, lse, dout, scale: float, ws, stream=None) -> None:
+    _sizes(plan, q=q, k=k, v=v, lse=lse, dout=dout)
     _check("splitkv_bwd_dq", _lib.splitkv_bwd_dq(
         plan.handle, _bf16_ptr(q), _bf16_ptr(k), _bf16_ptr(v), _f32_ptr(lse), _bf16_ptr(dout), float(scale),
         _ptr(ws), ws.numel() * ws.element_size(), _stream_ptr(stream)))
 
 
 def splitkv_bwd_reduce(plan: Plan, q, kb, vb, lse, dout, dq, dkb, dvb, scale: float, ws, stream=None) -> None:
+    _sizes(plan, q=q, kb=kb, vb=vb, lse=lse, dout=dout, dq=dq, dkb=dkb, dvb=dvb)
     _check("splitkv_bwd_reduce", _lib.splitkv_bwd_reduce(
         plan.handle, _bf16_ptr(q), _bf16_ptr(kb), _bf16_ptr(vb), _f32_ptr(lse), _bf16_ptr(dout), _f32_ptr(dq),
         _f32_ptr(dkb), _f32_ptr(dvb), float(scale), _ptr(ws), ws.numel() * ws.element_size(),
@@ -328,6 +360,7 @@ def splitkv_bwd_reduce(plan: Plan, q, kb, vb, lse, dout, dq, dkb, dvb, scale: fl
 
 def splitkv_attn_fwd_static_scratch(plan: Plan, q, k, v, kb, vb, scale: float, o, lse, stream=None) -> None:
     """Forward + merge with the partial records in the library's static device buffer (no allocation)."""
+    _sizes(plan, q=q, k=k, v=v, kb=kb, vb=vb, o=o, lse=lse)
     _check("splitkv_attn_fwd_static_scratch", _lib.splitkv_attn_fwd_static_scratch(
         plan.handle, _bf16_ptr(q), _bf16_ptr(k), _bf16_ptr(v), _bf16_ptr(kb), _bf16_ptr(vb), float(scale),
         _ptr(o), _o_dtype(o), _f32_ptr(lse), _stream_ptr(stream)))

@@ -60,3 +60,33 @@ def test_struct_layouts_match_header(tmp_path):
         size, offs = _c_layout(struct, fields, tmp_path)
         assert ctypes.sizeof(cls) == size, struct
         assert [getattr(cls, f).offset for f in fields] == offs, struct
+
+
+def test_bindings_check_tensor_sizes_against_the_plan(splitkv):
+    """The C entry points take bare pointers; the binding refuses a tensor whose element count
+    differs from the plan's layout before any pointer is taken (checked here on CPU tensors,
+    which then fail the CUDA check)."""
+    import pytest
+    import torch
+    plan = splitkv.splitkv_plan([300, 200], [10, 250, 400], 16, 4, 2, 64, 128, 8)
+    Nq, N = 3 * 16, 500
+    bf = dict(dtype=torch.bfloat16)
+    q, k, v = torch.zeros(Nq, 4, 64, **bf), torch.zeros(N, 2, 64, **bf), torch.zeros(N, 2, 64, **bf)
+    ws = torch.zeros(16, dtype=torch.uint8)
+    with pytest.raises(ValueError, match="k has"):
+        splitkv.splitkv_attn_fwd(plan, q, k[:-1], v, 0.1, ws)
+    with pytest.raises(ValueError, match="q has"):
+        splitkv.splitkv_attn_fwd(plan, q[:, :3], k, v, 0.1, ws)
+    with pytest.raises(ValueError, match="CUDA"):            # sizes right: the device check speaks
+        splitkv.splitkv_attn_fwd(plan, q, k, v, 0.1, ws)
+    o, lse = torch.zeros(Nq, 4, 64), torch.zeros(Nq, 4)
+    kb = torch.zeros(Nq, 2, 64, **bf)
+    with pytest.raises(ValueError, match="lse has"):
+        splitkv.splitkv_merge(plan, q, kb, kb, 0.1, ws, o, lse[:-1])
+    with pytest.raises(ValueError, match="dvb has"):
+        splitkv.splitkv_attn_bwd(plan, q, k, v, kb, kb, o, lse, q, o, o.new_zeros(N, 2, 64), o.new_zeros(N, 2, 64),
+                                 o.new_zeros(Nq, 2, 64), o.new_zeros(Nq, 2, 65), 0.1, ws)
+    # the sizes follow the plan through an update
+    splitkv.splitkv_plan_update(plan, [300, 300], [10, 250, 400])
+    with pytest.raises(ValueError, match="k has"):
+        splitkv.splitkv_attn_fwd(plan, q, k, v, 0.1, ws)

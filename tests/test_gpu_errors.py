@@ -49,8 +49,9 @@ def test_unsupported_head_dim(splitkv):
     plan = skv.splitkv_plan(w.sample_lens, w.anchors, w.block_size, 2, 1, 96, w.kv_chunk, 148)
     plan.upload()
     ws = torch.empty(skv.splitkv_workspace_size(plan, skv.WS_FWD), dtype=torch.uint8, device="cuda")
-    x = torch.zeros(16, dtype=torch.bfloat16, device="cuda")
-    with pytest.raises(skv.SplitKVError) as ei:
-        skv.splitkv_attn_fwd(plan, x, x, x, 1.0, ws)
+    q = torch.zeros((w.num_queries, 2, 96), dtype=torch.bfloat16, device="cuda")
+    kv = torch.zeros((w.context_len, 1, 96), dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(skv.SplitKVError) as ei:            # right sizes: the library refuses d = 96
+        skv.splitkv_attn_fwd(plan, q, kv, kv, 1.0, ws)
     assert ei.value.status == -2
     torch.cuda.synchronize()
