@@ -398,8 +398,9 @@ def run_ours(args, world, rank, local):
     for k in kernels:
         b_, a_ = work[k]
         s_ = max(per_kernel[k] * 1e-3, 1e-9)
-        kern[k] = {"ms": per_kernel[k],
-                   ("tflops" if b_ == "tensor" else "gbs"): (a_ / s_ / 1e12 if b_ == "tensor" else a_ / s_ / 1e9)}
+        rate = a_ / s_ / 1e12 if b_ == "tensor" else a_ / s_ / 1e9
+        kern[k] = {"ms": per_kernel[k], ("tflops" if b_ == "tensor" else "gbs"): rate,
+                   "frac": rate / (peaks["bf16_tflops"] if b_ == "tensor" else peaks["hbm_gbs"])}
     fwd_ms = per_kernel["fwd_partial"] + per_kernel["merge"]
     bwd_ms = sum(per_kernel[k] for k in ("bwd_delta", "bwd_dkdv", "bwd_dq", "bwd_reduce"))
 
