@@ -240,7 +240,7 @@ def bench_config(args, w, W, Wb, world):
             "seed": args.seed if args.seed is not None else 1000 + w.config.index,
             "q_slice": args.q_slice, "partial_records": "bf16" if args.partial_bf16 else "f32",
             "lpt_cost": args.lpt_cost, "fwd_lpt_cost": args.fwd_lpt_cost,
-            "item_claims": "run-time" if args.dynamic_claim else "static",
+            "schedule": args.schedule, "item_claims": "run-time" if args.dynamic_claim else "static",
             "parallelism": "replicas" if world > 1 else "single",
             "l2": "no flush: each step touches ~4 GB (> 126 MB L2)"}
 
@@ -279,7 +279,7 @@ def run_ours(args, world, rank, local):
     plan = skv.splitkv_plan(w.sample_lens, w.anchors, w.block_size, Hq, w.num_kv_heads, d, w.kv_chunk, W,
                             num_bwd_workers=Wb, q_slice=args.q_slice, partial_bf16=args.partial_bf16,
                             tile_cost=args.lpt_cost == "tiles", fwd_tile_cost=args.fwd_lpt_cost == "tiles",
-                            dynamic_claim=args.dynamic_claim)
+                            dynamic_claim=args.dynamic_claim, contiguous_schedule=args.schedule == "contiguous")
     plan.upload(stream)
     st = plan.stats()
     if args.dump_plan and rank == 0:
@@ -577,7 +577,7 @@ def run_e2e(args, w, plan, dev, stream, flops_step, world=1):
                            num_workers=plan.problem.num_workers, num_bwd_workers=plan.problem.num_bwd_workers,
                            q_slice=plan.problem.q_slice, device=dev, partial_bf16=args.partial_bf16,
                            tile_cost=args.lpt_cost == "tiles", fwd_tile_cost=args.fwd_lpt_cost == "tiles",
-                           dynamic_claim=args.dynamic_claim)
+                           dynamic_claim=args.dynamic_claim, contiguous_schedule=args.schedule == "contiguous")
     dv = {n: torch.empty(x.shape, dtype=x.dtype, device=dev) for n, x in host.items()}
     outs_h = {"o": torch.empty((Nq, Hq, d), dtype=torch.float32).pin_memory(),
               "lse": torch.empty((Nq, Hq), dtype=torch.float32).pin_memory()}
@@ -735,6 +735,9 @@ def parse_args(argv=None):
     ap.add_argument("--dump-cta-times", default=None, metavar="PATH",
                     help="write the measured per-CTA busy times of the last step (fwd partial and dK/dV "
                          "kernels, ns) with the schedule options to PATH as JSON")
+    ap.add_argument("--schedule", choices=["lpt", "contiguous"], default="lpt",
+                    help="contiguous: the pages' unbalanced baseline (chunks in order, equal counts) on the "
+                         "kernels, static lists, to time what LPT saves")
     ap.add_argument("--dump-plan", default=None, metavar="PATH",
                     help="write the run's plan (problem, stats, every table) to PATH (.npz)")
     ap.add_argument("--emulate-ranks", type=int, default=0, metavar="R",
@@ -744,7 +747,7 @@ def parse_args(argv=None):
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
-    args.dynamic_claim = args.claims == "run-time"
+    args.dynamic_claim = args.claims == "run-time" and args.schedule == "lpt"
     return args
 
 

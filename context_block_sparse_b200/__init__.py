@@ -25,7 +25,8 @@ from ._abi import (  # noqa: F401
     DTYPE_BF16, DTYPE_F32, EXPORT_BWD_LOADS, EXPORT_BWD_SCHEDULE, EXPORT_CHUNK_PAIRS,
     EXPORT_BWD_LPT_ORDER, EXPORT_CHUNK_OWNER, EXPORT_CONTIG_LOADS, EXPORT_ENTRIES, EXPORT_FWD_LOADS,
     EXPORT_FWD_LPT_ORDER, EXPORT_QUERY_SHARD, MAX_RANKS,
-    EXPORT_FWD_SCHEDULE, FLAG_BLOCK_KEYS_IN_CONTEXT, FLAG_DYNAMIC_CLAIM, FLAG_EQUAL_COUNT, FLAG_FWD_TILE_COST,
+    EXPORT_FWD_SCHEDULE, FLAG_BLOCK_KEYS_IN_CONTEXT, FLAG_CONTIGUOUS_SCHEDULE, FLAG_DYNAMIC_CLAIM, FLAG_EQUAL_COUNT,
+    FLAG_FWD_TILE_COST,
     FLAG_PARTIAL_BF16, FLAG_TILE_COST,
     STATIC_SCRATCH_BYTES, WS_BWD, WS_FWD,
 )
@@ -161,7 +162,8 @@ class Plan:
 
 def _problem(sample_lens, anchors, block_size, num_q_heads, num_kv_heads, head_dim, kv_chunk,
              num_workers, num_bwd_workers, q_slice, equal_count, block_keys_in_context=False,
-             partial_bf16=False, tile_cost=False, fwd_tile_cost=False, dynamic_claim=False):
+             partial_bf16=False, tile_cost=False, fwd_tile_cost=False, dynamic_claim=False,
+             contiguous_schedule=False):
     lens = np.ascontiguousarray(sample_lens, dtype=np.int32)
     anc = np.ascontiguousarray(anchors, dtype=np.int32)
     p = _abi.Problem()
@@ -179,7 +181,8 @@ def _problem(sample_lens, anchors, block_size, num_q_heads, num_kv_heads, head_d
     p.q_slice = int(q_slice)
     p.flags = ((FLAG_EQUAL_COUNT if equal_count else 0) | (FLAG_BLOCK_KEYS_IN_CONTEXT if block_keys_in_context else 0)
                | (FLAG_PARTIAL_BF16 if partial_bf16 else 0) | (FLAG_TILE_COST if tile_cost else 0)
-               | (FLAG_FWD_TILE_COST if fwd_tile_cost else 0) | (FLAG_DYNAMIC_CLAIM if dynamic_claim else 0))
+               | (FLAG_FWD_TILE_COST if fwd_tile_cost else 0) | (FLAG_DYNAMIC_CLAIM if dynamic_claim else 0)
+               | (FLAG_CONTIGUOUS_SCHEDULE if contiguous_schedule else 0))
     return p, (lens, anc)
 
 
@@ -187,17 +190,19 @@ def splitkv_plan(sample_lens: Sequence[int], anchors: Sequence[int], block_size:
                  num_kv_heads: int, head_dim: int, kv_chunk: int, num_workers: int,
                  num_bwd_workers: int = 0, q_slice: int = 0, equal_count: bool = False,
                  block_keys_in_context: bool = False, partial_bf16: bool = False,
-                 tile_cost: bool = False, fwd_tile_cost: bool = False, dynamic_claim: bool = False) -> Plan:
+                 tile_cost: bool = False, fwd_tile_cost: bool = False, dynamic_claim: bool = False,
+                 contiguous_schedule: bool = False) -> Plan:
     """Host-side mask metadata + LPT schedules (no CUDA call).  block_keys_in_context
     selects reading B of the block keys (SPLITKV_FLAG_BLOCK_KEYS_IN_CONTEXT);
     partial_bf16 stores the partial records as bf16 (SPLITKV_FLAG_PARTIAL_BF16);
     tile_cost / fwd_tile_cost cost the backward / forward LPT items by the executed
     tile work of their kernels (SPLITKV_FLAG_TILE_COST / SPLITKV_FLAG_FWD_TILE_COST);
     dynamic_claim lets the CTAs claim the items in LPT order at run time
-    (SPLITKV_FLAG_DYNAMIC_CLAIM)."""
+    (SPLITKV_FLAG_DYNAMIC_CLAIM); contiguous_schedule replaces LPT by the contiguous
+    baseline schedule (SPLITKV_FLAG_CONTIGUOUS_SCHEDULE)."""
     p, keep = _problem(sample_lens, anchors, block_size, num_q_heads, num_kv_heads, head_dim, kv_chunk,
                        num_workers, num_bwd_workers, q_slice, equal_count, block_keys_in_context, partial_bf16,
-                       tile_cost, fwd_tile_cost, dynamic_claim)
+                       tile_cost, fwd_tile_cost, dynamic_claim, contiguous_schedule)
     h = ctypes.c_void_p()
     _check("splitkv_plan", _lib.splitkv_plan(ctypes.byref(p), ctypes.byref(h)))
     return Plan(h, p, keep)
@@ -228,7 +233,8 @@ def splitkv_plan_update(plan: Plan, sample_lens, anchors, **kw) -> Plan:
                 partial_bf16=bool(old.flags & FLAG_PARTIAL_BF16),
                 tile_cost=bool(old.flags & FLAG_TILE_COST),
                 fwd_tile_cost=bool(old.flags & FLAG_FWD_TILE_COST),
-                dynamic_claim=bool(old.flags & FLAG_DYNAMIC_CLAIM))
+                dynamic_claim=bool(old.flags & FLAG_DYNAMIC_CLAIM),
+                contiguous_schedule=bool(old.flags & FLAG_CONTIGUOUS_SCHEDULE))
     args.update(kw)
     p, keep = _problem(sample_lens, anchors, **args)
     _check("splitkv_plan_update", _lib.splitkv_plan_update(plan.handle, ctypes.byref(p)))

@@ -26,6 +26,7 @@ FLAG_PARTIAL_BF16 = 4
 FLAG_TILE_COST = 8
 FLAG_FWD_TILE_COST = 16
 FLAG_DYNAMIC_CLAIM = 32
+FLAG_CONTIGUOUS_SCHEDULE = 64
 
 STATIC_SCRATCH_BYTES = 16 << 20
 

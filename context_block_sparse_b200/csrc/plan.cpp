@@ -81,7 +81,11 @@ int validate(const splitkv_problem* p) {
     return SPLITKV_ERR_INVALID_ARG;
   if (p->num_q_heads % p->num_kv_heads) return SPLITKV_ERR_INVALID_ARG;
   if (p->flags & ~uint32_t(SPLITKV_FLAG_EQUAL_COUNT | SPLITKV_FLAG_BLOCK_KEYS_IN_CONTEXT | SPLITKV_FLAG_PARTIAL_BF16 |
-                           SPLITKV_FLAG_TILE_COST | SPLITKV_FLAG_FWD_TILE_COST | SPLITKV_FLAG_DYNAMIC_CLAIM))
+                           SPLITKV_FLAG_TILE_COST | SPLITKV_FLAG_FWD_TILE_COST | SPLITKV_FLAG_DYNAMIC_CLAIM |
+                           SPLITKV_FLAG_CONTIGUOUS_SCHEDULE))
+    return SPLITKV_ERR_INVALID_ARG;
+  if ((p->flags & SPLITKV_FLAG_CONTIGUOUS_SCHEDULE) &&
+      (p->flags & (SPLITKV_FLAG_EQUAL_COUNT | SPLITKV_FLAG_DYNAMIC_CLAIM)))
     return SPLITKV_ERR_INVALID_ARG;
   int64_t N = 0;
   for (int s = 0; s < p->num_samples; ++s) {
@@ -150,6 +154,25 @@ void sort_by_cost_desc(const std::vector<Item>& items, std::vector<int32_t>& out
     a.swap(b);
   }
   out.swap(a);
+}
+
+// The contiguous ("unbalanced") schedule: items in their (chunk, head, slice) order,
+// item i of n to worker floor(i W / n); `order` lists them worker by worker (which is
+// item order), and `sorted` receives the same order.
+void contiguous_schedule(const std::vector<Item>& items, int W, std::vector<int32_t>& worker_ptr,
+                         std::vector<int32_t>& order, std::vector<uint64_t>& loads, std::vector<int32_t>& sorted) {
+  const int64_t n = int64_t(items.size());
+  loads.assign(size_t(W), 0);
+  worker_ptr.assign(size_t(W) + 1, 0);
+  order.resize(size_t(n));
+  for (int64_t i = 0; i < n; ++i) {
+    const int64_t w = (i * W) / n;
+    loads[size_t(w)] += items[size_t(i)].cost;
+    worker_ptr[size_t(w) + 1]++;
+    order[size_t(i)] = int32_t(i);
+  }
+  for (int w = 0; w < W; ++w) worker_ptr[size_t(w) + 1] += worker_ptr[size_t(w)];
+  sorted = order;
 }
 
 void lpt_schedule(const std::vector<Item>& items, int W, bool equal_count,
@@ -453,8 +476,13 @@ int build(splitkv_plan_t* P, const splitkv_problem* p) {
   nonzero(P->fwd_items);
   nonzero(P->bwd_items);
   const bool eq = (P->flags & SPLITKV_FLAG_EQUAL_COUNT) != 0;
-  lpt_schedule(P->fwd_items, P->W, eq, P->fwd_worker_ptr, P->fwd_order, P->fwd_loads, P->fwd_lpt);
-  lpt_schedule(P->bwd_items, P->Wb, eq, P->bwd_worker_ptr, P->bwd_order, P->bwd_loads, P->bwd_lpt);
+  if (P->flags & SPLITKV_FLAG_CONTIGUOUS_SCHEDULE) {
+    contiguous_schedule(P->fwd_items, P->W, P->fwd_worker_ptr, P->fwd_order, P->fwd_loads, P->fwd_lpt);
+    contiguous_schedule(P->bwd_items, P->Wb, P->bwd_worker_ptr, P->bwd_order, P->bwd_loads, P->bwd_lpt);
+  } else {
+    lpt_schedule(P->fwd_items, P->W, eq, P->fwd_worker_ptr, P->fwd_order, P->fwd_loads, P->fwd_lpt);
+    lpt_schedule(P->bwd_items, P->Wb, eq, P->bwd_worker_ptr, P->bwd_order, P->bwd_loads, P->bwd_lpt);
+  }
 
   // contiguous ("unbalanced") baseline: the num_chunks * Hkv (chunk, head) items in
   // order, item i to worker floor(i W / n), zero-cost items included

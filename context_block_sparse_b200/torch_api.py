@@ -25,19 +25,20 @@ class SplitKVAttention:
                  num_bwd_workers: int = 0, q_slice: int = 0, equal_count: bool = False,
                  device: Optional[torch.device] = None, block_keys_in_context: bool = False,
                  partial_bf16: bool = False, tile_cost: bool = False, fwd_tile_cost: bool = False,
-                 dynamic_claim: bool = False):
+                 dynamic_claim: bool = False, contiguous_schedule: bool = False):
         """block_keys_in_context: reading B of the block keys (the block's own tokens are
         the context positions after its anchor); kb, vb are then unused (pass None)
         and backward() returns no dkb, dvb.  partial_bf16: bf16 partial records.
         tile_cost / fwd_tile_cost: backward / forward LPT items costed by executed tile work.
-        dynamic_claim: the CTAs claim the items in LPT order at run time."""
+        dynamic_claim: the CTAs claim the items in LPT order at run time.
+        contiguous_schedule: the contiguous baseline schedule instead of LPT."""
         self.device = torch.device("cuda") if device is None else torch.device(device)
         if num_workers is None:
             num_workers = torch.cuda.get_device_properties(self.device).multi_processor_count
         self.plan: Plan = splitkv_plan(sample_lens, anchors, block_size, num_q_heads, num_kv_heads, head_dim,
                                        kv_chunk, num_workers, num_bwd_workers, q_slice, equal_count,
                                        block_keys_in_context, partial_bf16, tile_cost, fwd_tile_cost,
-                                       dynamic_claim)
+                                       dynamic_claim, contiguous_schedule)
         self.block_keys_in_context = bool(block_keys_in_context)
         splitkv_plan_upload(self.plan)
         self.block_size = block_size

@@ -119,6 +119,14 @@ extern "C" {
  * of other plans return SPLITKV_ERR_UNSUPPORTED.  Launches of one kernel on one
  * plan must not overlap (they share its cursor). */
 #define SPLITKV_FLAG_DYNAMIC_CLAIM  32u
+/* Contiguous schedules instead of LPT (the "unbalanced" baseline of the news page,
+ * "Balance actual attention work", run on the kernels): each schedule keeps its
+ * non-zero-cost items in (chunk, KV head, slice) order and gives item i of n to
+ * worker floor(i W / n), whatever their costs.  Results are unchanged; the point is
+ * to time what LPT saves.  Not combinable with SPLITKV_FLAG_EQUAL_COUNT or
+ * SPLITKV_FLAG_DYNAMIC_CLAIM (INVALID_ARG).  The LPT-order exports then hold the
+ * items in schedule order. */
+#define SPLITKV_FLAG_CONTIGUOUS_SCHEDULE  64u
 
 /* ---- dtype codes (o) ------------------------------------------------------- */
 #define SPLITKV_DTYPE_F32   0

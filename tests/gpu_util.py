@@ -27,7 +27,7 @@ def small(name="tiny", lens=(700, 1100, 333), anchors=24, Hq=8, Hkv=2, d=128, bs
 
 
 def run(w, bwd=False, o_dtype="f32", W=148, Wb=0, q_slice=0, equal_count=False, repeat=1, rb=False,
-        partial_bf16=False, tile_cost=False, dynamic_claim=False):
+        partial_bf16=False, tile_cost=False, dynamic_claim=False, contiguous_schedule=False):
     """Run plan/fwd/merge (and bwd) on cuda:0; returns numpy outputs (+ the attention object).
     rb: reading B of the block keys (kb, vb not passed; no dkb, dvb)."""
     import torch
@@ -35,7 +35,7 @@ def run(w, bwd=False, o_dtype="f32", W=148, Wb=0, q_slice=0, equal_count=False, 
     att = SplitKVAttention(w.sample_lens, w.anchors, w.block_size, w.num_q_heads, w.num_kv_heads, w.head_dim,
                            w.kv_chunk, num_workers=W, num_bwd_workers=Wb, q_slice=q_slice,
                            equal_count=equal_count, block_keys_in_context=rb, partial_bf16=partial_bf16,
-                           tile_cost=tile_cost, dynamic_claim=dynamic_claim)
+                           tile_cost=tile_cost, dynamic_claim=dynamic_claim, contiguous_schedule=contiguous_schedule)
     t = {n: to_dev(b) for n, b in w.bits.items()}
     kb, vb = (None, None) if rb else (t["kb"], t["vb"])
     odt = torch.float32 if o_dtype == "f32" else torch.bfloat16

@@ -71,6 +71,7 @@ def test_small_ragged_fwd_bwd_elementwise(splitkv, case):
     dict(o_dtype="bf16"), dict(q_slice=2, tile_cost=True), dict(tile_cost=True, Wb=5),
     dict(dynamic_claim=True), dict(dynamic_claim=True, W=7, Wb=3, q_slice=1), dict(dynamic_claim=True, W=300),
     dict(dynamic_claim=True, W=1, Wb=1, q_slice=2, partial_bf16=True),
+    dict(contiguous_schedule=True, q_slice=2, W=37), dict(contiguous_schedule=True, tile_cost=True, Wb=5),
 ])
 def test_schedules_and_options_same_result(splitkv, opts):
     w = small()

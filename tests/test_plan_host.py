@@ -212,10 +212,12 @@ def test_dynamic_claim_keeps_the_static_plan(splitkv):
 
 
 def test_unknown_flag_bits_rejected(splitkv):
-    """Flags outside SPLITKV_FLAG_* (1, 2, 4, 8, 16, 32) are an invalid argument; each known bit alone is accepted."""
+    """Flags outside SPLITKV_FLAG_* (1, 2, ..., 64) are an invalid argument; each known bit alone is
+    accepted; the contiguous schedule (64) refuses the LPT-only bits 1 and 32."""
     import ctypes
     lib = splitkv._lib
-    for flags, want in [(1, 0), (2, 0), (4, 0), (8, 0), (16, 0), (32, 0), (63, 0), (64, -1), (1 << 31, -1)]:
+    for flags, want in [(1, 0), (2, 0), (4, 0), (8, 0), (16, 0), (32, 0), (63, 0), (64, 0), (64 | 30, 0),
+                        (64 | 1, -1), (64 | 32, -1), (128, -1), (1 << 31, -1)]:
         p, keep = splitkv._problem([64, 64], [10, 70], 16, 2, 1, 128, 32, 4, 0, 0, False)
         p.flags = flags
         h = ctypes.c_void_p()
@@ -271,3 +273,40 @@ def test_costs_above_32_bits_bit_exact(splitkv):
     assert max(omask.chunk_pairs(lens, anchors, 16, C)) * 8 > (1 << 32)
     _check_against_oracle(splitkv, lens, anchors, 16, 8, 1, C, 3, q_slice=1)
     _check_against_oracle(splitkv, lens, anchors, 16, 8, 1, C, 2, eq=True)
+
+
+@pytest.mark.parametrize("seed", range(12))
+def test_contiguous_schedule_bit_exact(splitkv, seed):
+    """SPLITKV_FLAG_CONTIGUOUS_SCHEDULE: the non-zero-cost items of each schedule in (chunk,
+    head, slice) order, item i of n to worker floor(i W / n) -- the oracle's contiguous
+    assignment over the same items."""
+    rng = np.random.default_rng(300 + seed)
+    lens = [int(x) for x in rng.integers(50, 900, size=int(rng.integers(1, 5)))]
+    anchors = [int(x) for x in rng.integers(0, sum(lens), size=int(rng.integers(1, 40)))]
+    Hq, Hkv = [(4, 1), (8, 2), (2, 2)][seed % 3]
+    bs, C = [4, 8, 16][seed % 3], int(rng.integers(16, 300))
+    W, Wb, qs = int(rng.integers(1, 40)), int(rng.integers(1, 40)), seed % 3
+    tc = bool(seed % 2)
+    plan = splitkv.splitkv_plan(lens, anchors, bs, Hq, Hkv, 64, C, W, num_bwd_workers=Wb, q_slice=qs,
+                                tile_cost=tc, contiguous_schedule=True)
+    for what, loads_what, order_what, workers, q_slice, mode in (
+            (splitkv.EXPORT_FWD_SCHEDULE, splitkv.EXPORT_FWD_LOADS, splitkv.EXPORT_FWD_LPT_ORDER, W, qs, False),
+            (splitkv.EXPORT_BWD_SCHEDULE, splitkv.EXPORT_BWD_LOADS, splitkv.EXPORT_BWD_LPT_ORDER, Wb, 0, tc)):
+        live = [it for it in olpt.work_items(lens, anchors, bs, C, Hq, Hkv, q_slice=q_slice, tile_cost=mode)
+                if it[1] > 0]
+        lists, loads = olpt.contiguous(live, workers)
+        got = [[] for _ in range(workers)]
+        for w_, c, g, s, _ in plan.export(what).reshape(-1, 5).tolist():
+            got[w_].append((c, g, s))
+        assert got == [list(l) for l in lists]
+        assert plan.export(loads_what).tolist() == loads
+        order = [((c, g, s), cst) for c, g, s, cst in plan.export(order_what).reshape(-1, 4).tolist()]
+        assert order == sorted(live)
+    plan.destroy()
+
+
+@pytest.mark.parametrize("other", ["equal_count", "dynamic_claim"])
+def test_contiguous_schedule_refuses_lpt_options(splitkv, other):
+    with pytest.raises(splitkv.SplitKVError) as ei:
+        splitkv.splitkv_plan([500], [100, 300], 4, 2, 1, 64, 64, 8, contiguous_schedule=True, **{other: True})
+    assert ei.value.status == -1
