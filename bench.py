@@ -369,6 +369,7 @@ def run_ours(args, world, rank, local):
             json.dump({"workload": args.workload, "anchors": int(w.anchors.size), "q_slice": args.q_slice,
                        "lpt_cost": args.lpt_cost, "fwd_lpt_cost": args.fwd_lpt_cost,
                        "dynamic_claim": bool(args.dynamic_claim), "partial_bf16": bool(args.partial_bf16),
+                       "schedule": args.schedule,
                        "fwd_workers": W, "bwd_workers": Wb,
                        "fwd_ns": [int(x) for x in cta_f], "bwd_ns": [int(x) for x in cta_b]}, f)
 
