@@ -16,6 +16,8 @@ Readings where the pages are silent:
   eligible rank of least load, ties to the lowest rank; with n = q R + r chunks
   a rank is eligible while it holds fewer than q, or q while fewer than r ranks
   hold q + 1;
+* the "unbalanced" baseline the pages compare against keeps chunks in order: chunk c
+  to rank floor(c R / n);
 * query side: blocks are split into R contiguous ranges, rank r owning
   [floor(r A / R), floor((r + 1) A / R)); the owner of a block holds its draft
   keys/values (kb, vb) and adds the in-block term;
@@ -62,6 +64,12 @@ def chunk_owners(sample_lens, anchors, block_size: int, kv_chunk: int, num_q_hea
         counts[best] += 1
         owner[c] = best
     return owner
+
+
+def chunk_owners_contiguous(num_chunks: int, num_ranks: int) -> List[int]:
+    """The "unbalanced" device baseline ([news] "Balance actual attention work"): chunks left
+    in order, chunk c to rank floor(c R / n) -- equal counts, whatever their costs."""
+    return [(c * int(num_ranks)) // int(num_chunks) for c in range(int(num_chunks))]
 
 
 def query_shard(num_blocks: int, num_ranks: int, rank: int) -> Tuple[int, int]:

@@ -236,3 +236,31 @@ def test_planted_combine_mistakes_are_caught():
     # a combine that lets one rank's row win outright (max instead of softmax weights)
     pick = np.take_along_axis(Op, Lp.argmax(axis=0)[None, :, :, None], axis=0)[0]
     assert np.abs(pick - Ou).max() > 1e-3
+
+
+def test_contiguous_ownership_hand_worked():
+    assert cp.chunk_owners_contiguous(4, 2) == [0, 0, 1, 1]
+    assert cp.chunk_owners_contiguous(5, 2) == [0, 0, 0, 1, 1]
+    assert cp.chunk_owners_contiguous(7, 3) == [0, 0, 0, 1, 1, 2, 2]
+    assert cp.chunk_owners_contiguous(2, 4) == [0, 2]
+    for n, R in ((13, 4), (100, 8), (8, 8)):
+        own = cp.chunk_owners_contiguous(n, R)
+        assert own == sorted(own)                              # in order
+        q, r = divmod(n, R)
+        assert sorted(own.count(w) for w in range(R)) == sorted([q + 1] * r + [q] * (R - r))
+
+
+def test_lpt_ownership_beats_contiguous_on_a_skewed_context():
+    """All anchors late in a first sample of 2000 tokens, none in the second of 6000: the
+    first 8 of 32 chunks carry every pair.  Left in order they all land on rank 0, which
+    then holds the whole load; LPT spreads them (the pages' point)."""
+    lens = [2000, 6000]
+    anchors = list(range(1900, 2000, 5))
+    C, R = 250, 4
+    pairs = [4 * p for p in mask.chunk_pairs(lens, anchors, 4, C)]
+    n = len(pairs)
+    loads = lambda own: [sum(pairs[c] for c in range(n) if own[c] == w) for w in range(R)]
+    lpt_own = cp.chunk_owners(lens, anchors, 4, C, 4, R)
+    con_own = cp.chunk_owners_contiguous(n, R)
+    assert max(loads(con_own)) == sum(pairs)
+    assert max(loads(con_own)) > 3 * max(loads(lpt_own))
