@@ -438,8 +438,12 @@ def run_ours(args, world, rank, local):
     if rank == 0:
         result["device_lpt"] = device_lpt_report(skv, w)
     if rank == 0 and world == 1 and args.emulate_ranks > 1:
-        result["split_kv_ranks"] = rank_emulation_report(skv, w, args, args.emulate_ranks, dev, stream, t, W, Wb,
-                                                          peaks)
+        lpt = rank_emulation_report(skv, w, args, args.emulate_ranks, dev, stream, t, W, Wb, peaks)
+        con = rank_emulation_report(skv, w, args, args.emulate_ranks, dev, stream, t, W, Wb, peaks,
+                                    contiguous=True)
+        step = lambda r: max(f + b for f, b in zip(r["fwd_ms"], r["bwd_ms"]))   # noqa: E731
+        result["split_kv_ranks"] = {"lpt_ownership": lpt, "contiguous_ownership": con,
+                                    "step_ms_contiguous_over_lpt": step(con) / step(lpt)}
     if not args.no_e2e:
         result["e2e"] = run_e2e(args, w, plan, dev, stream, flops_step, world=world)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -472,19 +476,20 @@ def device_lpt_report(skv, w, workers=(8, 16, 32, 64)):
     return out
 
 
-def rank_emulation_report(skv, w, args, R, dev, stream, t, W, Wb, peaks, reps=5):
+def rank_emulation_report(skv, w, args, R, dev, stream, t, W, Wb, peaks, reps=5, contiguous=False):
     """Split-KV over R ranks with one GPU standing in for each rank in turn (after the timed
     region, untimed by the bench line): per rank, the device time of its forward
     (splitkv_attn_fwd + splitkv_merge) and backward (splitkv_attn_bwd) on its rank plan, the
     median of `reps`; the measured rank imbalance (max / mean - 1 of forward + backward)
     against the planned one (the ranks' summed chunk costs, news page "Balance actual
     attention work"); and the combine / sum kernels of the exchange against the HBM peak.
-    The collectives themselves are not timed (one GPU)."""
+    The collectives themselves are not timed (one GPU).  contiguous: chunks owned in order
+    (the pages' unbalanced device baseline) instead of by LPT."""
     import torch
     f32 = dict(dtype=torch.float32, device=dev)
     d, Hq, Hkv, Nq, N = w.head_dim, w.num_q_heads, w.num_kv_heads, w.num_queries, w.context_len
     kw = dict(num_bwd_workers=Wb, q_slice=args.q_slice, partial_bf16=args.partial_bf16,
-              tile_cost=args.lpt_cost == "tiles", dynamic_claim=args.dynamic_claim)
+              tile_cost=args.lpt_cost == "tiles", dynamic_claim=args.dynamic_claim, contiguous_ranks=contiguous)
     args_p = (w.sample_lens, w.anchors, w.block_size, Hq, Hkv, d, w.kv_chunk, W)
     o_parts = torch.empty((R, Nq, Hq, d), **f32)
     lse_parts = torch.empty((R, Nq, Hq), **f32)

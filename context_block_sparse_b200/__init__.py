@@ -25,7 +25,8 @@ from ._abi import (  # noqa: F401
     DTYPE_BF16, DTYPE_F32, EXPORT_BWD_LOADS, EXPORT_BWD_SCHEDULE, EXPORT_CHUNK_PAIRS,
     EXPORT_BWD_LPT_ORDER, EXPORT_CHUNK_OWNER, EXPORT_CONTIG_LOADS, EXPORT_ENTRIES, EXPORT_FWD_LOADS,
     EXPORT_FWD_LPT_ORDER, EXPORT_QUERY_SHARD, MAX_RANKS,
-    EXPORT_FWD_SCHEDULE, FLAG_BLOCK_KEYS_IN_CONTEXT, FLAG_CONTIGUOUS_SCHEDULE, FLAG_DYNAMIC_CLAIM, FLAG_EQUAL_COUNT,
+    EXPORT_FWD_SCHEDULE, FLAG_BLOCK_KEYS_IN_CONTEXT, FLAG_CONTIGUOUS_RANKS, FLAG_CONTIGUOUS_SCHEDULE,
+    FLAG_DYNAMIC_CLAIM, FLAG_EQUAL_COUNT,
     FLAG_FWD_TILE_COST,
     FLAG_PARTIAL_BF16, FLAG_TILE_COST,
     STATIC_SCRATCH_BYTES, WS_BWD, WS_FWD,
@@ -163,7 +164,7 @@ class Plan:
 def _problem(sample_lens, anchors, block_size, num_q_heads, num_kv_heads, head_dim, kv_chunk,
              num_workers, num_bwd_workers, q_slice, equal_count, block_keys_in_context=False,
              partial_bf16=False, tile_cost=False, fwd_tile_cost=False, dynamic_claim=False,
-             contiguous_schedule=False):
+             contiguous_schedule=False, contiguous_ranks=False):
     lens = np.ascontiguousarray(sample_lens, dtype=np.int32)
     anc = np.ascontiguousarray(anchors, dtype=np.int32)
     p = _abi.Problem()
@@ -182,7 +183,8 @@ def _problem(sample_lens, anchors, block_size, num_q_heads, num_kv_heads, head_d
     p.flags = ((FLAG_EQUAL_COUNT if equal_count else 0) | (FLAG_BLOCK_KEYS_IN_CONTEXT if block_keys_in_context else 0)
                | (FLAG_PARTIAL_BF16 if partial_bf16 else 0) | (FLAG_TILE_COST if tile_cost else 0)
                | (FLAG_FWD_TILE_COST if fwd_tile_cost else 0) | (FLAG_DYNAMIC_CLAIM if dynamic_claim else 0)
-               | (FLAG_CONTIGUOUS_SCHEDULE if contiguous_schedule else 0))
+               | (FLAG_CONTIGUOUS_SCHEDULE if contiguous_schedule else 0)
+               | (FLAG_CONTIGUOUS_RANKS if contiguous_ranks else 0))
     return p, (lens, anc)
 
 
@@ -191,7 +193,7 @@ def splitkv_plan(sample_lens: Sequence[int], anchors: Sequence[int], block_size:
                  num_bwd_workers: int = 0, q_slice: int = 0, equal_count: bool = False,
                  block_keys_in_context: bool = False, partial_bf16: bool = False,
                  tile_cost: bool = False, fwd_tile_cost: bool = False, dynamic_claim: bool = False,
-                 contiguous_schedule: bool = False) -> Plan:
+                 contiguous_schedule: bool = False, contiguous_ranks: bool = False) -> Plan:
     """Host-side mask metadata + LPT schedules (no CUDA call).  block_keys_in_context
     selects reading B of the block keys (SPLITKV_FLAG_BLOCK_KEYS_IN_CONTEXT);
     partial_bf16 stores the partial records as bf16 (SPLITKV_FLAG_PARTIAL_BF16);
@@ -199,10 +201,11 @@ def splitkv_plan(sample_lens: Sequence[int], anchors: Sequence[int], block_size:
     tile work of their kernels (SPLITKV_FLAG_TILE_COST / SPLITKV_FLAG_FWD_TILE_COST);
     dynamic_claim lets the CTAs claim the items in LPT order at run time
     (SPLITKV_FLAG_DYNAMIC_CLAIM); contiguous_schedule replaces LPT by the contiguous
-    baseline schedule (SPLITKV_FLAG_CONTIGUOUS_SCHEDULE)."""
+    baseline schedule (SPLITKV_FLAG_CONTIGUOUS_SCHEDULE); contiguous_ranks only matters to rank
+    plans (SPLITKV_FLAG_CONTIGUOUS_RANKS)."""
     p, keep = _problem(sample_lens, anchors, block_size, num_q_heads, num_kv_heads, head_dim, kv_chunk,
                        num_workers, num_bwd_workers, q_slice, equal_count, block_keys_in_context, partial_bf16,
-                       tile_cost, fwd_tile_cost, dynamic_claim, contiguous_schedule)
+                       tile_cost, fwd_tile_cost, dynamic_claim, contiguous_schedule, contiguous_ranks)
     h = ctypes.c_void_p()
     _check("splitkv_plan", _lib.splitkv_plan(ctypes.byref(p), ctypes.byref(h)))
     return Plan(h, p, keep)
@@ -213,7 +216,7 @@ def splitkv_plan_shard(sample_lens: Sequence[int], anchors: Sequence[int], block
                        rank: int, **kw) -> Plan:
     """Rank `rank`'s plan of Split-KV over `num_ranks` ranks (splitkv_plan_shard): the
     chunks it owns and the in-block term of its block range; other options as
-    splitkv_plan."""
+    splitkv_plan, plus contiguous_ranks (chunks owned in order, the unbalanced baseline)."""
     p, keep = _problem(sample_lens, anchors, block_size, num_q_heads, num_kv_heads, head_dim, kv_chunk,
                        num_workers, kw.pop("num_bwd_workers", 0), kw.pop("q_slice", 0),
                        kw.pop("equal_count", False), **kw)
@@ -234,7 +237,8 @@ def splitkv_plan_update(plan: Plan, sample_lens, anchors, **kw) -> Plan:
                 tile_cost=bool(old.flags & FLAG_TILE_COST),
                 fwd_tile_cost=bool(old.flags & FLAG_FWD_TILE_COST),
                 dynamic_claim=bool(old.flags & FLAG_DYNAMIC_CLAIM),
-                contiguous_schedule=bool(old.flags & FLAG_CONTIGUOUS_SCHEDULE))
+                contiguous_schedule=bool(old.flags & FLAG_CONTIGUOUS_SCHEDULE),
+                contiguous_ranks=bool(old.flags & FLAG_CONTIGUOUS_RANKS))
     args.update(kw)
     p, keep = _problem(sample_lens, anchors, **args)
     _check("splitkv_plan_update", _lib.splitkv_plan_update(plan.handle, ctypes.byref(p)))

@@ -27,6 +27,7 @@ FLAG_TILE_COST = 8
 FLAG_FWD_TILE_COST = 16
 FLAG_DYNAMIC_CLAIM = 32
 FLAG_CONTIGUOUS_SCHEDULE = 64
+FLAG_CONTIGUOUS_RANKS = 128
 
 STATIC_SCRATCH_BYTES = 16 << 20
 

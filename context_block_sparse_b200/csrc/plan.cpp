@@ -82,7 +82,7 @@ int validate(const splitkv_problem* p) {
   if (p->num_q_heads % p->num_kv_heads) return SPLITKV_ERR_INVALID_ARG;
   if (p->flags & ~uint32_t(SPLITKV_FLAG_EQUAL_COUNT | SPLITKV_FLAG_BLOCK_KEYS_IN_CONTEXT | SPLITKV_FLAG_PARTIAL_BF16 |
                            SPLITKV_FLAG_TILE_COST | SPLITKV_FLAG_FWD_TILE_COST | SPLITKV_FLAG_DYNAMIC_CLAIM |
-                           SPLITKV_FLAG_CONTIGUOUS_SCHEDULE))
+                           SPLITKV_FLAG_CONTIGUOUS_SCHEDULE | SPLITKV_FLAG_CONTIGUOUS_RANKS))
     return SPLITKV_ERR_INVALID_ARG;
   if ((p->flags & SPLITKV_FLAG_CONTIGUOUS_SCHEDULE) &&
       (p->flags & (SPLITKV_FLAG_EQUAL_COUNT | SPLITKV_FLAG_DYNAMIC_CLAIM)))
@@ -346,12 +346,16 @@ int build(splitkv_plan_t* P, const splitkv_problem* p) {
 
   // ranks: whole chunks to ranks by LPT with equal counts (the pages' device rule), every
   // chunk an item -- zero-cost ones too, since its keys live somewhere -- of cost
-  // Hq * pairs_c; then keep this rank's entries (their pairs are the rank's work) and
-  // the in-block term of its contiguous block range [floor(r A / R), floor((r + 1) A / R))
+  // Hq * pairs_c (or, under SPLITKV_FLAG_CONTIGUOUS_RANKS, chunk c to rank floor(c R / n));
+  // then keep this rank's entries (their pairs are the rank's work) and the in-block
+  // term of its contiguous block range [floor(r A / R), floor((r + 1) A / R))
   P->chunk_owner.assign(size_t(P->num_chunks), 0);
   P->bt_lo = int32_t(int64_t(P->rank) * P->A / P->R);
   P->bt_hi = int32_t(int64_t(P->rank + 1) * P->A / P->R);
-  if (P->R > 1) {
+  if (P->R > 1 && (P->flags & SPLITKV_FLAG_CONTIGUOUS_RANKS)) {
+    for (int c = 0; c < P->num_chunks; ++c)
+      P->chunk_owner[size_t(c)] = int32_t((int64_t(c) * P->R) / P->num_chunks);
+  } else if (P->R > 1) {
     std::vector<Item> chunk_items(size_t(P->num_chunks));
     for (int c = 0; c < P->num_chunks; ++c)
       chunk_items[size_t(c)] = Item{c, 0, 0, 0, 0, P->chunk_pairs[size_t(c)] * uint64_t(P->Hq)};
@@ -361,6 +365,8 @@ int build(splitkv_plan_t* P, const splitkv_problem* p) {
     for (int r = 0; r < P->R; ++r)
       for (int k = rank_ptr[size_t(r)]; k < rank_ptr[size_t(r) + 1]; ++k)
         P->chunk_owner[size_t(chunk_items[size_t(rank_order[size_t(k)])].c)] = r;
+  }
+  if (P->R > 1) {
     std::vector<I4> kept;
     std::vector<int32_t> kept_ptr(size_t(P->num_chunks) + 1, 0);
     for (int c = 0; c < P->num_chunks; ++c) {

@@ -127,6 +127,11 @@ extern "C" {
  * SPLITKV_FLAG_DYNAMIC_CLAIM (INVALID_ARG).  The LPT-order exports then hold the
  * items in schedule order. */
 #define SPLITKV_FLAG_CONTIGUOUS_SCHEDULE  64u
+/* Rank plans (splitkv_plan_shard) only: chunks owned by ranks in order -- chunk c of n
+ * to rank floor(c R / n) -- instead of by LPT (the news page's "unbalanced" device
+ * baseline), to time what LPT ownership saves.  The CTA schedules inside a rank are
+ * unaffected. */
+#define SPLITKV_FLAG_CONTIGUOUS_RANKS  128u
 
 /* ---- dtype codes (o) ------------------------------------------------------- */
 #define SPLITKV_DTYPE_F32   0

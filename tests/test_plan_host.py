@@ -212,12 +212,12 @@ def test_dynamic_claim_keeps_the_static_plan(splitkv):
 
 
 def test_unknown_flag_bits_rejected(splitkv):
-    """Flags outside SPLITKV_FLAG_* (1, 2, ..., 64) are an invalid argument; each known bit alone is
-    accepted; the contiguous schedule (64) refuses the LPT-only bits 1 and 32."""
+    """Flags outside SPLITKV_FLAG_* (1, 2, ..., 128) are an invalid argument; each known bit alone
+    is accepted; the contiguous schedule (64) refuses the LPT-only bits 1 and 32."""
     import ctypes
     lib = splitkv._lib
     for flags, want in [(1, 0), (2, 0), (4, 0), (8, 0), (16, 0), (32, 0), (63, 0), (64, 0), (64 | 30, 0),
-                        (64 | 1, -1), (64 | 32, -1), (128, -1), (1 << 31, -1)]:
+                        (64 | 1, -1), (64 | 32, -1), (128, 0), (255 & ~33, 0), (256, -1), (1 << 31, -1)]:
         p, keep = splitkv._problem([64, 64], [10, 70], 16, 2, 1, 128, 32, 4, 0, 0, False)
         p.flags = flags
         h = ctypes.c_void_p()

@@ -138,3 +138,27 @@ def test_rank_workspaces_add_up(splitkv):
     full = splitkv.splitkv_plan(*args).stats()["num_entries"]
     parts = [splitkv.splitkv_plan_shard(*args, 4, r).stats()["num_entries"] for r in range(4)]
     assert sum(parts) == full and max(parts) < full
+
+
+@pytest.mark.parametrize("R", [2, 3, 5])
+def test_contiguous_rank_ownership_bit_exact(splitkv, R):
+    """SPLITKV_FLAG_CONTIGUOUS_RANKS: chunk c to rank floor(c R / n), the rest of each rank
+    plan as with LPT ownership."""
+    w = make_workload("drafter", seed=1001, with_grad=False)
+    args = (w.sample_lens, w.anchors, w.block_size, w.num_q_heads, w.num_kv_heads, 64, w.kv_chunk, 148)
+    n = omask.num_chunks(w.context_len, w.kv_chunk)
+    owner = ocp.chunk_owners_contiguous(n, R)
+    full_entries = omask.chunk_entries(w.sample_lens, w.anchors, w.kv_chunk, w.block_size)
+    union = []
+    for r in range(R):
+        p = splitkv.splitkv_plan_shard(*args, R, r, contiguous_ranks=True)
+        assert p.export(splitkv.EXPORT_CHUNK_OWNER).tolist() == owner
+        ent = p.export(splitkv.EXPORT_ENTRIES).reshape(-1, 4).tolist()
+        assert sorted(map(tuple, ent)) == sorted(e for e in full_entries if owner[e[0]] == r)
+        union += [tuple(e) for e in ent]
+        p.destroy()
+    assert sorted(union) == sorted(full_entries)
+    # a plain plan ignores the flag
+    a = splitkv.splitkv_plan(*args)
+    b = splitkv.splitkv_plan(*args, contiguous_ranks=True)
+    assert np.array_equal(a.export(splitkv.EXPORT_FWD_SCHEDULE), b.export(splitkv.EXPORT_FWD_SCHEDULE))
