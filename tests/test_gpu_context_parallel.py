@@ -29,6 +29,7 @@ CASES = {
     "mma_d64_R4": dict(w=dict(Hq=4, Hkv=2, d=64), R=4, plan=dict()),
     "chunk_not_dividing_R2": dict(w=dict(Hq=4, Hkv=1, d=128, C=100, lens=(257, 3, 1000, 61)), R=2, plan=dict()),
     "reading_b_R2": dict(w=dict(Hq=8, Hkv=1), R=2, plan=dict(block_keys_in_context=True)),
+    "contiguous_ranks_R3": dict(w=dict(), R=3, plan=dict(contiguous_ranks=True, q_slice=1)),
 }
 
 
