@@ -137,6 +137,17 @@ class SplitKVContextParallel:
             ops = ops(self)          # a factory given this rank's layout
         self.ops = ops
         self._saved = None
+        self._bufs = {}
+
+    def _buffer(self, name: str, like: torch.Tensor, zero: bool = False) -> torch.Tensor:
+        """A full-size (every query row) buffer kept across steps: the query side has the same
+        shape every step, and rows other ranks never send stay as first written (zero)."""
+        shape = (sum(self.row_counts),) + tuple(like.shape[1:])
+        b = self._bufs.get(name)
+        if b is None or tuple(b.shape) != shape or b.dtype != like.dtype or b.device != like.device:
+            b = (torch.zeros if zero else torch.empty)(shape, dtype=like.dtype, device=like.device)
+            self._bufs[name] = b
+        return b
 
     # ---- layout
     @property
@@ -154,9 +165,9 @@ class SplitKVContextParallel:
         return [(c * C, min((c + 1) * C, self.N)) for c, o in enumerate(self.chunk_owner) if o == self.rank]
 
     # ---- row movement
-    def _gather_rows(self, shard: torch.Tensor) -> torch.Tensor:
+    def _gather_rows(self, name: str, shard: torch.Tensor) -> torch.Tensor:
         """Every rank's block rows, in block order: one broadcast per rank into its rows."""
-        full = torch.empty((sum(self.row_counts),) + tuple(shard.shape[1:]), dtype=shard.dtype, device=shard.device)
+        full = self._buffer(name, shard)
         full[self.rows].copy_(shard)
         for r in range(self.R):
             if self.row_counts[r]:
@@ -165,11 +176,11 @@ class SplitKVContextParallel:
                                group=self.group)
         return full
 
-    def _place_rows(self, shard: Optional[torch.Tensor]) -> Optional[torch.Tensor]:
+    def _place_rows(self, name: str, shard: Optional[torch.Tensor]) -> Optional[torch.Tensor]:
         """A full-size buffer holding this rank's block rows (the only rows it reads)."""
         if shard is None:
             return None
-        full = torch.zeros((sum(self.row_counts),) + tuple(shard.shape[1:]), dtype=shard.dtype, device=shard.device)
+        full = self._buffer(name, shard, zero=True)
         full[self.rows].copy_(shard)
         return full
 
@@ -183,8 +194,8 @@ class SplitKVContextParallel:
 
     # ---- steps
     def forward(self, q, k, v, kb, vb, scale: float, out_dtype=torch.float32):
-        q_full = self._gather_rows(q)
-        kb_full, vb_full = self._place_rows(kb), self._place_rows(vb)
+        q_full = self._gather_rows("q", q)
+        kb_full, vb_full = self._place_rows("kb", kb), self._place_rows("vb", vb)
         o_r, lse_r = self.ops.local_fwd(q_full, k, v, kb_full, vb_full, scale)
         o, lse = self.ops.combine(self._to_owners(o_r), self._to_owners(lse_r), out_dtype)
         self._saved = (q_full, kb_full, vb_full)
@@ -194,7 +205,8 @@ class SplitKVContextParallel:
         if self._saved is None:
             raise RuntimeError("backward needs a forward first")
         q_full, kb_full, vb_full = self._saved
-        o_full, lse_full, dout_full = self._gather_rows(o), self._gather_rows(lse), self._gather_rows(dout)
+        o_full, lse_full, dout_full = (self._gather_rows("o", o), self._gather_rows("lse", lse),
+                                       self._gather_rows("dout", dout))
         g = self.ops.local_bwd(q_full, k, v, kb_full, vb_full, o_full, lse_full, dout_full, scale)
         out = {"dq": self.ops.sum(self._to_owners(g["dq"])), "dk": g["dk"], "dv": g["dv"]}
         for n in ("dkb", "dvb"):
