@@ -476,6 +476,84 @@ def device_lpt_report(skv, w, workers=(8, 16, 32, 64)):
     return out
 
 
+def run_split_kv(args, world, rank, local):
+    """Split-KV over the torchrun ranks (one GPU each): the whole workload split by chunk
+    ownership, a step = SplitKVContextParallel forward + backward (query-side broadcasts,
+    local kernels, all-to-all of result rows, combine, dq sum); every rank's K, V hold the
+    whole context (only its chunks are read).  Timed like the main arm: CUDA events on the
+    launch stream between barriers, max over ranks; `value` = the whole problem's FLOPs per
+    second (total work fixed as N grows: strong scaling)."""
+    import datetime
+
+    import torch
+    import torch.distributed as dist
+
+    from context_block_sparse_b200.context_parallel import SplitKVContextParallel
+    from synth import make_workload
+
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    if "MASTER_ADDR" not in os.environ:      # run without torchrun: a one-rank group
+        import socket
+        s = socket.socket()
+        s.bind(("127.0.0.1", 0))
+        os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(s.getsockname()[1]), RANK="0", WORLD_SIZE="1")
+        s.close()
+    dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=180), device_id=dev)
+    try:
+        w = make_workload(args.workload, num_anchors=args.anchors, seed=args.seed, with_grad=True)
+        W, Wb = _workers(args)
+        W = W or torch.cuda.get_device_properties(dev).multi_processor_count
+        Wb = Wb or W
+        cp = SplitKVContextParallel(w.sample_lens, w.anchors, w.block_size, w.num_q_heads, w.num_kv_heads,
+                                    w.head_dim, w.kv_chunk, num_workers=W, num_bwd_workers=Wb, q_slice=args.q_slice,
+                                    tile_cost=args.lpt_cost == "tiles", dynamic_claim=args.dynamic_claim,
+                                    partial_bf16=args.partial_bf16, contiguous_ranks=args.schedule == "contiguous")
+        up = lambda n: torch.from_numpy(w.bits[n].view(np.int16)).view(torch.bfloat16).to(dev)   # noqa: E731
+        t = {n: up(n) for n in ("q", "k", "v", "kb", "vb", "dout")}
+        rows = cp.rows
+        q, kb, vb, dout = (t[n][rows].contiguous() for n in ("q", "kb", "vb", "dout"))
+        stream = torch.cuda.current_stream(dev)
+
+        def step():
+            o, lse = cp.forward(q, t["k"], t["v"], kb, vb, w.scale)
+            cp.backward(t["k"], t["v"], o, lse, dout, w.scale)
+
+        for _ in range(args.warmup):
+            step()
+        torch.cuda.synchronize(dev)
+        dist.barrier()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(args.steps):
+            step()
+        b.record(stream)
+        torch.cuda.synchronize(dev)
+        dist.barrier()
+        ms = max_over_ranks(a.elapsed_time(b), dev)
+        full = skv_plan_stats_of(w, W)
+        flops_step = 14.0 * w.head_dim * (full["context_pairs"] + full["block_pairs"])
+        res = {"metric": METRIC, "value": flops_step * args.steps / (ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+               "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms / args.steps,
+               "higher_is_better": True, "scaling": "strong", "vs_baseline": None, "dtype": "bf16",
+               "data": "synthetic", "impl": "split-kv",
+               "config": {**bench_config(args, w, W, Wb, world), "parallelism": f"split-kv over {world} ranks",
+                          "chunk_ownership": "contiguous" if args.schedule == "contiguous" else "lpt"}}
+        return res if rank == 0 else None
+    finally:
+        dist.destroy_process_group()
+
+
+def skv_plan_stats_of(w, W):
+    """Pair counts of the whole (unsplit) problem, from a host-only plan."""
+    import context_block_sparse_b200 as skv
+    p = skv.splitkv_plan(w.sample_lens, w.anchors, w.block_size, w.num_q_heads, w.num_kv_heads, w.head_dim,
+                         w.kv_chunk, W)
+    st = p.stats()
+    p.destroy()
+    return st
+
+
 def rank_emulation_report(skv, w, args, R, dev, stream, t, W, Wb, peaks, reps=5, contiguous=False):
     """Split-KV over R ranks with one GPU standing in for each rank in turn (after the timed
     region, untimed by the bench line): per rank, the device time of its forward
@@ -746,6 +824,9 @@ def parse_args(argv=None):
                          "kernels, static lists, to time what LPT saves")
     ap.add_argument("--dump-plan", default=None, metavar="PATH",
                     help="write the run's plan (problem, stats, every table) to PATH (.npz)")
+    ap.add_argument("--split-kv", action="store_true",
+                    help="under torchrun: Split-KV over the ranks (chunks owned by LPT, or in order with "
+                         "--schedule contiguous), the whole workload split, strong scaling")
     ap.add_argument("--emulate-ranks", type=int, default=0, metavar="R",
                     help="also report Split-KV over R ranks, one GPU running each rank plan in turn")
     ap.add_argument("--partial-bf16", action="store_true",
@@ -753,7 +834,9 @@ def parse_args(argv=None):
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
-    args.dynamic_claim = args.claims == "run-time" and args.schedule == "lpt"
+    # the contiguous schedule is a CTA-level mode; under --split-kv --schedule contiguous names
+    # the chunk ownership over ranks instead, and the CTAs keep LPT
+    args.dynamic_claim = args.claims == "run-time" and (args.schedule == "lpt" or args.split_kv)
     return args
 
 
@@ -764,6 +847,8 @@ def main(argv=None):
         print(f"warning: --gpus {args.gpus} but WORLD_SIZE={world}", file=sys.stderr)
     if args.impl == "reference":
         res = run_reference(args, world, rank)
+    elif args.split_kv:
+        res = run_split_kv(args, world, rank, local)
     else:
         res = run_ours(args, world, rank, local)
     if res is not None:

@@ -105,3 +105,7 @@ def test_rank_emulation_option():
     assert bench.parse_args([]).emulate_ranks == 0                 # not part of the default run
     assert bench.parse_args(["--emulate-ranks", "4"]).emulate_ranks == 4
     assert callable(bench.rank_emulation_report)
+    a = bench.parse_args(["--split-kv", "--schedule", "contiguous"])
+    assert a.split_kv and a.dynamic_claim                           # contiguous names the rank ownership there
+    assert not bench.parse_args(["--schedule", "contiguous"]).dynamic_claim
+    assert callable(bench.run_split_kv)
