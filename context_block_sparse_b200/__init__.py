@@ -396,6 +396,21 @@ def splitkv_read_cta_times(plan: Plan, which: int, stream=None) -> np.ndarray:
     return out
 
 
+def splitkv_merge_to_owners(plan: Plan, q, kb, vb, scale: float, ws, o_dest, lse_dest, stream=None) -> None:
+    """The merge of a rank plan writing each block's rows into its owner's receive buffers:
+    o_dest, lse_dest are int64 CUDA tensors [R] of device addresses (o: float32 [R][rows_r][Hq][d],
+    lse: float32 [R][rows_r][Hq] on rank r)."""
+    import torch
+    shard = splitkv_plan_export(plan, EXPORT_QUERY_SHARD).tolist()
+    for name, t in (("o_dest", o_dest), ("lse_dest", lse_dest)):
+        if t.dtype != torch.int64 or t.numel() != shard[1]:
+            raise ValueError(f"{name} must be an int64 tensor of {shard[1]} device addresses")
+    _sizes(plan, q=q, kb=kb, vb=vb)
+    _check("splitkv_merge_to_owners", _lib.splitkv_merge_to_owners(
+        plan.handle, _bf16_ptr(q), _bf16_ptr(kb), _bf16_ptr(vb), float(scale), _ptr(ws),
+        ws.numel() * ws.element_size(), shard[1], shard[0], _ptr(o_dest), _ptr(lse_dest), _stream_ptr(stream)))
+
+
 def splitkv_combine_ranks(o_parts, lse_parts, o, lse, stream=None) -> None:
     """o_parts [R, rows..., d] and lse_parts [R, rows...] float32 -> o [rows..., d] (float32 or
     bfloat16) and lse [rows...]: the exact combine of R ranks' results."""

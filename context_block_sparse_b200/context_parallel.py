@@ -35,7 +35,8 @@ import torch.distributed as dist
 
 from . import (
     EXPORT_CHUNK_OWNER, EXPORT_QUERY_SHARD, WS_BWD, WS_FWD, splitkv_attn_bwd, splitkv_attn_fwd,
-    splitkv_combine_ranks, splitkv_merge, splitkv_plan_shard, splitkv_sum_ranks, splitkv_workspace_size,
+    splitkv_combine_ranks, splitkv_merge, splitkv_merge_to_owners, splitkv_plan_shard, splitkv_sum_ranks,
+    splitkv_workspace_size,
 )
 
 
@@ -64,6 +65,12 @@ class KernelOps:
         splitkv_attn_fwd(self.plan, q, k, v, scale, self.ws_fwd)
         splitkv_merge(self.plan, q, kb, vb, scale, self.ws_fwd, o, lse)
         return o, lse
+
+    def local_fwd_to_owners(self, q, k, v, kb, vb, scale: float, dest_o, dest_lse):
+        """The forward with the exchange fused into the merge: rows go straight into the
+        owners' receive buffers (device addresses in dest_o / dest_lse)."""
+        splitkv_attn_fwd(self.plan, q, k, v, scale, self.ws_fwd)
+        splitkv_merge_to_owners(self.plan, q, kb, vb, scale, self.ws_fwd, dest_o, dest_lse)
 
     def combine(self, o_parts, lse_parts, out_dtype):
         o = torch.empty(o_parts.shape[1:], dtype=out_dtype, device=self.device)
@@ -106,9 +113,16 @@ class SplitKVContextParallel:
     """
 
     def __init__(self, sample_lens, anchors, block_size: int, num_q_heads: int, num_kv_heads: int, head_dim: int,
-                 kv_chunk: int, group=None, num_workers: Optional[int] = None, device=None, ops=None, **plan_kw):
+                 kv_chunk: int, group=None, num_workers: Optional[int] = None, device=None, ops=None,
+                 exchange: str = "nccl", **plan_kw):
         """ops: the local steps (default: the library's kernels on `device`), or a factory
-        called with this object; plan_kw: options of splitkv_plan (q_slice, tile_cost, ...)."""
+        called with this object; exchange: "nccl" (all-to-all of result rows) or "p2p" (the
+        forward merge stores each row into its owner's receive buffer, mapped into every rank
+        by CUDA IPC; ranks of one node with peer access); plan_kw: options of splitkv_plan
+        (q_slice, tile_cost, ...)."""
+        if exchange not in ("nccl", "p2p"):
+            raise ValueError("exchange is 'nccl' or 'p2p'")
+        self.exchange = exchange
         self.group = group
         self.R = dist.get_world_size(group)
         self.rank = dist.get_rank(group)
@@ -138,6 +152,7 @@ class SplitKVContextParallel:
         self.ops = ops
         self._saved = None
         self._bufs = {}
+        self._p2p = None
 
     def _buffer(self, name: str, like: torch.Tensor, zero: bool = False) -> torch.Tensor:
         """A full-size (every query row) buffer kept across steps: the query side has the same
@@ -192,12 +207,46 @@ class SplitKVContextParallel:
         dist.all_to_all_single(out, full.contiguous(), [mine] * self.R, self.row_counts, group=self.group)
         return out.view((self.R, mine) + tuple(full.shape[1:]))
 
+    def _p2p_buffers(self, device):
+        """This rank's receive buffers ([R][rows][Hq][d], [R][rows][Hq]) and the device
+        addresses of every rank's, mapped here through CUDA IPC (set up once)."""
+        if self._p2p is None:
+            from torch.multiprocessing.reductions import reduce_tensor
+            mine = self.row_counts[self.rank]
+            f32 = dict(dtype=torch.float32, device=device)
+            recv_o = torch.zeros((self.R, mine, self.Hq, self.d), **f32)
+            recv_l = torch.zeros((self.R, mine, self.Hq), **f32)
+            handles = [None] * self.R
+            dist.all_gather_object(handles, (reduce_tensor(recv_o), reduce_tensor(recv_l)), group=self.group)
+            peers, ptr_o, ptr_l = [], [], []
+            for r, (ho, hl) in enumerate(handles):
+                to, tl = (recv_o, recv_l) if r == self.rank else (ho[0](*ho[1]), hl[0](*hl[1]))
+                peers.append((to, tl))          # keeps the mappings open
+                ptr_o.append(to.data_ptr())
+                ptr_l.append(tl.data_ptr())
+            self._p2p = {"o": recv_o, "lse": recv_l, "peers": peers,
+                         "dest_o": torch.tensor(ptr_o, dtype=torch.int64, device=device),
+                         "dest_lse": torch.tensor(ptr_l, dtype=torch.int64, device=device),
+                         "flag": torch.zeros(1, dtype=torch.float32, device=device)}
+        return self._p2p
+
+    def _stream_barrier(self, flag: torch.Tensor) -> None:
+        """Every rank past this point in stream order: a one-element all-reduce."""
+        dist.all_reduce(flag, group=self.group)
+
     # ---- steps
     def forward(self, q, k, v, kb, vb, scale: float, out_dtype=torch.float32):
         q_full = self._gather_rows("q", q)
         kb_full, vb_full = self._place_rows("kb", kb), self._place_rows("vb", vb)
-        o_r, lse_r = self.ops.local_fwd(q_full, k, v, kb_full, vb_full, scale)
-        o, lse = self.ops.combine(self._to_owners(o_r), self._to_owners(lse_r), out_dtype)
+        if self.exchange == "p2p":
+            b = self._p2p_buffers(q.device)
+            self.ops.local_fwd_to_owners(q_full, k, v, kb_full, vb_full, scale, b["dest_o"], b["dest_lse"])
+            self._stream_barrier(b["flag"])          # every rank's rows have landed
+            o, lse = self.ops.combine(b["o"], b["lse"], out_dtype)
+            self._stream_barrier(b["flag"])          # every owner has read before the next writes
+        else:
+            o_r, lse_r = self.ops.local_fwd(q_full, k, v, kb_full, vb_full, scale)
+            o, lse = self.ops.combine(self._to_owners(o_r), self._to_owners(lse_r), out_dtype)
         self._saved = (q_full, kb_full, vb_full)
         return o, lse
 

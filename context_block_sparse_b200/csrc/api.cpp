@@ -86,6 +86,27 @@ int splitkv_merge(const splitkv_plan_t* plan, const void* q, const void* kb, con
       static_cast<cudaStream_t>(stream)));
 }
 
+int splitkv_merge_to_owners(const splitkv_plan_t* plan, const void* q, const void* kb, const void* vb, float scale,
+                            const void* ws, size_t ws_bytes, int32_t num_ranks, int32_t rank,
+                            float* const* o_dest, float* const* lse_dest, void* stream) {
+  const DevPlan* dp = nullptr;
+  int st = check_plan(plan, &dp);
+  if (st != SPLITKV_OK) return st;
+  int R = 1, self = 0;
+  splitkv::plan_ranks(plan, &R, &self);
+  if (num_ranks != R || rank != self || !o_dest || !lse_dest || !aligned(o_dest, 8) || !aligned(lse_dest, 8))
+    return SPLITKV_ERR_INVALID_ARG;
+  if (!all_aligned16(q, ws) || !block_ptrs_ok(dp, kb, vb)) return SPLITKV_ERR_INVALID_ARG;
+  const splitkv::FwdWs L = splitkv::fwd_ws_layout(dp->E, dp->bs, dp->Hq, dp->d, rec_bytes(dp));
+  if (ws_bytes < L.total) return SPLITKV_ERR_WORKSPACE_TOO_SMALL;
+  const char* w = static_cast<const char*>(ws);
+  return cuda_status(splitkv::launch_merge(
+      *dp, static_cast<const uint16_t*>(q), static_cast<const uint16_t*>(kb), static_cast<const uint16_t*>(vb),
+      scale, static_cast<const void*>(w + L.o_off), reinterpret_cast<const float*>(w + L.m_off),
+      reinterpret_cast<const float*>(w + L.l_off), nullptr, 0, nullptr, static_cast<cudaStream_t>(stream),
+      splitkv::MergeDest{o_dest, lse_dest, R, self}));
+}
+
 int splitkv_bwd_delta(const splitkv_plan_t* plan, const void* o, int o_dtype, const void* dout, void* ws,
                       size_t ws_bytes, void* stream) {
   const DevPlan* dp = nullptr;

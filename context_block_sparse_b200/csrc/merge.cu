@@ -150,7 +150,7 @@ __global__ void __launch_bounds__(kMergeThreads, 2)
     merge_kernel(DevPlan p, const uint16_t* __restrict__ q, const uint16_t* __restrict__ kb,
                  const uint16_t* __restrict__ vb, float scale_log2, const void* __restrict__ part_o,
                  const float* __restrict__ part_m, const float* __restrict__ part_l, void* __restrict__ o,
-                 int o_bf16, float* __restrict__ lse) {
+                 int o_bf16, float* __restrict__ lse, const MergeDest dest) {
   constexpr int NG = D / 16;
   using RecT = Rec<kBf16Rec>;
   constexpr int EG = 64 / (NG * RecT::RW);   // entries whose records are in flight together
@@ -170,6 +170,26 @@ __global__ void __launch_bounds__(kMergeThreads, 2)
   const int e0 = p.block_entry_ptr[b], n = p.block_entry_ptr[b + 1] - e0;
   const int R = p.G * p.bs;
   const int n_block_keys = bterm ? p.bs : 0;   // none when they are context keys, or on another rank
+  // output rows: the plan's own outputs, or the owner's receive buffer (see MergeDest);
+  // row_base = this block's first row in the buffer written to
+  void* o_out = o;
+  float* lse_out = lse;
+  int out_bf16 = o_bf16;
+  size_t row_base = size_t(b) * p.bs;
+  bool out_ok = true;
+  if (dest.o != nullptr) {
+    const int own = int((int64_t(b + 1) * dest.R - 1) / p.A);
+    const int lo = int(int64_t(own) * p.A / dest.R), hi = int(int64_t(own + 1) * p.A / dest.R);
+    out_ok = own >= 0 && own < dest.R && b >= lo && b < hi && dest.self >= 0 && dest.self < dest.R;
+    if (out_ok) {
+      o_out = dest.o[own];
+      lse_out = dest.lse[own];
+      row_base = size_t(dest.self) * size_t(hi - lo) * p.bs + size_t(b - lo) * p.bs;
+    } else if (threadIdx.x == 0) {
+      atomicCAS(p.status, 0, SPLITKV_ERR_INVALID_ARG);   // never reached: the owner formula failed
+    }
+    out_bf16 = 0;
+  }
   for (int r0 = 0; r0 < R; r0 += kRowsPerPass) {
     // rows ordered (token, head): the 8 rows of a warp are contiguous records
     const int r = min(r0 + (tid >> 2), R - 1);          // rows past R compute, never store
@@ -258,10 +278,11 @@ __global__ void __launch_bounds__(kMergeThreads, 2)
         }
       }
     }
-    if (active) {
+    if (active && out_ok) {
+      const size_t orow = (row_base + tt) * p.Hq + head;   // = qrow for the plan's own outputs
       const float inv = L > 0.f ? 1.f / L : 0.f;
-      if (o_bf16) {
-        uint16_t* dst = static_cast<uint16_t*>(o) + qrow * D;
+      if (out_bf16) {
+        uint16_t* dst = static_cast<uint16_t*>(o_out) + orow * D;
 #pragma unroll
         for (int k = 0; k < NG; ++k) {
           uint2 w;
@@ -270,13 +291,13 @@ __global__ void __launch_bounds__(kMergeThreads, 2)
           *reinterpret_cast<uint2*>(dst + 4 * (u + 4 * k)) = w;
         }
       } else {
-        float* dst = static_cast<float*>(o) + qrow * D;
+        float* dst = static_cast<float*>(o_out) + orow * D;
 #pragma unroll
         for (int k = 0; k < NG; ++k)
           *reinterpret_cast<float4*>(dst + 4 * (u + 4 * k)) =
               make_float4(acc[k][0] * inv, acc[k][1] * inv, acc[k][2] * inv, acc[k][3] * inv);
       }
-      if (u == 0) lse[qrow] = L > 0.f ? (M + __log2f(L)) * kLn2 : -INFINITY;
+      if (u == 0) lse_out[orow] = L > 0.f ? (M + __log2f(L)) * kLn2 : -INFINITY;
     }
   }
 }
@@ -480,13 +501,13 @@ __global__ void __launch_bounds__(kMergeThreads, 2)
 template <int D, bool kBf16Rec>
 cudaError_t merge_d(const DevPlan& p, const uint16_t* q, const uint16_t* kb, const uint16_t* vb,
                     float scale, const void* po, const float* pm, const float* pl, void* o, int o_bf16,
-                    float* lse, cudaStream_t s) {
+                    float* lse, cudaStream_t s, const MergeDest& dest) {
   const size_t smem = size_t(2) * p.bs * D * sizeof(uint16_t) + kEStage * sizeof(int);
   cudaError_t e =
       cudaFuncSetAttribute(merge_kernel<D, kBf16Rec>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
   if (e != cudaSuccess) return e;
   merge_kernel<D, kBf16Rec><<<dim3(p.A, p.Hkv), kMergeThreads, smem, s>>>(p, q, kb, vb, scale * kLog2e, po, pm,
-                                                                            pl, o, o_bf16, lse);
+                                                                            pl, o, o_bf16, lse, dest);
   return cudaGetLastError();
 }
 
@@ -512,13 +533,13 @@ cudaError_t reduce_d(const DevPlan& p, const uint16_t* q, const uint16_t* kb, co
 
 cudaError_t launch_merge(const DevPlan& p, const uint16_t* q, const uint16_t* kb, const uint16_t* vb,
                          float scale, const void* part_o, const float* part_m, const float* part_l,
-                         void* o, int o_bf16, float* lse, cudaStream_t s) {
+                         void* o, int o_bf16, float* lse, cudaStream_t s, const MergeDest& dest) {
   if (p.partial_bf16) {
-    if (p.d == 64) return merge_d<64, true>(p, q, kb, vb, scale, part_o, part_m, part_l, o, o_bf16, lse, s);
-    return merge_d<128, true>(p, q, kb, vb, scale, part_o, part_m, part_l, o, o_bf16, lse, s);
+    if (p.d == 64) return merge_d<64, true>(p, q, kb, vb, scale, part_o, part_m, part_l, o, o_bf16, lse, s, dest);
+    return merge_d<128, true>(p, q, kb, vb, scale, part_o, part_m, part_l, o, o_bf16, lse, s, dest);
   }
-  if (p.d == 64) return merge_d<64, false>(p, q, kb, vb, scale, part_o, part_m, part_l, o, o_bf16, lse, s);
-  return merge_d<128, false>(p, q, kb, vb, scale, part_o, part_m, part_l, o, o_bf16, lse, s);
+  if (p.d == 64) return merge_d<64, false>(p, q, kb, vb, scale, part_o, part_m, part_l, o, o_bf16, lse, s, dest);
+  return merge_d<128, false>(p, q, kb, vb, scale, part_o, part_m, part_l, o, o_bf16, lse, s, dest);
 }
 
 cudaError_t launch_bwd_delta(const DevPlan& p, const void* o, int o_bf16, const uint16_t* dout,

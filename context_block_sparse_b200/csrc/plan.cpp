@@ -866,4 +866,8 @@ int splitkv_workspace_size(const splitkv_plan_t* P, int which, size_t* bytes) {
 // Accessors for the attention entry points (api.cu).
 namespace splitkv {
 const DevPlan* plan_device_view(const splitkv_plan_t* P) { return P->uploaded ? &P->dev : nullptr; }
+void plan_ranks(const splitkv_plan_t* P, int* R, int* rank) {
+  *R = P->R;
+  *rank = P->rank;
+}
 }  // namespace splitkv

@@ -7,6 +7,8 @@
 
 #include <cuda_runtime.h>
 
+#include "splitkv.h"
+
 namespace splitkv {
 
 // Rows of one query tile: 128 / (G * bs) blocks x G heads x bs tokens.
@@ -93,10 +95,25 @@ cudaError_t launch_fwd_partial(const DevPlan& p, const uint16_t* q, const uint16
                                const uint16_t* v, float scale, void* part_o, float* part_m,
                                float* part_l, cudaStream_t s);
 
+// Where the merge writes its rows.  o == nullptr: the plan's own outputs (o, lse, every
+// query row).  Otherwise the exchange of Split-KV over ranks fused into the merge: the
+// rows of block b go to the receive buffers of the rank that owns b (blocks
+// [floor(r A / R), floor((r + 1) A / R)) to rank r) -- o[r] float32 [R][rows_r][Hq][d],
+// lse[r] [R][rows_r][Hq] -- at slot `self`; o and lse are device arrays of R pointers,
+// which may point into other GPUs' memory (peer-mapped).
+struct MergeDest {
+  float* const* o;
+  float* const* lse;
+  int R, self;
+};
+
 cudaError_t launch_merge(const DevPlan& p, const uint16_t* q, const uint16_t* kb,
                          const uint16_t* vb, float scale, const void* part_o,
                          const float* part_m, const float* part_l, void* o, int o_bf16,
-                         float* lse, cudaStream_t s);
+                         float* lse, cudaStream_t s, const MergeDest& dest = MergeDest{nullptr, nullptr, 1, 0});
+
+// R and rank of a plan (1 and 0 unless made by splitkv_plan_shard).
+void plan_ranks(const splitkv_plan_t* plan, int* R, int* rank);
 
 cudaError_t launch_bwd_delta(const DevPlan& p, const void* o, int o_bf16, const uint16_t* dout,
                              float* delta, cudaStream_t s);

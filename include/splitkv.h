@@ -410,6 +410,22 @@ int splitkv_plan_status(const splitkv_plan_t* plan, void* stream, int32_t* site)
  * Errors: INVALID_ARG, CUDA. */
 int splitkv_selftest_exp2(const float* x, float* y, int64_t n, void* stream);
 
+/* splitkv_merge of a rank plan with the exchange of Split-KV over ranks fused in (news
+ * page, "Exchange the smaller side"): instead of writing every query row's result to
+ * local o, lse, the rows of block b go straight to the receive buffers of the rank that
+ * owns b (blocks [floor(r A / R), floor((r + 1) A / R)) to rank r, as the plan's
+ * SPLITKV_EXPORT_QUERY_SHARD): o_dest[r] float32 [R][rows_r][Hq][d] and lse_dest[r]
+ * float32 [R][rows_r][Hq], rows_r = bs * (blocks of rank r), at slot `rank` -- the
+ * layout splitkv_combine_ranks reads on rank r.  o_dest and lse_dest are DEVICE arrays of
+ * R device pointers (8-byte aligned); entries may be another GPU's memory mapped into this
+ * one (peer access), which the kernel writes with plain stores.  The caller orders the
+ * owners' combine after every rank's merge (a collective or a barrier).  num_ranks and
+ * rank must be the plan's (splitkv_plan_shard).  Errors: as splitkv_merge, INVALID_ARG
+ * also for a rank mismatch or a NULL / misaligned pointer array. */
+int splitkv_merge_to_owners(const splitkv_plan_t* plan, const void* q, const void* kb, const void* vb,
+                            float scale, const void* ws, size_t ws_bytes, int32_t num_ranks, int32_t rank,
+                            float* const* o_dest, float* const* lse_dest, void* stream);
+
 /* Exact combine of the ranks' results (news page, "Exchange the smaller side":
  * partials over disjoint key shares merged with their normalisation statistics).
  * o_parts [R][rows][head_dim] and lse_parts [R][rows] float32 (device; row =

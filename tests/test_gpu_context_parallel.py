@@ -148,6 +148,69 @@ def test_bwd_workload_over_four_ranks_sampled(splitkv):
         assert np.isfinite(out[n]).all(), n
 
 
+@pytest.mark.parametrize("R,case", [(2, "tcgen05"), (3, "tcgen05"), (3, "mma_d64")])
+def test_merge_to_owners_is_the_merge_laid_out_by_owner(splitkv, R, case):
+    """splitkv_merge_to_owners (the exchange fused into the merge) stores, for every rank,
+    exactly the rows its plain merge writes, each block's rows in its owner's receive buffer
+    [R][rows_owner] at the sender's slot (bit for bit); the owners' combines match the
+    oracle.  One GPU, so every destination is local memory."""
+    import torch
+    from context_block_sparse_b200.context_parallel import block_ranges
+    skv = splitkv
+    w = small() if case == "tcgen05" else small(Hq=4, Hkv=2, d=64)
+    t = {n: to_dev(b) for n, b in w.bits.items()}
+    Nq, Hq, d, bs = w.num_queries, w.num_q_heads, w.head_dim, w.block_size
+    f32 = dict(dtype=torch.float32, device="cuda")
+    ranges = block_ranges(w.anchors.size, R)
+    n_rows = [(hi - lo) * bs for lo, hi in ranges]
+    recv_o = [torch.full((R, n, Hq, d), float("nan"), **f32) for n in n_rows]
+    recv_l = [torch.full((R, n, Hq), float("nan"), **f32) for n in n_rows]
+    dest_o = torch.tensor([x.data_ptr() for x in recv_o], dtype=torch.int64, device="cuda")
+    dest_l = torch.tensor([x.data_ptr() for x in recv_l], dtype=torch.int64, device="cuda")
+    args = (w.sample_lens, w.anchors, bs, Hq, w.num_kv_heads, d, w.kv_chunk, 148)
+    o_loc = torch.empty((R, Nq, Hq, d), **f32)
+    l_loc = torch.empty((R, Nq, Hq), **f32)
+    for r in range(R):
+        plan = skv.splitkv_plan_shard(*args, R, r).upload()
+        ws = torch.empty(skv.splitkv_workspace_size(plan, skv.WS_FWD), dtype=torch.uint8, device="cuda")
+        skv.splitkv_attn_fwd(plan, t["q"], t["k"], t["v"], w.scale, ws)
+        skv.splitkv_merge(plan, t["q"], t["kb"], t["vb"], w.scale, ws, o_loc[r], l_loc[r])
+        skv.splitkv_merge_to_owners(plan, t["q"], t["kb"], t["vb"], w.scale, ws, dest_o, dest_l)
+        torch.cuda.synchronize()
+        skv.splitkv_plan_status(plan)
+        plan.destroy()
+    O, L = oracle_fwd(w)
+    for own, (lo, hi) in enumerate(ranges):
+        rows = slice(lo * bs, hi * bs)
+        assert torch.equal(recv_o[own], o_loc[:, rows]), f"owner {own}: o rows differ from the plain merge"
+        assert torch.equal(recv_l[own], l_loc[:, rows]), f"owner {own}: lse rows differ from the plain merge"
+        o = torch.empty((hi - lo) * bs, Hq, d, **f32)
+        lse = torch.empty((hi - lo) * bs, Hq, **f32)
+        skv.splitkv_combine_ranks(recv_o[own], recv_l[own], o, lse)
+        assert_close("O", o.cpu().numpy().astype(np.float64), O[rows], TOL_OUT)
+        assert_close("LSE", lse.cpu().numpy().astype(np.float64), L[rows], TOL_LSE)
+
+
+def test_merge_to_owners_refuses_a_rank_mismatch(splitkv):
+    import torch
+    skv = splitkv
+    w = small()
+    plan = skv.splitkv_plan_shard(w.sample_lens, w.anchors, w.block_size, w.num_q_heads, w.num_kv_heads,
+                                  w.head_dim, w.kv_chunk, 148, 2, 1).upload()
+    t = {n: to_dev(b) for n, b in w.bits.items()}
+    ws = torch.empty(skv.splitkv_workspace_size(plan, skv.WS_FWD), dtype=torch.uint8, device="cuda")
+    ptrs = torch.zeros(2, dtype=torch.int64, device="cuda")
+    st = skv._lib.splitkv_merge_to_owners(plan.handle, t["q"].data_ptr(), t["kb"].data_ptr(), t["vb"].data_ptr(),
+                                          0.1, ws.data_ptr(), ws.numel(), 2, 0, ptrs.data_ptr(), ptrs.data_ptr(),
+                                          None)
+    assert st == -1                                       # the plan is rank 1's, not rank 0's
+    st = skv._lib.splitkv_merge_to_owners(plan.handle, t["q"].data_ptr(), t["kb"].data_ptr(), t["vb"].data_ptr(),
+                                          0.1, ws.data_ptr(), ws.numel(), 3, 1, ptrs.data_ptr(), ptrs.data_ptr(),
+                                          None)
+    assert st == -1                                       # of 2 ranks, not 3
+    torch.cuda.synchronize()
+
+
 @pytest.mark.parametrize("R,d,o_bf16", [(1, 128, False), (3, 128, False), (5, 64, True), (8, 128, True)])
 def test_combine_kernel_against_oracle(splitkv, R, d, o_bf16):
     import torch
@@ -202,8 +265,10 @@ def test_combine_and_sum_reject_bad_arguments(splitkv):
     assert lib.splitkv_sum_ranks(2, 0, None, None, None) == 0
 
 
-def test_context_parallel_class_on_one_nccl_rank(splitkv):
-    """SplitKVContextParallel end to end (broadcasts, all-to-all, kernels) on a one-rank group."""
+@pytest.mark.parametrize("exchange", ["nccl", "p2p"])
+def test_context_parallel_class_on_one_nccl_rank(splitkv, exchange):
+    """SplitKVContextParallel end to end (broadcasts, all-to-all or the fused merge with its
+    stream barriers, kernels) on a one-rank group, two steps."""
     import socket
 
     import torch
@@ -219,11 +284,13 @@ def test_context_parallel_class_on_one_nccl_rank(splitkv):
         w = small()
         t = {n: to_dev(b) for n, b in w.bits.items()}
         cp = SplitKVContextParallel(w.sample_lens, w.anchors, w.block_size, w.num_q_heads, w.num_kv_heads,
-                                    w.head_dim, w.kv_chunk, q_slice=2, tile_cost=True, dynamic_claim=True)
+                                    w.head_dim, w.kv_chunk, q_slice=2, tile_cost=True, dynamic_claim=True,
+                                    exchange=exchange)
         assert cp.owned_rows() == [(c * w.kv_chunk, min((c + 1) * w.kv_chunk, w.context_len))
                                    for c in range(-(-w.context_len // w.kv_chunk))]
-        o, lse = cp.forward(t["q"], t["k"], t["v"], t["kb"], t["vb"], w.scale)
-        g = cp.backward(t["k"], t["v"], o, lse, t["dout"], w.scale)
+        for _ in range(2):
+            o, lse = cp.forward(t["q"], t["k"], t["v"], t["kb"], t["vb"], w.scale)
+            g = cp.backward(t["k"], t["v"], o, lse, t["dout"], w.scale)
         torch.cuda.synchronize()
         O, L = oracle_fwd(w)
         assert_close("O", o.cpu().numpy().astype(np.float64), O, TOL_OUT)

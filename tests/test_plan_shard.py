@@ -162,3 +162,34 @@ def test_contiguous_rank_ownership_bit_exact(splitkv, R):
     a = splitkv.splitkv_plan(*args)
     b = splitkv.splitkv_plan(*args, contiguous_ranks=True)
     assert np.array_equal(a.export(splitkv.EXPORT_FWD_SCHEDULE), b.export(splitkv.EXPORT_FWD_SCHEDULE))
+
+
+def _owner_slot(A, R, bs, src, b, t):
+    """The merge kernel's destination of row t of block b sent by rank `src` under
+    splitkv_merge_to_owners: (owner, row in the owner's [R][rows_owner] receive buffer)."""
+    own = ((b + 1) * R - 1) // A
+    lo, hi = (own * A) // R, ((own + 1) * A) // R
+    assert lo <= b < hi
+    return own, src * (hi - lo) * bs + (b - lo) * bs + t
+
+
+@pytest.mark.parametrize("bs", [1, 4, 16])
+def test_owner_scatter_is_the_all_to_all_layout(bs):
+    """Every (sender, row) lands once, at the place the all-to-all of SplitKVContextParallel
+    puts it: rank r's rows are blocks [floor(r A / R), floor((r + 1) A / R)), received as
+    [sender][row - first row]."""
+    from context_block_sparse_b200.context_parallel import block_ranges
+    for A in range(1, 40):
+        for R in range(1, 10):
+            ranges = block_ranges(A, R)
+            seen = set()
+            for src in range(R):
+                for b in range(A):
+                    for t in range(bs):
+                        own, slot = _owner_slot(A, R, bs, src, b, t)
+                        lo, hi = ranges[own]
+                        assert lo <= b < hi
+                        assert slot == src * (hi - lo) * bs + (b * bs + t - lo * bs)
+                        assert 0 <= slot < R * (hi - lo) * bs
+                        seen.add((own, slot))
+            assert len(seen) == R * A * bs
