@@ -508,7 +508,8 @@ def run_split_kv(args, world, rank, local):
         cp = SplitKVContextParallel(w.sample_lens, w.anchors, w.block_size, w.num_q_heads, w.num_kv_heads,
                                     w.head_dim, w.kv_chunk, num_workers=W, num_bwd_workers=Wb, q_slice=args.q_slice,
                                     tile_cost=args.lpt_cost == "tiles", dynamic_claim=args.dynamic_claim,
-                                    partial_bf16=args.partial_bf16, contiguous_ranks=args.schedule == "contiguous")
+                                    partial_bf16=args.partial_bf16, contiguous_ranks=args.schedule == "contiguous",
+                                    exchange=args.exchange)
         up = lambda n: torch.from_numpy(w.bits[n].view(np.int16)).view(torch.bfloat16).to(dev)   # noqa: E731
         t = {n: up(n) for n in ("q", "k", "v", "kb", "vb", "dout")}
         rows = cp.rows
@@ -538,7 +539,8 @@ def run_split_kv(args, world, rank, local):
                "higher_is_better": True, "scaling": "strong", "vs_baseline": None, "dtype": "bf16",
                "data": "synthetic", "impl": "split-kv",
                "config": {**bench_config(args, w, W, Wb, world), "parallelism": f"split-kv over {world} ranks",
-                          "chunk_ownership": "contiguous" if args.schedule == "contiguous" else "lpt"}}
+                          "chunk_ownership": "contiguous" if args.schedule == "contiguous" else "lpt",
+                          "exchange": args.exchange}}
         return res if rank == 0 else None
     finally:
         dist.destroy_process_group()
@@ -827,6 +829,9 @@ def parse_args(argv=None):
     ap.add_argument("--split-kv", action="store_true",
                     help="under torchrun: Split-KV over the ranks (chunks owned by LPT, or in order with "
                          "--schedule contiguous), the whole workload split, strong scaling")
+    ap.add_argument("--exchange", choices=["nccl", "p2p"], default="nccl",
+                    help="with --split-kv: the forward exchange as an NCCL all-to-all, or fused into the "
+                         "merge kernel as stores into the owners' peer-mapped buffers")
     ap.add_argument("--emulate-ranks", type=int, default=0, metavar="R",
                     help="also report Split-KV over R ranks, one GPU running each rank plan in turn")
     ap.add_argument("--partial-bf16", action="store_true",

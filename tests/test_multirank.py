@@ -109,3 +109,4 @@ def test_rank_emulation_option():
     assert a.split_kv and a.dynamic_claim                           # contiguous names the rank ownership there
     assert not bench.parse_args(["--schedule", "contiguous"]).dynamic_claim
     assert callable(bench.run_split_kv)
+    assert bench.parse_args(["--split-kv", "--exchange", "p2p"]).exchange == "p2p"
