@@ -411,6 +411,22 @@ def splitkv_merge_to_owners(plan: Plan, q, kb, vb, scale: float, ws, o_dest, lse
         ws.numel() * ws.element_size(), shard[1], shard[0], _ptr(o_dest), _ptr(lse_dest), _stream_ptr(stream)))
 
 
+def splitkv_bwd_reduce_to_owners(plan: Plan, q, kb, vb, lse, dout, dkb, dvb, scale: float, ws, dq_dest,
+                                 stream=None) -> None:
+    """The dQ reduce of a rank plan writing each block's dq rows into its owner's receive
+    buffer: dq_dest is an int64 CUDA tensor [R] of device addresses (float32 [R][rows_r][Hq][d]
+    on rank r)."""
+    import torch
+    shard = splitkv_plan_export(plan, EXPORT_QUERY_SHARD).tolist()
+    if dq_dest.dtype != torch.int64 or dq_dest.numel() != shard[1]:
+        raise ValueError(f"dq_dest must be an int64 tensor of {shard[1]} device addresses")
+    _sizes(plan, q=q, kb=kb, vb=vb, lse=lse, dout=dout, dkb=dkb, dvb=dvb)
+    _check("splitkv_bwd_reduce_to_owners", _lib.splitkv_bwd_reduce_to_owners(
+        plan.handle, _bf16_ptr(q), _bf16_ptr(kb), _bf16_ptr(vb), _f32_ptr(lse), _bf16_ptr(dout), _f32_ptr(dkb),
+        _f32_ptr(dvb), float(scale), _ptr(ws), ws.numel() * ws.element_size(), shard[1], shard[0], _ptr(dq_dest),
+        _stream_ptr(stream)))
+
+
 def splitkv_combine_ranks(o_parts, lse_parts, o, lse, stream=None) -> None:
     """o_parts [R, rows..., d] and lse_parts [R, rows...] float32 -> o [rows..., d] (float32 or
     bfloat16) and lse [rows...]: the exact combine of R ranks' results."""

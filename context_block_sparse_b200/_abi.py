@@ -107,6 +107,8 @@ SIGNATURES = {
     "splitkv_plan_shard": (_I, [ctypes.POINTER(Problem), ctypes.c_int32, ctypes.c_int32, ctypes.POINTER(_P)]),
     "splitkv_combine_ranks": (_I, [ctypes.c_int32, ctypes.c_int64, ctypes.c_int32, _P, _P, _P, _I, _P, _P]),
     "splitkv_merge_to_owners": (_I, [_P, _P, _P, _P, _F, _P, _SZ, ctypes.c_int32, ctypes.c_int32, _P, _P, _P]),
+    "splitkv_bwd_reduce_to_owners": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _F, _P, _SZ, ctypes.c_int32,
+                                          ctypes.c_int32, _P, _P]),
     "splitkv_sum_ranks": (_I, [ctypes.c_int32, ctypes.c_int64, _P, _P, _P]),
     "splitkv_plan_upload": (_I, [_P, _P]),
     "splitkv_plan_destroy": (_I, [_P]),

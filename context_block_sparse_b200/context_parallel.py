@@ -34,9 +34,9 @@ import torch
 import torch.distributed as dist
 
 from . import (
-    EXPORT_CHUNK_OWNER, EXPORT_QUERY_SHARD, WS_BWD, WS_FWD, splitkv_attn_bwd, splitkv_attn_fwd,
-    splitkv_combine_ranks, splitkv_merge, splitkv_merge_to_owners, splitkv_plan_shard, splitkv_sum_ranks,
-    splitkv_workspace_size,
+    EXPORT_CHUNK_OWNER, EXPORT_QUERY_SHARD, WS_BWD, WS_FWD, splitkv_attn_bwd, splitkv_attn_fwd, splitkv_bwd_delta,
+    splitkv_bwd_partial, splitkv_bwd_reduce_to_owners, splitkv_combine_ranks, splitkv_merge,
+    splitkv_merge_to_owners, splitkv_plan_shard, splitkv_sum_ranks, splitkv_workspace_size,
 )
 
 
@@ -78,7 +78,7 @@ class KernelOps:
         splitkv_combine_ranks(o_parts, lse_parts, o, lse)
         return o, lse
 
-    def local_bwd(self, q, k, v, kb, vb, o, lse, dout, scale: float) -> Dict[str, torch.Tensor]:
+    def _bwd_buffers(self) -> Dict[str, torch.Tensor]:
         f32 = dict(dtype=torch.float32, device=self.device)
         if self._ws_bwd is None:
             self._ws_bwd = torch.empty(splitkv_workspace_size(self.plan, WS_BWD), dtype=torch.uint8,
@@ -88,10 +88,23 @@ class KernelOps:
                          "dv": torch.zeros((self.N, self.Hkv, self.d), **f32),
                          "dkb": None if self.rb else torch.zeros((self.Nq, self.Hkv, self.d), **f32),
                          "dvb": None if self.rb else torch.zeros((self.Nq, self.Hkv, self.d), **f32)}
-        g = dict(self._dkv)
-        g["dq"] = torch.empty((self.Nq, self.Hq, self.d), **f32)
+        return dict(self._dkv)
+
+    def local_bwd(self, q, k, v, kb, vb, o, lse, dout, scale: float) -> Dict[str, torch.Tensor]:
+        g = self._bwd_buffers()
+        g["dq"] = torch.empty((self.Nq, self.Hq, self.d), dtype=torch.float32, device=self.device)
         splitkv_attn_bwd(self.plan, q, k, v, kb, vb, o, lse, dout, g["dq"], g["dk"], g["dv"], g["dkb"], g["dvb"],
                          scale, self._ws_bwd)
+        return g
+
+    def local_bwd_to_owners(self, q, k, v, kb, vb, o, lse, dout, scale: float, dest_dq) -> Dict[str, torch.Tensor]:
+        """The backward with the dq exchange fused into the dQ reduce: dq rows go straight into
+        the owners' receive buffers (device addresses in dest_dq); returns dk, dv, dkb, dvb."""
+        g = self._bwd_buffers()
+        splitkv_bwd_delta(self.plan, o, dout, self._ws_bwd)
+        splitkv_bwd_partial(self.plan, q, k, v, lse, dout, g["dk"], g["dv"], scale, self._ws_bwd)
+        splitkv_bwd_reduce_to_owners(self.plan, q, kb, vb, lse, dout, g["dkb"], g["dvb"], scale, self._ws_bwd,
+                                     dest_dq)
         return g
 
     def sum(self, parts):
@@ -256,8 +269,17 @@ class SplitKVContextParallel:
         q_full, kb_full, vb_full = self._saved
         o_full, lse_full, dout_full = (self._gather_rows("o", o), self._gather_rows("lse", lse),
                                        self._gather_rows("dout", dout))
-        g = self.ops.local_bwd(q_full, k, v, kb_full, vb_full, o_full, lse_full, dout_full, scale)
-        out = {"dq": self.ops.sum(self._to_owners(g["dq"])), "dk": g["dk"], "dv": g["dv"]}
+        if self.exchange == "p2p":
+            b = self._p2p_buffers(dout.device)      # the forward's receive buffers take the dq rows
+            g = self.ops.local_bwd_to_owners(q_full, k, v, kb_full, vb_full, o_full, lse_full, dout_full, scale,
+                                             b["dest_o"])
+            self._stream_barrier(b["flag"])          # every rank's dq rows have landed
+            dq = self.ops.sum(b["o"])
+            self._stream_barrier(b["flag"])          # every owner has read before the next writes
+        else:
+            g = self.ops.local_bwd(q_full, k, v, kb_full, vb_full, o_full, lse_full, dout_full, scale)
+            dq = self.ops.sum(self._to_owners(g["dq"]))
+        out = {"dq": dq, "dk": g["dk"], "dv": g["dv"]}
         for n in ("dkb", "dvb"):
             out[n] = None if g[n] is None else g[n][self.rows]
         return out

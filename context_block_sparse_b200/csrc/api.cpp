@@ -175,6 +175,28 @@ int splitkv_bwd_reduce(const splitkv_plan_t* plan, const void* q, const void* kb
       static_cast<const void*>(w + L.dq_off), scale, dq, dkb, dvb, static_cast<cudaStream_t>(stream)));
 }
 
+int splitkv_bwd_reduce_to_owners(const splitkv_plan_t* plan, const void* q, const void* kb, const void* vb,
+                                 const float* lse, const void* dout, float* dkb, float* dvb, float scale,
+                                 const void* ws, size_t ws_bytes, int32_t num_ranks, int32_t rank,
+                                 float* const* dq_dest, void* stream) {
+  const DevPlan* dp = nullptr;
+  int st = check_plan(plan, &dp);
+  if (st != SPLITKV_OK) return st;
+  int R = 1, self = 0;
+  splitkv::plan_ranks(plan, &R, &self);
+  if (num_ranks != R || rank != self || !dq_dest || !aligned(dq_dest, 8)) return SPLITKV_ERR_INVALID_ARG;
+  if (!all_aligned16(q, dout, ws) || !block_ptrs_ok(dp, kb, vb, dkb, dvb) || !lse || !aligned(lse, 4))
+    return SPLITKV_ERR_INVALID_ARG;
+  const splitkv::BwdWs L = splitkv::bwd_ws_layout(dp->E, dp->Nq, dp->bs, dp->Hq, dp->d, rec_bytes(dp));
+  if (ws_bytes < L.total) return SPLITKV_ERR_WORKSPACE_TOO_SMALL;
+  const char* w = static_cast<const char*>(ws);
+  return cuda_status(splitkv::launch_bwd_reduce(
+      *dp, static_cast<const uint16_t*>(q), static_cast<const uint16_t*>(kb), static_cast<const uint16_t*>(vb),
+      static_cast<const uint16_t*>(dout), lse, reinterpret_cast<const float*>(w + L.delta_off),
+      static_cast<const void*>(w + L.dq_off), scale, nullptr, dkb, dvb, static_cast<cudaStream_t>(stream),
+      splitkv::MergeDest{dq_dest, nullptr, R, self}));
+}
+
 int splitkv_attn_bwd(const splitkv_plan_t* plan, const void* q, const void* k, const void* v, const void* kb,
                      const void* vb, const void* o, int o_dtype, const float* lse, const void* dout, float* dq,
                      float* dk, float* dv, float* dkb, float* dvb, float scale, void* ws, size_t ws_bytes,

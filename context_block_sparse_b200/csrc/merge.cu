@@ -142,6 +142,20 @@ __device__ __forceinline__ void stage_entries(int* sE, const int* __restrict__ e
   __syncthreads();
 }
 
+// Rows of block b under a MergeDest: the owner's index (into dest.o / dest.lse) and the
+// block's first row in the owner's [R][rows_owner] receive buffer, at slot dest.self.
+// ok = false only if the owner formula failed; then nothing is stored and the status
+// word records it.
+__device__ __forceinline__ int dest_of_block(const DevPlan& p, const MergeDest& dest, int b, size_t& row_base,
+                                             bool& ok) {
+  const int own = int((int64_t(b + 1) * dest.R - 1) / p.A);
+  const int lo = int(int64_t(own) * p.A / dest.R), hi = int(int64_t(own + 1) * p.A / dest.R);
+  ok = own >= 0 && own < dest.R && b >= lo && b < hi && dest.self >= 0 && dest.self < dest.R;
+  row_base = ok ? size_t(dest.self) * size_t(hi - lo) * p.bs + size_t(b - lo) * p.bs : 0;
+  if (!ok && threadIdx.x == 0) atomicCAS(p.status, 0, SPLITKV_ERR_INVALID_ARG);
+  return ok ? own : 0;
+}
+
 // ---------------------------------------------------------------------------
 // merge: grid (A, Hkv); smem kb/vb rows of the block (bf16), staged entry ids
 // ---------------------------------------------------------------------------
@@ -178,16 +192,9 @@ __global__ void __launch_bounds__(kMergeThreads, 2)
   size_t row_base = size_t(b) * p.bs;
   bool out_ok = true;
   if (dest.o != nullptr) {
-    const int own = int((int64_t(b + 1) * dest.R - 1) / p.A);
-    const int lo = int(int64_t(own) * p.A / dest.R), hi = int(int64_t(own + 1) * p.A / dest.R);
-    out_ok = own >= 0 && own < dest.R && b >= lo && b < hi && dest.self >= 0 && dest.self < dest.R;
-    if (out_ok) {
-      o_out = dest.o[own];
-      lse_out = dest.lse[own];
-      row_base = size_t(dest.self) * size_t(hi - lo) * p.bs + size_t(b - lo) * p.bs;
-    } else if (threadIdx.x == 0) {
-      atomicCAS(p.status, 0, SPLITKV_ERR_INVALID_ARG);   // never reached: the owner formula failed
-    }
+    const int own = dest_of_block(p, dest, b, row_base, out_ok);
+    o_out = dest.o[own];
+    lse_out = dest.lse[own];
     out_bf16 = 0;
   }
   for (int r0 = 0; r0 < R; r0 += kRowsPerPass) {
@@ -339,7 +346,7 @@ __global__ void __launch_bounds__(kMergeThreads, 2)
                       const uint16_t* __restrict__ vb, const uint16_t* __restrict__ dout,
                       const float* __restrict__ lse, const float* __restrict__ delta,
                       const void* __restrict__ dq_part, float scale, float* __restrict__ dq,
-                      float* __restrict__ dkb, float* __restrict__ dvb, int stage_rows) {
+                      float* __restrict__ dkb, float* __restrict__ dvb, int stage_rows, const MergeDest dest) {
   constexpr int NG = D / 16;
   using RecT = Rec<kBf16Rec>;
   constexpr int EG = 64 / (NG * RecT::RW);   // entries whose partials are in flight together
@@ -365,6 +372,11 @@ __global__ void __launch_bounds__(kMergeThreads, 2)
     *reinterpret_cast<uint4*>(sVb + t * D + ch * 8) = *reinterpret_cast<const uint4*>(vb + src);
   }
   const int n_block_keys = bterm ? bs : 0;   // none when they are context keys, or on another rank
+  // dq rows: the plan's own dq, or the owner's receive buffer (see MergeDest; dest.o)
+  float* dq_out = dq;
+  size_t dq_base = size_t(b) * bs;
+  bool dq_ok = true;
+  if (dest.o != nullptr) dq_out = dest.o[dest_of_block(p, dest, b, dq_base, dq_ok)];
   const float scale_log2 = scale * kLog2e;
   const int e0 = p.block_entry_ptr[b], n = p.block_entry_ptr[b + 1] - e0;
   // phase 1, a quad per row: P, dS of the in-block keys; dq = in-block dq + sum of partials
@@ -455,8 +467,8 @@ __global__ void __launch_bounds__(kMergeThreads, 2)
           }
       }
     }
-    if (active) {
-      float* dst = dq + qrow * D;
+    if (active && dq_ok) {
+      float* dst = dq_out + ((dq_base + tt) * p.Hq + head) * D;   // = dq + qrow * D for the plan's own dq
 #pragma unroll
       for (int k = 0; k < NG; ++k) *reinterpret_cast<float4*>(dst + 4 * (u + 4 * k)) = tot[k];
     }
@@ -514,7 +526,7 @@ cudaError_t merge_d(const DevPlan& p, const uint16_t* q, const uint16_t* kb, con
 template <int D, bool kBf16Rec>
 cudaError_t reduce_d(const DevPlan& p, const uint16_t* q, const uint16_t* kb, const uint16_t* vb,
                      const uint16_t* dout, const float* lse, const float* delta, const void* dq_part,
-                     float scale, float* dq, float* dkb, float* dvb, cudaStream_t s) {
+                     float scale, float* dq, float* dkb, float* dvb, cudaStream_t s, const MergeDest& dest) {
   const size_t rows = size_t(p.G) * p.bs;
   const size_t base =
       size_t(2) * p.bs * D * sizeof(uint16_t) + 2 * rows * p.bs * sizeof(float) + kEStage * sizeof(int);
@@ -525,7 +537,7 @@ cudaError_t reduce_d(const DevPlan& p, const uint16_t* q, const uint16_t* kb, co
                                        int(smem));
   if (e != cudaSuccess) return e;
   bwd_reduce_kernel<D, kBf16Rec><<<dim3(p.A, p.Hkv), kMergeThreads, smem, s>>>(
-      p, q, kb, vb, dout, lse, delta, dq_part, scale, dq, dkb, dvb, stage_rows);
+      p, q, kb, vb, dout, lse, delta, dq_part, scale, dq, dkb, dvb, stage_rows, dest);
   return cudaGetLastError();
 }
 
@@ -559,13 +571,13 @@ cudaError_t launch_bwd_delta(const DevPlan& p, const void* o, int o_bf16, const 
 cudaError_t launch_bwd_reduce(const DevPlan& p, const uint16_t* q, const uint16_t* kb,
                               const uint16_t* vb, const uint16_t* dout, const float* lse,
                               const float* delta, const void* dq_part, float scale, float* dq,
-                              float* dkb, float* dvb, cudaStream_t s) {
+                              float* dkb, float* dvb, cudaStream_t s, const MergeDest& dest) {
   if (p.partial_bf16) {
-    if (p.d == 64) return reduce_d<64, true>(p, q, kb, vb, dout, lse, delta, dq_part, scale, dq, dkb, dvb, s);
-    return reduce_d<128, true>(p, q, kb, vb, dout, lse, delta, dq_part, scale, dq, dkb, dvb, s);
+    if (p.d == 64) return reduce_d<64, true>(p, q, kb, vb, dout, lse, delta, dq_part, scale, dq, dkb, dvb, s, dest);
+    return reduce_d<128, true>(p, q, kb, vb, dout, lse, delta, dq_part, scale, dq, dkb, dvb, s, dest);
   }
-  if (p.d == 64) return reduce_d<64, false>(p, q, kb, vb, dout, lse, delta, dq_part, scale, dq, dkb, dvb, s);
-  return reduce_d<128, false>(p, q, kb, vb, dout, lse, delta, dq_part, scale, dq, dkb, dvb, s);
+  if (p.d == 64) return reduce_d<64, false>(p, q, kb, vb, dout, lse, delta, dq_part, scale, dq, dkb, dvb, s, dest);
+  return reduce_d<128, false>(p, q, kb, vb, dout, lse, delta, dq_part, scale, dq, dkb, dvb, s, dest);
 }
 
 }  // namespace splitkv

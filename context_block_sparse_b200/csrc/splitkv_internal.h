@@ -100,7 +100,8 @@ cudaError_t launch_fwd_partial(const DevPlan& p, const uint16_t* q, const uint16
 // rows of block b go to the receive buffers of the rank that owns b (blocks
 // [floor(r A / R), floor((r + 1) A / R)) to rank r) -- o[r] float32 [R][rows_r][Hq][d],
 // lse[r] [R][rows_r][Hq] -- at slot `self`; o and lse are device arrays of R pointers,
-// which may point into other GPUs' memory (peer-mapped).
+// which may point into other GPUs' memory (peer-mapped).  The dQ reduce uses o for its dq
+// rows (same layout) and ignores lse.
 struct MergeDest {
   float* const* o;
   float* const* lse;
@@ -128,7 +129,8 @@ cudaError_t launch_bwd_partial(const DevPlan& p, const uint16_t* q, const uint16
 cudaError_t launch_bwd_reduce(const DevPlan& p, const uint16_t* q, const uint16_t* kb,
                               const uint16_t* vb, const uint16_t* dout, const float* lse,
                               const float* delta, const void* dq_part, float scale, float* dq,
-                              float* dkb, float* dvb, cudaStream_t s);
+                              float* dkb, float* dvb, cudaStream_t s,
+                              const MergeDest& dest = MergeDest{nullptr, nullptr, 1, 0});
 
 // True when the tcgen05 forward and backward kernels serve this plan (and no
 // SPLITKV_FWD_KERNEL / SPLITKV_BWD_KERNEL override selects mma.sync): bf16

@@ -426,6 +426,19 @@ int splitkv_merge_to_owners(const splitkv_plan_t* plan, const void* q, const voi
                             float scale, const void* ws, size_t ws_bytes, int32_t num_ranks, int32_t rank,
                             float* const* o_dest, float* const* lse_dest, void* stream);
 
+/* splitkv_bwd_reduce of a rank plan with the dq exchange fused in: each block's dq rows
+ * (this rank's share: its chunk partials, plus the in-block term for its own blocks) go
+ * straight to the owner's receive buffer dq_dest[r] float32 [R][rows_r][Hq][d] at slot
+ * `rank` (the layout splitkv_sum_ranks reads on rank r); dkb, dvb as splitkv_bwd_reduce
+ * (rows of this rank's blocks).  dq_dest is a DEVICE array of R device pointers; as for
+ * splitkv_merge_to_owners, entries may be peer-mapped and the caller orders the owners'
+ * sums after every rank's call.  Errors: as splitkv_bwd_reduce, INVALID_ARG also for a
+ * rank mismatch or a NULL / misaligned pointer array. */
+int splitkv_bwd_reduce_to_owners(const splitkv_plan_t* plan, const void* q, const void* kb, const void* vb,
+                                 const float* lse, const void* dout, float* dkb, float* dvb, float scale,
+                                 const void* ws, size_t ws_bytes, int32_t num_ranks, int32_t rank,
+                                 float* const* dq_dest, void* stream);
+
 /* Exact combine of the ranks' results (news page, "Exchange the smaller side":
  * partials over disjoint key shares merged with their normalisation statistics).
  * o_parts [R][rows][head_dim] and lse_parts [R][rows] float32 (device; row =

@@ -191,6 +191,61 @@ def test_merge_to_owners_is_the_merge_laid_out_by_owner(splitkv, R, case):
         assert_close("LSE", lse.cpu().numpy().astype(np.float64), L[rows], TOL_LSE)
 
 
+@pytest.mark.parametrize("R,case", [(2, "tcgen05"), (3, "mma_d64")])
+def test_bwd_reduce_to_owners_is_the_reduce_laid_out_by_owner(splitkv, R, case):
+    """splitkv_bwd_reduce_to_owners (the dq exchange fused into the dQ reduce) stores every
+    rank's dq rows exactly as its plain backward writes them, in the owners' receive buffers
+    (bit for bit), and leaves dkb, dvb as the plain backward does; the owners' sums match
+    the oracle's dq."""
+    import torch
+    from context_block_sparse_b200.context_parallel import block_ranges
+    skv = splitkv
+    w = small() if case == "tcgen05" else small(Hq=4, Hkv=2, d=64)
+    t = {n: to_dev(b) for n, b in w.bits.items()}
+    Nq, N, Hq, Hkv, d, bs = w.num_queries, w.context_len, w.num_q_heads, w.num_kv_heads, w.head_dim, w.block_size
+    f32 = dict(dtype=torch.float32, device="cuda")
+    args = (w.sample_lens, w.anchors, bs, Hq, Hkv, d, w.kv_chunk, 148)
+    plans = [skv.splitkv_plan_shard(*args, R, r).upload() for r in range(R)]
+    o_parts = torch.empty((R, Nq, Hq, d), **f32)
+    l_parts = torch.empty((R, Nq, Hq), **f32)
+    for r, plan in enumerate(plans):
+        ws = torch.empty(skv.splitkv_workspace_size(plan, skv.WS_FWD), dtype=torch.uint8, device="cuda")
+        skv.splitkv_attn_fwd(plan, t["q"], t["k"], t["v"], w.scale, ws)
+        skv.splitkv_merge(plan, t["q"], t["kb"], t["vb"], w.scale, ws, o_parts[r], l_parts[r])
+    o = torch.empty((Nq, Hq, d), **f32)
+    lse = torch.empty((Nq, Hq), **f32)
+    skv.splitkv_combine_ranks(o_parts, l_parts, o, lse)
+    ranges = block_ranges(w.anchors.size, R)
+    recv = [torch.full((R, (hi - lo) * bs, Hq, d), float("nan"), **f32) for lo, hi in ranges]
+    dest = torch.tensor([x.data_ptr() for x in recv], dtype=torch.int64, device="cuda")
+    dq_loc = torch.empty((R, Nq, Hq, d), **f32)
+    for r, plan in enumerate(plans):
+        ws = torch.empty(skv.splitkv_workspace_size(plan, skv.WS_BWD), dtype=torch.uint8, device="cuda")
+        z = lambda shape: torch.zeros(shape, **f32)   # noqa: E731
+        g1 = {n: z(s) for n, s in (("dk", (N, Hkv, d)), ("dv", (N, Hkv, d)), ("dkb", (Nq, Hkv, d)),
+                                   ("dvb", (Nq, Hkv, d)))}
+        g2 = {n: z(x.shape) for n, x in g1.items()}
+        skv.splitkv_attn_bwd(plan, t["q"], t["k"], t["v"], t["kb"], t["vb"], o, lse, t["dout"], dq_loc[r],
+                             g1["dk"], g1["dv"], g1["dkb"], g1["dvb"], w.scale, ws)
+        skv.splitkv_bwd_delta(plan, o, t["dout"], ws)
+        skv.splitkv_bwd_partial(plan, t["q"], t["k"], t["v"], lse, t["dout"], g2["dk"], g2["dv"], w.scale, ws)
+        skv.splitkv_bwd_reduce_to_owners(plan, t["q"], t["kb"], t["vb"], lse, t["dout"], g2["dkb"], g2["dvb"],
+                                         w.scale, ws, dest)
+        torch.cuda.synchronize()
+        skv.splitkv_plan_status(plan)
+        for n in ("dkb", "dvb"):
+            assert torch.equal(g1[n], g2[n]), n
+    g = oracle_bwd(w)
+    for own, (lo, hi) in enumerate(ranges):
+        rows = slice(lo * bs, hi * bs)
+        assert torch.equal(recv[own], dq_loc[:, rows]), f"owner {own}: dq rows differ from the plain backward"
+        dq = torch.empty(((hi - lo) * bs, Hq, d), **f32)
+        skv.splitkv_sum_ranks(recv[own], dq)
+        assert_close("dq", dq.cpu().numpy().astype(np.float64), g["dq"][rows], TOL_OUT)
+    for plan in plans:
+        plan.destroy()
+
+
 def test_merge_to_owners_refuses_a_rank_mismatch(splitkv):
     import torch
     skv = splitkv
