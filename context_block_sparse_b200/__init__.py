@@ -427,6 +427,12 @@ def splitkv_bwd_reduce_to_owners(plan: Plan, q, kb, vb, lse, dout, dkb, dvb, sca
         _stream_ptr(stream)))
 
 
+def splitkv_enable_peer_access(peer_device: int) -> None:
+    """Let kernels on the current device access memory of `peer_device` (no-op when it is
+    the current device or access is already on)."""
+    _check("splitkv_enable_peer_access", _lib.splitkv_enable_peer_access(int(peer_device)))
+
+
 def splitkv_combine_ranks(o_parts, lse_parts, o, lse, stream=None) -> None:
     """o_parts [R, rows..., d] and lse_parts [R, rows...] float32 -> o [rows..., d] (float32 or
     bfloat16) and lse [rows...]: the exact combine of R ranks' results."""

@@ -35,7 +35,8 @@ import torch.distributed as dist
 
 from . import (
     EXPORT_CHUNK_OWNER, EXPORT_QUERY_SHARD, WS_BWD, WS_FWD, splitkv_attn_bwd, splitkv_attn_fwd, splitkv_bwd_delta,
-    splitkv_bwd_partial, splitkv_bwd_reduce_to_owners, splitkv_combine_ranks, splitkv_merge,
+    splitkv_bwd_partial, splitkv_bwd_reduce_to_owners, splitkv_combine_ranks, splitkv_enable_peer_access,
+    splitkv_merge,
     splitkv_merge_to_owners, splitkv_plan_shard, splitkv_sum_ranks, splitkv_workspace_size,
 )
 
@@ -234,6 +235,11 @@ class SplitKVContextParallel:
             peers, ptr_o, ptr_l = [], [], []
             for r, (ho, hl) in enumerate(handles):
                 to, tl = (recv_o, recv_l) if r == self.rank else (ho[0](*ho[1]), hl[0](*hl[1]))
+                if to.device != recv_o.device:
+                    # the IPC mapping is opened under the owner's device: this device's
+                    # kernels store into it only with peer access switched on here
+                    with torch.cuda.device(recv_o.device):
+                        splitkv_enable_peer_access(to.device.index)
                 peers.append((to, tl))          # keeps the mappings open
                 ptr_o.append(to.data_ptr())
                 ptr_l.append(tl.data_ptr())

@@ -105,6 +105,24 @@ extern "C" int splitkv_combine_ranks(int32_t num_ranks, int64_t rows, int32_t he
   return cudaGetLastError() == cudaSuccess ? SPLITKV_OK : SPLITKV_ERR_CUDA;
 }
 
+extern "C" int splitkv_enable_peer_access(int32_t peer_device) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return SPLITKV_ERR_CUDA;
+  if (peer_device == dev) return SPLITKV_OK;
+  int n = 0;
+  if (cudaGetDeviceCount(&n) != cudaSuccess) return SPLITKV_ERR_CUDA;
+  if (peer_device < 0 || peer_device >= n) return SPLITKV_ERR_INVALID_ARG;
+  int can = 0;
+  if (cudaDeviceCanAccessPeer(&can, dev, peer_device) != cudaSuccess) return SPLITKV_ERR_CUDA;
+  if (!can) return SPLITKV_ERR_UNSUPPORTED;
+  const cudaError_t e = cudaDeviceEnablePeerAccess(peer_device, 0);
+  if (e == cudaErrorPeerAccessAlreadyEnabled) {
+    cudaGetLastError();   // clear the (non-sticky) error the call left: access is on, as asked
+    return SPLITKV_OK;
+  }
+  return e == cudaSuccess ? SPLITKV_OK : SPLITKV_ERR_CUDA;
+}
+
 extern "C" int splitkv_sum_ranks(int32_t num_ranks, int64_t n, const float* parts, float* out, void* stream) {
   if (num_ranks < 1 || num_ranks > SPLITKV_MAX_RANKS || n < 0 || n % 4 || n > (int64_t(1) << 42))
     return SPLITKV_ERR_INVALID_ARG;

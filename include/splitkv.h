@@ -439,6 +439,12 @@ int splitkv_bwd_reduce_to_owners(const splitkv_plan_t* plan, const void* q, cons
                                  const void* ws, size_t ws_bytes, int32_t num_ranks, int32_t rank,
                                  float* const* dq_dest, void* stream);
 
+/* Let kernels on the current device read and write memory of `peer_device` (the receive
+ * buffers of splitkv_merge_to_owners / splitkv_bwd_reduce_to_owners when they live on
+ * another GPU, mapped here by CUDA IPC).  Already enabled counts as success.  Errors:
+ * INVALID_ARG (no such device), UNSUPPORTED (the two GPUs have no peer path), CUDA. */
+int splitkv_enable_peer_access(int32_t peer_device);
+
 /* Exact combine of the ranks' results (news page, "Exchange the smaller side":
  * partials over disjoint key shares merged with their normalisation statistics).
  * o_parts [R][rows][head_dim] and lse_parts [R][rows] float32 (device; row =

@@ -246,6 +246,14 @@ def test_bwd_reduce_to_owners_is_the_reduce_laid_out_by_owner(splitkv, R, case):
         plan.destroy()
 
 
+def test_enable_peer_access_on_one_gpu(splitkv):
+    """The current device needs nothing; a device that does not exist is refused."""
+    import torch
+    splitkv.splitkv_enable_peer_access(torch.cuda.current_device())
+    assert splitkv._lib.splitkv_enable_peer_access(torch.cuda.device_count() + 7) == -1
+    assert splitkv._lib.splitkv_enable_peer_access(-1) == -1
+
+
 def test_merge_to_owners_refuses_a_rank_mismatch(splitkv):
     import torch
     skv = splitkv
