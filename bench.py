@@ -447,7 +447,12 @@ def run_ours(args, world, rank, local):
     if not args.no_e2e:
         result["e2e"] = run_e2e(args, w, plan, dev, stream, flops_step, world=world)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        result["cpu_baseline"] = cpu_baseline(w, budget_s=args.cpu_seconds)
+        def gpu_rows(rows):
+            idx = torch.as_tensor(rows, device=dev)
+            return {n: x.index_select(0, idx).double().cpu().numpy()
+                    for n, x in (("o", o), ("lse", lse), ("dq", g["dq"]), ("dkb", g["dkb"]), ("dvb", g["dvb"]))}
+
+        result["cpu_baseline"] = cpu_baseline(w, budget_s=args.cpu_seconds, gpu_rows=gpu_rows)
     if world > 1:
         dist.destroy_process_group()
     return result if rank == 0 else None
@@ -718,8 +723,9 @@ def _oracle_threads():
         return os.cpu_count() or 1
 
 
-def _oracle_blocks(w, budget_s: float, start: int = 0, stride: int = 37):
-    """Run the oracle forward + backward block by block until budget_s elapses; returns (flops, seconds, n)."""
+def _oracle_blocks(w, budget_s: float, start: int = 0, stride: int = 37, keep=None):
+    """Run the oracle forward + backward block by block until budget_s elapses; returns (flops, seconds, n).
+    keep: a list that receives (block, O, LSE, dq, dkb, dvb) of every block's rows."""
     from oracle import attention as oatt
     from oracle import mask as omask
     f = {n: w.f64(n) for n in ("q", "k", "v", "kb", "vb", "dout")}
@@ -730,10 +736,13 @@ def _oracle_blocks(w, budget_s: float, start: int = 0, stride: int = 37):
     t0 = time.perf_counter()
     b = start % A
     while True:
-        oatt.attention_fwd(f["q"], f["k"], f["v"], f["kb"], f["vb"], w.sample_lens, w.anchors, w.block_size,
-                           w.scale, blocks=[b])
-        oatt.attention_bwd(f["q"], f["k"], f["v"], f["kb"], f["vb"], f["dout"], w.sample_lens, w.anchors,
-                           w.block_size, w.scale, blocks=[b])
+        O, L = oatt.attention_fwd(f["q"], f["k"], f["v"], f["kb"], f["vb"], w.sample_lens, w.anchors,
+                                  w.block_size, w.scale, blocks=[b])
+        g = oatt.attention_bwd(f["q"], f["k"], f["v"], f["kb"], f["vb"], f["dout"], w.sample_lens, w.anchors,
+                               w.block_size, w.scale, blocks=[b])
+        if keep is not None:
+            r = slice(b * w.block_size, (b + 1) * w.block_size)
+            keep.append((b, O[r], L[r], g["dq"][r], g["dkb"][r], g["dvb"][r]))
         S, a = iv[b]
         flops += 14.0 * w.head_dim * w.num_q_heads * w.block_size * ((a - S) + w.block_size)
         n += 1
@@ -743,12 +752,28 @@ def _oracle_blocks(w, budget_s: float, start: int = 0, stride: int = 37):
     return flops, time.perf_counter() - t0, n
 
 
-def cpu_baseline(w, budget_s=15.0):
-    flops, secs, n = _oracle_blocks(w, budget_s)
+def cpu_baseline(w, budget_s=15.0, gpu_rows=None):
+    """The oracle timed on a bounded sample of the workload; with gpu_rows (rows -> the GPU's
+    o, lse, dq, dkb, dvb on those query rows) also the GPU's error on the sampled blocks."""
+    keep = [] if gpu_rows is not None else None
+    flops, secs, n = _oracle_blocks(w, budget_s, keep=keep)
     out = {"value": flops / secs / 1e12, "unit": "TFLOP/s", "cores": _oracle_threads(), "kind": "oracle",
            "sample": f"fp64 numpy oracle, forward + backward of {n} of {w.anchors.size} anchor blocks "
                      f"(every 37th, all {w.num_q_heads} heads), {secs:.1f} s; same masked-pair FLOP count",
            "host_cpu_count": os.cpu_count()}
+    if keep:
+        err = {n: 0.0 for n in ("o", "lse", "dq", "dkb", "dvb")}
+        ref = dict(err)
+        for b, *want in keep:
+            got = gpu_rows(np.arange(b * w.block_size, (b + 1) * w.block_size))
+            for name, x in zip(("o", "lse", "dq", "dkb", "dvb"), want):
+                err[name] = max(err[name], float(np.abs(got[name] - x).max()))
+                ref[name] = max(ref[name], float(np.abs(x).max()))
+        out["parity_sample"] = {
+            "blocks": len(keep), "max_abs": err,
+            "max_abs_over_max_oracle": {k: err[k] / ref[k] if ref[k] else 0.0 for k in err},
+            "tolerance": {"o": 2e-2, "dq": 2e-2, "dkb": 2e-2, "dvb": 2e-2, "lse": 1e-3},
+            "what": "the last timed step's outputs against the fp64 oracle on the sampled blocks' rows"}
     # the same oracle on one thread, on a shorter sample
     try:
         from threadpoolctl import threadpool_limits

@@ -110,3 +110,27 @@ def test_rank_emulation_option():
     assert not bench.parse_args(["--schedule", "contiguous"]).dynamic_claim
     assert callable(bench.run_split_kv)
     assert bench.parse_args(["--split-kv", "--exchange", "p2p"]).exchange == "p2p"
+
+
+def test_cpu_baseline_reports_the_error_on_its_sample():
+    """With the GPU's rows supplied, the oracle leg also reports their error on the blocks
+    it computed (here: the oracle's own rows, exact, then a copy off by 0.5 in dq)."""
+    sys.path.insert(0, ROOT)
+    import numpy as np
+    import bench
+    from oracle import attention as oatt
+    from synth import make_workload
+    w = make_workload("tiny", with_grad=True)
+    f = {n: w.f64(n) for n in ("q", "k", "v", "kb", "vb", "dout")}
+    O, L = oatt.attention_fwd(f["q"], f["k"], f["v"], f["kb"], f["vb"], w.sample_lens, w.anchors, w.block_size,
+                              w.scale)
+    g = oatt.attention_bwd(f["q"], f["k"], f["v"], f["kb"], f["vb"], f["dout"], w.sample_lens, w.anchors,
+                           w.block_size, w.scale)
+    full = {"o": O, "lse": L, "dq": g["dq"], "dkb": g["dkb"], "dvb": g["dvb"]}
+    exact = bench.cpu_baseline(w, budget_s=0.2, gpu_rows=lambda rows: {n: x[rows] for n, x in full.items()})
+    ps = exact["parity_sample"]
+    assert ps["blocks"] >= 1 and all(v < 1e-12 for v in ps["max_abs"].values())
+    off = dict(full, dq=full["dq"] + 0.5)
+    bad = bench.cpu_baseline(w, budget_s=0.2, gpu_rows=lambda rows: {n: x[rows] for n, x in off.items()})
+    assert abs(bad["parity_sample"]["max_abs"]["dq"] - 0.5) < 1e-9
+    assert bad["parity_sample"]["max_abs"]["o"] < 1e-12
