@@ -742,7 +742,8 @@ def _oracle_blocks(w, budget_s: float, start: int = 0, stride: int = 37, keep=No
                                w.block_size, w.scale, blocks=[b])
         if keep is not None:
             r = slice(b * w.block_size, (b + 1) * w.block_size)
-            keep.append((b, O[r], L[r], g["dq"][r], g["dkb"][r], g["dvb"][r]))
+            # copies: views would keep the oracle's full-size arrays of every block alive
+            keep.append((b, O[r].copy(), L[r].copy(), g["dq"][r].copy(), g["dkb"][r].copy(), g["dvb"][r].copy()))
         S, a = iv[b]
         flops += 14.0 * w.head_dim * w.num_q_heads * w.block_size * ((a - S) + w.block_size)
         n += 1
