@@ -264,3 +264,23 @@ def test_lpt_ownership_beats_contiguous_on_a_skewed_context():
     con_own = cp.chunk_owners_contiguous(n, R)
     assert max(loads(con_own)) == sum(pairs)
     assert max(loads(con_own)) > 3 * max(loads(lpt_own))
+
+
+def test_planted_backward_mistake_is_caught():
+    """A rank backward that normalises with its own LSE_r instead of the final LSE (a
+    plausible slip: each rank has its LSE_r at hand) no longer sums to the unsplit dq."""
+    lens, anchors, bs, t = _problem(3, Hq=4, Hkv=2)
+    C, scale, R = 6, 0.31, 3
+    owner = cp.chunk_owners(lens, anchors, bs, C, 4, R)
+    O, L = att.attention_fwd(t["q"], t["k"], t["v"], t["kb"], t["vb"], lens, anchors, bs, scale)
+    g = att.attention_bwd(t["q"], t["k"], t["v"], t["kb"], t["vb"], t["dout"], lens, anchors, bs, scale)
+    right = sum(cp.rank_bwd(t["q"], t["k"], t["v"], t["kb"], t["vb"], t["dout"], O, L, lens, anchors, bs, C,
+                            scale, owner, r, R)["dq"] for r in range(R))
+    np.testing.assert_allclose(right, g["dq"], rtol=0, atol=1e-12)
+    wrong = 0
+    for r in range(R):
+        O_r, L_r = cp.rank_fwd(t["q"], t["k"], t["v"], t["kb"], t["vb"], lens, anchors, bs, C, scale, owner, r, R)
+        L_r = np.where(np.isfinite(L_r), L_r, 0.0)
+        wrong = wrong + cp.rank_bwd(t["q"], t["k"], t["v"], t["kb"], t["vb"], t["dout"], O, L_r, lens, anchors,
+                                    bs, C, scale, owner, r, R)["dq"]
+    assert np.abs(wrong - g["dq"]).max() > 1e-3
