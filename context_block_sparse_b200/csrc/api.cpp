@@ -7,46 +7,20 @@
 #include "splitkv.h"
 #include "splitkv_internal.h"
 
-namespace splitkv {
-const DevPlan* plan_device_view(const splitkv_plan_t* P);
-}
-
 namespace {
 
+using splitkv::all_aligned16;
+using splitkv::block_ptrs_ok;
+using splitkv::check_plan;
 using splitkv::DevPlan;
+using splitkv::rec_bytes;
 
-bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
-
-// Shared checks of every attention call; on success *out points at the device view.
-int check_plan(const splitkv_plan_t* plan, const DevPlan** out) {
-  if (!plan) return SPLITKV_ERR_INVALID_ARG;
-  const DevPlan* dp = splitkv::plan_device_view(plan);
-  if (!dp) return SPLITKV_ERR_NOT_UPLOADED;
-  if (dp->d != 64 && dp->d != 128) return SPLITKV_ERR_UNSUPPORTED;
-  if ((dp->partial_bf16 || dp->dynamic) && !splitkv::tcgen05_supported(*dp)) return SPLITKV_ERR_UNSUPPORTED;
-  *out = dp;
-  return SPLITKV_OK;
-}
-
-size_t rec_bytes(const DevPlan* dp) { return dp->partial_bf16 ? 2 : 4; }
+bool aligned(const void* p, uintptr_t a) { return splitkv::ptr_aligned(p, a); }
 
 int cuda_status(cudaError_t e) {
   if (e == cudaSuccess) return SPLITKV_OK;
   cudaGetLastError();
   return SPLITKV_ERR_CUDA;
-}
-
-template <typename... Ps>
-bool all_aligned16(Ps... ps) {
-  return ((ps != nullptr && aligned(ps, 16)) && ...);
-}
-
-// Block-key tensors (kb, vb, dkb, dvb): required under reading A; under reading B
-// they may be NULL (never read or written) and are checked only for alignment.
-template <typename... Ps>
-bool block_ptrs_ok(const DevPlan* dp, Ps... ps) {
-  if (dp->block_term) return all_aligned16(ps...);
-  return ((ps == nullptr || aligned(ps, 16)) && ...);
 }
 
 }  // namespace

@@ -132,9 +132,42 @@ cudaError_t launch_bwd_reduce(const DevPlan& p, const uint16_t* q, const uint16_
                               float* dkb, float* dvb, cudaStream_t s,
                               const MergeDest& dest = MergeDest{nullptr, nullptr, 1, 0});
 
+// ---- argument checks shared by the C-ABI entry points (api.cpp, static_scratch.cu)
+const DevPlan* plan_device_view(const splitkv_plan_t* P);
+
+inline bool ptr_aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+// Non-null and 16-byte aligned, every one of them.
+template <typename... Ps>
+inline bool all_aligned16(Ps... ps) {
+  return ((ps != nullptr && ptr_aligned(ps, 16)) && ...);
+}
+
+// Block-key tensors (kb, vb, dkb, dvb): required under reading A; under reading B
+// they may be NULL (never read or written) and are checked only for alignment.
+template <typename... Ps>
+inline bool block_ptrs_ok(const DevPlan* dp, Ps... ps) {
+  if (dp->block_term) return all_aligned16(ps...);
+  return ((ps == nullptr || ptr_aligned(ps, 16)) && ...);
+}
+
+// Bytes of one O_c / dQ-partial element of the plan's records.
+inline size_t rec_bytes(const DevPlan* dp) { return dp->partial_bf16 ? 2 : 4; }
+
 // True when the tcgen05 forward and backward kernels serve this plan (and no
 // SPLITKV_FWD_KERNEL / SPLITKV_BWD_KERNEL override selects mma.sync): bf16
 // partial records and run-time claims exist on those kernels only.
 bool tcgen05_supported(const DevPlan& p);
+
+// Checks every attention call shares; on success *out points at the plan's device view.
+inline int check_plan(const splitkv_plan_t* plan, const DevPlan** out) {
+  if (!plan) return SPLITKV_ERR_INVALID_ARG;
+  const DevPlan* dp = plan_device_view(plan);
+  if (!dp) return SPLITKV_ERR_NOT_UPLOADED;
+  if (dp->d != 64 && dp->d != 128) return SPLITKV_ERR_UNSUPPORTED;
+  if ((dp->partial_bf16 || dp->dynamic) && !tcgen05_supported(*dp)) return SPLITKV_ERR_UNSUPPORTED;
+  *out = dp;
+  return SPLITKV_OK;
+}
 
 }  // namespace splitkv

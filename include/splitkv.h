@@ -43,7 +43,12 @@
  *   - Workspaces are caller-allocated device memory of at least the size
  *     splitkv_workspace_size reports; the library allocates no per-call memory.
  *   - Calls that share a plan or a workspace must not run concurrently on
- *     different streams.
+ *     different streams.  A plan's device memory holds the run-time claim
+ *     cursors of its partial kernels (SPLITKV_FLAG_DYNAMIC_CLAIM: reset before,
+ *     and advanced by, every launch) and its status words, so two launches of
+ *     one plan in flight at once take items from each other's lists (items are
+ *     skipped or run twice) even when their tensors and workspaces differ: give
+ *     each concurrent stream its own plan.
  */
 #ifndef SPLITKV_H_
 #define SPLITKV_H_
@@ -382,15 +387,20 @@ int splitkv_bwd_dq(const splitkv_plan_t* plan, const void* q, const void* k, con
  * synchronisation, plug-ins handed raw pointers without an allocator).
  * The caller passes the inputs and outputs exactly as for splitkv_attn_fwd and
  * splitkv_merge; the plan must already have its device copy
- * (splitkv_plan_upload, a set-up step) on the current device.  The first call
- * on a device looks up the buffer's device address (cudaGetSymbolAddress),
- * so make that first call before any stream capture.  Every call shares the one
- * buffer, and calls whose kernels overlap on the GPU (different streams, or
- * different host threads) race on it: serialise them.  Each call writes every
- * record it reads, so left-over contents of an earlier call are never used.
- * Errors: as splitkv_merge, plus WORKSPACE_TOO_SMALL when the problem's forward
- * workspace (splitkv_workspace_size, SPLITKV_WS_FWD) exceeds
- * SPLITKV_STATIC_SCRATCH_BYTES. */
+ * (splitkv_plan_upload, a set-up step) in the CUDA context current at the
+ * call.  The first call in a context looks up the buffer's device address
+ * (cudaGetSymbolAddress; cached per context, keyed by the context's id, so a
+ * caller's own driver-API context or a re-created primary context gets its
+ * own lookup), so make that first call before any stream capture.  Every call
+ * shares the one buffer, and calls whose kernels overlap on the GPU (different
+ * streams, or different host threads) race on it: serialise them.  Each call
+ * writes every record it reads, so left-over contents of an earlier call are
+ * never used.
+ * Errors: INVALID_ARG, NOT_UPLOADED and UNSUPPORTED as splitkv_merge;
+ * WORKSPACE_TOO_SMALL when the problem's forward workspace
+ * (splitkv_workspace_size, SPLITKV_WS_FWD) exceeds SPLITKV_STATIC_SCRATCH_BYTES
+ * (checked before any CUDA call); CUDA when the current context cannot be
+ * queried, the buffer's address cannot be looked up, or a launch fails. */
 int splitkv_attn_fwd_static_scratch(const splitkv_plan_t* plan, const void* q, const void* k,
                                     const void* v, const void* kb, const void* vb, float scale,
                                     void* o, int o_dtype, float* lse, void* stream);
