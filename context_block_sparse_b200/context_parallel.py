@@ -231,10 +231,14 @@ class SplitKVContextParallel:
             recv_o = torch.zeros((self.R, mine, self.Hq, self.d), **f32)
             recv_l = torch.zeros((self.R, mine, self.Hq), **f32)
             handles = [None] * self.R
-            dist.all_gather_object(handles, (reduce_tensor(recv_o), reduce_tensor(recv_l)), group=self.group)
+            if self.R > 1:
+                # one-rank groups share nothing: an IPC handle that no other process opens
+                # would stay registered with torch's producer-side reference count until exit
+                dist.all_gather_object(handles, (reduce_tensor(recv_o), reduce_tensor(recv_l)),
+                                       group=self.group)
             peers, ptr_o, ptr_l = [], [], []
-            for r, (ho, hl) in enumerate(handles):
-                to, tl = (recv_o, recv_l) if r == self.rank else (ho[0](*ho[1]), hl[0](*hl[1]))
+            for r, h in enumerate(handles):
+                to, tl = (recv_o, recv_l) if r == self.rank else (h[0][0](*h[0][1]), h[1][0](*h[1][1]))
                 if to.device != recv_o.device:
                     # the IPC mapping is opened under the owner's device: this device's
                     # kernels store into it only with peer access switched on here
