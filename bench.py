@@ -452,7 +452,12 @@ def run_ours(args, world, rank, local):
             return {n: x.index_select(0, idx).double().cpu().numpy()
                     for n, x in (("o", o), ("lse", lse), ("dq", g["dq"]), ("dkb", g["dkb"]), ("dvb", g["dvb"]))}
 
-        result["cpu_baseline"] = cpu_baseline(w, budget_s=args.cpu_seconds, gpu_rows=gpu_rows)
+        def gpu_keys(keys):
+            idx = torch.as_tensor(keys, device=dev)
+            return {n: g[n].index_select(0, idx).double().cpu().numpy() for n in ("dk", "dv")}
+
+        result["cpu_baseline"] = cpu_baseline(w, budget_s=args.cpu_seconds, gpu_rows=gpu_rows,
+                                              gpu_keys=gpu_keys)
     if world > 1:
         dist.destroy_process_group()
     return result if rank == 0 else None
@@ -753,9 +758,53 @@ def _oracle_blocks(w, budget_s: float, start: int = 0, stride: int = 37, keep=No
     return flops, time.perf_counter() - t0, n
 
 
-def cpu_baseline(w, budget_s=15.0, gpu_rows=None):
+def parity_chunks(w):
+    """KV chunks whose dK, dV the oracle checks at full size, with the blocks that read them:
+    the last chunk of the first and of a middle sample (few readers each) and the first chunk
+    of the shortest sample (read by every block of that sample, so its gradient sums many
+    blocks).  Returns (chunks, reader blocks, key positions)."""
+    from oracle import mask as omask
+    C = w.kv_chunk
+    starts = list(omask.sample_starts(w.sample_lens)) + [w.context_len]
+
+    def last_inside(s):     # the last chunk inside sample s (else the one holding its last key)
+        c = starts[s + 1] // C - 1
+        return c if c * C >= starts[s] else (starts[s + 1] - 1) // C
+
+    def first_inside(s):    # the first chunk inside sample s (else the one holding its first key)
+        c = -(-starts[s] // C)
+        return c if (c + 1) * C <= starts[s + 1] else starts[s] // C
+
+    mid = len(w.sample_lens) // 2
+    short = int(np.argmin(w.sample_lens))
+    chunks = sorted({last_inside(0), last_inside(mid), first_inside(short)})
+    iv = omask.context_interval(w.sample_lens, w.anchors)
+    readers = [b for b, (S, a) in enumerate(iv) if any(S < (c + 1) * C and a > c * C for c in chunks)]
+    keys = np.concatenate([np.arange(c * C, min((c + 1) * C, w.context_len)) for c in chunks])
+    return chunks, readers, keys
+
+
+def _dkdv_parity(w, gpu_keys):
+    """The GPU's dK, dV on the keys of parity_chunks(w) against the oracle's, which sums
+    the backward of every block that reads them (untimed)."""
+    from oracle import attention as oatt
+    chunks, readers, keys = parity_chunks(w)
+    f = {n: w.f64(n) for n in ("q", "k", "v", "kb", "vb", "dout")}
+    g = oatt.attention_bwd(f["q"], f["k"], f["v"], f["kb"], f["vb"], f["dout"], w.sample_lens, w.anchors,
+                           w.block_size, w.scale, blocks=readers)
+    got = gpu_keys(keys)
+    err = {n: float(np.abs(got[n] - g[n][keys]).max()) for n in ("dk", "dv")}
+    ref = {n: float(np.abs(g[n][keys]).max()) for n in ("dk", "dv")}
+    return {"chunks": [int(c) for c in chunks], "reader_blocks": len(readers), "keys": int(keys.size),
+            "max_abs": err, "max_abs_over_max_oracle": {n: err[n] / ref[n] if ref[n] else 0.0 for n in err},
+            "tolerance": {"dk": 2e-2, "dv": 2e-2}}
+
+
+def cpu_baseline(w, budget_s=15.0, gpu_rows=None, gpu_keys=None):
     """The oracle timed on a bounded sample of the workload; with gpu_rows (rows -> the GPU's
-    o, lse, dq, dkb, dvb on those query rows) also the GPU's error on the sampled blocks."""
+    o, lse, dq, dkb, dvb on those query rows) also the GPU's error on the sampled blocks, and
+    with gpu_keys (key positions -> the GPU's dk, dv there) its dK, dV error on the keys of a
+    few chunks (parity_chunks)."""
     keep = [] if gpu_rows is not None else None
     flops, secs, n = _oracle_blocks(w, budget_s, keep=keep)
     out = {"value": flops / secs / 1e12, "unit": "TFLOP/s", "cores": _oracle_threads(), "kind": "oracle",
@@ -778,6 +827,11 @@ def cpu_baseline(w, budget_s=15.0, gpu_rows=None):
                 "what": "the last timed step's outputs against the fp64 oracle on the sampled blocks' rows"}
         except Exception as e:      # a report, never a reason to lose the bench line
             out["parity_sample"] = {"error": f"{type(e).__name__}: {e}"}
+    if gpu_keys is not None and "parity_sample" in out:
+        try:
+            out["parity_sample"]["dkdv"] = _dkdv_parity(w, gpu_keys)
+        except Exception as e:      # a report, never a reason to lose the bench line
+            out["parity_sample"]["dkdv"] = {"error": f"{type(e).__name__}: {e}"}
     # the same oracle on one thread, on a shorter sample
     try:
         from threadpoolctl import threadpool_limits

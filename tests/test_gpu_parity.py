@@ -345,10 +345,14 @@ def test_skew_fwd_sampled(splitkv):
 
 
 def test_bwd_config_sampled(splitkv):
-    """fwd+bwd at 64k context / 8k queries: O, LSE, dQ, dKb, dVb on sampled blocks; dK, dV on the keys of
-    sampled chunks, with the oracle summing over every block that reads them."""
+    """fwd+bwd at 64k context / 8k queries in the bench's launch configuration (query slices of
+    two tiles, backward LPT by tile cost, run-time claims): O, LSE, dQ, dKb, dVb on sampled
+    blocks; dK, dV on the keys of three chunks (the bench's parity chunks: two read by few
+    blocks, one read by every block of the shortest sample), with the oracle summing over every
+    block that reads them."""
+    from bench import parity_chunks
     w = make_workload("bwd")
-    out, _, _ = run(w, bwd=True)
+    out, _, _ = run(w, bwd=True, dynamic_claim=True, q_slice=2, tile_cost=True)
     blocks = _sample_blocks(w, n=6)
     _check_fwd(w, out, blocks)
     g = oracle_bwd(w, blocks)
@@ -356,19 +360,27 @@ def test_bwd_config_sampled(splitkv):
     rows = np.concatenate([np.arange(b * bs, (b + 1) * bs) for b in blocks])
     for n in ("dq", "dkb", "dvb"):
         assert_close(n, out[n][rows], g[n][rows], TOL_OUT)
-    # dK, dV on two chunks: the last chunks of the first and of a middle sample (few readers each)
-    C = w.kv_chunk
-    starts = omask.sample_starts(w.sample_lens) + [w.context_len]
-    mid = len(w.sample_lens) // 2
-    chunks = sorted({(starts[1] - 1) // C, (starts[mid + 1] - 1) // C})
-    iv = omask.context_interval(w.sample_lens, w.anchors)
-    readers = [b for b, (S, a) in enumerate(iv) if any(S < (c + 1) * C and a > c * C for c in chunks)]
+    chunks, readers, keys = parity_chunks(w)
+    assert len(chunks) == 3 and len(readers) > 0
     g2 = oracle_bwd(w, readers)
-    keys = np.concatenate([np.arange(c * C, min((c + 1) * C, w.context_len)) for c in chunks])
     for n in ("dk", "dv"):
         assert_close(n, out[n][keys], g2[n][keys], TOL_OUT)
     for n in ("dq", "dk", "dv", "dkb", "dvb"):
         assert np.isfinite(out[n]).all(), n
+
+
+def test_bwd_config_static_schedule_sampled(splitkv):
+    """The same workload on the library's default schedule (static worker lists, pair cost,
+    no slices): sampled rows and the dK, dV of the parity chunks against the oracle."""
+    from bench import parity_chunks
+    w = make_workload("bwd")
+    out, _, _ = run(w, bwd=True)
+    blocks = _sample_blocks(w, n=3, seed=11)
+    _check_fwd(w, out, blocks)
+    chunks, readers, keys = parity_chunks(w)
+    g2 = oracle_bwd(w, readers)
+    for n in ("dk", "dv"):
+        assert_close(n, out[n][keys], g2[n][keys], TOL_OUT)
 
 
 def test_cta_timers_recorded(splitkv):
