@@ -353,28 +353,35 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (!mbar_wait(&B->kv_full, kt_count & 1, wctx, 2 * 10000 + __LINE__)) { ok = false; break; }
           tc_fence_after();
           int u = 0;
+          bool s_issued = false;   // S^T of this pair was issued ahead, right after the previous dV
           for (int t = item.z; t < item.w; ++t) {
             const int4 tile = p.tiles[t];
             if (!(tile.z < k0 + BT && tile.w > k0)) continue;
             const int s = qd_count & 1;
-            if (!mbar_wait(&B->qd_full[s], (qd_count >> 1) & 1, wctx, 2 * 10000 + __LINE__)) { ok = false; break; }
-            tc_fence_after();
-            // S^T = K Q^T (cols 0..127), dP^T = V dO^T (cols 128..255); the P^T pass
-            // starts when S^T lands, while dP^T is still being computed
-            for (int kk = 0; kk < D / 16; ++kk)
-              mma_ss(tmem + 0, kmajor(aK, kk), kmajor(aQ + s * kTile, kk), kIdescKM, kk > 0 ? 1u : 0u);
-            mma_commit(&B->st_ready);
+            if (!s_issued) {
+              if (!mbar_wait(&B->qd_full[s], (qd_count >> 1) & 1, wctx, 2 * 10000 + __LINE__)) { ok = false; break; }
+              tc_fence_after();
+              // S^T = K Q^T (cols 0..127); the P^T pass starts when it lands
+              for (int kk = 0; kk < D / 16; ++kk)
+                mma_ss(tmem + 0, kmajor(aK, kk), kmajor(aQ + s * kTile, kk), kIdescKM, kk > 0 ? 1u : 0u);
+              mma_commit(&B->st_ready);
+            }
+            s_issued = false;
+            // dP^T = V dO^T (cols 128..255): after dK of the previous pair, which read dS^T there
             for (int kk = 0; kk < D / 16; ++kk)
               mma_ss(tmem + 128, kmajor(aV, kk), kmajor(adO + s * kTile, kk), kIdescKM, kk > 0 ? 1u : 0u);
             mma_commit(&B->dpt_ready);
-            {   // K and V are read only by S^T / dP^T: release them after the key tile's last pair
-              bool later = false;
-              for (int t2 = t + 1; t2 < item.w && !later; ++t2) {
-                const int4 tl2 = p.tiles[t2];
-                later = tl2.z < k0 + BT && tl2.w > k0;
+            // the next pair of this key tile, if any
+            int tn = -1;
+            for (int t2 = t + 1; t2 < item.w; ++t2) {
+              const int4 tl2 = p.tiles[t2];
+              if (tl2.z < k0 + BT && tl2.w > k0) {
+                tn = t2;
+                break;
               }
-              if (!later) mma_commit(&B->kv_empty);
             }
+            // K and V are read only by S^T / dP^T: release them after the key tile's last pair
+            if (tn < 0) mma_commit(&B->kv_empty);
             if (!mbar_wait(&B->pt_ready, pds_cnt & 1, wctx, 2 * 10000 + __LINE__)) { ok = false; break; }
             if (u == 0) {
               if (!mbar_wait(&B->dkv_free, (dkvf_cnt & 1) ^ 1, wctx, 2 * 10000 + __LINE__)) { ok = false; break; }
@@ -385,6 +392,18 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int kk = 0; kk < BT / 16; ++kk)
               mma_ts(tmem + 384, tmem + 0 + packed_col(kk), mnmajor(adO + s * kTile, kk), kIdescMN,
                      (u > 0 || kk > 0) ? 1u : 0u);
+            if (tn >= 0) {
+              // the next pair's S^T right behind dV, which is the last reader of this pair's
+              // P^T in cols 0..127 (the dS^T pass keeps P in registers): its P^T pass can then
+              // start as soon as the element-wise warps finish this pair, while dK runs
+              const int s1 = (qd_count + 1) & 1;
+              if (!mbar_wait(&B->qd_full[s1], ((qd_count + 1) >> 1) & 1, wctx, 2 * 10000 + __LINE__)) { ok = false; break; }
+              tc_fence_after();
+              for (int kk = 0; kk < D / 16; ++kk)
+                mma_ss(tmem + 0, kmajor(aK, kk), kmajor(aQ + s1 * kTile, kk), kIdescKM, kk > 0 ? 1u : 0u);
+              mma_commit(&B->st_ready);
+              s_issued = true;
+            }
             if (!mbar_wait(&B->dst_ready, pds_cnt & 1, wctx, 2 * 10000 + __LINE__)) { ok = false; break; }
             ++pds_cnt;
             tc_fence_after();
