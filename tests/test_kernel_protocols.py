@@ -212,7 +212,8 @@ class Forward(Core):
 
 
 # ---------------------------------------------------------------------------
-# dK/dV kernel: K, V stationary per key tile, Q / dO double-buffered per pair
+# dK/dV kernel: K, V stationary per key tile, Q / dO double-buffered per pair; within a
+# key tile the next pair's S^T is issued right after this pair's dV
 # ---------------------------------------------------------------------------
 class DKDV(Core):
     def __init__(self, ktiles, seed, drop=None):
@@ -255,24 +256,30 @@ class DKDV(Core):
         q, pds, tiles_done = 0, 0, 0
         for k, n in enumerate(self.kt):
             yield from self.wait("kv_full", k)
+            s_issued = False      # S^T of this pair issued ahead, right after the previous dV
+
+            def st_mma(qq, k=k):
+                def st(qq=qq, ss=qq % 2, k=k):
+                    self.check(self.KV == k and self.Q[ss] == qq, f"S^T({qq}) reads KV {self.KV} Q {self.Q[ss]}")
+                    self.check(self.ST is None or self.ST[0] == "read", f"S^T({qq}) overwrites {self.ST}")
+                    self.ST = ("S", qq)
+                self.mma(st)
+                self.commit("st_ready")
             for u in range(n):
                 s = q % 2
-                yield from self.wait(f"qd_full{s}", q // 2)
-
-                def st(q=q, s=s, k=k):
-                    self.check(self.KV == k and self.Q[s] == q, f"S^T({q}) reads KV {self.KV} Q {self.Q[s]}")
-                    self.check(self.ST is None or self.ST[0] == "read", f"S^T({q}) overwrites {self.ST}")
-                    self.ST = ("S", q)
+                if not s_issued:
+                    yield from self.wait(f"qd_full{s}", q // 2)
+                    st_mma(q)
+                s_issued = False
 
                 def dpt(q=q, s=s, k=k):
                     self.check(self.KV == k and self.Q[s] == q, f"dP^T({q}) reads KV {self.KV} Q {self.Q[s]}")
                     self.check(self.DP is None or self.DP[0] == "read", f"dP^T({q}) overwrites {self.DP}")
                     self.DP = ("dP", q)
-                self.mma(st)
-                self.commit("st_ready")
                 self.mma(dpt)
                 self.commit("dpt_ready")
-                if u + 1 == n:
+                last = u + 1 == n
+                if last:
                     self.commit("kv_empty")
                 yield from self.wait("pt_ready", pds)
                 if u == 0 and tiles_done >= 1 and self.drop != "dkv_free":
@@ -284,7 +291,16 @@ class DKDV(Core):
                         self.check(self.ACC is None or self.ACC[0] == "stored", f"dV overwrites {self.ACC}")
                         self.ACC = ("acc", k, 0)
                     self.ST = ("read", q)
+                if not last and self.drop == "lookahead_before_dv":
+                    yield from self.wait(f"qd_full{(q + 1) % 2}", (q + 1) // 2)
+                    st_mma(q + 1)
+                    s_issued = True
                 self.mma(dv)
+                if not last and self.drop != "lookahead_before_dv":
+                    # the next pair's S^T right behind dV, its P^T's last reader
+                    yield from self.wait(f"qd_full{(q + 1) % 2}", (q + 1) // 2)
+                    st_mma(q + 1)
+                    s_issued = True
                 yield from self.wait("dst_ready", pds)
                 pds += 1
 
@@ -486,10 +502,12 @@ def test_protocol_holds_on_random_schedules(kernel):
 
 
 @pytest.mark.parametrize("kernel,drop", [("forward", "kv_empty"), ("forward", "q_empty"), ("dkdv", "qd_empty"),
-                                         ("dkdv", "kv_empty"), ("dq", "kv_empty"), ("dq", "qd_empty")])
+                                         ("dkdv", "kv_empty"), ("dkdv", "lookahead_before_dv"), ("dq", "kv_empty"),
+                                         ("dq", "qd_empty")])
 def test_each_producer_guard_is_needed(kernel, drop):
     """Removing one of the producer's waits lets some schedule overwrite a stage that an
-    MMA has not read yet."""
+    MMA has not read yet; issuing the dK/dV kernel's look-ahead S^T before dV instead of
+    after it overwrites a P^T that dV has not read."""
     rng = random.Random(5)
     caught = 0
     for seed in range(300):
