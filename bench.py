@@ -359,6 +359,7 @@ def run_ours(args, world, rank, local):
     # measured per-CTA busy time of the last step (untimed read)
     cta_f = skv.splitkv_read_cta_times(plan, skv.WS_FWD, stream)
     cta_b = skv.splitkv_read_cta_times(plan, skv.WS_BWD, stream)
+    cta_q = skv.splitkv_read_cta_times(plan, skv.TIMES_DQ, stream) if _bwd_is_two_launches(w) else None
 
     def imb(x):
         x = np.asarray(x, dtype=np.float64)
@@ -371,7 +372,8 @@ def run_ours(args, world, rank, local):
                        "dynamic_claim": bool(args.dynamic_claim), "partial_bf16": bool(args.partial_bf16),
                        "schedule": args.schedule,
                        "fwd_workers": W, "bwd_workers": Wb,
-                       "fwd_ns": [int(x) for x in cta_f], "bwd_ns": [int(x) for x in cta_b]}, f)
+                       "fwd_ns": [int(x) for x in cta_f], "bwd_ns": [int(x) for x in cta_b],
+                       "dq_ns": None if cta_q is None else [int(x) for x in cta_q]}, f)
 
     pairs = st["context_pairs"] + st["block_pairs"]
     flops_fwd = 4.0 * d * pairs
@@ -424,7 +426,8 @@ def run_ours(args, world, rank, local):
         "pct_of_bf16_peak": 100.0 * value / world / peaks["bf16_tflops"],
         "lpt_imbalance_pct": {"fwd_plan": 100 * st["fwd_imbalance"], "bwd_plan": 100 * st["bwd_imbalance"],
                               "contiguous_plan": 100 * st["contig_imbalance"], "fwd_measured": 100 * imb(cta_f),
-                              "bwd_measured": 100 * imb(cta_b)},
+                              "bwd_measured": 100 * imb(cta_b),
+                              "dq_measured": None if cta_q is None else 100 * imb(cta_q)},
         "plan_us": float(np.median(plan_us)) if plan_us else None,
         "kernels": kern,
         "roofline": roof,

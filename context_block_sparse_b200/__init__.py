@@ -29,7 +29,7 @@ from ._abi import (  # noqa: F401
     FLAG_DYNAMIC_CLAIM, FLAG_EQUAL_COUNT,
     FLAG_FWD_TILE_COST,
     FLAG_PARTIAL_BF16, FLAG_TILE_COST,
-    STATIC_SCRATCH_BYTES, WS_BWD, WS_FWD,
+    STATIC_SCRATCH_BYTES, TIMES_DQ, WS_BWD, WS_FWD,
 )
 
 _lib = _abi.load()
@@ -387,9 +387,10 @@ def splitkv_plan_status(plan: Plan, stream=None) -> None:
 
 
 def splitkv_read_cta_times(plan: Plan, which: int, stream=None) -> np.ndarray:
-    """Per-CTA busy nanoseconds of the last forward (WS_FWD) or backward (WS_BWD) partial kernel."""
+    """Per-CTA busy nanoseconds of the last forward (WS_FWD), dK/dV (WS_BWD) or dQ (TIMES_DQ)
+    partial kernel."""
     st = plan.stats()
-    n = st["num_workers"] if which == WS_FWD else st["num_bwd_workers"]
+    n = st["num_bwd_workers"] if which == WS_BWD else st["num_workers"]
     out = np.zeros(n, dtype=np.int64)
     _check("splitkv_read_cta_times", _lib.splitkv_read_cta_times(
         plan.handle, which, out.ctypes.data_as(ctypes.POINTER(ctypes.c_int64)), n, _stream_ptr(stream)))

@@ -36,6 +36,7 @@ DTYPE_BF16 = 1
 
 WS_FWD = 0
 WS_BWD = 1
+TIMES_DQ = 2
 
 EXPORT_ENTRIES = 0
 EXPORT_CHUNK_PAIRS = 1

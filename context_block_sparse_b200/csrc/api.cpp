@@ -213,10 +213,12 @@ int splitkv_read_cta_times(const splitkv_plan_t* plan, int which, int64_t* out_n
   if (!plan || !out_ns) return SPLITKV_ERR_INVALID_ARG;
   const DevPlan* dp = splitkv::plan_device_view(plan);
   if (!dp) return SPLITKV_ERR_NOT_UPLOADED;
-  if (which != SPLITKV_WS_FWD && which != SPLITKV_WS_BWD) return SPLITKV_ERR_INVALID_ARG;
-  const int n = which == SPLITKV_WS_FWD ? dp->W : dp->Wb;
+  if (which != SPLITKV_WS_FWD && which != SPLITKV_WS_BWD && which != SPLITKV_TIMES_DQ) return SPLITKV_ERR_INVALID_ARG;
+  // stamps: forward CTAs, then dK/dV CTAs, then dQ CTAs
+  const int n = which == SPLITKV_WS_BWD ? dp->Wb : dp->W;
   if (capacity < n) return SPLITKV_ERR_WORKSPACE_TOO_SMALL;
-  const long long* src = dp->timers + (which == SPLITKV_WS_FWD ? 0 : 2 * size_t(dp->W));
+  const size_t first = which == SPLITKV_WS_FWD ? 0 : which == SPLITKV_WS_BWD ? size_t(dp->W) : size_t(dp->W + dp->Wb);
+  const long long* src = dp->timers + 2 * first;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   // stamps are small: copy to a host array synchronously on the stream
   long long* host = new (std::nothrow) long long[2 * size_t(n)];

@@ -651,7 +651,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int w = blockIdx.x;
   volatile int* abort_flag = &B->abort_flag;
   const WaitCtx wctx{abort_flag, p.status};
-  if (tid == 0) B->abort_flag = 0;
+  if (tid == 0) {
+    p.timers[(p.W + p.Wb + w) * 2 + 0] = global_timer_ns();
+    B->abort_flag = 0;
+  }
   {
     // commits count 1; element-wise / metadata signals count warps (warp_arrive)
     const uint32_t counts[kDqNumBars] = {1, 1, 1, 1, 1, 1, 1, 1, 1, 1, 1, 8, 1, 8, 1, 1, 1, 8, 8};
@@ -895,6 +898,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   if (warp == 2) tmem_dealloc(tmem, 512);
+  if (tid == 0) p.timers[(p.W + p.Wb + w) * 2 + 1] = global_timer_ns();
 }
 
 }  // namespace

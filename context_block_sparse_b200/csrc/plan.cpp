@@ -658,7 +658,7 @@ int splitkv_plan_upload(splitkv_plan_t* P, void* stream) {
   }
   const size_t table_bytes = off;
   const size_t timer_off = table_bytes;
-  const size_t status_off = timer_off + splitkv::align_up(size_t(P->W + P->Wb) * 2 * sizeof(long long), 256);
+  const size_t status_off = timer_off + splitkv::align_up(size_t(2 * P->W + P->Wb) * 2 * sizeof(long long), 256);
   const size_t total = status_off + 256;
 
   if (P->upload_pending) {

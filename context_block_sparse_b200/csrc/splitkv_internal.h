@@ -26,7 +26,7 @@ struct DevPlan {
   const int*  block_entry_ptr;  // [A+1]
   const int*  block_entries;    // [E]   entry ids of each block, ascending chunk
   const int*  zero_chunks;      // [Z]   chunks no block reads (backward zero fill)
-  long long*  timers;           // [W + Wb][2] global-timer stamps: forward CTAs, then backward CTAs
+  long long*  timers;           // [2W + Wb][2] global-timer stamps: forward, dK/dV, then dQ CTAs
   int*        status;           // device status word: 0, or a SPLITKV_ERR_* code a kernel recorded
   int num_zero_chunks;
   int N, Nq, A, bs, Hq, Hkv, G, d, C, num_chunks, E, W, Wb;

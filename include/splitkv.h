@@ -145,6 +145,8 @@ extern "C" {
 /* ---- workspace kinds --------------------------------------------------------- */
 #define SPLITKV_WS_FWD  0
 #define SPLITKV_WS_BWD  1
+/* splitkv_read_cta_times only: the dQ kernel of the backward (tcgen05 path) */
+#define SPLITKV_TIMES_DQ  2
 
 /* ---- export selectors (splitkv_plan_export) ------------------------------- */
 #define SPLITKV_EXPORT_ENTRIES        0  /* 4 per entry: chunk, block, lo, hi (record order)      */
@@ -475,10 +477,12 @@ int splitkv_combine_ranks(int32_t num_ranks, int64_t rows, int32_t head_dim, con
  * multiple of 4.  Asynchronous on `stream`.  Errors: INVALID_ARG, CUDA. */
 int splitkv_sum_ranks(int32_t num_ranks, int64_t n, const float* parts, float* out, void* stream);
 
-/* Per-CTA busy time of the last splitkv_attn_fwd (which = SPLITKV_WS_FWD) or
- * backward partial kernel (SPLITKV_WS_BWD) on this plan: out_ns[w] = end - start
- * of worker w's CTA in nanoseconds (device global timer), for the schedule's
- * worker count.  Synchronises `stream`.  Errors: INVALID_ARG, NOT_UPLOADED,
+/* Per-CTA busy time of the last splitkv_attn_fwd (which = SPLITKV_WS_FWD), the
+ * last dK/dV partial kernel (SPLITKV_WS_BWD; the single backward kernel of the
+ * mma.sync path) or the last dQ partial kernel (SPLITKV_TIMES_DQ; tcgen05 path,
+ * zeros before its first launch) on this plan: out_ns[w] = end - start of
+ * worker w's CTA in nanoseconds (device global timer), for the schedule's
+ * worker count (num_workers for the forward and dQ kernels).  Synchronises `stream`.  Errors: INVALID_ARG, NOT_UPLOADED,
  * WORKSPACE_TOO_SMALL (capacity below the worker count), CUDA. */
 int splitkv_read_cta_times(const splitkv_plan_t* plan, int which, int64_t* out_ns,
                            int64_t capacity, void* stream);

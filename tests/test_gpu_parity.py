@@ -389,3 +389,13 @@ def test_cta_timers_recorded(splitkv):
     out, att, _ = run(w)
     t = skv.splitkv_read_cta_times(att.plan, skv.WS_FWD)
     assert t.shape == (148,) and (t > 0).all()
+
+
+def test_cta_timers_of_every_partial_kernel(splitkv):
+    """Forward, dK/dV and dQ kernels each stamp their CTAs (W, Wb and W of them)."""
+    import context_block_sparse_b200 as skv
+    w = small()
+    _, att, _ = run(w, bwd=True, W=11, Wb=5)
+    for which, n in ((skv.WS_FWD, 11), (skv.WS_BWD, 5), (skv.TIMES_DQ, 11)):
+        t = skv.splitkv_read_cta_times(att.plan, which)
+        assert t.shape == (n,) and (t > 0).all(), which
