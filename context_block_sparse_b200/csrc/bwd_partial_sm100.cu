@@ -586,13 +586,13 @@ __global__ void __launch_bounds__(kThreads, 1)
 // dq kernel
 // ============================================================================
 struct DqBars {
-  uint64_t qd_full, qd_empty, k_full[2], v_full[2], kv_empty[2], s_ready[2], dp_ready, ds_ready, dq_ready, dq_free,
-      mma_done, meta_ready[2], meta_free[2];
+  uint64_t qd_full, qd_empty, k_full[2], v_full[2], k_empty[2], v_empty[2], s_ready[2], dp_ready, ds_ready, dq_ready,
+      dq_free, mma_done, meta_ready[2], meta_free[2];
   ClaimRing ring;   // run-time claims: producer -> MMA thread, metadata warp, 8 element-wise warps
   uint32_t tmem_base;
   int abort_flag;
 };
-constexpr int kDqNumBars = 19;
+constexpr int kDqNumBars = 21;
 static_assert(sizeof(DqBars) <= 256, "barrier block");
 
 // Per-row metadata of a query tile for the dq kernel (shared memory).
@@ -657,7 +657,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   {
     // commits count 1; element-wise / metadata signals count warps (warp_arrive)
-    const uint32_t counts[kDqNumBars] = {1, 1, 1, 1, 1, 1, 1, 1, 1, 1, 1, 8, 1, 8, 1, 1, 1, 8, 8};
+    const uint32_t counts[kDqNumBars] = {1, 1, 1, 1, 1, 1, 1, 1, 1, 1, 1, 1, 1, 8, 1, 8, 1, 1, 1, 8, 8};
     if (tid == 0) claim_ring_init(&B->ring, kClaimConsumers);
     setup_common(&B->qd_full, kDqNumBars, counts, &B->tmem_base, warp);
   }
@@ -672,33 +672,45 @@ __global__ void __launch_bounds__(kThreads, 1)
       TileIter ti;
       ti.init(&p, w, &B->ring, kClaimProducer, &wctx);
       int t, g;
-      uint32_t tile_count = 0, kv_count = 0, q_issued = 0;
+      uint32_t tile_count = 0, kv_count = 0, q_issued = 0, k_issued = 0, v_issued = 0;
       bool ok = true;
+      // key tile c of this CTA: V first (its stage frees once dP has read it), then K
+      // (its stage frees only after dQ += dS K)
+      auto load_kv = [&](uint32_t c, int k0) -> bool {
+        const int s = int(c & 1);
+        if (!mbar_wait(&B->v_empty[s], ((c >> 1) & 1) ^ 1, wctx, 2 * 10000 + __LINE__)) return false;
+        mbar_expect_tx(&B->v_full[s], kTile);
+        for (int dh = 0; dh < 2; ++dh) tma_load_3d(sV + s * kTile + dh * kHalf, &tm_v, &B->v_full[s], dh * 64, g, k0);
+        ++v_issued;
+        if (!mbar_wait(&B->k_empty[s], ((c >> 1) & 1) ^ 1, wctx, 2 * 10000 + __LINE__)) return false;
+        mbar_expect_tx(&B->k_full[s], kTile);
+        for (int dh = 0; dh < 2; ++dh) tma_load_3d(sK + s * kTile + dh * kHalf, &tm_k, &B->k_full[s], dh * 64, g, k0);
+        ++k_issued;
+        return true;
+      };
       while (ok && ti.next(t, g)) {
         const int4 tile = p.tiles[t];
+        const int n_kt = (tile.w - tile.z + BT - 1) / BT;
+        // the tile's first key tile needs only free stages: request it before the Q / dO
+        // buffer frees (the previous tile's last S and dP), so that it lands meanwhile
+        if (!load_kv(kv_count, tile.z)) { ok = false; break; }
         if (!mbar_wait(&B->qd_empty, (tile_count & 1) ^ 1, wctx, 2 * 10000 + __LINE__)) { ok = false; break; }
         mbar_expect_tx(&B->qd_full, 2 * kTile);
         load_query_tile(p, tile, g, sQ, &tm_q, &B->qd_full);
         load_query_tile(p, tile, g, sdO, &tm_do, &B->qd_full);
         ++q_issued;
-        const int n_kt = (tile.w - tile.z + BT - 1) / BT;
-        for (int j = 0; j < n_kt; ++j, ++kv_count) {
-          const int s = kv_count & 1;
-          if (!mbar_wait(&B->kv_empty[s], ((kv_count >> 1) & 1) ^ 1, wctx, 2 * 10000 + __LINE__)) { ok = false; break; }
-          const int k0 = tile.z + j * BT;
-          mbar_expect_tx(&B->k_full[s], kTile);
-          for (int dh = 0; dh < 2; ++dh) tma_load_3d(sK + s * kTile + dh * kHalf, &tm_k, &B->k_full[s], dh * 64, g, k0);
-          mbar_expect_tx(&B->v_full[s], kTile);
-          for (int dh = 0; dh < 2; ++dh) tma_load_3d(sV + s * kTile + dh * kHalf, &tm_v, &B->v_full[s], dh * 64, g, k0);
-        }
+        for (int j = 1; j < n_kt && ok; ++j)
+          if (!load_kv(kv_count + j, tile.z + j * BT)) ok = false;
+        if (!ok) break;
+        kv_count += n_kt;
         ++tile_count;
       }
       if (!ok) *abort_flag = 1;
       if (q_issued > 0) mbar_drain(&B->qd_full, (q_issued - 1) & 1, wctx, 2 * 10000 + __LINE__);
-      for (uint32_t c = kv_count >= 2 ? kv_count - 2 : 0; c < kv_count; ++c) {
+      for (uint32_t c = k_issued >= 2 ? k_issued - 2 : 0; c < k_issued; ++c)
         mbar_drain(&B->k_full[c & 1], (c >> 1) & 1, wctx, 2 * 10000 + __LINE__);
+      for (uint32_t c = v_issued >= 2 ? v_issued - 2 : 0; c < v_issued; ++c)
         mbar_drain(&B->v_full[c & 1], (c >> 1) & 1, wctx, 2 * 10000 + __LINE__);
-      }
     }
   } else if (warp == 1) {
     if (lane == 0) {
@@ -725,6 +737,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int kk = 0; kk < D / 16; ++kk)
             mma_ss(tmem + 256, kmajor(adO, kk), kmajor(aV + s * kTile, kk), kIdescKM, kk > 0 ? 1u : 0u);
           mma_commit(&B->dp_ready);
+          mma_commit(&B->v_empty[s]);   // V is read by dP only
         }
         for (int j = 0; j < n_kt; ++j) {
           const uint32_t c = c0 + j;
@@ -752,12 +765,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int kk = 0; kk < D / 16; ++kk)
               mma_ss(tmem + 256, kmajor(adO, kk), kmajor(aV + s1 * kTile, kk), kIdescKM, kk > 0 ? 1u : 0u);
             mma_commit(&B->dp_ready);
+            mma_commit(&B->v_empty[s1]);
             if (j + 2 == n_kt) mma_commit(&B->qd_empty);   // Q, dO: no further reader after this S / dP
           }
           for (int kk = 0; kk < BT / 16; ++kk)
             mma_ts(tmem + 384, tmem + s * 128 + packed_col(kk), mnmajor(aK + s * kTile, kk), kIdescMN,
                    (j > 0 || kk > 0) ? 1u : 0u);
-          mma_commit(&B->kv_empty[s]);
+          mma_commit(&B->k_empty[s]);   // K is read by S and by dQ += dS K
         }
         if (!ok) break;
         mma_commit(&B->dq_ready);
