@@ -757,8 +757,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             ++dqf_cnt;
           }
           tc_fence_after();
-          // the next dP first (the element-wise step of key tile j + 1 waits on it), then
-          // dQ (cols 384..) += dS K : dS in TMEM (columns 0..63 of S buffer s), K MN-major
+          // dQ (cols 384..) += dS K first -- dS in TMEM (columns 0..63 of S buffer s), K
+          // MN-major -- so that K stage s frees one product earlier for the load of key
+          // tile j + 2 (the loads, not the element-wise steps, set the pace), then the next dP
+          for (int kk = 0; kk < BT / 16; ++kk)
+            mma_ts(tmem + 384, tmem + s * 128 + packed_col(kk), mnmajor(aK + s * kTile, kk), kIdescMN,
+                   (j > 0 || kk > 0) ? 1u : 0u);
+          mma_commit(&B->k_empty[s]);   // K is read by S and by dQ += dS K
           if (more) {
             if (!mbar_wait(&B->v_full[s1], ((c + 1) >> 1) & 1, wctx, 2 * 10000 + __LINE__)) { ok = false; break; }
             tc_fence_after();
@@ -768,10 +773,6 @@ __global__ void __launch_bounds__(kThreads, 1)
             mma_commit(&B->v_empty[s1]);
             if (j + 2 == n_kt) mma_commit(&B->qd_empty);   // Q, dO: no further reader after this S / dP
           }
-          for (int kk = 0; kk < BT / 16; ++kk)
-            mma_ts(tmem + 384, tmem + s * 128 + packed_col(kk), mnmajor(aK + s * kTile, kk), kIdescMN,
-                   (j > 0 || kk > 0) ? 1u : 0u);
-          mma_commit(&B->k_empty[s]);   // K is read by S and by dQ += dS K
         }
         if (!ok) break;
         mma_commit(&B->dq_ready);
