@@ -351,13 +351,15 @@ class DKDV(Core):
 
 
 # ---------------------------------------------------------------------------
-# dQ kernel: Q / dO per query tile, two-stage K/V ring, S double-buffered
+# dQ kernel: Q / dO per query tile; K and V rings of two stages each (V released once dP
+# has read it, K after dQ += dS K; V loaded first; a tile's first K/V before its Q / dO);
+# S double-buffered; dQ issued before the next dP
 # ---------------------------------------------------------------------------
 class DQ(Core):
     def __init__(self, tiles, seed, drop=None):
-        names = ["qd_full", "qd_empty", "k_full0", "k_full1", "v_full0", "v_full1", "kv_empty0", "kv_empty1",
-                 "s_ready0", "s_ready1", "dp_ready", "ds_ready", "dq_ready", "dq_free", "meta_ready0",
-                 "meta_ready1", "meta_free0", "meta_free1"]
+        names = ["qd_full", "qd_empty", "k_full0", "k_full1", "v_full0", "v_full1", "k_empty0", "k_empty1",
+                 "v_empty0", "v_empty1", "s_ready0", "s_ready1", "dp_ready", "ds_ready", "dq_ready", "dq_free",
+                 "meta_ready0", "meta_ready1", "meta_free0", "meta_free1"]
         super().__init__(seed, names)
         self.tiles = tiles
         self.drop = drop
@@ -368,17 +370,22 @@ class DQ(Core):
 
     def producer(self):
         kv = 0
+
+        def load_kv(c):
+            s = c % 2
+            if c >= 2 and self.drop != "kv_empty":
+                yield from self.wait(f"v_empty{s}", c // 2 - 1)
+            self.load(f"v_full{s}", lambda s=s, c=c: self.V.__setitem__(s, c))
+            if c >= 2 and self.drop != "kv_empty":
+                yield from self.wait(f"k_empty{s}", c // 2 - 1)
+            self.load(f"k_full{s}", lambda s=s, c=c: self.K.__setitem__(s, c))
         for n, nkt in enumerate(self.tiles):
+            yield from load_kv(kv)
             if n >= 1 and self.drop != "qd_empty":
                 yield from self.wait("qd_empty", n - 1)
             self.load("qd_full", lambda n=n: setattr(self, "QD", n))
-            for j in range(nkt):
-                c = kv + j
-                s = c % 2
-                if c >= 2 and self.drop != "kv_empty":
-                    yield from self.wait(f"kv_empty{s}", c // 2 - 1)
-                self.load(f"k_full{s}", lambda s=s, c=c: self.K.__setitem__(s, c))
-                self.load(f"v_full{s}", lambda s=s, c=c: self.V.__setitem__(s, c))
+            for j in range(1, nkt):
+                yield from load_kv(kv + j)
             kv += nkt
             yield
 
@@ -411,6 +418,7 @@ class DQ(Core):
                     self.DP = ("dP", c)
                 self.mma(ex)
                 self.commit("dp_ready")
+                self.commit(f"v_empty{c % 2}")
             c0 = kv
             yield from self.wait(f"k_full{c0 % 2}", c0 // 2)
             s_mma(c0)
@@ -426,11 +434,6 @@ class DQ(Core):
                 ds += 1
                 if j == 0 and n >= 1 and self.drop != "dq_free":
                     yield from self.wait("dq_free", n - 1)
-                if more and self.drop != "dp_after_ds":
-                    yield from self.wait(f"v_full{(c + 1) % 2}", (c + 1) // 2)
-                    dp_mma(c + 1)
-                    if j + 2 == nkt:
-                        self.commit("qd_empty")
 
                 def dq(b=c % 2, c=c, j=j, n=n):
                     self.check(self.S[b] == ("dS", c) and self.K[b] == c, f"dQ({c}) reads {self.S[b]} K {self.K[b]}")
@@ -442,7 +445,12 @@ class DQ(Core):
                         self.DQ = ("acc", n, j + 1)
                     self.S[b] = ("read", c)
                 self.mma(dq)
-                self.commit(f"kv_empty{c % 2}")
+                self.commit(f"k_empty{c % 2}")
+                if more:
+                    yield from self.wait(f"v_full{(c + 1) % 2}", (c + 1) // 2)
+                    dp_mma(c + 1)
+                    if j + 2 == nkt:
+                        self.commit("qd_empty")
             self.commit("dq_ready")
             if nkt == 1:
                 self.commit("qd_empty")
