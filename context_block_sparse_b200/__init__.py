@@ -456,5 +456,12 @@ def splitkv_sum_ranks(parts, out, stream=None) -> None:
     _check("splitkv_sum_ranks", _lib.splitkv_sum_ranks(R, n, _f32_ptr(parts), _f32_ptr(out), _stream_ptr(stream)))
 
 
+def splitkv_selftest_wait_timeout(stream=None):
+    """Run the bounded-wait self-test; returns the status words (code, site) it recorded."""
+    out = (ctypes.c_int32 * 2)()
+    _check("splitkv_selftest_wait_timeout", _lib.splitkv_selftest_wait_timeout(out, _stream_ptr(stream)))
+    return int(out[0]), int(out[1])
+
+
 def library_path() -> str:
     return _abi.LIB_PATH

@@ -477,6 +477,15 @@ int splitkv_combine_ranks(int32_t num_ranks, int64_t rows, int32_t head_dim, con
  * multiple of 4.  Asynchronous on `stream`.  Errors: INVALID_ARG, CUDA. */
 int splitkv_sum_ranks(int32_t num_ranks, int64_t n, const float* parts, float* out, void* stream);
 
+/* Self-test of the kernels' failure detection: one CTA waits, with the same bounded
+ * mbarrier waits the attention kernels use, on a barrier nothing ever completes.  The
+ * wait gives up after its time limit (2 s of the device global timer) and records
+ * SPLITKV_ERR_TIMEOUT and its source site, which come back in status_out[0] and
+ * status_out[1] (the kernel does not hang and the context stays usable).  Synchronises
+ * `stream`; takes about two seconds.  Not part of the method.
+ * Errors: INVALID_ARG, NO_MEMORY, CUDA. */
+int splitkv_selftest_wait_timeout(int32_t* status_out, void* stream);
+
 /* Per-CTA busy time of the last splitkv_attn_fwd (which = SPLITKV_WS_FWD), the
  * last dK/dV partial kernel (SPLITKV_WS_BWD; the single backward kernel of the
  * mma.sync path) or the last dQ partial kernel (SPLITKV_TIMES_DQ; tcgen05 path,

@@ -55,3 +55,21 @@ def test_unsupported_head_dim(splitkv):
         skv.splitkv_attn_fwd(plan, q, kv, kv, 1.0, ws)
     assert ei.value.status == -2
     torch.cuda.synchronize()
+
+
+def test_a_wait_nothing_completes_times_out_and_the_context_survives(splitkv):
+    """Failure detection without a fault: a bounded wait on a barrier no one completes gives
+    up after its limit and reports SPLITKV_ERR_TIMEOUT with its site; afterwards the same
+    context runs a forward and backward that match the oracle."""
+    import time
+    from gpu_util import TOL_OUT, assert_close, oracle_bwd, run
+    t0 = time.time()
+    code, site = splitkv.splitkv_selftest_wait_timeout()
+    elapsed = time.time() - t0
+    assert code == -5                       # SPLITKV_ERR_TIMEOUT
+    assert site // 10000 == 9               # a wait of the self-test
+    assert 1.5 < elapsed < 60               # the two-second limit, not a hang
+    w = small(Hq=4, Hkv=1, d=128)
+    out, _, _ = run(w, bwd=True)
+    g = oracle_bwd(w)
+    assert_close("dq", out["dq"], g["dq"], TOL_OUT)
