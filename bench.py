@@ -662,7 +662,8 @@ def rank_emulation_report(skv, w, args, R, dev, stream, t, W, Wb, peaks, reps=5,
 
 def run_e2e(args, w, plan, dev, stream, flops_step, world=1):
     """Same metric through the public API from pinned HOST buffers: every step copies its inputs in and
-    its results (o, lse, dq, dk, dv, dkb, dvb) out inside the timed region."""
+    its results (o, lse, dq, dk, dv, dkb, dvb) out inside the timed region, the copies overlapping the
+    computation of the neighbouring steps (two device buffer sets, one stream per copy direction)."""
     import torch
     import torch.distributed as dist
 
@@ -677,40 +678,71 @@ def run_e2e(args, w, plan, dev, stream, flops_step, world=1):
                            q_slice=plan.problem.q_slice, device=dev, partial_bf16=args.partial_bf16,
                            tile_cost=args.lpt_cost == "tiles", fwd_tile_cost=args.fwd_lpt_cost == "tiles",
                            dynamic_claim=args.dynamic_claim, contiguous_schedule=args.schedule == "contiguous")
-    dv = {n: torch.empty(x.shape, dtype=x.dtype, device=dev) for n, x in host.items()}
-    outs_h = {"o": torch.empty((Nq, Hq, d), dtype=torch.float32).pin_memory(),
-              "lse": torch.empty((Nq, Hq), dtype=torch.float32).pin_memory()}
-    for n in ("q", "k", "v", "kb", "vb"):
-        outs_h["d" + n] = torch.empty(host[n].shape, dtype=torch.float32).pin_memory()
+    # two device sets of inputs and outputs, so that the next step's inputs go up and the
+    # last step's results come down while a step computes; uploads and downloads on copy
+    # streams of their own (the two PCIe directions run at once)
+    dvs = [{n: torch.empty(x.shape, dtype=x.dtype, device=dev) for n, x in host.items()} for _ in range(2)]
+    f32 = dict(dtype=torch.float32, device=dev)
+    outs_d = [{"o": torch.empty((Nq, Hq, d), **f32), "lse": torch.empty((Nq, Hq), **f32),
+               **{"d" + n: torch.empty(host[n].shape, **f32) for n in ("q", "k", "v", "kb", "vb")}}
+              for _ in range(2)]
+    outs_h = {n: torch.empty(x.shape, dtype=torch.float32).pin_memory() for n, x in outs_d[0].items()}
     h2d = sum(x.numel() * x.element_size() for x in host.values()) + 4 * (w.sample_lens.size + w.anchors.size)
     d2h = sum(x.numel() * x.element_size() for x in outs_h.values())
     steps = max(1, min(args.steps, args.e2e_steps))
+    up_s = torch.cuda.Stream(dev)
+    down_s = torch.cuda.Stream(dev)
+    ev = lambda: torch.cuda.Event()   # noqa: E731
+    computed = [None, None]   # per set: the step's kernels are done (its inputs and outputs are free)
+    downloaded = [None, None]  # per set: its outputs have reached the host
 
-    def step():
-        for n in host:
-            dv[n].copy_(host[n], non_blocking=True)
+    def step(k):
+        b = k % 2
+        x, y = dvs[b], outs_d[b]
+        # inputs: after the kernels of step k - 2 have read this set
+        if computed[b] is not None:
+            up_s.wait_event(computed[b])
+        with torch.cuda.stream(up_s):
+            for n in host:
+                x[n].copy_(host[n], non_blocking=True)
+        uploaded = ev()
+        uploaded.record(up_s)
+        # compute: after the inputs landed and step k - 2's results left this set
+        stream.wait_event(uploaded)
+        if downloaded[b] is not None:
+            stream.wait_event(downloaded[b])
         skv.splitkv_plan_update(att.plan, w.sample_lens, w.anchors)
         att.plan.upload(stream)
-        o, lse = att.forward(dv["q"], dv["k"], dv["v"], dv["kb"], dv["vb"], w.scale)
-        g = att.backward(dv["q"], dv["k"], dv["v"], dv["kb"], dv["vb"], o, lse, dv["dout"], w.scale)
-        outs_h["o"].copy_(o, non_blocking=True)
-        outs_h["lse"].copy_(lse, non_blocking=True)
-        for n, x in g.items():
-            outs_h[n].copy_(x, non_blocking=True)
+        o, lse = att.forward(x["q"], x["k"], x["v"], x["kb"], x["vb"], w.scale, o=y["o"], lse=y["lse"])
+        att.backward(x["q"], x["k"], x["v"], x["kb"], x["vb"], o, lse, x["dout"], w.scale,
+                     grads={n: y[n] for n in ("dq", "dk", "dv", "dkb", "dvb")})
+        computed[b] = ev()
+        computed[b].record(stream)
+        # results: down while the next step computes
+        down_s.wait_event(computed[b])
+        with torch.cuda.stream(down_s):
+            for n, t in y.items():
+                outs_h[n].copy_(t, non_blocking=True)
+        downloaded[b] = ev()
+        downloaded[b].record(down_s)
 
-    for _ in range(2):
-        step()
+    for k in range(2):
+        step(k)
     torch.cuda.synchronize(dev)
     if world > 1:
         dist.barrier()
     a = torch.cuda.Event(enable_timing=True)
-    b = torch.cuda.Event(enable_timing=True)
+    bev = torch.cuda.Event(enable_timing=True)
     a.record(stream)
-    for _ in range(steps):
-        step()
-    b.record(stream)
+    up_s.wait_event(a)      # the first upload of the timed steps starts after the start mark
+    down_s.wait_event(a)
+    for k in range(2, 2 + steps):
+        step(k)
+    stream.wait_event(downloaded[(1 + steps) % 2])   # the last results are on the host
+    stream.wait_event(downloaded[steps % 2])
+    bev.record(stream)
     torch.cuda.synchronize(dev)
-    ms = max_over_ranks(a.elapsed_time(b), dev)
+    ms = max_over_ranks(a.elapsed_time(bev), dev)
     if world > 1:
         dist.barrier()
     return {"value": whole_job_tflops(world, steps, flops_step, ms), "unit": "TFLOP/s",
