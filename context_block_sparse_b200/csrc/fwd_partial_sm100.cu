@@ -11,7 +11,10 @@
 // tiles are taken two at a time (A and B) so that each K/V tile loaded into
 // shared memory feeds two 128x128 score tiles.  Roles (384 threads):
 //   warp 0      TMA producer: Q tiles (3-D boxes of bs tokens x G heads per
-//               block) and 128-key K/V tiles into a 2-stage ring;
+//               block) and 128-key K and V tiles into two-stage rings of their
+//               own (a K stage refills once its S products are done, a V stage
+//               once its PV products are; a pair's first K/V tiles go out before
+//               its Q buffer frees);
 //   warp 1      MMA issuer (one thread): S_X = Q_X K^T into TMEM, then
 //               O_X += P_X V with P_X read from TMEM (bf16, aliasing S_X);
 //   warp 2      tensor-memory allocation (512 columns: S_A, S_B, O_A, O_B);
@@ -69,7 +72,7 @@ static_assert(kSmemBytes <= 232448, "shared memory per block");
 
 struct Bars {
   uint64_t q_full, q_empty;
-  uint64_t k_full[kStages], v_full[kStages], kv_empty[kStages];
+  uint64_t k_full[kStages], v_full[kStages], k_empty[kStages], v_empty[kStages];
   uint64_t s_ready[2], p_ready[2], o_ready[2], o_free[2];
   uint64_t mma_done;
   ClaimRing ring;   // run-time claims: the producer hands items to the MMA thread and the 8 softmax warps
@@ -191,7 +194,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&bars->k_full[s], 1);
       mbar_init(&bars->v_full[s], 1);
-      mbar_init(&bars->kv_empty[s], 1);
+      mbar_init(&bars->k_empty[s], 1);
+      mbar_init(&bars->v_empty[s], 1);
     }
     for (int x = 0; x < 2; ++x) {
       mbar_init(&bars->s_ready[x], 1);
@@ -225,9 +229,31 @@ __global__ void __launch_bounds__(kThreads, 1)
       PairIter pi;
       pi.init(&p, w, &bars->ring, kClaimProducer, &wctx);
       int tA, tB, g, klo, khi;
-      uint32_t kv_count = 0, pair_count = 0, q_issued = 0;
+      uint32_t kv_count = 0, pair_count = 0, q_issued = 0, k_issued = 0, v_issued = 0;
       bool ok = true;
+      // key tile j of the current pair into the next K and V stages: each stage is
+      // refilled once the last product reading it (S for K, PV for V) has completed
+      auto load_kv = [&](int j) -> bool {
+        const int s = kv_count % kStages;
+        const uint32_t ph = ((kv_count / kStages) & 1) ^ 1;
+        const int k0 = klo + j * BN;
+        if (!mbar_wait(&bars->k_empty[s], ph, wctx, 1 * 10000 + __LINE__)) return false;
+        mbar_expect_tx(&bars->k_full[s], kTile);
+        for (int dh = 0; dh < 2; ++dh)
+          tma_load_3d(smem + kOffK + s * kTile + dh * kHalf, &tm_k, &bars->k_full[s], dh * 64, g, k0);
+        ++k_issued;
+        if (!mbar_wait(&bars->v_empty[s], ph, wctx, 1 * 10000 + __LINE__)) return false;
+        mbar_expect_tx(&bars->v_full[s], kTile);
+        for (int dh = 0; dh < 2; ++dh)
+          tma_load_3d(smem + kOffV + s * kTile + dh * kHalf, &tm_v, &bars->v_full[s], dh * 64, g, k0);
+        ++v_issued;
+        ++kv_count;
+        return true;
+      };
       while (ok && pi.next(tA, tB, g, klo, khi)) {
+        const int n_kt = (khi - klo + BN - 1) / BN;
+        // the pair's first K / V tiles go out before its Q buffer frees
+        if (!load_kv(0)) { ok = false; break; }
         if (!mbar_wait(&bars->q_empty, (pair_count & 1) ^ 1, wctx, 1 * 10000 + __LINE__)) { ok = false; break; }
         const int4 ta = p.tiles[tA];
         const int nA = ta.y - ta.x;
@@ -252,28 +278,19 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
         ++q_issued;
-        const int n_kt = (khi - klo + BN - 1) / BN;
-        for (int j = 0; j < n_kt; ++j, ++kv_count) {
-          const int s = kv_count % kStages;
-          if (!mbar_wait(&bars->kv_empty[s], ((kv_count / kStages) & 1) ^ 1, wctx, 1 * 10000 + __LINE__)) { ok = false; break; }
-          const int k0 = klo + j * BN;
-          mbar_expect_tx(&bars->k_full[s], kTile);
-          for (int dh = 0; dh < 2; ++dh)
-            tma_load_3d(smem + kOffK + s * kTile + dh * kHalf, &tm_k, &bars->k_full[s], dh * 64, g, k0);
-          mbar_expect_tx(&bars->v_full[s], kTile);
-          for (int dh = 0; dh < 2; ++dh)
-            tma_load_3d(smem + kOffV + s * kTile + dh * kHalf, &tm_v, &bars->v_full[s], dh * 64, g, k0);
-        }
+        for (int j = 1; j < n_kt; ++j)
+          if (!load_kv(j)) { ok = false; break; }
+        if (!ok) break;
         ++pair_count;
       }
       if (!ok) *abort_flag = 1;
       // copies still in flight land before the CTA may exit: wait for the last
       // fill of every buffer (bounded; completed phases return at once)
       if (q_issued > 0) mbar_drain(&bars->q_full, (q_issued - 1) & 1, wctx, 1 * 10000 + __LINE__);
-      for (uint32_t c = kv_count >= kStages ? kv_count - kStages : 0; c < kv_count; ++c) {
+      for (uint32_t c = k_issued >= kStages ? k_issued - kStages : 0; c < k_issued; ++c)
         mbar_drain(&bars->k_full[c % kStages], (c / kStages) & 1, wctx, 1 * 10000 + __LINE__);
+      for (uint32_t c = v_issued >= kStages ? v_issued - kStages : 0; c < v_issued; ++c)
         mbar_drain(&bars->v_full[c % kStages], (c / kStages) & 1, wctx, 1 * 10000 + __LINE__);
-      }
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
@@ -303,6 +320,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             mma_commit(&bars->s_ready[x]);
           }
+          mma_commit(&bars->k_empty[s0]);   // K_s0 free once its S products complete
         }
         for (int j = 0; j < n_kt && ok; ++j) {
           const uint32_t c = kv_count + j;
@@ -326,6 +344,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               mma_ts(tmem + 256 + x * 128, tmem + x * 128 + kk * 8, b, kIdescPV, (j > 0 || kk > 0) ? 1u : 0u);
             }
             mma_commit(&bars->o_ready[x]);
+            if (x == nx - 1) mma_commit(&bars->v_empty[s]);   // V_s: its last PV issued
             if (more) {
               if (x == 0) {
                 if (!mbar_wait(&bars->k_full[s1], ((c + 1) / kStages) & 1, wctx, 1 * 10000 + __LINE__)) { ok = false; break; }
@@ -338,12 +357,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                 mma_ss(tmem + x * 128, a, b, kIdescQK, kk > 0 ? 1u : 0u);
               }
               mma_commit(&bars->s_ready[x]);
-              // the pair's last S: Q_A / Q_B have no further reader
-              if (j + 2 == n_kt && x == nx - 1) mma_commit(&bars->q_empty);
+              if (x == nx - 1) {
+                mma_commit(&bars->k_empty[s1]);   // K_s1: its last S issued
+                // the pair's last S: Q_A / Q_B have no further reader
+                if (j + 2 == n_kt) mma_commit(&bars->q_empty);
+              }
             }
           }
           if (!ok) break;
-          mma_commit(&bars->kv_empty[s]);   // K_s, V_s free once everything issued so far completes
         }
         if (!ok) break;
         if (n_kt == 1) mma_commit(&bars->q_empty);

@@ -95,12 +95,14 @@ class Core:
 
 
 # ---------------------------------------------------------------------------
-# forward kernel: query tiles two at a time (A, B), one two-stage K/V ring
+# forward kernel: query tiles two at a time (A, B), K and V rings of two stages each (a
+# pair's first K/V tiles requested before its Q buffer frees)
 # ---------------------------------------------------------------------------
 class Forward(Core):
     def __init__(self, pairs, seed, drop=None):
-        names = ["q_full", "q_empty", "k_full0", "k_full1", "v_full0", "v_full1", "kv_empty0", "kv_empty1",
-                 "s_ready0", "s_ready1", "p_ready0", "p_ready1", "o_ready0", "o_ready1", "o_free0", "o_free1"]
+        names = ["q_full", "q_empty", "k_full0", "k_full1", "v_full0", "v_full1", "k_empty0", "k_empty1",
+                 "v_empty0", "v_empty1", "s_ready0", "s_ready1", "p_ready0", "p_ready1", "o_ready0", "o_ready1",
+                 "o_free0", "o_free1"]
         super().__init__(seed, names)
         self.pairs = pairs            # [(nx, n_kt)]
         self.drop = drop
@@ -113,17 +115,22 @@ class Forward(Core):
 
     def producer(self):
         kv = 0
+
+        def load_kv(c):
+            s = c % 2
+            if c >= 2 and self.drop != "kv_empty":
+                yield from self.wait(f"k_empty{s}", c // 2 - 1)
+            self.load(f"k_full{s}", lambda s=s, c=c: self.K.__setitem__(s, c))
+            if c >= 2 and self.drop != "kv_empty":
+                yield from self.wait(f"v_empty{s}", c // 2 - 1)
+            self.load(f"v_full{s}", lambda s=s, c=c: self.V.__setitem__(s, c))
         for i, (nx, nkt) in enumerate(self.pairs):
+            yield from load_kv(kv)
             if i >= 1 and self.drop != "q_empty":
                 yield from self.wait("q_empty", i - 1)
             self.load("q_full", lambda i=i: setattr(self, "Q", i))
-            for j in range(nkt):
-                c = kv + j
-                s = c % 2
-                if c >= 2 and self.drop != "kv_empty":
-                    yield from self.wait(f"kv_empty{s}", c // 2 - 1)
-                self.load(f"k_full{s}", lambda s=s, c=c: self.K.__setitem__(s, c))
-                self.load(f"v_full{s}", lambda s=s, c=c: self.V.__setitem__(s, c))
+            for j in range(1, nkt):
+                yield from load_kv(kv + j)
             kv += nkt
             yield
 
@@ -143,6 +150,7 @@ class Forward(Core):
             yield from self.wait(f"k_full{kv % 2}", kv // 2)
             for x in range(nx):
                 s_mma(x, kv)
+            self.commit(f"k_empty{kv % 2}")
             for j in range(nkt):
                 c = kv + j
                 more = j + 1 < nkt
@@ -169,13 +177,16 @@ class Forward(Core):
                             self.O[x] = ("acc", i, j + 1)
                     self.mma(pv)
                     self.commit(f"o_ready{x}")
+                    if x == nx - 1:
+                        self.commit(f"v_empty{c % 2}")
                     if more:
                         if x == 0:
                             yield from self.wait(f"k_full{(c + 1) % 2}", (c + 1) // 2)
                         s_mma(x, c + 1)
-                        if j + 2 == nkt and x == nx - 1:
-                            self.commit("q_empty")
-                self.commit(f"kv_empty{c % 2}")
+                        if x == nx - 1:
+                            self.commit(f"k_empty{(c + 1) % 2}")
+                            if j + 2 == nkt:
+                                self.commit("q_empty")
             if nkt == 1:
                 self.commit("q_empty")
             kv += nkt
