@@ -9,7 +9,7 @@
 //
 // One persistent CTA per worker walks its LPT items; every item's 128-row query
 // tiles are taken two at a time (A and B) so that each K/V tile loaded into
-// shared memory feeds two 128x128 score tiles.  Roles (384 threads):
+// shared memory feeds two 128x128 score tiles.  Roles (512 threads):
 //   warp 0      TMA producer: Q tiles (3-D boxes of bs tokens x G heads per
 //               block) and 128-key K and V tiles into two-stage rings of their
 //               own (a K stage refills once its S products are done, a V stage
@@ -18,8 +18,11 @@
 //   warp 1      MMA issuer (one thread): S_X = Q_X K^T into TMEM, then
 //               O_X += P_X V with P_X read from TMEM (bf16, aliasing S_X);
 //   warp 2      tensor-memory allocation (512 columns: S_A, S_B, O_A, O_B);
-//   warps 4-7   softmax / epilogue of tile A (thread = row = TMEM lane);
-//   warps 8-11  softmax / epilogue of tile B.
+//   warps 4-7   softmax of tile A (thread = row = TMEM lane);
+//   warps 8-11  softmax of tile B;
+//   warps 12-15 record epilogue of both tiles: O_X / l from TMEM to the record,
+//               so that the softmax warps go on to the next pair at once and the
+//               output columns return to the MMA right after their last read.
 // The softmax keeps, per row, a reference maximum m_ref, taken from the first
 // key tile in which the row has allowed keys (the only tile that reads S from
 // TMEM twice); later tiles exponentiate against it in one pass and only when a
@@ -27,10 +30,9 @@
 // written rescaled to a new reference -- the result is the same, the reference
 // is exact bookkeeping.  The record written is m_c = the row's true maximum
 // (natural units), l_c = sum exp(s - m_c) and O_c = sum exp(s - m_c) v / l_c.
-// Rows are masked to their block's [lo, hi).  When a warp's 32 rows are whole
-// tokens of one block (G * bs a multiple of 32), O_c leaves through bulk tensor
-// stores of 32-row x 16-column boxes staged in two 2 KB buffers per warp (32-row x
-// 32-column bf16 boxes when the plan stores bf16 records).
+// Rows are masked to their block's [lo, hi).  The epilogue stores go through a
+// 4 KB per-warp staging buffer so that every store instruction writes whole
+// 128-byte row segments (bf16 records: 64 bytes per row straight from registers).
 //
 // Every mbarrier wait is bounded; on a timeout the kernel records
 // SPLITKV_ERR_TIMEOUT in the plan's status word, lets every role wind down,
@@ -51,7 +53,7 @@ constexpr int D = 128;
 constexpr int BM = 128;               // query rows per tile
 constexpr int BN = 128;               // keys per key tile
 constexpr int kStages = 2;            // K/V ring depth
-constexpr int kThreads = 384;
+constexpr int kThreads = 512;
 constexpr uint32_t kHalf = 128 * 128; // bytes of one 64-column half of a 128-row tile
 constexpr uint32_t kTile = 2 * kHalf; // 32 KB: a 128 x 128 bf16 tile
 constexpr uint32_t kIdescQK = idesc_bf16_f32(128, 128, 0);
@@ -65,22 +67,27 @@ constexpr float kHeadroomLog2 = 32.0f;
 constexpr uint32_t kOffQ = 0;                              // Q_A, Q_B
 constexpr uint32_t kOffK = kOffQ + 2 * kTile;              // K stages
 constexpr uint32_t kOffV = kOffK + kStages * kTile;        // V stages
-constexpr uint32_t kOffScratch = kOffV + kStages * kTile; // epilogue buffers, 4 KB per softmax warp
-constexpr uint32_t kOffBar = kOffScratch + 8 * 4096;       // mbarriers
-constexpr uint32_t kSmemBytes = kOffBar + 256 + 1024;      // + alignment slack
+constexpr uint32_t kOffScratch = kOffV + kStages * kTile; // record staging, 4 KB per epilogue warp
+constexpr uint32_t kOffStats = kOffScratch + 4 * 4096;     // row statistics [2 pair parities][2 tiles][128] float4
+constexpr uint32_t kOffBar = kOffStats + 2 * 2 * BM * 16;  // mbarriers
+constexpr uint32_t kSmemBytes = kOffBar + 512 + 1024;      // + alignment slack
 static_assert(kSmemBytes <= 232448, "shared memory per block");
 
 struct Bars {
   uint64_t q_full, q_empty;
   uint64_t k_full[kStages], v_full[kStages], k_empty[kStages], v_empty[kStages];
   uint64_t s_ready[2], p_ready[2], o_ready[2], o_free[2];
+  // o_full[x]: tile x's last PV of a pair has completed (the epilogue reads O);
+  // stats_ready[x][b]: the softmax warps of tile x left the row statistics of a pair
+  // in stats buffer b = pair parity
+  uint64_t o_full[2], stats_ready[2][2];
   uint64_t mma_done;
   ClaimRing ring;   // run-time claims: the producer hands items to the MMA thread and the 8 softmax warps
   uint32_t tmem_base;
   int abort_flag;
 };
-static_assert(sizeof(Bars) <= 256, "barrier block");
-constexpr uint32_t kClaimConsumers = 1 + 8;
+static_assert(sizeof(Bars) <= 512, "barrier block");
+constexpr uint32_t kClaimConsumers = 1 + 8 + 4;
 
 // The sequence of tile pairs a worker processes (identical in every role): the
 // worker's items of the static schedule, or the items it claims at run time.
@@ -176,8 +183,8 @@ __device__ __forceinline__ float exp_pack_store(const uint32_t (&v)[64], int a, 
 
 __global__ void __launch_bounds__(kThreads, 1)
     fwd_partial_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                             const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
-                             DevPlan p, float scale_log2, int bulk_o, void* __restrict__ part_o,
+                             const __grid_constant__ CUtensorMap tm_v, DevPlan p, float scale_log2,
+                             void* __restrict__ part_o,
                              float* __restrict__ part_m, float* __restrict__ part_l) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -201,7 +208,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&bars->s_ready[x], 1);
       mbar_init(&bars->p_ready[x], 4);    // one arrival per softmax warp
       mbar_init(&bars->o_ready[x], 1);
-      mbar_init(&bars->o_free[x], 4);
+      mbar_init(&bars->o_free[x], 4);      // one arrival per epilogue warp
+      mbar_init(&bars->o_full[x], 1);
+      mbar_init(&bars->stats_ready[x][0], 4);
+      mbar_init(&bars->stats_ready[x][1], 4);
     }
     mbar_init(&bars->mma_done, 1);
     claim_ring_init(&bars->ring, kClaimConsumers);
@@ -344,6 +354,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               mma_ts(tmem + 256 + x * 128, tmem + x * 128 + kk * 8, b, kIdescPV, (j > 0 || kk > 0) ? 1u : 0u);
             }
             mma_commit(&bars->o_ready[x]);
+            if (!more) mma_commit(&bars->o_full[x]);           // tile x's output complete
             if (x == nx - 1) mma_commit(&bars->v_empty[s]);   // V_s: its last PV issued
             if (more) {
               if (x == 0) {
@@ -376,17 +387,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       mma_commit(&bars->mma_done);
       mbar_drain(&bars->mma_done, 0, wctx, 1 * 10000 + __LINE__);
     }
-  } else if (warp >= 4) {
-    // ------------------------------------------------------------ softmax + epilogue
+  } else if (warp >= 4 && warp < 12) {
+    // ------------------------------------------------------------ softmax
     const int x = (warp - 4) >> 2;            // tile A (warps 4-7) or B (warps 8-11)
     const int r = ((warp & 3) << 5) + lane;   // row of the tile = TMEM lane
     const uint32_t lane_addr = uint32_t((warp & 3) << 5) << 16;
     const uint32_t tS = tmem + lane_addr + x * 128;
-    const uint32_t tO = tmem + lane_addr + 256 + x * 128;
+    const uint32_t tO = tmem + lane_addr + 256 + x * 128;   // O_X: rescaled in place on a new reference
     PairIter pi;
     pi.init(&p, w, &bars->ring, kClaimWarp, &wctx);
     int tA, tB, g, klo, khi;
-    uint32_t s_cnt = 0, o_cnt = 0;
+    uint32_t s_cnt = 0, o_cnt = 0, st_cnt = 0;
     bool ok = true;
     while (ok && pi.next(tA, tB, g, klo, khi)) {
       const int t = x == 0 ? tA : tB;
@@ -394,16 +405,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int n_kt = (khi - klo + BN - 1) / BN;
       const int4 tile = p.tiles[t];
       const int slot = r / rows_per_slot;
-      const int within = r - slot * rows_per_slot;
-      const int tt = within / p.G, hh = within - tt * p.G;
       const bool valid = slot < tile.y - tile.x;
-      int lo = 0, hi = 0, rec = 0;
+      int lo = 0, hi = 0;   // the row's allowed keys (none for a padding row)
       if (valid) {
-        const int e = tile.x + slot;
-        const int4 ent = p.entries[e];
+        const int4 ent = p.entries[tile.x + slot];
         lo = ent.y;
         hi = ent.z;
-        rec = (e * p.bs + tt) * p.Hq + g * p.G + hh;
       }
       float m_ref = -INFINITY, m_true = -INFINITY, l = 0.f;
       for (int j = 0; j < n_kt && ok; ++j) {
@@ -497,86 +504,77 @@ __global__ void __launch_bounds__(kThreads, 1)
         warp_arrive(&bars->p_ready[x]);
       }
       if (!ok) break;
-      // epilogue: wait for the last PV of this tile, then write the record
-      if (!warp_wait(&bars->o_ready[x], (o_cnt + n_kt - 1) & 1, wctx, 1 * 10000 + __LINE__)) { ok = false; break; }
       o_cnt += n_kt;
-      tc_fence_after();
-      const float inv = l > 0.f ? 1.f / l : 0.f;
-      float* scratch = reinterpret_cast<float*>(smem + kOffScratch) + (warp - 4) * 1024;
-      if (bulk_o && p.partial_bf16) {
-        // bf16 records: one 32-row x 32-column box per TMEM load, two buffers
-        const int z0 = __shfl_sync(0xffffffffu, valid ? rec / p.Hq : 0, 0);
-        if (valid) {
-          uint32_t va[32], vb[32];
-          tmem_ld32(tO, va);
-          tmem_wait_ld();
-          reg_fence<32>(va);
-#pragma unroll
-          for (int cch = 0; cch < D / 32; cch += 2) {
-            tmem_ld32(tO + (cch + 1) * 32, vb);
-            warp_bulk_store32_bf16<1>(scratch, va, inv, &tm_o, cch * 32, g * p.G, z0);
-            tmem_wait_ld();
-            reg_fence<32>(vb);
-            if (cch + 2 < D / 32) tmem_ld32(tO + (cch + 2) * 32, va);
-            warp_bulk_store32_bf16<1>(scratch + 512, vb, inv, &tm_o, (cch + 1) * 32, g * p.G, z0);
-            tmem_wait_ld();
-            reg_fence<32>(va);
-          }
-        }
-      } else if (p.partial_bf16) {
-#pragma unroll 1
-        for (int cch = 0; cch < D / 32; ++cch) {
-          uint32_t v[32];
-          tmem_ld32(tO + cch * 32, v);
-          tmem_wait_ld();
-          reg_fence<32>(v);
-          if (valid) lane_store32_bf16(static_cast<uint16_t*>(part_o) + size_t(rec) * D + cch * 32, v, inv);
-          __syncwarp();   // valid differs across the warp's rows: converge before the next tcgen05.ld
-        }
-      } else if (bulk_o) {
-        // the warp's rows: tokens tt0 .. tt0 + 32/G - 1 of one block, all G heads
-        // (valid is warp-uniform here: a slot holds whole warps)
-        const int z0 = __shfl_sync(0xffffffffu, valid ? rec / p.Hq : 0, 0);
-        if (valid) {
-          uint32_t va[32], vb[32];
-          tmem_ld32(tO, va);
-          tmem_wait_ld();
-          reg_fence<32>(va);
-#pragma unroll
-          for (int cch = 0; cch < D / 32; cch += 2) {
-            tmem_ld32(tO + (cch + 1) * 32, vb);
-            warp_bulk_store16<1>(scratch, va, inv, &tm_o, cch * 32, g * p.G, z0);
-            warp_bulk_store16<1>(scratch + 512, va + 16, inv, &tm_o, cch * 32 + 16, g * p.G, z0);
-            tmem_wait_ld();
-            reg_fence<32>(vb);
-            if (cch + 2 < D / 32) tmem_ld32(tO + (cch + 2) * 32, va);
-            warp_bulk_store16<1>(scratch, vb, inv, &tm_o, (cch + 1) * 32, g * p.G, z0);
-            warp_bulk_store16<1>(scratch + 512, vb + 16, inv, &tm_o, (cch + 1) * 32 + 16, g * p.G, z0);
-            tmem_wait_ld();
-            reg_fence<32>(va);
-          }
-        }
-      } else {
-#pragma unroll 1
-        for (int cch = 0; cch < D / 32; ++cch) {
-          uint32_t v[32];
-          tmem_ld32(tO + cch * 32, v);
-          tmem_wait_ld();
-          reg_fence<32>(v);
-          warp_store_rows<32>(scratch, reinterpret_cast<const float*>(v), inv,
-                              valid ? static_cast<float*>(part_o) + size_t(rec) * D + cch * 32 : nullptr);
-        }
+      // the row's statistics for the epilogue warps: 1 / l, and the record's m_c (the
+      // true maximum, natural units) and l_c (the sum relative to it)
+      {
+        float4* st = reinterpret_cast<float4*>(smem + kOffStats) + ((st_cnt & 1) * 2 + x) * BM + r;
+        *st = make_float4(l > 0.f ? 1.f / l : 0.f, (l > 0.f) ? m_true * kLn2 : -INFINITY,
+                          (l > 0.f) ? l * fast_exp2(m_ref - m_true) : 0.f, 0.f);
+        __threadfence_block();
+        warp_arrive(&bars->stats_ready[x][st_cnt & 1]);
+        ++st_cnt;
       }
-      if (valid) {
-        // record (true max, sum relative to it)
-        part_m[rec] = (l > 0.f) ? m_true * kLn2 : -INFINITY;
-        part_l[rec] = (l > 0.f) ? l * fast_exp2(m_ref - m_true) : 0.f;
-      }
-      tc_fence_before();
-      warp_arrive(&bars->o_free[x]);
     }
-    // bulk stores of this warp complete before the CTA exits
-    if (lane == 0) bulk_wait0();
+    if (!ok) *abort_flag = 1;
+  } else if (warp >= 12) {
+    // ------------------------------------------------------------ record epilogue
+    // O_x of a finished tile from tensor memory to the record (times 1 / l), then the
+    // record's m_c and l_c; the output columns are released to the MMA right after the
+    // last TMEM read, so the next pair's first PV does not wait for the stores.
+    const int wq = warp & 3;
+    const int r = (wq << 5) + lane;   // row of the tile = TMEM lane
+    const uint32_t lane_addr = uint32_t(wq << 5) << 16;
+    float* scratch = reinterpret_cast<float*>(smem + kOffScratch) + wq * 1024;
+    PairIter pi;
+    pi.init(&p, w, &bars->ring, kClaimWarp, &wctx);
+    int tA, tB, g, klo, khi;
+    uint32_t pc[2] = {0, 0};
+    bool ok = true;
+    while (ok && pi.next(tA, tB, g, klo, khi)) {
+      for (int x = 0; x < 2; ++x) {
+        const int t = x == 0 ? tA : tB;
+        if (t < 0) continue;
+        const uint32_t tO = tmem + lane_addr + 256 + x * 128;
+        const int4 tile = p.tiles[t];
+        const int slot = r / rows_per_slot;
+        const int within = r - slot * rows_per_slot;
+        const int tt = within / p.G, hh = within - tt * p.G;
+        const bool valid = slot < tile.y - tile.x;
+        const int rec = valid ? ((tile.x + slot) * p.bs + tt) * p.Hq + g * p.G + hh : 0;
+        if (!warp_wait(&bars->o_full[x], pc[x] & 1, wctx, 1 * 10000 + __LINE__)) { ok = false; break; }
+        if (!warp_wait(&bars->stats_ready[x][pc[x] & 1], (pc[x] >> 1) & 1, wctx, 1 * 10000 + __LINE__)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const float4 st = reinterpret_cast<const float4*>(smem + kOffStats)[((pc[x] & 1) * 2 + x) * BM + r];
+        ++pc[x];
+#pragma unroll 1
+        for (int cch = 0; cch < D / 32; ++cch) {
+          uint32_t v[32];
+          tmem_ld32(tO + cch * 32, v);
+          tmem_wait_ld();
+          reg_fence<32>(v);
+          if (cch == D / 32 - 1) {
+            // every TMEM read of O_x done: the MMA may start the next pair's products into it
+            tc_fence_before();
+            warp_arrive(&bars->o_free[x]);
+          }
+          if (p.partial_bf16) {
+            if (valid) lane_store32_bf16(static_cast<uint16_t*>(part_o) + size_t(rec) * D + cch * 32, v, st.x);
+            __syncwarp();   // valid differs across the warp's rows: converge before the next tcgen05.ld
+          } else {
+            warp_store_rows<32>(scratch, reinterpret_cast<const float*>(v), st.x,
+                                valid ? static_cast<float*>(part_o) + size_t(rec) * D + cch * 32 : nullptr);
+          }
+        }
+        if (valid) {
+          part_m[rec] = st.y;
+          part_l[rec] = st.z;
+        }
+      }
+    }
     __syncwarp();
     if (!ok) *abort_flag = 1;
   }
@@ -597,17 +595,8 @@ bool fwd_sm100_supported(const DevPlan& p) {
 
 cudaError_t launch_fwd_partial_sm100(const DevPlan& p, const uint16_t* q, const uint16_t* k, const uint16_t* v,
                                      float scale, void* part_o, float* part_m, float* part_l, cudaStream_t s) {
-  CUtensorMap tq, tk, tv, to;
+  CUtensorMap tq, tk, tv;
   if (!make_bf16_map_3d(&tq, q, D, p.Hq, p.Nq, p.G, p.bs)) return cudaErrorInvalidValue;
-  // bulk record stores when a warp's 32 rows are 32/G whole tokens of one block
-  const bool bulk = 32 % p.G == 0 && (p.G * p.bs) % 32 == 0 && p.E > 0;
-  if (bulk) {
-    const bool ok = p.partial_bf16 ? make_bf16_store_map_3d(&to, part_o, D, p.Hq, uint64_t(p.E) * p.bs, p.G, 32 / p.G)
-                                   : make_f32_map_3d(&to, part_o, D, p.Hq, uint64_t(p.E) * p.bs, 16, p.G, 32 / p.G);
-    if (!ok) return cudaErrorInvalidValue;
-  } else {
-    memset(&to, 0, sizeof(to));
-  }
   if (!make_bf16_map_3d(&tk, k, D, p.Hkv, p.N, 1, BN)) return cudaErrorInvalidValue;
   if (!make_bf16_map_3d(&tv, v, D, p.Hkv, p.N, 1, BN)) return cudaErrorInvalidValue;
   cudaError_t e = cudaFuncSetAttribute(fwd_partial_sm100_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -615,8 +604,8 @@ cudaError_t launch_fwd_partial_sm100(const DevPlan& p, const uint16_t* q, const 
   if (e != cudaSuccess) return e;
   // run-time claims start from item 0 at every launch
   if (p.dynamic && (e = cudaMemsetAsync(p.claim + 0, 0, sizeof(int), s)) != cudaSuccess) return e;
-  fwd_partial_sm100_kernel<<<p.W, kThreads, kSmemBytes, s>>>(tq, tk, tv, to, p, scale * kLog2e, bulk ? 1 : 0,
-                                                             part_o, part_m, part_l);
+  fwd_partial_sm100_kernel<<<p.W, kThreads, kSmemBytes, s>>>(tq, tk, tv, p, scale * kLog2e, part_o, part_m,
+                                                             part_l);
   return cudaGetLastError();
 }
 

@@ -96,13 +96,15 @@ class Core:
 
 # ---------------------------------------------------------------------------
 # forward kernel: query tiles two at a time (A, B), K and V rings of two stages each (a
-# pair's first K/V tiles requested before its Q buffer frees)
+# pair's first K/V tiles requested before its Q buffer frees); the records leave through
+# separate epilogue warps (the tile's last PV and the softmax's row statistics, double-
+# buffered by pair parity, hand each tile over; the epilogue releases O after reading it)
 # ---------------------------------------------------------------------------
 class Forward(Core):
     def __init__(self, pairs, seed, drop=None):
         names = ["q_full", "q_empty", "k_full0", "k_full1", "v_full0", "v_full1", "k_empty0", "k_empty1",
                  "v_empty0", "v_empty1", "s_ready0", "s_ready1", "p_ready0", "p_ready1", "o_ready0", "o_ready1",
-                 "o_free0", "o_free1"]
+                 "o_free0", "o_free1", "o_full0", "o_full1", "stats0_0", "stats0_1", "stats1_0", "stats1_1"]
         super().__init__(seed, names)
         self.pairs = pairs            # [(nx, n_kt)]
         self.drop = drop
@@ -111,6 +113,7 @@ class Forward(Core):
         self.V = [None, None]
         self.S = [None, None]
         self.O = [None, None]
+        self.ST = {}                  # (tile, buffer) -> pair whose statistics it holds
         self.rescale = {}
 
     def producer(self):
@@ -177,6 +180,8 @@ class Forward(Core):
                             self.O[x] = ("acc", i, j + 1)
                     self.mma(pv)
                     self.commit(f"o_ready{x}")
+                    if not more:
+                        self.commit(f"o_full{x}")
                     if x == nx - 1:
                         self.commit(f"v_empty{c % 2}")
                     if more:
@@ -194,7 +199,7 @@ class Forward(Core):
 
     def softmax(self, x):
         kv = 0
-        s_cnt, o_cnt = 0, 0
+        s_cnt, o_cnt, st_cnt = 0, 0, 0
         for i, (nx, nkt) in enumerate(self.pairs):
             if x >= nx:
                 kv += nkt
@@ -210,16 +215,37 @@ class Forward(Core):
                 yield
                 self.S[x] = ("P", i, c)
                 self.B[f"p_ready{x}"].arrive()
-            yield from self.wait(f"o_ready{x}", o_cnt + nkt - 1)
             o_cnt += nkt
-            self.check(self.O[x] == ("acc", i, nkt), f"epilogue({x}) of pair {i} finds {self.O[x]}")
-            yield
-            self.O[x] = ("stored", i)
-            self.B[f"o_free{x}"].arrive()
+            yield                         # the statistics are written after the last P is handed over
+            b = st_cnt % 2
+            self.check(self.ST.get((x, b), ("read",))[0] == "read", f"stats({x},{b}) of pair {i} overwrite unread "
+                       f"{self.ST.get((x, b))}")
+            self.ST[(x, b)] = ("written", i)
+            self.B[f"stats{x}_{b}"].arrive()
+            st_cnt += 1
             kv += nkt
 
+    def epilogue(self):
+        pc = [0, 0]
+        for i, (nx, nkt) in enumerate(self.pairs):
+            for x in range(nx):
+                yield from self.wait(f"o_full{x}", pc[x])
+                b = pc[x] % 2
+                if self.drop != "stats":
+                    yield from self.wait(f"stats{x}_{b}", pc[x] // 2)
+                self.check(self.ST.get((x, b)) == ("written", i), f"epilogue({x}) of pair {i} finds stats "
+                           f"{self.ST.get((x, b))}")
+                self.ST[(x, b)] = ("read", i)
+                self.check(self.O[x] == ("acc", i, nkt), f"epilogue({x}) of pair {i} finds {self.O[x]}")
+                pc[x] += 1
+                yield
+                self.O[x] = ("stored", i)
+                self.B[f"o_free{x}"].arrive()
+                yield
+
     def go(self):
-        self.run({"prod": self.producer(), "mma": self.mma_thread(), "smA": self.softmax(0), "smB": self.softmax(1)})
+        self.run({"prod": self.producer(), "mma": self.mma_thread(), "smA": self.softmax(0), "smB": self.softmax(1),
+                  "epi": self.epilogue()})
 
 
 # ---------------------------------------------------------------------------
@@ -520,13 +546,16 @@ def test_protocol_holds_on_random_schedules(kernel):
         CASES[kernel](rng, seed).go()
 
 
-@pytest.mark.parametrize("kernel,drop", [("forward", "kv_empty"), ("forward", "q_empty"), ("dkdv", "qd_empty"),
+@pytest.mark.parametrize("kernel,drop", [("forward", "kv_empty"), ("forward", "q_empty"), ("forward", "o_free"),
+                                         ("forward", "stats"),
+                                         ("dkdv", "qd_empty"),
                                          ("dkdv", "kv_empty"), ("dkdv", "lookahead_before_dv"), ("dq", "kv_empty"),
                                          ("dq", "qd_empty")])
 def test_each_producer_guard_is_needed(kernel, drop):
     """Removing one of the producer's waits lets some schedule overwrite a stage that an
     MMA has not read yet; issuing the dK/dV kernel's look-ahead S^T before dV instead of
-    after it overwrites a P^T that dV has not read."""
+    after it overwrites a P^T that dV has not read; without the forward MMA's wait for the
+    epilogue warps to release O, the next pair's first PV overwrites an O not yet read."""
     rng = random.Random(5)
     caught = 0
     for seed in range(300):
@@ -537,12 +566,13 @@ def test_each_producer_guard_is_needed(kernel, drop):
     assert caught > 0
 
 
-@pytest.mark.parametrize("kernel,drop", [("forward", "o_free"), ("dkdv", "dkv_free"), ("dq", "dq_free")])
+@pytest.mark.parametrize("kernel,drop", [("dkdv", "dkv_free"), ("dq", "dq_free")])
 def test_epilogue_release_is_implied_by_program_order(kernel, drop):
-    """The MMA thread's wait for the epilogue to release an accumulator is redundant: the
-    epilogue runs on the element-wise warps before their next pass, which the first product
-    into the accumulator already waits for.  The kernels keep the wait as a guard; these
-    schedules show that nothing depends on it."""
+    """In the backward kernels the MMA thread's wait for the epilogue to release an
+    accumulator is redundant: the epilogue runs on the element-wise warps before their next
+    pass, which the first product into the accumulator already waits for.  The kernels keep
+    the wait as a guard; these schedules show that nothing depends on it.  (The forward's
+    epilogue runs on warps of its own, so there the wait is needed: see above.)"""
     rng = random.Random(6)
     for seed in range(150):
         CASES[kernel](rng, seed, drop).go()
