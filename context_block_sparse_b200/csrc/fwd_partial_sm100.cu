@@ -24,12 +24,11 @@
 //               so that the softmax warps go on to the next pair at once and the
 //               output columns return to the MMA right after their last read.
 // The softmax keeps, per row, a reference maximum m_ref, taken from the first
-// key tile in which the row has allowed keys (the only tile that reads S from
-// TMEM twice); later tiles exponentiate against it in one pass and only when a
-// score exceeds m_ref by more than 2^32 (in P) are O, l and the P already
-// written rescaled to a new reference -- the result is the same, the reference
-// is exact bookkeeping.  The record written is m_c = the row's true maximum
-// (natural units), l_c = sum exp(s - m_c) and O_c = sum exp(s - m_c) v / l_c.
+// 64-column half in which the row has allowed keys; every half is exponentiated
+// against it in one pass, and only when a score exceeds m_ref by more than 2^32
+// (in P) are O, l and the P already written rescaled to a new reference -- the
+// result is the same, the reference is exact bookkeeping.  The record written
+// is m_c = the row's true maximum (natural units), l_c = sum exp(s - m_c) and O_c = sum exp(s - m_c) v / l_c.
 // Rows are masked to their block's [lo, hi).  The epilogue stores go through a
 // 4 KB per-warp staging buffer so that every store instruction writes whole
 // 128-byte row segments (bf16 records: 64 bytes per row straight from registers).
@@ -423,22 +422,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         const bool none = b <= 0 || a >= BN;
         // warp-uniform: the two exp_pack_store variants issue warp-collective tcgen05.st
         const bool full = __all_sync(0xffffffffu, a <= 0 && b >= BN);
-        // first allowed keys of a row: its reference is this tile's maximum (O and
-        // l of the row are still zero, nothing to rescale)
-        if (__any_sync(0xffffffffu, m_ref == -INFINITY && !none)) {
-          float mxr = -INFINITY;
-#pragma unroll 1
-          for (int h = 0; h < BN / 64; ++h) {
-            uint32_t v[64];
-            tmem_ld32p(tS + h * 64, v);
-            tmem_ld32p(tS + h * 64 + 32, v + 32);
-            tmem_wait_ld();
-            reg_fence<64>(v);
-            mxr = fmaxf(mxr, full ? row_max<false>(v, a - h * 64, b - h * 64)
-                                  : row_max<true>(v, a - h * 64, b - h * 64));
-          }
-          if (m_ref == -INFINITY && !none) m_ref = mxr * scale_log2;
-        }
         // one pass per 64-column half: maximum, P = exp2(s * scale_log2 - m_ref)
         // (masked -> 0), row sum, bf16 P into TMEM columns 32h..32h+31 of S_X
         // (columns already read)
@@ -453,6 +436,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           const float mh = scale_log2 * (full ? row_max<false>(v, a - h * 64, b - h * 64)
                                               : row_max<true>(v, a - h * 64, b - h * 64));
           mx = fmaxf(mx, mh);
+          // a row's first allowed keys set its reference (its O and l are still zero);
+          // later halves past the headroom take the rescale below
+          if (m_ref == -INFINITY) m_ref = mh;
           const bool over = mh > m_ref + kHeadroomLog2;
           if (__any_sync(0xffffffffu, over)) {
             // new reference for the rows past the headroom: rescale O (after PV(j-1)),
