@@ -376,6 +376,12 @@ def splitkv_attn_fwd_static_scratch(plan: Plan, q, k, v, kb, vb, scale: float, o
         _ptr(o), _o_dtype(o), _f32_ptr(lse), _stream_ptr(stream)))
 
 
+def splitkv_plan_set_wait_limit(plan: Plan, ns: int) -> None:
+    """Time limit (ns) of the mbarrier waits in this plan's tcgen05 kernels (default 2e9);
+    from the next launch on."""
+    _check("splitkv_plan_set_wait_limit", _lib.splitkv_plan_set_wait_limit(plan.handle, int(ns)))
+
+
 def splitkv_plan_status(plan: Plan, stream=None) -> None:
     """Raise SplitKVError if a kernel of this plan recorded an error (e.g. a timed-out wait)."""
     site = ctypes.c_int32(0)

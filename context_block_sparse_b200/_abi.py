@@ -128,6 +128,7 @@ SIGNATURES = {
     "splitkv_bwd_dq": (_I, [_P, _P, _P, _P, _P, _P, _F, _P, _SZ, _P]),
     "splitkv_attn_fwd_static_scratch": (_I, [_P, _P, _P, _P, _P, _P, _F, _P, _I, _P, _P]),
     "splitkv_plan_status": (_I, [_P, _P, ctypes.POINTER(ctypes.c_int32)]),
+    "splitkv_plan_set_wait_limit": (_I, [_P, ctypes.c_int64]),
     "splitkv_selftest_exp2": (_I, [_P, _P, ctypes.c_int64, _P]),
     "splitkv_selftest_wait_timeout": (_I, [ctypes.POINTER(ctypes.c_int32), _P]),
     "splitkv_read_cta_times": (_I, [_P, _I, ctypes.POINTER(ctypes.c_int64), ctypes.c_int64, _P]),

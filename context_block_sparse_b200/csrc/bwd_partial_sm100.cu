@@ -286,7 +286,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int w = blockIdx.x;
   volatile int* abort_flag = &B->abort_flag;
-  const WaitCtx wctx{abort_flag, p.status};
+  const WaitCtx wctx{abort_flag, p.status, p.wait_limit_ns};
   if (tid == 0) {
     p.timers[(p.W + w) * 2 + 0] = global_timer_ns();
     B->abort_flag = 0;
@@ -650,7 +650,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int w = blockIdx.x;
   volatile int* abort_flag = &B->abort_flag;
-  const WaitCtx wctx{abort_flag, p.status};
+  const WaitCtx wctx{abort_flag, p.status, p.wait_limit_ns};
   if (tid == 0) {
     p.timers[(p.W + p.Wb + w) * 2 + 0] = global_timer_ns();
     B->abort_flag = 0;

@@ -34,6 +34,9 @@ struct Item {
 
 }  // namespace
 
+// Largest wait limit a plan accepts (a minute): a wait that long has failed.
+constexpr int64_t kMaxWaitLimitNs = 60000000000LL;
+
 struct splitkv_plan_s {
   // problem
   int32_t S = 0, A = 0, bs = 0, Hq = 0, Hkv = 0, d = 0, C = 0, W = 0, Wb = 0, q_slice = 0;
@@ -68,6 +71,7 @@ struct splitkv_plan_s {
   cudaEvent_t upload_ev = nullptr;
   bool upload_pending = false;
   bool uploaded = false;
+  int64_t wait_limit_ns = 2000000000LL;            // splitkv_plan_set_wait_limit
   DevPlan dev{};
 };
 
@@ -740,7 +744,15 @@ int splitkv_plan_upload(splitkv_plan_t* P, void* stream) {
   v.n_fwd_items = int(P->fwd_items.size());
   v.n_bwd_items = int(P->bwd_items.size());
   v.claim = reinterpret_cast<int*>(d + status_off + 128);   // after the two status words
+  v.wait_limit_ns = P->wait_limit_ns;
   P->uploaded = true;
+  return SPLITKV_OK;
+}
+
+int splitkv_plan_set_wait_limit(splitkv_plan_t* P, int64_t ns) {
+  if (!P || ns < 0 || ns > kMaxWaitLimitNs) return SPLITKV_ERR_INVALID_ARG;
+  P->wait_limit_ns = ns;
+  P->dev.wait_limit_ns = ns;   // takes effect from the next launch (the device view is passed by value)
   return SPLITKV_OK;
 }
 

@@ -35,7 +35,7 @@ __global__ void wait_timeout_kernel(int* status) {
     splitkv::sm100::mbar_fence_init();
   }
   __syncthreads();
-  const splitkv::sm100::WaitCtx c{&abort_flag, status};
+  const splitkv::sm100::WaitCtx c{&abort_flag, status, splitkv::sm100::kWaitLimitNs};
   if (threadIdx.x == 0)
     splitkv::sm100::mbar_wait(&bar, 0, c, 9 * 10000 + __LINE__);
   else if (threadIdx.x >= 32)

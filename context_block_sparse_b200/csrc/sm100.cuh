@@ -15,7 +15,10 @@ namespace sm100 {
 // A wait that has not completed after this long has failed (a bug): the
 // kernel records a timeout and the waiting site in its status words and winds
 // down instead of hanging the GPU.  Bounded in time, not in iterations, because
-// mbarrier.try_wait may suspend the thread between polls.
+// mbarrier.try_wait may suspend the thread between polls.  The kernels' ordinary
+// waits take the plan's limit (this by default; a test may shorten it to make a
+// wait run out); the drains of copies and products in flight on the way out
+// always take this one, so that nothing is left writing after the CTA exits.
 constexpr long long kWaitLimitNs = 2000000000LL;
 
 // ---------------------------------------------------------------- mbarrier
@@ -57,6 +60,7 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 struct WaitCtx {
   volatile int* abort_flag;
   int* status;
+  long long limit_ns;   // time limit of mbar_wait / warp_wait
 };
 
 __device__ __forceinline__ void record_timeout(const WaitCtx& c, int site) {
@@ -66,15 +70,17 @@ __device__ __forceinline__ void record_timeout(const WaitCtx& c, int site) {
 }
 
 // Wait for the phase of `parity` to complete.  Returns false when the time
-// limit passes (recorded with `site`) or another role has flagged an abort.
+// limit passes (recorded with `site`) or another role has flagged an abort.  The
+// clock is read every 64 polls, or at every poll under a limit below 1 us (a
+// limit of 0 gives up at the first poll that finds the phase incomplete).
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const WaitCtx& c, int site) {
   if (mbar_try_wait(bar, parity)) return true;
   const long long t0 = global_timer_ns();
   for (uint32_t i = 1;; ++i) {
     if (mbar_try_wait(bar, parity)) return true;
-    if ((i & 63u) == 0) {
+    if ((i & 63u) == 0 || c.limit_ns < 1000) {
       if (*c.abort_flag) return false;
-      if (global_timer_ns() - t0 > kWaitLimitNs) {
+      if (global_timer_ns() - t0 >= c.limit_ns) {
         record_timeout(c, site);
         return false;
       }
@@ -457,12 +463,13 @@ __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.
 // and subtracting 1.5 * 2^23), f in [-0.5, 0.5], a cubic fitted here to 2^f on
 // that interval (weighted least squares on the relative error, max relative
 // error 7.6e-5 in fp32, far below bf16's 3.9e-3), and the exponent n added
-// to the result's bits.  x is clamped at -126 (the result is then below 2^-125,
-// i.e. zero for bf16 P and negligible in fp32 sums).
+// to the result's bits.  Below -126 (and for -inf, a masked score) the result
+// is exactly 0, as MUFU's is for -inf.
 constexpr float kExpMagic = 12582912.0f;   // 1.5 * 2^23
 constexpr float kExpC0 = 0.99992758f, kExpC1 = 0.69326109f, kExpC2 = 0.24261758f, kExpC3 = 0.055174146f;
 
 __device__ __forceinline__ void exp2_poly2(float x0, float x1, float& y0, float& y1) {
+  const bool z0 = x0 < -126.f, z1 = x1 < -126.f;
   x0 = fmaxf(x0, -126.f);
   x1 = fmaxf(x1, -126.f);
   float t0, t1, n0, n1, f0, f1, p0, p1;
@@ -472,8 +479,8 @@ __device__ __forceinline__ void exp2_poly2(float x0, float x1, float& y0, float&
   ffma2(p0, p1, f0, f1, kExpC3, kExpC3, kExpC2, kExpC2);
   ffma2(p0, p1, p0, p1, f0, f1, kExpC1, kExpC1);
   ffma2(p0, p1, p0, p1, f0, f1, kExpC0, kExpC0);
-  y0 = __uint_as_float(__float_as_uint(p0) + (__float_as_uint(t0) << 23));
-  y1 = __uint_as_float(__float_as_uint(p1) + (__float_as_uint(t1) << 23));
+  y0 = z0 ? 0.f : __uint_as_float(__float_as_uint(p0) + (__float_as_uint(t0) << 23));
+  y1 = z1 ? 0.f : __uint_as_float(__float_as_uint(p1) + (__float_as_uint(t1) << 23));
 }
 
 // exp2 of two lanes on MUFU (poly = false) or on the FMA pipe (poly = true);

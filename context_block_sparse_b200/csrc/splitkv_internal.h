@@ -39,6 +39,9 @@ struct DevPlan {
   int dynamic;
   int n_fwd_items, n_bwd_items;
   int* claim;                   // [4]
+  // time limit of the kernels' mbarrier waits (ns; splitkv_plan_set_wait_limit), after
+  // which a wait records SPLITKV_ERR_TIMEOUT and the kernel winds down
+  long long wait_limit_ns;
 };
 
 // Byte offsets of the forward workspace (partial records).

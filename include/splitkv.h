@@ -407,6 +407,18 @@ int splitkv_attn_fwd_static_scratch(const splitkv_plan_t* plan, const void* q, c
                                     const void* v, const void* kb, const void* vb, float scale,
                                     void* o, int o_dtype, float* lse, void* stream);
 
+/* Time limit of the mbarrier waits inside this plan's tcgen05 kernels, in
+ * nanoseconds of the device global timer (default 2e9, the limit of every
+ * wait; 0 <= ns <= 6e10, else INVALID_ARG).  A wait that runs past it records
+ * SPLITKV_ERR_TIMEOUT and its site in the plan's status words (read by
+ * splitkv_plan_status), and the kernel winds down: every role stops, the copies
+ * and products already in flight are awaited (with the default limit) and the
+ * tensor memory is freed, so the context stays usable and the next launch runs
+ * normally.  Takes effect from the next launch; host-only.  This is the failure
+ * detection of the kernels made testable: a test sets a limit no wait can meet
+ * and checks the status.  The pages have no counterpart to it. */
+int splitkv_plan_set_wait_limit(splitkv_plan_t* plan, int64_t ns);
+
 /* Device status of the plan's kernels: synchronises `stream`, returns
  * SPLITKV_OK, or the SPLITKV_ERR_* code a kernel recorded since the last call
  * (SPLITKV_ERR_TIMEOUT: a wait inside a kernel passed its 2-second limit and

@@ -73,3 +73,60 @@ def test_a_wait_nothing_completes_times_out_and_the_context_survives(splitkv):
     out, _, _ = run(w, bwd=True)
     g = oracle_bwd(w)
     assert_close("dq", out["dq"], g["dq"], TOL_OUT)
+
+
+@pytest.mark.parametrize("claims", [False, True])
+def test_waits_past_the_plan_limit_wind_the_attention_kernels_down(splitkv, claims):
+    """Failure detection of the attention kernels themselves: under a plan wait limit of 0 a
+    wait gives up at the first poll that finds its barrier incomplete.  The forward kernel and
+    the two backward kernels then record SPLITKV_ERR_TIMEOUT with the site of the wait, drain
+    their copies and products in flight, free their tensor memory and return (no hang, no
+    fault); with the default limit restored, the same plan on the same device matches the
+    oracle again."""
+    import torch
+    from context_block_sparse_b200.torch_api import SplitKVAttention
+    from gpu_util import TOL_LSE, TOL_OUT, assert_close, oracle_bwd, oracle_fwd
+    skv = splitkv
+    w = small(Hq=4, Hkv=1, d=128)                      # the smallest shape of the tcgen05 kernels
+    t = {n: to_dev(b) for n, b in w.bits.items()}
+    att = SplitKVAttention(w.sample_lens, w.anchors, w.block_size, w.num_q_heads, w.num_kv_heads, w.head_dim,
+                           w.kv_chunk, q_slice=1 if claims else 0, dynamic_claim=claims)
+    o, lse = att.forward(t["q"], t["k"], t["v"], t["kb"], t["vb"], w.scale)
+    torch.cuda.synchronize()
+    skv.splitkv_plan_status(att.plan)                  # a normal run first: no error
+
+    skv.splitkv_plan_set_wait_limit(att.plan, 0)
+    att.forward(t["q"], t["k"], t["v"], t["kb"], t["vb"], w.scale)
+    torch.cuda.synchronize()
+    with pytest.raises(skv.SplitKVError) as ei:
+        skv.splitkv_plan_status(att.plan)
+    assert ei.value.status == -5 and ei.value.site // 10000 == 1, (ei.value.status, ei.value.site)
+    skv.splitkv_plan_status(att.plan)                  # read and cleared
+    att.backward(t["q"], t["k"], t["v"], t["kb"], t["vb"], o, lse, t["dout"], w.scale)
+    torch.cuda.synchronize()
+    with pytest.raises(skv.SplitKVError) as ei:
+        skv.splitkv_plan_status(att.plan)
+    assert ei.value.status == -5 and ei.value.site // 10000 == 2, (ei.value.status, ei.value.site)
+
+    skv.splitkv_plan_set_wait_limit(att.plan, 2_000_000_000)
+    o, lse = att.forward(t["q"], t["k"], t["v"], t["kb"], t["vb"], w.scale)
+    g = att.backward(t["q"], t["k"], t["v"], t["kb"], t["vb"], o, lse, t["dout"], w.scale)
+    torch.cuda.synchronize()
+    skv.splitkv_plan_status(att.plan)
+    O, L = oracle_fwd(w)
+    assert_close("O", o.cpu().numpy().astype("float64"), O, TOL_OUT)
+    assert_close("LSE", lse.cpu().numpy().astype("float64"), L, TOL_LSE)
+    ref = oracle_bwd(w)
+    for n in ("dq", "dk", "dv"):
+        assert_close(n, g[n].cpu().numpy().astype("float64"), ref[n], TOL_OUT)
+
+
+def test_wait_limit_argument_checks(splitkv):
+    skv = splitkv
+    w = small(Hq=4, Hkv=1, d=128, grad=False)
+    plan = skv.splitkv_plan(w.sample_lens, w.anchors, w.block_size, w.num_q_heads, w.num_kv_heads, w.head_dim,
+                            w.kv_chunk, 148)
+    assert skv._lib.splitkv_plan_set_wait_limit(plan.handle, -1) == -1
+    assert skv._lib.splitkv_plan_set_wait_limit(plan.handle, 61_000_000_000) == -1
+    assert skv._lib.splitkv_plan_set_wait_limit(None, 5) == -1
+    assert skv._lib.splitkv_plan_set_wait_limit(plan.handle, 5) == 0

@@ -22,3 +22,15 @@ def test_poly_exp2_relative_error(splitkv):
     assert float(rel.max()) < 1e-4, float(rel.max())
     tiny = y[~keep]
     assert bool((tiny >= 0).all()) and float(tiny.max()) < 1e-30
+
+
+def test_poly_exp2_is_zero_below_the_normal_range_and_for_minus_infinity(splitkv):
+    """Masked scores reach the exponential as -inf: the FMA-pipe exp2 gives exactly 0 there,
+    as the MUFU one does, and for any input below -126."""
+    import torch
+    x = torch.tensor([float("-inf"), -1e30, -300.0, -127.0, -126.5], device="cuda")
+    y = torch.full_like(x, 1.0)
+    st = splitkv._lib.splitkv_selftest_exp2(x.data_ptr(), y.data_ptr(), ctypes.c_int64(x.numel()),
+                                            ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+    assert st == 0
+    assert y.cpu().tolist() == [0.0] * 5
