@@ -18,8 +18,10 @@
 //   warp 1      MMA issuer (one thread): S_X = Q_X K^T into TMEM, then
 //               O_X += P_X V with P_X read from TMEM (bf16, aliasing S_X);
 //   warp 2      tensor-memory allocation (512 columns: S_A, S_B, O_A, O_B);
-//   warps 4-7   softmax of tile A (thread = row = TMEM lane);
-//   warps 8-11  softmax of tile B;
+//   warps 4-11  softmax of both tiles (A, then B, at every key tile): warps 4-7
+//               take score columns 0..63, warps 8-11 columns 64..127 (thread =
+//               row = TMEM lane); the two threads of a row agree on the key
+//               tile's row maximum through shared memory before exponentiating;
 //   warps 12-15 record epilogue of both tiles: O_X / l from TMEM to the record,
 //               so that the softmax warps go on to the next pair at once and the
 //               output columns return to the MMA right after their last read.
@@ -68,7 +70,8 @@ constexpr uint32_t kOffK = kOffQ + 2 * kTile;              // K stages
 constexpr uint32_t kOffV = kOffK + kStages * kTile;        // V stages
 constexpr uint32_t kOffScratch = kOffV + kStages * kTile; // record staging, 4 KB per epilogue warp
 constexpr uint32_t kOffStats = kOffScratch + 4 * 4096;     // row statistics [2 pair parities][2 tiles][128] float4
-constexpr uint32_t kOffBar = kOffStats + 2 * 2 * BM * 16;  // mbarriers
+constexpr uint32_t kOffXchg = kOffStats + 2 * 2 * BM * 16;  // half maxima [2 exchange parities][2 halves][128] float
+constexpr uint32_t kOffBar = kOffXchg + 2 * 2 * BM * 4;     // mbarriers
 constexpr uint32_t kSmemBytes = kOffBar + 512 + 1024;      // + alignment slack
 static_assert(kSmemBytes <= 232448, "shared memory per block");
 
@@ -80,6 +83,9 @@ struct Bars {
   // stats_ready[x][b]: the softmax warps of tile x left the row statistics of a pair
   // in stats buffer b = pair parity
   uint64_t o_full[2], stats_ready[2][2];
+  // xchg[q]: the two warps holding rows 32q..32q+31 (one per 64-column half) have
+  // left their halves' maxima of a key tile (count 2 warps)
+  uint64_t xchg[4];
   uint64_t mma_done;
   ClaimRing ring;   // run-time claims: the producer hands items to the MMA thread and the 8 softmax warps
   uint32_t tmem_base;
@@ -133,30 +139,33 @@ struct PairIter {
 };
 
 
-// Maximum of 64 raw scores of one row over its allowed columns [a, b) of them
-// (-inf when none is allowed).
-template <bool kMasked>
-__device__ __forceinline__ float row_max(const uint32_t (&v)[64], int a, int b) {
+// One row of one query tile in the softmax warps: its allowed keys [lo, hi), the
+// reference maximum and the true maximum (log2 units) and the sum of P (relative to
+// the reference) over this thread's half of the columns.
+struct RowState {
+  int lo, hi;
+  float m_ref, m_true, l;
+};
+
+// Maximum of 64 raw scores of one row (masked scores are -inf).
+__device__ __forceinline__ float row_max(const uint32_t (&v)[64]) {
   float m0 = -INFINITY, m1 = -INFINITY, m2 = -INFINITY, m3 = -INFINITY;
 #pragma unroll
   for (int i = 0; i < 64; i += 8) {
-    float u[8];
-#pragma unroll
-    for (int k = 0; k < 8; ++k)
-      u[k] = (!kMasked || (i + k >= a && i + k < b)) ? __uint_as_float(v[i + k]) : -INFINITY;
-    m0 = fmax3(m0, u[0], u[1]);
-    m1 = fmax3(m1, u[2], u[3]);
-    m2 = fmax3(m2, u[4], u[5]);
-    m3 = fmax3(m3, u[6], u[7]);
+    m0 = fmax3(m0, __uint_as_float(v[i]), __uint_as_float(v[i + 1]));
+    m1 = fmax3(m1, __uint_as_float(v[i + 2]), __uint_as_float(v[i + 3]));
+    m2 = fmax3(m2, __uint_as_float(v[i + 4]), __uint_as_float(v[i + 5]));
+    m3 = fmax3(m3, __uint_as_float(v[i + 6]), __uint_as_float(v[i + 7]));
   }
   return fmaxf(fmaxf(m0, m1), fmaxf(m2, m3));
 }
 
-// P = exp2(v * c + nm) over 64 columns of a row (0 outside [a, b)), packed to
-// bf16 pairs into 32 TMEM columns at tS; returns the row sum of the fp32 P.
-template <bool kMasked>
-__device__ __forceinline__ float exp_pack_store(const uint32_t (&v)[64], int a, int b, float c, float nm,
-                                                uint32_t tS) {
+// P = exp2(v * c + nm) over 64 columns of a row (exactly 0 for a masked score,
+// -inf), packed to bf16 pairs into 32 TMEM columns at tS; returns the row sum of
+// the fp32 P.  MUFU for every pair: the two softmax warps of an SM sub-partition
+// share one tile, so its exponentials take 1024 MUFU cycles, below the tile's two
+// products; the FMA-pipe polynomial would only add registers (and spills).
+__device__ __forceinline__ float exp_pack_store(const uint32_t (&v)[64], float c, float nm, uint32_t tS) {
   float s0 = 0.f, s1 = 0.f;
 #pragma unroll
   for (int cch = 0; cch < 2; ++cch) {
@@ -166,12 +175,7 @@ __device__ __forceinline__ float exp_pack_store(const uint32_t (&v)[64], int a, 
       const int col = cch * 32 + 2 * i;
       float x0, x1;
       ffma2(x0, x1, __uint_as_float(v[col]), __uint_as_float(v[col + 1]), c, c, nm, nm);
-      float p0, p1;
-      exp2_pair((i % kPolyEvery) == 1, x0, x1, p0, p1);
-      if (kMasked) {
-        p0 = (col >= a && col < b) ? p0 : 0.f;
-        p1 = (col + 1 >= a && col + 1 < b) ? p1 : 0.f;
-      }
+      const float p0 = fast_exp2(x0), p1 = fast_exp2(x1);
       fadd2(s0, s1, s0, s1, p0, p1);
       pk[i] = pack_bf16(p0, p1);
     }
@@ -191,7 +195,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int w = blockIdx.x;
   volatile int* abort_flag = &bars->abort_flag;
-  const WaitCtx wctx{abort_flag, p.status};
+  const WaitCtx wctx{abort_flag, p.status, p.wait_limit_ns};
 
   if (tid == 0) {
     p.timers[w * 2 + 0] = global_timer_ns();
@@ -205,14 +209,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int x = 0; x < 2; ++x) {
       mbar_init(&bars->s_ready[x], 1);
-      mbar_init(&bars->p_ready[x], 4);    // one arrival per softmax warp
+      mbar_init(&bars->p_ready[x], 8);    // one arrival per softmax warp
       mbar_init(&bars->o_ready[x], 1);
       mbar_init(&bars->o_free[x], 4);      // one arrival per epilogue warp
       mbar_init(&bars->o_full[x], 1);
-      mbar_init(&bars->stats_ready[x][0], 4);
-      mbar_init(&bars->stats_ready[x][1], 4);
+      mbar_init(&bars->stats_ready[x][0], 8);
+      mbar_init(&bars->stats_ready[x][1], 8);
     }
     mbar_init(&bars->mma_done, 1);
+    for (int q = 0; q < 4; ++q) mbar_init(&bars->xchg[q], 2);
     claim_ring_init(&bars->ring, kClaimConsumers);
     bars->abort_flag = 0;
     mbar_fence_init();
@@ -347,10 +352,13 @@ __global__ void __launch_bounds__(kThreads, 1)
               if (!mbar_wait(&bars->v_full[s], (c / kStages) & 1, wctx, 1 * 10000 + __LINE__)) { ok = false; break; }
             }
             tc_fence_after();
-            // O_X (+)= P_X V : P in TMEM (columns 0..63 of S_X), V MN-major in smem
+            // O_X (+)= P_X V : P in TMEM (keys 0..63 in columns 0..31 of S_X, keys
+            // 64..127 in columns 64..95: each half written over the scores it replaces),
+            // V MN-major in smem
             for (int kk = 0; kk < BN / 16; ++kk) {
               const uint64_t b = smem_desc_sw128(sV + s * kTile + kk * 2048, kHalf, 1024);
-              mma_ts(tmem + 256 + x * 128, tmem + x * 128 + kk * 8, b, kIdescPV, (j > 0 || kk > 0) ? 1u : 0u);
+              const uint32_t pcol = kk < 4 ? kk * 8 : 64 + (kk - 4) * 8;
+              mma_ts(tmem + 256 + x * 128, tmem + x * 128 + pcol, b, kIdescPV, (j > 0 || kk > 0) ? 1u : 0u);
             }
             mma_commit(&bars->o_ready[x]);
             if (!more) mma_commit(&bars->o_full[x]);           // tile x's output complete
@@ -388,118 +396,138 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp >= 4 && warp < 12) {
     // ------------------------------------------------------------ softmax
-    const int x = (warp - 4) >> 2;            // tile A (warps 4-7) or B (warps 8-11)
-    const int r = ((warp & 3) << 5) + lane;   // row of the tile = TMEM lane
-    const uint32_t lane_addr = uint32_t((warp & 3) << 5) << 16;
-    const uint32_t tS = tmem + lane_addr + x * 128;
-    const uint32_t tO = tmem + lane_addr + 256 + x * 128;   // O_X: rescaled in place on a new reference
+    // Warps 4-7 take columns 0..63 of every score tile, warps 8-11 columns 64..127;
+    // both tiles of a pair go through the same warps (A then B at every key tile).
+    // The two threads of a row agree on its key-tile maximum through shared memory
+    // before exponentiating, so they keep one reference and one O.
+    const int h = (warp - 4) >> 2;            // column half
+    const int wq = warp & 3;
+    const int r = (wq << 5) + lane;           // row of the tile = TMEM lane
+    const uint32_t lane_addr = uint32_t(wq << 5) << 16;
+    float* xs = reinterpret_cast<float*>(smem + kOffXchg);
     PairIter pi;
     pi.init(&p, w, &bars->ring, kClaimWarp, &wctx);
     int tA, tB, g, klo, khi;
-    uint32_t s_cnt = 0, o_cnt = 0, st_cnt = 0;
+    uint32_t s_cntA = 0, s_cntB = 0, o_cntA = 0, o_cntB = 0, st_cntA = 0, st_cntB = 0, n_x = 0;
     bool ok = true;
     while (ok && pi.next(tA, tB, g, klo, khi)) {
-      const int t = x == 0 ? tA : tB;
-      if (t < 0) continue;                    // no tile B in this pair
+      const int nx = tB >= 0 ? 2 : 1;
       const int n_kt = (khi - klo + BN - 1) / BN;
-      const int4 tile = p.tiles[t];
-      const int slot = r / rows_per_slot;
-      const bool valid = slot < tile.y - tile.x;
-      int lo = 0, hi = 0;   // the row's allowed keys (none for a padding row)
-      if (valid) {
-        const int4 ent = p.entries[tile.x + slot];
-        lo = ent.y;
-        hi = ent.z;
-      }
-      float m_ref = -INFINITY, m_true = -INFINITY, l = 0.f;
-      for (int j = 0; j < n_kt && ok; ++j) {
-        if (!warp_wait(&bars->s_ready[x], s_cnt & 1, wctx, 1 * 10000 + __LINE__)) { ok = false; break; }
-        ++s_cnt;
-        tc_fence_after();
-        const int k0 = klo + j * BN;
-        // the row's allowed columns in this key tile: [a, b)
-        const int a = lo - k0, b = hi - k0;
-        const bool none = b <= 0 || a >= BN;
-        // warp-uniform: the two exp_pack_store variants issue warp-collective tcgen05.st
-        const bool full = __all_sync(0xffffffffu, a <= 0 && b >= BN);
-        // one pass per 64-column half: maximum, P = exp2(s * scale_log2 - m_ref)
-        // (masked -> 0), row sum, bf16 P into TMEM columns 32h..32h+31 of S_X
-        // (columns already read)
-        float mx = -INFINITY;
-#pragma unroll 1
-        for (int h = 0; h < BN / 64; ++h) {
+      RowState rsA, rsB;
+      auto init_row = [&](RowState& st, const int t) {
+        st.lo = st.hi = 0;   // the row's allowed keys (none for a padding row)
+        st.m_ref = st.m_true = -INFINITY;
+        st.l = 0.f;
+        if (t >= 0) {
+          const int4 tile = p.tiles[t];
+          const int slot = r / rows_per_slot;
+          if (slot < tile.y - tile.x) {
+            const int4 ent = p.entries[tile.x + slot];
+            st.lo = ent.y;
+            st.hi = ent.z;
+          }
+        }
+      };
+      init_row(rsA, tA);
+      init_row(rsB, tB);
+      // key tile j of tile x: false when a wait gave up
+      auto step = [&](RowState& st, uint32_t& sc, const uint32_t oc, const int x, const int j) -> bool {
+          const uint32_t tS = tmem + lane_addr + x * 128;
+          const uint32_t tO = tmem + lane_addr + 256 + x * 128;   // O_X: rescaled in place on a new reference
+          if (!warp_wait(&bars->s_ready[x], sc & 1, wctx, 1 * 10000 + __LINE__)) return false;
+          ++sc;
+          tc_fence_after();
+          // the row's allowed columns in this half of the key tile: [a, b)
+          const int k0 = klo + j * BN + h * 64;
+          const int a = st.lo - k0, b = st.hi - k0;
           uint32_t v[64];
           tmem_ld32p(tS + h * 64, v);
           tmem_ld32p(tS + h * 64 + 32, v + 32);
           tmem_wait_ld();
           reg_fence<64>(v);
-          const float mh = scale_log2 * (full ? row_max<false>(v, a - h * 64, b - h * 64)
-                                              : row_max<true>(v, a - h * 64, b - h * 64));
-          mx = fmaxf(mx, mh);
+          // masked scores become -inf (their exponentials are exactly 0)
+          if (!__all_sync(0xffffffffu, a <= 0 && b >= 64)) {
+#pragma unroll
+            for (int i = 0; i < 64; ++i) v[i] = (i >= a && i < b) ? v[i] : 0xff800000u;
+          }
+          const float mh = scale_log2 * row_max(v);
+          // the other half's maximum of this row (exchange slots alternate by parity)
+          float* slot = xs + (n_x & 1) * 2 * BM;
+          slot[h * BM + r] = mh;
+          __threadfence_block();
+          warp_arrive(&bars->xchg[wq]);
+          if (!warp_wait(&bars->xchg[wq], n_x & 1, wctx, 1 * 10000 + __LINE__)) return false;
+          const float mt = fmaxf(mh, slot[(h ^ 1) * BM + r]);   // -inf: no allowed key in the tile
+          ++n_x;
           // a row's first allowed keys set its reference (its O and l are still zero);
-          // later halves past the headroom take the rescale below
-          if (m_ref == -INFINITY) m_ref = mh;
-          const bool over = mh > m_ref + kHeadroomLog2;
+          // a later maximum past the headroom rescales O and l to a new reference
+          if (st.m_ref == -INFINITY) st.m_ref = mt;
+          const bool over = mt > st.m_ref + kHeadroomLog2;
           if (__any_sync(0xffffffffu, over)) {
-            // new reference for the rows past the headroom: rescale O (after PV(j-1)),
-            // the P of half 0 already in TMEM, and l
-            const float f = over ? fast_exp2(m_ref - mh) : 1.f;
+            const float f = over ? fast_exp2(st.m_ref - mt) : 1.f;
             if (j > 0) {
-              if (!warp_wait(&bars->o_ready[x], (o_cnt + j - 1) & 1, wctx, 1 * 10000 + __LINE__)) {
-                ok = false;
-                break;
-              }
+              // this half's O columns, after PV(j-1)
+              if (!warp_wait(&bars->o_ready[x], (oc + j - 1) & 1, wctx, 1 * 10000 + __LINE__)) return false;
               tc_fence_after();
 #pragma unroll 1
-              for (int cch = 0; cch < D / 16; ++cch) {
+              for (int cch = 0; cch < 4; ++cch) {
                 uint32_t o[16];
-                tmem_ld16(tO + cch * 16, o);
+                tmem_ld16(tO + h * 64 + cch * 16, o);
                 tmem_wait_ld();
                 reg_fence<16>(o);
 #pragma unroll
                 for (int i = 0; i < 16; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * f);
-                tmem_st16(tO + cch * 16, o);
+                tmem_st16(tO + h * 64 + cch * 16, o);
               }
-            }
-            if (h > 0) {
               tmem_wait_st();
-#pragma unroll 1
-              for (int cch = 0; cch < 2; ++cch) {
-                uint32_t pk[16];
-                tmem_ld16(tS + cch * 16, pk);
-                tmem_wait_ld();
-                reg_fence<16>(pk);
-#pragma unroll
-                for (int i = 0; i < 16; ++i)
-                  pk[i] = pack_bf16(__uint_as_float(pk[i] << 16) * f, __uint_as_float(pk[i] & 0xffff0000u) * f);
-                tmem_st16(tS + cch * 16, pk);
-              }
             }
-            tmem_wait_st();
-            l *= f;
-            if (over) m_ref = mh;
+            st.l *= f;
+            if (over) st.m_ref = mt;
           }
-          const float m_use = (m_ref == -INFINITY) ? 0.f : m_ref;
-          l += full ? exp_pack_store<false>(v, a - h * 64, b - h * 64, scale_log2, -m_use, tS + h * 32)
-                    : exp_pack_store<true>(v, a - h * 64, b - h * 64, scale_log2, -m_use, tS + h * 32);
+          const float m_use = (st.m_ref == -INFINITY) ? 0.f : st.m_ref;
+          // P of this half over the scores it replaces: columns 0..31 (half 0), 64..95 (half 1)
+          st.l += exp_pack_store(v, scale_log2, -m_use, tS + h * 64);
+          st.m_true = fmaxf(st.m_true, mt);
+          tmem_wait_st();
+          tc_fence_before();
+          warp_arrive(&bars->p_ready[x]);
+          return true;
+      };
+      for (int j = 0; j < n_kt && ok; ++j) {
+#pragma unroll 1
+        for (int x = 0; x < nx && ok; ++x) {
+          RowState st = x == 0 ? rsA : rsB;
+          uint32_t sc = x == 0 ? s_cntA : s_cntB;
+          ok = step(st, sc, x == 0 ? o_cntA : o_cntB, x, j);
+          if (x == 0) {
+            rsA = st;
+            s_cntA = sc;
+          } else {
+            rsB = st;
+            s_cntB = sc;
+          }
         }
-        if (!ok) break;
-        m_true = fmaxf(m_true, none ? -INFINITY : mx);
-        tmem_wait_st();
-        tc_fence_before();
-        warp_arrive(&bars->p_ready[x]);
       }
       if (!ok) break;
-      o_cnt += n_kt;
-      // the row's statistics for the epilogue warps: 1 / l, and the record's m_c (the
-      // true maximum, natural units) and l_c (the sum relative to it)
-      {
-        float4* st = reinterpret_cast<float4*>(smem + kOffStats) + ((st_cnt & 1) * 2 + x) * BM + r;
-        *st = make_float4(l > 0.f ? 1.f / l : 0.f, (l > 0.f) ? m_true * kLn2 : -INFINITY,
-                          (l > 0.f) ? l * fast_exp2(m_ref - m_true) : 0.f, 0.f);
+      // the rows' statistics for the epilogue warps: half 0 leaves its sum, the true
+      // maximum and the reference, half 1 its sum (fields of one float4 per row)
+#pragma unroll
+      for (int x = 0; x < 2; ++x) {
+        if (x >= nx) break;
+        const RowState& st = x == 0 ? rsA : rsB;
+        uint32_t& stc = x == 0 ? st_cntA : st_cntB;
+        (x == 0 ? o_cntA : o_cntB) += n_kt;
+        float* st4 = reinterpret_cast<float*>(smem + kOffStats) + (((stc & 1) * 2 + x) * BM + r) * 4;
+        if (h == 0) {
+          st4[0] = st.l;
+          st4[1] = st.m_true;
+          st4[2] = st.m_ref;
+        } else {
+          st4[3] = st.l;
+        }
         __threadfence_block();
-        warp_arrive(&bars->stats_ready[x][st_cnt & 1]);
-        ++st_cnt;
+        warp_arrive(&bars->stats_ready[x][stc & 1]);
+        ++stc;
       }
     }
     if (!ok) *abort_flag = 1;
@@ -534,8 +562,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           break;
         }
         tc_fence_after();
-        const float4 st = reinterpret_cast<const float4*>(smem + kOffStats)[((pc[x] & 1) * 2 + x) * BM + r];
+        const float4 sx = reinterpret_cast<const float4*>(smem + kOffStats)[((pc[x] & 1) * 2 + x) * BM + r];
         ++pc[x];
+        // 1 / l, and the record: m_c = the true maximum (natural units), l_c = the sum
+        // relative to it (the halves' sums are relative to the common reference)
+        const float l = sx.x + sx.w;
+        const float4 st = make_float4(l > 0.f ? 1.f / l : 0.f, (l > 0.f) ? sx.y * kLn2 : -INFINITY,
+                                      (l > 0.f) ? l * fast_exp2(sx.z - sx.y) : 0.f, 0.f);
 #pragma unroll 1
         for (int cch = 0; cch < D / 32; ++cch) {
           uint32_t v[32];

@@ -96,16 +96,22 @@ class Core:
 
 # ---------------------------------------------------------------------------
 # forward kernel: query tiles two at a time (A, B), K and V rings of two stages each (a
-# pair's first K/V tiles requested before its Q buffer frees); the records leave through
-# separate epilogue warps (the tile's last PV and the softmax's row statistics, double-
-# buffered by pair parity, hand each tile over; the epilogue releases O after reading it)
+# pair's first K/V tiles requested before its Q buffer frees); two softmax warpgroups,
+# one per 64-column half of every score tile, take tile A then tile B at each key tile
+# and exchange their halves' row maxima through shared memory (slots alternating by
+# exchange parity); the records leave through separate epilogue warps (the tile's last
+# PV and the softmax's row statistics, double-buffered by pair parity, hand each tile
+# over; the epilogue releases O after reading it)
 # ---------------------------------------------------------------------------
 class Forward(Core):
     def __init__(self, pairs, seed, drop=None):
         names = ["q_full", "q_empty", "k_full0", "k_full1", "v_full0", "v_full1", "k_empty0", "k_empty1",
                  "v_empty0", "v_empty1", "s_ready0", "s_ready1", "p_ready0", "p_ready1", "o_ready0", "o_ready1",
-                 "o_free0", "o_free1", "o_full0", "o_full1", "stats0_0", "stats0_1", "stats1_0", "stats1_1"]
+                 "o_free0", "o_free1", "o_full0", "o_full1", "stats0_0", "stats0_1", "stats1_0", "stats1_1",
+                 "xchg"]
         super().__init__(seed, names)
+        for n in ("p_ready0", "p_ready1", "stats0_0", "stats0_1", "stats1_0", "stats1_1", "xchg"):
+            self.B[n] = Bar(2)        # one arrival per column half
         self.pairs = pairs            # [(nx, n_kt)]
         self.drop = drop
         self.Q = None
@@ -113,7 +119,9 @@ class Forward(Core):
         self.V = [None, None]
         self.S = [None, None]
         self.O = [None, None]
-        self.ST = {}                  # (tile, buffer) -> pair whose statistics it holds
+        self.ST = {}                  # (tile, buffer) -> (pair, halves written) or ("read",)
+        self.PH = [set(), set()]      # halves whose P of the current key tile is in S_x
+        self.XS = {}                  # exchange slot (parity, half) -> exchange index written
         self.rescale = {}
 
     def producer(self):
@@ -169,7 +177,9 @@ class Forward(Core):
                         yield from self.wait(f"v_full{c % 2}", c // 2)
 
                     def pv(x=x, c=c, j=j, i=i):
-                        self.check(self.S[x] == ("P", i, c), f"PV({x},{c}) reads {self.S[x]}")
+                        self.check(self.S[x] == ("S", i, c) and self.PH[x] == {0, 1},
+                                   f"PV({x},{c}) reads {self.S[x]} with P halves {self.PH[x]}")
+                        self.PH[x] = set()
                         self.check(self.V[c % 2] == c, f"PV({x},{c}) reads V {self.V[c % 2]}")
                         self.S[x] = ("read", i, c)
                         if j == 0:
@@ -197,32 +207,41 @@ class Forward(Core):
             kv += nkt
             yield
 
-    def softmax(self, x):
+    def softmax(self, h):
         kv = 0
-        s_cnt, o_cnt, st_cnt = 0, 0, 0
+        s_cnt, o_cnt, st_cnt, n = [0, 0], [0, 0], [0, 0], 0
         for i, (nx, nkt) in enumerate(self.pairs):
-            if x >= nx:
-                kv += nkt
-                continue
             for j in range(nkt):
                 c = kv + j
-                yield from self.wait(f"s_ready{x}", s_cnt)
-                s_cnt += 1
-                self.check(self.S[x] == ("S", i, c), f"softmax({x},{c}) finds {self.S[x]}")
-                if j > 0 and self.rng.random() < 0.2:   # the rare rescale of O after PV(j - 1)
-                    yield from self.wait(f"o_ready{x}", o_cnt + j - 1)
-                    self.check(self.O[x] == ("acc", i, j), f"rescale finds O {self.O[x]}")
-                yield
-                self.S[x] = ("P", i, c)
-                self.B[f"p_ready{x}"].arrive()
-            o_cnt += nkt
-            yield                         # the statistics are written after the last P is handed over
-            b = st_cnt % 2
-            self.check(self.ST.get((x, b), ("read",))[0] == "read", f"stats({x},{b}) of pair {i} overwrite unread "
-                       f"{self.ST.get((x, b))}")
-            self.ST[(x, b)] = ("written", i)
-            self.B[f"stats{x}_{b}"].arrive()
-            st_cnt += 1
+                for x in range(nx):
+                    yield from self.wait(f"s_ready{x}", s_cnt[x])
+                    s_cnt[x] += 1
+                    self.check(self.S[x] == ("S", i, c) and h not in self.PH[x],
+                               f"softmax half {h} ({x},{c}) finds {self.S[x]}")
+                    self.XS[(n % 2, h)] = n
+                    self.B["xchg"].arrive()
+                    if self.drop != "xchg":
+                        yield from self.wait("xchg", n)
+                    self.check(self.XS.get((n % 2, 1 - h)) == n,
+                               f"half {h} reads exchange {self.XS.get((n % 2, 1 - h))} for {n}")
+                    n += 1
+                    if j > 0 and self.rng.random() < 0.2:   # the rare rescale of O after PV(j - 1)
+                        yield from self.wait(f"o_ready{x}", o_cnt[x] + j - 1)
+                        self.check(self.O[x] == ("acc", i, j), f"rescale finds O {self.O[x]}")
+                    yield
+                    self.PH[x].add(h)
+                    self.B[f"p_ready{x}"].arrive()
+            for x in range(nx):
+                o_cnt[x] += nkt
+                b = st_cnt[x] % 2
+                old = self.ST.get((x, b), ("read",))
+                fresh = old == ("read",)
+                self.check(fresh or (old[0] == i and h not in old[1]),
+                           f"stats({x},{b}) of pair {i} overwrite unread {old}")
+                self.ST[(x, b)] = (i, (set() if fresh else old[1]) | {h})
+                self.B[f"stats{x}_{b}"].arrive()
+                st_cnt[x] += 1
+                yield                     # the next half's statistics follow later
             kv += nkt
 
     def epilogue(self):
@@ -233,9 +252,9 @@ class Forward(Core):
                 b = pc[x] % 2
                 if self.drop != "stats":
                     yield from self.wait(f"stats{x}_{b}", pc[x] // 2)
-                self.check(self.ST.get((x, b)) == ("written", i), f"epilogue({x}) of pair {i} finds stats "
+                self.check(self.ST.get((x, b)) == (i, {0, 1}), f"epilogue({x}) of pair {i} finds stats "
                            f"{self.ST.get((x, b))}")
-                self.ST[(x, b)] = ("read", i)
+                self.ST[(x, b)] = ("read",)
                 self.check(self.O[x] == ("acc", i, nkt), f"epilogue({x}) of pair {i} finds {self.O[x]}")
                 pc[x] += 1
                 yield
@@ -244,7 +263,7 @@ class Forward(Core):
                 yield
 
     def go(self):
-        self.run({"prod": self.producer(), "mma": self.mma_thread(), "smA": self.softmax(0), "smB": self.softmax(1),
+        self.run({"prod": self.producer(), "mma": self.mma_thread(), "sm0": self.softmax(0), "sm1": self.softmax(1),
                   "epi": self.epilogue()})
 
 
@@ -547,7 +566,7 @@ def test_protocol_holds_on_random_schedules(kernel):
 
 
 @pytest.mark.parametrize("kernel,drop", [("forward", "kv_empty"), ("forward", "q_empty"), ("forward", "o_free"),
-                                         ("forward", "stats"),
+                                         ("forward", "stats"), ("forward", "xchg"),
                                          ("dkdv", "qd_empty"),
                                          ("dkdv", "kv_empty"), ("dkdv", "lookahead_before_dv"), ("dq", "kv_empty"),
                                          ("dq", "qd_empty")])
