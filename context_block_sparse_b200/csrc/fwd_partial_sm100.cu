@@ -506,29 +506,28 @@ __global__ void __launch_bounds__(kThreads, 1)
             rsB = st;
             s_cntB = sc;
           }
+          if (ok && j == n_kt - 1) {
+            // the tile's last key tile: its rows' statistics go to the epilogue warps
+            // at once (half 0 leaves its sum, the true maximum and the reference, half 1
+            // its sum: fields of one float4 per row)
+            uint32_t stc = x == 0 ? st_cntA : st_cntB;
+            float* st4 = reinterpret_cast<float*>(smem + kOffStats) + (((stc & 1) * 2 + x) * BM + r) * 4;
+            if (h == 0) {
+              st4[0] = st.l;
+              st4[1] = st.m_true;
+              st4[2] = st.m_ref;
+            } else {
+              st4[3] = st.l;
+            }
+            __threadfence_block();
+            warp_arrive(&bars->stats_ready[x][stc & 1]);
+            if (x == 0) ++st_cntA; else ++st_cntB;
+          }
         }
       }
       if (!ok) break;
-      // the rows' statistics for the epilogue warps: half 0 leaves its sum, the true
-      // maximum and the reference, half 1 its sum (fields of one float4 per row)
-#pragma unroll
-      for (int x = 0; x < 2; ++x) {
-        if (x >= nx) break;
-        const RowState& st = x == 0 ? rsA : rsB;
-        uint32_t& stc = x == 0 ? st_cntA : st_cntB;
-        (x == 0 ? o_cntA : o_cntB) += n_kt;
-        float* st4 = reinterpret_cast<float*>(smem + kOffStats) + (((stc & 1) * 2 + x) * BM + r) * 4;
-        if (h == 0) {
-          st4[0] = st.l;
-          st4[1] = st.m_true;
-          st4[2] = st.m_ref;
-        } else {
-          st4[3] = st.l;
-        }
-        __threadfence_block();
-        warp_arrive(&bars->stats_ready[x][stc & 1]);
-        ++stc;
-      }
+      o_cntA += n_kt;
+      if (nx == 2) o_cntB += n_kt;
     }
     if (!ok) *abort_flag = 1;
   } else if (warp >= 12) {
@@ -557,11 +556,19 @@ __global__ void __launch_bounds__(kThreads, 1)
         const bool valid = slot < tile.y - tile.x;
         const int rec = valid ? ((tile.x + slot) * p.bs + tt) * p.Hq + g * p.G + hh : 0;
         if (!warp_wait(&bars->o_full[x], pc[x] & 1, wctx, 1 * 10000 + __LINE__)) { ok = false; break; }
+        tc_fence_after();
+        // O in two rounds of two 32-column chunks; the output columns are released after
+        // the second round's TMEM reads, before its stores
+        uint32_t va[32], vb[32];
+        tmem_ld32(tO, va);
+        tmem_ld32(tO + 32, vb);
+        tmem_wait_ld();
+        reg_fence<32>(va);
+        reg_fence<32>(vb);
         if (!warp_wait(&bars->stats_ready[x][pc[x] & 1], (pc[x] >> 1) & 1, wctx, 1 * 10000 + __LINE__)) {
           ok = false;
           break;
         }
-        tc_fence_after();
         const float4 sx = reinterpret_cast<const float4*>(smem + kOffStats)[((pc[x] & 1) * 2 + x) * BM + r];
         ++pc[x];
         // 1 / l, and the record: m_c = the true maximum (natural units), l_c = the sum
@@ -569,25 +576,30 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float l = sx.x + sx.w;
         const float4 st = make_float4(l > 0.f ? 1.f / l : 0.f, (l > 0.f) ? sx.y * kLn2 : -INFINITY,
                                       (l > 0.f) ? l * fast_exp2(sx.z - sx.y) : 0.f, 0.f);
-#pragma unroll 1
-        for (int cch = 0; cch < D / 32; ++cch) {
-          uint32_t v[32];
-          tmem_ld32(tO + cch * 32, v);
-          tmem_wait_ld();
-          reg_fence<32>(v);
-          if (cch == D / 32 - 1) {
-            // every TMEM read of O_x done: the MMA may start the next pair's products into it
-            tc_fence_before();
-            warp_arrive(&bars->o_free[x]);
-          }
+        // stores of two 32-column chunks held in va, vb
+        auto store2 = [&](int col) {
           if (p.partial_bf16) {
-            if (valid) lane_store32_bf16(static_cast<uint16_t*>(part_o) + size_t(rec) * D + cch * 32, v, st.x);
+            if (valid) {
+              lane_store32_bf16(static_cast<uint16_t*>(part_o) + size_t(rec) * D + col, va, st.x);
+              lane_store32_bf16(static_cast<uint16_t*>(part_o) + size_t(rec) * D + col + 32, vb, st.x);
+            }
             __syncwarp();   // valid differs across the warp's rows: converge before the next tcgen05.ld
           } else {
-            warp_store_rows<32>(scratch, reinterpret_cast<const float*>(v), st.x,
-                                valid ? static_cast<float*>(part_o) + size_t(rec) * D + cch * 32 : nullptr);
+            float* dst = valid ? static_cast<float*>(part_o) + size_t(rec) * D + col : nullptr;
+            warp_store_rows<32>(scratch, reinterpret_cast<const float*>(va), st.x, dst);
+            warp_store_rows<32>(scratch, reinterpret_cast<const float*>(vb), st.x, valid ? dst + 32 : nullptr);
           }
-        }
+        };
+        store2(0);
+        tmem_ld32(tO + 64, va);
+        tmem_ld32(tO + 96, vb);
+        tmem_wait_ld();
+        reg_fence<32>(va);
+        reg_fence<32>(vb);
+        // every TMEM read of O_x done: the MMA may start the next pair's products into it
+        tc_fence_before();
+        warp_arrive(&bars->o_free[x]);
+        store2(64);
         if (valid) {
           part_m[rec] = st.y;
           part_l[rec] = st.z;

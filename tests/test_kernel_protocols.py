@@ -231,17 +231,18 @@ class Forward(Core):
                     yield
                     self.PH[x].add(h)
                     self.B[f"p_ready{x}"].arrive()
+                    if j == nkt - 1:
+                        yield             # the statistics follow the tile's last P
+                        b = st_cnt[x] % 2
+                        old = self.ST.get((x, b), ("read",))
+                        fresh = old == ("read",)
+                        self.check(fresh or (old[0] == i and h not in old[1]),
+                                   f"stats({x},{b}) of pair {i} overwrite unread {old}")
+                        self.ST[(x, b)] = (i, (set() if fresh else old[1]) | {h})
+                        self.B[f"stats{x}_{b}"].arrive()
+                        st_cnt[x] += 1
             for x in range(nx):
                 o_cnt[x] += nkt
-                b = st_cnt[x] % 2
-                old = self.ST.get((x, b), ("read",))
-                fresh = old == ("read",)
-                self.check(fresh or (old[0] == i and h not in old[1]),
-                           f"stats({x},{b}) of pair {i} overwrite unread {old}")
-                self.ST[(x, b)] = (i, (set() if fresh else old[1]) | {h})
-                self.B[f"stats{x}_{b}"].arrive()
-                st_cnt[x] += 1
-                yield                     # the next half's statistics follow later
             kv += nkt
 
     def epilogue(self):
