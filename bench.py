@@ -49,12 +49,12 @@ METRIC = "masked-pair attn TFLOP/s fwd/bwd, % of BF16 tensor peak; LPT imbalance
 # kernel, with the sha256 of the sources the kernel was built from when it was
 # taken; a changed source voids the figure.
 NCU_TRAFFIC = {
-    "fwd_partial": {"bytes": 2075161140, "src": "9a3f68c6308f2a0e"},
-    "merge": {"bytes": 1558043085, "src": "b87601659b20c86d"},
-    "bwd_delta": {"bytes": 201970791, "src": "b87601659b20c86d"},
-    "bwd_dkdv": {"bytes": 1653801319, "src": "1ddaa484886212e9"},
-    "bwd_dq": {"bytes": 2306389299, "src": "1ddaa484886212e9"},
-    "bwd_reduce": {"bytes": 1554170317, "src": "b87601659b20c86d"},
+    # dram__bytes_read.sum + dram__bytes_write.sum of one launch at the 64k / 8k fwd+bwd
+    # workload (ncu --clock-control none, one pass), with a hash of the kernel's sources at
+    # the capture: a kernel whose sources changed since reports traffic null
+    "fwd_partial": {"bytes": 926102528 + 1152824576, "src": "5960367354c328d5"},
+    "bwd_dkdv": {"bytes": 1137947904 + 486652928, "src": "4aac18d0056134d0"},
+    "bwd_dq": {"bytes": 1161585920 + 1140958464, "src": "4aac18d0056134d0"},
 }
 _KERNEL_SOURCES = {
     "fwd_partial": ("fwd_partial_sm100.cu", "sm100.cuh", "splitkv_internal.h"),
