@@ -1,5 +1,5 @@
 // Backward of the chunk partial attention on the 5th-generation tensor cores
-// (tcgen05 / TMEM / TMA), head_dim 128.
+// (tcgen05 / TMEM / TMA), head_dim 64 or 128.
 //
 // News page "Split-KV speeds diffusion drafter training by keeping long-context
 // data local", section "Exchange the smaller side": keys and values stay local
@@ -47,19 +47,26 @@ namespace {
 
 using namespace sm100;
 
-constexpr int D = 128;
 constexpr int BT = 128;                // keys per key tile = rows per query tile
 constexpr int kThreads = 384;
 constexpr uint32_t kHalf = 128 * 128;  // one 64-column half of a 128-row bf16 tile
-constexpr uint32_t kTile = 2 * kHalf;  // 32 KB
 constexpr uint32_t kIdescKM = idesc_bf16_f32(128, 128, 0);  // B K-major
-constexpr uint32_t kIdescMN = idesc_bf16_f32(128, D, 1);    // B MN-major
-// 6 tiles | row metadata (8 KB) | epilogue scratch (2 KB per element-wise warp) | barriers
-constexpr uint32_t kOffMeta = 6 * kTile;
-constexpr uint32_t kOffScratch = kOffMeta + 8192;
-constexpr uint32_t kOffBars = kOffScratch + 8 * 2048;
-constexpr uint32_t kSmemBytes = kOffBars + 256 + 1024;
-static_assert(kSmemBytes <= 232448, "shared memory per block");
+
+// Sizes that follow the head dimension D (64 or 128): a 128-row bf16 tile of D
+// columns is D / 64 halves of 16 KB; the products into dK, dV, dQ have N = D.
+// Shared memory: 6 tiles | row metadata (8 KB) | epilogue scratch (2 KB per
+// element-wise warp) | barriers.
+template <int D>
+struct Dims {
+  static_assert(D == 64 || D == 128, "head dimension");
+  static constexpr uint32_t kTile = uint32_t(D / 64) * kHalf;
+  static constexpr uint32_t kIdescMN = idesc_bf16_f32(128, D, 1);   // B MN-major, N = D
+  static constexpr uint32_t kOffMeta = 6 * kTile;
+  static constexpr uint32_t kOffScratch = kOffMeta + 8192;
+  static constexpr uint32_t kOffBars = kOffScratch + 8 * 2048;
+  static constexpr uint32_t kSmemBytes = kOffBars + 256 + 1024;
+  static_assert(kSmemBytes <= 232448, "shared memory per block");
+};
 
 
 // K-major SW128 descriptor of the k-th 16-column step of a 128-row tile.
@@ -103,9 +110,10 @@ __device__ __forceinline__ RowMeta row_meta(const DevPlan& p, const int4& tile, 
 }
 
 // TMA of one query tile's rows (Q or dO layout) into a 128-row SW128 tile
-// (kTile bytes).  Slots past the tile's last block are loaded from token
+// (D / 64 halves).  Slots past the tile's last block are loaded from token
 // coordinate Nq, outside the tensor, so that the hardware fills them with
 // zeros: the dK/dV products contract over all 128 rows.
+template <int D>
 __device__ __forceinline__ void load_query_tile(const DevPlan& p, const int4& tile, int g, uint8_t* dst,
                                                 const CUtensorMap* map, uint64_t* bar) {
   const int rps = p.G * p.bs;
@@ -113,7 +121,8 @@ __device__ __forceinline__ void load_query_tile(const DevPlan& p, const int4& ti
   const int n = tile.y - tile.x;
   for (int s = 0; s < BT / rps; ++s) {
     const int z = s < n ? p.entries[tile.x + s].x * p.bs : p.Nq;
-    for (int dh = 0; dh < 2; ++dh) tma_load_3d(dst + dh * kHalf + s * slot_bytes, map, bar, dh * 64, g * p.G, z);
+    for (int dh = 0; dh < D / 64; ++dh)
+      tma_load_3d(dst + dh * kHalf + s * slot_bytes, map, bar, dh * 64, g * p.G, z);
   }
 }
 
@@ -144,6 +153,8 @@ __device__ __forceinline__ void ds_tile(uint32_t tS, uint32_t tdP, int hf, int a
     tmem_ld32(tS + q * 32, sv);
     tmem_ld32(tdP + q * 32, dpv);
     tmem_wait_ld();
+    reg_fence<32>(sv);
+    reg_fence<32>(dpv);
     uint32_t pk[16];
 #pragma unroll
     for (int i = 0; i < 16; ++i) {
@@ -267,6 +278,7 @@ __device__ __forceinline__ void bwd_item_seq(ItemSeq& s, const DevPlan& p, int w
     s.init_static(p.bwd_worker_ptr[w], p.bwd_worker_ptr[w + 1]);
 }
 
+template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
     bwd_dkdv_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_do,
                           const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
@@ -275,14 +287,17 @@ __global__ void __launch_bounds__(kThreads, 1)
                           float* __restrict__ dk, float* __restrict__ dv) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  using Dm = Dims<D>;
+  constexpr uint32_t kTile = Dm::kTile;
+  constexpr uint32_t kIdescMN = Dm::kIdescMN;
   uint8_t* sK = smem;
   uint8_t* sV = smem + kTile;
   uint8_t* sQ = smem + 2 * kTile;   // [2 stages]
   uint8_t* sdO = smem + 4 * kTile;  // [2 stages]
-  float* meta_l2 = reinterpret_cast<float*>(smem + 6 * kTile);               // [2][128] lse2 per row
-  float* meta_dl = reinterpret_cast<float*>(smem + 6 * kTile + 1024);        // [2][128] delta per row
-  int2* meta_slot = reinterpret_cast<int2*>(smem + 6 * kTile + 2048);         // [2][16] (lo, hi) per slot
-  DkdvBars* B = reinterpret_cast<DkdvBars*>(smem + kOffBars);
+  float* meta_l2 = reinterpret_cast<float*>(smem + Dm::kOffMeta);               // [2][128] lse2 per row
+  float* meta_dl = reinterpret_cast<float*>(smem + Dm::kOffMeta + 1024);        // [2][128] delta per row
+  int2* meta_slot = reinterpret_cast<int2*>(smem + Dm::kOffMeta + 2048);         // [2][16] (lo, hi) per slot
+  DkdvBars* B = reinterpret_cast<DkdvBars*>(smem + Dm::kOffBars);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int w = blockIdx.x;
   volatile int* abort_flag = &B->abort_flag;
@@ -317,7 +332,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int k0 = c0; ok && k0 < c1; k0 += BT) {
           if (!mbar_wait(&B->kv_empty, (kt_count & 1) ^ 1, wctx, 2 * 10000 + __LINE__)) { ok = false; break; }
           mbar_expect_tx(&B->kv_full, 2 * kTile);
-          for (int dh = 0; dh < 2; ++dh) {
+          for (int dh = 0; dh < D / 64; ++dh) {
             tma_load_3d(sK + dh * kHalf, &tm_k, &B->kv_full, dh * 64, g, k0);
             tma_load_3d(sV + dh * kHalf, &tm_v, &B->kv_full, dh * 64, g, k0);
           }
@@ -328,8 +343,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int s = qd_count & 1;
             if (!mbar_wait(&B->qd_empty[s], ((qd_count >> 1) & 1) ^ 1, wctx, 2 * 10000 + __LINE__)) { ok = false; break; }
             mbar_expect_tx(&B->qd_full[s], 2 * kTile);
-            load_query_tile(p, tile, g, sQ + s * kTile, &tm_q, &B->qd_full[s]);
-            load_query_tile(p, tile, g, sdO + s * kTile, &tm_do, &B->qd_full[s]);
+            load_query_tile<D>(p, tile, g, sQ + s * kTile, &tm_q, &B->qd_full[s]);
+            load_query_tile<D>(p, tile, g, sdO + s * kTile, &tm_do, &B->qd_full[s]);
             ++qd_count;
           }
         }
@@ -540,7 +555,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (!warp_wait(&B->dkv_ready, dkv_cnt & 1, wctx, 2 * 10000 + __LINE__)) { ok = false; break; }
           ++dkv_cnt;
           tc_fence_after();
-          float* scratch = reinterpret_cast<float*>(smem + kOffScratch) + (warp - 4) * 512;
+          float* scratch = reinterpret_cast<float*>(smem + Dm::kOffScratch) + (warp - 4) * 512;
           if (__all_sync(0xffffffffu, own)) {
             // the warp's 32 keys all belong to this chunk (and lie below N): bulk
             // tensor stores of 32 keys x 16 columns
@@ -634,6 +649,7 @@ struct TileIter {
   }
 };
 
+template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
     bwd_dq_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_do,
                         const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
@@ -641,12 +657,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                         const float* __restrict__ delta, float scale, int bulk, void* __restrict__ dq_part) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  using Dm = Dims<D>;
+  constexpr uint32_t kTile = Dm::kTile;
+  constexpr uint32_t kIdescMN = Dm::kIdescMN;
   uint8_t* sQ = smem;
   uint8_t* sdO = smem + kTile;
   uint8_t* sK = smem + 2 * kTile;   // [2 stages]
   uint8_t* sV = smem + 4 * kTile;   // [2 stages]
-  DqRow* meta = reinterpret_cast<DqRow*>(smem + 6 * kTile);   // [2][128]
-  DqBars* B = reinterpret_cast<DqBars*>(smem + kOffBars);
+  DqRow* meta = reinterpret_cast<DqRow*>(smem + Dm::kOffMeta);   // [2][128]
+  DqBars* B = reinterpret_cast<DqBars*>(smem + Dm::kOffBars);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int w = blockIdx.x;
   volatile int* abort_flag = &B->abort_flag;
@@ -680,11 +699,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int s = int(c & 1);
         if (!mbar_wait(&B->v_empty[s], ((c >> 1) & 1) ^ 1, wctx, 2 * 10000 + __LINE__)) return false;
         mbar_expect_tx(&B->v_full[s], kTile);
-        for (int dh = 0; dh < 2; ++dh) tma_load_3d(sV + s * kTile + dh * kHalf, &tm_v, &B->v_full[s], dh * 64, g, k0);
+        for (int dh = 0; dh < D / 64; ++dh)
+          tma_load_3d(sV + s * kTile + dh * kHalf, &tm_v, &B->v_full[s], dh * 64, g, k0);
         ++v_issued;
         if (!mbar_wait(&B->k_empty[s], ((c >> 1) & 1) ^ 1, wctx, 2 * 10000 + __LINE__)) return false;
         mbar_expect_tx(&B->k_full[s], kTile);
-        for (int dh = 0; dh < 2; ++dh) tma_load_3d(sK + s * kTile + dh * kHalf, &tm_k, &B->k_full[s], dh * 64, g, k0);
+        for (int dh = 0; dh < D / 64; ++dh)
+          tma_load_3d(sK + s * kTile + dh * kHalf, &tm_k, &B->k_full[s], dh * 64, g, k0);
         ++k_issued;
         return true;
       };
@@ -696,8 +717,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!load_kv(kv_count, tile.z)) { ok = false; break; }
         if (!mbar_wait(&B->qd_empty, (tile_count & 1) ^ 1, wctx, 2 * 10000 + __LINE__)) { ok = false; break; }
         mbar_expect_tx(&B->qd_full, 2 * kTile);
-        load_query_tile(p, tile, g, sQ, &tm_q, &B->qd_full);
-        load_query_tile(p, tile, g, sdO, &tm_do, &B->qd_full);
+        load_query_tile<D>(p, tile, g, sQ, &tm_q, &B->qd_full);
+        load_query_tile<D>(p, tile, g, sdO, &tm_do, &B->qd_full);
         ++q_issued;
         for (int j = 1; j < n_kt && ok; ++j)
           if (!load_kv(kv_count + j, tile.z + j * BT)) ok = false;
@@ -820,7 +841,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int r = ((warp & 3) << 5) + lane;
     const uint32_t lane_addr = uint32_t((warp & 3) << 5) << 16;
     const uint32_t tdP = tmem + lane_addr + 256;
-    const uint32_t tdQ = tmem + lane_addr + 384 + hf * 64;   // this warpgroup's 64 dQ columns
+    constexpr int kHalfD = D / 2;                            // dQ columns per warpgroup
+    const uint32_t tdQ = tmem + lane_addr + 384 + hf * kHalfD;   // this warpgroup's dQ columns
     const float scale_log2 = scale * kLog2e;
     TileIter ti;
     ti.init(&p, w, &B->ring, kClaimWarp, &wctx);
@@ -860,21 +882,22 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!warp_wait(&B->dq_ready, dq_cnt & 1, wctx, 2 * 10000 + __LINE__)) { ok = false; break; }
       ++dq_cnt;
       tc_fence_after();
-      float* scratch = reinterpret_cast<float*>(smem + kOffScratch) + (warp - 4) * 512;
+      float* scratch = reinterpret_cast<float*>(smem + Dm::kOffScratch) + (warp - 4) * 512;
       if (p.partial_bf16) {
-        // bf16 dq partials: two 32-column chunks of this warpgroup's 64 columns
+        // bf16 dq partials: 32-column chunks of this warpgroup's D / 2 columns
         const int z0 = __shfl_sync(0xffffffffu, m.valid ? m.rec / p.Hq : 0, 0);
         const bool wv = __shfl_sync(0xffffffffu, m.valid ? 1 : 0, 0) != 0;
 #pragma unroll 1
-        for (int cc = 0; cc < 2; ++cc) {
+        for (int cc = 0; cc < kHalfD / 32; ++cc) {
           uint32_t v[32];
           tmem_ld32(tdQ + cc * 32, v);
           tmem_wait_ld();
           reg_fence<32>(v);
           if (bulk)
-            warp_bulk_store32_bf16<0>(scratch, v, scale, &tm_dq, hf * 64 + cc * 32, g * p.G, z0, wv);
+            warp_bulk_store32_bf16<0>(scratch, v, scale, &tm_dq, hf * kHalfD + cc * 32, g * p.G, z0, wv);
           else if (m.valid)
-            lane_store32_bf16(static_cast<uint16_t*>(dq_part) + size_t(m.rec) * D + hf * 64 + cc * 32, v, scale);
+            lane_store32_bf16(static_cast<uint16_t*>(dq_part) + size_t(m.rec) * D + hf * kHalfD + cc * 32, v,
+                              scale);
           __syncwarp();   // m.valid differs across the warp's rows: converge before the next tcgen05.ld
         }
       } else if (bulk) {
@@ -883,17 +906,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int z0 = __shfl_sync(0xffffffffu, m.valid ? m.rec / p.Hq : 0, 0);
         const bool wv = __shfl_sync(0xffffffffu, m.valid ? 1 : 0, 0) != 0;
 #pragma unroll 1
-        for (int cc = 0; cc < 4; ++cc) {
+        for (int cc = 0; cc < kHalfD / 16; ++cc) {
           uint32_t v[16];
           tmem_ld16(tdQ + cc * 16, v);
           tmem_wait_ld();
           reg_fence<16>(v);
-          warp_bulk_store16<0>(scratch, v, scale, &tm_dq, hf * 64 + cc * 16, g * p.G, z0, wv);
+          warp_bulk_store16<0>(scratch, v, scale, &tm_dq, hf * kHalfD + cc * 16, g * p.G, z0, wv);
         }
       } else {
-        float* dst = static_cast<float*>(dq_part) + size_t(m.rec) * D + hf * 64;
+        float* dst = static_cast<float*>(dq_part) + size_t(m.rec) * D + hf * kHalfD;
 #pragma unroll 1
-        for (int cc = 0; cc < 4; ++cc) {
+        for (int cc = 0; cc < kHalfD / 16; ++cc) {
           uint32_t v[16];
           tmem_ld16(tdQ + cc * 16, v);
           tmem_wait_ld();
@@ -920,12 +943,16 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 bool bwd_sm100_supported(const DevPlan& p) {
   const int rows = p.G * p.bs;
-  return p.d == D && rows % 8 == 0 && rows <= BT && tensor_maps_available();
+  return (p.d == 64 || p.d == 128) && rows % 8 == 0 && rows <= BT && tensor_maps_available();
 }
 
-cudaError_t launch_bwd_partial_sm100(const DevPlan& p, const uint16_t* q, const uint16_t* k, const uint16_t* v,
-                                     const uint16_t* dout, const float* lse, const float* delta, float scale,
-                                     float* dk, float* dv, void* dq_part, cudaStream_t s, int which) {
+namespace {
+
+template <int D>
+cudaError_t launch_bwd_sm100(const DevPlan& p, const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                             const uint16_t* dout, const float* lse, const float* delta, float scale, float* dk,
+                             float* dv, void* dq_part, cudaStream_t s, int which) {
+  constexpr uint32_t kSmem = Dims<D>::kSmemBytes;
   CUtensorMap tq, tdo, tk, tv, tdk, tdv, tdq;
   if (!make_bf16_map_3d(&tq, q, D, p.Hq, p.Nq, p.G, p.bs) || !make_bf16_map_3d(&tdo, dout, D, p.Hq, p.Nq, p.G, p.bs) ||
       !make_bf16_map_3d(&tk, k, D, p.Hkv, p.N, 1, BT) || !make_bf16_map_3d(&tv, v, D, p.Hkv, p.N, 1, BT) ||
@@ -941,25 +968,34 @@ cudaError_t launch_bwd_partial_sm100(const DevPlan& p, const uint16_t* q, const 
   } else {
     memset(&tdq, 0, sizeof(tdq));
   }
-  cudaError_t e = cudaFuncSetAttribute(bwd_dkdv_sm100_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       int(kSmemBytes));
+  cudaError_t e = cudaFuncSetAttribute(bwd_dkdv_sm100_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       int(kSmem));
   if (e != cudaSuccess) return e;
-  e = cudaFuncSetAttribute(bwd_dq_sm100_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(kSmemBytes));
+  e = cudaFuncSetAttribute(bwd_dq_sm100_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(kSmem));
   if (e != cudaSuccess) return e;
   // run-time claims start from item 0 at every launch (each kernel its own cursor)
   if (which != 2) {
     if (p.dynamic && (e = cudaMemsetAsync(p.claim + 1, 0, sizeof(int), s)) != cudaSuccess) return e;
-    bwd_dkdv_sm100_kernel<<<p.Wb, kThreads, kSmemBytes, s>>>(tq, tdo, tk, tv, tdk, tdv, p, lse, delta, scale, dk, dv);
+    bwd_dkdv_sm100_kernel<D><<<p.Wb, kThreads, kSmem, s>>>(tq, tdo, tk, tv, tdk, tdv, p, lse, delta, scale, dk, dv);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
   if (which != 1) {
     if (p.dynamic && (e = cudaMemsetAsync(p.claim + 2, 0, sizeof(int), s)) != cudaSuccess) return e;
-    bwd_dq_sm100_kernel<<<p.W, kThreads, kSmemBytes, s>>>(tq, tdo, tk, tv, tdq, p, lse, delta, scale,
-                                                          bulk_dq ? 1 : 0, dq_part);
+    bwd_dq_sm100_kernel<D><<<p.W, kThreads, kSmem, s>>>(tq, tdo, tk, tv, tdq, p, lse, delta, scale,
+                                                        bulk_dq ? 1 : 0, dq_part);
     e = cudaGetLastError();
   }
   return e;
+}
+
+}  // namespace
+
+cudaError_t launch_bwd_partial_sm100(const DevPlan& p, const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                                     const uint16_t* dout, const float* lse, const float* delta, float scale,
+                                     float* dk, float* dv, void* dq_part, cudaStream_t s, int which) {
+  if (p.d == 64) return launch_bwd_sm100<64>(p, q, k, v, dout, lse, delta, scale, dk, dv, dq_part, s, which);
+  return launch_bwd_sm100<128>(p, q, k, v, dout, lse, delta, scale, dk, dv, dq_part, s, which);
 }
 
 }  // namespace splitkv

@@ -1,5 +1,5 @@
 // Partial attention of every (chunk, block) entry on the 5th-generation tensor
-// cores (tcgen05 / TMEM / TMA), head_dim 128.
+// cores (tcgen05 / TMEM / TMA), head_dim 64 or 128.
 //
 // News page "Split-KV speeds diffusion drafter training by keeping long-context
 // data local", section "Exchange the smaller side": each key/value shard (here
@@ -50,30 +50,35 @@ namespace {
 
 using namespace sm100;
 
-constexpr int D = 128;
 constexpr int BM = 128;               // query rows per tile
 constexpr int BN = 128;               // keys per key tile
 constexpr int kStages = 2;            // K/V ring depth
 constexpr int kThreads = 512;
 constexpr uint32_t kHalf = 128 * 128; // bytes of one 64-column half of a 128-row tile
-constexpr uint32_t kTile = 2 * kHalf; // 32 KB: a 128 x 128 bf16 tile
 constexpr uint32_t kIdescQK = idesc_bf16_f32(128, 128, 0);
-constexpr uint32_t kIdescPV = idesc_bf16_f32(128, D, 1);
 // A row's reference maximum stays while P = exp2(s - m_ref) <= 2^kHeadroomLog2;
 // P (bf16), l and O (fp32) hold such values exactly as well as near 1, and
 // O = sum P v stays far inside the fp32 range.
 constexpr float kHeadroomLog2 = 32.0f;
 
-// shared-memory map (offsets from a 1024-aligned base)
-constexpr uint32_t kOffQ = 0;                              // Q_A, Q_B
-constexpr uint32_t kOffK = kOffQ + 2 * kTile;              // K stages
-constexpr uint32_t kOffV = kOffK + kStages * kTile;        // V stages
-constexpr uint32_t kOffScratch = kOffV + kStages * kTile; // record staging, 4 KB per epilogue warp
-constexpr uint32_t kOffStats = kOffScratch + 4 * 4096;     // row statistics [2 pair parities][2 tiles][128] float4
-constexpr uint32_t kOffXchg = kOffStats + 2 * 2 * BM * 16;  // half maxima [2 exchange parities][2 halves][128] float
-constexpr uint32_t kOffBar = kOffXchg + 2 * 2 * BM * 4;     // mbarriers
-constexpr uint32_t kSmemBytes = kOffBar + 512 + 1024;      // + alignment slack
-static_assert(kSmemBytes <= 232448, "shared memory per block");
+// Sizes that follow the head dimension D (64 or 128): a 128-row bf16 tile of D
+// columns is D / 64 halves of 16 KB, PV has N = D, O takes D TMEM columns.
+// Shared-memory map (offsets from a 1024-aligned base).
+template <int D>
+struct Dims {
+  static_assert(D == 64 || D == 128, "head dimension");
+  static constexpr uint32_t kTile = uint32_t(D / 64) * kHalf;    // a 128 x D bf16 tile
+  static constexpr uint32_t kIdescPV = idesc_bf16_f32(128, D, 1);
+  static constexpr uint32_t kOffQ = 0;                              // Q_A, Q_B
+  static constexpr uint32_t kOffK = kOffQ + 2 * kTile;              // K stages
+  static constexpr uint32_t kOffV = kOffK + kStages * kTile;        // V stages
+  static constexpr uint32_t kOffScratch = kOffV + kStages * kTile;  // record staging, 4 KB per epilogue warp
+  static constexpr uint32_t kOffStats = kOffScratch + 4 * 4096;     // row statistics [2 pair parities][2 tiles][128] float4
+  static constexpr uint32_t kOffXchg = kOffStats + 2 * 2 * BM * 16; // half maxima [2 exchange parities][2 halves][128]
+  static constexpr uint32_t kOffBar = kOffXchg + 2 * 2 * BM * 4;    // mbarriers
+  static constexpr uint32_t kSmemBytes = kOffBar + 512 + 1024;      // + alignment slack
+  static_assert(kSmemBytes <= 232448, "shared memory per block");
+};
 
 struct Bars {
   uint64_t q_full, q_empty;
@@ -184,6 +189,7 @@ __device__ __forceinline__ float exp_pack_store(const uint32_t (&v)[64], float c
   return s0 + s1;
 }
 
+template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
     fwd_partial_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                              const __grid_constant__ CUtensorMap tm_v, DevPlan p, float scale_log2,
@@ -191,7 +197,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                              float* __restrict__ part_m, float* __restrict__ part_l) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  Bars* bars = reinterpret_cast<Bars*>(smem + kOffBar);
+  using Dm = Dims<D>;
+  constexpr uint32_t kTile = Dm::kTile;
+  constexpr uint32_t kIdescPV = Dm::kIdescPV;
+  constexpr uint32_t kOffQ = Dm::kOffQ, kOffK = Dm::kOffK, kOffV = Dm::kOffV;
+  Bars* bars = reinterpret_cast<Bars*>(smem + Dm::kOffBar);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int w = blockIdx.x;
   volatile int* abort_flag = &bars->abort_flag;
@@ -253,12 +263,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int k0 = klo + j * BN;
         if (!mbar_wait(&bars->k_empty[s], ph, wctx, 1 * 10000 + __LINE__)) return false;
         mbar_expect_tx(&bars->k_full[s], kTile);
-        for (int dh = 0; dh < 2; ++dh)
+        for (int dh = 0; dh < D / 64; ++dh)
           tma_load_3d(smem + kOffK + s * kTile + dh * kHalf, &tm_k, &bars->k_full[s], dh * 64, g, k0);
         ++k_issued;
         if (!mbar_wait(&bars->v_empty[s], ph, wctx, 1 * 10000 + __LINE__)) return false;
         mbar_expect_tx(&bars->v_full[s], kTile);
-        for (int dh = 0; dh < 2; ++dh)
+        for (int dh = 0; dh < D / 64; ++dh)
           tma_load_3d(smem + kOffV + s * kTile + dh * kHalf, &tm_v, &bars->v_full[s], dh * 64, g, k0);
         ++v_issued;
         ++kv_count;
@@ -287,7 +297,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           uint8_t* qbuf = smem + kOffQ + x * kTile;
           for (int s = 0; s < BM / rows_per_slot; ++s) {
             const int z = s < n ? p.entries[e0 + s].x * p.bs : p.Nq;
-            for (int dh = 0; dh < 2; ++dh)
+            for (int dh = 0; dh < D / 64; ++dh)
               tma_load_3d(qbuf + dh * kHalf + s * slot_bytes, &tm_q, &bars->q_full, dh * 64, g * p.G, z);
           }
         }
@@ -404,7 +414,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int wq = warp & 3;
     const int r = (wq << 5) + lane;           // row of the tile = TMEM lane
     const uint32_t lane_addr = uint32_t(wq << 5) << 16;
-    float* xs = reinterpret_cast<float*>(smem + kOffXchg);
+    float* xs = reinterpret_cast<float*>(smem + Dm::kOffXchg);
     PairIter pi;
     pi.init(&p, w, &bars->ring, kClaimWarp, &wctx);
     int tA, tB, g, klo, khi;
@@ -470,14 +480,14 @@ __global__ void __launch_bounds__(kThreads, 1)
               if (!warp_wait(&bars->o_ready[x], (oc + j - 1) & 1, wctx, 1 * 10000 + __LINE__)) return false;
               tc_fence_after();
 #pragma unroll 1
-              for (int cch = 0; cch < 4; ++cch) {
+              for (int cch = 0; cch < D / 32; ++cch) {   // this half's D / 2 columns of O
                 uint32_t o[16];
-                tmem_ld16(tO + h * 64 + cch * 16, o);
+                tmem_ld16(tO + h * (D / 2) + cch * 16, o);
                 tmem_wait_ld();
                 reg_fence<16>(o);
 #pragma unroll
                 for (int i = 0; i < 16; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * f);
-                tmem_st16(tO + h * 64 + cch * 16, o);
+                tmem_st16(tO + h * (D / 2) + cch * 16, o);
               }
               tmem_wait_st();
             }
@@ -511,7 +521,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             // at once (half 0 leaves its sum, the true maximum and the reference, half 1
             // its sum: fields of one float4 per row)
             uint32_t stc = x == 0 ? st_cntA : st_cntB;
-            float* st4 = reinterpret_cast<float*>(smem + kOffStats) + (((stc & 1) * 2 + x) * BM + r) * 4;
+            float* st4 = reinterpret_cast<float*>(smem + Dm::kOffStats) + (((stc & 1) * 2 + x) * BM + r) * 4;
             if (h == 0) {
               st4[0] = st.l;
               st4[1] = st.m_true;
@@ -538,7 +548,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int wq = warp & 3;
     const int r = (wq << 5) + lane;   // row of the tile = TMEM lane
     const uint32_t lane_addr = uint32_t(wq << 5) << 16;
-    float* scratch = reinterpret_cast<float*>(smem + kOffScratch) + wq * 1024;
+    float* scratch = reinterpret_cast<float*>(smem + Dm::kOffScratch) + wq * 1024;
     PairIter pi;
     pi.init(&p, w, &bars->ring, kClaimWarp, &wctx);
     int tA, tB, g, klo, khi;
@@ -557,19 +567,23 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int rec = valid ? ((tile.x + slot) * p.bs + tt) * p.Hq + g * p.G + hh : 0;
         if (!warp_wait(&bars->o_full[x], pc[x] & 1, wctx, 1 * 10000 + __LINE__)) { ok = false; break; }
         tc_fence_after();
-        // O in two rounds of two 32-column chunks; the output columns are released after
-        // the second round's TMEM reads, before its stores
+        // O in rounds of two 32-column chunks (two rounds at D = 128, one at D = 64); the
+        // output columns are released after the last round's TMEM reads, before its stores
         uint32_t va[32], vb[32];
         tmem_ld32(tO, va);
         tmem_ld32(tO + 32, vb);
         tmem_wait_ld();
         reg_fence<32>(va);
         reg_fence<32>(vb);
+        if (D == 64) {
+          tc_fence_before();
+          warp_arrive(&bars->o_free[x]);
+        }
         if (!warp_wait(&bars->stats_ready[x][pc[x] & 1], (pc[x] >> 1) & 1, wctx, 1 * 10000 + __LINE__)) {
           ok = false;
           break;
         }
-        const float4 sx = reinterpret_cast<const float4*>(smem + kOffStats)[((pc[x] & 1) * 2 + x) * BM + r];
+        const float4 sx = reinterpret_cast<const float4*>(smem + Dm::kOffStats)[((pc[x] & 1) * 2 + x) * BM + r];
         ++pc[x];
         // 1 / l, and the record: m_c = the true maximum (natural units), l_c = the sum
         // relative to it (the halves' sums are relative to the common reference)
@@ -591,15 +605,17 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         };
         store2(0);
-        tmem_ld32(tO + 64, va);
-        tmem_ld32(tO + 96, vb);
-        tmem_wait_ld();
-        reg_fence<32>(va);
-        reg_fence<32>(vb);
-        // every TMEM read of O_x done: the MMA may start the next pair's products into it
-        tc_fence_before();
-        warp_arrive(&bars->o_free[x]);
-        store2(64);
+        if (D == 128) {
+          tmem_ld32(tO + 64, va);
+          tmem_ld32(tO + 96, vb);
+          tmem_wait_ld();
+          reg_fence<32>(va);
+          reg_fence<32>(vb);
+          // every TMEM read of O_x done: the MMA may start the next pair's products into it
+          tc_fence_before();
+          warp_arrive(&bars->o_free[x]);
+          store2(64);
+        }
         if (valid) {
           part_m[rec] = st.y;
           part_l[rec] = st.z;
@@ -621,23 +637,34 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 bool fwd_sm100_supported(const DevPlan& p) {
   const int rows = p.G * p.bs;
-  return p.d == D && rows % 8 == 0 && rows <= BM && tensor_maps_available();
+  return (p.d == 64 || p.d == 128) && rows % 8 == 0 && rows <= BM && tensor_maps_available();
 }
 
-cudaError_t launch_fwd_partial_sm100(const DevPlan& p, const uint16_t* q, const uint16_t* k, const uint16_t* v,
-                                     float scale, void* part_o, float* part_m, float* part_l, cudaStream_t s) {
+namespace {
+
+template <int D>
+cudaError_t launch_fwd_sm100(const DevPlan& p, const uint16_t* q, const uint16_t* k, const uint16_t* v, float scale,
+                             void* part_o, float* part_m, float* part_l, cudaStream_t s) {
+  constexpr uint32_t kSmem = Dims<D>::kSmemBytes;
   CUtensorMap tq, tk, tv;
   if (!make_bf16_map_3d(&tq, q, D, p.Hq, p.Nq, p.G, p.bs)) return cudaErrorInvalidValue;
   if (!make_bf16_map_3d(&tk, k, D, p.Hkv, p.N, 1, BN)) return cudaErrorInvalidValue;
   if (!make_bf16_map_3d(&tv, v, D, p.Hkv, p.N, 1, BN)) return cudaErrorInvalidValue;
-  cudaError_t e = cudaFuncSetAttribute(fwd_partial_sm100_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       int(kSmemBytes));
+  cudaError_t e = cudaFuncSetAttribute(fwd_partial_sm100_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       int(kSmem));
   if (e != cudaSuccess) return e;
   // run-time claims start from item 0 at every launch
   if (p.dynamic && (e = cudaMemsetAsync(p.claim + 0, 0, sizeof(int), s)) != cudaSuccess) return e;
-  fwd_partial_sm100_kernel<<<p.W, kThreads, kSmemBytes, s>>>(tq, tk, tv, p, scale * kLog2e, part_o, part_m,
-                                                             part_l);
+  fwd_partial_sm100_kernel<D><<<p.W, kThreads, kSmem, s>>>(tq, tk, tv, p, scale * kLog2e, part_o, part_m, part_l);
   return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_fwd_partial_sm100(const DevPlan& p, const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                                     float scale, void* part_o, float* part_m, float* part_l, cudaStream_t s) {
+  if (p.d == 64) return launch_fwd_sm100<64>(p, q, k, v, scale, part_o, part_m, part_l, s);
+  return launch_fwd_sm100<128>(p, q, k, v, scale, part_o, part_m, part_l, s);
 }
 
 }  // namespace splitkv

@@ -29,7 +29,8 @@ CASES = {
     "tcgen05_static": dict(w=dict(), plan=dict()),
     "tcgen05_claims_bf16": dict(w=dict(), plan=dict(q_slice=2, tile_cost=True, dynamic_claim=True,
                                                       partial_bf16=True)),
-    "mma_d64": dict(w=dict(Hq=4, Hkv=2, d=64), plan=dict()),
+    "tcgen05_d64": dict(w=dict(Hq=4, Hkv=2, d=64), plan=dict()),
+    "mma_bs1": dict(w=dict(Hq=2, Hkv=1, d=64, bs=1, anchors=200, C=64), plan=dict()),
     "reading_b": dict(w=dict(Hq=8, Hkv=1), plan=dict(block_keys_in_context=True)),
 }
 

@@ -26,7 +26,7 @@ CASES = {
     "tcgen05_R2": dict(w=dict(), R=2, plan=dict()),
     "tcgen05_R3_claims_bf16": dict(w=dict(), R=3, plan=dict(q_slice=2, tile_cost=True, dynamic_claim=True,
                                                             partial_bf16=True)),
-    "mma_d64_R4": dict(w=dict(Hq=4, Hkv=2, d=64), R=4, plan=dict()),
+    "d64_R4": dict(w=dict(Hq=4, Hkv=2, d=64), R=4, plan=dict()),
     "chunk_not_dividing_R2": dict(w=dict(Hq=4, Hkv=1, d=128, C=100, lens=(257, 3, 1000, 61)), R=2, plan=dict()),
     "reading_b_R2": dict(w=dict(Hq=8, Hkv=1), R=2, plan=dict(block_keys_in_context=True)),
     "contiguous_ranks_R3": dict(w=dict(), R=3, plan=dict(contiguous_ranks=True, q_slice=1)),
@@ -148,7 +148,7 @@ def test_bwd_workload_over_four_ranks_sampled(splitkv):
         assert np.isfinite(out[n]).all(), n
 
 
-@pytest.mark.parametrize("R,case", [(2, "tcgen05"), (3, "tcgen05"), (3, "mma_d64")])
+@pytest.mark.parametrize("R,case", [(2, "tcgen05"), (3, "tcgen05"), (3, "d64")])
 def test_merge_to_owners_is_the_merge_laid_out_by_owner(splitkv, R, case):
     """splitkv_merge_to_owners (the exchange fused into the merge) stores, for every rank,
     exactly the rows its plain merge writes, each block's rows in its owner's receive buffer
@@ -191,7 +191,7 @@ def test_merge_to_owners_is_the_merge_laid_out_by_owner(splitkv, R, case):
         assert_close("LSE", lse.cpu().numpy().astype(np.float64), L[rows], TOL_LSE)
 
 
-@pytest.mark.parametrize("R,case", [(2, "tcgen05"), (3, "mma_d64")])
+@pytest.mark.parametrize("R,case", [(2, "tcgen05"), (3, "d64")])
 def test_bwd_reduce_to_owners_is_the_reduce_laid_out_by_owner(splitkv, R, case):
     """splitkv_bwd_reduce_to_owners (the dq exchange fused into the dQ reduce) stores every
     rank's dq rows exactly as its plain backward writes them, in the owners' receive buffers

@@ -182,6 +182,8 @@ def test_block_keys_in_context_fwd_bwd(splitkv, case):
 
 BF16_CASES = {
     "gqa4_d128": dict(Hq=8, Hkv=2, d=128),                           # records by bulk tensor stores
+    "gqa4_d64": dict(Hq=8, Hkv=2, d=64),                             # head_dim 64 on the tcgen05 kernels
+    "mha_bs16_d64": dict(Hq=1, Hkv=1, d=64),                         # the tiny workload's layout
     "g1_bs8_d128": dict(Hq=2, Hkv=2, d=128, bs=8, anchors=40),      # 8-row slots: per-lane stores
     "gqa8_d128": dict(Hq=8, Hkv=1, d=128),
     "chunk_not_dividing": dict(Hq=4, Hkv=1, d=128, C=100, lens=(257, 3, 1000, 61)),
@@ -220,15 +222,20 @@ def test_partial_bf16_records(splitkv):
         assert_close("m_c", m[e].astype(np.float64), p["m"], TOL_LSE)
 
 
+# rows of a 128-row tile in slots of G * bs: with G * bs not a multiple of 8 (here bs = 1)
+# the forward and backward run on the mma.sync kernels, which offer neither option
+MMA_ONLY = dict(Hq=2, Hkv=2, d=64, bs=1, anchors=200, C=64)
+
+
 def test_partial_bf16_needs_the_tcgen05_path(splitkv):
-    w = small(Hq=2, Hkv=2, d=64)
+    w = small(**MMA_ONLY)
     with pytest.raises(splitkv.SplitKVError) as ei:
         run(w, partial_bf16=True)
     assert ei.value.status == -2   # SPLITKV_ERR_UNSUPPORTED
 
 
 def test_dynamic_claim_needs_the_tcgen05_path(splitkv):
-    w = small(Hq=2, Hkv=2, d=64)
+    w = small(**MMA_ONLY)
     with pytest.raises(splitkv.SplitKVError) as ei:
         run(w, dynamic_claim=True)
     assert ei.value.status == -2   # SPLITKV_ERR_UNSUPPORTED

@@ -79,10 +79,7 @@ def test_static_scratch_matches_oracle_and_workspace_path_on_consecutive_calls(s
     flags = OPTIONS[opt]
     rb = bool(flags.get("block_keys_in_context"))
     wa = small(Hq=8, Hkv=2, d=128, grad=False)
-    # the second problem: d = 64 takes the mma.sync path, which offers neither run-time
-    # claims nor bf16 records; those options run it at d = 128
-    d_b = 128 if (flags.get("dynamic_claim") or flags.get("partial_bf16")) else 64
-    wb = small(Hq=4, Hkv=1, d=d_b, lens=(900, 1500), anchors=30, seed=5, grad=False)
+    wb = small(Hq=4, Hkv=1, d=64, lens=(900, 1500), anchors=30, seed=5, grad=False)   # another head_dim
     ta, pa = _setup(skv, wa, **flags)
     tb, pb = _setup(skv, wb, **flags)
     want_a = oracle_fwd(wa, rb=rb)
