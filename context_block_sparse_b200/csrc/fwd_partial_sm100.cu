@@ -18,19 +18,19 @@
 //   warp 1      MMA issuer (one thread): S_X = Q_X K^T into TMEM, then
 //               O_X += P_X V with P_X read from TMEM (bf16, aliasing S_X);
 //   warp 2      tensor-memory allocation (512 columns: S_A, S_B, O_A, O_B);
-//   warps 4-11  softmax of both tiles (A, then B, at every key tile): warps 4-7
-//               take score columns 0..63, warps 8-11 columns 64..127 (thread =
-//               row = TMEM lane); the two threads of a row agree on the key
-//               tile's row maximum through shared memory before exponentiating;
+//   warps 4-11  softmax of both tiles (A, then B, at every key tile): warp 4 + q
+//               holds rows 32q..32q+15 and warp 8 + q rows 32q+16..32q+31 through
+//               the 16-lane TMEM shapes, two rows and 32 columns per thread, so
+//               that the four threads of a row reduce its maximum by shuffles;
 //   warps 12-15 record epilogue of both tiles: O_X / l from TMEM to the record,
 //               so that the softmax warps go on to the next pair at once and the
 //               output columns return to the MMA right after their last read.
 // The softmax keeps, per row, a reference maximum m_ref, taken from the first
-// 64-column half in which the row has allowed keys; every half is exponentiated
-// against it in one pass, and only when a score exceeds m_ref by more than 2^32
-// (in P) are O, l and the P already written rescaled to a new reference -- the
-// result is the same, the reference is exact bookkeeping.  The record written
-// is m_c = the row's true maximum (natural units), l_c = sum exp(s - m_c) and O_c = sum exp(s - m_c) v / l_c.
+// key tile in which the row has allowed keys; later tiles exponentiate against
+// it, and only when a score exceeds m_ref by more than 2^32 (in P) are O and l
+// rescaled to a new reference -- the result is the same, the reference is exact
+// bookkeeping.  The record written is m_c = the row's true maximum (natural
+// units), l_c = sum exp(s - m_c) and O_c = sum exp(s - m_c) v / l_c.
 // Rows are masked to their block's [lo, hi).  The epilogue stores go through a
 // 4 KB per-warp staging buffer so that every store instruction writes whole
 // 128-byte row segments (bf16 records: 64 bytes per row straight from registers).
@@ -74,8 +74,8 @@ struct Dims {
   static constexpr uint32_t kOffV = kOffK + kStages * kTile;        // V stages
   static constexpr uint32_t kOffScratch = kOffV + kStages * kTile;  // record staging, 4 KB per epilogue warp
   static constexpr uint32_t kOffStats = kOffScratch + 4 * 4096;     // row statistics [2 pair parities][2 tiles][128] float4
-  static constexpr uint32_t kOffXchg = kOffStats + 2 * 2 * BM * 16; // half maxima [2 exchange parities][2 halves][128]
-  static constexpr uint32_t kOffBar = kOffXchg + 2 * 2 * BM * 4;    // mbarriers
+  static constexpr uint32_t kOffRows = kOffStats + 2 * 2 * BM * 16; // allowed keys (lo, hi) [2 tiles][128] int2
+  static constexpr uint32_t kOffBar = kOffRows + 2 * BM * 8;         // mbarriers
   static constexpr uint32_t kSmemBytes = kOffBar + 512 + 1024;      // + alignment slack
   static_assert(kSmemBytes <= 232448, "shared memory per block");
 };
@@ -88,9 +88,6 @@ struct Bars {
   // stats_ready[x][b]: the softmax warps of tile x left the row statistics of a pair
   // in stats buffer b = pair parity
   uint64_t o_full[2], stats_ready[2][2];
-  // xchg[q]: the two warps holding rows 32q..32q+31 (one per 64-column half) have
-  // left their halves' maxima of a key tile (count 2 warps)
-  uint64_t xchg[4];
   uint64_t mma_done;
   ClaimRing ring;   // run-time claims: the producer hands items to the MMA thread and the 8 softmax warps
   uint32_t tmem_base;
@@ -144,49 +141,60 @@ struct PairIter {
 };
 
 
-// One row of one query tile in the softmax warps: its allowed keys [lo, hi), the
-// reference maximum and the true maximum (log2 units) and the sum of P (relative to
-// the reference) over this thread's half of the columns.
-struct RowState {
-  int lo, hi;
-  float m_ref, m_true, l;
+// The two rows a softmax thread holds in one query tile (16x256b fragments: rows
+// t/4 and t/4 + 8 of its warp's 16 lanes): the reference maximum and the true
+// maximum (log2 units), and the sum of P relative to the reference over this
+// thread's 32 columns of each row (the four threads of a row add theirs at the
+// end of the tile).  The rows' allowed keys live in shared memory.
+struct Rows2 {
+  float m_ref[2], m_true[2], l[2];
 };
 
-// Maximum of 64 raw scores of one row (masked scores are -inf).
-__device__ __forceinline__ float row_max(const uint32_t (&v)[64]) {
-  float m0 = -INFINITY, m1 = -INFINITY, m2 = -INFINITY, m3 = -INFINITY;
+// Row maxima of the 64 scores a thread holds (32 per row; masked scores -inf),
+// reduced over the four threads of each row.
+__device__ __forceinline__ void row_max2(const uint32_t (&v)[64], float& m0, float& m1) {
+  float a0 = -INFINITY, a1 = -INFINITY, b0 = -INFINITY, b1 = -INFINITY;
 #pragma unroll
-  for (int i = 0; i < 64; i += 8) {
-    m0 = fmax3(m0, __uint_as_float(v[i]), __uint_as_float(v[i + 1]));
-    m1 = fmax3(m1, __uint_as_float(v[i + 2]), __uint_as_float(v[i + 3]));
-    m2 = fmax3(m2, __uint_as_float(v[i + 4]), __uint_as_float(v[i + 5]));
-    m3 = fmax3(m3, __uint_as_float(v[i + 6]), __uint_as_float(v[i + 7]));
+  for (int i = 0; i < 16; i += 2) {
+    a0 = fmax3(a0, __uint_as_float(v[4 * i]), __uint_as_float(v[4 * i + 1]));
+    b0 = fmax3(b0, __uint_as_float(v[4 * i + 2]), __uint_as_float(v[4 * i + 3]));
+    a1 = fmax3(a1, __uint_as_float(v[4 * i + 4]), __uint_as_float(v[4 * i + 5]));
+    b1 = fmax3(b1, __uint_as_float(v[4 * i + 6]), __uint_as_float(v[4 * i + 7]));
   }
-  return fmaxf(fmaxf(m0, m1), fmaxf(m2, m3));
+  m0 = fmaxf(a0, a1);
+  m1 = fmaxf(b0, b1);
+  m0 = fmaxf(m0, __shfl_xor_sync(0xffffffffu, m0, 1));
+  m1 = fmaxf(m1, __shfl_xor_sync(0xffffffffu, m1, 1));
+  m0 = fmaxf(m0, __shfl_xor_sync(0xffffffffu, m0, 2));
+  m1 = fmaxf(m1, __shfl_xor_sync(0xffffffffu, m1, 2));
 }
 
-// P = exp2(v * c + nm) over 64 columns of a row (exactly 0 for a masked score,
-// -inf), packed to bf16 pairs into 32 TMEM columns at tS; returns the row sum of
-// the fp32 P.  MUFU for every pair: the two softmax warps of an SM sub-partition
-// share one tile, so its exponentials take 1024 MUFU cycles, below the tile's two
-// products; the FMA-pipe polynomial would only add registers (and spills).
-__device__ __forceinline__ float exp_pack_store(const uint32_t (&v)[64], float c, float nm, uint32_t tS) {
-  float s0 = 0.f, s1 = 0.f;
+// P = exp2(v * c - m_row) for the thread's 64 scores (exactly 0 for a masked
+// score, -inf), packed to bf16 pairs and stored with 16x128b over the scores'
+// first 64 TMEM columns (P of keys 2k, 2k + 1 in column k); adds the rows' sums of
+// the fp32 P to l0, l1.  MUFU for every exponential.
+__device__ __forceinline__ void exp_pack_store2(const uint32_t (&v)[64], float c, float nm0, float nm1,
+                                                uint32_t tS, float& l0, float& l1) {
+  float s00 = 0.f, s01 = 0.f, s10 = 0.f, s11 = 0.f;
 #pragma unroll
-  for (int cch = 0; cch < 2; ++cch) {
+  for (int half = 0; half < 2; ++half) {
     uint32_t pk[16];
 #pragma unroll
-    for (int i = 0; i < 16; ++i) {
-      const int col = cch * 32 + 2 * i;
-      float x0, x1;
-      ffma2(x0, x1, __uint_as_float(v[col]), __uint_as_float(v[col + 1]), c, c, nm, nm);
-      const float p0 = fast_exp2(x0), p1 = fast_exp2(x1);
-      fadd2(s0, s1, s0, s1, p0, p1);
-      pk[i] = pack_bf16(p0, p1);
+    for (int i = 0; i < 8; ++i) {
+      const int q = 4 * (half * 8 + i);
+      float x0, x1, y0, y1;
+      ffma2(x0, x1, __uint_as_float(v[q]), __uint_as_float(v[q + 1]), c, c, nm0, nm0);
+      ffma2(y0, y1, __uint_as_float(v[q + 2]), __uint_as_float(v[q + 3]), c, c, nm1, nm1);
+      const float p0 = fast_exp2(x0), p1 = fast_exp2(x1), r0 = fast_exp2(y0), r1 = fast_exp2(y1);
+      fadd2(s00, s01, s00, s01, p0, p1);
+      fadd2(s10, s11, s10, s11, r0, r1);
+      pk[2 * i] = pack_bf16(p0, p1);
+      pk[2 * i + 1] = pack_bf16(r0, r1);
     }
-    tmem_st16p(tS + cch * 16, pk);
+    tmem_st16x128b_x8(tS + half * 32, pk);
   }
-  return s0 + s1;
+  l0 += s00 + s01;
+  l1 += s10 + s11;
 }
 
 template <int D>
@@ -227,7 +235,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&bars->stats_ready[x][1], 8);
     }
     mbar_init(&bars->mma_done, 1);
-    for (int q = 0; q < 4; ++q) mbar_init(&bars->xchg[q], 2);
     claim_ring_init(&bars->ring, kClaimConsumers);
     bars->abort_flag = 0;
     mbar_fence_init();
@@ -362,13 +369,11 @@ __global__ void __launch_bounds__(kThreads, 1)
               if (!mbar_wait(&bars->v_full[s], (c / kStages) & 1, wctx, 1 * 10000 + __LINE__)) { ok = false; break; }
             }
             tc_fence_after();
-            // O_X (+)= P_X V : P in TMEM (keys 0..63 in columns 0..31 of S_X, keys
-            // 64..127 in columns 64..95: each half written over the scores it replaces),
-            // V MN-major in smem
+            // O_X (+)= P_X V : P in TMEM (keys 2k, 2k + 1 in column k of S_X), V MN-major
+            // in smem
             for (int kk = 0; kk < BN / 16; ++kk) {
               const uint64_t b = smem_desc_sw128(sV + s * kTile + kk * 2048, kHalf, 1024);
-              const uint32_t pcol = kk < 4 ? kk * 8 : 64 + (kk - 4) * 8;
-              mma_ts(tmem + 256 + x * 128, tmem + x * 128 + pcol, b, kIdescPV, (j > 0 || kk > 0) ? 1u : 0u);
+              mma_ts(tmem + 256 + x * 128, tmem + x * 128 + kk * 8, b, kIdescPV, (j > 0 || kk > 0) ? 1u : 0u);
             }
             mma_commit(&bars->o_ready[x]);
             if (!more) mma_commit(&bars->o_full[x]);           // tile x's output complete
@@ -406,98 +411,122 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp >= 4 && warp < 12) {
     // ------------------------------------------------------------ softmax
-    // Warps 4-7 take columns 0..63 of every score tile, warps 8-11 columns 64..127;
-    // both tiles of a pair go through the same warps (A then B at every key tile).
-    // The two threads of a row agree on its key-tile maximum through shared memory
-    // before exponentiating, so they keep one reference and one O.
-    const int h = (warp - 4) >> 2;            // column half
-    const int wq = warp & 3;
-    const int r = (wq << 5) + lane;           // row of the tile = TMEM lane
-    const uint32_t lane_addr = uint32_t(wq << 5) << 16;
-    float* xs = reinterpret_cast<float*>(smem + Dm::kOffXchg);
+    // Warps 4-11 take both tiles of a pair, A then B at every key tile.  Warp 4 + q
+    // holds rows 32q..32q+15 of a tile and warp 8 + q rows 32q+16..32q+31, through
+    // the 16-lane TMEM shapes: each thread has two rows (t/4 and t/4 + 8 of its
+    // warp's 16) and 32 of their 128 columns, the four threads of a row sit in one
+    // warp and reduce its maximum with two shuffles.
+    const int wq = warp & 3, h = (warp - 4) >> 2;
+    const int rbase = wq * 32 + h * 16;           // the warp's first row = TMEM lane
+    const int r0 = rbase + (lane >> 2), r1 = r0 + 8;
+    const uint32_t lane_addr = uint32_t(rbase) << 16;
+    const int cpair = 2 * (lane & 3);             // this thread's column pair in every 8 columns
+    int2* rows_lh = reinterpret_cast<int2*>(smem + Dm::kOffRows);
     PairIter pi;
     pi.init(&p, w, &bars->ring, kClaimWarp, &wctx);
     int tA, tB, g, klo, khi;
-    uint32_t s_cntA = 0, s_cntB = 0, o_cntA = 0, o_cntB = 0, st_cntA = 0, st_cntB = 0, n_x = 0;
+    uint32_t s_cntA = 0, s_cntB = 0, o_cntA = 0, o_cntB = 0, st_cntA = 0, st_cntB = 0;
     bool ok = true;
     while (ok && pi.next(tA, tB, g, klo, khi)) {
       const int nx = tB >= 0 ? 2 : 1;
       const int n_kt = (khi - klo + BN - 1) / BN;
-      RowState rsA, rsB;
-      auto init_row = [&](RowState& st, const int t) {
-        st.lo = st.hi = 0;   // the row's allowed keys (none for a padding row)
-        st.m_ref = st.m_true = -INFINITY;
-        st.l = 0.f;
-        if (t >= 0) {
-          const int4 tile = p.tiles[t];
-          const int slot = r / rows_per_slot;
-          if (slot < tile.y - tile.x) {
-            const int4 ent = p.entries[tile.x + slot];
-            st.lo = ent.y;
-            st.hi = ent.z;
+      Rows2 rsA, rsB;
+#pragma unroll
+      for (int k = 0; k < 2; ++k) {
+        rsA.m_ref[k] = rsA.m_true[k] = rsB.m_ref[k] = rsB.m_true[k] = -INFINITY;
+        rsA.l[k] = rsB.l[k] = 0.f;
+      }
+      // the allowed keys of this thread's rows in both tiles (none for a padding row),
+      // kept in shared memory by the first thread of each row (read by the row's four)
+      if ((lane & 3) == 0) {
+#pragma unroll
+        for (int x = 0; x < 2; ++x) {
+          const int t = x == 0 ? tA : tB;
+          int4 tile = make_int4(0, 0, 0, 0);
+          if (t >= 0) tile = p.tiles[t];
+#pragma unroll
+          for (int k = 0; k < 2; ++k) {
+            const int rr = k == 0 ? r0 : r1;
+            const int slot = rr / rows_per_slot;
+            int2 lh = make_int2(0, 0);
+            if (t >= 0 && slot < tile.y - tile.x) {
+              const int4 ent = p.entries[tile.x + slot];
+              lh = make_int2(ent.y, ent.z);
+            }
+            rows_lh[x * BM + rr] = lh;
           }
         }
-      };
-      init_row(rsA, tA);
-      init_row(rsB, tB);
+      }
+      __syncwarp();
       // key tile j of tile x: false when a wait gave up
-      auto step = [&](RowState& st, uint32_t& sc, const uint32_t oc, const int x, const int j) -> bool {
+      auto step = [&](Rows2& st, uint32_t& sc, const uint32_t oc, const int x, const int j) -> bool {
           const uint32_t tS = tmem + lane_addr + x * 128;
           const uint32_t tO = tmem + lane_addr + 256 + x * 128;   // O_X: rescaled in place on a new reference
           if (!warp_wait(&bars->s_ready[x], sc & 1, wctx, 1 * 10000 + __LINE__)) return false;
           ++sc;
           tc_fence_after();
-          // the row's allowed columns in this half of the key tile: [a, b)
-          const int k0 = klo + j * BN + h * 64;
-          const int a = st.lo - k0, b = st.hi - k0;
           uint32_t v[64];
-          tmem_ld32p(tS + h * 64, v);
-          tmem_ld32p(tS + h * 64 + 32, v + 32);
+          tmem_ld16x256b_x16(tS, v);
           tmem_wait_ld();
           reg_fence<64>(v);
-          // masked scores become -inf (their exponentials are exactly 0)
-          if (!__all_sync(0xffffffffu, a <= 0 && b >= 64)) {
+          // the rows' allowed columns in this key tile: [a, b); masked scores become -inf
+          const int k0 = klo + j * BN;
+          const int2 lh0 = rows_lh[x * BM + r0], lh1 = rows_lh[x * BM + r1];
+          const int a0 = lh0.x - k0, b0 = lh0.y - k0, a1 = lh1.x - k0, b1 = lh1.y - k0;
+          if (!__all_sync(0xffffffffu, a0 <= 0 && b0 >= BN && a1 <= 0 && b1 >= BN)) {
 #pragma unroll
-            for (int i = 0; i < 64; ++i) v[i] = (i >= a && i < b) ? v[i] : 0xff800000u;
+            for (int i = 0; i < 16; ++i) {
+#pragma unroll
+              for (int e = 0; e < 2; ++e) {
+                const int col = 8 * i + cpair + e;
+                v[4 * i + e] = (col >= a0 && col < b0) ? v[4 * i + e] : 0xff800000u;
+                v[4 * i + 2 + e] = (col >= a1 && col < b1) ? v[4 * i + 2 + e] : 0xff800000u;
+              }
+            }
           }
-          const float mh = scale_log2 * row_max(v);
-          // the other half's maximum of this row (exchange slots alternate by parity)
-          float* slot = xs + (n_x & 1) * 2 * BM;
-          slot[h * BM + r] = mh;
-          __threadfence_block();
-          warp_arrive(&bars->xchg[wq]);
-          if (!warp_wait(&bars->xchg[wq], n_x & 1, wctx, 1 * 10000 + __LINE__)) return false;
-          const float mt = fmaxf(mh, slot[(h ^ 1) * BM + r]);   // -inf: no allowed key in the tile
-          ++n_x;
+          float mt0, mt1;
+          row_max2(v, mt0, mt1);
+          mt0 *= scale_log2;   // -inf: no allowed key of the row in this tile
+          mt1 *= scale_log2;
           // a row's first allowed keys set its reference (its O and l are still zero);
           // a later maximum past the headroom rescales O and l to a new reference
-          if (st.m_ref == -INFINITY) st.m_ref = mt;
-          const bool over = mt > st.m_ref + kHeadroomLog2;
-          if (__any_sync(0xffffffffu, over)) {
-            const float f = over ? fast_exp2(st.m_ref - mt) : 1.f;
+          if (st.m_ref[0] == -INFINITY) st.m_ref[0] = mt0;
+          if (st.m_ref[1] == -INFINITY) st.m_ref[1] = mt1;
+          const bool over0 = mt0 > st.m_ref[0] + kHeadroomLog2, over1 = mt1 > st.m_ref[1] + kHeadroomLog2;
+          if (__any_sync(0xffffffffu, over0 || over1)) {
+            const float f0 = over0 ? fast_exp2(st.m_ref[0] - mt0) : 1.f;
+            const float f1 = over1 ? fast_exp2(st.m_ref[1] - mt1) : 1.f;
             if (j > 0) {
-              // this half's O columns, after PV(j-1)
+              // the rows' O, after PV(j-1): 32 columns per 16x256b.x4 round trip
               if (!warp_wait(&bars->o_ready[x], (oc + j - 1) & 1, wctx, 1 * 10000 + __LINE__)) return false;
               tc_fence_after();
 #pragma unroll 1
-              for (int cch = 0; cch < D / 32; ++cch) {   // this half's D / 2 columns of O
+              for (int cch = 0; cch < D / 32; ++cch) {
                 uint32_t o[16];
-                tmem_ld16(tO + h * (D / 2) + cch * 16, o);
+                tmem_ld16x256b_x4(tO + cch * 32, o);
                 tmem_wait_ld();
                 reg_fence<16>(o);
 #pragma unroll
-                for (int i = 0; i < 16; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * f);
-                tmem_st16(tO + h * (D / 2) + cch * 16, o);
+                for (int i = 0; i < 4; ++i) {
+                  o[4 * i] = __float_as_uint(__uint_as_float(o[4 * i]) * f0);
+                  o[4 * i + 1] = __float_as_uint(__uint_as_float(o[4 * i + 1]) * f0);
+                  o[4 * i + 2] = __float_as_uint(__uint_as_float(o[4 * i + 2]) * f1);
+                  o[4 * i + 3] = __float_as_uint(__uint_as_float(o[4 * i + 3]) * f1);
+                }
+                tmem_st16x256b_x4(tO + cch * 32, o);
               }
               tmem_wait_st();
             }
-            st.l *= f;
-            if (over) st.m_ref = mt;
+            st.l[0] *= f0;
+            st.l[1] *= f1;
+            if (over0) st.m_ref[0] = mt0;
+            if (over1) st.m_ref[1] = mt1;
           }
-          const float m_use = (st.m_ref == -INFINITY) ? 0.f : st.m_ref;
-          // P of this half over the scores it replaces: columns 0..31 (half 0), 64..95 (half 1)
-          st.l += exp_pack_store(v, scale_log2, -m_use, tS + h * 64);
-          st.m_true = fmaxf(st.m_true, mt);
+          // P over the scores' first 64 columns (every score of these rows is in registers)
+          exp_pack_store2(v, scale_log2, st.m_ref[0] == -INFINITY ? 0.f : -st.m_ref[0],
+                          st.m_ref[1] == -INFINITY ? 0.f : -st.m_ref[1], tS, st.l[0], st.l[1]);
+          st.m_true[0] = fmaxf(st.m_true[0], mt0);
+          st.m_true[1] = fmaxf(st.m_true[1], mt1);
           tmem_wait_st();
           tc_fence_before();
           warp_arrive(&bars->p_ready[x]);
@@ -506,7 +535,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int j = 0; j < n_kt && ok; ++j) {
 #pragma unroll 1
         for (int x = 0; x < nx && ok; ++x) {
-          RowState st = x == 0 ? rsA : rsB;
+          Rows2 st = x == 0 ? rsA : rsB;
           uint32_t sc = x == 0 ? s_cntA : s_cntB;
           ok = step(st, sc, x == 0 ? o_cntA : o_cntB, x, j);
           if (x == 0) {
@@ -517,17 +546,16 @@ __global__ void __launch_bounds__(kThreads, 1)
             s_cntB = sc;
           }
           if (ok && j == n_kt - 1) {
-            // the tile's last key tile: its rows' statistics go to the epilogue warps
-            // at once (half 0 leaves its sum, the true maximum and the reference, half 1
-            // its sum: fields of one float4 per row)
+            // the tile's last key tile: its rows' statistics go to the epilogue warps at
+            // once (the sum over the row's four threads, the true maximum, the reference)
             uint32_t stc = x == 0 ? st_cntA : st_cntB;
-            float* st4 = reinterpret_cast<float*>(smem + Dm::kOffStats) + (((stc & 1) * 2 + x) * BM + r) * 4;
-            if (h == 0) {
-              st4[0] = st.l;
-              st4[1] = st.m_true;
-              st4[2] = st.m_ref;
-            } else {
-              st4[3] = st.l;
+            float4* st4 = reinterpret_cast<float4*>(smem + Dm::kOffStats) + ((stc & 1) * 2 + x) * BM;
+#pragma unroll
+            for (int k = 0; k < 2; ++k) {
+              float lk = st.l[k];
+              lk += __shfl_xor_sync(0xffffffffu, lk, 1);
+              lk += __shfl_xor_sync(0xffffffffu, lk, 2);
+              if ((lane & 3) == 0) st4[k == 0 ? r0 : r1] = make_float4(lk, st.m_true[k], st.m_ref[k], 0.f);
             }
             __threadfence_block();
             warp_arrive(&bars->stats_ready[x][stc & 1]);

@@ -97,9 +97,8 @@ class Core:
 # ---------------------------------------------------------------------------
 # forward kernel: query tiles two at a time (A, B), K and V rings of two stages each (a
 # pair's first K/V tiles requested before its Q buffer frees); two softmax warpgroups,
-# one per 64-column half of every score tile, take tile A then tile B at each key tile
-# and exchange their halves' row maxima through shared memory (slots alternating by
-# exchange parity); the records leave through separate epilogue warps (the tile's last
+# one per half of the rows of every score tile, take tile A then tile B at each key
+# tile; the records leave through separate epilogue warps (the tile's last
 # PV and the softmax's row statistics, double-buffered by pair parity, hand each tile
 # over; the epilogue releases O after reading it)
 # ---------------------------------------------------------------------------
@@ -107,11 +106,10 @@ class Forward(Core):
     def __init__(self, pairs, seed, drop=None):
         names = ["q_full", "q_empty", "k_full0", "k_full1", "v_full0", "v_full1", "k_empty0", "k_empty1",
                  "v_empty0", "v_empty1", "s_ready0", "s_ready1", "p_ready0", "p_ready1", "o_ready0", "o_ready1",
-                 "o_free0", "o_free1", "o_full0", "o_full1", "stats0_0", "stats0_1", "stats1_0", "stats1_1",
-                 "xchg"]
+                 "o_free0", "o_free1", "o_full0", "o_full1", "stats0_0", "stats0_1", "stats1_0", "stats1_1"]
         super().__init__(seed, names)
-        for n in ("p_ready0", "p_ready1", "stats0_0", "stats0_1", "stats1_0", "stats1_1", "xchg"):
-            self.B[n] = Bar(2)        # one arrival per column half
+        for n in ("p_ready0", "p_ready1", "stats0_0", "stats0_1", "stats1_0", "stats1_1"):
+            self.B[n] = Bar(2)        # one arrival per softmax warpgroup
         self.pairs = pairs            # [(nx, n_kt)]
         self.drop = drop
         self.Q = None
@@ -120,8 +118,7 @@ class Forward(Core):
         self.S = [None, None]
         self.O = [None, None]
         self.ST = {}                  # (tile, buffer) -> (pair, halves written) or ("read",)
-        self.PH = [set(), set()]      # halves whose P of the current key tile is in S_x
-        self.XS = {}                  # exchange slot (parity, half) -> exchange index written
+        self.PH = [set(), set()]      # warpgroups whose rows' P of the current key tile is in S_x
         self.rescale = {}
 
     def producer(self):
@@ -209,7 +206,7 @@ class Forward(Core):
 
     def softmax(self, h):
         kv = 0
-        s_cnt, o_cnt, st_cnt, n = [0, 0], [0, 0], [0, 0], 0
+        s_cnt, o_cnt, st_cnt = [0, 0], [0, 0], [0, 0]
         for i, (nx, nkt) in enumerate(self.pairs):
             for j in range(nkt):
                 c = kv + j
@@ -218,13 +215,6 @@ class Forward(Core):
                     s_cnt[x] += 1
                     self.check(self.S[x] == ("S", i, c) and h not in self.PH[x],
                                f"softmax half {h} ({x},{c}) finds {self.S[x]}")
-                    self.XS[(n % 2, h)] = n
-                    self.B["xchg"].arrive()
-                    if self.drop != "xchg":
-                        yield from self.wait("xchg", n)
-                    self.check(self.XS.get((n % 2, 1 - h)) == n,
-                               f"half {h} reads exchange {self.XS.get((n % 2, 1 - h))} for {n}")
-                    n += 1
                     if j > 0 and self.rng.random() < 0.2:   # the rare rescale of O after PV(j - 1)
                         yield from self.wait(f"o_ready{x}", o_cnt[x] + j - 1)
                         self.check(self.O[x] == ("acc", i, j), f"rescale finds O {self.O[x]}")
@@ -567,7 +557,7 @@ def test_protocol_holds_on_random_schedules(kernel):
 
 
 @pytest.mark.parametrize("kernel,drop", [("forward", "kv_empty"), ("forward", "q_empty"), ("forward", "o_free"),
-                                         ("forward", "stats"), ("forward", "xchg"),
+                                         ("forward", "stats"),
                                          ("dkdv", "qd_empty"),
                                          ("dkdv", "kv_empty"), ("dkdv", "lookahead_before_dv"), ("dq", "kv_empty"),
                                          ("dq", "qd_empty")])
