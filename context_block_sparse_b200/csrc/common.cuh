@@ -57,6 +57,18 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
+// Named CTA barriers (ids 1..15; id 0 is __syncthreads): count = all threads taking part,
+// a multiple of 32.  arrive releases the caller's earlier shared-memory writes to the
+// threads that sync on the same barrier; sync waits for count arrivals.
+template <int kId>
+__device__ __forceinline__ void named_sync(int count) {
+  asm volatile("bar.sync %0, %1;" ::"n"(kId), "r"(count) : "memory");
+}
+template <int kId>
+__device__ __forceinline__ void named_arrive(int count) {
+  asm volatile("bar.arrive %0, %1;" ::"n"(kId), "r"(count) : "memory");
+}
+
 // Hardware base-2 exponential (MUFU.EX2); exp2(-inf) = 0.
 __device__ __forceinline__ float fast_exp2(float x) {
   float y;

@@ -336,70 +336,125 @@ __global__ void __launch_bounds__(kMergeThreads)
 }
 
 // ---------------------------------------------------------------------------
-// dq reduce + in-block backward: grid (A, Hkv)
-// smem: kb, vb [bs][D] bf16; P, dS [rows][bs] fp32 (rows = G*bs, ordered
-// (token, head)); q, dout [rows][D] bf16 when stage_rows; entry ids
+// dq reduce + in-block backward: grid (A, Hkv), two roles of 128 threads that run
+// side by side, so that the partial stream keeps HBM busy while the in-block term is
+// computed:
+//   stream role (warps 0-3): for 32 rows at a time, the sum of the chunk dq partials
+//     in ascending chunk order (EG records in flight per thread), plus the rows'
+//     in-block dq taken from a shared-memory slot -> dq;
+//   block role (warps 4-7): P, dS of the bs block keys and the rows' in-block dq
+//     (-> the slot of the same 32 rows), then dkb = scale dS^T Q and dvb = P^T dO.
+// The two slots are handed over with named barriers (full: block -> stream, empty:
+// stream -> block).  The block role runs its products on the tensor cores (mma.sync
+// m16n8k16: bf16 operands, P and dS rounded to bf16 as in the chunk kernels; fp32
+// accumulators) when the rows and the block keys come in multiples of 16, otherwise
+// on the FMA pipes in fp32.
 // ---------------------------------------------------------------------------
-template <int D, bool kBf16Rec>
-__global__ void __launch_bounds__(kMergeThreads, 2)
-    bwd_reduce_kernel(DevPlan p, const uint16_t* __restrict__ q, const uint16_t* __restrict__ kb,
-                      const uint16_t* __restrict__ vb, const uint16_t* __restrict__ dout,
-                      const float* __restrict__ lse, const float* __restrict__ delta,
-                      const void* __restrict__ dq_part, float scale, float* __restrict__ dq,
-                      float* __restrict__ dkb, float* __restrict__ dvb, int stage_rows, const MergeDest dest) {
+constexpr int kRoleThreads = kMergeThreads / 2;
+constexpr int kRoleRows = kRoleThreads / 4;   // rows of one pass (a quad per row in the stream role)
+constexpr int kBarStream = 1, kBarBlock = 2, kBarFull = 3, kBarEmpty = 5;   // full / empty: + slot
+
+// Shared memory of the reduce kernel (byte offsets, 16-byte aligned):
+//   slot   [2][32][D] fp32    in-block dq of a pass, block role -> stream role
+//   kb, vb [bs][D] bf16       the block's keys and values
+//   p, ds  [rows][bs] fp32 (FMA path) or [rows][bs + 8] bf16 (tensor path)
+//   e      [kEStage] int      entry ids (stream role)
+//   qr, dr [rows][D] bf16     the rows' q and dout (tensor path; FMA path when stage_rows)
+// rows = G * bs ordered (token, head).  On the tensor path the kb, vb, qr, dr tiles are
+// 16-byte-chunk swizzled (swz) for conflict-free ldmatrix.
+struct ReduceSmem {
+  size_t slot, kb, vb, p, ds, e, qr, dr, total;
+};
+__host__ __device__ inline size_t al16(size_t x) { return (x + 15) & ~size_t(15); }
+__host__ __device__ inline ReduceSmem reduce_smem(int D, int bs, int R, bool tc, bool stage_rows) {
+  ReduceSmem L;
+  size_t o = 0;
+  L.slot = o;
+  o += al16(size_t(2) * kRoleRows * D * 4);
+  L.kb = o;
+  o += al16(size_t(bs) * D * 2);
+  L.vb = o;
+  o += al16(size_t(bs) * D * 2);
+  const size_t pds = tc ? size_t(R) * (bs + 8) * 2 : size_t(R) * bs * 4;
+  L.p = o;
+  o += al16(pds);
+  L.ds = o;
+  o += al16(pds);
+  L.e = o;
+  o += al16(size_t(kEStage) * 4);
+  const size_t rows = (tc || stage_rows) ? size_t(R) * D * 2 : 0;
+  L.qr = o;
+  o += al16(rows);
+  L.dr = o;
+  o += al16(rows);
+  L.total = o;
+  return L;
+}
+
+// float4 granule gi of row rl in a [32][D] fp32 slot; rows rl and rl ^ 1 use opposite
+// halves of the banks for the same granule, so a quad's 16-byte accesses from two rows
+// (one 128-byte wavefront) never share a bank.
+template <int D>
+__device__ __forceinline__ int slot_off(int rl, int gi) {
+  return rl * D + 4 * (gi ^ ((rl & 1) << 2));
+}
+
+struct BlockIO {   // global operands of the block role
+  const uint16_t* q;
+  const uint16_t* kb;
+  const uint16_t* vb;
+  const uint16_t* dout;
+  const float* lse;
+  const float* delta;
+  float scale;
+  float* dkb;
+  float* dvb;
+};
+
+template <int kSlot>
+__device__ __forceinline__ void slot_handoff_wait(int j) {   // block role: slot kSlot free again
+  if (j >= 2) named_sync<kBarEmpty + kSlot>(kMergeThreads);
+}
+
+// Block role on the FMA pipes (any rows / block keys): a quad per row for P, dS and
+// the in-block dq; a warp per pair of block keys for dkb, dvb.
+template <int D>
+__device__ __forceinline__ void block_role_fma(const DevPlan& p, int b, int g, const BlockIO& io, int stage_rows,
+                                               float* sSlot, uint16_t* sKb, uint16_t* sVb, float* sP, float* sdS,
+                                               uint16_t* sQr, uint16_t* sDr) {
   constexpr int NG = D / 16;
-  using RecT = Rec<kBf16Rec>;
-  constexpr int EG = 64 / (NG * RecT::RW);   // entries whose partials are in flight together
   constexpr int DPL = D / 32;
-  extern __shared__ __align__(16) uint8_t smem_raw[];
-  const int bs = p.bs;
-  const int R = p.G * bs;
-  uint16_t* sKb = reinterpret_cast<uint16_t*>(smem_raw);
-  uint16_t* sVb = sKb + bs * D;
-  float* sP = reinterpret_cast<float*>(sVb + bs * D);    // [rows][bs]
-  float* sdS = sP + R * bs;                               // [rows][bs]
-  int* sE = reinterpret_cast<int*>(sdS + R * bs);         // [kEStage]
-  uint16_t* sQr = reinterpret_cast<uint16_t*>(sE + kEStage);   // [rows][D] when stage_rows
-  uint16_t* sDr = sQr + R * D;
-  const int b = blockIdx.x, g = blockIdx.y;
-  const int tid = threadIdx.x, u = tid & 3, warp = tid >> 5, lane = tid & 31;
-  const int nwarps = blockDim.x >> 5;
-  const bool bterm = p.block_term && b >= p.bt_lo && b < p.bt_hi;   // in-block term of this block here
-  for (int idx = tid; bterm && idx < bs * (D / 8); idx += blockDim.x) {
+  const int bs = p.bs, R = p.G * bs;
+  const int gt = threadIdx.x - kRoleThreads, u = gt & 3, rl = gt >> 2, bwarp = gt >> 5, lane = threadIdx.x & 31;
+  for (int idx = gt; idx < bs * (D / 8); idx += kRoleThreads) {
     const int t = idx / (D / 8), ch = idx % (D / 8);
     const size_t src = (size_t(b * bs + t) * p.Hkv + g) * D + ch * 8;
-    *reinterpret_cast<uint4*>(sKb + t * D + ch * 8) = *reinterpret_cast<const uint4*>(kb + src);
-    *reinterpret_cast<uint4*>(sVb + t * D + ch * 8) = *reinterpret_cast<const uint4*>(vb + src);
+    *reinterpret_cast<uint4*>(sKb + t * D + ch * 8) = *reinterpret_cast<const uint4*>(io.kb + src);
+    *reinterpret_cast<uint4*>(sVb + t * D + ch * 8) = *reinterpret_cast<const uint4*>(io.vb + src);
   }
-  const int n_block_keys = bterm ? bs : 0;   // none when they are context keys, or on another rank
-  // dq rows: the plan's own dq, or the owner's receive buffer (see MergeDest; dest.o)
-  float* dq_out = dq;
-  size_t dq_base = size_t(b) * bs;
-  bool dq_ok = true;
-  if (dest.o != nullptr) dq_out = dest.o[dest_of_block(p, dest, b, dq_base, dq_ok)];
-  const float scale_log2 = scale * kLog2e;
-  const int e0 = p.block_entry_ptr[b], n = p.block_entry_ptr[b + 1] - e0;
-  // phase 1, a quad per row: P, dS of the in-block keys; dq = in-block dq + sum of partials
-  for (int r0 = 0; r0 < R; r0 += kRowsPerPass) {
-    const int r = min(r0 + (tid >> 2), R - 1);          // rows past R compute, never store
-    const bool active = r0 + (tid >> 2) < R;
+  named_sync<kBarBlock>(kRoleThreads);
+  const float scale_log2 = io.scale * kLog2e;
+  const int npass = (R + kRoleRows - 1) / kRoleRows;
+  for (int j = 0; j < npass; ++j) {
+    const int r = min(j * kRoleRows + rl, R - 1);
+    const bool active = j * kRoleRows + rl < R;
     const int tt = r / p.G, hh = r - tt * p.G;
-    const int head = g * p.G + hh;
-    const size_t qrow = size_t(b * bs + tt) * p.Hq + head;
-    stage_entries(sE, p.block_entries + e0, 0, min(n, kEStage));
+    const size_t qrow = size_t(b * bs + tt) * p.Hq + g * p.G + hh;
     float acc[NG][4];
     {
       float qv[NG][4], dov[NG][4];
-      load_bf16_quad<NG>(q + qrow * D, u, qv);
-      load_bf16_quad<NG>(dout + qrow * D, u, dov);
-      const float l2 = lse[qrow] * kLog2e;
-      const float dl = delta[qrow];
+      load_bf16_quad<NG>(io.q + qrow * D, u, qv);
+      load_bf16_quad<NG>(io.dout + qrow * D, u, dov);
+      const float l2 = io.lse[qrow] * kLog2e;
+      const float dl = io.delta[qrow];
 #pragma unroll
       for (int k = 0; k < NG; ++k)
 #pragma unroll
         for (int i = 0; i < 4; ++i) acc[k][i] = 0.f;
-      for (int key = 0; key < n_block_keys; ++key) {
-        float sd = 0.f, dp = 0.f;
+#pragma unroll 1
+      for (int key = 0; key < bs; ++key) {
+        // four partial sums per dot product: dependent chains of NG, not 4 * NG, FMAs
+        float sd4[4] = {0.f, 0.f, 0.f, 0.f}, dp4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
         for (int k = 0; k < NG; ++k) {
           float kv[1][4], vv[1][4];
@@ -407,12 +462,12 @@ __global__ void __launch_bounds__(kMergeThreads, 2)
           load_bf16_quad<1>(sVb + key * D + 16 * k, u, vv);
 #pragma unroll
           for (int i = 0; i < 4; ++i) {
-            sd = fmaf(qv[k][i], kv[0][i], sd);
-            dp = fmaf(dov[k][i], vv[0][i], dp);
+            sd4[i] = fmaf(qv[k][i], kv[0][i], sd4[i]);
+            dp4[i] = fmaf(dov[k][i], vv[0][i], dp4[i]);
           }
         }
-        sd = quad_sum(sd);
-        dp = quad_sum(dp);
+        const float sd = quad_sum((sd4[0] + sd4[1]) + (sd4[2] + sd4[3]));
+        const float dp = quad_sum((dp4[0] + dp4[1]) + (dp4[2] + dp4[3]));
         const float pr = (l2 == -INFINITY) ? 0.f : fast_exp2(sd * scale_log2 - l2);
         const float ds = pr * (dp - dl);
         if (active && u == 0) {
@@ -427,58 +482,36 @@ __global__ void __launch_bounds__(kMergeThreads, 2)
           for (int i = 0; i < 4; ++i) acc[k][i] = fmaf(ds, kv[0][i], acc[k][i]);
         }
       }
-      if (stage_rows && active && bterm) {   // keep q and dout of this row for the dkb / dvb pass
+      if (stage_rows && active) {   // keep q and dout of this row for the dkb / dvb pass
 #pragma unroll
         for (int k = 0; k < NG; ++k) {
           const int off = r * D + 4 * (u + 4 * k);
-          *reinterpret_cast<uint2*>(sQr + off) = *reinterpret_cast<const uint2*>(q + qrow * D + 4 * (u + 4 * k));
-          *reinterpret_cast<uint2*>(sDr + off) = *reinterpret_cast<const uint2*>(dout + qrow * D + 4 * (u + 4 * k));
+          *reinterpret_cast<uint2*>(sQr + off) = *reinterpret_cast<const uint2*>(io.q + qrow * D + 4 * (u + 4 * k));
+          *reinterpret_cast<uint2*>(sDr + off) =
+              *reinterpret_cast<const uint2*>(io.dout + qrow * D + 4 * (u + 4 * k));
         }
       }
     }
-    // the in-block term, then the chunk partials in ascending chunk order, EG in flight
-    float4 tot[NG];
+    const int sl = j & 1;
+    sl ? slot_handoff_wait<1>(j) : slot_handoff_wait<0>(j);
+    float* slot = sSlot + sl * kRoleRows * D;
 #pragma unroll
     for (int k = 0; k < NG; ++k)
-      tot[k] = make_float4(scale * acc[k][0], scale * acc[k][1], scale * acc[k][2], scale * acc[k][3]);
-    for (int c0 = 0; c0 < n; c0 += kEStage) {
-      const int cnt = min(kEStage, n - c0);
-      if (c0 > 0) stage_entries(sE, p.block_entries + e0, c0, cnt);
-      for (int i0 = 0; i0 < cnt; i0 += EG) {
-        uint32_t pv[EG][NG][RecT::RW];
-#pragma unroll
-        for (int v = 0; v < EG; ++v) {
-          if (i0 + v < cnt) {
-            const size_t rec = size_t(sE[i0 + v] * bs + tt) * p.Hq + head;
-            RecT::template load<NG>(dq_part, rec * D, u, pv[v]);
-          } else {
-            RecT::template zero<NG>(pv[v]);
-          }
-        }
-#pragma unroll
-        for (int v = 0; v < EG; ++v)
-#pragma unroll
-          for (int k = 0; k < NG; ++k) {
-            const float4 x = RecT::get(pv[v][k]);
-            tot[k].x += x.x;
-            tot[k].y += x.y;
-            tot[k].z += x.z;
-            tot[k].w += x.w;
-          }
-      }
-    }
-    if (active && dq_ok) {
-      float* dst = dq_out + ((dq_base + tt) * p.Hq + head) * D;   // = dq + qrow * D for the plan's own dq
-#pragma unroll
-      for (int k = 0; k < NG; ++k) *reinterpret_cast<float4*>(dst + 4 * (u + 4 * k)) = tot[k];
-    }
+      *reinterpret_cast<float4*>(slot + slot_off<D>(rl, u + 4 * k)) =
+          make_float4(io.scale * acc[k][0], io.scale * acc[k][1], io.scale * acc[k][2], io.scale * acc[k][3]);
+    sl ? named_arrive<kBarFull + 1>(kMergeThreads) : named_arrive<kBarFull>(kMergeThreads);
   }
-  __syncthreads();
-  // phase 2, one warp per block key: dkb = scale * sum_r dS[r] q_r, dvb = sum_r P[r] dout_r
-  for (int key = warp; key < n_block_keys; key += nwarps) {
-    float ak[DPL], av[DPL];
+  named_sync<kBarBlock>(kRoleThreads);   // P, dS (and the staged rows) of every row written
+  // a warp per pair of block keys (k0, k0 + 1), sharing each row's loads:
+  // dkb = scale * sum_r dS[r] q_r, dvb = sum_r P[r] dout_r
+  for (int k0 = 2 * bwarp; k0 < bs; k0 += 2 * (kRoleThreads / 32)) {
+    const int nk = min(2, bs - k0);
+    float ak[2][DPL], av[2][DPL];
 #pragma unroll
-    for (int i = 0; i < DPL; ++i) ak[i] = av[i] = 0.f;
+    for (int x = 0; x < 2; ++x)
+#pragma unroll
+      for (int i = 0; i < DPL; ++i) ak[x][i] = av[x][i] = 0.f;
+#pragma unroll 4
     for (int r = 0; r < R; ++r) {
       float qv[DPL], dov[DPL];
       if (stage_rows) {
@@ -487,27 +520,302 @@ __global__ void __launch_bounds__(kMergeThreads, 2)
       } else {
         const int tt = r / p.G, hh = r - tt * p.G;
         const size_t qrow = size_t(b * bs + tt) * p.Hq + g * p.G + hh;
-        load_bf16_row<DPL>(q + qrow * D + lane * DPL, qv);
-        load_bf16_row<DPL>(dout + qrow * D + lane * DPL, dov);
+        load_bf16_row<DPL>(io.q + qrow * D + lane * DPL, qv);
+        load_bf16_row<DPL>(io.dout + qrow * D + lane * DPL, dov);
       }
-      const float ds = sdS[r * bs + key], pr = sP[r * bs + key];
+      const int k1 = k0 + nk - 1;   // = k0 when the pair is a single key
+      const float ds0 = sdS[r * bs + k0], pr0 = sP[r * bs + k0];
+      const float ds1 = sdS[r * bs + k1], pr1 = sP[r * bs + k1];
 #pragma unroll
       for (int i = 0; i < DPL; ++i) {
-        ak[i] = fmaf(ds, qv[i], ak[i]);
-        av[i] = fmaf(pr, dov[i], av[i]);
+        ak[0][i] = fmaf(ds0, qv[i], ak[0][i]);
+        av[0][i] = fmaf(pr0, dov[i], av[0][i]);
+        ak[1][i] = fmaf(ds1, qv[i], ak[1][i]);
+        av[1][i] = fmaf(pr1, dov[i], av[1][i]);
       }
     }
-    const size_t krow = size_t(b * bs + key) * p.Hkv + g;
-    float* dk_dst = dkb + krow * D + lane * DPL;
-    float* dv_dst = dvb + krow * D + lane * DPL;
-    if constexpr (DPL == 4) {
-      *reinterpret_cast<float4*>(dk_dst) = make_float4(scale * ak[0], scale * ak[1], scale * ak[2], scale * ak[3]);
-      *reinterpret_cast<float4*>(dv_dst) = make_float4(av[0], av[1], av[2], av[3]);
-    } else {
-      *reinterpret_cast<float2*>(dk_dst) = make_float2(scale * ak[0], scale * ak[1]);
-      *reinterpret_cast<float2*>(dv_dst) = make_float2(av[0], av[1]);
+    for (int x = 0; x < nk; ++x) {
+      const size_t krow = size_t(b * bs + k0 + x) * p.Hkv + g;
+      float* dk_dst = io.dkb + krow * D + lane * DPL;
+      float* dv_dst = io.dvb + krow * D + lane * DPL;
+      if constexpr (DPL == 4) {
+        *reinterpret_cast<float4*>(dk_dst) =
+            make_float4(io.scale * ak[x][0], io.scale * ak[x][1], io.scale * ak[x][2], io.scale * ak[x][3]);
+        *reinterpret_cast<float4*>(dv_dst) = make_float4(av[x][0], av[x][1], av[x][2], av[x][3]);
+      } else {
+        *reinterpret_cast<float2*>(dk_dst) = make_float2(io.scale * ak[x][0], io.scale * ak[x][1]);
+        *reinterpret_cast<float2*>(dv_dst) = make_float2(av[x][0], av[x][1]);
+      }
     }
   }
+}
+
+// Block role on the tensor cores (rows R and block keys bs multiples of 16).  Pass j
+// (rows 32j..32j+31) gives warp w the 16-row tile 2j + (w & 1) and half w >> 1 of the
+// head dim: S = Q K^T and dP = dO V^T over the block keys, 16 at a time (the two warps
+// of a tile compute them both), P and dS in registers, the warp's half of the in-block
+// dq += dS K.  Then dkb = scale dS^T Q and dvb = P^T dO, contracting over the rows,
+// in items of (product, 16 keys, 32 columns).  Fragment layouts of m16n8k16: element
+// e of an accumulator n-tile is row gq + 8 (e >> 1), column 2 tq + (e & 1).
+template <int D>
+__device__ __forceinline__ void block_role_tc(const DevPlan& p, int b, int g, const BlockIO& io, float* sSlot,
+                                              uint16_t* sKb, uint16_t* sVb, uint16_t* sPb, uint16_t* sdSb,
+                                              uint16_t* sQr, uint16_t* sDr) {
+  constexpr int kNH = D / 16;   // 8-column n-tiles in half the head dim
+  const int bs = p.bs, R = p.G * bs, SB = bs + 8;
+  const int gt = threadIdx.x - kRoleThreads, w = gt >> 5, lane = threadIdx.x & 31;
+  const int gq = lane >> 2, tq = lane & 3;
+  for (int idx = gt; idx < bs * (D / 8); idx += kRoleThreads) {
+    const int t = idx / (D / 8), ch = idx % (D / 8);
+    const size_t src = (size_t(b * bs + t) * p.Hkv + g) * D + ch * 8;
+    *reinterpret_cast<uint4*>(sKb + swz<D>(t, ch)) = *reinterpret_cast<const uint4*>(io.kb + src);
+    *reinterpret_cast<uint4*>(sVb + swz<D>(t, ch)) = *reinterpret_cast<const uint4*>(io.vb + src);
+  }
+  for (int idx = gt; idx < R * (D / 8); idx += kRoleThreads) {
+    const int r = idx / (D / 8), ch = idx % (D / 8);
+    const int tt = r / p.G, hh = r - tt * p.G;
+    const size_t src = (size_t(b * bs + tt) * p.Hq + g * p.G + hh) * D + ch * 8;
+    *reinterpret_cast<uint4*>(sQr + swz<D>(r, ch)) = *reinterpret_cast<const uint4*>(io.q + src);
+    *reinterpret_cast<uint4*>(sDr + swz<D>(r, ch)) = *reinterpret_cast<const uint4*>(io.dout + src);
+  }
+  named_sync<kBarBlock>(kRoleThreads);
+  const float scale_log2 = io.scale * kLog2e;
+  const int npass = (R + kRoleRows - 1) / kRoleRows;
+  const int nmt = R / 16;
+  const int dh = w >> 1;
+  for (int j = 0; j < npass; ++j) {
+    const int mt = 2 * j + (w & 1);
+    float dqa[kNH][4];
+#pragma unroll
+    for (int nn = 0; nn < kNH; ++nn)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) dqa[nn][e] = 0.f;
+    if (mt < nmt) {
+      const int r0 = mt * 16;
+      float l2[2], dl[2];   // statistics of the thread's rows r0 + gq, r0 + gq + 8
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int r = r0 + gq + 8 * h, tt = r / p.G, hh = r - tt * p.G;
+        const size_t qrow = size_t(b * bs + tt) * p.Hq + g * p.G + hh;
+        l2[h] = io.lse[qrow] * kLog2e;
+        dl[h] = io.delta[qrow];
+      }
+      for (int kc = 0; kc < bs; kc += 16) {
+        float s[2][4], dp[2][4];
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) s[nt][e] = dp[nt][e] = 0.f;
+#pragma unroll
+        for (int ks = 0; ks < D / 16; ++ks) {
+          uint32_t qa[4], da[4], kf[4], vf[4];
+          const int ar = r0 + (lane & 15), ach = 2 * ks + (lane >> 4);
+          ldsm_x4(qa[0], qa[1], qa[2], qa[3], sQr + swz<D>(ar, ach));
+          ldsm_x4(da[0], da[1], da[2], da[3], sDr + swz<D>(ar, ach));
+          const int br = kc + (lane & 7) + ((lane >> 4) << 3), bch = 2 * ks + ((lane >> 3) & 1);
+          ldsm_x4(kf[0], kf[1], kf[2], kf[3], sKb + swz<D>(br, bch));
+          ldsm_x4(vf[0], vf[1], vf[2], vf[3], sVb + swz<D>(br, bch));
+          mma_bf16_16816(s[0], qa, kf[0], kf[1]);
+          mma_bf16_16816(s[1], qa, kf[2], kf[3]);
+          mma_bf16_16816(dp[0], da, vf[0], vf[1]);
+          mma_bf16_16816(dp[1], da, vf[2], vf[3]);
+        }
+        // P = exp2(s c - lse2), dS = P (dP - Delta), packed as the A operand of dS K:
+        // word 2 nt + h holds row gq + 8h, keys kc + 8 nt + 2 tq and + 1
+        uint32_t pa[4], sa[4];
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            float pr[2], ds[2];
+#pragma unroll
+            for (int c = 0; c < 2; ++c) {
+              pr[c] = (l2[h] == -INFINITY) ? 0.f : fast_exp2(s[nt][2 * h + c] * scale_log2 - l2[h]);
+              ds[c] = pr[c] * (dp[nt][2 * h + c] - dl[h]);
+            }
+            pa[2 * nt + h] = pack_bf16(pr[0], pr[1]);
+            sa[2 * nt + h] = pack_bf16(ds[0], ds[1]);
+          }
+        if (dh == 0) {   // P, dS of the tile for dvb, dkb (one of the tile's two warps)
+#pragma unroll
+          for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              const int off = (r0 + gq + 8 * h) * SB + kc + 8 * nt + 2 * tq;
+              *reinterpret_cast<uint32_t*>(sPb + off) = pa[2 * nt + h];
+              *reinterpret_cast<uint32_t*>(sdSb + off) = sa[2 * nt + h];
+            }
+        }
+#pragma unroll
+        for (int nn = 0; nn < kNH; nn += 2) {   // in-block dq (the warp's columns) += dS K
+          const int kr = kc + (lane & 7) + 8 * ((lane >> 3) & 1);
+          const int ch = dh * (D / 16) + nn + (lane >> 4);
+          uint32_t b0, b1, b2, b3;
+          ldsm_x4_t(b0, b1, b2, b3, sKb + swz<D>(kr, ch));
+          mma_bf16_16816(dqa[nn], sa, b0, b1);
+          mma_bf16_16816(dqa[nn + 1], sa, b2, b3);
+        }
+      }
+    }
+    const int sl = j & 1;
+    sl ? slot_handoff_wait<1>(j) : slot_handoff_wait<0>(j);
+    if (mt < nmt) {
+      float* slot = sSlot + sl * kRoleRows * D;
+#pragma unroll
+      for (int nn = 0; nn < kNH; ++nn)
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const int rl = (w & 1) * 16 + gq + 8 * h;
+          const int col = dh * (D / 2) + nn * 8 + 2 * tq;
+          *reinterpret_cast<float2*>(slot + slot_off<D>(rl, col >> 2) + (col & 3)) =
+              make_float2(io.scale * dqa[nn][2 * h], io.scale * dqa[nn][2 * h + 1]);
+        }
+    }
+    sl ? named_arrive<kBarFull + 1>(kMergeThreads) : named_arrive<kBarFull>(kMergeThreads);
+  }
+  named_sync<kBarBlock>(kRoleThreads);   // P, dS of every row in shared memory
+  const int nitems = 2 * (bs / 16) * (D / 32);
+  for (int it = w; it < nitems; it += kRoleThreads / 32) {
+    const int prod = it & 1, rest = it >> 1, km = rest / (D / 32), ng = rest % (D / 32);
+    const uint16_t* sA = prod ? sPb : sdSb;   // A = P^T or dS^T (keys x rows), stored [rows][keys]
+    const uint16_t* sB = prod ? sDr : sQr;    // B = dout or q (rows x columns)
+    float acc[4][4];
+#pragma unroll
+    for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) acc[nt][e] = 0.f;
+    for (int kr0 = 0; kr0 < R; kr0 += 16) {
+      uint32_t a[4];
+      const int mi = lane >> 3;
+      ldsm_x4_t(a[0], a[1], a[2], a[3], sA + (kr0 + (lane & 7) + (mi >> 1) * 8) * SB + km * 16 + (mi & 1) * 8);
+#pragma unroll
+      for (int np = 0; np < 2; ++np) {
+        const int br = kr0 + (lane & 7) + 8 * ((lane >> 3) & 1);
+        const int ch = ng * 4 + np * 2 + (lane >> 4);
+        uint32_t b0, b1, b2, b3;
+        ldsm_x4_t(b0, b1, b2, b3, sB + swz<D>(br, ch));
+        mma_bf16_16816(acc[2 * np], a, b0, b1);
+        mma_bf16_16816(acc[2 * np + 1], a, b2, b3);
+      }
+    }
+    float* dst = prod ? io.dvb : io.dkb;
+    const float f = prod ? 1.f : io.scale;
+#pragma unroll
+    for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int key = km * 16 + gq + 8 * h;
+        const int col = ng * 32 + nt * 8 + 2 * tq;
+        *reinterpret_cast<float2*>(dst + (size_t(b * bs + key) * p.Hkv + g) * D + col) =
+            make_float2(f * acc[nt][2 * h], f * acc[nt][2 * h + 1]);
+      }
+  }
+}
+
+template <int D, bool kBf16Rec, bool kTC>
+__global__ void __launch_bounds__(kMergeThreads, 2)
+    bwd_reduce_kernel(DevPlan p, const uint16_t* __restrict__ q, const uint16_t* __restrict__ kb,
+                      const uint16_t* __restrict__ vb, const uint16_t* __restrict__ dout,
+                      const float* __restrict__ lse, const float* __restrict__ delta,
+                      const void* __restrict__ dq_part, float scale, float* __restrict__ dq,
+                      float* __restrict__ dkb, float* __restrict__ dvb, int stage_rows, const MergeDest dest) {
+  constexpr int NG = D / 16;
+  using RecT = Rec<kBf16Rec>;
+  constexpr int EG = 64 / (NG * RecT::RW);   // entries whose partials are in flight together
+  extern __shared__ __align__(16) uint8_t smem_raw[];
+  const int bs = p.bs;
+  const int R = p.G * bs;
+  const ReduceSmem L = reduce_smem(D, bs, R, kTC, stage_rows != 0);
+  float* sSlot = reinterpret_cast<float*>(smem_raw + L.slot);
+  int* sE = reinterpret_cast<int*>(smem_raw + L.e);
+  const int b = blockIdx.x, g = blockIdx.y;
+  const int tid = threadIdx.x;
+  const bool bterm = p.block_term && b >= p.bt_lo && b < p.bt_hi;   // in-block term of this block here
+  const int npass = (R + kRoleRows - 1) / kRoleRows;
+
+  if (tid < kRoleThreads) {
+    // ---- stream role ----
+    const int gt = tid, u = gt & 3, rl = gt >> 2;
+    const int e0 = p.block_entry_ptr[b], n = p.block_entry_ptr[b + 1] - e0;
+    // dq rows: the plan's own dq, or the owner's receive buffer (see MergeDest; dest.o)
+    float* dq_out = dq;
+    size_t dq_base = size_t(b) * bs;
+    bool dq_ok = true;
+    if (dest.o != nullptr) dq_out = dest.o[dest_of_block(p, dest, b, dq_base, dq_ok)];
+    for (int j = 0; j < npass; ++j) {
+      const int r = min(j * kRoleRows + rl, R - 1);        // rows past R compute, never store
+      const bool active = j * kRoleRows + rl < R;
+      const int tt = r / p.G, hh = r - tt * p.G;
+      const int head = g * p.G + hh;
+      float4 tot[NG];
+#pragma unroll
+      for (int k = 0; k < NG; ++k) tot[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int c0 = 0; c0 < n; c0 += kEStage) {
+        const int cnt = min(kEStage, n - c0);
+        if (j == 0 || n > kEStage) {   // entry ids staged once when they fit
+          named_sync<kBarStream>(kRoleThreads);
+          for (int i = gt; i < cnt; i += kRoleThreads) sE[i] = p.block_entries[e0 + c0 + i];
+          named_sync<kBarStream>(kRoleThreads);
+        }
+        for (int i0 = 0; i0 < cnt; i0 += EG) {
+          uint32_t pv[EG][NG][RecT::RW];
+#pragma unroll
+          for (int v = 0; v < EG; ++v) {
+            if (i0 + v < cnt) {
+              const size_t rec = size_t(sE[i0 + v] * bs + tt) * p.Hq + head;
+              RecT::template load<NG>(dq_part, rec * D, u, pv[v]);
+            } else {
+              RecT::template zero<NG>(pv[v]);
+            }
+          }
+#pragma unroll
+          for (int v = 0; v < EG; ++v)
+#pragma unroll
+            for (int k = 0; k < NG; ++k) {
+              const float4 x = RecT::get(pv[v][k]);
+              tot[k].x += x.x;
+              tot[k].y += x.y;
+              tot[k].z += x.z;
+              tot[k].w += x.w;
+            }
+        }
+      }
+      if (bterm) {   // + the rows' in-block dq
+        const int sl = j & 1;
+        sl ? named_sync<kBarFull + 1>(kMergeThreads) : named_sync<kBarFull>(kMergeThreads);
+        const float* slot = sSlot + sl * kRoleRows * D;
+#pragma unroll
+        for (int k = 0; k < NG; ++k) {
+          const float4 x = *reinterpret_cast<const float4*>(slot + slot_off<D>(rl, u + 4 * k));
+          tot[k].x += x.x;
+          tot[k].y += x.y;
+          tot[k].z += x.z;
+          tot[k].w += x.w;
+        }
+        if (j + 2 < npass) sl ? named_arrive<kBarEmpty + 1>(kMergeThreads) : named_arrive<kBarEmpty>(kMergeThreads);
+      }
+      if (active && dq_ok) {
+        float* dst = dq_out + ((dq_base + tt) * p.Hq + head) * D;   // = dq + qrow * D for the plan's own dq
+#pragma unroll
+        for (int k = 0; k < NG; ++k) *reinterpret_cast<float4*>(dst + 4 * (u + 4 * k)) = tot[k];
+      }
+    }
+    return;
+  }
+
+  // ---- block role ----
+  if (!bterm) return;   // its keys are context keys, or the term is computed on another rank
+  const BlockIO io{q, kb, vb, dout, lse, delta, scale, dkb, dvb};
+  uint16_t* sKb = reinterpret_cast<uint16_t*>(smem_raw + L.kb);
+  uint16_t* sVb = reinterpret_cast<uint16_t*>(smem_raw + L.vb);
+  uint16_t* sQr = reinterpret_cast<uint16_t*>(smem_raw + L.qr);
+  uint16_t* sDr = reinterpret_cast<uint16_t*>(smem_raw + L.dr);
+  if constexpr (kTC)
+    block_role_tc<D>(p, b, g, io, sSlot, sKb, sVb, reinterpret_cast<uint16_t*>(smem_raw + L.p),
+                     reinterpret_cast<uint16_t*>(smem_raw + L.ds), sQr, sDr);
+  else
+    block_role_fma<D>(p, b, g, io, stage_rows, sSlot, sKb, sVb, reinterpret_cast<float*>(smem_raw + L.p),
+                      reinterpret_cast<float*>(smem_raw + L.ds), sQr, sDr);
 }
 
 template <int D, bool kBf16Rec>
@@ -523,22 +831,35 @@ cudaError_t merge_d(const DevPlan& p, const uint16_t* q, const uint16_t* kb, con
   return cudaGetLastError();
 }
 
+template <int D, bool kBf16Rec, bool kTC>
+cudaError_t reduce_launch(const DevPlan& p, const uint16_t* q, const uint16_t* kb, const uint16_t* vb,
+                          const uint16_t* dout, const float* lse, const float* delta, const void* dq_part,
+                          float scale, float* dq, float* dkb, float* dvb, cudaStream_t s, const MergeDest& dest,
+                          int stage_rows, size_t smem) {
+  cudaError_t e = cudaFuncSetAttribute(bwd_reduce_kernel<D, kBf16Rec, kTC>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+  if (e != cudaSuccess) return e;
+  bwd_reduce_kernel<D, kBf16Rec, kTC><<<dim3(p.A, p.Hkv), kMergeThreads, smem, s>>>(
+      p, q, kb, vb, dout, lse, delta, dq_part, scale, dq, dkb, dvb, stage_rows, dest);
+  return cudaGetLastError();
+}
+
 template <int D, bool kBf16Rec>
 cudaError_t reduce_d(const DevPlan& p, const uint16_t* q, const uint16_t* kb, const uint16_t* vb,
                      const uint16_t* dout, const float* lse, const float* delta, const void* dq_part,
                      float scale, float* dq, float* dkb, float* dvb, cudaStream_t s, const MergeDest& dest) {
-  const size_t rows = size_t(p.G) * p.bs;
-  const size_t base =
-      size_t(2) * p.bs * D * sizeof(uint16_t) + 2 * rows * p.bs * sizeof(float) + kEStage * sizeof(int);
-  const size_t staged = base + 2 * rows * D * sizeof(uint16_t);
-  const int stage_rows = staged <= size_t(64) * 1024 ? 1 : 0;   // small enough to keep occupancy
-  const size_t smem = stage_rows ? staged : base;
-  cudaError_t e = cudaFuncSetAttribute(bwd_reduce_kernel<D, kBf16Rec>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       int(smem));
-  if (e != cudaSuccess) return e;
-  bwd_reduce_kernel<D, kBf16Rec><<<dim3(p.A, p.Hkv), kMergeThreads, smem, s>>>(
-      p, q, kb, vb, dout, lse, delta, dq_part, scale, dq, dkb, dvb, stage_rows, dest);
-  return cudaGetLastError();
+  const int R = p.G * p.bs;
+  constexpr size_t kMaxSmem = size_t(227) * 1024;
+  // tensor path: rows and block keys in 16s, and its tiles fit in shared memory
+  const size_t tc_smem = reduce_smem(D, p.bs, R, true, true).total;
+  if (R % 16 == 0 && p.bs % 16 == 0 && tc_smem <= kMaxSmem)
+    return reduce_launch<D, kBf16Rec, true>(p, q, kb, vb, dout, lse, delta, dq_part, scale, dq, dkb, dvb, s, dest,
+                                            1, tc_smem);
+  const size_t staged = reduce_smem(D, p.bs, R, false, true).total;
+  const int stage_rows = staged <= size_t(110) * 1024 ? 1 : 0;   // small enough for two CTAs per SM
+  const size_t smem = reduce_smem(D, p.bs, R, false, stage_rows != 0).total;
+  return reduce_launch<D, kBf16Rec, false>(p, q, kb, vb, dout, lse, delta, dq_part, scale, dq, dkb, dvb, s, dest,
+                                           stage_rows, smem);
 }
 
 }  // namespace

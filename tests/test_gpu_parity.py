@@ -55,6 +55,10 @@ SMALL_CASES = {
     "g1_bs8_d128": dict(Hq=2, Hkv=2, d=128, bs=8, anchors=40),
     # tcgen05 path with a whole 128-row tile per block (G = 8)
     "gqa8_d128": dict(Hq=8, Hkv=1, d=128),
+    # in-block term on the tensor cores: 64 block keys (four 16-key steps), 128 rows
+    "bs64_g2_d128": dict(Hq=4, Hkv=2, d=128, bs=64, anchors=8),
+    # 32 block keys, 32 rows (one pass of the reduce kernel)
+    "bs32_g1_d128": dict(Hq=2, Hkv=2, d=128, bs=32, anchors=12),
 }
 
 

@@ -533,6 +533,71 @@ class DQ(Core):
 
 
 # ---------------------------------------------------------------------------
+# dq reduce kernel: the block role computes the in-block dq of 32 rows at a time into one
+# of two shared-memory slots and arrives on the slot's "full" named barrier; the stream
+# role sums the rows' chunk partials, syncs on "full", adds the slot, and arrives on the
+# slot's "empty" barrier when the block role will write that slot again (pass j + 2);
+# the block role syncs on "empty" before its third and later passes.  A named barrier
+# (bar.sync / bar.arrive with a count of both roles' threads) completes a phase at every
+# second group arrival, whoever makes it.
+# ---------------------------------------------------------------------------
+class NamedBar:
+    def __init__(self):
+        self.arr, self.phase = 0, 0
+
+    def arrive(self):
+        ph = self.phase
+        self.arr += 1
+        if self.arr == 2:
+            self.arr = 0
+            self.phase += 1
+        return ph
+
+
+class Reduce(Core):
+    def __init__(self, npass, seed, drop=None):
+        super().__init__(seed, [])
+        self.npass, self.drop = npass, drop
+        self.N = {f"{k}{s}": NamedBar() for k in ("full", "empty") for s in (0, 1)}
+        self.slot = [None, None]   # pass whose in-block dq the slot holds (None: consumed)
+
+    def sync(self, name):
+        ph = self.N[name].arrive()
+        while self.N[name].phase <= ph:
+            yield
+
+    def stream(self):
+        for j in range(self.npass):
+            for _ in range(self.rng.randint(1, 4)):   # the chunk partials of the rows
+                yield
+            sl = j & 1
+            yield from self.sync(f"full{sl}")
+            self.check(self.slot[sl] == j, f"stream pass {j} read slot {sl} holding {self.slot[sl]}")
+            self.slot[sl] = None
+            if j + 2 < self.npass:
+                self.N[f"empty{sl}"].arrive()
+            yield
+
+    def block(self):
+        for j in range(self.npass):
+            for _ in range(self.rng.randint(1, 3)):   # P, dS and the in-block dq of the rows
+                yield
+            sl = j & 1
+            if j >= 2 and self.drop != "empty":
+                yield from self.sync(f"empty{sl}")
+            self.check(self.slot[sl] is None, f"block pass {j} overwrote slot {sl} holding {self.slot[sl]}")
+            self.slot[sl] = j
+            self.N[f"full{sl}"].arrive()
+            yield
+        for _ in range(self.rng.randint(0, 3)):   # dkb, dvb
+            yield
+
+    def go(self):
+        self.run({"stream": self.stream(), "block": self.block()})
+        self.check(all(b.arr == 0 for b in self.N.values()), "a named barrier left with a pending arrival")
+
+
+# ---------------------------------------------------------------------------
 def _fwd_case(rng, seed, drop=None):
     pairs = [(rng.choice([1, 2, 2]), rng.choice([1, 1, 2, 3, 4, 6])) for _ in range(rng.randint(1, 12))]
     return Forward(pairs, seed, drop)
@@ -546,7 +611,11 @@ def _dq_case(rng, seed, drop=None):
     return DQ([rng.choice([1, 1, 2, 3, 4, 6]) for _ in range(rng.randint(1, 12))], seed, drop)
 
 
-CASES = {"forward": _fwd_case, "dkdv": _dkdv_case, "dq": _dq_case}
+def _reduce_case(rng, seed, drop=None):
+    return Reduce(rng.randint(1, 6), seed, drop)
+
+
+CASES = {"forward": _fwd_case, "dkdv": _dkdv_case, "dq": _dq_case, "reduce": _reduce_case}
 
 
 @pytest.mark.parametrize("kernel", list(CASES))
@@ -560,7 +629,7 @@ def test_protocol_holds_on_random_schedules(kernel):
                                          ("forward", "stats"),
                                          ("dkdv", "qd_empty"),
                                          ("dkdv", "kv_empty"), ("dkdv", "lookahead_before_dv"), ("dq", "kv_empty"),
-                                         ("dq", "qd_empty")])
+                                         ("dq", "qd_empty"), ("reduce", "empty")])
 def test_each_producer_guard_is_needed(kernel, drop):
     """Removing one of the producer's waits lets some schedule overwrite a stage that an
     MMA has not read yet; issuing the dK/dV kernel's look-ahead S^T before dV instead of
