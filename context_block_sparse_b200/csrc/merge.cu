@@ -157,9 +157,192 @@ __device__ __forceinline__ int dest_of_block(const DevPlan& p, const MergeDest& 
 }
 
 // ---------------------------------------------------------------------------
-// merge: grid (A, Hkv); smem kb/vb rows of the block (bf16), staged entry ids
+// Helpers of the merge and reduce kernels.  The reduce kernel runs two roles of
+// 128 threads: the stream role reads the block's chunk records (the HBM-bound part)
+// 32 rows at a time, a quad per row; the block role computes the in-block term of
+// the same rows (bs keys of the block itself) and hands it over per pass of 32 rows
+// through one of two shared-memory slots: "full" (block -> stream) and "empty"
+// (stream -> block, before the slot's next use two passes later) are named barriers
+// over both roles.
 // ---------------------------------------------------------------------------
-template <int D, bool kBf16Rec>
+constexpr int kRoleThreads = kMergeThreads / 2;
+constexpr int kRoleRows = kRoleThreads / 4;   // rows of one pass (a quad per row in the stream role)
+constexpr int kBarStream = 1, kBarBlock = 2, kBarFull = 3, kBarEmpty = 5;   // full / empty: + slot
+
+__host__ __device__ inline size_t al16(size_t x) { return (x + 15) & ~size_t(15); }
+
+// float4 granule gi of row rl in a [32][D] fp32 slot; rows rl and rl ^ 1 use opposite
+// halves of the banks for the same granule, so a quad's 16-byte accesses from two rows
+// (one 128-byte wavefront) never share a bank.
+template <int D>
+__device__ __forceinline__ int slot_off(int rl, int gi) {
+  return rl * D + 4 * (gi ^ ((rl & 1) << 2));
+}
+
+template <int kSlot>
+__device__ __forceinline__ void slot_handoff_wait(int j) {   // block role: slot kSlot free again
+  if (j >= 2) named_sync<kBarEmpty + kSlot>(kMergeThreads);
+}
+
+__device__ __forceinline__ void slot_full_arrive(int sl) {
+  sl ? named_arrive<kBarFull + 1>(kMergeThreads) : named_arrive<kBarFull>(kMergeThreads);
+}
+
+__device__ __forceinline__ float quad_max(float x) {
+  x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, 1));
+  x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, 2));
+  return x;
+}
+
+// Stage the block's keys and values into shared memory, 16-byte chunks, by the
+// reduce kernel's block role.
+template <int D, bool kSwz>
+__device__ __forceinline__ void stage_block_rows(const DevPlan& p, int b, int g, const uint16_t* __restrict__ kb,
+                                                 const uint16_t* __restrict__ vb, uint16_t* sKb, uint16_t* sVb) {
+  const int gt = threadIdx.x - kRoleThreads, bs = p.bs;
+  for (int idx = gt; idx < bs * (D / 8); idx += kRoleThreads) {
+    const int t = idx / (D / 8), ch = idx % (D / 8);
+    const size_t src = (size_t(b * bs + t) * p.Hkv + g) * D + ch * 8;
+    const int dst = kSwz ? swz<D>(t, ch) : t * D + ch * 8;
+    *reinterpret_cast<uint4*>(sKb + dst) = *reinterpret_cast<const uint4*>(kb + src);
+    *reinterpret_cast<uint4*>(sVb + dst) = *reinterpret_cast<const uint4*>(vb + src);
+  }
+}
+// Stage the rows' q (or dout) into a swizzled [rows][D] tile, by the block role.
+template <int D>
+__device__ __forceinline__ void stage_query_rows(const DevPlan& p, int b, int g, const uint16_t* __restrict__ src_rows,
+                                                 uint16_t* sRows) {
+  const int gt = threadIdx.x - kRoleThreads, bs = p.bs, R = p.G * bs;
+  for (int idx = gt; idx < R * (D / 8); idx += kRoleThreads) {
+    const int r = idx / (D / 8), ch = idx % (D / 8);
+    const int tt = r / p.G, hh = r - tt * p.G;
+    const size_t src = (size_t(b * bs + tt) * p.Hq + g * p.G + hh) * D + ch * 8;
+    *reinterpret_cast<uint4*>(sRows + swz<D>(r, ch)) = *reinterpret_cast<const uint4*>(src_rows + src);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// merge: grid (A, Hkv), all 256 threads; a CTA combines the G * bs rows of block b
+// under KV head g, 64 rows a pass, a quad per row.  Per row: the in-block term --
+// online softmax over the bs block keys: M_in (base 2), L_in and the unnormalised
+// acc_in = sum_k 2^(s_k - M_in) v_k -- then the chunk records in ascending chunk
+// order (EG in flight) with an online reference maximum M: acc += l_c 2^(m_c - M) O_c,
+// L += l_c 2^(m_c - M); o = acc / L, lse = (M + log2 L) ln 2.
+// When rows and block keys come in multiples of 16 the in-block term of every row
+// is computed first, on the tensor cores (mma.sync; P rounded to bf16 for P V, as in
+// the chunk kernels), into shared memory, and each row's pass starts from it; other
+// shapes compute it per row on the FMA pipes in fp32.
+// smem: kb, vb [bs][D] bf16 | entry ids [kEStage] | tensor path: q rows [rows][D] bf16,
+// in-block acc [rows][D] fp32, (M_in, L_in) [rows] float2; tensor-path bf16 tiles swizzled.
+// ---------------------------------------------------------------------------
+struct MergeSmem {
+  size_t kb, vb, e, qr, ib, ml, total;
+};
+__host__ __device__ inline MergeSmem merge_smem(int D, int bs, int R, bool tc) {
+  MergeSmem L;
+  size_t o = 0;
+  L.kb = o;
+  o += al16(size_t(bs) * D * 2);
+  L.vb = o;
+  o += al16(size_t(bs) * D * 2);
+  L.e = o;
+  o += al16(size_t(kEStage) * 4);
+  L.qr = o;
+  o += al16(tc ? size_t(R) * D * 2 : 0);
+  L.ib = o;
+  o += al16(tc ? size_t(R) * D * 4 : 0);
+  L.ml = o;
+  o += al16(tc ? size_t(R) * 8 : 0);
+  L.total = o;
+  return L;
+}
+
+// In-block term of every row on the tensor cores: task t = (16-row tile t >> 1, half
+// t & 1 of the head dim), tasks spread over the 8 warps.  S = Q K^T over 16 block keys
+// at a time, an online maximum per row (quad max), P = 2^(s - M) and the half's
+// acc += P V.  Fragment layouts of m16n8k16: element e of an accumulator n-tile is row
+// gq + 8 (e >> 1), column 2 tq + (e & 1).  Results: sIb rows (slot_off layout), sML.
+template <int D>
+__device__ __forceinline__ void merge_block_tc(const DevPlan& p, float scale_log2, const uint16_t* sKb,
+                                               const uint16_t* sVb, const uint16_t* sQr, float* sIb, float2* sML) {
+  constexpr int kNH = D / 16;   // 8-column n-tiles in half the head dim
+  const int bs = p.bs, R = p.G * bs;
+  const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int gq = lane >> 2, tq = lane & 3;
+  for (int task = w; task < 2 * (R / 16); task += kMergeThreads / 32) {
+    const int r0 = (task >> 1) * 16, dh = task & 1;
+    float acc[kNH][4];
+#pragma unroll
+    for (int nn = 0; nn < kNH; ++nn)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) acc[nn][e] = 0.f;
+    float M[2] = {-INFINITY, -INFINITY}, L[2] = {0.f, 0.f};   // rows gq, gq + 8 (L: this thread's columns)
+    for (int kc = 0; kc < bs; kc += 16) {
+      float s[2][4];
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) s[nt][e] = 0.f;
+#pragma unroll
+      for (int ks = 0; ks < D / 16; ++ks) {
+        uint32_t qa[4], kf[4];
+        ldsm_x4(qa[0], qa[1], qa[2], qa[3], sQr + swz<D>(r0 + (lane & 15), 2 * ks + (lane >> 4)));
+        ldsm_x4(kf[0], kf[1], kf[2], kf[3],
+                sKb + swz<D>(kc + (lane & 7) + ((lane >> 4) << 3), 2 * ks + ((lane >> 3) & 1)));
+        mma_bf16_16816(s[0], qa, kf[0], kf[1]);
+        mma_bf16_16816(s[1], qa, kf[2], kf[3]);
+      }
+      uint32_t pa[4];   // word 2 nt + h: row gq + 8h, keys kc + 8 nt + 2 tq and + 1
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        float x[4];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) x[c] = s[c >> 1][2 * h + (c & 1)] * scale_log2;
+        const float mn = fmaxf(M[h], quad_max(fmaxf(fmaxf(x[0], x[1]), fmaxf(x[2], x[3]))));
+        const float corr = fast_exp2(M[h] - mn);   // 0 on the first keys (M = -inf)
+        M[h] = mn;
+        float e4[4];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) e4[c] = fast_exp2(x[c] - mn);
+        L[h] = L[h] * corr + ((e4[0] + e4[1]) + (e4[2] + e4[3]));
+#pragma unroll
+        for (int nn = 0; nn < kNH; ++nn) {
+          acc[nn][2 * h] *= corr;
+          acc[nn][2 * h + 1] *= corr;
+        }
+        pa[h] = pack_bf16(e4[0], e4[1]);
+        pa[2 + h] = pack_bf16(e4[2], e4[3]);
+      }
+#pragma unroll
+      for (int nn = 0; nn < kNH; nn += 2) {   // acc (the task's columns) += P V
+        const int kr = kc + (lane & 7) + 8 * ((lane >> 3) & 1);
+        const int ch = dh * (D / 16) + nn + (lane >> 4);
+        uint32_t b0, b1, b2, b3;
+        ldsm_x4_t(b0, b1, b2, b3, sVb + swz<D>(kr, ch));
+        mma_bf16_16816(acc[nn], pa, b0, b1);
+        mma_bf16_16816(acc[nn + 1], pa, b2, b3);
+      }
+    }
+#pragma unroll
+    for (int nn = 0; nn < kNH; ++nn)
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int r = r0 + gq + 8 * h;
+        const int col = dh * (D / 2) + nn * 8 + 2 * tq;
+        *reinterpret_cast<float2*>(sIb + slot_off<D>(r, col >> 2) + (col & 3)) =
+            make_float2(acc[nn][2 * h], acc[nn][2 * h + 1]);
+      }
+    if (dh == 0) {
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const float l = quad_sum(L[h]);
+        if (tq == 0) sML[r0 + gq + 8 * h] = make_float2(M[h], l);
+      }
+    }
+  }
+}
+
+template <int D, bool kBf16Rec, bool kTC>
 __global__ void __launch_bounds__(kMergeThreads, 2)
     merge_kernel(DevPlan p, const uint16_t* __restrict__ q, const uint16_t* __restrict__ kb,
                  const uint16_t* __restrict__ vb, float scale_log2, const void* __restrict__ part_o,
@@ -169,27 +352,44 @@ __global__ void __launch_bounds__(kMergeThreads, 2)
   using RecT = Rec<kBf16Rec>;
   constexpr int EG = 64 / (NG * RecT::RW);   // entries whose records are in flight together
   extern __shared__ __align__(16) uint8_t smem_raw[];
-  uint16_t* sKb = reinterpret_cast<uint16_t*>(smem_raw);   // [bs][D]
-  uint16_t* sVb = sKb + p.bs * D;
-  int* sE = reinterpret_cast<int*>(sVb + p.bs * D);        // [kEStage]
+  const int bs = p.bs, R = p.G * bs;
+  const MergeSmem S = merge_smem(D, bs, R, kTC);
+  uint16_t* sKb = reinterpret_cast<uint16_t*>(smem_raw + S.kb);
+  uint16_t* sVb = reinterpret_cast<uint16_t*>(smem_raw + S.vb);
+  int* sE = reinterpret_cast<int*>(smem_raw + S.e);
+  float* sIb = reinterpret_cast<float*>(smem_raw + S.ib);
+  float2* sML = reinterpret_cast<float2*>(smem_raw + S.ml);
   const int b = blockIdx.x, g = blockIdx.y;
   const int tid = threadIdx.x, u = tid & 3;
   const bool bterm = p.block_term && b >= p.bt_lo && b < p.bt_hi;   // in-block term of this block here
-  for (int idx = tid; bterm && idx < p.bs * (D / 8); idx += blockDim.x) {
+  for (int idx = tid; bterm && idx < bs * (D / 8); idx += kMergeThreads) {
     const int t = idx / (D / 8), ch = idx % (D / 8);
-    const size_t src = (size_t(b * p.bs + t) * p.Hkv + g) * D + ch * 8;
-    *reinterpret_cast<uint4*>(sKb + t * D + ch * 8) = *reinterpret_cast<const uint4*>(kb + src);
-    *reinterpret_cast<uint4*>(sVb + t * D + ch * 8) = *reinterpret_cast<const uint4*>(vb + src);
+    const size_t src = (size_t(b * bs + t) * p.Hkv + g) * D + ch * 8;
+    const int dst = kTC ? swz<D>(t, ch) : t * D + ch * 8;
+    *reinterpret_cast<uint4*>(sKb + dst) = *reinterpret_cast<const uint4*>(kb + src);
+    *reinterpret_cast<uint4*>(sVb + dst) = *reinterpret_cast<const uint4*>(vb + src);
+  }
+  if constexpr (kTC) {
+    if (bterm) {
+      uint16_t* sQr = reinterpret_cast<uint16_t*>(smem_raw + S.qr);
+      for (int idx = tid; idx < R * (D / 8); idx += kMergeThreads) {
+        const int r = idx / (D / 8), ch = idx % (D / 8);
+        const int tt = r / p.G, hh = r - tt * p.G;
+        const size_t src = (size_t(b * bs + tt) * p.Hq + g * p.G + hh) * D + ch * 8;
+        *reinterpret_cast<uint4*>(sQr + swz<D>(r, ch)) = *reinterpret_cast<const uint4*>(q + src);
+      }
+      __syncthreads();
+      merge_block_tc<D>(p, scale_log2, sKb, sVb, sQr, sIb, sML);
+    }
   }
   const int e0 = p.block_entry_ptr[b], n = p.block_entry_ptr[b + 1] - e0;
-  const int R = p.G * p.bs;
-  const int n_block_keys = bterm ? p.bs : 0;   // none when they are context keys, or on another rank
+  const int n_block_keys = (bterm && !kTC) ? bs : 0;   // in-block term computed per row (FMA path)
   // output rows: the plan's own outputs, or the owner's receive buffer (see MergeDest);
   // row_base = this block's first row in the buffer written to
   void* o_out = o;
   float* lse_out = lse;
   int out_bf16 = o_bf16;
-  size_t row_base = size_t(b) * p.bs;
+  size_t row_base = size_t(b) * bs;
   bool out_ok = true;
   if (dest.o != nullptr) {
     const int own = dest_of_block(p, dest, b, row_base, out_ok);
@@ -203,27 +403,40 @@ __global__ void __launch_bounds__(kMergeThreads, 2)
     const bool active = r0 + (tid >> 2) < R;
     const int tt = r / p.G, hh = r - tt * p.G;
     const int head = g * p.G + hh;
-    const size_t qrow = size_t(b * p.bs + tt) * p.Hq + head;
-    stage_entries(sE, p.block_entries + e0, 0, min(n, kEStage));
-    // in-block term: online softmax over the bs block keys (base 2), unnormalised
+    const size_t qrow = size_t(b * bs + tt) * p.Hq + head;
+    stage_entries(sE, p.block_entries + e0, 0, min(n, kEStage));   // (its barrier also publishes sIb, sML)
     float acc[NG][4];
     float M = -INFINITY, L = 0.f;
-    {
-      float qv[NG][4];
-      load_bf16_quad<NG>(q + qrow * D, u, qv);
+    if (kTC && bterm) {   // the row's in-block state
+      const float2 ml = sML[r];
+      M = ml.x;
+      L = ml.y;
+#pragma unroll
+      for (int k = 0; k < NG; ++k) {
+        const float4 x = *reinterpret_cast<const float4*>(sIb + slot_off<D>(r, u + 4 * k));
+        acc[k][0] = x.x;
+        acc[k][1] = x.y;
+        acc[k][2] = x.z;
+        acc[k][3] = x.w;
+      }
+    } else {
 #pragma unroll
       for (int k = 0; k < NG; ++k)
 #pragma unroll
         for (int i = 0; i < 4; ++i) acc[k][i] = 0.f;
+    }
+    if (n_block_keys > 0) {   // in-block term per row: online softmax over the block keys (base 2)
+      float qv[NG][4];
+      load_bf16_quad<NG>(q + qrow * D, u, qv);
       for (int key = 0; key < n_block_keys; ++key) {
         float kv[NG][4];
         load_bf16_quad<NG>(sKb + key * D, u, kv);
-        float dot = 0.f;
+        float d4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
         for (int k = 0; k < NG; ++k)
 #pragma unroll
-          for (int i = 0; i < 4; ++i) dot = fmaf(qv[k][i], kv[k][i], dot);
-        const float sc = quad_sum(dot) * scale_log2;
+          for (int i = 0; i < 4; ++i) d4[i] = fmaf(qv[k][i], kv[k][i], d4[i]);
+        const float sc = quad_sum((d4[0] + d4[1]) + (d4[2] + d4[3])) * scale_log2;
         const float mn = fmaxf(M, sc);
         const float corr = fast_exp2(M - mn);
         const float pr = fast_exp2(sc - mn);
@@ -249,7 +462,7 @@ __global__ void __launch_bounds__(kMergeThreads, 2)
           lx[v] = 0.f;
           mx[v] = -INFINITY;
           if (i0 + v < cnt) {
-            const size_t rec = size_t(sE[i0 + v] * p.bs + tt) * p.Hq + head;
+            const size_t rec = size_t(sE[i0 + v] * bs + tt) * p.Hq + head;
             RecT::template load<NG>(part_o, rec * D, u, ov[v]);
             const float lr = __ldg(part_l + rec), mr = __ldg(part_m + rec);
             lx[v] = lr;
@@ -350,10 +563,6 @@ __global__ void __launch_bounds__(kMergeThreads)
 // accumulators) when the rows and the block keys come in multiples of 16, otherwise
 // on the FMA pipes in fp32.
 // ---------------------------------------------------------------------------
-constexpr int kRoleThreads = kMergeThreads / 2;
-constexpr int kRoleRows = kRoleThreads / 4;   // rows of one pass (a quad per row in the stream role)
-constexpr int kBarStream = 1, kBarBlock = 2, kBarFull = 3, kBarEmpty = 5;   // full / empty: + slot
-
 // Shared memory of the reduce kernel (byte offsets, 16-byte aligned):
 //   slot   [2][32][D] fp32    in-block dq of a pass, block role -> stream role
 //   kb, vb [bs][D] bf16       the block's keys and values
@@ -365,7 +574,6 @@ constexpr int kBarStream = 1, kBarBlock = 2, kBarFull = 3, kBarEmpty = 5;   // f
 struct ReduceSmem {
   size_t slot, kb, vb, p, ds, e, qr, dr, total;
 };
-__host__ __device__ inline size_t al16(size_t x) { return (x + 15) & ~size_t(15); }
 __host__ __device__ inline ReduceSmem reduce_smem(int D, int bs, int R, bool tc, bool stage_rows) {
   ReduceSmem L;
   size_t o = 0;
@@ -391,14 +599,6 @@ __host__ __device__ inline ReduceSmem reduce_smem(int D, int bs, int R, bool tc,
   return L;
 }
 
-// float4 granule gi of row rl in a [32][D] fp32 slot; rows rl and rl ^ 1 use opposite
-// halves of the banks for the same granule, so a quad's 16-byte accesses from two rows
-// (one 128-byte wavefront) never share a bank.
-template <int D>
-__device__ __forceinline__ int slot_off(int rl, int gi) {
-  return rl * D + 4 * (gi ^ ((rl & 1) << 2));
-}
-
 struct BlockIO {   // global operands of the block role
   const uint16_t* q;
   const uint16_t* kb;
@@ -411,11 +611,6 @@ struct BlockIO {   // global operands of the block role
   float* dvb;
 };
 
-template <int kSlot>
-__device__ __forceinline__ void slot_handoff_wait(int j) {   // block role: slot kSlot free again
-  if (j >= 2) named_sync<kBarEmpty + kSlot>(kMergeThreads);
-}
-
 // Block role on the FMA pipes (any rows / block keys): a quad per row for P, dS and
 // the in-block dq; a warp per pair of block keys for dkb, dvb.
 template <int D>
@@ -426,12 +621,7 @@ __device__ __forceinline__ void block_role_fma(const DevPlan& p, int b, int g, c
   constexpr int DPL = D / 32;
   const int bs = p.bs, R = p.G * bs;
   const int gt = threadIdx.x - kRoleThreads, u = gt & 3, rl = gt >> 2, bwarp = gt >> 5, lane = threadIdx.x & 31;
-  for (int idx = gt; idx < bs * (D / 8); idx += kRoleThreads) {
-    const int t = idx / (D / 8), ch = idx % (D / 8);
-    const size_t src = (size_t(b * bs + t) * p.Hkv + g) * D + ch * 8;
-    *reinterpret_cast<uint4*>(sKb + t * D + ch * 8) = *reinterpret_cast<const uint4*>(io.kb + src);
-    *reinterpret_cast<uint4*>(sVb + t * D + ch * 8) = *reinterpret_cast<const uint4*>(io.vb + src);
-  }
+  stage_block_rows<D, false>(p, b, g, io.kb, io.vb, sKb, sVb);
   named_sync<kBarBlock>(kRoleThreads);
   const float scale_log2 = io.scale * kLog2e;
   const int npass = (R + kRoleRows - 1) / kRoleRows;
@@ -499,7 +689,7 @@ __device__ __forceinline__ void block_role_fma(const DevPlan& p, int b, int g, c
     for (int k = 0; k < NG; ++k)
       *reinterpret_cast<float4*>(slot + slot_off<D>(rl, u + 4 * k)) =
           make_float4(io.scale * acc[k][0], io.scale * acc[k][1], io.scale * acc[k][2], io.scale * acc[k][3]);
-    sl ? named_arrive<kBarFull + 1>(kMergeThreads) : named_arrive<kBarFull>(kMergeThreads);
+    slot_full_arrive(sl);
   }
   named_sync<kBarBlock>(kRoleThreads);   // P, dS (and the staged rows) of every row written
   // a warp per pair of block keys (k0, k0 + 1), sharing each row's loads:
@@ -565,19 +755,9 @@ __device__ __forceinline__ void block_role_tc(const DevPlan& p, int b, int g, co
   const int bs = p.bs, R = p.G * bs, SB = bs + 8;
   const int gt = threadIdx.x - kRoleThreads, w = gt >> 5, lane = threadIdx.x & 31;
   const int gq = lane >> 2, tq = lane & 3;
-  for (int idx = gt; idx < bs * (D / 8); idx += kRoleThreads) {
-    const int t = idx / (D / 8), ch = idx % (D / 8);
-    const size_t src = (size_t(b * bs + t) * p.Hkv + g) * D + ch * 8;
-    *reinterpret_cast<uint4*>(sKb + swz<D>(t, ch)) = *reinterpret_cast<const uint4*>(io.kb + src);
-    *reinterpret_cast<uint4*>(sVb + swz<D>(t, ch)) = *reinterpret_cast<const uint4*>(io.vb + src);
-  }
-  for (int idx = gt; idx < R * (D / 8); idx += kRoleThreads) {
-    const int r = idx / (D / 8), ch = idx % (D / 8);
-    const int tt = r / p.G, hh = r - tt * p.G;
-    const size_t src = (size_t(b * bs + tt) * p.Hq + g * p.G + hh) * D + ch * 8;
-    *reinterpret_cast<uint4*>(sQr + swz<D>(r, ch)) = *reinterpret_cast<const uint4*>(io.q + src);
-    *reinterpret_cast<uint4*>(sDr + swz<D>(r, ch)) = *reinterpret_cast<const uint4*>(io.dout + src);
-  }
+  stage_block_rows<D, true>(p, b, g, io.kb, io.vb, sKb, sVb);
+  stage_query_rows<D>(p, b, g, io.q, sQr);
+  stage_query_rows<D>(p, b, g, io.dout, sDr);
   named_sync<kBarBlock>(kRoleThreads);
   const float scale_log2 = io.scale * kLog2e;
   const int npass = (R + kRoleRows - 1) / kRoleRows;
@@ -671,7 +851,7 @@ __device__ __forceinline__ void block_role_tc(const DevPlan& p, int b, int g, co
               make_float2(io.scale * dqa[nn][2 * h], io.scale * dqa[nn][2 * h + 1]);
         }
     }
-    sl ? named_arrive<kBarFull + 1>(kMergeThreads) : named_arrive<kBarFull>(kMergeThreads);
+    slot_full_arrive(sl);
   }
   named_sync<kBarBlock>(kRoleThreads);   // P, dS of every row in shared memory
   const int nitems = 2 * (bs / 16) * (D / 32);
@@ -818,17 +998,27 @@ __global__ void __launch_bounds__(kMergeThreads, 2)
                       reinterpret_cast<float*>(smem_raw + L.ds), sQr, sDr);
 }
 
+template <int D, bool kBf16Rec, bool kTC>
+cudaError_t merge_launch(const DevPlan& p, const uint16_t* q, const uint16_t* kb, const uint16_t* vb, float scale,
+                         const void* po, const float* pm, const float* pl, void* o, int o_bf16, float* lse,
+                         cudaStream_t s, const MergeDest& dest) {
+  const size_t smem = merge_smem(D, p.bs, p.G * p.bs, kTC).total;
+  cudaError_t e =
+      cudaFuncSetAttribute(merge_kernel<D, kBf16Rec, kTC>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+  if (e != cudaSuccess) return e;
+  merge_kernel<D, kBf16Rec, kTC><<<dim3(p.A, p.Hkv), kMergeThreads, smem, s>>>(p, q, kb, vb, scale * kLog2e, po, pm,
+                                                                                pl, o, o_bf16, lse, dest);
+  return cudaGetLastError();
+}
+
 template <int D, bool kBf16Rec>
 cudaError_t merge_d(const DevPlan& p, const uint16_t* q, const uint16_t* kb, const uint16_t* vb,
                     float scale, const void* po, const float* pm, const float* pl, void* o, int o_bf16,
                     float* lse, cudaStream_t s, const MergeDest& dest) {
-  const size_t smem = size_t(2) * p.bs * D * sizeof(uint16_t) + kEStage * sizeof(int);
-  cudaError_t e =
-      cudaFuncSetAttribute(merge_kernel<D, kBf16Rec>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
-  if (e != cudaSuccess) return e;
-  merge_kernel<D, kBf16Rec><<<dim3(p.A, p.Hkv), kMergeThreads, smem, s>>>(p, q, kb, vb, scale * kLog2e, po, pm,
-                                                                            pl, o, o_bf16, lse, dest);
-  return cudaGetLastError();
+  // tensor path: rows and block keys in 16s (its tiles always fit: at most 163 KB)
+  if ((p.G * p.bs) % 16 == 0 && p.bs % 16 == 0)
+    return merge_launch<D, kBf16Rec, true>(p, q, kb, vb, scale, po, pm, pl, o, o_bf16, lse, s, dest);
+  return merge_launch<D, kBf16Rec, false>(p, q, kb, vb, scale, po, pm, pl, o, o_bf16, lse, s, dest);
 }
 
 template <int D, bool kBf16Rec, bool kTC>
