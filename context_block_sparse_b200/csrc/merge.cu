@@ -195,12 +195,13 @@ __device__ __forceinline__ float quad_max(float x) {
 }
 
 // Stage the block's keys and values into shared memory, 16-byte chunks, by the
-// reduce kernel's block role.
+// nthr threads from t0 on (swizzled for ldmatrix when kSwz).
 template <int D, bool kSwz>
 __device__ __forceinline__ void stage_block_rows(const DevPlan& p, int b, int g, const uint16_t* __restrict__ kb,
-                                                 const uint16_t* __restrict__ vb, uint16_t* sKb, uint16_t* sVb) {
-  const int gt = threadIdx.x - kRoleThreads, bs = p.bs;
-  for (int idx = gt; idx < bs * (D / 8); idx += kRoleThreads) {
+                                                 const uint16_t* __restrict__ vb, uint16_t* sKb, uint16_t* sVb,
+                                                 int t0, int nthr) {
+  const int gt = threadIdx.x - t0, bs = p.bs;
+  for (int idx = gt; idx < bs * (D / 8); idx += nthr) {
     const int t = idx / (D / 8), ch = idx % (D / 8);
     const size_t src = (size_t(b * bs + t) * p.Hkv + g) * D + ch * 8;
     const int dst = kSwz ? swz<D>(t, ch) : t * D + ch * 8;
@@ -208,12 +209,13 @@ __device__ __forceinline__ void stage_block_rows(const DevPlan& p, int b, int g,
     *reinterpret_cast<uint4*>(sVb + dst) = *reinterpret_cast<const uint4*>(vb + src);
   }
 }
-// Stage the rows' q (or dout) into a swizzled [rows][D] tile, by the block role.
+// Stage the rows' q (or dout) into a swizzled [rows][D] tile, by the nthr threads
+// from t0 on.
 template <int D>
 __device__ __forceinline__ void stage_query_rows(const DevPlan& p, int b, int g, const uint16_t* __restrict__ src_rows,
-                                                 uint16_t* sRows) {
-  const int gt = threadIdx.x - kRoleThreads, bs = p.bs, R = p.G * bs;
-  for (int idx = gt; idx < R * (D / 8); idx += kRoleThreads) {
+                                                 uint16_t* sRows, int t0, int nthr) {
+  const int gt = threadIdx.x - t0, bs = p.bs, R = p.G * bs;
+  for (int idx = gt; idx < R * (D / 8); idx += nthr) {
     const int r = idx / (D / 8), ch = idx % (D / 8);
     const int tt = r / p.G, hh = r - tt * p.G;
     const size_t src = (size_t(b * bs + tt) * p.Hq + g * p.G + hh) * D + ch * 8;
@@ -549,32 +551,33 @@ __global__ void __launch_bounds__(kMergeThreads)
 }
 
 // ---------------------------------------------------------------------------
-// dq reduce + in-block backward: grid (A, Hkv), two roles of 128 threads that run
-// side by side, so that the partial stream keeps HBM busy while the in-block term is
-// computed:
-//   stream role (warps 0-3): for 32 rows at a time, the sum of the chunk dq partials
-//     in ascending chunk order (EG records in flight per thread), plus the rows'
-//     in-block dq taken from a shared-memory slot -> dq;
-//   block role (warps 4-7): P, dS of the bs block keys and the rows' in-block dq
-//     (-> the slot of the same 32 rows), then dkb = scale dS^T Q and dvb = P^T dO.
-// The two slots are handed over with named barriers (full: block -> stream, empty:
-// stream -> block).  The block role runs its products on the tensor cores (mma.sync
-// m16n8k16: bf16 operands, P and dS rounded to bf16 as in the chunk kernels; fp32
-// accumulators) when the rows and the block keys come in multiples of 16, otherwise
-// on the FMA pipes in fp32.
+// dq reduce + in-block backward: grid (A, Hkv); a CTA handles the G * bs rows of
+// block b under KV head g: dq = the in-block term's dq + the chunk dq partials in
+// ascending chunk order; dkb, dvb of the in-block term.  Two kernels:
+//
+//  bwd_reduce_tc_kernel (rows and block keys in multiples of 16): all 256 threads.
+//    First the in-block term of every row on the tensor cores (mma.sync m16n8k16:
+//    bf16 operands, P and dS rounded to bf16 as in the chunk kernels; fp32
+//    accumulators), its dq into shared memory; then 64 rows a pass, a quad per row,
+//    dq = that + the partials (EG records in flight per thread); last dkb = scale dS^T Q
+//    and dvb = P^T dO from P, dS kept in shared memory.
+//
+//  bwd_reduce_kernel (any shape): the two roles above run side by side -- the
+//    stream role sums the partials of 32 rows a pass and adds the slot's in-block dq;
+//    the block role computes P, dS and the in-block dq on the FMA pipes in fp32 (a quad
+//    per row), then dkb, dvb (a warp per pair of block keys).
 // ---------------------------------------------------------------------------
-// Shared memory of the reduce kernel (byte offsets, 16-byte aligned):
+// Shared memory of bwd_reduce_kernel (byte offsets, 16-byte aligned):
 //   slot   [2][32][D] fp32    in-block dq of a pass, block role -> stream role
 //   kb, vb [bs][D] bf16       the block's keys and values
-//   p, ds  [rows][bs] fp32 (FMA path) or [rows][bs + 8] bf16 (tensor path)
+//   p, ds  [rows][bs] fp32
 //   e      [kEStage] int      entry ids (stream role)
-//   qr, dr [rows][D] bf16     the rows' q and dout (tensor path; FMA path when stage_rows)
-// rows = G * bs ordered (token, head).  On the tensor path the kb, vb, qr, dr tiles are
-// 16-byte-chunk swizzled (swz) for conflict-free ldmatrix.
+//   qr, dr [rows][D] bf16     the rows' q and dout (when stage_rows)
+// rows = G * bs ordered (token, head).
 struct ReduceSmem {
   size_t slot, kb, vb, p, ds, e, qr, dr, total;
 };
-__host__ __device__ inline ReduceSmem reduce_smem(int D, int bs, int R, bool tc, bool stage_rows) {
+__host__ __device__ inline ReduceSmem reduce_smem(int D, int bs, int R, bool stage_rows) {
   ReduceSmem L;
   size_t o = 0;
   L.slot = o;
@@ -583,18 +586,46 @@ __host__ __device__ inline ReduceSmem reduce_smem(int D, int bs, int R, bool tc,
   o += al16(size_t(bs) * D * 2);
   L.vb = o;
   o += al16(size_t(bs) * D * 2);
-  const size_t pds = tc ? size_t(R) * (bs + 8) * 2 : size_t(R) * bs * 4;
   L.p = o;
-  o += al16(pds);
+  o += al16(size_t(R) * bs * 4);
   L.ds = o;
-  o += al16(pds);
+  o += al16(size_t(R) * bs * 4);
   L.e = o;
   o += al16(size_t(kEStage) * 4);
-  const size_t rows = (tc || stage_rows) ? size_t(R) * D * 2 : 0;
+  const size_t rows = stage_rows ? size_t(R) * D * 2 : 0;
   L.qr = o;
   o += al16(rows);
   L.dr = o;
   o += al16(rows);
+  L.total = o;
+  return L;
+}
+
+// Shared memory of bwd_reduce_tc_kernel: kb, vb [bs][D] and qr, dr [rows][D] bf16
+// (swizzled for ldmatrix); p, ds [rows][bs + 8] bf16 (the pad keeps ldmatrix rows on
+// distinct banks); ib [rows][D] fp32 in-block dq (slot_off layout); entry ids.
+struct ReduceTcSmem {
+  size_t kb, vb, qr, dr, p, ds, ib, e, total;
+};
+__host__ __device__ inline ReduceTcSmem reduce_tc_smem(int D, int bs, int R) {
+  ReduceTcSmem L;
+  size_t o = 0;
+  L.kb = o;
+  o += al16(size_t(bs) * D * 2);
+  L.vb = o;
+  o += al16(size_t(bs) * D * 2);
+  L.qr = o;
+  o += al16(size_t(R) * D * 2);
+  L.dr = o;
+  o += al16(size_t(R) * D * 2);
+  L.p = o;
+  o += al16(size_t(R) * (bs + 8) * 2);
+  L.ds = o;
+  o += al16(size_t(R) * (bs + 8) * 2);
+  L.ib = o;
+  o += al16(size_t(R) * D * 4);
+  L.e = o;
+  o += al16(size_t(kEStage) * 4);
   L.total = o;
   return L;
 }
@@ -621,7 +652,7 @@ __device__ __forceinline__ void block_role_fma(const DevPlan& p, int b, int g, c
   constexpr int DPL = D / 32;
   const int bs = p.bs, R = p.G * bs;
   const int gt = threadIdx.x - kRoleThreads, u = gt & 3, rl = gt >> 2, bwarp = gt >> 5, lane = threadIdx.x & 31;
-  stage_block_rows<D, false>(p, b, g, io.kb, io.vb, sKb, sVb);
+  stage_block_rows<D, false>(p, b, g, io.kb, io.vb, sKb, sVb, kRoleThreads, kRoleThreads);
   named_sync<kBarBlock>(kRoleThreads);
   const float scale_log2 = io.scale * kLog2e;
   const int npass = (R + kRoleRows - 1) / kRoleRows;
@@ -740,122 +771,115 @@ __device__ __forceinline__ void block_role_fma(const DevPlan& p, int b, int g, c
   }
 }
 
-// Block role on the tensor cores (rows R and block keys bs multiples of 16).  Pass j
-// (rows 32j..32j+31) gives warp w the 16-row tile 2j + (w & 1) and half w >> 1 of the
-// head dim: S = Q K^T and dP = dO V^T over the block keys, 16 at a time (the two warps
-// of a tile compute them both), P and dS in registers, the warp's half of the in-block
-// dq += dS K.  Then dkb = scale dS^T Q and dvb = P^T dO, contracting over the rows,
-// in items of (product, 16 keys, 32 columns).  Fragment layouts of m16n8k16: element
-// e of an accumulator n-tile is row gq + 8 (e >> 1), column 2 tq + (e & 1).
+// In-block term of every row on the tensor cores: task t = (16-row tile t >> 1, half
+// t & 1 of the head dim), tasks spread over the 8 warps.  S = Q K^T and dP = dO V^T over
+// the block keys 16 at a time (both tasks of a tile compute them), P = exp2(s c - lse2),
+// dS = P (dP - Delta) in registers, the half's in-block dq += dS K -> sIb (times scale);
+// the tile's P, dS (bf16) -> sPb, sdSb.  Fragment layouts of m16n8k16: element e of an
+// accumulator n-tile is row gq + 8 (e >> 1), column 2 tq + (e & 1).
 template <int D>
-__device__ __forceinline__ void block_role_tc(const DevPlan& p, int b, int g, const BlockIO& io, float* sSlot,
-                                              uint16_t* sKb, uint16_t* sVb, uint16_t* sPb, uint16_t* sdSb,
-                                              uint16_t* sQr, uint16_t* sDr) {
+__device__ __forceinline__ void reduce_inblock_tc(const DevPlan& p, int b, int g, const BlockIO& io,
+                                                  const uint16_t* sKb, const uint16_t* sVb, const uint16_t* sQr,
+                                                  const uint16_t* sDr, uint16_t* sPb, uint16_t* sdSb, float* sIb) {
   constexpr int kNH = D / 16;   // 8-column n-tiles in half the head dim
   const int bs = p.bs, R = p.G * bs, SB = bs + 8;
-  const int gt = threadIdx.x - kRoleThreads, w = gt >> 5, lane = threadIdx.x & 31;
+  const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int gq = lane >> 2, tq = lane & 3;
-  stage_block_rows<D, true>(p, b, g, io.kb, io.vb, sKb, sVb);
-  stage_query_rows<D>(p, b, g, io.q, sQr);
-  stage_query_rows<D>(p, b, g, io.dout, sDr);
-  named_sync<kBarBlock>(kRoleThreads);
   const float scale_log2 = io.scale * kLog2e;
-  const int npass = (R + kRoleRows - 1) / kRoleRows;
-  const int nmt = R / 16;
-  const int dh = w >> 1;
-  for (int j = 0; j < npass; ++j) {
-    const int mt = 2 * j + (w & 1);
+  for (int task = w; task < 2 * (R / 16); task += kMergeThreads / 32) {
+    const int r0 = (task >> 1) * 16, dh = task & 1;
     float dqa[kNH][4];
 #pragma unroll
     for (int nn = 0; nn < kNH; ++nn)
 #pragma unroll
       for (int e = 0; e < 4; ++e) dqa[nn][e] = 0.f;
-    if (mt < nmt) {
-      const int r0 = mt * 16;
-      float l2[2], dl[2];   // statistics of the thread's rows r0 + gq, r0 + gq + 8
+    float l2[2], dl[2];   // statistics of the thread's rows r0 + gq, r0 + gq + 8
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        const int r = r0 + gq + 8 * h, tt = r / p.G, hh = r - tt * p.G;
-        const size_t qrow = size_t(b * bs + tt) * p.Hq + g * p.G + hh;
-        l2[h] = io.lse[qrow] * kLog2e;
-        dl[h] = io.delta[qrow];
+    for (int h = 0; h < 2; ++h) {
+      const int r = r0 + gq + 8 * h, tt = r / p.G, hh = r - tt * p.G;
+      const size_t qrow = size_t(b * bs + tt) * p.Hq + g * p.G + hh;
+      l2[h] = io.lse[qrow] * kLog2e;
+      dl[h] = io.delta[qrow];
+    }
+    for (int kc = 0; kc < bs; kc += 16) {
+      float s[2][4], dp[2][4];
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) s[nt][e] = dp[nt][e] = 0.f;
+#pragma unroll
+      for (int ks = 0; ks < D / 16; ++ks) {
+        uint32_t qa[4], da[4], kf[4], vf[4];
+        const int ar = r0 + (lane & 15), ach = 2 * ks + (lane >> 4);
+        ldsm_x4(qa[0], qa[1], qa[2], qa[3], sQr + swz<D>(ar, ach));
+        ldsm_x4(da[0], da[1], da[2], da[3], sDr + swz<D>(ar, ach));
+        const int br = kc + (lane & 7) + ((lane >> 4) << 3), bch = 2 * ks + ((lane >> 3) & 1);
+        ldsm_x4(kf[0], kf[1], kf[2], kf[3], sKb + swz<D>(br, bch));
+        ldsm_x4(vf[0], vf[1], vf[2], vf[3], sVb + swz<D>(br, bch));
+        mma_bf16_16816(s[0], qa, kf[0], kf[1]);
+        mma_bf16_16816(s[1], qa, kf[2], kf[3]);
+        mma_bf16_16816(dp[0], da, vf[0], vf[1]);
+        mma_bf16_16816(dp[1], da, vf[2], vf[3]);
       }
-      for (int kc = 0; kc < bs; kc += 16) {
-        float s[2][4], dp[2][4];
+      // P = exp2(s c - lse2), dS = P (dP - Delta), packed as the A operand of dS K:
+      // word 2 nt + h holds row gq + 8h, keys kc + 8 nt + 2 tq and + 1
+      uint32_t pa[4], sa[4];
 #pragma unroll
-        for (int nt = 0; nt < 2; ++nt)
+      for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
-          for (int e = 0; e < 4; ++e) s[nt][e] = dp[nt][e] = 0.f;
+        for (int h = 0; h < 2; ++h) {
+          float pr[2], ds[2];
 #pragma unroll
-        for (int ks = 0; ks < D / 16; ++ks) {
-          uint32_t qa[4], da[4], kf[4], vf[4];
-          const int ar = r0 + (lane & 15), ach = 2 * ks + (lane >> 4);
-          ldsm_x4(qa[0], qa[1], qa[2], qa[3], sQr + swz<D>(ar, ach));
-          ldsm_x4(da[0], da[1], da[2], da[3], sDr + swz<D>(ar, ach));
-          const int br = kc + (lane & 7) + ((lane >> 4) << 3), bch = 2 * ks + ((lane >> 3) & 1);
-          ldsm_x4(kf[0], kf[1], kf[2], kf[3], sKb + swz<D>(br, bch));
-          ldsm_x4(vf[0], vf[1], vf[2], vf[3], sVb + swz<D>(br, bch));
-          mma_bf16_16816(s[0], qa, kf[0], kf[1]);
-          mma_bf16_16816(s[1], qa, kf[2], kf[3]);
-          mma_bf16_16816(dp[0], da, vf[0], vf[1]);
-          mma_bf16_16816(dp[1], da, vf[2], vf[3]);
+          for (int c = 0; c < 2; ++c) {
+            pr[c] = (l2[h] == -INFINITY) ? 0.f : fast_exp2(s[nt][2 * h + c] * scale_log2 - l2[h]);
+            ds[c] = pr[c] * (dp[nt][2 * h + c] - dl[h]);
+          }
+          pa[2 * nt + h] = pack_bf16(pr[0], pr[1]);
+          sa[2 * nt + h] = pack_bf16(ds[0], ds[1]);
         }
-        // P = exp2(s c - lse2), dS = P (dP - Delta), packed as the A operand of dS K:
-        // word 2 nt + h holds row gq + 8h, keys kc + 8 nt + 2 tq and + 1
-        uint32_t pa[4], sa[4];
+      if (dh == 0) {   // P, dS of the tile for dvb, dkb (one of the tile's two tasks)
 #pragma unroll
         for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
           for (int h = 0; h < 2; ++h) {
-            float pr[2], ds[2];
-#pragma unroll
-            for (int c = 0; c < 2; ++c) {
-              pr[c] = (l2[h] == -INFINITY) ? 0.f : fast_exp2(s[nt][2 * h + c] * scale_log2 - l2[h]);
-              ds[c] = pr[c] * (dp[nt][2 * h + c] - dl[h]);
-            }
-            pa[2 * nt + h] = pack_bf16(pr[0], pr[1]);
-            sa[2 * nt + h] = pack_bf16(ds[0], ds[1]);
+            const int off = (r0 + gq + 8 * h) * SB + kc + 8 * nt + 2 * tq;
+            *reinterpret_cast<uint32_t*>(sPb + off) = pa[2 * nt + h];
+            *reinterpret_cast<uint32_t*>(sdSb + off) = sa[2 * nt + h];
           }
-        if (dh == 0) {   // P, dS of the tile for dvb, dkb (one of the tile's two warps)
+      }
 #pragma unroll
-          for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-              const int off = (r0 + gq + 8 * h) * SB + kc + 8 * nt + 2 * tq;
-              *reinterpret_cast<uint32_t*>(sPb + off) = pa[2 * nt + h];
-              *reinterpret_cast<uint32_t*>(sdSb + off) = sa[2 * nt + h];
-            }
-        }
-#pragma unroll
-        for (int nn = 0; nn < kNH; nn += 2) {   // in-block dq (the warp's columns) += dS K
-          const int kr = kc + (lane & 7) + 8 * ((lane >> 3) & 1);
-          const int ch = dh * (D / 16) + nn + (lane >> 4);
-          uint32_t b0, b1, b2, b3;
-          ldsm_x4_t(b0, b1, b2, b3, sKb + swz<D>(kr, ch));
-          mma_bf16_16816(dqa[nn], sa, b0, b1);
-          mma_bf16_16816(dqa[nn + 1], sa, b2, b3);
-        }
+      for (int nn = 0; nn < kNH; nn += 2) {   // in-block dq (the task's columns) += dS K
+        const int kr = kc + (lane & 7) + 8 * ((lane >> 3) & 1);
+        const int ch = dh * (D / 16) + nn + (lane >> 4);
+        uint32_t b0, b1, b2, b3;
+        ldsm_x4_t(b0, b1, b2, b3, sKb + swz<D>(kr, ch));
+        mma_bf16_16816(dqa[nn], sa, b0, b1);
+        mma_bf16_16816(dqa[nn + 1], sa, b2, b3);
       }
     }
-    const int sl = j & 1;
-    sl ? slot_handoff_wait<1>(j) : slot_handoff_wait<0>(j);
-    if (mt < nmt) {
-      float* slot = sSlot + sl * kRoleRows * D;
 #pragma unroll
-      for (int nn = 0; nn < kNH; ++nn)
+    for (int nn = 0; nn < kNH; ++nn)
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          const int rl = (w & 1) * 16 + gq + 8 * h;
-          const int col = dh * (D / 2) + nn * 8 + 2 * tq;
-          *reinterpret_cast<float2*>(slot + slot_off<D>(rl, col >> 2) + (col & 3)) =
-              make_float2(io.scale * dqa[nn][2 * h], io.scale * dqa[nn][2 * h + 1]);
-        }
-    }
-    slot_full_arrive(sl);
+      for (int h = 0; h < 2; ++h) {
+        const int r = r0 + gq + 8 * h;
+        const int col = dh * (D / 2) + nn * 8 + 2 * tq;
+        *reinterpret_cast<float2*>(sIb + slot_off<D>(r, col >> 2) + (col & 3)) =
+            make_float2(io.scale * dqa[nn][2 * h], io.scale * dqa[nn][2 * h + 1]);
+      }
   }
-  named_sync<kBarBlock>(kRoleThreads);   // P, dS of every row in shared memory
+}
+
+// dkb = scale dS^T Q and dvb = P^T dO on the tensor cores, contracting over the rows,
+// in items (product, 16 keys, 32 columns) spread over the 8 warps.
+template <int D>
+__device__ __forceinline__ void reduce_kv_tc(const DevPlan& p, int b, int g, const BlockIO& io,
+                                             const uint16_t* sQr, const uint16_t* sDr, const uint16_t* sPb,
+                                             const uint16_t* sdSb) {
+  const int bs = p.bs, R = p.G * bs, SB = bs + 8;
+  const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int gq = lane >> 2, tq = lane & 3;
   const int nitems = 2 * (bs / 16) * (D / 32);
-  for (int it = w; it < nitems; it += kRoleThreads / 32) {
+  for (int it = w; it < nitems; it += kMergeThreads / 32) {
     const int prod = it & 1, rest = it >> 1, km = rest / (D / 32), ng = rest % (D / 32);
     const uint16_t* sA = prod ? sPb : sdSb;   // A = P^T or dS^T (keys x rows), stored [rows][keys]
     const uint16_t* sB = prod ? sDr : sQr;    // B = dout or q (rows x columns)
@@ -892,7 +916,92 @@ __device__ __forceinline__ void block_role_tc(const DevPlan& p, int b, int g, co
   }
 }
 
-template <int D, bool kBf16Rec, bool kTC>
+template <int D, bool kBf16Rec>
+__global__ void __launch_bounds__(kMergeThreads, 2)
+    bwd_reduce_tc_kernel(DevPlan p, const uint16_t* __restrict__ q, const uint16_t* __restrict__ kb,
+                         const uint16_t* __restrict__ vb, const uint16_t* __restrict__ dout,
+                         const float* __restrict__ lse, const float* __restrict__ delta,
+                         const void* __restrict__ dq_part, float scale, float* __restrict__ dq,
+                         float* __restrict__ dkb, float* __restrict__ dvb, const MergeDest dest) {
+  constexpr int NG = D / 16;
+  using RecT = Rec<kBf16Rec>;
+  constexpr int EG = 64 / (NG * RecT::RW);   // entries whose partials are in flight together
+  extern __shared__ __align__(16) uint8_t smem_raw[];
+  const int bs = p.bs, R = p.G * bs;
+  const ReduceTcSmem L = reduce_tc_smem(D, bs, R);
+  uint16_t* sKb = reinterpret_cast<uint16_t*>(smem_raw + L.kb);
+  uint16_t* sVb = reinterpret_cast<uint16_t*>(smem_raw + L.vb);
+  uint16_t* sQr = reinterpret_cast<uint16_t*>(smem_raw + L.qr);
+  uint16_t* sDr = reinterpret_cast<uint16_t*>(smem_raw + L.dr);
+  uint16_t* sPb = reinterpret_cast<uint16_t*>(smem_raw + L.p);
+  uint16_t* sdSb = reinterpret_cast<uint16_t*>(smem_raw + L.ds);
+  float* sIb = reinterpret_cast<float*>(smem_raw + L.ib);
+  int* sE = reinterpret_cast<int*>(smem_raw + L.e);
+  const int b = blockIdx.x, g = blockIdx.y;
+  const int tid = threadIdx.x, u = tid & 3;
+  const bool bterm = p.block_term && b >= p.bt_lo && b < p.bt_hi;   // in-block term of this block here
+  const BlockIO io{q, kb, vb, dout, lse, delta, scale, dkb, dvb};
+  if (bterm) {
+    stage_block_rows<D, true>(p, b, g, kb, vb, sKb, sVb, 0, kMergeThreads);
+    stage_query_rows<D>(p, b, g, q, sQr, 0, kMergeThreads);
+    stage_query_rows<D>(p, b, g, dout, sDr, 0, kMergeThreads);
+    __syncthreads();
+    reduce_inblock_tc<D>(p, b, g, io, sKb, sVb, sQr, sDr, sPb, sdSb, sIb);
+  }
+  // dq rows: the plan's own dq, or the owner's receive buffer (see MergeDest; dest.o)
+  float* dq_out = dq;
+  size_t dq_base = size_t(b) * bs;
+  bool dq_ok = true;
+  if (dest.o != nullptr) dq_out = dest.o[dest_of_block(p, dest, b, dq_base, dq_ok)];
+  const int e0 = p.block_entry_ptr[b], n = p.block_entry_ptr[b + 1] - e0;
+  for (int r0 = 0; r0 < R; r0 += kRowsPerPass) {
+    const int r = min(r0 + (tid >> 2), R - 1);          // rows past R compute, never store
+    const bool active = r0 + (tid >> 2) < R;
+    const int tt = r / p.G, hh = r - tt * p.G;
+    const int head = g * p.G + hh;
+    stage_entries(sE, p.block_entries + e0, 0, min(n, kEStage));   // (its barrier also publishes sIb)
+    float4 tot[NG];
+#pragma unroll
+    for (int k = 0; k < NG; ++k)
+      tot[k] = bterm ? *reinterpret_cast<const float4*>(sIb + slot_off<D>(r, u + 4 * k))
+                     : make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int c0 = 0; c0 < n; c0 += kEStage) {
+      const int cnt = min(kEStage, n - c0);
+      if (c0 > 0) stage_entries(sE, p.block_entries + e0, c0, cnt);
+      for (int i0 = 0; i0 < cnt; i0 += EG) {
+        uint32_t pv[EG][NG][RecT::RW];
+#pragma unroll
+        for (int v = 0; v < EG; ++v) {
+          if (i0 + v < cnt) {
+            const size_t rec = size_t(sE[i0 + v] * bs + tt) * p.Hq + head;
+            RecT::template load<NG>(dq_part, rec * D, u, pv[v]);
+          } else {
+            RecT::template zero<NG>(pv[v]);
+          }
+        }
+#pragma unroll
+        for (int v = 0; v < EG; ++v)
+#pragma unroll
+          for (int k = 0; k < NG; ++k) {
+            const float4 x = RecT::get(pv[v][k]);
+            tot[k].x += x.x;
+            tot[k].y += x.y;
+            tot[k].z += x.z;
+            tot[k].w += x.w;
+          }
+      }
+    }
+    if (active && dq_ok) {
+      float* dst = dq_out + ((dq_base + tt) * p.Hq + head) * D;   // = dq + qrow * D for the plan's own dq
+#pragma unroll
+      for (int k = 0; k < NG; ++k) *reinterpret_cast<float4*>(dst + 4 * (u + 4 * k)) = tot[k];
+    }
+  }
+  // P, dS of every row were published by the pass loop's barrier
+  if (bterm) reduce_kv_tc<D>(p, b, g, io, sQr, sDr, sPb, sdSb);
+}
+
+template <int D, bool kBf16Rec>
 __global__ void __launch_bounds__(kMergeThreads, 2)
     bwd_reduce_kernel(DevPlan p, const uint16_t* __restrict__ q, const uint16_t* __restrict__ kb,
                       const uint16_t* __restrict__ vb, const uint16_t* __restrict__ dout,
@@ -905,7 +1014,7 @@ __global__ void __launch_bounds__(kMergeThreads, 2)
   extern __shared__ __align__(16) uint8_t smem_raw[];
   const int bs = p.bs;
   const int R = p.G * bs;
-  const ReduceSmem L = reduce_smem(D, bs, R, kTC, stage_rows != 0);
+  const ReduceSmem L = reduce_smem(D, bs, R, stage_rows != 0);
   float* sSlot = reinterpret_cast<float*>(smem_raw + L.slot);
   int* sE = reinterpret_cast<int*>(smem_raw + L.e);
   const int b = blockIdx.x, g = blockIdx.y;
@@ -990,12 +1099,8 @@ __global__ void __launch_bounds__(kMergeThreads, 2)
   uint16_t* sVb = reinterpret_cast<uint16_t*>(smem_raw + L.vb);
   uint16_t* sQr = reinterpret_cast<uint16_t*>(smem_raw + L.qr);
   uint16_t* sDr = reinterpret_cast<uint16_t*>(smem_raw + L.dr);
-  if constexpr (kTC)
-    block_role_tc<D>(p, b, g, io, sSlot, sKb, sVb, reinterpret_cast<uint16_t*>(smem_raw + L.p),
-                     reinterpret_cast<uint16_t*>(smem_raw + L.ds), sQr, sDr);
-  else
-    block_role_fma<D>(p, b, g, io, stage_rows, sSlot, sKb, sVb, reinterpret_cast<float*>(smem_raw + L.p),
-                      reinterpret_cast<float*>(smem_raw + L.ds), sQr, sDr);
+  block_role_fma<D>(p, b, g, io, stage_rows, sSlot, sKb, sVb, reinterpret_cast<float*>(smem_raw + L.p),
+                    reinterpret_cast<float*>(smem_raw + L.ds), sQr, sDr);
 }
 
 template <int D, bool kBf16Rec, bool kTC>
@@ -1021,19 +1126,6 @@ cudaError_t merge_d(const DevPlan& p, const uint16_t* q, const uint16_t* kb, con
   return merge_launch<D, kBf16Rec, false>(p, q, kb, vb, scale, po, pm, pl, o, o_bf16, lse, s, dest);
 }
 
-template <int D, bool kBf16Rec, bool kTC>
-cudaError_t reduce_launch(const DevPlan& p, const uint16_t* q, const uint16_t* kb, const uint16_t* vb,
-                          const uint16_t* dout, const float* lse, const float* delta, const void* dq_part,
-                          float scale, float* dq, float* dkb, float* dvb, cudaStream_t s, const MergeDest& dest,
-                          int stage_rows, size_t smem) {
-  cudaError_t e = cudaFuncSetAttribute(bwd_reduce_kernel<D, kBf16Rec, kTC>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
-  if (e != cudaSuccess) return e;
-  bwd_reduce_kernel<D, kBf16Rec, kTC><<<dim3(p.A, p.Hkv), kMergeThreads, smem, s>>>(
-      p, q, kb, vb, dout, lse, delta, dq_part, scale, dq, dkb, dvb, stage_rows, dest);
-  return cudaGetLastError();
-}
-
 template <int D, bool kBf16Rec>
 cudaError_t reduce_d(const DevPlan& p, const uint16_t* q, const uint16_t* kb, const uint16_t* vb,
                      const uint16_t* dout, const float* lse, const float* delta, const void* dq_part,
@@ -1041,15 +1133,24 @@ cudaError_t reduce_d(const DevPlan& p, const uint16_t* q, const uint16_t* kb, co
   const int R = p.G * p.bs;
   constexpr size_t kMaxSmem = size_t(227) * 1024;
   // tensor path: rows and block keys in 16s, and its tiles fit in shared memory
-  const size_t tc_smem = reduce_smem(D, p.bs, R, true, true).total;
-  if (R % 16 == 0 && p.bs % 16 == 0 && tc_smem <= kMaxSmem)
-    return reduce_launch<D, kBf16Rec, true>(p, q, kb, vb, dout, lse, delta, dq_part, scale, dq, dkb, dvb, s, dest,
-                                            1, tc_smem);
-  const size_t staged = reduce_smem(D, p.bs, R, false, true).total;
+  const size_t tc_smem = reduce_tc_smem(D, p.bs, R).total;
+  if (R % 16 == 0 && p.bs % 16 == 0 && tc_smem <= kMaxSmem) {
+    cudaError_t e = cudaFuncSetAttribute(bwd_reduce_tc_kernel<D, kBf16Rec>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, int(tc_smem));
+    if (e != cudaSuccess) return e;
+    bwd_reduce_tc_kernel<D, kBf16Rec><<<dim3(p.A, p.Hkv), kMergeThreads, tc_smem, s>>>(
+        p, q, kb, vb, dout, lse, delta, dq_part, scale, dq, dkb, dvb, dest);
+    return cudaGetLastError();
+  }
+  const size_t staged = reduce_smem(D, p.bs, R, true).total;
   const int stage_rows = staged <= size_t(110) * 1024 ? 1 : 0;   // small enough for two CTAs per SM
-  const size_t smem = reduce_smem(D, p.bs, R, false, stage_rows != 0).total;
-  return reduce_launch<D, kBf16Rec, false>(p, q, kb, vb, dout, lse, delta, dq_part, scale, dq, dkb, dvb, s, dest,
-                                           stage_rows, smem);
+  const size_t smem = reduce_smem(D, p.bs, R, stage_rows != 0).total;
+  cudaError_t e = cudaFuncSetAttribute(bwd_reduce_kernel<D, kBf16Rec>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       int(smem));
+  if (e != cudaSuccess) return e;
+  bwd_reduce_kernel<D, kBf16Rec><<<dim3(p.A, p.Hkv), kMergeThreads, smem, s>>>(
+      p, q, kb, vb, dout, lse, delta, dq_part, scale, dq, dkb, dvb, stage_rows, dest);
+  return cudaGetLastError();
 }
 
 }  // namespace
