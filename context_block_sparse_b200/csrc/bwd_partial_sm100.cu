@@ -600,9 +600,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 // ============================================================================
 // dq kernel
 // ============================================================================
+// K goes through a ring of three stages (read by S and by dQ += dS K, so a stage frees
+// late), V through one (read by dP only); the stages' shared memory equals two of each.
+constexpr int kDqKStages = 3;
 struct DqBars {
-  uint64_t qd_full, qd_empty, k_full[2], v_full[2], k_empty[2], v_empty[2], s_ready[2], dp_ready, ds_ready, dq_ready,
-      dq_free, mma_done, meta_ready[2], meta_free[2];
+  uint64_t qd_full, qd_empty, k_full[kDqKStages], v_full, k_empty[kDqKStages], v_empty, s_ready[2], dp_ready,
+      ds_ready, dq_ready, dq_free, mma_done, meta_ready[2], meta_free[2];
   ClaimRing ring;   // run-time claims: producer -> MMA thread, metadata warp, 8 element-wise warps
   uint32_t tmem_base;
   int abort_flag;
@@ -662,8 +665,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   constexpr uint32_t kIdescMN = Dm::kIdescMN;
   uint8_t* sQ = smem;
   uint8_t* sdO = smem + kTile;
-  uint8_t* sK = smem + 2 * kTile;   // [2 stages]
-  uint8_t* sV = smem + 4 * kTile;   // [2 stages]
+  uint8_t* sK = smem + 2 * kTile;   // [kDqKStages stages]
+  uint8_t* sV = smem + (2 + kDqKStages) * kTile;
   DqRow* meta = reinterpret_cast<DqRow*>(smem + Dm::kOffMeta);   // [2][128]
   DqBars* B = reinterpret_cast<DqBars*>(smem + Dm::kOffBars);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -693,20 +696,21 @@ __global__ void __launch_bounds__(kThreads, 1)
       int t, g;
       uint32_t tile_count = 0, kv_count = 0, q_issued = 0, k_issued = 0, v_issued = 0;
       bool ok = true;
-      // key tile c of this CTA: V first (its stage frees once dP has read it), then K
-      // (its stage frees only after dQ += dS K)
+      // key tile c of this CTA, in the order the MMA thread reads them: K (its stage of
+      // three frees after dQ += dS K of key tile c - 3), then V (its one stage frees once
+      // dP of key tile c - 1 has read it)
       auto load_kv = [&](uint32_t c, int k0) -> bool {
-        const int s = int(c & 1);
-        if (!mbar_wait(&B->v_empty[s], ((c >> 1) & 1) ^ 1, wctx, 2 * 10000 + __LINE__)) return false;
-        mbar_expect_tx(&B->v_full[s], kTile);
-        for (int dh = 0; dh < D / 64; ++dh)
-          tma_load_3d(sV + s * kTile + dh * kHalf, &tm_v, &B->v_full[s], dh * 64, g, k0);
-        ++v_issued;
-        if (!mbar_wait(&B->k_empty[s], ((c >> 1) & 1) ^ 1, wctx, 2 * 10000 + __LINE__)) return false;
+        const int s = int(c % kDqKStages);
+        if (!mbar_wait(&B->k_empty[s], ((c / kDqKStages) & 1) ^ 1, wctx, 2 * 10000 + __LINE__)) return false;
         mbar_expect_tx(&B->k_full[s], kTile);
         for (int dh = 0; dh < D / 64; ++dh)
           tma_load_3d(sK + s * kTile + dh * kHalf, &tm_k, &B->k_full[s], dh * 64, g, k0);
         ++k_issued;
+        if (!mbar_wait(&B->v_empty, (c & 1) ^ 1, wctx, 2 * 10000 + __LINE__)) return false;
+        mbar_expect_tx(&B->v_full, kTile);
+        for (int dh = 0; dh < D / 64; ++dh)
+          tma_load_3d(sV + dh * kHalf, &tm_v, &B->v_full, dh * 64, g, k0);
+        ++v_issued;
         return true;
       };
       while (ok && ti.next(t, g)) {
@@ -728,10 +732,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (!ok) *abort_flag = 1;
       if (q_issued > 0) mbar_drain(&B->qd_full, (q_issued - 1) & 1, wctx, 2 * 10000 + __LINE__);
-      for (uint32_t c = k_issued >= 2 ? k_issued - 2 : 0; c < k_issued; ++c)
-        mbar_drain(&B->k_full[c & 1], (c >> 1) & 1, wctx, 2 * 10000 + __LINE__);
-      for (uint32_t c = v_issued >= 2 ? v_issued - 2 : 0; c < v_issued; ++c)
-        mbar_drain(&B->v_full[c & 1], (c >> 1) & 1, wctx, 2 * 10000 + __LINE__);
+      for (uint32_t c = k_issued >= kDqKStages ? k_issued - kDqKStages : 0; c < k_issued; ++c)
+        mbar_drain(&B->k_full[c % kDqKStages], (c / kDqKStages) & 1, wctx, 2 * 10000 + __LINE__);
+      if (v_issued > 0) mbar_drain(&B->v_full, (v_issued - 1) & 1, wctx, 2 * 10000 + __LINE__);
     }
   } else if (warp == 1) {
     if (lane == 0) {
@@ -747,53 +750,54 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!mbar_wait(&B->qd_full, tile_count & 1, wctx, 2 * 10000 + __LINE__)) { ok = false; break; }
         const uint32_t c0 = kv_count;
         {
-          const int s = c0 & 1;
-          if (!mbar_wait(&B->k_full[s], (c0 >> 1) & 1, wctx, 2 * 10000 + __LINE__)) { ok = false; break; }
+          const int s = c0 & 1, ks = int(c0 % kDqKStages);   // S buffer, K stage
+          if (!mbar_wait(&B->k_full[ks], (c0 / kDqKStages) & 1, wctx, 2 * 10000 + __LINE__)) { ok = false; break; }
           tc_fence_after();
           for (int kk = 0; kk < D / 16; ++kk)
-            mma_ss(tmem + s * 128, kmajor(aQ, kk), kmajor(aK + s * kTile, kk), kIdescKM, kk > 0 ? 1u : 0u);
+            mma_ss(tmem + s * 128, kmajor(aQ, kk), kmajor(aK + ks * kTile, kk), kIdescKM, kk > 0 ? 1u : 0u);
           mma_commit(&B->s_ready[s]);
-          if (!mbar_wait(&B->v_full[s], (c0 >> 1) & 1, wctx, 2 * 10000 + __LINE__)) { ok = false; break; }
+          if (!mbar_wait(&B->v_full, c0 & 1, wctx, 2 * 10000 + __LINE__)) { ok = false; break; }
           tc_fence_after();
           for (int kk = 0; kk < D / 16; ++kk)
-            mma_ss(tmem + 256, kmajor(adO, kk), kmajor(aV + s * kTile, kk), kIdescKM, kk > 0 ? 1u : 0u);
+            mma_ss(tmem + 256, kmajor(adO, kk), kmajor(aV, kk), kIdescKM, kk > 0 ? 1u : 0u);
           mma_commit(&B->dp_ready);
-          mma_commit(&B->v_empty[s]);   // V is read by dP only
+          mma_commit(&B->v_empty);   // V is read by dP only
         }
         for (int j = 0; j < n_kt; ++j) {
           const uint32_t c = c0 + j;
-          const int s = c & 1, s1 = (c + 1) & 1;
+          const int s = c & 1, s1 = (c + 1) & 1;   // S buffers
+          const int ks = int(c % kDqKStages), ks1 = int((c + 1) % kDqKStages);   // K stages
           const bool more = j + 1 < n_kt;
           if (more) {   // next S into the other buffer while this tile's dS is formed
-            if (!mbar_wait(&B->k_full[s1], ((c + 1) >> 1) & 1, wctx, 2 * 10000 + __LINE__)) { ok = false; break; }
+            if (!mbar_wait(&B->k_full[ks1], ((c + 1) / kDqKStages) & 1, wctx, 2 * 10000 + __LINE__)) { ok = false; break; }
             tc_fence_after();
             for (int kk = 0; kk < D / 16; ++kk)
-              mma_ss(tmem + s1 * 128, kmajor(aQ, kk), kmajor(aK + s1 * kTile, kk), kIdescKM, kk > 0 ? 1u : 0u);
+              mma_ss(tmem + s1 * 128, kmajor(aQ, kk), kmajor(aK + ks1 * kTile, kk), kIdescKM, kk > 0 ? 1u : 0u);
             mma_commit(&B->s_ready[s1]);
           }
           if (!mbar_wait(&B->ds_ready, ds_cnt & 1, wctx, 2 * 10000 + __LINE__)) { ok = false; break; }
           ++ds_cnt;
+          // the next dP first (the element-wise warps have read this one's dP): their next
+          // pass then waits for one product, not two; dQ += dS K runs during that pass
+          if (more) {
+            if (!mbar_wait(&B->v_full, (c + 1) & 1, wctx, 2 * 10000 + __LINE__)) { ok = false; break; }
+            tc_fence_after();
+            for (int kk = 0; kk < D / 16; ++kk)
+              mma_ss(tmem + 256, kmajor(adO, kk), kmajor(aV, kk), kIdescKM, kk > 0 ? 1u : 0u);
+            mma_commit(&B->dp_ready);
+            mma_commit(&B->v_empty);
+            if (j + 2 == n_kt) mma_commit(&B->qd_empty);   // Q, dO: no further reader after this S / dP
+          }
           if (j == 0) {
             if (!mbar_wait(&B->dq_free, (dqf_cnt & 1) ^ 1, wctx, 2 * 10000 + __LINE__)) { ok = false; break; }
             ++dqf_cnt;
           }
           tc_fence_after();
-          // dQ (cols 384..) += dS K first -- dS in TMEM (columns 0..63 of S buffer s), K
-          // MN-major -- so that K stage s frees one product earlier for the load of key
-          // tile j + 2 (the loads, not the element-wise steps, set the pace), then the next dP
+          // dQ (cols 384..) += dS K -- dS in TMEM (columns 0..63 of S buffer s), K MN-major
           for (int kk = 0; kk < BT / 16; ++kk)
-            mma_ts(tmem + 384, tmem + s * 128 + packed_col(kk), mnmajor(aK + s * kTile, kk), kIdescMN,
+            mma_ts(tmem + 384, tmem + s * 128 + packed_col(kk), mnmajor(aK + ks * kTile, kk), kIdescMN,
                    (j > 0 || kk > 0) ? 1u : 0u);
-          mma_commit(&B->k_empty[s]);   // K is read by S and by dQ += dS K
-          if (more) {
-            if (!mbar_wait(&B->v_full[s1], ((c + 1) >> 1) & 1, wctx, 2 * 10000 + __LINE__)) { ok = false; break; }
-            tc_fence_after();
-            for (int kk = 0; kk < D / 16; ++kk)
-              mma_ss(tmem + 256, kmajor(adO, kk), kmajor(aV + s1 * kTile, kk), kIdescKM, kk > 0 ? 1u : 0u);
-            mma_commit(&B->dp_ready);
-            mma_commit(&B->v_empty[s1]);
-            if (j + 2 == n_kt) mma_commit(&B->qd_empty);   // Q, dO: no further reader after this S / dP
-          }
+          mma_commit(&B->k_empty[ks]);   // K is read by S and by dQ += dS K
         }
         if (!ok) break;
         mma_commit(&B->dq_ready);

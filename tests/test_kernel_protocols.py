@@ -398,34 +398,34 @@ class DKDV(Core):
 
 
 # ---------------------------------------------------------------------------
-# dQ kernel: Q / dO per query tile; K and V rings of two stages each (V released once dP
-# has read it, K after dQ += dS K; V loaded first; a tile's first K/V before its Q / dO);
-# S double-buffered; dQ issued before the next dP
+# dQ kernel: Q / dO per query tile; a K ring of three stages (released after dQ += dS K)
+# and one V stage (released once dP has read it), K loaded before V; a tile's first K/V
+# before its Q / dO; S double-buffered; the next dP issued before dQ
 # ---------------------------------------------------------------------------
 class DQ(Core):
     def __init__(self, tiles, seed, drop=None):
-        names = ["qd_full", "qd_empty", "k_full0", "k_full1", "v_full0", "v_full1", "k_empty0", "k_empty1",
-                 "v_empty0", "v_empty1", "s_ready0", "s_ready1", "dp_ready", "ds_ready", "dq_ready", "dq_free",
+        names = ["qd_full", "qd_empty", "k_full0", "k_full1", "k_full2", "v_full", "k_empty0", "k_empty1",
+                 "k_empty2", "v_empty", "s_ready0", "s_ready1", "dp_ready", "ds_ready", "dq_ready", "dq_free",
                  "meta_ready0", "meta_ready1", "meta_free0", "meta_free1"]
         super().__init__(seed, names)
         self.tiles = tiles
         self.drop = drop
         self.QD = None
-        self.K, self.V, self.S = [None, None], [None, None], [None, None]
+        self.K, self.V, self.S = [None, None, None], [None], [None, None]
         self.DP, self.DQ = None, None
         self.META = [None, None]
 
     def producer(self):
         kv = 0
 
-        def load_kv(c):
-            s = c % 2
-            if c >= 2 and self.drop != "kv_empty":
-                yield from self.wait(f"v_empty{s}", c // 2 - 1)
-            self.load(f"v_full{s}", lambda s=s, c=c: self.V.__setitem__(s, c))
-            if c >= 2 and self.drop != "kv_empty":
-                yield from self.wait(f"k_empty{s}", c // 2 - 1)
+        def load_kv(c):   # K: a ring of three stages; V: one stage
+            s = c % 3
+            if c >= 3 and self.drop != "kv_empty":
+                yield from self.wait(f"k_empty{s}", c // 3 - 1)
             self.load(f"k_full{s}", lambda s=s, c=c: self.K.__setitem__(s, c))
+            if c >= 1 and self.drop != "v_empty":
+                yield from self.wait("v_empty", c - 1)
+            self.load("v_full", lambda c=c: self.V.__setitem__(0, c))
         for n, nkt in enumerate(self.tiles):
             yield from load_kv(kv)
             if n >= 1 and self.drop != "qd_empty":
@@ -452,38 +452,44 @@ class DQ(Core):
 
             def s_mma(c, n=n):
                 def ex(b=c % 2, c=c, n=n):
-                    self.check(self.QD == n and self.K[b] == c, f"S({c}) reads QD {self.QD} K {self.K[b]}")
+                    self.check(self.QD == n and self.K[c % 3] == c, f"S({c}) reads QD {self.QD} K {self.K[c % 3]}")
                     self.check(self.S[b] is None or self.S[b][0] == "read", f"S({c}) overwrites {self.S[b]}")
                     self.S[b] = ("S", c)
                 self.mma(ex)
                 self.commit(f"s_ready{c % 2}")
 
             def dp_mma(c, n=n):
-                def ex(b=c % 2, c=c, n=n):
-                    self.check(self.QD == n and self.V[b] == c, f"dP({c}) reads QD {self.QD} V {self.V[b]}")
+                def ex(c=c, n=n):
+                    self.check(self.QD == n and self.V[0] == c, f"dP({c}) reads QD {self.QD} V {self.V[0]}")
                     self.check(self.DP is None or self.DP[0] == "read", f"dP({c}) overwrites {self.DP}")
                     self.DP = ("dP", c)
                 self.mma(ex)
                 self.commit("dp_ready")
-                self.commit(f"v_empty{c % 2}")
+                self.commit("v_empty")
             c0 = kv
-            yield from self.wait(f"k_full{c0 % 2}", c0 // 2)
+            yield from self.wait(f"k_full{c0 % 3}", c0 // 3)
             s_mma(c0)
-            yield from self.wait(f"v_full{c0 % 2}", c0 // 2)
+            yield from self.wait("v_full", c0)
             dp_mma(c0)
             for j in range(nkt):
                 c = c0 + j
                 more = j + 1 < nkt
                 if more:
-                    yield from self.wait(f"k_full{(c + 1) % 2}", (c + 1) // 2)
+                    yield from self.wait(f"k_full{(c + 1) % 3}", (c + 1) // 3)
                     s_mma(c + 1)
                 yield from self.wait("ds_ready", ds)
                 ds += 1
+                if more:
+                    yield from self.wait("v_full", c + 1)
+                    dp_mma(c + 1)
+                    if j + 2 == nkt:
+                        self.commit("qd_empty")
                 if j == 0 and n >= 1 and self.drop != "dq_free":
                     yield from self.wait("dq_free", n - 1)
 
                 def dq(b=c % 2, c=c, j=j, n=n):
-                    self.check(self.S[b] == ("dS", c) and self.K[b] == c, f"dQ({c}) reads {self.S[b]} K {self.K[b]}")
+                    self.check(self.S[b] == ("dS", c) and self.K[c % 3] == c,
+                               f"dQ({c}) reads {self.S[b]} K {self.K[c % 3]}")
                     if j == 0:
                         self.check(self.DQ is None or self.DQ[0] == "stored", f"dQ overwrites {self.DQ}")
                         self.DQ = ("acc", n, 1)
@@ -492,12 +498,7 @@ class DQ(Core):
                         self.DQ = ("acc", n, j + 1)
                     self.S[b] = ("read", c)
                 self.mma(dq)
-                self.commit(f"k_empty{c % 2}")
-                if more:
-                    yield from self.wait(f"v_full{(c + 1) % 2}", (c + 1) // 2)
-                    dp_mma(c + 1)
-                    if j + 2 == nkt:
-                        self.commit("qd_empty")
+                self.commit(f"k_empty{c % 3}")
             self.commit("dq_ready")
             if nkt == 1:
                 self.commit("qd_empty")
@@ -628,8 +629,8 @@ def test_protocol_holds_on_random_schedules(kernel):
 @pytest.mark.parametrize("kernel,drop", [("forward", "kv_empty"), ("forward", "q_empty"), ("forward", "o_free"),
                                          ("forward", "stats"),
                                          ("dkdv", "qd_empty"),
-                                         ("dkdv", "kv_empty"), ("dkdv", "lookahead_before_dv"), ("dq", "kv_empty"),
-                                         ("dq", "qd_empty"), ("reduce", "empty")])
+                                         ("dkdv", "kv_empty"), ("dkdv", "lookahead_before_dv"),
+                                         ("dq", "kv_empty"), ("dq", "v_empty"), ("reduce", "empty")])
 def test_each_producer_guard_is_needed(kernel, drop):
     """Removing one of the producer's waits lets some schedule overwrite a stage that an
     MMA has not read yet; issuing the dK/dV kernel's look-ahead S^T before dV instead of
@@ -645,13 +646,16 @@ def test_each_producer_guard_is_needed(kernel, drop):
     assert caught > 0
 
 
-@pytest.mark.parametrize("kernel,drop", [("dkdv", "dkv_free"), ("dq", "dq_free")])
-def test_epilogue_release_is_implied_by_program_order(kernel, drop):
-    """In the backward kernels the MMA thread's wait for the epilogue to release an
-    accumulator is redundant: the epilogue runs on the element-wise warps before their next
-    pass, which the first product into the accumulator already waits for.  The kernels keep
-    the wait as a guard; these schedules show that nothing depends on it.  (The forward's
-    epilogue runs on warps of its own, so there the wait is needed: see above.)"""
+@pytest.mark.parametrize("kernel,drop", [("dkdv", "dkv_free"), ("dq", "dq_free"), ("dq", "qd_empty")])
+def test_guard_is_implied_by_program_order(kernel, drop):
+    """Some waits are redundant, kept as guards; these schedules show that nothing depends
+    on them.  In the backward kernels the MMA thread's wait for the epilogue to release an
+    accumulator: the epilogue runs on the element-wise warps before their next pass, which
+    the first product into the accumulator already waits for.  (The forward's epilogue runs
+    on warps of its own, so there the wait is needed: see above.)  In the dQ kernel the
+    producer's wait for the Q / dO buffer: it loads a tile's Q / dO only after the single
+    V stage was released by the previous tile's last dP, which the tensor pipe executes
+    after the last products reading Q / dO."""
     rng = random.Random(6)
     for seed in range(150):
         CASES[kernel](rng, seed, drop).go()
