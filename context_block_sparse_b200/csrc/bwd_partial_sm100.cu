@@ -26,15 +26,17 @@
 //      dQ += dS K                           (A operand from TMEM)
 //    then scale * dQ is written once as the (chunk, block) entry's dq partial.
 //
-// Roles per CTA (384 threads): warp 0 TMA producer, warp 1 MMA issuer (one
-// thread), warp 2 tensor-memory allocation, warp 3 prefetches the row
-// metadata of upcoming query tiles into shared memory, warps 4-11 element-wise work and
-// epilogue in two warpgroups that split the 128 columns of every tile between
-// them (thread = TMEM lane; warpgroup h takes columns 64h..64h+63).  Each
-// warpgroup writes its bf16 results into its own columns (the MMA addresses the
-// 16-wide K-steps one by one), so neither overwrites scores the other has not
-// read yet.  Waits are bounded; a timeout is recorded in the plan's status word
-// and every role winds down.
+// Roles per CTA: warp 0 TMA producer, warp 1 MMA issuer (one thread), warp 2
+// tensor-memory allocation, warp 3 prefetches the row metadata of upcoming query
+// tiles into shared memory, warps 4-11 element-wise work in two warpgroups that
+// split the 128 columns of every tile between them (thread = TMEM lane; warpgroup
+// h takes columns 64h..64h+63).  Each warpgroup writes its bf16 results into its
+// own columns (the MMA addresses the 16-wide K-steps one by one), so neither
+// overwrites scores the other has not read yet.  The dK/dV kernel (384 threads)
+// writes dK, dV from the element-wise warps after each key tile; the dQ kernel
+// (512 threads) has warps 12-15 of its own for the dq-partial epilogue, so the
+// element-wise warps go on with the next query tile meanwhile.  Waits are bounded;
+// a timeout is recorded in the plan's status word and every role winds down.
 #include <cfloat>
 #include <cstring>
 
@@ -54,8 +56,9 @@ constexpr uint32_t kIdescKM = idesc_bf16_f32(128, 128, 0);  // B K-major
 
 // Sizes that follow the head dimension D (64 or 128): a 128-row bf16 tile of D
 // columns is D / 64 halves of 16 KB; the products into dK, dV, dQ have N = D.
-// Shared memory: 6 tiles | row metadata (8 KB) | epilogue scratch (2 KB per
-// element-wise warp) | barriers.
+// Shared memory: 6 tiles | row metadata (8 KB) | epilogue scratch (8 x 2 KB: one
+// per element-wise warp of the dK/dV kernel, one per epilogue warp of the dQ
+// kernel) | barriers.
 template <int D>
 struct Dims {
   static_assert(D == 64 || D == 128, "head dimension");
@@ -611,6 +614,10 @@ struct DqBars {
   int abort_flag;
 };
 constexpr int kDqNumBars = 21;
+// dQ kernel roles (512 threads): warps 0-3 as in the dK/dV kernel, 4-11 element-wise,
+// 12-15 the dq-partial epilogue; claim-ring consumers: MMA thread, warp 3, warps 4-15
+constexpr int kDqThreads = 512;
+constexpr uint32_t kDqClaimConsumers = 1 + 1 + 8 + 4;
 static_assert(sizeof(DqBars) <= 256, "barrier block");
 
 // Per-row metadata of a query tile for the dq kernel (shared memory).
@@ -653,7 +660,7 @@ struct TileIter {
 };
 
 template <int D>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kDqThreads, 1)
     bwd_dq_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_do,
                         const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                         const __grid_constant__ CUtensorMap tm_dq, DevPlan p, const float* __restrict__ lse,
@@ -679,8 +686,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   {
     // commits count 1; element-wise / metadata signals count warps (warp_arrive)
-    const uint32_t counts[kDqNumBars] = {1, 1, 1, 1, 1, 1, 1, 1, 1, 1, 1, 1, 1, 8, 1, 8, 1, 1, 1, 8, 8};
-    if (tid == 0) claim_ring_init(&B->ring, kClaimConsumers);
+    const uint32_t counts[kDqNumBars] = {1, 1, 1, 1, 1, 1, 1, 1, 1, 1, 1, 1, 1, 8, 1, 4, 1, 1, 1, 8, 8};
+    if (tid == 0) claim_ring_init(&B->ring, kDqClaimConsumers);
     setup_common(&B->qd_full, kDqNumBars, counts, &B->tmem_base, warp);
   }
   const uint32_t tmem = B->tmem_base;
@@ -840,18 +847,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       ++mcount;
     }
     if (!ok) *abort_flag = 1;
-  } else if (warp >= 4) {
+  } else if (warp >= 4 && warp < 12) {
     const int hf = (warp - 4) >> 2;           // warpgroup: keys 64hf..64hf+63 of every key tile
-    const int r = ((warp & 3) << 5) + lane;
     const uint32_t lane_addr = uint32_t((warp & 3) << 5) << 16;
     const uint32_t tdP = tmem + lane_addr + 256;
-    constexpr int kHalfD = D / 2;                            // dQ columns per warpgroup
-    const uint32_t tdQ = tmem + lane_addr + 384 + hf * kHalfD;   // this warpgroup's dQ columns
+    const int r = ((warp & 3) << 5) + lane;
     const float scale_log2 = scale * kLog2e;
     TileIter ti;
     ti.init(&p, w, &B->ring, kClaimWarp, &wctx);
     int t, g;
-    uint32_t kv_count = 0, dp_cnt = 0, dq_cnt = 0, mcount = 0;
+    uint32_t kv_count = 0, dp_cnt = 0, mcount = 0;
     bool ok = true;
     while (ok && ti.next(t, g)) {
       const int4 tile = p.tiles[t];
@@ -883,53 +888,75 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (!ok) break;
       kv_count += n_kt;
+    }
+    if (!ok) *abort_flag = 1;
+  } else if (warp >= 12) {
+    // epilogue warps 12-15: warp 12 + q stores rows 32q..32q+31 (TMEM lanes) of each
+    // tile's dQ, all D columns, as the (chunk, block) entries' dq partials; dQ is
+    // released to the MMA thread after its last TMEM read
+    const int r = ((warp & 3) << 5) + lane;
+    const uint32_t tdQ = tmem + (uint32_t((warp & 3) << 5) << 16) + 384;
+    float* scratch = reinterpret_cast<float*>(smem + Dm::kOffScratch) + (warp - 12) * 512;
+    TileIter ti;
+    ti.init(&p, w, &B->ring, kClaimWarp, &wctx);
+    int t, g;
+    uint32_t dq_cnt = 0;
+    bool ok = true;
+    while (ok && ti.next(t, g)) {
+      const int4 tile = p.tiles[t];
+      const RowMeta m = row_meta(p, tile, g, r);
       if (!warp_wait(&B->dq_ready, dq_cnt & 1, wctx, 2 * 10000 + __LINE__)) { ok = false; break; }
       ++dq_cnt;
       tc_fence_after();
-      float* scratch = reinterpret_cast<float*>(smem + Dm::kOffScratch) + (warp - 4) * 512;
+      // the warp's 32 rows are 32/G whole tokens of one block, all G heads of KV head g
+      // (valid is warp-uniform when bulk stores are used)
+      const int z0 = __shfl_sync(0xffffffffu, m.valid ? m.rec / p.Hq : 0, 0);
+      const bool wv = __shfl_sync(0xffffffffu, m.valid ? 1 : 0, 0) != 0;
       if (p.partial_bf16) {
-        // bf16 dq partials: 32-column chunks of this warpgroup's D / 2 columns
-        const int z0 = __shfl_sync(0xffffffffu, m.valid ? m.rec / p.Hq : 0, 0);
-        const bool wv = __shfl_sync(0xffffffffu, m.valid ? 1 : 0, 0) != 0;
 #pragma unroll 1
-        for (int cc = 0; cc < kHalfD / 32; ++cc) {
+        for (int cc = 0; cc < D / 32; ++cc) {
           uint32_t v[32];
           tmem_ld32(tdQ + cc * 32, v);
           tmem_wait_ld();
           reg_fence<32>(v);
+          if (cc == D / 32 - 1) {   // dQ read: the next tile's first dQ += dS K may start
+            tc_fence_before();
+            warp_arrive(&B->dq_free);
+          }
           if (bulk)
-            warp_bulk_store32_bf16<0>(scratch, v, scale, &tm_dq, hf * kHalfD + cc * 32, g * p.G, z0, wv);
+            warp_bulk_store32_bf16<0>(scratch, v, scale, &tm_dq, cc * 32, g * p.G, z0, wv);
           else if (m.valid)
-            lane_store32_bf16(static_cast<uint16_t*>(dq_part) + size_t(m.rec) * D + hf * kHalfD + cc * 32, v,
-                              scale);
+            lane_store32_bf16(static_cast<uint16_t*>(dq_part) + size_t(m.rec) * D + cc * 32, v, scale);
           __syncwarp();   // m.valid differs across the warp's rows: converge before the next tcgen05.ld
         }
       } else if (bulk) {
-        // the warp's 32 rows are 32/G whole tokens of one block, all G heads of KV
-        // head g (valid is warp-uniform): bulk tensor stores of 32 x 16 boxes
-        const int z0 = __shfl_sync(0xffffffffu, m.valid ? m.rec / p.Hq : 0, 0);
-        const bool wv = __shfl_sync(0xffffffffu, m.valid ? 1 : 0, 0) != 0;
 #pragma unroll 1
-        for (int cc = 0; cc < kHalfD / 16; ++cc) {
+        for (int cc = 0; cc < D / 16; ++cc) {
           uint32_t v[16];
           tmem_ld16(tdQ + cc * 16, v);
           tmem_wait_ld();
           reg_fence<16>(v);
-          warp_bulk_store16<0>(scratch, v, scale, &tm_dq, hf * kHalfD + cc * 16, g * p.G, z0, wv);
+          if (cc == D / 16 - 1) {
+            tc_fence_before();
+            warp_arrive(&B->dq_free);
+          }
+          warp_bulk_store16<0>(scratch, v, scale, &tm_dq, cc * 16, g * p.G, z0, wv);
         }
       } else {
-        float* dst = static_cast<float*>(dq_part) + size_t(m.rec) * D + hf * kHalfD;
+        float* dst = static_cast<float*>(dq_part) + size_t(m.rec) * D;
 #pragma unroll 1
-        for (int cc = 0; cc < kHalfD / 16; ++cc) {
+        for (int cc = 0; cc < D / 16; ++cc) {
           uint32_t v[16];
           tmem_ld16(tdQ + cc * 16, v);
           tmem_wait_ld();
           reg_fence<16>(v);
+          if (cc == D / 16 - 1) {
+            tc_fence_before();
+            warp_arrive(&B->dq_free);
+          }
           warp_store_rows<16>(scratch, reinterpret_cast<const float*>(v), scale, m.valid ? dst + cc * 16 : nullptr);
         }
       }
-      tc_fence_before();
-      warp_arrive(&B->dq_free);
     }
     // bulk stores of this warp complete before the CTA exits
     if (lane == 0) bulk_wait0();
@@ -986,7 +1013,7 @@ cudaError_t launch_bwd_sm100(const DevPlan& p, const uint16_t* q, const uint16_t
   }
   if (which != 1) {
     if (p.dynamic && (e = cudaMemsetAsync(p.claim + 2, 0, sizeof(int), s)) != cudaSuccess) return e;
-    bwd_dq_sm100_kernel<D><<<p.W, kThreads, kSmem, s>>>(tq, tdo, tk, tv, tdq, p, lse, delta, scale,
+    bwd_dq_sm100_kernel<D><<<p.W, kDqThreads, kSmem, s>>>(tq, tdo, tk, tv, tdq, p, lse, delta, scale,
                                                         bulk_dq ? 1 : 0, dq_part);
     e = cudaGetLastError();
   }

@@ -400,7 +400,8 @@ class DKDV(Core):
 # ---------------------------------------------------------------------------
 # dQ kernel: Q / dO per query tile; a K ring of three stages (released after dQ += dS K)
 # and one V stage (released once dP has read it), K loaded before V; a tile's first K/V
-# before its Q / dO; S double-buffered; the next dP issued before dQ
+# before its Q / dO; S double-buffered; the next dP issued before dQ; dQ read and
+# released by epilogue warps of its own
 # ---------------------------------------------------------------------------
 class DQ(Core):
     def __init__(self, tiles, seed, drop=None):
@@ -523,6 +524,9 @@ class DQ(Core):
                 self.DP = ("read", c)
                 self.B["ds_ready"].arrive()
             kv += nkt
+
+    def epilogue(self):   # warps of its own: reads dQ, releases it, then stores
+        for n, nkt in enumerate(self.tiles):
             yield from self.wait("dq_ready", n)
             self.check(self.DQ == ("acc", n, nkt), f"epilogue {n} finds {self.DQ}")
             yield
@@ -530,7 +534,8 @@ class DQ(Core):
             self.B["dq_free"].arrive()
 
     def go(self):
-        self.run({"prod": self.producer(), "mma": self.mma_thread(), "ew": self.elementwise(), "meta": self.meta()})
+        self.run({"prod": self.producer(), "mma": self.mma_thread(), "ew": self.elementwise(), "meta": self.meta(),
+                  "epi": self.epilogue()})
 
 
 # ---------------------------------------------------------------------------
@@ -630,12 +635,14 @@ def test_protocol_holds_on_random_schedules(kernel):
                                          ("forward", "stats"),
                                          ("dkdv", "qd_empty"),
                                          ("dkdv", "kv_empty"), ("dkdv", "lookahead_before_dv"),
-                                         ("dq", "kv_empty"), ("dq", "v_empty"), ("reduce", "empty")])
+                                         ("dq", "kv_empty"), ("dq", "v_empty"), ("dq", "dq_free"),
+                                         ("reduce", "empty")])
 def test_each_producer_guard_is_needed(kernel, drop):
     """Removing one of the producer's waits lets some schedule overwrite a stage that an
     MMA has not read yet; issuing the dK/dV kernel's look-ahead S^T before dV instead of
     after it overwrites a P^T that dV has not read; without the forward MMA's wait for the
-    epilogue warps to release O, the next pair's first PV overwrites an O not yet read."""
+    epilogue warps to release O, the next pair's first PV overwrites an O not yet read (and
+    likewise the dQ kernel's next tile's first dQ += dS K)."""
     rng = random.Random(5)
     caught = 0
     for seed in range(300):
@@ -646,13 +653,14 @@ def test_each_producer_guard_is_needed(kernel, drop):
     assert caught > 0
 
 
-@pytest.mark.parametrize("kernel,drop", [("dkdv", "dkv_free"), ("dq", "dq_free"), ("dq", "qd_empty")])
+@pytest.mark.parametrize("kernel,drop", [("dkdv", "dkv_free"), ("dq", "qd_empty")])
 def test_guard_is_implied_by_program_order(kernel, drop):
     """Some waits are redundant, kept as guards; these schedules show that nothing depends
-    on them.  In the backward kernels the MMA thread's wait for the epilogue to release an
-    accumulator: the epilogue runs on the element-wise warps before their next pass, which
-    the first product into the accumulator already waits for.  (The forward's epilogue runs
-    on warps of its own, so there the wait is needed: see above.)  In the dQ kernel the
+    on them.  In the dK/dV kernel the MMA thread's wait for the epilogue to release the
+    accumulators: the epilogue runs on the element-wise warps before their next pass, which
+    the first product into an accumulator already waits for.  (The forward's and the dQ
+    kernel's epilogues run on warps of their own, so there the wait is needed: see above.)
+    In the dQ kernel the
     producer's wait for the Q / dO buffer: it loads a tile's Q / dO only after the single
     V stage was released by the previous tile's last dP, which the tensor pipe executes
     after the last products reading Q / dO."""
