@@ -448,7 +448,9 @@ def run_ours(args, world, rank, local):
         result["split_kv_ranks"] = {"lpt_ownership": lpt, "contiguous_ownership": con,
                                     "step_ms_contiguous_over_lpt": step(con) / step(lpt)}
     if not args.no_e2e:
-        result["e2e"] = run_e2e(args, w, plan, dev, stream, flops_step, world=world)
+        result["e2e"] = run_e2e(args, w, plan, dev, stream, flops_step, world=world, out_bf16=True)
+        e32 = run_e2e(args, w, plan, dev, stream, flops_step, world=world, out_bf16=False)
+        result["e2e"]["f32_outputs"] = {k: e32[k] for k in ("value", "ms_per_step", "d2h_bytes_per_step")}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         def gpu_rows(rows):
             idx = torch.as_tensor(rows, device=dev)
@@ -660,10 +662,12 @@ def rank_emulation_report(skv, w, args, R, dev, stream, t, W, Wb, peaks, reps=5,
     }
 
 
-def run_e2e(args, w, plan, dev, stream, flops_step, world=1):
+def run_e2e(args, w, plan, dev, stream, flops_step, world=1, out_bf16=True):
     """Same metric through the public API from pinned HOST buffers: every step copies its inputs in and
     its results (o, lse, dq, dk, dv, dkb, dvb) out inside the timed region, the copies overlapping the
-    computation of the neighbouring steps (two device buffer sets, one stream per copy direction)."""
+    computation of the neighbouring steps (two device buffer sets, one stream per copy direction).
+    out_bf16: o and the gradients come back as bf16 (the kernels accumulate in fp32; o is stored as
+    bf16 by the merge, the gradients rounded on the GPU by splitkv_cast_bf16), lse as fp32."""
     import torch
     import torch.distributed as dist
 
@@ -683,10 +687,11 @@ def run_e2e(args, w, plan, dev, stream, flops_step, world=1):
     # streams of their own (the two PCIe directions run at once)
     dvs = [{n: torch.empty(x.shape, dtype=x.dtype, device=dev) for n, x in host.items()} for _ in range(2)]
     f32 = dict(dtype=torch.float32, device=dev)
-    outs_d = [{"o": torch.empty((Nq, Hq, d), **f32), "lse": torch.empty((Nq, Hq), **f32),
-               **{"d" + n: torch.empty(host[n].shape, **f32) for n in ("q", "k", "v", "kb", "vb")}}
+    odt = torch.bfloat16 if out_bf16 else torch.float32
+    outs_d = [{"o": torch.empty((Nq, Hq, d), dtype=odt, device=dev), "lse": torch.empty((Nq, Hq), **f32),
+               **{"d" + n: torch.empty(host[n].shape, dtype=odt, device=dev) for n in ("q", "k", "v", "kb", "vb")}}
               for _ in range(2)]
-    outs_h = {n: torch.empty(x.shape, dtype=torch.float32).pin_memory() for n, x in outs_d[0].items()}
+    outs_h = {n: torch.empty(x.shape, dtype=x.dtype).pin_memory() for n, x in outs_d[0].items()}
     h2d = sum(x.numel() * x.element_size() for x in host.values()) + 4 * (w.sample_lens.size + w.anchors.size)
     d2h = sum(x.numel() * x.element_size() for x in outs_h.values())
     steps = max(1, min(args.steps, args.e2e_steps))
@@ -715,7 +720,7 @@ def run_e2e(args, w, plan, dev, stream, flops_step, world=1):
         att.plan.upload(stream)
         o, lse = att.forward(x["q"], x["k"], x["v"], x["kb"], x["vb"], w.scale, o=y["o"], lse=y["lse"])
         att.backward(x["q"], x["k"], x["v"], x["kb"], x["vb"], o, lse, x["dout"], w.scale,
-                     grads={n: y[n] for n in ("dq", "dk", "dv", "dkb", "dvb")})
+                     grads={n: y[n] for n in ("dq", "dk", "dv", "dkb", "dvb")}, grad_dtype=odt)
         computed[b] = ev()
         computed[b].record(stream)
         # results: down while the next step computes
@@ -747,7 +752,9 @@ def run_e2e(args, w, plan, dev, stream, flops_step, world=1):
         dist.barrier()
     return {"value": whole_job_tflops(world, steps, flops_step, ms), "unit": "TFLOP/s",
             "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "steps": steps,
-            "ms_per_step": ms / steps}
+            "ms_per_step": ms / steps,
+            "outputs": ("bf16 o, dq, dk, dv, dkb, dvb (fp32 accumulation, rounded on the GPU); fp32 lse"
+                        if out_bf16 else "fp32 o, lse, dq, dk, dv, dkb, dvb")}
 
 
 # ---------------------------------------------------------------------------

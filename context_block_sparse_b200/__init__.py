@@ -462,6 +462,16 @@ def splitkv_sum_ranks(parts, out, stream=None) -> None:
     _check("splitkv_sum_ranks", _lib.splitkv_sum_ranks(R, n, _f32_ptr(parts), _f32_ptr(out), _stream_ptr(stream)))
 
 
+def splitkv_cast_bf16(src, dst, stream=None) -> None:
+    """dst (bfloat16) = src (float32) rounded to nearest even, element by element."""
+    import torch
+    if src.dtype != torch.float32 or dst.dtype != torch.bfloat16:
+        raise ValueError("src must be float32 and dst bfloat16")
+    if src.numel() != dst.numel() or not src.is_contiguous() or not dst.is_contiguous():
+        raise ValueError("src and dst must be contiguous with the same number of elements")
+    _check("splitkv_cast_bf16", _lib.splitkv_cast_bf16(int(src.numel()), _ptr(src), _ptr(dst), _stream_ptr(stream)))
+
+
 def splitkv_selftest_wait_timeout(stream=None):
     """Run the bounded-wait self-test; returns the status words (code, site) it recorded."""
     out = (ctypes.c_int32 * 2)()

@@ -111,6 +111,7 @@ SIGNATURES = {
     "splitkv_bwd_reduce_to_owners": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _F, _P, _SZ, ctypes.c_int32,
                                           ctypes.c_int32, _P, _P]),
     "splitkv_sum_ranks": (_I, [ctypes.c_int32, ctypes.c_int64, _P, _P, _P]),
+    "splitkv_cast_bf16": (_I, [ctypes.c_int64, _P, _P, _P]),
     "splitkv_enable_peer_access": (_I, [ctypes.c_int32]),
     "splitkv_plan_upload": (_I, [_P, _P]),
     "splitkv_plan_destroy": (_I, [_P]),

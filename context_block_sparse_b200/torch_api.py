@@ -12,7 +12,7 @@ from typing import Optional
 import torch
 
 from . import (
-    WS_BWD, WS_FWD, Plan, splitkv_attn_bwd, splitkv_attn_fwd, splitkv_merge, splitkv_plan,
+    WS_BWD, WS_FWD, Plan, splitkv_attn_bwd, splitkv_attn_fwd, splitkv_cast_bf16, splitkv_merge, splitkv_plan,
     splitkv_plan_upload, splitkv_workspace_size,
 )
 
@@ -47,6 +47,7 @@ class SplitKVAttention:
         self.head_dim = head_dim
         self.ws_fwd = torch.empty(splitkv_workspace_size(self.plan, WS_FWD), dtype=torch.uint8, device=self.device)
         self._ws_bwd = None
+        self._grad32 = None   # float32 gradients behind bf16 ones (grad_dtype=torch.bfloat16)
 
     def ws_bwd(self) -> torch.Tensor:
         if self._ws_bwd is None:
@@ -64,16 +65,34 @@ class SplitKVAttention:
         splitkv_merge(self.plan, q, kb, vb, scale, self.ws_fwd, o, lse)
         return o, lse
 
-    def backward(self, q, k, v, kb, vb, o, lse, dout, scale: float, grads=None):
+    def _grad_buffers(self, q, k, v, kb, vb, dtype):
+        a = dict(dtype=dtype, device=q.device)
+        return {
+            "dq": torch.empty(q.shape, **a),
+            "dk": torch.empty(k.shape, **a),
+            "dv": torch.empty(v.shape, **a),
+            "dkb": None if self.block_keys_in_context else torch.empty(kb.shape, **a),
+            "dvb": None if self.block_keys_in_context else torch.empty(vb.shape, **a),
+        }
+
+    def backward(self, q, k, v, kb, vb, o, lse, dout, scale: float, grads=None, grad_dtype=torch.float32):
+        """Gradients dq, dk, dv (and dkb, dvb).  grad_dtype=torch.bfloat16 returns them in bf16:
+        the kernels still accumulate in fp32 (into buffers kept by this object), and
+        splitkv_cast_bf16 rounds the finished arrays."""
+        if grad_dtype not in (torch.float32, torch.bfloat16):
+            raise ValueError("grad_dtype must be torch.float32 or torch.bfloat16")
         if grads is None:
-            f32 = dict(dtype=torch.float32, device=q.device)
-            grads = {
-                "dq": torch.empty(q.shape, **f32),
-                "dk": torch.empty(k.shape, **f32),
-                "dv": torch.empty(v.shape, **f32),
-                "dkb": None if self.block_keys_in_context else torch.empty(kb.shape, **f32),
-                "dvb": None if self.block_keys_in_context else torch.empty(vb.shape, **f32),
-            }
-        splitkv_attn_bwd(self.plan, q, k, v, kb, vb, o, lse, dout, grads["dq"], grads["dk"], grads["dv"],
-                         grads["dkb"], grads["dvb"], scale, self.ws_bwd())
+            grads = self._grad_buffers(q, k, v, kb, vb, grad_dtype)
+        if grad_dtype == torch.float32:
+            g32 = grads
+        else:
+            if self._grad32 is None or self._grad32["dq"].shape != q.shape or self._grad32["dk"].shape != k.shape:
+                self._grad32 = self._grad_buffers(q, k, v, kb, vb, torch.float32)
+            g32 = self._grad32
+        splitkv_attn_bwd(self.plan, q, k, v, kb, vb, o, lse, dout, g32["dq"], g32["dk"], g32["dv"],
+                         g32["dkb"], g32["dvb"], scale, self.ws_bwd())
+        if grad_dtype == torch.bfloat16:
+            for n, t in grads.items():
+                if t is not None:
+                    splitkv_cast_bf16(g32[n], t)
         return grads

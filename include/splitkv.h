@@ -483,6 +483,17 @@ int splitkv_enable_peer_access(int32_t peer_device);
 int splitkv_combine_ranks(int32_t num_ranks, int64_t rows, int32_t head_dim, const float* o_parts,
                           const float* lse_parts, void* o, int o_dtype, float* lse, void* stream);
 
+/* Conversion of a finished float32 result array (o, dq, dk, dv, dkb, dvb) to
+ * bfloat16, round to nearest even: dst[i] = bf16(src[i]) for i < n.  The pages
+ * have no counterpart: the method's arithmetic is unchanged (it computes and
+ * accumulates in fp32); this halves the bytes of results a caller keeps in bf16,
+ * e.g. gradients copied back to the host.  src (float32) and dst (bfloat16, as
+ * uint16) are DEVICE arrays of n elements owned by the caller, not overlapping;
+ * 16-byte aligned pointers take the vector path, others an element-wise one.
+ * Asynchronous on `stream`.  Errors: INVALID_ARG (n < 0 or above 2^42, NULL
+ * pointer with n > 0), CUDA (launch failure). */
+int splitkv_cast_bf16(int64_t n, const float* src, uint16_t* dst, void* stream);
+
 /* Sum of the ranks' shares: out[i] = sum_r parts[r * n + i], ranks added in
  * ascending order (the dq of Split-KV over ranks: every rank's dq share of the
  * rows a rank owns).  parts [R][n] and out [n] float32, 16-byte aligned, n a

@@ -90,3 +90,12 @@ def test_bindings_check_tensor_sizes_against_the_plan(splitkv):
     splitkv.splitkv_plan_update(plan, [300, 300], [10, 250, 400])
     with pytest.raises(ValueError, match="k has"):
         splitkv.splitkv_attn_fwd(plan, q, k, v, 0.1, ws)
+
+
+def test_cast_bf16_rejects_bad_arguments_on_the_host(splitkv):
+    """splitkv_cast_bf16 checks its size and pointers before any CUDA call."""
+    lib = splitkv._lib
+    assert lib.splitkv_cast_bf16(-1, None, None, None) == splitkv._abi.ERR_INVALID_ARG
+    assert lib.splitkv_cast_bf16(4, None, None, None) == splitkv._abi.ERR_INVALID_ARG
+    assert lib.splitkv_cast_bf16(1 << 43, 16, 16, None) == splitkv._abi.ERR_INVALID_ARG
+    assert lib.splitkv_cast_bf16(0, None, None, None) == splitkv._abi.OK   # nothing to do
