@@ -52,10 +52,16 @@ NCU_TRAFFIC = {
     # dram__bytes_read.sum + dram__bytes_write.sum of one launch at the 64k / 8k fwd+bwd
     # workload (ncu --clock-control none, one pass), with a hash of the kernel's sources at
     # the capture: a kernel whose sources changed since reports traffic null
-    "fwd_partial": {"bytes": 926102528 + 1152824576, "src": "5960367354c328d5"},
-    "bwd_dkdv": {"bytes": 1137947904 + 486652928, "src": "4aac18d0056134d0"},
-    "bwd_dq": {"bytes": 1161585920 + 1140958464, "src": "4aac18d0056134d0"},
+    "fwd_partial": {"bytes": 926116864 + 1154541568, "src": "f9c145e1db5443a1"},
+    "bwd_dkdv": {"bytes": 1206263552 + 487801856, "src": "3b45b20da4cc6420"},
+    "bwd_dq": {"bytes": 1162170112 + 1140885248, "src": "3b45b20da4cc6420"},
+    "merge": {"bytes": 1430378752 + 126864896, "src": "650d9add59a164a1"},
+    "bwd_reduce": {"bytes": 1365891072 + 188002560, "src": "650d9add59a164a1"},
+    "bwd_delta": {"bytes": 201351424 + 736768, "src": "650d9add59a164a1"},
 }
+# the workload and schedule the figures were taken on (bench.py's defaults)
+NCU_TRAFFIC_CONFIG = {"workload": "bwd", "anchors": None, "schedule": "lpt", "lpt_cost": "tiles",
+                      "fwd_lpt_cost": "pairs", "q_slice": 2, "partial_bf16": False, "claims": "run-time"}
 _KERNEL_SOURCES = {
     "fwd_partial": ("fwd_partial_sm100.cu", "sm100.cuh", "splitkv_internal.h"),
     "bwd_dkdv": ("bwd_partial_sm100.cu", "sm100.cuh", "splitkv_internal.h"),
@@ -386,7 +392,8 @@ def run_ours(args, world, rank, local):
     bound, amount = work[dom]
     dom_s = per_kernel[dom] * 1e-3
     tr = NCU_TRAFFIC.get(dom)
-    traffic = tr["bytes"] if tr and tr.get("src") == _src_hash(dom) else None
+    same_config = all(getattr(args, k) == v for k, v in NCU_TRAFFIC_CONFIG.items())
+    traffic = tr["bytes"] if tr and same_config and tr.get("src") == _src_hash(dom) else None
     if bound == "tensor":
         achieved = amount / dom_s / 1e12
         roof = {"kernel": dom, "bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"],
