@@ -53,8 +53,8 @@ NCU_TRAFFIC = {
     # workload (ncu --clock-control none, one pass), with a hash of the kernel's sources at
     # the capture: a kernel whose sources changed since reports traffic null
     "fwd_partial": {"bytes": 926116864 + 1154541568, "src": "f9c145e1db5443a1"},
-    "bwd_dkdv": {"bytes": 1206263552 + 487801856, "src": "3b45b20da4cc6420"},
-    "bwd_dq": {"bytes": 1162170112 + 1140885248, "src": "3b45b20da4cc6420"},
+    "bwd_dkdv": {"bytes": 1148916992 + 486914048, "src": "981b70cc1d42b122"},
+    "bwd_dq": {"bytes": 1159078656 + 1141427968, "src": "981b70cc1d42b122"},
     "merge": {"bytes": 1430378752 + 126864896, "src": "650d9add59a164a1"},
     "bwd_reduce": {"bytes": 1365891072 + 188002560, "src": "650d9add59a164a1"},
     "bwd_delta": {"bytes": 201351424 + 736768, "src": "650d9add59a164a1"},

@@ -144,6 +144,10 @@ __device__ __forceinline__ void setup_common(uint64_t* bars, int nbars, const ui
   tc_fence_after();
 }
 
+// The dQ pass takes one exponential pair in eight on the FMA-pipe polynomial (measured:
+// 1/8 and all-MUFU ~2 % faster than the dK/dV pass's one in four, one in two 5 % slower).
+constexpr int kPolyEveryDq = 8;
+
 // dq kernel, half hf of one key tile for one row (thread = TMEM lane): dS =
 // P (dP - Delta) with P = exp2(s * c - lse2), zero outside the row's columns
 // [a, b) of the tile; bf16 pairs of dS go to packed_col() of the score buffer.
@@ -165,7 +169,7 @@ __device__ __forceinline__ void ds_tile(uint32_t tS, uint32_t tdP, int hf, int a
       float x0, x1, d0, d1, g0, g1;
       ffma2(x0, x1, __uint_as_float(sv[2 * i]), __uint_as_float(sv[2 * i + 1]), c, c, -l2, -l2);
       float p0, p1;
-      exp2_pair((i % kPolyEvery) == 1, x0, x1, p0, p1);
+      exp2_pair((i % kPolyEveryDq) == 1, x0, x1, p0, p1);
       if (kMasked) {
         p0 = (col >= a && col < b) ? p0 : 0.f;
         p1 = (col + 1 >= a && col + 1 < b) ? p1 : 0.f;
