@@ -59,6 +59,10 @@ SMALL_CASES = {
     "bs64_g2_d128": dict(Hq=4, Hkv=2, d=128, bs=64, anchors=8),
     # 32 block keys, 32 rows (one pass of the reduce kernel)
     "bs32_g1_d128": dict(Hq=2, Hkv=2, d=128, bs=32, anchors=12),
+    # 128 block keys: the tensor-core reduce with eight 16-key steps (d = 64), and at
+    # d = 128 the two-role reduce at its largest shared memory (226 KB) beside the tensor-core merge
+    "bs128_g1_d64": dict(Hq=2, Hkv=2, d=64, bs=128, anchors=6),
+    "bs128_g1_d128": dict(Hq=2, Hkv=2, d=128, bs=128, anchors=6),
 }
 
 
